@@ -1,0 +1,49 @@
+"""End-to-end accuracy of the oracle against the page's printed figure.
+
+"Issue 5 probe: int8 quantized DiT serve paths on the RTX 3090", Round two,
+kernel-path verification: the raw ops match a float32 reference at 0.17%
+rel-L2 across (64,256,128) / (512,4096,4096) / (512,4096,12288).  Reading (see
+tests/golden/relL2_verification.json): the reference is the fp32 product of
+the dequantised operands, so 0.17% is the bf16 output rounding floor.  A wrong
+scale, a dropped term or a transposed operand moves the error by orders of
+magnitude, so this pins the composition of the three steps.
+"""
+import json
+import os
+
+import numpy as np
+import pytest
+
+import oracle
+from w8a8_int8_dynamic_b200.workloads import WORKLOADS, bf16_bits_to_f32, make_inputs
+
+GOLD = json.load(open(os.path.join(os.path.dirname(__file__), "golden", "relL2_verification.json")))
+
+
+def _rel_l2(a, b):
+    return float(np.linalg.norm(a - b) / np.linalg.norm(b))
+
+
+@pytest.mark.parametrize("name,rows", [
+    ("small_64x128x256", None),
+    ("square_512x4096x4096", 48),
+    ("fused_qkv_512x12288x4096", 32),
+])
+def test_rel_l2_matches_page_figure(name, rows):
+    wl = WORKLOADS[name]
+    assert [wl.M, wl.K, wl.N] in GOLD["shapes_M_K_N"]
+    inp = make_inputs(wl)
+    x = inp.x if rows is None else np.concatenate([inp.x[:rows - 1], inp.x[-1:]])
+    y, q, a_s, acc = oracle.linear(x, inp.w, inp.w_scale, inp.bias)
+    yf = bf16_bits_to_f32(y).astype(np.float64)
+    bias = 0.0 if inp.bias is None else bf16_bits_to_f32(inp.bias).astype(np.float64)
+    wdq = inp.w.astype(np.float64) * inp.w_scale[:, None].astype(np.float64)
+    ref = (q.astype(np.float64) * a_s[:, None].astype(np.float64)) @ wdq.T + bias
+    err = _rel_l2(yf, ref)
+    target = GOLD["rel_l2"]
+    assert 0.6 * target <= err <= 1.5 * target, err
+    # the unquantised-activation error is much larger with outlier channels;
+    # reported, not gated, but it must stay a few percent
+    xf = bf16_bits_to_f32(x).astype(np.float64)
+    err_unq = _rel_l2(yf, xf @ wdq.T + bias)
+    assert err_unq < 0.08
