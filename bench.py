@@ -1,0 +1,479 @@
+"""Benchmark of the W8A8 int8-dynamic linear path on B200.
+
+One step = one pass of the hot path over one batch: dynamic per-token int8
+quantisation of the activations, the int8 x int8 -> int32 tensor-core GEMM
+against pre-packed int8 weights, and the dequantising bf16 epilogue
+(w8a8_linear), on the square 512 x 4096 x 4096 projection with bias and an
+all-zero row.  Weights are packed once before timing (load time).
+
+Prints ONE JSON line (rank 0).  ``value`` is whole-job int8 TOPS (2*M*N*K per
+step, summed over ranks, divided by the max-over-ranks device time).  Inputs
+rotate over enough buffer sets to exceed the 126 MB L2, and each set's step is
+replayed from a CUDA graph so host launch overhead stays out of the device
+timing.  Also reported: the dominant kernel's roofline (GEMM alone, CUDA
+events on its stream), an end-to-end figure through the public API with
+host buffers, the oracle's CPU throughput, SM clocks sampled during the timed
+region, and a sweep over the other workloads.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                  [--no-sweep] [--workload NAME]
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+import torch
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, HERE)
+
+from w8a8_int8_dynamic_b200.workloads import WORKLOADS, make_inputs  # noqa: E402
+
+MAIN_WORKLOAD = "square_512x4096x4096"
+L2_BYTES = 126 * 1024 * 1024
+SPEC_INT8_TOPS = 4500.0
+
+
+# ----------------------------------------------------------------------------- peaks
+def load_peaks():
+    path = os.path.join(HERE, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        p = json.load(open(path))
+        return {"hbm_gbs": float(p["hbm_gbs"]), "bf16_tflops": float(p["bf16_tflops"]),
+                "bf16_tflops_sustained": float(p.get("bf16_tflops_sustained", p["bf16_tflops"])),
+                "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+            "source": "fallback"}
+
+
+# ----------------------------------------------------------------------------- clocks
+class ClockSampler:
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        os.makedirs(os.path.join(HERE, "gpurun_out"), exist_ok=True)
+        self.path = os.path.join(HERE, "gpurun_out", f"clocks_rank{self.index}.csv")
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "50"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except (FileNotFoundError, OSError):
+            self.proc = None
+        time.sleep(0.3)
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"],
+                    "samples": 0}
+        time.sleep(0.15)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        rows = []
+        for line in open(self.path):
+            parts = [t.strip() for t in line.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                rows.append((float(parts[0]), float(parts[1]), parts[2], parts[3:]))
+            except ValueError:
+                continue
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        names = ["active_mask", "hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown",
+                 "sw_power_cap"]
+        reasons = set()
+        for r in rows:
+            for n, v in zip(names[1:], r[3][1:]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        loaded = [r[0] for r in rows if r[0] > 500] or [r[0] for r in rows]
+        return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": max(r[1] for r in rows),
+                "reasons": sorted(reasons), "samples": len(rows)}
+
+
+# ----------------------------------------------------------------------------- helpers
+def bf16_dev(a_u16: np.ndarray, device) -> torch.Tensor:
+    return torch.from_numpy(np.ascontiguousarray(a_u16).view(np.int16)).to(device).view(torch.bfloat16)
+
+
+def algorithmic(wl, M=None):
+    M = wl.M if M is None else M
+    N, K = wl.N, wl.K
+    bias = 2 * N if wl.bias else 0
+    ops = 2 * M * N * K
+    gemm_bytes = M * K + N * K + 2 * M * N + 4 * M + 4 * N + bias
+    quant_bytes = 3 * M * K + 4 * M
+    fused_bytes = 2 * M * K + N * K + 2 * M * N + 4 * N + bias
+    return ops, gemm_bytes, quant_bytes, fused_bytes
+
+
+class LayerSets:
+    """``nsets`` independent copies of a workload's tensors on the device."""
+
+    def __init__(self, w8, wl, nsets, device, M=None):
+        inp = make_inputs(wl, M)
+        self.M, self.N, self.K = inp.x.shape[0], wl.N, wl.K
+        self.sets = []
+        x0 = bf16_dev(inp.x, device)
+        w0 = torch.from_numpy(inp.w).to(device)
+        packed0 = w8.pack_weight(w0)
+        del w0
+        ws0 = torch.from_numpy(inp.w_scale).to(device)
+        b0 = None if inp.bias is None else bf16_dev(inp.bias, device)
+        wsb = w8.linear_workspace_bytes(self.M, self.N, self.K)
+        mmws = w8.scaled_mm_workspace_bytes(self.M, self.N, self.K)
+        for i in range(nsets):
+            s = {
+                "x": x0 if i == 0 else x0.clone(),
+                "packed": packed0 if i == 0 else packed0.clone(),
+                "w_scale": ws0 if i == 0 else ws0.clone(),
+                "bias": None if b0 is None else (b0 if i == 0 else b0.clone()),
+                "y": torch.empty((self.M, self.N), dtype=torch.bfloat16, device=device),
+                "ws": torch.empty((wsb,), dtype=torch.uint8, device=device),
+                "mmws": torch.empty((max(mmws, 16),), dtype=torch.uint8, device=device)
+                if mmws else None,
+            }
+            s["q"], s["a_scale"] = w8.quant_act(s["x"])
+            self.sets.append(s)
+        torch.cuda.synchronize()
+
+    def set_bytes(self):
+        s = self.sets[0]
+        return sum(t.numel() * t.element_size() for k, t in s.items()
+                   if isinstance(t, torch.Tensor))
+
+
+def sets_needed(w8, wl, M=None):
+    probe_M = wl.M if M is None else M
+    per = (probe_M * wl.K * 3 + wl.N * wl.K + 2 * probe_M * wl.N + 8 * wl.N
+           + w8.linear_workspace_bytes(probe_M, wl.N, wl.K))
+    n = 1
+    while n * per <= 1.5 * L2_BYTES and n < 16:
+        n += 1
+    return n, per
+
+
+def capture(fn, stream):
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        fn()
+    return g
+
+
+def time_graphs(graphs, steps, stream):
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        start.record(stream)
+        for i in range(steps):
+            graphs[i % len(graphs)].replay()
+        end.record(stream)
+    end.synchronize()
+    return start.elapsed_time(end) / 1e3  # seconds
+
+
+# ----------------------------------------------------------------------------- our arm
+def run_workload(w8, wl, steps, warmup, device, stream, M=None, with_quant=True):
+    nsets, _ = sets_needed(w8, wl, M)
+    ls = LayerSets(w8, wl, nsets, device, M)
+    before = w8.launch_count()
+    layer_graphs, mm_graphs, q_graphs = [], [], []
+    for s in ls.sets:
+        def step(s=s):
+            w8.linear(s["x"], s["packed"], s["w_scale"], s["bias"], ls.N, out=s["y"],
+                      workspace=s["ws"], stream=stream)
+        def mm(s=s):
+            w8.scaled_mm(s["q"], s["a_scale"], s["packed"], s["w_scale"], s["bias"], ls.N,
+                         out=s["y"], workspace=s["mmws"], stream=stream)
+        def qa(s=s):
+            w8.quant_act(s["x"], q=s["q"], a_scale=s["a_scale"], stream=stream)
+        with torch.cuda.stream(stream):
+            step(); mm(); qa()  # warm the launch path (attributes, tensor maps) before capture
+        torch.cuda.synchronize()
+        c0 = w8.launch_count()
+        layer_graphs.append(capture(step, stream))
+        per_step = w8.launch_count() - c0
+        mm_graphs.append(capture(mm, stream))
+        q_graphs.append(capture(qa, stream))
+    torch.cuda.synchronize()
+    assert w8.poll_status() == 0
+    for g in (layer_graphs, mm_graphs, q_graphs):
+        time_graphs(g, max(warmup, 3) * len(g), stream)
+    res = {"launches_per_step": per_step, "nsets": nsets, "set_bytes": ls.set_bytes(),
+           "M": ls.M, "N": ls.N, "K": ls.K}
+    res["t_step"] = time_graphs(layer_graphs, steps, stream) / steps
+    res["t_gemm"] = time_graphs(mm_graphs, steps, stream) / steps
+    if with_quant:
+        res["t_quant"] = time_graphs(q_graphs, steps, stream) / steps
+    assert w8.poll_status() == 0, "device-side timeout during the benchmark"
+    del before
+    return ls, layer_graphs, res
+
+
+def run_ours(args, rank, world, device):
+    import w8a8_int8_dynamic_b200 as w8
+    w8.lib()
+    peaks = load_peaks()
+    int8_peak = 2.0 * peaks["bf16_tflops"]  # nominal int8 : bf16 dense rate = 2
+    stream = torch.cuda.Stream(device=device)
+    wl = WORKLOADS[args.workload]
+    ops, gemm_bytes, quant_bytes, fused_bytes = algorithmic(wl)
+
+    ls, layer_graphs, base = run_workload(w8, wl, max(args.warmup, 3), args.warmup, device, stream)
+    # ---- the timed region: exactly K steps, barrier + sync on both sides
+    sampler = ClockSampler(torch.cuda.current_device() if "CUDA_VISIBLE_DEVICES" in os.environ
+                           else device.index or 0)
+    sampler.start()
+    for _ in range(args.warmup):
+        time_graphs(layer_graphs, len(layer_graphs), stream)
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        start.record(stream)
+        for i in range(args.steps):
+            layer_graphs[i % len(layer_graphs)].replay()
+        end.record(stream)
+    end.synchronize()
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    elapsed = start.elapsed_time(end) / 1e3
+    clocks = sampler.stop()
+    assert w8.poll_status() == 0, "device-side timeout during the timed region"
+    t_max = elapsed
+    if world > 1:
+        t = torch.tensor([elapsed], dtype=torch.float64, device=device)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        t_max = float(t.item())
+    value = ops * args.steps * world / t_max / 1e12
+    ms_per_step = t_max / args.steps * 1e3
+
+    # ---- dominant kernel (the GEMM) alone, CUDA events on its stream
+    gemm_tops = ops / base["t_gemm"] / 1e12
+    roofline = {"bound": "tensor", "achieved": round(gemm_tops, 2), "peak": round(int8_peak, 1),
+                "unit": "TOPS", "frac": round(gemm_tops / int8_peak, 4), "traffic": None,
+                "kernel": "gemm_kernel (persistent tcgen05 kind::i8 + epilogue)",
+                "peak_note": f"int8 = 2 x {peaks['source']} bf16 burst {peaks['bf16_tflops']} TFLOP/s",
+                "frac_vs_spec_4500": round(gemm_tops / SPEC_INT8_TOPS, 4),
+                "gemm_us": round(base["t_gemm"] * 1e6, 3),
+                "quant_us": round(base["t_quant"] * 1e6, 3),
+                "quant_gbs": round(quant_bytes / base["t_quant"] / 1e9, 1),
+                "quant_frac_hbm": round(quant_bytes / base["t_quant"] / 1e9 / peaks["hbm_gbs"], 4)}
+    traffic_file = os.path.join(HERE, "profiles", "traffic.json")
+    if os.path.exists(traffic_file):
+        tr = json.load(open(traffic_file)).get(args.workload, {})
+        if tr.get("gemm_bytes_per_launch") is not None:
+            roofline["traffic"] = tr["gemm_bytes_per_launch"]
+
+    # ---- end to end through the public API, host buffers
+    e2e = run_e2e(w8, ls, args, stream, ops)
+
+    out = {
+        "metric": "W8A8 quant+scaled-GEMM TOPS and % of int8 roofline on one B200",
+        "value": round(value, 2), "unit": "TOPS", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(ms_per_step, 5), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "int8 x int8 -> int32, bf16 in/out",
+        "data": "synthetic (seeded; N(0,1) activations with 1% outlier channels x10, "
+                "int8 weights uniform [-127,127], fp32 scales, bf16 bias)",
+        "config": {"workload": args.workload, "M": wl.M, "N": wl.N, "K": wl.K,
+                   "step": "w8a8_linear = quant kernel + tcgen05 GEMM/epilogue (2 launches, PDL)",
+                   "l2": f"rotating {base['nsets']} input sets of {base['set_bytes'] / 2**20:.1f} MiB "
+                         f"(> 126 MB L2)",
+                   "launch": "per-set CUDA graph replay", "parallelism": f"replicas x{world}"},
+        "roofline": roofline,
+        "fused_frac_of_roofline": round(max(ops / (int8_peak * 1e12),
+                                            fused_bytes / (peaks["hbm_gbs"] * 1e9)) / (t_max / args.steps),
+                                        4),
+        "e2e": e2e,
+        "gpu_launches": int(base["launches_per_step"] * args.steps),
+        "clocks": clocks,
+    }
+    if rank == 0 and not args.no_cpu_baseline:
+        out["cpu_baseline"] = cpu_baseline(wl, budget_s=args.cpu_seconds)
+    if not args.no_sweep:
+        out["sweep"] = sweep(w8, args, device, stream, peaks, int8_peak)
+    return out
+
+
+def run_e2e(w8, ls, args, stream, ops):
+    """Public API, host buffers: per step H2D of x from pinned memory, the
+    layer call, D2H of y into pinned memory, all inside the timed region."""
+    s0 = ls.sets[0]
+    M, N, K = ls.M, ls.N, ls.K
+    nbuf = 4
+    xs = [s0["x"].cpu().pin_memory() for _ in range(nbuf)]
+    ys = [torch.empty((M, N), dtype=torch.bfloat16).pin_memory() for _ in range(nbuf)]
+    xd = torch.empty_like(s0["x"])
+    layer_args = (s0["packed"], s0["w_scale"], s0["bias"], N)
+    steps = max(10, min(args.steps, 2000))
+    with torch.cuda.stream(stream):
+        for i in range(3):
+            xd.copy_(xs[i % nbuf], non_blocking=True)
+            y = w8.linear(xd, *layer_args, workspace=s0["ws"], stream=stream)
+            ys[i % nbuf].copy_(y, non_blocking=True)
+        torch.cuda.synchronize()
+        start = torch.cuda.Event(enable_timing=True)
+        end = torch.cuda.Event(enable_timing=True)
+        start.record(stream)
+        for i in range(steps):
+            xd.copy_(xs[i % nbuf], non_blocking=True)
+            y = w8.linear(xd, *layer_args, workspace=s0["ws"], stream=stream)
+            ys[i % nbuf].copy_(y, non_blocking=True)
+        end.record(stream)
+        end.synchronize()
+    t = start.elapsed_time(end) / 1e3 / steps
+    return {"value": round(ops / t / 1e12, 3), "unit": "TOPS", "h2d_bytes_per_step": M * K * 2,
+            "d2h_bytes_per_step": M * N * 2, "steps": steps, "ms_per_step": round(t * 1e3, 4),
+            "api": "w8a8_int8_dynamic_b200.linear (ctypes -> w8a8_linear)"}
+
+
+def sweep(w8, args, device, stream, peaks, int8_peak):
+    out = {}
+    names = ["small_64x128x256", "square_512x4096x4096", "fused_qkv_512x12288x4096",
+             "dit_mlp_up_4096x12288x3072", "dit_mlp_down_4096x3072x12288",
+             "decode_m1_27648x5120", "decode_m4_27648x5120", "decode_m16_27648x5120"]
+    for name in names:
+        wl = WORKLOADS[name]
+        ops, gemm_bytes, quant_bytes, fused_bytes = algorithmic(wl)
+        steps = 200 if wl.M * wl.N * wl.K > 1e11 else 1000
+        ls, graphs, r = run_workload(w8, wl, steps, 3, device, stream)
+        t_roof_gemm = max(ops / (int8_peak * 1e12), gemm_bytes / (peaks["hbm_gbs"] * 1e9))
+        t_roof_fused = max(ops / (int8_peak * 1e12), fused_bytes / (peaks["hbm_gbs"] * 1e9))
+        bound = "tensor" if ops / (int8_peak * 1e12) >= gemm_bytes / (peaks["hbm_gbs"] * 1e9) else "hbm"
+        out[name] = {
+            "M": wl.M, "N": wl.N, "K": wl.K, "bound": bound,
+            "step_us": round(r["t_step"] * 1e6, 3), "gemm_us": round(r["t_gemm"] * 1e6, 3),
+            "quant_us": round(r["t_quant"] * 1e6, 3),
+            "step_tops": round(ops / r["t_step"] / 1e12, 2),
+            "gemm_tops": round(ops / r["t_gemm"] / 1e12, 2),
+            "gemm_gbs": round(gemm_bytes / r["t_gemm"] / 1e9, 1),
+            "gemm_frac_roofline": round(t_roof_gemm / r["t_gemm"], 4),
+            "gemm_frac_spec_int8": round(ops / r["t_gemm"] / 1e12 / SPEC_INT8_TOPS, 4),
+            "quant_gbs": round(quant_bytes / r["t_quant"] / 1e9, 1),
+            "quant_frac_hbm": round(quant_bytes / r["t_quant"] / 1e9 / peaks["hbm_gbs"], 4),
+            "step_frac_roofline": round(t_roof_fused / r["t_step"], 4),
+            "l2_sets": r["nsets"],
+        }
+        del ls, graphs
+        torch.cuda.empty_cache()
+    return out
+
+
+# ----------------------------------------------------------------------------- CPU oracle
+def cpu_baseline(wl, budget_s=12.0):
+    """The oracle as it stands, on the host cores: whole layers of the same
+    workload, repeated until about budget_s seconds have elapsed."""
+    import oracle
+    inp = make_inputs(wl)
+    ops = 2 * wl.M * wl.N * wl.K
+    oracle.linear(inp.x[:8], inp.w[:64], inp.w_scale[:64], None if inp.bias is None else inp.bias[:64])
+    t0 = time.perf_counter()
+    reps = 0
+    while True:
+        oracle.linear(inp.x, inp.w, inp.w_scale, inp.bias)
+        reps += 1
+        if time.perf_counter() - t0 >= budget_s or reps >= 50:
+            break
+    t = (time.perf_counter() - t0) / reps
+    return {"value": round(ops / t / 1e12, 5), "unit": "TOPS", "cores": oracle.num_threads(),
+            "kind": "oracle",
+            "sample": f"{reps} full {wl.name} layers (quant + int32 GEMM + epilogue), "
+                      f"{t:.3f} s each, OpenMP over rows"}
+
+
+def run_reference(args):
+    wl = WORKLOADS[args.workload]
+    import oracle
+    inp = make_inputs(wl)
+    ops = 2 * wl.M * wl.N * wl.K
+    # bounded sample per step: a slice of rows of the same workload
+    rows = max(1, min(wl.M, int(args.ref_rows)))
+    x = inp.x[:rows]
+    for _ in range(args.warmup):
+        oracle.linear(x, inp.w, inp.w_scale, inp.bias)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        oracle.linear(x, inp.w, inp.w_scale, inp.bias)
+    t = (time.perf_counter() - t0) / args.steps
+    sample_ops = 2 * rows * wl.N * wl.K
+    value = sample_ops / t / 1e12
+    return {
+        "metric": "W8A8 quant+scaled-GEMM TOPS and % of int8 roofline on one B200",
+        "impl": "reference", "value": round(value, 5), "unit": "TOPS", "n_gpus": 1,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(t * 1e3, 3),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "int8 x int8 -> int32, bf16 in/out", "data": "synthetic (seeded)",
+        "config": {"workload": args.workload, "M": wl.M, "N": wl.N, "K": wl.K,
+                   "sample_rows_per_step": rows},
+        "cpu_baseline": {"value": round(value, 5), "unit": "TOPS", "cores": oracle.num_threads(),
+                         "kind": "oracle",
+                         "sample": f"{rows} of {wl.M} rows of {wl.name} per step "
+                                   f"({sample_ops / ops:.3f} of a layer)"},
+        "e2e": {"value": round(value, 5), "unit": "TOPS", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+
+
+# ----------------------------------------------------------------------------- main
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20000)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default=MAIN_WORKLOAD, choices=list(WORKLOADS))
+    ap.add_argument("--no-sweep", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--ref-rows", type=int, default=64)
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        if rank == 0:
+            print(json.dumps(run_reference(args)), flush=True)
+        return 0
+
+    device = torch.device("cuda", local_rank)
+    torch.cuda.set_device(device)
+    if world > 1:
+        import datetime
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=device)
+    try:
+        out = run_ours(args, rank, world, device)
+        if rank == 0:
+            print(json.dumps(out), flush=True)
+    finally:
+        if world > 1:
+            torch.distributed.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

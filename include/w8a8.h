@@ -1,0 +1,185 @@
+/*
+ * w8a8.h -- C ABI of libw8a8.so: W8A8 int8-dynamic linear layers for NVIDIA
+ * B200 (sm_100a).
+ *
+ * The method (sources by page title and section):
+ *   "Issue 5 probe: int8 quantized DiT serve paths on the RTX 3090",
+ *   Round two: int8 weights with fp32 per-output-channel scales, dynamic
+ *   per-token symmetric int8 activations, an int8 scaled matmul, and the
+ *   layer path "load -> transpose-repack -> apply" with fused Q/K/V and
+ *   row-parallel layers.  "INT8 Quant for Dual-Max Recipe": int8 x int8 on
+ *   the integer tensor cores with no dequantisation of the weights.
+ *   "Online Quantization", Parameters: activation_scheme "dynamic".
+ *
+ * Arithmetic (identical, bit for bit, to the CPU oracle of this repository):
+ *   a_scale[m] = amax_k |x[m,k]| / 127                (fp32, IEEE division)
+ *   q[m,k]     = clamp(rint_half_even(x[m,k] / a_scale[m]), -127, 127)
+ *                (q = 0 and a_scale = 0 for a row whose amax is 0)
+ *   acc[m,n]   = sum_k q[m,k] * w[n,k]                 (exact int32)
+ *   y[m,n]     = bf16_rne(((float)acc * a_scale[m]) * w_scale[n] + bias[n])
+ *                (each step one fp32 operation rounded to nearest even)
+ *
+ * Conventions for every entry point:
+ *   - Pointers marked "device" are CUDA device pointers of the current
+ *     device; the caller allocates and owns them.  The library allocates no
+ *     device memory per call (it keeps one 4-byte status word per device).
+ *   - Matrices are row-major.  x: bf16 [M, K] with row stride ldx elements;
+ *     q: int8 [M, K] dense; w: int8 [N, K] (K contiguous, i.e. out x in);
+ *     y: bf16 [M, N] dense.  bf16 is passed as raw 16-bit storage.
+ *   - All work is enqueued on `stream` (NULL = legacy default stream) and is
+ *     asynchronous; no entry point synchronises except w8a8_poll_status.
+ *   - Argument checks run on the host before any launch; on failure nothing
+ *     is launched and the status says why.  A launch failure returns
+ *     W8A8_ERR_CUDA.  Kernels never trap: a device-side wait that exceeds
+ *     its time limit (about one second) records W8A8_ERR_TIMEOUT in the
+ *     device status word, which w8a8_poll_status reports.
+ *   - Shape limits: 1 <= M <= 2^31-1, 1 <= N, 16 <= K <= 131072, K % 16 == 0
+ *     (16-byte rows for TMA), N % 8 == 0 (16-byte output rows), all pointers
+ *     16-byte aligned.  K <= 131072 keeps |acc| <= 131072*127*128 < 2^31.
+ *   - Calls that share buffers and overlap on the GPU race; use one stream
+ *     or events.
+ */
+#ifndef W8A8_H_
+#define W8A8_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same object as cudaStream_t / CUstream. */
+typedef struct CUstream_st *w8a8_stream_t;
+
+typedef enum w8a8_status {
+  W8A8_OK = 0,
+  W8A8_ERR_INVALID_ARG = 1,       /* null pointer, negative size, bad enum */
+  W8A8_ERR_ALIGNMENT = 2,         /* pointer or stride not 16-byte aligned */
+  W8A8_ERR_UNSUPPORTED_SHAPE = 3, /* K % 16, N % 8, K range, M range */
+  W8A8_ERR_CUDA = 4,              /* a CUDA runtime / launch error */
+  W8A8_ERR_TIMEOUT = 5,           /* a device-side wait gave up (kernel output invalid) */
+  W8A8_ERR_BUFFER_TOO_SMALL = 6   /* packed or workspace buffer too small */
+} w8a8_status;
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char *w8a8_status_string(int status);
+
+/* ABI version of this header: (major << 16) | minor. */
+int w8a8_abi_version(void);
+
+/* ---- step 1: dynamic per-token activation quantisation ------------------
+ * Source: "Issue 5 probe ...", Round two ("dynamic per-token symmetric int8
+ * activations", op scaled_int8_quant); "Online Quantization", Parameters.
+ *   x       device, bf16 [M, K], row stride ldx >= K elements (ldx % 8 == 0)
+ *   q       device, int8 [M, K] dense (output)
+ *   a_scale device, fp32 [M]   (output)
+ * One pass over x: 2*M*K bytes read, M*K + 4*M bytes written. */
+w8a8_status w8a8_quant_act(const void *x, int64_t M, int64_t K, int64_t ldx,
+                           int8_t *q, float *a_scale, w8a8_stream_t stream);
+
+/* ---- step 2 (load time): weight repack ------------------------------------
+ * Source: "Issue 5 probe ...", Round two, kernel-path verification
+ * ("load -> transpose-repack -> apply"); the layout is this library's own:
+ * 128x128-byte tiles, each the K-major 128-byte-swizzled shared-memory image
+ * the tensor core reads, N padded to 256 and K to 128 with zeros.
+ *   Byte size of the packed buffer for an [N, K] weight: */
+w8a8_status w8a8_packed_weight_bytes(int64_t N, int64_t K, size_t *bytes);
+
+/*   w      device, int8 [N, K] row-major (K contiguous)
+ *   packed device, packed_bytes >= w8a8_packed_weight_bytes(N, K)
+ * Every byte of `packed` is written (padding with zeros).  Fused Q/K/V:
+ * concatenate the three [hidden, K] blocks along N (and their scales) and
+ * pack once; the output's column slices are the three projections. */
+w8a8_status w8a8_pack_weight(const int8_t *w, int64_t N, int64_t K,
+                             void *packed, size_t packed_bytes,
+                             w8a8_stream_t stream);
+
+/* Inverse of w8a8_pack_weight (test and inspection use): packed -> w [N, K]. */
+w8a8_status w8a8_unpack_weight(const void *packed, int64_t N, int64_t K,
+                               int8_t *w, w8a8_stream_t stream);
+
+/* ---- steps 3+4: int8 GEMM with the dequantising epilogue -----------------
+ * Source: "Issue 5 probe ...", Round two (op cutlass_scaled_mm: int8 x int8
+ * with per-token and per-channel fp32 scales); "INT8 Quant for Dual-Max
+ * Recipe" (native int8 tensor-core path, no weight dequantisation).
+ *   q        device, int8 [M, K] dense (from w8a8_quant_act)
+ *   a_scale  device, fp32 [M]
+ *   packed_w device, from w8a8_pack_weight(N, K)
+ *   w_scale  device, fp32 [N]
+ *   bias     device, bf16 [N], or NULL for no bias
+ *   y        device, bf16 [M, N] (output)
+ *   workspace device scratch of ws_bytes >= w8a8_scaled_mm_workspace_bytes,
+ *            or NULL.  Only the small-M (decode) kernel uses it: int32 split-K
+ *            partials and one counter per 128-row weight block.  With NULL,
+ *            every M runs the large-M kernel.
+ * Large M runs the persistent tcgen05 GEMM; M <= 16 with a workspace runs
+ * the weight-streaming swap-AB kernel.  Both give bit-identical results. */
+w8a8_status w8a8_scaled_mm_workspace_bytes(int64_t M, int64_t N, int64_t K,
+                                           size_t *bytes);
+w8a8_status w8a8_scaled_mm(const int8_t *q, const float *a_scale,
+                           const void *packed_w, const float *w_scale,
+                           const void *bias, void *y, int64_t M, int64_t N,
+                           int64_t K, void *workspace, size_t ws_bytes,
+                           w8a8_stream_t stream);
+
+/* The int32 accumulators acc[M, N] of the same GEMM, without the epilogue
+ * (test and inspection use; acc device, int32 [M, N]). */
+w8a8_status w8a8_scaled_mm_i32(const int8_t *q, const void *packed_w,
+                               int32_t *acc, int64_t M, int64_t N, int64_t K,
+                               w8a8_stream_t stream);
+
+/* ---- the whole layer: quantise + GEMM + epilogue --------------------------
+ * Source: "Issue 5 probe ...", Round two (the layer path: the activation
+ * quantisation feeds the scaled matmul).  Two launches on `stream`; the GEMM
+ * is launched as a programmatic dependent of the quantisation so that its
+ * set-up overlaps the quantisation's tail.
+ *   x         device, bf16 [M, K], row stride ldx
+ *   workspace device, ws_bytes >= w8a8_linear_workspace_bytes(M, N, K); holds
+ *             q and a_scale (and split-K partials for small M).  Its contents
+ *             on entry do not matter.
+ * N-D activations [..., K] are flattened by the caller to [M, K] and y is
+ * viewed back as [..., N] (the "Diffusion Quantization Reference", GGUF
+ * rules and the output-rank failure in "Common Failures"). */
+w8a8_status w8a8_linear_workspace_bytes(int64_t M, int64_t N, int64_t K,
+                                        size_t *bytes);
+w8a8_status w8a8_linear(const void *x, int64_t ldx, const void *packed_w,
+                        const float *w_scale, const void *bias, void *y,
+                        int64_t M, int64_t N, int64_t K, void *workspace,
+                        size_t ws_bytes, w8a8_stream_t stream);
+
+/* ---- path selection (tests and benchmarks) ---------------------------------
+ * 0 = automatic (default); 1 = always the persistent large-M GEMM (automatic
+ * tile width); 2 = the small-M weight-streaming kernel (M <= 16 only, else
+ * W8A8_ERR_INVALID_ARG); 3 / 4 = the large-M GEMM with 128- / 256-wide
+ * output tiles.  Process-wide; not synchronised with concurrent calls. */
+w8a8_status w8a8_set_path(int path);
+
+/* ---- harness kernel: GELU (tanh form), bf16 -> bf16 ------------------------
+ * Not on the pages; it joins the up and down projections of the DiT MLP
+ * workload.  y = 0.5 x (1 + tanh(sqrt(2/pi)(x + 0.044715 x^3))) in fp32,
+ * rounded to bf16.  x, y device bf16 [n]; y may alias x. */
+w8a8_status w8a8_gelu_tanh(const void *x, void *y, int64_t n,
+                           w8a8_stream_t stream);
+
+/* ---- errors ----------------------------------------------------------------
+ * Synchronises `stream`, then returns and clears the device status word of
+ * the current device: W8A8_ERR_TIMEOUT if any kernel gave up on a wait since
+ * the last poll, W8A8_ERR_CUDA on an asynchronous CUDA error, else W8A8_OK. */
+w8a8_status w8a8_poll_status(w8a8_stream_t stream);
+
+/* Self-test of the bounded-wait path: launches one block that waits on a
+ * barrier nothing will ever complete, with a limit of timeout_ns
+ * nanoseconds (clamped to [1e3, 5e9]); the wait gives up, records
+ * W8A8_ERR_TIMEOUT in the status word and the kernel exits normally. */
+w8a8_status w8a8_selftest_wait_timeout(int64_t timeout_ns,
+                                       w8a8_stream_t stream);
+
+/* Number of kernels this library has launched in this process (all devices). */
+int64_t w8a8_launch_count(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* W8A8_H_ */

@@ -258,8 +258,11 @@ int64_t w8a8o_packed_bytes(int64_t N, int64_t K) {
 
 /* ---- GELU (tanh form), bf16 -> bf16 ----------------------------------------
  * Only used between the up and down projections of the DiT MLP workload; the
- * pages do not define it.  0.5 x (1 + tanh( sqrt(2/pi) (x + 0.044715 x^3) ))
- * evaluated in double and rounded once to bf16. */
+ * pages do not define it.  GELU_tanh(x) = 0.5 x (1 + tanh(u)) with
+ * u = sqrt(2/pi) (x + 0.044715 x^3).  Since 0.5 (1 + tanh(u)) = 1 / (1 + e^(-2u))
+ * exactly, it is evaluated in double as x * sigma(2u), with sigma written so
+ * that no step cancels (1 + tanh(u) loses every digit once tanh(u) rounds to
+ * -1, e.g. u < -19 in double), then rounded once to bf16. */
 int w8a8o_gelu_tanh(const uint16_t *x, int64_t n, uint16_t *y) {
   if (!x || !y || n < 0) return ORACLE_EINVAL;
   const double c = sqrt(2.0 / 3.14159265358979323846);
@@ -267,8 +270,10 @@ int w8a8o_gelu_tanh(const uint16_t *x, int64_t n, uint16_t *y) {
 #pragma omp parallel for schedule(static)
   for (i = 0; i < n; ++i) {
     double v = (double)bf16_to_f32(x[i]);
-    double g = 0.5 * v * (1.0 + tanh(c * (v + 0.044715 * v * v * v)));
-    y[i] = f64_to_bf16_rne(g);
+    double u = c * (v + 0.044715 * v * v * v);
+    double e = exp(-2.0 * fabs(u));           /* in (0, 1] */
+    double sig = u >= 0.0 ? 1.0 / (1.0 + e) : e / (1.0 + e);
+    y[i] = f64_to_bf16_rne(v * sig);
   }
   return ORACLE_OK;
 }

@@ -3,6 +3,8 @@ down projections of the DiT MLP workload (the pages do not define it).
 
 Pinned by closed forms of the tanh form, its odd-part identity, and its known
 distance from the exact erf GELU (a library routine)."""
+from decimal import Decimal, getcontext
+
 import numpy as np
 from scipy.special import erf
 
@@ -45,3 +47,32 @@ def test_positive_part_monotone():
     v = np.linspace(0, 8, 2001, dtype=np.float32)
     y, _ = _g(v)
     assert (np.diff(y) >= 0).all()
+
+
+def _gelu_decimal(x: float) -> Decimal:
+    """GELU_tanh at 60 significant digits: 0.5 x (1 + tanh(u)) with tanh
+    written through exp, evaluated in decimal arithmetic."""
+    getcontext().prec = 60
+    d = Decimal(x)
+    pi = Decimal("3.14159265358979323846264338327950288419716939937510582097494")
+    u = (Decimal(2) / pi).sqrt() * (d + Decimal("0.044715") * d * d * d)
+    t = ((2 * u).exp() - 1) / ((2 * u).exp() + 1)  # tanh(u)
+    return Decimal("0.5") * d * (1 + t)
+
+
+def test_matches_high_precision_including_negative_tail():
+    """Against a 60-digit evaluation of the tanh form, including the tail
+    x in [-12, -3] where 1 + tanh(u) cancels in binary floating point."""
+    rng = np.random.default_rng(3)
+    v = np.concatenate([rng.uniform(-12, -3, 600), rng.uniform(-3, 3, 300),
+                        rng.uniform(3, 12, 100)]).astype(np.float32)
+    y, x = _g(v)
+    for xi, yi in zip(x, y):
+        ref = _gelu_decimal(float(xi))
+        if ref == 0:
+            assert yi == 0
+            continue
+        # one correct rounding to bf16: half an ulp of 8 significant bits, or
+        # half the smallest bf16 subnormal (2^-133) below the normal range
+        tol = max(abs(ref) * Decimal(2) ** -8, Decimal(2) ** -134)
+        assert abs(Decimal(float(yi)) - ref) <= tol, (xi, yi, ref)

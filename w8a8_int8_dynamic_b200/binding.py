@@ -1,0 +1,268 @@
+"""Thin ctypes binding of libw8a8.so.
+
+Argument marshalling only: every step of the path runs in the library's CUDA
+kernels.  PyTorch is used for device memory and the current stream.  There is
+no fallback: if the shared library is missing or a call fails, this raises.
+
+N-D activations [..., K] are flattened to [M, K] around the call and the
+output is viewed back as [..., N] (the "Diffusion Quantization Reference",
+GGUF rules: flatten N-D activations around the matmul and restore the shape;
+its "Common Failures" table lists the output-rank collapse this avoids).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional, Tuple
+
+import torch
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libw8a8.so")
+
+OK = 0
+STATUS_NAMES = {
+    0: "W8A8_OK", 1: "W8A8_ERR_INVALID_ARG", 2: "W8A8_ERR_ALIGNMENT",
+    3: "W8A8_ERR_UNSUPPORTED_SHAPE", 4: "W8A8_ERR_CUDA", 5: "W8A8_ERR_TIMEOUT",
+    6: "W8A8_ERR_BUFFER_TOO_SMALL",
+}
+
+PATH_AUTO, PATH_LARGE, PATH_SMALL, PATH_LARGE_BN128, PATH_LARGE_BN256 = 0, 1, 2, 3, 4
+
+
+class W8A8Error(RuntimeError):
+    def __init__(self, what: str, status: int):
+        super().__init__(f"{what} failed: {STATUS_NAMES.get(status, status)}")
+        self.status = status
+
+
+_lib = None
+
+_P = ctypes.c_void_p
+_I64 = ctypes.c_int64
+_SZ = ctypes.c_size_t
+
+_SIGNATURES = {
+    "w8a8_status_string": ([ctypes.c_int], ctypes.c_char_p),
+    "w8a8_abi_version": ([], ctypes.c_int),
+    "w8a8_quant_act": ([_P, _I64, _I64, _I64, _P, _P, _P], ctypes.c_int),
+    "w8a8_packed_weight_bytes": ([_I64, _I64, ctypes.POINTER(_SZ)], ctypes.c_int),
+    "w8a8_pack_weight": ([_P, _I64, _I64, _P, _SZ, _P], ctypes.c_int),
+    "w8a8_unpack_weight": ([_P, _I64, _I64, _P, _P], ctypes.c_int),
+    "w8a8_scaled_mm_workspace_bytes": ([_I64, _I64, _I64, ctypes.POINTER(_SZ)], ctypes.c_int),
+    "w8a8_scaled_mm": ([_P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _P, _SZ, _P], ctypes.c_int),
+    "w8a8_scaled_mm_i32": ([_P, _P, _P, _I64, _I64, _I64, _P], ctypes.c_int),
+    "w8a8_linear_workspace_bytes": ([_I64, _I64, _I64, ctypes.POINTER(_SZ)], ctypes.c_int),
+    "w8a8_linear": ([_P, _I64, _P, _P, _P, _P, _I64, _I64, _I64, _P, _SZ, _P], ctypes.c_int),
+    "w8a8_set_path": ([ctypes.c_int], ctypes.c_int),
+    "w8a8_gelu_tanh": ([_P, _P, _I64, _P], ctypes.c_int),
+    "w8a8_poll_status": ([_P], ctypes.c_int),
+    "w8a8_selftest_wait_timeout": ([_I64, _P], ctypes.c_int),
+    "w8a8_launch_count": ([], ctypes.c_int64),
+}
+
+
+def lib() -> ctypes.CDLL:
+    """Load libw8a8.so (built in-tree by ``w8a8_int8_dynamic_b200.build``)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(
+                f"libw8a8.so not found at {LIB_PATH}; build it with "
+                "`python -m w8a8_int8_dynamic_b200.build` (nvcc, sm_100a)")
+        L = ctypes.CDLL(LIB_PATH)
+        for name, (args, res) in _SIGNATURES.items():
+            fn = getattr(L, name)
+            fn.argtypes = args
+            fn.restype = res
+        _lib = L
+    return _lib
+
+
+def _check(rc: int, what: str):
+    if rc != OK:
+        raise W8A8Error(what, rc)
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream=None):
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _need_cuda(t: torch.Tensor, name: str, dtype=None):
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if dtype is not None and t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+
+
+# ---- sizes -------------------------------------------------------------------
+def packed_weight_bytes(N: int, K: int) -> int:
+    out = _SZ()
+    _check(lib().w8a8_packed_weight_bytes(N, K, ctypes.byref(out)), "w8a8_packed_weight_bytes")
+    return out.value
+
+
+def linear_workspace_bytes(M: int, N: int, K: int) -> int:
+    out = _SZ()
+    _check(lib().w8a8_linear_workspace_bytes(M, N, K, ctypes.byref(out)),
+           "w8a8_linear_workspace_bytes")
+    return out.value
+
+
+def scaled_mm_workspace_bytes(M: int, N: int, K: int) -> int:
+    out = _SZ()
+    _check(lib().w8a8_scaled_mm_workspace_bytes(M, N, K, ctypes.byref(out)),
+           "w8a8_scaled_mm_workspace_bytes")
+    return out.value
+
+
+# ---- ops ---------------------------------------------------------------------
+def quant_act(x: torch.Tensor, q: Optional[torch.Tensor] = None,
+              a_scale: Optional[torch.Tensor] = None, stream=None) -> Tuple[torch.Tensor, torch.Tensor]:
+    """x bf16 [M, K] (row stride may exceed K) -> (q int8 [M, K], a_scale fp32 [M])."""
+    _need_cuda(x, "x", torch.bfloat16)
+    M, K = x.shape
+    if x.stride(1) != 1:
+        raise ValueError("x must have unit stride along K")
+    if q is None:
+        q = torch.empty((M, K), dtype=torch.int8, device=x.device)
+    if a_scale is None:
+        a_scale = torch.empty((M,), dtype=torch.float32, device=x.device)
+    _check(lib().w8a8_quant_act(_ptr(x), M, K, x.stride(0), _ptr(q), _ptr(a_scale), _stream(stream)),
+           "w8a8_quant_act")
+    return q, a_scale
+
+
+def pack_weight(w: torch.Tensor, stream=None) -> torch.Tensor:
+    """int8 [N, K] (K contiguous) -> packed tile image (uint8, flat)."""
+    _need_cuda(w, "w", torch.int8)
+    w = w.contiguous()
+    N, K = w.shape
+    nbytes = packed_weight_bytes(N, K)
+    packed = torch.empty((nbytes,), dtype=torch.uint8, device=w.device)
+    _check(lib().w8a8_pack_weight(_ptr(w), N, K, _ptr(packed), nbytes, _stream(stream)),
+           "w8a8_pack_weight")
+    return packed
+
+
+def unpack_weight(packed: torch.Tensor, N: int, K: int, stream=None) -> torch.Tensor:
+    _need_cuda(packed, "packed")
+    w = torch.empty((N, K), dtype=torch.int8, device=packed.device)
+    _check(lib().w8a8_unpack_weight(_ptr(packed), N, K, _ptr(w), _stream(stream)),
+           "w8a8_unpack_weight")
+    return w
+
+
+def scaled_mm(q: torch.Tensor, a_scale: torch.Tensor, packed_w: torch.Tensor,
+              w_scale: torch.Tensor, bias: Optional[torch.Tensor], N: int,
+              out: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None,
+              stream=None) -> torch.Tensor:
+    """q int8 [M, K] x packed W -> y bf16 [M, N]."""
+    _need_cuda(q, "q", torch.int8)
+    M, K = q.shape
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.bfloat16, device=q.device)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(lib().w8a8_scaled_mm(_ptr(q), _ptr(a_scale), _ptr(packed_w), _ptr(w_scale), _ptr(bias),
+                                _ptr(out), M, N, K, _ptr(workspace), ws_bytes, _stream(stream)),
+           "w8a8_scaled_mm")
+    return out
+
+
+def scaled_mm_i32(q: torch.Tensor, packed_w: torch.Tensor, N: int,
+                  out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    _need_cuda(q, "q", torch.int8)
+    M, K = q.shape
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.int32, device=q.device)
+    _check(lib().w8a8_scaled_mm_i32(_ptr(q), _ptr(packed_w), _ptr(out), M, N, K, _stream(stream)),
+           "w8a8_scaled_mm_i32")
+    return out
+
+
+def linear(x: torch.Tensor, packed_w: torch.Tensor, w_scale: torch.Tensor,
+           bias: Optional[torch.Tensor], N: int, out: Optional[torch.Tensor] = None,
+           workspace: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """The whole layer: y[..., N] = W8A8(x[..., K])."""
+    _need_cuda(x, "x", torch.bfloat16)
+    lead = x.shape[:-1]
+    K = x.shape[-1]
+    x2 = x.reshape(-1, K)
+    if x2.stride(1) != 1:
+        x2 = x2.contiguous()
+    M = x2.shape[0]
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.bfloat16, device=x.device)
+    need = linear_workspace_bytes(M, N, K)
+    if workspace is None:
+        workspace = torch.empty((need,), dtype=torch.uint8, device=x.device)
+    ws_bytes = workspace.numel() * workspace.element_size()
+    _check(lib().w8a8_linear(_ptr(x2), x2.stride(0), _ptr(packed_w), _ptr(w_scale), _ptr(bias),
+                             _ptr(out), M, N, K, _ptr(workspace), ws_bytes, _stream(stream)),
+           "w8a8_linear")
+    return out.view(*lead, N)
+
+
+def gelu_tanh(x: torch.Tensor, out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    _need_cuda(x, "x", torch.bfloat16)
+    x = x.contiguous()
+    if out is None:
+        out = torch.empty_like(x)
+    _check(lib().w8a8_gelu_tanh(_ptr(x), _ptr(out), x.numel(), _stream(stream)), "w8a8_gelu_tanh")
+    return out
+
+
+def set_path(path: int):
+    _check(lib().w8a8_set_path(path), "w8a8_set_path")
+
+
+def poll_status(stream=None) -> int:
+    return int(lib().w8a8_poll_status(_stream(stream)))
+
+
+def selftest_wait_timeout(timeout_ns: int, stream=None):
+    _check(lib().w8a8_selftest_wait_timeout(timeout_ns, _stream(stream)), "w8a8_selftest_wait_timeout")
+
+
+def launch_count() -> int:
+    return int(lib().w8a8_launch_count())
+
+
+class W8A8Linear:
+    """A pre-quantised linear layer: int8 weights [N, K] packed once at load
+    time ("load -> transpose-repack -> apply"), fp32 per-output-channel
+    scales, optional bf16 bias.  For fused Q/K/V, build it from the three
+    blocks with :meth:`from_blocks` and split the output with :meth:`split`.
+    """
+
+    def __init__(self, w: torch.Tensor, w_scale: torch.Tensor, bias: Optional[torch.Tensor] = None,
+                 splits: Optional[Tuple[int, ...]] = None):
+        _need_cuda(w, "w", torch.int8)
+        self.N, self.K = w.shape
+        self.packed = pack_weight(w)
+        self.w_scale = w_scale.to(device=w.device, dtype=torch.float32).contiguous()
+        self.bias = None if bias is None else bias.to(device=w.device, dtype=torch.bfloat16).contiguous()
+        self.splits = tuple(splits) if splits else (self.N,)
+        self._ws = None
+
+    @classmethod
+    def from_blocks(cls, blocks, scales, biases=None):
+        w = torch.cat(list(blocks), dim=0)
+        s = torch.cat(list(scales), dim=0)
+        b = None if biases is None else torch.cat(list(biases), dim=0)
+        return cls(w, s, b, splits=tuple(int(t.shape[0]) for t in blocks))
+
+    def __call__(self, x: torch.Tensor) -> torch.Tensor:
+        M = x.numel() // x.shape[-1]
+        need = linear_workspace_bytes(M, self.N, self.K)
+        if self._ws is None or self._ws.numel() < need or self._ws.device != x.device:
+            self._ws = torch.empty((need,), dtype=torch.uint8, device=x.device)
+        return linear(x, self.packed, self.w_scale, self.bias, self.N, workspace=self._ws)
+
+    def split(self, y: torch.Tensor):
+        return torch.split(y, list(self.splits), dim=-1)

@@ -1,0 +1,66 @@
+// gelu.cu -- GELU (tanh form), bf16 -> bf16, fp32 arithmetic.
+//
+// Not part of the method on the pages: it joins the up- and down-projections
+// of the DiT MLP workload (image-token-scale transformer block), so that the
+// down-projection is fed what a real block feeds it.  HBM-bound, 4 bytes per
+// element; 8 elements per thread with 128-bit loads and stores.
+#include <cuda_bf16.h>
+
+#include "internal.h"
+
+namespace w8a8 {
+namespace {
+
+// GELU_tanh(x) = 0.5 x (1 + tanh(u)), u = sqrt(2/pi)(x + 0.044715 x^3),
+// evaluated as x * sigma(2u) (the same function: 0.5(1 + tanh(u)) = 1/(1 + e^-2u)),
+// with sigma written so nothing cancels: 1 + tanh(u) in fp32 is exactly 0
+// once tanh(u) rounds to -1 (u < -9), which would flush whole ranges of
+// small negative outputs to -0.
+__device__ __forceinline__ float gelu_f(float x) {
+  const float c = 0.7978845608028654f;  // sqrt(2 / pi)
+  const float u = c * (x + 0.044715f * x * x * x);
+  const float e = expf(-2.0f * fabsf(u));  // in (0, 1]
+  const float sig = u >= 0.0f ? 1.0f / (1.0f + e) : e / (1.0f + e);
+  return x * sig;
+}
+
+__device__ __forceinline__ uint32_t gelu2(uint32_t v) {
+  const float a = gelu_f(__uint_as_float(v << 16));
+  const float b = gelu_f(__uint_as_float(v & 0xFFFF0000u));
+  const __nv_bfloat162 r = __floats2bfloat162_rn(a, b);
+  return *reinterpret_cast<const uint32_t *>(&r);
+}
+
+__global__ void gelu_kernel(const uint4 *__restrict__ x, uint4 *__restrict__ y, int64_t n8,
+                            const uint16_t *__restrict__ xt, uint16_t *__restrict__ yt,
+                            int64_t tail) {
+  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n8;
+       i += (int64_t)gridDim.x * blockDim.x) {
+    const uint4 v = x[i];
+    y[i] = make_uint4(gelu2(v.x), gelu2(v.y), gelu2(v.z), gelu2(v.w));
+  }
+  if (blockIdx.x == 0 && threadIdx.x < tail) {
+    const float a = gelu_f(__uint_as_float((uint32_t)xt[threadIdx.x] << 16));
+    const __nv_bfloat16 r = __float2bfloat16_rn(a);
+    yt[threadIdx.x] = *reinterpret_cast<const uint16_t *>(&r);
+  }
+}
+
+}  // namespace
+}  // namespace w8a8
+
+using namespace w8a8;
+
+extern "C" w8a8_status w8a8_gelu_tanh(const void *x, void *y, int64_t n, w8a8_stream_t stream) {
+  if (!x || !y || n < 0) return W8A8_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(y)) return W8A8_ERR_ALIGNMENT;
+  if (n == 0) return W8A8_OK;
+  const int64_t n8 = n / 8, tail = n % 8;
+  const int64_t blocks =
+      std::max<int64_t>(1, std::min<int64_t>((n8 + 255) / 256, (int64_t)sm_count() * 8));
+  gelu_kernel<<<(unsigned)blocks, 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+      static_cast<const uint4 *>(x), static_cast<uint4 *>(y), n8,
+      static_cast<const uint16_t *>(x) + n8 * 8, static_cast<uint16_t *>(y) + n8 * 8, tail);
+  count_launch();
+  return from_cuda(cudaGetLastError());
+}

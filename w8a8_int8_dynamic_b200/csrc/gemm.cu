@@ -1,0 +1,823 @@
+// gemm.cu -- int8 x int8 -> int32 GEMM on the sm_100a tensor cores with the
+// dequantising epilogue, plus the fused quantise+GEMM layer entry point.
+//
+// Source: "Issue 5 probe: int8 quantized DiT serve paths on the RTX 3090",
+// Round two: the cutlass_scaled_mm op (int8 activations x int8 weights,
+// per-token and per-output-channel fp32 scales, bf16 out), fused Q/K/V and
+// row-parallel layer shapes.  "INT8 Quant for Dual-Max Recipe": W8A8 runs
+// int8 x int8 natively on the integer tensor cores, weights never
+// dequantised; prefill is compute-bound, decode is weight-bandwidth-bound.
+//
+//   acc[m,n] = sum_k q[m,k] w[n,k]                     (exact int32, TMEM)
+//   y[m,n]   = bf16_rne(((float)acc * a_scale[m]) * w_scale[n] + bias[n])
+//
+// Two kernels share the tile image, descriptors and epilogue arithmetic:
+//
+// 1. gemm_kernel (large M): persistent, one CTA per SM, 192 threads.
+//    warp 0: producer -- TMA 2-D load of the q tile (128 rows x 128 bytes,
+//            128-byte swizzle) and a 16 KB bulk copy per 128-row weight slab
+//            from the packed image, onto a STAGES-deep mbarrier ring;
+//    warp 1: MMA issuer -- 4 x tcgen05.mma.kind::i8 (M=128, N=BN, K=32) per
+//            stage, int32 accumulators in TMEM, double-buffered so the
+//            epilogue of tile i overlaps the main loop of tile i+1;
+//    warps 2-5: epilogue -- tcgen05.ld of 32 columns at a time, the scale /
+//            bias arithmetic in fp32 (each step rounded separately, so the
+//            result is bit-identical to the definition), bf16 stores.
+// 2. decode_kernel (small M <= 16, weight streaming): swap-AB -- the weight
+//    tile is the MMA's M=128 operand and the (zero-padded) 16 activation rows
+//    are its N=16 operand, so the tensor core consumes W straight from the
+//    packed image.  The (128-row block, 128-byte k-block) units are split
+//    evenly over all SMs (stream-K); a 128-row block whose K range spans
+//    several CTAs is finished by the last CTA to arrive (atomic counter),
+//    which adds the others' int32 partials (exact, order-free) and runs the
+//    epilogue.  Nothing ever waits on another CTA.
+//
+// Every mbarrier wait is time-bounded (ptx.cuh); a wait that gives up sets
+// the device status word to W8A8_ERR_TIMEOUT and the block drains and exits.
+#include <cuda_bf16.h>
+
+#include <algorithm>
+
+#include "internal.h"
+#include "ptx.cuh"
+
+namespace w8a8 {
+namespace {
+
+constexpr int kBM = 128;                 // tile rows (MMA M)
+constexpr int kBK = 128;                 // bytes of K per pipeline stage
+constexpr int kTileBytes = 128 * kBK;    // one 128 x 128 int8 tile = 16 KB
+constexpr int kThreads = 192;            // 6 warps
+constexpr int kDecodeNT = 16;            // activation rows per decode MMA (N)
+
+struct GemmArgs {
+  const uint8_t *packed_w;
+  const float *a_scale;
+  const float *w_scale;
+  const uint16_t *bias;  // may be null
+  void *out;             // bf16 [M, N] or int32 [M, N]
+  int M, N;
+  int num_kb;            // K blocks of 128 bytes (= packed K / 128)
+  int tiles_m, tiles_n;
+  int *status;
+};
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  const __nv_bfloat162 r = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<const uint32_t *>(&r);
+}
+
+__device__ __forceinline__ float dequant(int32_t acc, float as, float ws) {
+  return __fmul_rn(__fmul_rn(__int2float_rn(acc), as), ws);
+}
+
+// ============================================================================
+// Large-M persistent GEMM
+// ============================================================================
+template <int BN, int STAGES>
+struct LargeSmem {
+  static constexpr int kA = 0;
+  static constexpr int kB = STAGES * kTileBytes;
+  static constexpr int kBars = kB + STAGES * BN * kBK;  // full[S], empty[S], tfull[2], tempty[2], mma_done
+  static constexpr int kMisc = kBars + (2 * STAGES + 5) * 8;
+  static constexpr int kUsed = kMisc + 16;
+  static constexpr int kAlloc = kUsed + 1024;  // slack for 1024-byte alignment
+};
+
+template <int BN, bool OUT_I32>
+__device__ __forceinline__ void epilogue_tile(const GemmArgs &a, uint32_t tmem_cols, int quarter,
+                                              int lane, int mb, int nb) {
+  const int row = mb * kBM + quarter * 32 + lane;
+  const bool row_ok = row < a.M;
+  const float as = (!OUT_I32 && row_ok) ? __ldg(a.a_scale + row) : 0.0f;
+  const uint32_t taddr = tmem_cols + ((uint32_t)(quarter * 32) << 16);
+#pragma unroll 1
+  for (int c = 0; c < BN / 32; ++c) {
+    const int n0 = nb * BN + c * 32;
+    if (n0 >= a.N) break;  // uniform across the warp
+    uint32_t r[32];
+    tmem_ld_32x32b_x32(taddr + c * 32, r);
+    tmem_ld_wait();
+    if (OUT_I32) {
+      if (row_ok) {
+        int32_t *dst = static_cast<int32_t *>(a.out) + (int64_t)row * a.N + n0;
+#pragma unroll
+        for (int g = 0; g < 8; ++g)
+          if (n0 + 4 * g < a.N)
+            *reinterpret_cast<uint4 *>(dst + 4 * g) =
+                make_uint4(r[4 * g], r[4 * g + 1], r[4 * g + 2], r[4 * g + 3]);
+      }
+    } else {
+#pragma unroll
+      for (int g = 0; g < 4; ++g) {
+        const int nn = n0 + 8 * g;
+        if (nn >= a.N) break;  // N % 8 == 0: groups of 8 are all in or all out
+        const float4 w0 = __ldg(reinterpret_cast<const float4 *>(a.w_scale + nn));
+        const float4 w1 = __ldg(reinterpret_cast<const float4 *>(a.w_scale + nn + 4));
+        float t[8];
+        t[0] = dequant((int32_t)r[8 * g + 0], as, w0.x);
+        t[1] = dequant((int32_t)r[8 * g + 1], as, w0.y);
+        t[2] = dequant((int32_t)r[8 * g + 2], as, w0.z);
+        t[3] = dequant((int32_t)r[8 * g + 3], as, w0.w);
+        t[4] = dequant((int32_t)r[8 * g + 4], as, w1.x);
+        t[5] = dequant((int32_t)r[8 * g + 5], as, w1.y);
+        t[6] = dequant((int32_t)r[8 * g + 6], as, w1.z);
+        t[7] = dequant((int32_t)r[8 * g + 7], as, w1.w);
+        if (a.bias) {
+          const uint4 b = __ldg(reinterpret_cast<const uint4 *>(a.bias + nn));
+          const uint32_t bw[4] = {b.x, b.y, b.z, b.w};
+#pragma unroll
+          for (int h = 0; h < 4; ++h) {
+            t[2 * h] = __fadd_rn(t[2 * h], __uint_as_float(bw[h] << 16));
+            t[2 * h + 1] = __fadd_rn(t[2 * h + 1], __uint_as_float(bw[h] & 0xFFFF0000u));
+          }
+        }
+        if (row_ok) {
+          uint16_t *dst = static_cast<uint16_t *>(a.out) + (int64_t)row * a.N + nn;
+          *reinterpret_cast<uint4 *>(dst) =
+              make_uint4(pack_bf16x2(t[0], t[1]), pack_bf16x2(t[2], t[3]),
+                         pack_bf16x2(t[4], t[5]), pack_bf16x2(t[6], t[7]));
+        }
+      }
+    }
+  }
+}
+
+template <int BN, int STAGES, bool OUT_I32>
+__global__ void __launch_bounds__(kThreads, 1)
+    gemm_kernel(const __grid_constant__ CUtensorMap tmap_q, const GemmArgs args) {
+  using L = LargeSmem<BN, STAGES>;
+  constexpr uint32_t kTmemCols = 2 * BN;  // two accumulator buffers
+  constexpr uint32_t kStageBytes = kTileBytes + BN * kBK;
+  constexpr uint32_t kIdesc = idesc_i8(kBM, BN);
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint8_t *sA = smem + L::kA;
+  uint8_t *sB = smem + L::kB;
+  uint64_t *full = reinterpret_cast<uint64_t *>(smem + L::kBars);
+  uint64_t *empty = full + STAGES;
+  uint64_t *tfull = empty + STAGES;
+  uint64_t *tempty = tfull + 2;
+  uint64_t *mma_done = tempty + 2;
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + L::kMisc);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + L::kMisc + 4);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&tfull[b], 1);
+      mbar_init(&tempty[b], 4);  // one arrival per epilogue warp
+    }
+    mbar_init(mma_done, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 0 && lane == 0) prefetch_tmap(&tmap_q);
+  if (warp == 1) tmem_alloc(tmem_slot, kTmemCols);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  // Inputs written by the preceding kernel of the stream are visible from here.
+  griddep_wait();
+
+  const int num_tiles = args.tiles_m * args.tiles_n;
+  const int num_kb = args.num_kb;
+
+  // Roles run as whole warps (so every warp reaches the block barriers
+  // converged); lane 0 waits and issues, and shares each wait's outcome.
+  if (warp == 0) {
+    // ---------------- producer ----------------
+    uint32_t it = 0;
+    uint32_t last_par[STAGES];
+    uint32_t issued = 0;
+    bool ok = true;
+    for (int tile = blockIdx.x; ok && tile < num_tiles; tile += gridDim.x) {
+      const int mb = tile % args.tiles_m, nb = tile / args.tiles_m;
+      const uint8_t *wslab = args.packed_w + (size_t)nb * (BN / 128) * num_kb * kTileBytes;
+      for (int kb = 0; kb < num_kb; ++kb, ++it) {
+        const uint32_t s = it % STAGES, ph = (it / STAGES) & 1;
+        int w_ok = 0;
+        if (lane == 0) w_ok = mbar_wait_bounded(&empty[s], ph ^ 1, abort_flag, args.status);
+        if (!__shfl_sync(0xFFFFFFFFu, w_ok, 0)) {
+          ok = false;
+          break;
+        }
+        if (lane == 0) {
+          mbar_arrive_expect_tx(&full[s], kStageBytes);
+          tma_load_2d(sA + s * kTileBytes, &tmap_q, kb * kBK, mb * kBM, &full[s]);
+#pragma unroll
+          for (int h = 0; h < BN / 128; ++h)
+            bulk_load(sB + s * (BN * kBK) + h * kTileBytes,
+                      wslab + ((size_t)h * num_kb + kb) * kTileBytes, kTileBytes, &full[s]);
+        }
+        __syncwarp();
+        last_par[s] = ph;
+        ++issued;
+      }
+    }
+    if (!ok && lane == 0) {
+      // Drain: wait (bounded) for the copies still in flight into our smem.
+      const uint32_t n = issued < STAGES ? issued : STAGES;
+      for (uint32_t s = 0; s < n; ++s) {
+        volatile int no_abort = 0;
+        (void)mbar_wait_bounded(&full[s], last_par[s], &no_abort, args.status);
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ---------------- MMA issuer ----------------
+    uint32_t it = 0, t_local = 0;
+    bool ok = true;
+    for (int tile = blockIdx.x; ok && tile < num_tiles; tile += gridDim.x, ++t_local) {
+      const uint32_t b = t_local & 1, bph = (t_local >> 1) & 1;
+      int w_ok = 0;
+      if (lane == 0) w_ok = mbar_wait_bounded(&tempty[b], bph ^ 1, abort_flag, args.status);
+      if (!__shfl_sync(0xFFFFFFFFu, w_ok, 0)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      const uint32_t d_tmem = tmem_base + b * BN;
+      for (int kb = 0; kb < num_kb; ++kb, ++it) {
+        const uint32_t s = it % STAGES, ph = (it / STAGES) & 1;
+        if (lane == 0) w_ok = mbar_wait_bounded(&full[s], ph, abort_flag, args.status);
+        if (!__shfl_sync(0xFFFFFFFFu, w_ok, 0)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        if (lane == 0) {
+          const uint64_t a_desc = sw128_kmajor_desc(sA + s * kTileBytes);
+          const uint64_t b_desc = sw128_kmajor_desc(sB + s * (BN * kBK));
+#pragma unroll
+          for (int k = 0; k < kBK / 32; ++k)
+            mma_i8(d_tmem, a_desc + 2 * k, b_desc + 2 * k, kIdesc, (kb | k) != 0);
+          mma_commit(&empty[s]);  // frees the stage when these MMAs finish
+        }
+        __syncwarp();
+      }
+      if (ok && lane == 0) mma_commit(&tfull[b]);
+      __syncwarp();
+    }
+    if (!ok && lane == 0) {
+      // Wait (bounded) for MMAs still in flight before TMEM is released.
+      mma_commit(mma_done);
+      volatile int no_abort = 0;
+      (void)mbar_wait_bounded(mma_done, 0, &no_abort, args.status);
+    }
+    __syncwarp();
+  } else {
+    // ---------------- epilogue (warps 2..5) ----------------
+    const int quarter = warp & 3;  // TMEM lanes this warp may access
+    uint32_t t_local = 0;
+    for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++t_local) {
+      const uint32_t b = t_local & 1, bph = (t_local >> 1) & 1;
+      int ok = 0;
+      if (lane == 0) ok = mbar_wait_bounded(&tfull[b], bph, abort_flag, args.status);
+      ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
+      if (!ok) break;
+      tc_fence_after();
+      const int mb = tile % args.tiles_m, nb = tile / args.tiles_m;
+      epilogue_tile<BN, OUT_I32>(args, tmem_base + b * BN, quarter, lane, mb, nb);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&tempty[b]);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, kTmemCols);
+  }
+}
+
+// ============================================================================
+// Small-M (decode) swap-AB stream-K kernel
+// ============================================================================
+template <int STAGES>
+struct DecodeSmem {
+  static constexpr int kW = 0;                                  // STAGES x 16 KB weight tiles
+  static constexpr int kQ = STAGES * kTileBytes;                // STAGES x 2 KB activation tiles
+  static constexpr int kBars = kQ + STAGES * kDecodeNT * kBK;   // full, empty, tfull[2], tempty[2], done
+  static constexpr int kMisc = kBars + (2 * STAGES + 5) * 8;
+  static constexpr int kUsed = kMisc + 32;
+  static constexpr int kAlloc = kUsed + 1024;
+};
+
+struct DecodeArgs {
+  const uint8_t *packed_w;
+  const float *a_scale;
+  const float *w_scale;
+  const uint16_t *bias;
+  uint16_t *y;
+  int M, N;
+  int num_kb;          // k blocks per 128-row slab
+  int num_nb;          // 128-row slabs covering N
+  int64_t units;       // num_nb * num_kb
+  int max_contrib;     // partial slots per slab
+  int32_t *partials;   // [num_nb][max_contrib][128][16]
+  uint32_t *counters;  // [num_nb], zero on entry
+  int *status;
+};
+
+__device__ __forceinline__ int64_t unit_begin(int64_t units, int grid, int c) {
+  return units * c / grid;
+}
+
+// First CTA whose unit range contains unit u (ranges are [begin(c), begin(c+1))).
+__device__ __forceinline__ int cta_of_unit(int64_t units, int grid, int64_t u) {
+  int c = (int)((u * grid) / units);
+  while (c + 1 < grid && unit_begin(units, grid, c + 1) <= u) ++c;
+  while (c > 0 && unit_begin(units, grid, c) > u) --c;
+  return c;
+}
+
+template <int STAGES>
+__global__ void __launch_bounds__(kThreads, 1)
+    decode_kernel(const __grid_constant__ CUtensorMap tmap_q, const DecodeArgs args) {
+  using L = DecodeSmem<STAGES>;
+  constexpr uint32_t kTmemCols = 32;  // two 16-column accumulators
+  constexpr uint32_t kQBytes = kDecodeNT * kBK;
+  constexpr uint32_t kStageBytes = kTileBytes + kQBytes;
+  constexpr uint32_t kIdesc = idesc_i8(kBM, kDecodeNT);
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint8_t *sW = smem + L::kW;
+  uint8_t *sQ = smem + L::kQ;
+  uint64_t *full = reinterpret_cast<uint64_t *>(smem + L::kBars);
+  uint64_t *empty = full + STAGES;
+  uint64_t *tfull = empty + STAGES;
+  uint64_t *tempty = tfull + 2;
+  uint64_t *mma_done = tempty + 2;
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + L::kMisc);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + L::kMisc + 4);
+  volatile int *last_flag = reinterpret_cast<volatile int *>(smem + L::kMisc + 8);
+  volatile int *seg_ok = reinterpret_cast<volatile int *>(smem + L::kMisc + 16);  // [2]
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&tfull[b], 1);
+      mbar_init(&tempty[b], 4);
+    }
+    mbar_init(mma_done, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 0 && lane == 0) prefetch_tmap(&tmap_q);
+  if (warp == 1) tmem_alloc(tmem_slot, kTmemCols);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  const uint64_t evict_first = policy_evict_first();
+  const int64_t u_begin = unit_begin(args.units, gridDim.x, blockIdx.x);
+  const int64_t u_end = unit_begin(args.units, gridDim.x, blockIdx.x + 1);
+  const int nkb = args.num_kb;
+
+  if (warp == 0) {
+    // ---------------- producer (whole warp; lane 0 issues) ----------------
+    // The weight stream does not depend on the preceding kernel: start it
+    // before waiting for the activations.
+    uint32_t it = 0, issued = 0;
+    uint32_t last_par[STAGES];
+    bool ok = true, waited = false;
+    for (int64_t u = u_begin; u < u_end; ++u, ++it) {
+      const uint32_t s = it % STAGES, ph = (it / STAGES) & 1;
+      int w_ok = 0;
+      if (lane == 0) w_ok = mbar_wait_bounded(&empty[s], ph ^ 1, abort_flag, args.status);
+      if (!__shfl_sync(0xFFFFFFFFu, w_ok, 0)) {
+        ok = false;
+        break;
+      }
+      const int kb = (int)(u % nkb);
+      if (lane == 0) {
+        mbar_arrive_expect_tx(&full[s], kStageBytes);
+        bulk_load_hint(sW + s * kTileBytes, args.packed_w + (size_t)u * kTileBytes, kTileBytes,
+                       &full[s], evict_first);
+      }
+      if (!waited) {
+        griddep_wait();
+        waited = true;
+      }
+      if (lane == 0) tma_load_2d(sQ + s * kQBytes, &tmap_q, kb * kBK, 0, &full[s]);
+      __syncwarp();
+      last_par[s] = ph;
+      ++issued;
+    }
+    if (!waited) griddep_wait();
+    if (!ok && lane == 0) {
+      const uint32_t n = issued < STAGES ? issued : STAGES;
+      for (uint32_t s = 0; s < n; ++s) {
+        volatile int no_abort = 0;
+        (void)mbar_wait_bounded(&full[s], last_par[s], &no_abort, args.status);
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ---------------- MMA issuer (whole warp; lane 0 issues) ----------------
+    uint32_t it = 0, seg = 0;
+    bool ok = true;
+    int64_t u = u_begin;
+    while (ok && u < u_end) {
+      const int nb = (int)(u / nkb);
+      const int64_t seg_end = std::min<int64_t>(u_end, (int64_t)(nb + 1) * nkb);
+      const uint32_t b = seg & 1, bph = (seg >> 1) & 1;
+      int w_ok = 0;
+      if (lane == 0) w_ok = mbar_wait_bounded(&tempty[b], bph ^ 1, abort_flag, args.status);
+      if (!__shfl_sync(0xFFFFFFFFu, w_ok, 0)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      const uint32_t d_tmem = tmem_base + b * kDecodeNT;
+      bool first = true;
+      for (; u < seg_end; ++u, ++it) {
+        const uint32_t s = it % STAGES, ph = (it / STAGES) & 1;
+        if (lane == 0) w_ok = mbar_wait_bounded(&full[s], ph, abort_flag, args.status);
+        if (!__shfl_sync(0xFFFFFFFFu, w_ok, 0)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        if (lane == 0) {
+          const uint64_t a_desc = sw128_kmajor_desc(sW + s * kTileBytes);
+          const uint64_t b_desc = sw128_kmajor_desc(sQ + s * kQBytes);
+#pragma unroll
+          for (int k = 0; k < kBK / 32; ++k)
+            mma_i8(d_tmem, a_desc + 2 * k, b_desc + 2 * k, kIdesc, (first && k == 0) ? 0u : 1u);
+          mma_commit(&empty[s]);
+        }
+        __syncwarp();
+        first = false;
+      }
+      if (ok && lane == 0) mma_commit(&tfull[b]);
+      __syncwarp();
+      ++seg;
+    }
+    if (!ok && lane == 0) {
+      mma_commit(mma_done);
+      volatile int no_abort = 0;
+      (void)mbar_wait_bounded(mma_done, 0, &no_abort, args.status);
+    }
+    __syncwarp();
+  } else {
+    // ---------------- epilogue (warps 2..5): one output channel per thread ----
+    // The four warps take every decision together: thread 0 of the group
+    // waits on the barrier and publishes the outcome behind a named barrier,
+    // so no warp can be left alone at a later named barrier.
+    griddep_wait();  // a_scale may come from the preceding kernel
+    const int quarter = warp & 3;
+    const int et = threadIdx.x - 64;  // 0..127
+    uint32_t seg = 0;
+    int64_t u = u_begin;
+    while (u < u_end) {
+      const int nb = (int)(u / nkb);
+      const int64_t slab_begin = (int64_t)nb * nkb, slab_end = slab_begin + nkb;
+      const int64_t seg_end = std::min<int64_t>(u_end, slab_end);
+      const bool whole = (u == slab_begin) && (seg_end == slab_end);
+      const uint32_t b = seg & 1, bph = (seg >> 1) & 1;
+      if (et == 0) seg_ok[b] = mbar_wait_bounded(&tfull[b], bph, abort_flag, args.status) ? 1 : 0;
+      __syncwarp();
+      asm volatile("bar.sync 1, 128;" ::: "memory");
+      if (!seg_ok[b]) break;
+      tc_fence_after();
+      uint32_t r[kDecodeNT];
+      tmem_ld_32x32b_x16(tmem_base + ((uint32_t)(quarter * 32) << 16) + b * kDecodeNT, r);
+      tmem_ld_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&tempty[b]);
+
+      const int n_local = quarter * 32 + lane;  // TMEM lane = weight row in the slab
+      const int n = nb * 128 + n_local;
+      bool finish = whole;
+      if (!whole) {
+        // contributor rank of this CTA among the CTAs covering this slab
+        const int first_cta = cta_of_unit(args.units, gridDim.x, slab_begin);
+        const int last_cta = cta_of_unit(args.units, gridDim.x, slab_end - 1);
+        const int contributors = last_cta - first_cta + 1;
+        const int rank = blockIdx.x - first_cta;
+        int32_t *slot = args.partials +
+                        ((size_t)nb * args.max_contrib + rank) * (128 * kDecodeNT) + n_local;
+#pragma unroll
+        for (int m = 0; m < kDecodeNT; ++m) slot[m * 128] = (int32_t)r[m];
+        __threadfence();
+        __syncwarp();
+        asm volatile("bar.sync 1, 128;" ::: "memory");
+        if (et == 0) {
+          const uint32_t prev = atomicAdd(args.counters + nb, 1u);
+          const bool last = prev + 1 == (uint32_t)contributors;
+          if (last) args.counters[nb] = 0;  // leave it clean for the next call
+          *last_flag = last ? 1 : 0;
+        }
+        __syncwarp();
+        asm volatile("bar.sync 1, 128;" ::: "memory");
+        finish = *last_flag != 0;
+        if (finish) {
+          __threadfence();
+          int32_t sum[kDecodeNT];
+#pragma unroll
+          for (int m = 0; m < kDecodeNT; ++m) sum[m] = 0;
+          for (int c = 0; c < contributors; ++c) {
+            const int32_t *o = args.partials +
+                               ((size_t)nb * args.max_contrib + c) * (128 * kDecodeNT) + n_local;
+#pragma unroll
+            for (int m = 0; m < kDecodeNT; ++m) sum[m] += __ldcg(o + m * 128);
+          }
+#pragma unroll
+          for (int m = 0; m < kDecodeNT; ++m) r[m] = (uint32_t)sum[m];
+        }
+      }
+      if (finish && n < args.N) {
+        const float ws = __ldg(args.w_scale + n);
+        const float bv = args.bias ? __uint_as_float((uint32_t)__ldg(args.bias + n) << 16) : 0.0f;
+#pragma unroll
+        for (int m = 0; m < kDecodeNT; ++m) {
+          if (m < args.M) {
+            float t = dequant((int32_t)r[m], __ldg(args.a_scale + m), ws);
+            if (args.bias) t = __fadd_rn(t, bv);
+            const __nv_bfloat16 h = __float2bfloat16_rn(t);
+            args.y[(int64_t)m * args.N + n] = *reinterpret_cast<const uint16_t *>(&h);
+          }
+        }
+      }
+      u = seg_end;
+      ++seg;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, kTmemCols);
+  }
+}
+
+// ============================================================================
+// host side
+// ============================================================================
+constexpr int kLargeStages128 = 6;
+constexpr int kLargeStages256 = 4;
+constexpr int kDecodeStages = 10;
+
+bool g_attr_done[64][8];
+
+template <typename Kernel>
+cudaError_t set_smem_attr(Kernel k, int bytes, int slot) {
+  const int d = current_device();
+  if (d >= 0 && d < 64 && g_attr_done[d][slot]) return cudaSuccess;
+  cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e == cudaSuccess && d >= 0 && d < 64) g_attr_done[d][slot] = true;
+  return e;
+}
+
+template <typename Kernel, typename Args>
+cudaError_t launch_ex(Kernel k, int grid, int smem, cudaStream_t stream, bool pdl,
+                      const CUtensorMap &tmap, const Args &args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)grid);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = (size_t)smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = pdl ? attr : nullptr;
+  cfg.numAttrs = pdl ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, k, tmap, args);
+}
+
+template <int BN, int STAGES, bool OUT_I32>
+w8a8_status run_large(const CUtensorMap &tmap, GemmArgs args, cudaStream_t stream, bool pdl,
+                      int slot) {
+  using L = LargeSmem<BN, STAGES>;
+  auto k = gemm_kernel<BN, STAGES, OUT_I32>;
+  cudaError_t e = set_smem_attr(k, L::kAlloc, slot);
+  if (e != cudaSuccess) return W8A8_ERR_CUDA;
+  args.tiles_n = (int)((args.N + BN - 1) / BN);
+  const int tiles = args.tiles_m * args.tiles_n;
+  const int grid = std::min(tiles, sm_count());
+  e = launch_ex(k, grid, L::kAlloc, stream, pdl, tmap, args);
+  count_launch();
+  return from_cuda(e);
+}
+
+// Tile width for the large-M kernel: fewest waves x tile time, with the
+// narrower tile charged for its lower tensor-pipe efficiency.
+int choose_bn(int64_t M, int64_t N) {
+  const int path = forced_path();
+  if (path == 3) return 128;
+  if (path == 4) return 256;
+  const int64_t sms = sm_count();
+  const int64_t tm = (M + kBM - 1) / kBM;
+  const int64_t t128 = tm * ((N + 127) / 128), t256 = tm * ((N + 255) / 256);
+  const double c128 = (double)((t128 + sms - 1) / sms) * 128.0 / 0.85;
+  const double c256 = (double)((t256 + sms - 1) / sms) * 256.0;
+  return c256 <= c128 ? 256 : 128;
+}
+
+}  // namespace
+
+// Decode workspace: counters + partial slots.
+static int64_t decode_units(int64_t N, int64_t K) {
+  return (packed_rows(N) / 128) * (packed_cols(K) / 128);
+}
+
+static void decode_geometry(int64_t N, int64_t K, int *grid, int *max_contrib) {
+  const int64_t units = decode_units(N, K);
+  const int64_t g = std::min<int64_t>(units, sm_count());
+  const int64_t per = units / g;  // smallest range length
+  const int64_t nkb = packed_cols(K) / 128;
+  *grid = (int)g;
+  *max_contrib = (int)((nkb + per - 1) / per + 1);
+}
+
+int64_t decode_workspace_bytes(int64_t N, int64_t K) {
+  int grid, mc;
+  decode_geometry(N, K, &grid, &mc);
+  const int64_t nb = packed_rows(N) / 128;
+  const int64_t counters = round_up(nb * 4, 256);
+  return counters + nb * mc * 128 * kDecodeNT * 4;
+}
+
+bool use_decode_path(int64_t M) {
+  const int p = forced_path();
+  if (p == 2) return M <= kDecodeNT;
+  if (p == 1 || p == 3 || p == 4) return false;
+  return M <= kDecodeNT;
+}
+
+w8a8_status launch_decode(const int8_t *q, const float *a_scale, const void *packed_w,
+                          const float *w_scale, const void *bias, void *y, int64_t M,
+                          int64_t N, int64_t K, void *workspace, cudaStream_t stream, bool pdl) {
+  CUtensorMap tmap;
+  if (!make_tmap_u8_2d(&tmap, q, (uint64_t)M, (uint64_t)K, (uint64_t)K, kDecodeNT, kBK))
+    return W8A8_ERR_CUDA;
+  int grid, mc;
+  decode_geometry(N, K, &grid, &mc);
+  const int64_t nb = packed_rows(N) / 128;
+  uint8_t *ws = static_cast<uint8_t *>(workspace);
+  DecodeArgs a;
+  a.packed_w = static_cast<const uint8_t *>(packed_w);
+  a.a_scale = a_scale;
+  a.w_scale = w_scale;
+  a.bias = static_cast<const uint16_t *>(bias);
+  a.y = static_cast<uint16_t *>(y);
+  a.M = (int)M;
+  a.N = (int)N;
+  a.num_kb = (int)(packed_cols(K) / 128);
+  a.num_nb = (int)nb;
+  a.units = nb * a.num_kb;
+  a.max_contrib = mc;
+  a.counters = reinterpret_cast<uint32_t *>(ws);
+  a.partials = reinterpret_cast<int32_t *>(ws + round_up(nb * 4, 256));
+  a.status = status_word();
+  if (!a.status) return W8A8_ERR_CUDA;
+  cudaError_t e = cudaMemsetAsync(ws, 0, (size_t)nb * 4, stream);
+  if (e != cudaSuccess) return W8A8_ERR_CUDA;
+  using L = DecodeSmem<kDecodeStages>;
+  auto k = decode_kernel<kDecodeStages>;
+  e = set_smem_attr(k, L::kAlloc, 7);
+  if (e != cudaSuccess) return W8A8_ERR_CUDA;
+  // The memset sits between the producer of q and this kernel, so a
+  // programmatic launch would only overlap the memset; keep it plain.
+  (void)pdl;
+  e = launch_ex(k, grid, L::kAlloc, stream, false, tmap, a);
+  count_launch();
+  return from_cuda(e);
+}
+
+w8a8_status launch_scaled_mm(const int8_t *q, const float *a_scale, const void *packed_w,
+                             const float *w_scale, const void *bias, void *out, bool out_i32,
+                             int64_t M, int64_t N, int64_t K, cudaStream_t stream, bool pdl) {
+  CUtensorMap tmap;
+  if (!make_tmap_u8_2d(&tmap, q, (uint64_t)M, (uint64_t)K, (uint64_t)K, kBM, kBK))
+    return W8A8_ERR_CUDA;
+  GemmArgs a;
+  a.packed_w = static_cast<const uint8_t *>(packed_w);
+  a.a_scale = a_scale;
+  a.w_scale = w_scale;
+  a.bias = static_cast<const uint16_t *>(bias);
+  a.out = out;
+  a.M = (int)M;
+  a.N = (int)N;
+  a.num_kb = (int)(packed_cols(K) / 128);
+  a.tiles_m = (int)((M + kBM - 1) / kBM);
+  a.tiles_n = 0;
+  a.status = status_word();
+  if (!a.status) return W8A8_ERR_CUDA;
+  const int bn = choose_bn(M, N);
+  if (out_i32) {
+    return bn == 256 ? run_large<256, kLargeStages256, true>(tmap, a, stream, pdl, 0)
+                     : run_large<128, kLargeStages128, true>(tmap, a, stream, pdl, 1);
+  }
+  return bn == 256 ? run_large<256, kLargeStages256, false>(tmap, a, stream, pdl, 2)
+                   : run_large<128, kLargeStages128, false>(tmap, a, stream, pdl, 3);
+}
+
+static w8a8_status check_gemm_args(const void *q, const void *packed_w, const void *out,
+                                   int64_t M, int64_t N, int64_t K) {
+  if (!q || !packed_w || !out) return W8A8_ERR_INVALID_ARG;
+  if (M < 1 || M > 0x7FFFFFFF || N < 1 || K < 1) return W8A8_ERR_INVALID_ARG;
+  if (K % 16 != 0 || K > kMaxK || N % 8 != 0 || N > ((int64_t)1 << 30))
+    return W8A8_ERR_UNSUPPORTED_SHAPE;
+  if (!aligned16(q) || !aligned16(packed_w) || !aligned16(out)) return W8A8_ERR_ALIGNMENT;
+  return W8A8_OK;
+}
+
+}  // namespace w8a8
+
+using namespace w8a8;
+
+extern "C" {
+
+w8a8_status w8a8_scaled_mm_workspace_bytes(int64_t M, int64_t N, int64_t K, size_t *bytes) {
+  if (!bytes || M < 1 || N < 1 || K < 1) return W8A8_ERR_INVALID_ARG;
+  if (K % 16 != 0 || K > kMaxK || N % 8 != 0) return W8A8_ERR_UNSUPPORTED_SHAPE;
+  *bytes = M <= kDecodeNT ? (size_t)decode_workspace_bytes(N, K) : 0;
+  return W8A8_OK;
+}
+
+w8a8_status w8a8_scaled_mm(const int8_t *q, const float *a_scale, const void *packed_w,
+                           const float *w_scale, const void *bias, void *y, int64_t M, int64_t N,
+                           int64_t K, void *workspace, size_t ws_bytes, w8a8_stream_t stream) {
+  w8a8_status st = check_gemm_args(q, packed_w, y, M, N, K);
+  if (st != W8A8_OK) return st;
+  if (!a_scale || !w_scale) return W8A8_ERR_INVALID_ARG;
+  if (!aligned16(a_scale) || !aligned16(w_scale) || (bias && !aligned16(bias)))
+    return W8A8_ERR_ALIGNMENT;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (use_decode_path(M) && workspace) {
+    if (!aligned16(workspace)) return W8A8_ERR_ALIGNMENT;
+    if ((int64_t)ws_bytes < decode_workspace_bytes(N, K)) return W8A8_ERR_BUFFER_TOO_SMALL;
+    return launch_decode(q, a_scale, packed_w, w_scale, bias, y, M, N, K, workspace, s, false);
+  }
+  if (forced_path() == 2) return W8A8_ERR_INVALID_ARG;  // small path needs M <= 16 and a workspace
+  return launch_scaled_mm(q, a_scale, packed_w, w_scale, bias, y, false, M, N, K, s, false);
+}
+
+w8a8_status w8a8_scaled_mm_i32(const int8_t *q, const void *packed_w, int32_t *acc, int64_t M,
+                               int64_t N, int64_t K, w8a8_stream_t stream) {
+  w8a8_status st = check_gemm_args(q, packed_w, acc, M, N, K);
+  if (st != W8A8_OK) return st;
+  return launch_scaled_mm(q, nullptr, packed_w, nullptr, nullptr, acc, true, M, N, K,
+                          reinterpret_cast<cudaStream_t>(stream), false);
+}
+
+w8a8_status w8a8_linear_workspace_bytes(int64_t M, int64_t N, int64_t K, size_t *bytes) {
+  if (!bytes || M < 1 || N < 1 || K < 1) return W8A8_ERR_INVALID_ARG;
+  if (K % 16 != 0 || K > kMaxK || N % 8 != 0) return W8A8_ERR_UNSUPPORTED_SHAPE;
+  int64_t b = round_up(M * K, 256) + round_up(M * 4, 256);
+  if (M <= kDecodeNT) b += decode_workspace_bytes(N, K);
+  *bytes = (size_t)b;
+  return W8A8_OK;
+}
+
+w8a8_status w8a8_linear(const void *x, int64_t ldx, const void *packed_w, const float *w_scale,
+                        const void *bias, void *y, int64_t M, int64_t N, int64_t K,
+                        void *workspace, size_t ws_bytes, w8a8_stream_t stream) {
+  w8a8_status st = check_gemm_args(x, packed_w, y, M, N, K);
+  if (st != W8A8_OK) return st;
+  if (!w_scale || !workspace) return W8A8_ERR_INVALID_ARG;
+  if (ldx < K) return W8A8_ERR_INVALID_ARG;
+  if (ldx % 8 != 0 || !aligned16(w_scale) || !aligned16(workspace) ||
+      (bias && !aligned16(bias)))
+    return W8A8_ERR_ALIGNMENT;
+  size_t need = 0;
+  st = w8a8_linear_workspace_bytes(M, N, K, &need);
+  if (st != W8A8_OK) return st;
+  if (ws_bytes < need) return W8A8_ERR_BUFFER_TOO_SMALL;
+  uint8_t *ws = static_cast<uint8_t *>(workspace);
+  int8_t *q = reinterpret_cast<int8_t *>(ws);
+  float *a_scale = reinterpret_cast<float *>(ws + round_up(M * K, 256));
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  st = launch_quant(x, M, K, ldx, q, a_scale, s);
+  if (st != W8A8_OK) return st;
+  if (use_decode_path(M)) {
+    void *dws = ws + round_up(M * K, 256) + round_up(M * 4, 256);
+    return launch_decode(q, a_scale, packed_w, w_scale, bias, y, M, N, K, dws, s, true);
+  }
+  if (forced_path() == 2) return W8A8_ERR_INVALID_ARG;
+  return launch_scaled_mm(q, a_scale, packed_w, w_scale, bias, y, false, M, N, K, s, true);
+}
+
+}  // extern "C"

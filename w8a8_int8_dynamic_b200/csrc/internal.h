@@ -1,0 +1,55 @@
+// internal.h -- host-side helpers shared by the translation units of libw8a8.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "w8a8.h"
+
+namespace w8a8 {
+
+// Device pointer to this device's status word (0 = OK, else a w8a8_status).
+int *status_word();
+
+// Number of SMs of the current device (cached per device).
+int sm_count();
+
+// Current device ordinal (cached per host thread).
+int current_device();
+
+// Counts one kernel launch (for the benchmark's launch accounting).
+void count_launch(int n = 1);
+
+// Path override set by w8a8_set_path: 0 auto, 1 large-M GEMM, 2 small-M.
+int forced_path();
+
+// 2-D tiled tensor map over a row-major uint8 matrix [rows, cols] with row
+// stride ld bytes, box {box_cols, box_rows}, 128-byte swizzle, zero fill out
+// of bounds.  Returns false if the driver rejects it.
+bool make_tmap_u8_2d(CUtensorMap *map, const void *base, uint64_t rows, uint64_t cols,
+                     uint64_t ld, uint32_t box_rows, uint32_t box_cols);
+
+inline bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+inline w8a8_status from_cuda(cudaError_t e) { return e == cudaSuccess ? W8A8_OK : W8A8_ERR_CUDA; }
+
+// Size limits shared by the entry points.
+constexpr int64_t kMaxK = 131072;
+
+inline int64_t round_up(int64_t v, int64_t m) { return (v + m - 1) / m * m; }
+
+// Packed weight geometry: N padded to 256, K to 128; tiles of 128x128 bytes.
+inline int64_t packed_rows(int64_t N) { return round_up(N, 256); }
+inline int64_t packed_cols(int64_t K) { return round_up(K, 128); }
+
+// GEMM launchers (gemm.cu).
+w8a8_status launch_scaled_mm(const int8_t *q, const float *a_scale, const void *packed_w,
+                             const float *w_scale, const void *bias, void *out, bool out_i32,
+                             int64_t M, int64_t N, int64_t K, cudaStream_t stream, bool pdl);
+// Quantisation launcher (quant.cu).
+w8a8_status launch_quant(const void *x, int64_t M, int64_t K, int64_t ldx, int8_t *q,
+                         float *a_scale, cudaStream_t stream);
+
+}  // namespace w8a8

@@ -1,0 +1,160 @@
+// runtime.cu -- status word, error polling, device queries, tensor-map
+// encoding and the bounded-wait self-test of libw8a8.
+#include <atomic>
+#include <cudaTypedefs.h>
+#include <mutex>
+
+#include "internal.h"
+#include "ptx.cuh"
+
+namespace w8a8 {
+
+// One status word per device (module globals are instantiated per device).
+__device__ int g_status_word;
+
+namespace {
+constexpr int kMaxDevices = 64;
+int *g_status_ptr[kMaxDevices];
+int g_sm_count[kMaxDevices];
+std::mutex g_mu;
+std::atomic<int64_t> g_launches{0};
+std::atomic<int> g_forced_path{0};
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+}  // namespace
+
+int current_device() {
+  int d = 0;
+  cudaGetDevice(&d);
+  return d;
+}
+
+int *status_word() {
+  const int d = current_device();
+  if (d < 0 || d >= kMaxDevices) return nullptr;
+  if (!g_status_ptr[d]) {
+    std::lock_guard<std::mutex> lk(g_mu);
+    if (!g_status_ptr[d]) {
+      void *p = nullptr;
+      if (cudaGetSymbolAddress(&p, g_status_word) != cudaSuccess) return nullptr;
+      g_status_ptr[d] = static_cast<int *>(p);
+    }
+  }
+  return g_status_ptr[d];
+}
+
+int sm_count() {
+  const int d = current_device();
+  if (d < 0 || d >= kMaxDevices) return 148;
+  if (!g_sm_count[d]) {
+    int n = 0;
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, d);
+    g_sm_count[d] = n > 0 ? n : 148;
+  }
+  return g_sm_count[d];
+}
+
+void count_launch(int n) { g_launches.fetch_add(n, std::memory_order_relaxed); }
+
+int forced_path() { return g_forced_path.load(std::memory_order_relaxed); }
+
+bool make_tmap_u8_2d(CUtensorMap *map, const void *base, uint64_t rows, uint64_t cols,
+                     uint64_t ld, uint32_t box_rows, uint32_t box_cols) {
+  if (!g_encode) {
+    std::lock_guard<std::mutex> lk(g_mu);
+    if (!g_encode) {
+      void *fn = nullptr;
+      cudaDriverEntryPointQueryResult q;
+      if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) !=
+              cudaSuccess ||
+          q != cudaDriverEntryPointSuccess || !fn)
+        return false;
+      g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+    }
+  }
+  const cuuint64_t dims[2] = {cols, rows};
+  const cuuint64_t strides[1] = {ld};
+  const cuuint32_t box[2] = {box_cols, box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  const CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void *>(base),
+                              dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                              CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+// Waits on a barrier that nothing arrives at; the bounded wait must give up.
+__global__ void selftest_wait_kernel(int *status, uint64_t limit_ns) {
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    abort_flag = 0;
+    fence_barrier_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    // phase 0 never completes: the single expected arrival never comes
+    (void)mbar_wait_bounded(&bar, 0, &abort_flag, status, limit_ns);
+  }
+  __syncthreads();
+}
+
+}  // namespace w8a8
+
+using namespace w8a8;
+
+extern "C" {
+
+const char *w8a8_status_string(int status) {
+  switch (status) {
+    case W8A8_OK: return "W8A8_OK";
+    case W8A8_ERR_INVALID_ARG: return "W8A8_ERR_INVALID_ARG";
+    case W8A8_ERR_ALIGNMENT: return "W8A8_ERR_ALIGNMENT";
+    case W8A8_ERR_UNSUPPORTED_SHAPE: return "W8A8_ERR_UNSUPPORTED_SHAPE";
+    case W8A8_ERR_CUDA: return "W8A8_ERR_CUDA";
+    case W8A8_ERR_TIMEOUT: return "W8A8_ERR_TIMEOUT";
+    case W8A8_ERR_BUFFER_TOO_SMALL: return "W8A8_ERR_BUFFER_TOO_SMALL";
+    default: return "W8A8_ERR_UNKNOWN";
+  }
+}
+
+int w8a8_abi_version(void) { return (1 << 16) | 0; }
+
+w8a8_status w8a8_set_path(int path) {
+  if (path < 0 || path > 4) return W8A8_ERR_INVALID_ARG;
+  g_forced_path.store(path);
+  return W8A8_OK;
+}
+
+int64_t w8a8_launch_count(void) { return g_launches.load(); }
+
+w8a8_status w8a8_poll_status(w8a8_stream_t stream) {
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  int *sw = status_word();
+  if (!sw) return W8A8_ERR_CUDA;
+  int host = 0;
+  cudaError_t e = cudaMemcpyAsync(&host, sw, sizeof(int), cudaMemcpyDeviceToHost, s);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) return W8A8_ERR_CUDA;
+  if (host != 0) {
+    const int zero = 0;
+    e = cudaMemcpyAsync(sw, &zero, sizeof(int), cudaMemcpyHostToDevice, s);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+    if (e != cudaSuccess) return W8A8_ERR_CUDA;
+    return static_cast<w8a8_status>(host);
+  }
+  return W8A8_OK;
+}
+
+w8a8_status w8a8_selftest_wait_timeout(int64_t timeout_ns, w8a8_stream_t stream) {
+  if (timeout_ns < 1000) timeout_ns = 1000;
+  if (timeout_ns > 5000000000LL) timeout_ns = 5000000000LL;
+  int *sw = status_word();
+  if (!sw) return W8A8_ERR_CUDA;
+  selftest_wait_kernel<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+      sw, static_cast<uint64_t>(timeout_ns));
+  count_launch();
+  return from_cuda(cudaGetLastError());
+}
+
+}  // extern "C"
