@@ -78,18 +78,43 @@ template <int BN, int STAGES>
 struct LargeSmem {
   static constexpr int kA = 0;
   static constexpr int kB = STAGES * kTileBytes;
-  static constexpr int kBars = kB + STAGES * BN * kBK;  // full[S], empty[S], tfull[2], tempty[2], mma_done
+  // per epilogue warp: the tile's BN w_scale (fp32) and BN bias (bf16) values
+  static constexpr int kEpiPerWarp = BN * 4 + BN * 2;
+  static constexpr int kEpi = kB + STAGES * BN * kBK;
+  static constexpr int kBars = kEpi + 4 * kEpiPerWarp;  // full[S], empty[S], tfull[2], tempty[2], mma_done
   static constexpr int kMisc = kBars + (2 * STAGES + 5) * 8;
   static constexpr int kUsed = kMisc + 16;
   static constexpr int kAlloc = kUsed + 1024;  // slack for 1024-byte alignment
 };
 
+// Stages this tile's per-column scale and bias into the warp's own smem
+// slice (all lanes then read them as broadcasts).
+template <int BN>
+__device__ __forceinline__ void stage_columns(const GemmArgs &a, int nb, int lane, float *s_ws,
+                                              uint16_t *s_bias) {
+  const int n0 = nb * BN;
+#pragma unroll
+  for (int j = lane * 4; j < BN; j += 128) {
+    float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (n0 + j < a.N) v = __ldg(reinterpret_cast<const float4 *>(a.w_scale + n0 + j));
+    *reinterpret_cast<float4 *>(s_ws + j) = v;
+  }
+  if (a.bias) {
+#pragma unroll
+    for (int j = lane * 8; j < BN; j += 256) {
+      uint4 v = make_uint4(0, 0, 0, 0);
+      if (n0 + j < a.N) v = __ldg(reinterpret_cast<const uint4 *>(a.bias + n0 + j));
+      *reinterpret_cast<uint4 *>(s_bias + j) = v;
+    }
+  }
+}
+
 template <int BN, bool OUT_I32>
 __device__ __forceinline__ void epilogue_tile(const GemmArgs &a, uint32_t tmem_cols, int quarter,
-                                              int lane, int mb, int nb) {
+                                              int lane, int mb, int nb, float as,
+                                              const float *s_ws, const uint16_t *s_bias) {
   const int row = mb * kBM + quarter * 32 + lane;
   const bool row_ok = row < a.M;
-  const float as = (!OUT_I32 && row_ok) ? __ldg(a.a_scale + row) : 0.0f;
   const uint32_t taddr = tmem_cols + ((uint32_t)(quarter * 32) << 16);
 #pragma unroll 1
   for (int c = 0; c < BN / 32; ++c) {
@@ -108,12 +133,14 @@ __device__ __forceinline__ void epilogue_tile(const GemmArgs &a, uint32_t tmem_c
                 make_uint4(r[4 * g], r[4 * g + 1], r[4 * g + 2], r[4 * g + 3]);
       }
     } else {
+      const float *ws = s_ws + c * 32;
+      const uint16_t *bs = s_bias + c * 32;
 #pragma unroll
       for (int g = 0; g < 4; ++g) {
         const int nn = n0 + 8 * g;
         if (nn >= a.N) break;  // N % 8 == 0: groups of 8 are all in or all out
-        const float4 w0 = __ldg(reinterpret_cast<const float4 *>(a.w_scale + nn));
-        const float4 w1 = __ldg(reinterpret_cast<const float4 *>(a.w_scale + nn + 4));
+        const float4 w0 = *reinterpret_cast<const float4 *>(ws + 8 * g);
+        const float4 w1 = *reinterpret_cast<const float4 *>(ws + 8 * g + 4);
         float t[8];
         t[0] = dequant((int32_t)r[8 * g + 0], as, w0.x);
         t[1] = dequant((int32_t)r[8 * g + 1], as, w0.y);
@@ -124,7 +151,7 @@ __device__ __forceinline__ void epilogue_tile(const GemmArgs &a, uint32_t tmem_c
         t[6] = dequant((int32_t)r[8 * g + 6], as, w1.z);
         t[7] = dequant((int32_t)r[8 * g + 7], as, w1.w);
         if (a.bias) {
-          const uint4 b = __ldg(reinterpret_cast<const uint4 *>(a.bias + nn));
+          const uint4 b = *reinterpret_cast<const uint4 *>(bs + 8 * g);
           const uint32_t bw[4] = {b.x, b.y, b.z, b.w};
 #pragma unroll
           for (int h = 0; h < 4; ++h) {
@@ -185,76 +212,84 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
 
-  // Inputs written by the preceding kernel of the stream are visible from here.
-  griddep_wait();
-
   const int num_tiles = args.tiles_m * args.tiles_n;
   const int num_kb = args.num_kb;
+  const int my_tiles = blockIdx.x < num_tiles ? (num_tiles - 1 - blockIdx.x) / gridDim.x + 1 : 0;
+  const uint32_t my_iters = (uint32_t)my_tiles * num_kb;
 
-  // Roles run as whole warps (so every warp reaches the block barriers
-  // converged); lane 0 waits and issues, and shares each wait's outcome.
+  // Roles: lane 0 of warps 0 and 1 runs the producer / MMA loop alone; the
+  // rest of those warps wait at __syncwarp so every warp reaches the block
+  // barrier below converged.
   if (warp == 0) {
-    // ---------------- producer ----------------
-    uint32_t it = 0;
-    uint32_t last_par[STAGES];
-    uint32_t issued = 0;
-    bool ok = true;
-    for (int tile = blockIdx.x; ok && tile < num_tiles; tile += gridDim.x) {
-      const int mb = tile % args.tiles_m, nb = tile / args.tiles_m;
-      const uint8_t *wslab = args.packed_w + (size_t)nb * (BN / 128) * num_kb * kTileBytes;
-      for (int kb = 0; kb < num_kb; ++kb, ++it) {
+    if (lane == 0) {
+      // ---------------- producer ----------------
+      uint32_t last_par[STAGES];
+      bool ok = true;
+      auto b_src = [&](uint32_t it, int h) {
+        const int tile = blockIdx.x + (int)(it / num_kb) * gridDim.x;
+        const int nb = tile / args.tiles_m, kb = (int)(it % num_kb);
+        return args.packed_w + (((size_t)nb * (BN / 128) + h) * num_kb + kb) * kTileBytes;
+      };
+      // The weight tiles of the first stages do not depend on the preceding
+      // kernel of the stream: issue them before waiting for it.
+      const uint32_t pre = my_iters < (uint32_t)STAGES ? my_iters : (uint32_t)STAGES;
+      for (uint32_t it = 0; it < pre; ++it) {
+        mbar_arrive_expect_tx(&full[it], kStageBytes);
+#pragma unroll
+        for (int h = 0; h < BN / 128; ++h)
+          bulk_load(sB + it * (BN * kBK) + h * kTileBytes, b_src(it, h), kTileBytes, &full[it]);
+        last_par[it] = 0;
+      }
+      griddep_wait();
+      for (uint32_t it = 0; it < pre; ++it) {
+        const int tile = blockIdx.x + (int)(it / num_kb) * gridDim.x;
+        tma_load_2d(sA + it * kTileBytes, &tmap_q, (int)(it % num_kb) * kBK,
+                    (tile % args.tiles_m) * kBM, &full[it]);
+      }
+      for (uint32_t it = pre; it < my_iters; ++it) {
         const uint32_t s = it % STAGES, ph = (it / STAGES) & 1;
-        int w_ok = 0;
-        if (lane == 0) w_ok = mbar_wait_bounded(&empty[s], ph ^ 1, abort_flag, args.status);
-        if (!__shfl_sync(0xFFFFFFFFu, w_ok, 0)) {
+        if (!mbar_wait(&empty[s], ph ^ 1, abort_flag, args.status)) {
           ok = false;
           break;
         }
-        if (lane == 0) {
-          mbar_arrive_expect_tx(&full[s], kStageBytes);
-          tma_load_2d(sA + s * kTileBytes, &tmap_q, kb * kBK, mb * kBM, &full[s]);
+        const int tile = blockIdx.x + (int)(it / num_kb) * gridDim.x;
+        mbar_arrive_expect_tx(&full[s], kStageBytes);
+        tma_load_2d(sA + s * kTileBytes, &tmap_q, (int)(it % num_kb) * kBK,
+                    (tile % args.tiles_m) * kBM, &full[s]);
 #pragma unroll
-          for (int h = 0; h < BN / 128; ++h)
-            bulk_load(sB + s * (BN * kBK) + h * kTileBytes,
-                      wslab + ((size_t)h * num_kb + kb) * kTileBytes, kTileBytes, &full[s]);
-        }
-        __syncwarp();
+        for (int h = 0; h < BN / 128; ++h)
+          bulk_load(sB + s * (BN * kBK) + h * kTileBytes, b_src(it, h), kTileBytes, &full[s]);
         last_par[s] = ph;
-        ++issued;
       }
-    }
-    if (!ok && lane == 0) {
-      // Drain: wait (bounded) for the copies still in flight into our smem.
-      const uint32_t n = issued < STAGES ? issued : STAGES;
-      for (uint32_t s = 0; s < n; ++s) {
-        volatile int no_abort = 0;
-        (void)mbar_wait_bounded(&full[s], last_par[s], &no_abort, args.status);
+      if (!ok) {
+        // Drain: wait (bounded) for the copies still in flight into our smem.
+        for (uint32_t s = 0; s < (uint32_t)STAGES && s < my_iters; ++s) {
+          volatile int no_abort = 0;
+          (void)mbar_wait_bounded(&full[s], last_par[s], &no_abort, args.status);
+        }
       }
     }
     __syncwarp();
   } else if (warp == 1) {
-    // ---------------- MMA issuer ----------------
-    uint32_t it = 0, t_local = 0;
-    bool ok = true;
-    for (int tile = blockIdx.x; ok && tile < num_tiles; tile += gridDim.x, ++t_local) {
-      const uint32_t b = t_local & 1, bph = (t_local >> 1) & 1;
-      int w_ok = 0;
-      if (lane == 0) w_ok = mbar_wait_bounded(&tempty[b], bph ^ 1, abort_flag, args.status);
-      if (!__shfl_sync(0xFFFFFFFFu, w_ok, 0)) {
-        ok = false;
-        break;
-      }
-      tc_fence_after();
-      const uint32_t d_tmem = tmem_base + b * BN;
-      for (int kb = 0; kb < num_kb; ++kb, ++it) {
-        const uint32_t s = it % STAGES, ph = (it / STAGES) & 1;
-        if (lane == 0) w_ok = mbar_wait_bounded(&full[s], ph, abort_flag, args.status);
-        if (!__shfl_sync(0xFFFFFFFFu, w_ok, 0)) {
+    if (lane == 0) {
+      // ---------------- MMA issuer ----------------
+      uint32_t it = 0;
+      bool ok = true;
+      for (int t = 0; ok && t < my_tiles; ++t) {
+        const uint32_t b = t & 1, bph = (t >> 1) & 1;
+        if (!mbar_wait(&tempty[b], bph ^ 1, abort_flag, args.status)) {
           ok = false;
           break;
         }
         tc_fence_after();
-        if (lane == 0) {
+        const uint32_t d_tmem = tmem_base + b * BN;
+        for (int kb = 0; kb < num_kb; ++kb, ++it) {
+          const uint32_t s = it % STAGES, ph = (it / STAGES) & 1;
+          if (!mbar_wait(&full[s], ph, abort_flag, args.status)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
           const uint64_t a_desc = sw128_kmajor_desc(sA + s * kTileBytes);
           const uint64_t b_desc = sw128_kmajor_desc(sB + s * (BN * kBK));
 #pragma unroll
@@ -262,31 +297,40 @@ __global__ void __launch_bounds__(kThreads, 1)
             mma_i8(d_tmem, a_desc + 2 * k, b_desc + 2 * k, kIdesc, (kb | k) != 0);
           mma_commit(&empty[s]);  // frees the stage when these MMAs finish
         }
-        __syncwarp();
+        if (ok) mma_commit(&tfull[b]);
       }
-      if (ok && lane == 0) mma_commit(&tfull[b]);
-      __syncwarp();
-    }
-    if (!ok && lane == 0) {
-      // Wait (bounded) for MMAs still in flight before TMEM is released.
-      mma_commit(mma_done);
-      volatile int no_abort = 0;
-      (void)mbar_wait_bounded(mma_done, 0, &no_abort, args.status);
+      if (!ok) {
+        // Wait (bounded) for MMAs still in flight before TMEM is released.
+        mma_commit(mma_done);
+        volatile int no_abort = 0;
+        (void)mbar_wait_bounded(mma_done, 0, &no_abort, args.status);
+      }
     }
     __syncwarp();
   } else {
     // ---------------- epilogue (warps 2..5) ----------------
+    griddep_wait();  // a_scale comes from the preceding kernel
     const int quarter = warp & 3;  // TMEM lanes this warp may access
-    uint32_t t_local = 0;
-    for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++t_local) {
-      const uint32_t b = t_local & 1, bph = (t_local >> 1) & 1;
+    float *s_ws = reinterpret_cast<float *>(smem + L::kEpi + (warp - 2) * L::kEpiPerWarp);
+    uint16_t *s_bias = reinterpret_cast<uint16_t *>(s_ws + BN);
+    for (int t = 0; t < my_tiles; ++t) {
+      const int tile = blockIdx.x + t * gridDim.x;
+      const int mb = tile % args.tiles_m, nb = tile / args.tiles_m;
+      const uint32_t b = t & 1, bph = (t >> 1) & 1;
+      // operands of the epilogue, fetched while the main loop runs
+      float as = 0.0f;
+      if (!OUT_I32) {
+        stage_columns<BN>(args, nb, lane, s_ws, s_bias);
+        const int row = mb * kBM + quarter * 32 + lane;
+        if (row < args.M) as = __ldg(args.a_scale + row);
+      }
+      __syncwarp();
       int ok = 0;
-      if (lane == 0) ok = mbar_wait_bounded(&tfull[b], bph, abort_flag, args.status);
+      if (lane == 0) ok = mbar_wait(&tfull[b], bph, abort_flag, args.status);
       ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
       if (!ok) break;
       tc_fence_after();
-      const int mb = tile % args.tiles_m, nb = tile / args.tiles_m;
-      epilogue_tile<BN, OUT_I32>(args, tmem_base + b * BN, quarter, lane, mb, nb);
+      epilogue_tile<BN, OUT_I32>(args, tmem_base + b * BN, quarter, lane, mb, nb, as, s_ws, s_bias);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&tempty[b]);
@@ -393,89 +437,84 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int nkb = args.num_kb;
 
   if (warp == 0) {
-    // ---------------- producer (whole warp; lane 0 issues) ----------------
-    // The weight stream does not depend on the preceding kernel: start it
-    // before waiting for the activations.
-    uint32_t it = 0, issued = 0;
-    uint32_t last_par[STAGES];
-    bool ok = true, waited = false;
-    for (int64_t u = u_begin; u < u_end; ++u, ++it) {
-      const uint32_t s = it % STAGES, ph = (it / STAGES) & 1;
-      int w_ok = 0;
-      if (lane == 0) w_ok = mbar_wait_bounded(&empty[s], ph ^ 1, abort_flag, args.status);
-      if (!__shfl_sync(0xFFFFFFFFu, w_ok, 0)) {
-        ok = false;
-        break;
+    if (lane == 0) {
+      // ---------------- producer ----------------
+      // The weight stream does not depend on the preceding kernel: the first
+      // stages' weight tiles go out before waiting for the activations.
+      uint32_t last_par[STAGES];
+      bool ok = true;
+      const int64_t n_units = u_end - u_begin;
+      const uint32_t pre = n_units < STAGES ? (uint32_t)n_units : (uint32_t)STAGES;
+      for (uint32_t i = 0; i < pre; ++i) {
+        mbar_arrive_expect_tx(&full[i], kStageBytes);
+        bulk_load_hint(sW + i * kTileBytes, args.packed_w + (size_t)(u_begin + i) * kTileBytes,
+                       kTileBytes, &full[i], evict_first);
+        last_par[i] = 0;
       }
-      const int kb = (int)(u % nkb);
-      if (lane == 0) {
+      griddep_wait();
+      for (uint32_t i = 0; i < pre; ++i)
+        tma_load_2d(sQ + i * kQBytes, &tmap_q, (int)((u_begin + i) % nkb) * kBK, 0, &full[i]);
+      uint32_t it = pre;
+      for (int64_t u = u_begin + pre; u < u_end; ++u, ++it) {
+        const uint32_t s = it % STAGES, ph = (it / STAGES) & 1;
+        if (!mbar_wait(&empty[s], ph ^ 1, abort_flag, args.status)) {
+          ok = false;
+          break;
+        }
         mbar_arrive_expect_tx(&full[s], kStageBytes);
         bulk_load_hint(sW + s * kTileBytes, args.packed_w + (size_t)u * kTileBytes, kTileBytes,
                        &full[s], evict_first);
+        tma_load_2d(sQ + s * kQBytes, &tmap_q, (int)(u % nkb) * kBK, 0, &full[s]);
+        last_par[s] = ph;
       }
-      if (!waited) {
-        griddep_wait();
-        waited = true;
-      }
-      if (lane == 0) tma_load_2d(sQ + s * kQBytes, &tmap_q, kb * kBK, 0, &full[s]);
-      __syncwarp();
-      last_par[s] = ph;
-      ++issued;
-    }
-    if (!waited) griddep_wait();
-    if (!ok && lane == 0) {
-      const uint32_t n = issued < STAGES ? issued : STAGES;
-      for (uint32_t s = 0; s < n; ++s) {
-        volatile int no_abort = 0;
-        (void)mbar_wait_bounded(&full[s], last_par[s], &no_abort, args.status);
+      if (!ok) {
+        for (uint32_t s = 0; s < (uint32_t)STAGES && (int64_t)s < n_units; ++s) {
+          volatile int no_abort = 0;
+          (void)mbar_wait_bounded(&full[s], last_par[s], &no_abort, args.status);
+        }
       }
     }
     __syncwarp();
   } else if (warp == 1) {
-    // ---------------- MMA issuer (whole warp; lane 0 issues) ----------------
-    uint32_t it = 0, seg = 0;
-    bool ok = true;
-    int64_t u = u_begin;
-    while (ok && u < u_end) {
-      const int nb = (int)(u / nkb);
-      const int64_t seg_end = std::min<int64_t>(u_end, (int64_t)(nb + 1) * nkb);
-      const uint32_t b = seg & 1, bph = (seg >> 1) & 1;
-      int w_ok = 0;
-      if (lane == 0) w_ok = mbar_wait_bounded(&tempty[b], bph ^ 1, abort_flag, args.status);
-      if (!__shfl_sync(0xFFFFFFFFu, w_ok, 0)) {
-        ok = false;
-        break;
-      }
-      tc_fence_after();
-      const uint32_t d_tmem = tmem_base + b * kDecodeNT;
-      bool first = true;
-      for (; u < seg_end; ++u, ++it) {
-        const uint32_t s = it % STAGES, ph = (it / STAGES) & 1;
-        if (lane == 0) w_ok = mbar_wait_bounded(&full[s], ph, abort_flag, args.status);
-        if (!__shfl_sync(0xFFFFFFFFu, w_ok, 0)) {
+    if (lane == 0) {
+      // ---------------- MMA issuer ----------------
+      uint32_t it = 0, seg = 0;
+      bool ok = true;
+      int64_t u = u_begin;
+      while (ok && u < u_end) {
+        const int nb = (int)(u / nkb);
+        const int64_t seg_end = min(u_end, (int64_t)(nb + 1) * nkb);
+        const uint32_t b = seg & 1, bph = (seg >> 1) & 1;
+        if (!mbar_wait(&tempty[b], bph ^ 1, abort_flag, args.status)) {
           ok = false;
           break;
         }
         tc_fence_after();
-        if (lane == 0) {
+        const uint32_t d_tmem = tmem_base + b * kDecodeNT;
+        bool first = true;
+        for (; u < seg_end; ++u, ++it) {
+          const uint32_t s = it % STAGES, ph = (it / STAGES) & 1;
+          if (!mbar_wait(&full[s], ph, abort_flag, args.status)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
           const uint64_t a_desc = sw128_kmajor_desc(sW + s * kTileBytes);
           const uint64_t b_desc = sw128_kmajor_desc(sQ + s * kQBytes);
 #pragma unroll
           for (int k = 0; k < kBK / 32; ++k)
             mma_i8(d_tmem, a_desc + 2 * k, b_desc + 2 * k, kIdesc, (first && k == 0) ? 0u : 1u);
+          first = false;
           mma_commit(&empty[s]);
         }
-        __syncwarp();
-        first = false;
+        if (ok) mma_commit(&tfull[b]);
+        ++seg;
       }
-      if (ok && lane == 0) mma_commit(&tfull[b]);
-      __syncwarp();
-      ++seg;
-    }
-    if (!ok && lane == 0) {
-      mma_commit(mma_done);
-      volatile int no_abort = 0;
-      (void)mbar_wait_bounded(mma_done, 0, &no_abort, args.status);
+      if (!ok) {
+        mma_commit(mma_done);
+        volatile int no_abort = 0;
+        (void)mbar_wait_bounded(mma_done, 0, &no_abort, args.status);
+      }
     }
     __syncwarp();
   } else {
@@ -491,10 +530,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     while (u < u_end) {
       const int nb = (int)(u / nkb);
       const int64_t slab_begin = (int64_t)nb * nkb, slab_end = slab_begin + nkb;
-      const int64_t seg_end = std::min<int64_t>(u_end, slab_end);
+      const int64_t seg_end = min(u_end, slab_end);
       const bool whole = (u == slab_begin) && (seg_end == slab_end);
       const uint32_t b = seg & 1, bph = (seg >> 1) & 1;
-      if (et == 0) seg_ok[b] = mbar_wait_bounded(&tfull[b], bph, abort_flag, args.status) ? 1 : 0;
+      if (et == 0) seg_ok[b] = mbar_wait(&tfull[b], bph, abort_flag, args.status) ? 1 : 0;
       __syncwarp();
       asm volatile("bar.sync 1, 128;" ::: "memory");
       if (!seg_ok[b]) break;

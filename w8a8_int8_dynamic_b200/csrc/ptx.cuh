@@ -82,6 +82,16 @@ static __device__ __noinline__ bool mbar_wait_bounded(uint64_t *bar, uint32_t pa
   }
 }
 
+// Common case inline (one try_wait); the bounded polling loop only when the
+// phase has not completed yet.  The out-of-line call alone costs a few
+// hundred cycles, more than a 128x128x128 int8 MMA stage, so it must stay off
+// the fast path.
+__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity,
+                                          volatile int *abort_flag, int *status) {
+  if (mbar_try_wait(smem_addr(bar), parity)) return true;
+  return mbar_wait_bounded(bar, parity, abort_flag, status);
+}
+
 // ---- TMA and bulk copies (global -> shared, completion on an mbarrier) ------
 __device__ __forceinline__ void prefetch_tmap(const CUtensorMap *map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
