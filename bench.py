@@ -53,6 +53,25 @@ def load_peaks():
             "source": "fallback"}
 
 
+def recorded_traffic(workload):
+    """DRAM bytes per launch of the GEMM from the committed ncu capture, or
+    None when there is none or the kernel sources changed since it was taken."""
+    import hashlib
+    path = os.path.join(HERE, "profiles", "traffic.json")
+    if not os.path.exists(path):
+        return None
+    rec = json.load(open(path)).get(workload)
+    if not rec:
+        return None
+    csrc = os.path.join(HERE, "w8a8_int8_dynamic_b200", "csrc")
+    h = hashlib.sha256()
+    for f in ("gemm.cu", "ptx.cuh"):
+        h.update(open(os.path.join(csrc, f), "rb").read())
+    if h.hexdigest()[:16] != rec.get("source_sha256_16"):
+        return None
+    return rec.get("gemm_bytes_per_launch")
+
+
 # ----------------------------------------------------------------------------- clocks
 class ClockSampler:
     FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
@@ -280,11 +299,7 @@ def run_ours(args, rank, world, device):
                 "quant_us": round(base["t_quant"] * 1e6, 3),
                 "quant_gbs": round(quant_bytes / base["t_quant"] / 1e9, 1),
                 "quant_frac_hbm": round(quant_bytes / base["t_quant"] / 1e9 / peaks["hbm_gbs"], 4)}
-    traffic_file = os.path.join(HERE, "profiles", "traffic.json")
-    if os.path.exists(traffic_file):
-        tr = json.load(open(traffic_file)).get(args.workload, {})
-        if tr.get("gemm_bytes_per_launch") is not None:
-            roofline["traffic"] = tr["gemm_bytes_per_launch"]
+    roofline["traffic"] = recorded_traffic(args.workload)
 
     # ---- end to end through the public API, host buffers
     e2e = run_e2e(w8, ls, args, stream, ops)
