@@ -145,8 +145,9 @@ def test_gemm_i32_extreme_values():
 
 
 @pytest.mark.parametrize("bias", [False, True])
-@pytest.mark.parametrize("path", [w8.PATH_LARGE_BN128, w8.PATH_LARGE_BN256])
-@pytest.mark.parametrize("M,N,K", [(64, 128, 256), (129, 392, 400), (300, 1000, 528), (512, 1024, 4096)])
+@pytest.mark.parametrize("path", [w8.PATH_LARGE_BN128, w8.PATH_LARGE_BN256, w8.PATH_LARGE_PAIR])
+@pytest.mark.parametrize("M,N,K", [(64, 128, 256), (129, 392, 400), (300, 1000, 528), (512, 1024, 4096),
+                                   (257, 264, 272), (700, 520, 144)])
 def test_scaled_mm_matches_oracle(M, N, K, path, bias):
     w8.set_path(path)
     inp = random_case(M + N + K, M, N, K, bias=bias, n_outliers=K // 64, zero_row=True)
@@ -160,7 +161,9 @@ def test_scaled_mm_matches_oracle(M, N, K, path, bias):
     assert np.array_equal(y_h, y_ref), "expected bit-exact bf16"
 
 
-def test_scaled_mm_does_not_write_outside_y():
+@pytest.mark.parametrize("path", [w8.PATH_LARGE_BN128, w8.PATH_LARGE_PAIR])
+def test_scaled_mm_does_not_write_outside_y(path):
+    w8.set_path(path)
     M, N, K = 130, 264, 272
     inp = random_case(9, M, N, K, bias=True)
     q_ref, s_ref = oracle.quant_act(inp.x)
@@ -194,9 +197,11 @@ def test_decode_path_matches_oracle(M, N, K):
 
 
 # ---------------------------------------------------------------- fused layer
+@pytest.mark.parametrize("path", [w8.PATH_AUTO, w8.PATH_LARGE_PAIR])
 @pytest.mark.parametrize("M,N,K", [(1, 264, 400), (16, 1024, 1024), (17, 1024, 1024),
                                    (64, 128, 256), (300, 1000, 528), (512, 4096, 4096)])
-def test_linear_matches_oracle(M, N, K):
+def test_linear_matches_oracle(M, N, K, path):
+    w8.set_path(path)
     inp = random_case(M * 5 + N + K, M, N, K, bias=True, n_outliers=K // 100, zero_row=True)
     y_ref, q_ref, s_ref, _ = oracle.linear(inp.x, inp.w, inp.w_scale, inp.bias)
     layer = w8.W8A8Linear(dev(inp.w), dev(inp.w_scale), dev_bf16(inp.bias))

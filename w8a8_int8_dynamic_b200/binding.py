@@ -27,7 +27,7 @@ STATUS_NAMES = {
     6: "W8A8_ERR_BUFFER_TOO_SMALL",
 }
 
-PATH_AUTO, PATH_LARGE, PATH_SMALL, PATH_LARGE_BN128, PATH_LARGE_BN256 = 0, 1, 2, 3, 4
+PATH_AUTO, PATH_LARGE, PATH_SMALL, PATH_LARGE_BN128, PATH_LARGE_BN256, PATH_LARGE_PAIR = 0, 1, 2, 3, 4, 5
 
 
 class W8A8Error(RuntimeError):

@@ -38,38 +38,10 @@
 
 #include <algorithm>
 
-#include "internal.h"
-#include "ptx.cuh"
+#include "gemm_common.cuh"
 
 namespace w8a8 {
 namespace {
-
-constexpr int kBM = 128;                 // tile rows (MMA M)
-constexpr int kBK = 128;                 // bytes of K per pipeline stage
-constexpr int kTileBytes = 128 * kBK;    // one 128 x 128 int8 tile = 16 KB
-constexpr int kThreads = 192;            // 6 warps
-constexpr int kDecodeNT = 16;            // activation rows per decode MMA (N)
-
-struct GemmArgs {
-  const uint8_t *packed_w;
-  const float *a_scale;
-  const float *w_scale;
-  const uint16_t *bias;  // may be null
-  void *out;             // bf16 [M, N] or int32 [M, N]
-  int M, N;
-  int num_kb;            // K blocks of 128 bytes (= packed K / 128)
-  int tiles_m, tiles_n;
-  int *status;
-};
-
-__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
-  const __nv_bfloat162 r = __floats2bfloat162_rn(lo, hi);
-  return *reinterpret_cast<const uint32_t *>(&r);
-}
-
-__device__ __forceinline__ float dequant(int32_t acc, float as, float ws) {
-  return __fmul_rn(__fmul_rn(__int2float_rn(acc), as), ws);
-}
 
 // ============================================================================
 // Large-M persistent GEMM
@@ -86,89 +58,6 @@ struct LargeSmem {
   static constexpr int kUsed = kMisc + 16;
   static constexpr int kAlloc = kUsed + 1024;  // slack for 1024-byte alignment
 };
-
-// Stages this tile's per-column scale and bias into the warp's own smem
-// slice (all lanes then read them as broadcasts).
-template <int BN>
-__device__ __forceinline__ void stage_columns(const GemmArgs &a, int nb, int lane, float *s_ws,
-                                              uint16_t *s_bias) {
-  const int n0 = nb * BN;
-#pragma unroll
-  for (int j = lane * 4; j < BN; j += 128) {
-    float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-    if (n0 + j < a.N) v = __ldg(reinterpret_cast<const float4 *>(a.w_scale + n0 + j));
-    *reinterpret_cast<float4 *>(s_ws + j) = v;
-  }
-  if (a.bias) {
-#pragma unroll
-    for (int j = lane * 8; j < BN; j += 256) {
-      uint4 v = make_uint4(0, 0, 0, 0);
-      if (n0 + j < a.N) v = __ldg(reinterpret_cast<const uint4 *>(a.bias + n0 + j));
-      *reinterpret_cast<uint4 *>(s_bias + j) = v;
-    }
-  }
-}
-
-template <int BN, bool OUT_I32>
-__device__ __forceinline__ void epilogue_tile(const GemmArgs &a, uint32_t tmem_cols, int quarter,
-                                              int lane, int mb, int nb, float as,
-                                              const float *s_ws, const uint16_t *s_bias) {
-  const int row = mb * kBM + quarter * 32 + lane;
-  const bool row_ok = row < a.M;
-  const uint32_t taddr = tmem_cols + ((uint32_t)(quarter * 32) << 16);
-#pragma unroll 1
-  for (int c = 0; c < BN / 32; ++c) {
-    const int n0 = nb * BN + c * 32;
-    if (n0 >= a.N) break;  // uniform across the warp
-    uint32_t r[32];
-    tmem_ld_32x32b_x32(taddr + c * 32, r);
-    tmem_ld_wait();
-    if (OUT_I32) {
-      if (row_ok) {
-        int32_t *dst = static_cast<int32_t *>(a.out) + (int64_t)row * a.N + n0;
-#pragma unroll
-        for (int g = 0; g < 8; ++g)
-          if (n0 + 4 * g < a.N)
-            *reinterpret_cast<uint4 *>(dst + 4 * g) =
-                make_uint4(r[4 * g], r[4 * g + 1], r[4 * g + 2], r[4 * g + 3]);
-      }
-    } else {
-      const float *ws = s_ws + c * 32;
-      const uint16_t *bs = s_bias + c * 32;
-#pragma unroll
-      for (int g = 0; g < 4; ++g) {
-        const int nn = n0 + 8 * g;
-        if (nn >= a.N) break;  // N % 8 == 0: groups of 8 are all in or all out
-        const float4 w0 = *reinterpret_cast<const float4 *>(ws + 8 * g);
-        const float4 w1 = *reinterpret_cast<const float4 *>(ws + 8 * g + 4);
-        float t[8];
-        t[0] = dequant((int32_t)r[8 * g + 0], as, w0.x);
-        t[1] = dequant((int32_t)r[8 * g + 1], as, w0.y);
-        t[2] = dequant((int32_t)r[8 * g + 2], as, w0.z);
-        t[3] = dequant((int32_t)r[8 * g + 3], as, w0.w);
-        t[4] = dequant((int32_t)r[8 * g + 4], as, w1.x);
-        t[5] = dequant((int32_t)r[8 * g + 5], as, w1.y);
-        t[6] = dequant((int32_t)r[8 * g + 6], as, w1.z);
-        t[7] = dequant((int32_t)r[8 * g + 7], as, w1.w);
-        if (a.bias) {
-          const uint4 b = *reinterpret_cast<const uint4 *>(bs + 8 * g);
-          const uint32_t bw[4] = {b.x, b.y, b.z, b.w};
-#pragma unroll
-          for (int h = 0; h < 4; ++h) {
-            t[2 * h] = __fadd_rn(t[2 * h], __uint_as_float(bw[h] << 16));
-            t[2 * h + 1] = __fadd_rn(t[2 * h + 1], __uint_as_float(bw[h] & 0xFFFF0000u));
-          }
-        }
-        if (row_ok) {
-          uint16_t *dst = static_cast<uint16_t *>(a.out) + (int64_t)row * a.N + nn;
-          *reinterpret_cast<uint4 *>(dst) =
-              make_uint4(pack_bf16x2(t[0], t[1]), pack_bf16x2(t[2], t[3]),
-                         pack_bf16x2(t[4], t[5]), pack_bf16x2(t[6], t[7]));
-        }
-      }
-    }
-  }
-}
 
 template <int BN, int STAGES, bool OUT_I32>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -330,7 +219,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
       if (!ok) break;
       tc_fence_after();
-      epilogue_tile<BN, OUT_I32>(args, tmem_base + b * BN, quarter, lane, mb, nb, as, s_ws, s_bias);
+      epilogue_tile<BN, OUT_I32>(args, tmem_base + b * BN, quarter, lane, mb * kBM, nb, as, s_ws,
+                                 s_bias);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&tempty[b]);
@@ -660,18 +550,27 @@ w8a8_status run_large(const CUtensorMap &tmap, GemmArgs args, cudaStream_t strea
   return from_cuda(e);
 }
 
-// Tile width for the large-M kernel: fewest waves x tile time, with the
-// narrower tile charged for its lower tensor-pipe efficiency.
-int choose_bn(int64_t M, int64_t N) {
+// Kernel choice for large M.  Per-SM feed from L2 limits how much of the
+// int8 rate each tile shape reaches (measured: the 128 x 128 1-SM tile needs
+// ~128 B/clk per SM, the 128 x 256 tile ~94, the 2-SM 256 x 256 tile ~64),
+// so the cost of a shape is its wave count times its per-SM tile work divided
+// by the fraction of the rate it sustains.
+enum class LargeKind { k128, k256, kPair };
+
+LargeKind choose_large(int64_t M, int64_t N) {
   const int path = forced_path();
-  if (path == 3) return 128;
-  if (path == 4) return 256;
+  if (path == 3) return LargeKind::k128;
+  if (path == 4) return LargeKind::k256;
+  if (path == 5) return LargeKind::kPair;
   const int64_t sms = sm_count();
   const int64_t tm = (M + kBM - 1) / kBM;
   const int64_t t128 = tm * ((N + 127) / 128), t256 = tm * ((N + 255) / 256);
-  const double c128 = (double)((t128 + sms - 1) / sms) * 128.0 / 0.85;
-  const double c256 = (double)((t256 + sms - 1) / sms) * 256.0;
-  return c256 <= c128 ? 256 : 128;
+  const int64_t tpair = pair_tiles(M, N), pairs = sms / 2;
+  const double c128 = (double)((t128 + sms - 1) / sms) * 128.0 / 0.45;
+  const double c256 = (double)((t256 + sms - 1) / sms) * 256.0 / 0.60;
+  const double cpair = (double)((tpair + pairs - 1) / pairs) * 256.0 / 0.85;
+  if (cpair <= c128 && cpair <= c256) return LargeKind::kPair;
+  return c256 <= c128 ? LargeKind::k256 : LargeKind::k128;
 }
 
 }  // namespace
@@ -701,7 +600,7 @@ int64_t decode_workspace_bytes(int64_t N, int64_t K) {
 bool use_decode_path(int64_t M) {
   const int p = forced_path();
   if (p == 2) return M <= kDecodeNT;
-  if (p == 1 || p == 3 || p == 4) return false;
+  if (p == 1 || p == 3 || p == 4 || p == 5) return false;
   return M <= kDecodeNT;
 }
 
@@ -764,13 +663,20 @@ w8a8_status launch_scaled_mm(const int8_t *q, const float *a_scale, const void *
   a.tiles_n = 0;
   a.status = status_word();
   if (!a.status) return W8A8_ERR_CUDA;
-  const int bn = choose_bn(M, N);
   if (out_i32) {
-    return bn == 256 ? run_large<256, kLargeStages256, true>(tmap, a, stream, pdl, 0)
-                     : run_large<128, kLargeStages128, true>(tmap, a, stream, pdl, 1);
+    // the int32 export always uses the 1-SM kernel (tests and inspection)
+    const LargeKind kind = choose_large(M, N);
+    return kind == LargeKind::k128 ? run_large<128, kLargeStages128, true>(tmap, a, stream, pdl, 1)
+                                   : run_large<256, kLargeStages256, true>(tmap, a, stream, pdl, 0);
   }
-  return bn == 256 ? run_large<256, kLargeStages256, false>(tmap, a, stream, pdl, 2)
-                   : run_large<128, kLargeStages128, false>(tmap, a, stream, pdl, 3);
+  switch (choose_large(M, N)) {
+    case LargeKind::kPair:
+      return launch_gemm2sm(q, a_scale, packed_w, w_scale, bias, out, M, N, K, stream, pdl);
+    case LargeKind::k256:
+      return run_large<256, kLargeStages256, false>(tmap, a, stream, pdl, 2);
+    default:
+      return run_large<128, kLargeStages128, false>(tmap, a, stream, pdl, 3);
+  }
 }
 
 static w8a8_status check_gemm_args(const void *q, const void *packed_w, const void *out,

@@ -31,6 +31,11 @@ int forced_path();
 bool make_tmap_u8_2d(CUtensorMap *map, const void *base, uint64_t rows, uint64_t cols,
                      uint64_t ld, uint32_t box_rows, uint32_t box_cols);
 
+// Same, without swizzle: for the packed weight image, whose bytes are already
+// in the tensor core's shared-memory order.
+bool make_tmap_u8_2d_plain(CUtensorMap *map, const void *base, uint64_t rows, uint64_t cols,
+                           uint64_t ld, uint32_t box_rows, uint32_t box_cols);
+
 inline bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 inline w8a8_status from_cuda(cudaError_t e) { return e == cudaSuccess ? W8A8_OK : W8A8_ERR_CUDA; }
@@ -48,6 +53,11 @@ inline int64_t packed_cols(int64_t K) { return round_up(K, 128); }
 w8a8_status launch_scaled_mm(const int8_t *q, const float *a_scale, const void *packed_w,
                              const float *w_scale, const void *bias, void *out, bool out_i32,
                              int64_t M, int64_t N, int64_t K, cudaStream_t stream, bool pdl);
+// 2-SM (CTA pair) GEMM with the bf16 epilogue (gemm2sm.cu).
+w8a8_status launch_gemm2sm(const int8_t *q, const float *a_scale, const void *packed_w,
+                           const float *w_scale, const void *bias, void *y, int64_t M, int64_t N,
+                           int64_t K, cudaStream_t stream, bool pdl);
+int64_t pair_tiles(int64_t M, int64_t N);
 // Quantisation launcher (quant.cu).
 w8a8_status launch_quant(const void *x, int64_t M, int64_t K, int64_t ldx, int8_t *q,
                          float *a_scale, cudaStream_t stream);

@@ -57,8 +57,9 @@ void count_launch(int n) { g_launches.fetch_add(n, std::memory_order_relaxed); }
 
 int forced_path() { return g_forced_path.load(std::memory_order_relaxed); }
 
-bool make_tmap_u8_2d(CUtensorMap *map, const void *base, uint64_t rows, uint64_t cols,
-                     uint64_t ld, uint32_t box_rows, uint32_t box_cols) {
+static bool encode_u8_2d(CUtensorMap *map, const void *base, uint64_t rows, uint64_t cols,
+                         uint64_t ld, uint32_t box_rows, uint32_t box_cols,
+                         CUtensorMapSwizzle swizzle) {
   if (!g_encode) {
     std::lock_guard<std::mutex> lk(g_mu);
     if (!g_encode) {
@@ -76,10 +77,20 @@ bool make_tmap_u8_2d(CUtensorMap *map, const void *base, uint64_t rows, uint64_t
   const cuuint32_t box[2] = {box_cols, box_rows};
   const cuuint32_t estr[2] = {1, 1};
   const CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void *>(base),
-                              dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                              CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                              dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle,
+                              CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
+}
+
+bool make_tmap_u8_2d(CUtensorMap *map, const void *base, uint64_t rows, uint64_t cols,
+                     uint64_t ld, uint32_t box_rows, uint32_t box_cols) {
+  return encode_u8_2d(map, base, rows, cols, ld, box_rows, box_cols, CU_TENSOR_MAP_SWIZZLE_128B);
+}
+
+bool make_tmap_u8_2d_plain(CUtensorMap *map, const void *base, uint64_t rows, uint64_t cols,
+                           uint64_t ld, uint32_t box_rows, uint32_t box_cols) {
+  return encode_u8_2d(map, base, rows, cols, ld, box_rows, box_cols, CU_TENSOR_MAP_SWIZZLE_NONE);
 }
 
 // Waits on a barrier that nothing arrives at; the bounded wait must give up.
@@ -121,7 +132,7 @@ const char *w8a8_status_string(int status) {
 int w8a8_abi_version(void) { return (1 << 16) | 0; }
 
 w8a8_status w8a8_set_path(int path) {
-  if (path < 0 || path > 4) return W8A8_ERR_INVALID_ARG;
+  if (path < 0 || path > 5) return W8A8_ERR_INVALID_ARG;
   g_forced_path.store(path);
   return W8A8_OK;
 }
