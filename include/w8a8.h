@@ -148,6 +148,26 @@ w8a8_status w8a8_linear(const void *x, int64_t ldx, const void *packed_w,
                         int64_t M, int64_t N, int64_t K, void *workspace,
                         size_t ws_bytes, w8a8_stream_t stream);
 
+/* ---- the whole layer without a caller-provided workspace ---------------------
+ * No counterpart on the pages: an addition for callers that cannot allocate
+ * device memory when they run a layer (a plugin whose host framework owns all
+ * device memory and forbids cudaMalloc inside execution callbacks, or a
+ * latency-critical loop that cannot afford the device-wide synchronisation of
+ * cudaMalloc / cudaFree).  Same arguments, arithmetic and results as
+ * w8a8_linear, minus the workspace: the codes, scales and small-M partials go
+ * to one scratch array of w8a8_linear_noalloc_max_bytes() bytes (8 MiB) that
+ * every GPU loading this library holds until the process exits.  Nothing is
+ * allocated.  Returns W8A8_ERR_BUFFER_TOO_SMALL, launching nothing, when
+ * w8a8_linear_workspace_bytes(M, N, K) exceeds that size.  The first call on
+ * each device looks up the array's device address (make it before any stream
+ * capture).  All calls on a device share the array: calls that overlap on the
+ * GPU (different streams without ordering) race and corrupt each other. */
+size_t w8a8_linear_noalloc_max_bytes(void);
+w8a8_status w8a8_linear_noalloc(const void *x, int64_t ldx, const void *packed_w,
+                                const float *w_scale, const void *bias, void *y,
+                                int64_t M, int64_t N, int64_t K,
+                                w8a8_stream_t stream);
+
 /* ---- path selection (tests and benchmarks) ---------------------------------
  * 0 = automatic (default); 1 = always the persistent large-M GEMM (automatic
  * tile width); 2 = the small-M weight-streaming kernel (M <= 16 only, else

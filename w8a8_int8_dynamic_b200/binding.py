@@ -54,6 +54,8 @@ _SIGNATURES = {
     "w8a8_scaled_mm_i32": ([_P, _P, _P, _I64, _I64, _I64, _P], ctypes.c_int),
     "w8a8_linear_workspace_bytes": ([_I64, _I64, _I64, ctypes.POINTER(_SZ)], ctypes.c_int),
     "w8a8_linear": ([_P, _I64, _P, _P, _P, _P, _I64, _I64, _I64, _P, _SZ, _P], ctypes.c_int),
+    "w8a8_linear_noalloc_max_bytes": ([], _SZ),
+    "w8a8_linear_noalloc": ([_P, _I64, _P, _P, _P, _P, _I64, _I64, _I64, _P], ctypes.c_int),
     "w8a8_set_path": ([ctypes.c_int], ctypes.c_int),
     "w8a8_gelu_tanh": ([_P, _P, _I64, _P], ctypes.c_int),
     "w8a8_poll_status": ([_P], ctypes.c_int),
@@ -206,6 +208,33 @@ def linear(x: torch.Tensor, packed_w: torch.Tensor, w_scale: torch.Tensor,
                              _ptr(out), M, N, K, _ptr(workspace), ws_bytes, _stream(stream)),
            "w8a8_linear")
     return out.view(*lead, N)
+
+
+def linear_noalloc(x: torch.Tensor, packed_w: torch.Tensor, w_scale: torch.Tensor,
+                   bias: Optional[torch.Tensor], N: int, out: Optional[torch.Tensor] = None,
+                   stream=None) -> torch.Tensor:
+    """The whole layer with no workspace argument, for callers that cannot
+    allocate device memory when they run a layer: the library keeps one
+    scratch array per GPU (``linear_noalloc_max_bytes()`` bytes) for the codes,
+    scales and small-M partials.  Calls that overlap on the GPU share it and
+    race; order them on one stream."""
+    _need_cuda(x, "x", torch.bfloat16)
+    lead = x.shape[:-1]
+    K = x.shape[-1]
+    x2 = x.reshape(-1, K)
+    if x2.stride(1) != 1:
+        x2 = x2.contiguous()
+    M = x2.shape[0]
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.bfloat16, device=x.device)
+    _check(lib().w8a8_linear_noalloc(_ptr(x2), x2.stride(0), _ptr(packed_w), _ptr(w_scale), _ptr(bias),
+                                     _ptr(out), M, N, K, _stream(stream)),
+           "w8a8_linear_noalloc")
+    return out.view(*lead, N)
+
+
+def linear_noalloc_max_bytes() -> int:
+    return int(lib().w8a8_linear_noalloc_max_bytes())
 
 
 def gelu_tanh(x: torch.Tensor, out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
