@@ -37,6 +37,7 @@
 #include <cuda_bf16.h>
 
 #include <algorithm>
+#include <cstring>
 
 #include "gemm_common.cuh"
 
@@ -53,7 +54,8 @@ struct LargeSmem {
   // per epilogue warp: the tile's BN w_scale (fp32) and BN bias (bf16) values
   static constexpr int kEpiPerWarp = BN * 4 + BN * 2;
   static constexpr int kEpi = kB + STAGES * BN * kBK;
-  static constexpr int kBars = kEpi + 4 * kEpiPerWarp;  // full[S], empty[S], tfull[2], tempty[2], mma_done
+  static constexpr int kOut = kEpi + 4 * kEpiPerWarp + 1024 - (kEpi + 4 * kEpiPerWarp) % 1024;
+  static constexpr int kBars = kOut + 4 * kEpiStagePerWarp;  // full[S], empty[S], tfull[2], tempty[2], done
   static constexpr int kMisc = kBars + (2 * STAGES + 5) * 8;
   static constexpr int kUsed = kMisc + 16;
   static constexpr int kAlloc = kUsed + 1024;  // slack for 1024-byte alignment
@@ -61,7 +63,8 @@ struct LargeSmem {
 
 template <int BN, int STAGES, bool OUT_I32>
 __global__ void __launch_bounds__(kThreads, 1)
-    gemm_kernel(const __grid_constant__ CUtensorMap tmap_q, const GemmArgs args) {
+    gemm_kernel(const __grid_constant__ CUtensorMap tmap_q,
+                const __grid_constant__ CUtensorMap tmap_y, const GemmArgs args) {
   using L = LargeSmem<BN, STAGES>;
   constexpr uint32_t kTmemCols = 2 * BN;  // two accumulator buffers
   constexpr uint32_t kStageBytes = kTileBytes + BN * kBK;
@@ -202,6 +205,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int quarter = warp & 3;  // TMEM lanes this warp may access
     float *s_ws = reinterpret_cast<float *>(smem + L::kEpi + (warp - 2) * L::kEpiPerWarp);
     uint16_t *s_bias = reinterpret_cast<uint16_t *>(s_ws + BN);
+    uint8_t *s_out = smem + L::kOut + (warp - 2) * kEpiStagePerWarp;
+    uint32_t out_count = 0;
     for (int t = 0; t < my_tiles; ++t) {
       const int tile = blockIdx.x + t * gridDim.x;
       const int mb = tile % args.tiles_m, nb = tile / args.tiles_m;
@@ -219,12 +224,18 @@ __global__ void __launch_bounds__(kThreads, 1)
       ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
       if (!ok) break;
       tc_fence_after();
-      epilogue_tile<BN, OUT_I32>(args, tmem_base + b * BN, quarter, lane, mb * kBM, nb, as, s_ws,
-                                 s_bias);
+      if (OUT_I32)
+        epilogue_tile<BN, true>(args, tmem_base + b * BN, quarter, lane, mb * kBM, nb, as, s_ws,
+                                s_bias);
+      else
+        epilogue_tile_tma<BN>(args, &tmap_y, tmem_base + b * BN, quarter, lane, mb * kBM, nb, as,
+                              s_ws, s_bias, s_out, out_count, nullptr, NoExtra());
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&tempty[b]);
     }
+    if (lane == 0) bulk_wait_group_all();  // output stores complete before exit
+    __syncwarp();
   }
 
   tc_fence_before();
@@ -519,9 +530,9 @@ cudaError_t set_smem_attr(Kernel k, int bytes, int slot) {
   return e;
 }
 
-template <typename Kernel, typename Args>
+template <typename Kernel, typename... Args>
 cudaError_t launch_ex(Kernel k, int grid, int smem, cudaStream_t stream, bool pdl,
-                      const CUtensorMap &tmap, const Args &args) {
+                      const Args &...args) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)grid);
   cfg.blockDim = dim3(kThreads);
@@ -532,12 +543,12 @@ cudaError_t launch_ex(Kernel k, int grid, int smem, cudaStream_t stream, bool pd
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = pdl ? attr : nullptr;
   cfg.numAttrs = pdl ? 1 : 0;
-  return cudaLaunchKernelEx(&cfg, k, tmap, args);
+  return cudaLaunchKernelEx(&cfg, k, args...);
 }
 
 template <int BN, int STAGES, bool OUT_I32>
-w8a8_status run_large(const CUtensorMap &tmap, GemmArgs args, cudaStream_t stream, bool pdl,
-                      int slot) {
+w8a8_status run_large(const CUtensorMap &tmap, const CUtensorMap &tmap_y, GemmArgs args,
+                      cudaStream_t stream, bool pdl, int slot) {
   using L = LargeSmem<BN, STAGES>;
   auto k = gemm_kernel<BN, STAGES, OUT_I32>;
   cudaError_t e = set_smem_attr(k, L::kAlloc, slot);
@@ -545,7 +556,7 @@ w8a8_status run_large(const CUtensorMap &tmap, GemmArgs args, cudaStream_t strea
   args.tiles_n = (int)((args.N + BN - 1) / BN);
   const int tiles = args.tiles_m * args.tiles_n;
   const int grid = std::min(tiles, sm_count());
-  e = launch_ex(k, grid, L::kAlloc, stream, pdl, tmap, args);
+  e = launch_ex(k, grid, L::kAlloc, stream, pdl, tmap, tmap_y, args);
   count_launch();
   return from_cuda(e);
 }
@@ -555,22 +566,31 @@ w8a8_status run_large(const CUtensorMap &tmap, GemmArgs args, cudaStream_t strea
 // ~128 B/clk per SM, the 128 x 256 tile ~94, the 2-SM 256 x 256 tile ~64),
 // so the cost of a shape is its wave count times its per-SM tile work divided
 // by the fraction of the rate it sustains.
-enum class LargeKind { k128, k256, kPair };
+enum class LargeKind { k128, k256, kPair, kPairSplit };
 
-LargeKind choose_large(int64_t M, int64_t N) {
+LargeKind choose_large(int64_t M, int64_t N, int64_t K) {
   const int path = forced_path();
   if (path == 3) return LargeKind::k128;
   if (path == 4) return LargeKind::k256;
   if (path == 5) return LargeKind::kPair;
+  if (path == 6) return LargeKind::kPairSplit;
   const int64_t sms = sm_count();
   const int64_t tm = (M + kBM - 1) / kBM;
   const int64_t t128 = tm * ((N + 127) / 128), t256 = tm * ((N + 255) / 256);
-  const int64_t tpair = pair_tiles(M, N), pairs = sms / 2;
+  const int64_t tpair = pair_tiles(M, N), pairs = sms / 2, quads = sms / 4;
   const double c128 = (double)((t128 + sms - 1) / sms) * 128.0 / 0.45;
   const double c256 = (double)((t256 + sms - 1) / sms) * 256.0 / 0.60;
   const double cpair = (double)((tpair + pairs - 1) / pairs) * 256.0 / 0.85;
-  if (cpair <= c128 && cpair <= c256) return LargeKind::kPair;
-  return c256 <= c128 ? LargeKind::k256 : LargeKind::k128;
+  // half the K per cluster of two pairs, plus the exchange of one partial
+  const bool can_split = (packed_cols(K) / 128 + 1) / 2 >= 2;
+  const double csplit =
+      can_split ? (double)((tpair + quads - 1) / quads) * 128.0 / 0.85 * 1.15 : 1e30;
+  double best = c128;
+  LargeKind kind = LargeKind::k128;
+  if (c256 < best) best = c256, kind = LargeKind::k256;
+  if (cpair <= best) best = cpair, kind = LargeKind::kPair;
+  if (csplit < best) best = csplit, kind = LargeKind::kPairSplit;
+  return kind;
 }
 
 }  // namespace
@@ -600,7 +620,7 @@ int64_t decode_workspace_bytes(int64_t N, int64_t K) {
 bool use_decode_path(int64_t M) {
   const int p = forced_path();
   if (p == 2) return M <= kDecodeNT;
-  if (p == 1 || p == 3 || p == 4 || p == 5) return false;
+  if (p == 1 || p >= 3) return false;
   return M <= kDecodeNT;
 }
 
@@ -663,19 +683,26 @@ w8a8_status launch_scaled_mm(const int8_t *q, const float *a_scale, const void *
   a.tiles_n = 0;
   a.status = status_word();
   if (!a.status) return W8A8_ERR_CUDA;
+  CUtensorMap tmap_y;
   if (out_i32) {
-    // the int32 export always uses the 1-SM kernel (tests and inspection)
-    const LargeKind kind = choose_large(M, N);
-    return kind == LargeKind::k128 ? run_large<128, kLargeStages128, true>(tmap, a, stream, pdl, 1)
-                                   : run_large<256, kLargeStages256, true>(tmap, a, stream, pdl, 0);
+    // the int32 export always uses the 1-SM kernel (tests and inspection); it
+    // stores from registers and takes no output tensor map
+    memset(&tmap_y, 0, sizeof(tmap_y));
+    const LargeKind kind = choose_large(M, N, K);
+    return kind == LargeKind::k128
+               ? run_large<128, kLargeStages128, true>(tmap, tmap_y, a, stream, pdl, 1)
+               : run_large<256, kLargeStages256, true>(tmap, tmap_y, a, stream, pdl, 0);
   }
-  switch (choose_large(M, N)) {
+  if (!make_tmap_out_bf16(&tmap_y, out, (uint64_t)M, (uint64_t)N)) return W8A8_ERR_CUDA;
+  switch (choose_large(M, N, K)) {
     case LargeKind::kPair:
-      return launch_gemm2sm(q, a_scale, packed_w, w_scale, bias, out, M, N, K, stream, pdl);
+      return launch_gemm2sm(q, a_scale, packed_w, w_scale, bias, out, M, N, K, stream, pdl, 1);
+    case LargeKind::kPairSplit:
+      return launch_gemm2sm(q, a_scale, packed_w, w_scale, bias, out, M, N, K, stream, pdl, 2);
     case LargeKind::k256:
-      return run_large<256, kLargeStages256, false>(tmap, a, stream, pdl, 2);
+      return run_large<256, kLargeStages256, false>(tmap, tmap_y, a, stream, pdl, 2);
     default:
-      return run_large<128, kLargeStages128, false>(tmap, a, stream, pdl, 3);
+      return run_large<128, kLargeStages128, false>(tmap, tmap_y, a, stream, pdl, 3);
   }
 }
 

@@ -3,14 +3,13 @@
 // Same arithmetic as gemm.cu ("Issue 5 probe: int8 quantized DiT serve paths
 // on the RTX 3090", Round two: int8 scaled matmul with per-token and
 // per-channel fp32 scales; "INT8 Quant for Dual-Max Recipe": native int8 x int8
-// on the tensor cores), organised for a CTA pair (a 2-CTA cluster):
+// on the tensor cores), organised for CTA pairs:
 //
-//   * output tiles are 256 x 256; the even CTA owns rows 0..127 of the tile,
-//     the odd CTA rows 128..255.  Each CTA loads only its own 128 rows of q
-//     and its own 128-row slab of the packed weights (the tile's N half), so
-//     per SM a k-block moves 32 KB for 128 x 256 x 128 MACs -- two thirds of
-//     what a 1-SM 128 x 256 tile moves, which is what lets the tensor pipe be
-//     fed from L2 at the int8 rate;
+//   * output tiles are 256 x 256; the even CTA of a pair owns rows 0..127 of
+//     the tile, the odd CTA rows 128..255.  Each CTA loads only its own 128
+//     rows of q and its own 128-row slab of the packed weights (the tile's N
+//     half), so per SM a k-block moves 32 KB for 128 x 256 x 128 MACs -- two
+//     thirds of what a 1-SM 128 x 256 tile moves;
 //   * a pipeline stage holds two k-blocks (64 KB per CTA), fetched with three
 //     TMA copies (two q boxes, one 32 KB box of two contiguous packed weight
 //     tiles), all completing on the even CTA's "full" barrier;
@@ -18,12 +17,19 @@
 //     (M = 256, N = 256, K = 32), which reads both CTAs' shared memory and
 //     accumulates into both CTAs' TMEM; its commits arrive on the "empty" and
 //     "accumulator full" barriers of both CTAs (commit multicast);
-//   * both CTAs run the epilogue on their own 128 TMEM lanes and tell the
-//     even CTA when an accumulator buffer may be reused.
+//   * both CTAs run the epilogue on their own 128 TMEM lanes.
 //
-// No TMA load uses cluster multicast.  Every wait is time-bounded; a block
-// that gives up drains its copies, the pair meets at a cluster barrier and
-// frees TMEM.
+// SPLIT = 1: persistent clusters of 2 CTAs, double-buffered accumulators.
+// SPLIT = 2: clusters of 4 CTAs = two pairs computing one tile over the two
+//   halves of K (for problems with too few tiles to fill the GPU).  The second
+//   pair writes its int32 partial into its own (then idle) stage buffers and
+//   ships it with one DSMEM bulk copy into the first pair's stage buffers; the
+//   first pair adds it -- exactly, in int32 -- before the scale arithmetic.
+//
+// No TMA load uses cluster multicast.  Every wait is time-bounded (the waits
+// between the two pairs of a cluster are safe: a cluster's CTAs are
+// co-scheduled); a block that gives up drains its copies, the cluster meets
+// at a barrier and frees TMEM.
 #include <algorithm>
 
 #include "gemm_common.cuh"
@@ -31,9 +37,10 @@
 namespace w8a8 {
 namespace {
 
-constexpr int kPairBN = 256;                 // tile N (both CTAs)
-constexpr int kStageK = 2;                   // k-blocks per stage
+constexpr int kPairBN = 256;                      // tile N (both CTAs)
+constexpr int kStageK = 2;                        // k-blocks per stage
 constexpr int kHalfStage = kStageK * kTileBytes;  // 32 KB: one operand of one stage
+constexpr int kPartialBytes = 128 * kPairBN * 4;  // one CTA's int32 partial: 128 KB
 
 template <int STAGES>
 struct PairSmem {
@@ -41,16 +48,28 @@ struct PairSmem {
   static constexpr int kB = STAGES * kHalfStage;        // STAGES x 32 KB weight tiles
   static constexpr int kEpiPerWarp = kPairBN * 4 + kPairBN * 2;
   static constexpr int kEpi = kB + STAGES * kHalfStage;
-  static constexpr int kBars = kEpi + 4 * kEpiPerWarp;  // full, empty, tfull[2], tempty[2], done
-  static constexpr int kMisc = kBars + (2 * STAGES + 5) * 8;
+  static constexpr int kOut = kEpi + 4 * kEpiPerWarp + 1024 - (kEpi + 4 * kEpiPerWarp) % 1024;
+  // full[S], empty[S], tfull[2], tempty[2], done, ready, recv
+  static constexpr int kBars = kOut + 4 * kEpiStagePerWarp;
+  static constexpr int kMisc = kBars + (2 * STAGES + 7) * 8;
   static constexpr int kUsed = kMisc + 16;
   static constexpr int kAlloc = kUsed + 1024;
+  static_assert(2 * STAGES * kHalfStage >= kPartialBytes, "partial must fit the stage buffers");
 };
 
-template <int STAGES>
+// int32 partial layout in shared memory: element (row r, column j) at
+// ((j / 4) * 128 + r) * 4 + j % 4, so the 32 lanes (rows) of a warp move 512
+// contiguous bytes per 16-byte access.
+__device__ __forceinline__ int partial_index(int r, int j) { return ((j >> 2) * 128 + r) * 4 + (j & 3); }
+struct PartialIndex {
+  __device__ int operator()(int r, int j) const { return partial_index(r, j); }
+};
+
+template <int STAGES, int SPLIT>
 __global__ void __launch_bounds__(kThreads, 1)
     gemm2sm_kernel(const __grid_constant__ CUtensorMap tmap_q,
-                   const __grid_constant__ CUtensorMap tmap_w, const GemmArgs args) {
+                   const __grid_constant__ CUtensorMap tmap_w,
+                   const __grid_constant__ CUtensorMap tmap_y, const GemmArgs args) {
   using L = PairSmem<STAGES>;
   constexpr uint32_t kTmemCols = 2 * kPairBN;
   constexpr uint32_t kIdesc = idesc_i8(256, kPairBN);
@@ -65,11 +84,20 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t *tfull = empty + STAGES;
   uint64_t *tempty = tfull + 2;
   uint64_t *mma_done = tempty + 2;
+  uint64_t *ready = mma_done + 1;  // (second pair) the first pair's buffers are free
+  uint64_t *recv = ready + 1;      // (first pair) the partial has arrived
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + L::kMisc);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + L::kMisc + 4);
+  int32_t *partial = reinterpret_cast<int32_t *>(smem);  // aliases the stage buffers
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const uint32_t rank = cluster_ctarank();  // 0: even CTA (issues the MMAs), 1: odd CTA
+  const uint32_t crank = cluster_ctarank();
+  const uint32_t rank = crank & 1;      // 0: even CTA of the pair (issues the MMAs)
+  const uint32_t ksplit = crank >> 1;   // which K part this pair computes (SPLIT = 2)
+  const uint32_t lead = crank & ~1u;    // cluster rank of this pair's even CTA
+  // commit multicast masks are in cluster-rank space
+  const uint16_t pair_mask = (uint16_t)(0x3u << lead);
+  const uint16_t self_mask = (uint16_t)(0x1u << crank);
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(&full[s], 2);  // one expect_tx arrival from each CTA of the pair
@@ -80,6 +108,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&tempty[b], 8);  // four epilogue warps in each CTA
     }
     mbar_init(mma_done, 1);
+    mbar_init(ready, 1);
+    mbar_init(recv, 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -89,33 +119,37 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   if (warp == 1) tmem_alloc_pair(tmem_slot, kTmemCols);
   tc_fence_before();
-  cluster_sync();  // barriers of both CTAs initialised, TMEM allocated in both
+  cluster_sync();  // barriers of the cluster initialised, TMEM allocated
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
 
   const int num_tiles = args.tiles_m * args.tiles_n;  // 256 x 256 tiles
   const int num_kb = args.num_kb;
-  const int num_stages_k = (num_kb + kStageK - 1) / kStageK;
-  const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
-  const int my_tiles = pair < num_tiles ? (num_tiles - 1 - pair) / npairs + 1 : 0;
-  const uint32_t my_iters = (uint32_t)my_tiles * num_stages_k;
-  const uint32_t full0 = map_to_cta(smem_addr(full), 0);  // even CTA's full[0]
-  const uint32_t tempty0 = map_to_cta(smem_addr(tempty), 0);
+  const int stages_total = (num_kb + kStageK - 1) / kStageK;
+  // this pair's share of the K stages
+  const int st_begin = SPLIT == 1 ? 0 : (ksplit == 0 ? 0 : stages_total / 2);
+  const int st_end = SPLIT == 1 ? stages_total : (ksplit == 0 ? stages_total / 2 : stages_total);
+  const int nst = st_end - st_begin;
+  const int slot = SPLIT == 1 ? (int)(blockIdx.x >> 1) : (int)(blockIdx.x >> 2);
+  const int nslots = SPLIT == 1 ? (int)(gridDim.x >> 1) : (int)(gridDim.x >> 2);
+  const int my_tiles = slot < num_tiles ? (num_tiles - 1 - slot) / nslots + 1 : 0;
+  const uint32_t my_iters = (uint32_t)my_tiles * nst;
+  const uint32_t full0 = map_to_cta(smem_addr(full), lead);  // pair leader's full[0]
+  const uint32_t tempty0 = map_to_cta(smem_addr(tempty), lead);
 
   if (warp == 0) {
     if (lane == 0) {
-      // ---------------- producer (both CTAs) ----------------
-      auto tile_of = [&](uint32_t it) { return pair + (int)(it / num_stages_k) * npairs; };
+      // ---------------- producer (every CTA) ----------------
       auto issue = [&](uint32_t it, uint32_t s, bool weights, bool acts) {
-        const int tile = tile_of(it);
+        const int tile = slot + (int)(it / nst) * nslots;
         const int mb = tile % args.tiles_m, nb = tile / args.tiles_m;
-        const int kb0 = (int)(it % num_stages_k) * kStageK;
+        const int kb0 = (st_begin + (int)(it % nst)) * kStageK;
         const int nk = min(kStageK, num_kb - kb0);
         const uint32_t bar = full0 + s * 8;
         if (weights) {
           // two contiguous packed tiles (k-blocks kb0, kb0+1) of this CTA's slab
-          const int slab = nb * 2 + (int)rank;
-          tma_load_2d_pair(sB + s * kHalfStage, &tmap_w, 0, (slab * num_kb + kb0) * 128, bar);
+          const int wslab = nb * 2 + (int)rank;
+          tma_load_2d_pair(sB + s * kHalfStage, &tmap_w, 0, (wslab * num_kb + kb0) * 128, bar);
         }
         if (acts) {
           const int row0 = mb * 256 + (int)rank * 128;
@@ -125,7 +159,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       };
       auto stage_bytes = [&](uint32_t it) {
-        const int kb0 = (int)(it % num_stages_k) * kStageK;
+        const int kb0 = (st_begin + (int)(it % nst)) * kStageK;
         return (uint32_t)(kHalfStage + min(kStageK, num_kb - kb0) * kTileBytes);
       };
       uint32_t last_par[STAGES];
@@ -151,17 +185,17 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       // Wait until every stage this CTA filled has been consumed: the MMA
       // commits that release them also arrive here, and must land before the
-      // pair may leave.  On abort, wait for our own copies instead.
+      // CTA may leave (and, with SPLIT = 2, before the stage buffers are
+      // reused for the partial).
       for (uint32_t s = 0; s < (uint32_t)STAGES && s < my_iters; ++s) {
         volatile int no_abort = 0;
-        if (ok)
-          (void)mbar_wait_bounded(&empty[s], last_par[s], &no_abort, args.status);
+        if (ok) (void)mbar_wait_bounded(&empty[s], last_par[s], &no_abort, args.status);
       }
     }
     __syncwarp();
   } else if (warp == 1) {
     if (lane == 0 && rank == 0) {
-      // ---------------- MMA issuer (even CTA) ----------------
+      // ---------------- MMA issuer (even CTA of each pair) ----------------
       uint32_t it = 0;
       bool ok = true;
       for (int t = 0; ok && t < my_tiles; ++t) {
@@ -172,14 +206,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + b * kPairBN;
-        for (int j = 0; j < num_stages_k; ++j, ++it) {
+        for (int j = 0; j < nst; ++j, ++it) {
           const uint32_t s = it % STAGES, ph = (it / STAGES) & 1;
           if (!mbar_wait(&full[s], ph, abort_flag, args.status)) {
             ok = false;
             break;
           }
           tc_fence_after();
-          const int nk = min(kStageK, num_kb - j * kStageK);
+          const int nk = min(kStageK, num_kb - (st_begin + j) * kStageK);
           for (int h = 0; h < nk; ++h) {
             const uint64_t a_desc = sw128_kmajor_desc(sA + s * kHalfStage + h * kTileBytes);
             const uint64_t b_desc = sw128_kmajor_desc(sB + s * kHalfStage + h * kTileBytes);
@@ -187,29 +221,32 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int k = 0; k < kBK / 32; ++k)
               mma_i8_pair(d_tmem, a_desc + 2 * k, b_desc + 2 * k, kIdesc, (j | h | k) != 0);
           }
-          mma_commit_pair(&empty[s], 0x3);  // frees the stage in both CTAs
+          mma_commit_pair(&empty[s], pair_mask);  // frees the stage in both CTAs
         }
-        if (ok) mma_commit_pair(&tfull[b], 0x3);
+        if (ok) mma_commit_pair(&tfull[b], pair_mask);
       }
       if (!ok) {
-        mma_commit_pair(mma_done, 0x1);
+        mma_commit_pair(mma_done, self_mask);
         volatile int no_abort = 0;
         (void)mbar_wait_bounded(mma_done, 0, &no_abort, args.status);
       }
     }
     __syncwarp();
   } else {
-    // ---------------- epilogue (warps 2..5, both CTAs) ----------------
+    // ---------------- epilogue (warps 2..5, every CTA) ----------------
     griddep_wait();  // a_scale comes from the preceding kernel
     const int quarter = warp & 3;
+    const int et = threadIdx.x - 64;  // 0..127
     float *s_ws = reinterpret_cast<float *>(smem + L::kEpi + (warp - 2) * L::kEpiPerWarp);
     uint16_t *s_bias = reinterpret_cast<uint16_t *>(s_ws + kPairBN);
+    uint8_t *s_out = smem + L::kOut + (warp - 2) * kEpiStagePerWarp;
+    uint32_t out_count = 0;
     for (int t = 0; t < my_tiles; ++t) {
-      const int tile = pair + t * npairs;
+      const int tile = slot + t * nslots;
       const int mb = tile % args.tiles_m, nb = tile / args.tiles_m;
       const int row_base = mb * 256 + (int)rank * 128;
       const uint32_t b = t & 1, bph = (t >> 1) & 1;
-      stage_columns<kPairBN>(args, nb, lane, s_ws, s_bias);
+      if (SPLIT == 1 || ksplit == 0) stage_columns<kPairBN>(args, nb, lane, s_ws, s_bias);
       const int row = row_base + quarter * 32 + lane;
       const float as = row < args.M ? __ldg(args.a_scale + row) : 0.0f;
       __syncwarp();
@@ -218,16 +255,61 @@ __global__ void __launch_bounds__(kThreads, 1)
       ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
       if (!ok) break;
       tc_fence_after();
-      epilogue_tile<kPairBN, false>(args, tmem_base + b * kPairBN, quarter, lane, row_base, nb, as,
-                                    s_ws, s_bias);
+      const uint32_t taddr = tmem_base + b * kPairBN + ((uint32_t)(quarter * 32) << 16);
+      const int r = quarter * 32 + lane;  // row within this CTA's 128
+      if (SPLIT == 2 && ksplit == 1) {
+        // Second pair: stage the int32 partial in this CTA's stage buffers
+        // (all consumed: the producer waited for that) and ship it to the
+        // first pair's CTA of the same rank once its buffers are free.
+#pragma unroll 1
+        for (int c = 0; c < kPairBN / 32; ++c) {
+          uint32_t v[32];
+          tmem_ld_32x32b_x32(taddr + c * 32, v);
+          tmem_ld_wait();
+#pragma unroll
+          for (int g = 0; g < 8; ++g)
+            *reinterpret_cast<uint4 *>(partial + partial_index(r, c * 32 + 4 * g)) =
+                make_uint4(v[4 * g], v[4 * g + 1], v[4 * g + 2], v[4 * g + 3]);
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        asm volatile("bar.sync 1, 128;" ::: "memory");
+        if (et == 0) {
+          if (mbar_wait(ready, 0, abort_flag, args.status)) {
+            const uint32_t dst_cta = crank - 2;
+            bulk_copy_s2cluster(map_to_cta(smem_addr(partial), dst_cta), partial, kPartialBytes,
+                                map_to_cta(smem_addr(recv), dst_cta));
+          }
+        }
+        __syncwarp();
+      } else {
+        if (SPLIT == 2) {
+          // First pair: every stage is consumed (tfull), so the stage buffers
+          // may receive the partner pair's partial now.
+          if (et == 0) {
+            mbar_arrive_expect_tx(recv, kPartialBytes);
+            mbar_arrive_cluster(map_to_cta(smem_addr(ready), crank + 2));
+          }
+          int got = 0;
+          if (lane == 0) got = mbar_wait(recv, 0, abort_flag, args.status);
+          got = __shfl_sync(0xFFFFFFFFu, got, 0);
+          if (!got) break;
+        }
+        // dequantise: (acc [+ partner partial]) * a_scale * w_scale + bias
+        epilogue_tile_tma<kPairBN>(args, &tmap_y, tmem_base + b * kPairBN, quarter, lane,
+                                   row_base, nb, as, s_ws, s_bias, s_out, out_count,
+                                   SPLIT == 2 ? partial : nullptr, PartialIndex());
+      }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive_cluster(tempty0 + b * 8);
+      if (SPLIT == 1 && lane == 0) mbar_arrive_cluster(tempty0 + b * 8);
     }
+    if (lane == 0) bulk_wait_group_all();  // output stores complete before exit
+    __syncwarp();
   }
 
   tc_fence_before();
-  cluster_sync();  // no CTA leaves while its peer may still touch its memory
+  cluster_sync();  // no CTA leaves while a peer may still touch its memory
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc_pair(tmem_base, kTmemCols);
@@ -235,7 +317,42 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 constexpr int kPairStages = 3;
-bool g_pair_attr_done[64];
+bool g_pair_attr_done[64][2];
+
+template <int SPLIT>
+w8a8_status run_pair(const CUtensorMap &tq, const CUtensorMap &tw, const CUtensorMap &ty,
+                     const GemmArgs &a, cudaStream_t stream, bool pdl) {
+  using L = PairSmem<kPairStages>;
+  auto k = gemm2sm_kernel<kPairStages, SPLIT>;
+  const int d = current_device();
+  if (d < 0 || d >= 64 || !g_pair_attr_done[d][SPLIT - 1]) {
+    if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kAlloc) !=
+        cudaSuccess)
+      return W8A8_ERR_CUDA;
+    if (d >= 0 && d < 64) g_pair_attr_done[d][SPLIT - 1] = true;
+  }
+  const int tiles = a.tiles_m * a.tiles_n;
+  const int cta_per_cluster = 2 * SPLIT;
+  // SPLIT = 1: persistent, one pair per two SMs; SPLIT = 2: one tile per cluster.
+  const int clusters = SPLIT == 1 ? std::max(1, std::min(tiles, sm_count() / 2)) : tiles;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)(cta_per_cluster * clusters));
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = (size_t)L::kAlloc;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = (unsigned)cta_per_cluster;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 2 : 1;
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, k, tq, tw, ty, a);
+  count_launch();
+  return from_cuda(e);
+}
 
 }  // namespace
 
@@ -244,10 +361,11 @@ int64_t pair_tiles(int64_t M, int64_t N) { return ((M + 255) / 256) * ((N + 255)
 
 w8a8_status launch_gemm2sm(const int8_t *q, const float *a_scale, const void *packed_w,
                            const float *w_scale, const void *bias, void *y, int64_t M, int64_t N,
-                           int64_t K, cudaStream_t stream, bool pdl) {
-  CUtensorMap tq, tw;
+                           int64_t K, cudaStream_t stream, bool pdl, int split) {
+  CUtensorMap tq, tw, ty;
   if (!make_tmap_u8_2d(&tq, q, (uint64_t)M, (uint64_t)K, (uint64_t)K, kBM, kBK))
     return W8A8_ERR_CUDA;
+  if (!make_tmap_out_bf16(&ty, y, (uint64_t)M, (uint64_t)N)) return W8A8_ERR_CUDA;
   const uint64_t wrows = (uint64_t)(packed_rows(N) * packed_cols(K) / 128);
   if (!make_tmap_u8_2d_plain(&tw, packed_w, wrows, 128, 128, 256, 128)) return W8A8_ERR_CUDA;
   GemmArgs a;
@@ -263,34 +381,10 @@ w8a8_status launch_gemm2sm(const int8_t *q, const float *a_scale, const void *pa
   a.tiles_n = (int)((N + 255) / 256);
   a.status = status_word();
   if (!a.status) return W8A8_ERR_CUDA;
-  using L = PairSmem<kPairStages>;
-  auto k = gemm2sm_kernel<kPairStages>;
-  const int d = current_device();
-  if (d < 0 || d >= 64 || !g_pair_attr_done[d]) {
-    if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kAlloc) !=
-        cudaSuccess)
-      return W8A8_ERR_CUDA;
-    if (d >= 0 && d < 64) g_pair_attr_done[d] = true;
-  }
-  const int tiles = a.tiles_m * a.tiles_n;
-  const int pairs = std::max(1, std::min(tiles, sm_count() / 2));
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((unsigned)(2 * pairs));
-  cfg.blockDim = dim3(kThreads);
-  cfg.dynamicSmemBytes = (size_t)L::kAlloc;
-  cfg.stream = stream;
-  cudaLaunchAttribute attr[2];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = 2;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[1].val.programmaticStreamSerializationAllowed = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = pdl ? 2 : 1;
-  const cudaError_t e = cudaLaunchKernelEx(&cfg, k, tq, tw, a);
-  count_launch();
-  return from_cuda(e);
+  // the split needs at least one stage per half
+  if (split == 2 && (a.num_kb + kStageK - 1) / kStageK >= 2)
+    return run_pair<2>(tq, tw, ty, a, stream, pdl);
+  return run_pair<1>(tq, tw, ty, a, stream, pdl);
 }
 
 }  // namespace w8a8

@@ -36,6 +36,9 @@ bool make_tmap_u8_2d(CUtensorMap *map, const void *base, uint64_t rows, uint64_t
 bool make_tmap_u8_2d_plain(CUtensorMap *map, const void *base, uint64_t rows, uint64_t cols,
                            uint64_t ld, uint32_t box_rows, uint32_t box_cols);
 
+// bf16 output y[M, N] for TMA stores: box 32 x 32, 64-byte swizzle.
+bool make_tmap_out_bf16(CUtensorMap *map, const void *y, uint64_t M, uint64_t N);
+
 inline bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 inline w8a8_status from_cuda(cudaError_t e) { return e == cudaSuccess ? W8A8_OK : W8A8_ERR_CUDA; }
@@ -56,7 +59,7 @@ w8a8_status launch_scaled_mm(const int8_t *q, const float *a_scale, const void *
 // 2-SM (CTA pair) GEMM with the bf16 epilogue (gemm2sm.cu).
 w8a8_status launch_gemm2sm(const int8_t *q, const float *a_scale, const void *packed_w,
                            const float *w_scale, const void *bias, void *y, int64_t M, int64_t N,
-                           int64_t K, cudaStream_t stream, bool pdl);
+                           int64_t K, cudaStream_t stream, bool pdl, int split);
 int64_t pair_tiles(int64_t M, int64_t N);
 // Quantisation launcher (quant.cu).
 w8a8_status launch_quant(const void *x, int64_t M, int64_t K, int64_t ldx, int8_t *q,

@@ -93,6 +93,22 @@ bool make_tmap_u8_2d_plain(CUtensorMap *map, const void *base, uint64_t rows, ui
   return encode_u8_2d(map, base, rows, cols, ld, box_rows, box_cols, CU_TENSOR_MAP_SWIZZLE_NONE);
 }
 
+bool make_tmap_out_bf16(CUtensorMap *map, const void *y, uint64_t M, uint64_t N) {
+  if (!g_encode) {
+    CUtensorMap tmp;
+    if (!encode_u8_2d(&tmp, y, 1, 16, 16, 1, 16, CU_TENSOR_MAP_SWIZZLE_NONE)) return false;
+  }
+  const cuuint64_t dims[2] = {N, M};
+  const cuuint64_t strides[1] = {N * 2};
+  const cuuint32_t box[2] = {32, 32};
+  const cuuint32_t estr[2] = {1, 1};
+  const CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(y),
+                              dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                              CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+                              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 // Waits on a barrier that nothing arrives at; the bounded wait must give up.
 __global__ void selftest_wait_kernel(int *status, uint64_t limit_ns) {
   __shared__ uint64_t bar;
@@ -132,7 +148,7 @@ const char *w8a8_status_string(int status) {
 int w8a8_abi_version(void) { return (1 << 16) | 0; }
 
 w8a8_status w8a8_set_path(int path) {
-  if (path < 0 || path > 5) return W8A8_ERR_INVALID_ARG;
+  if (path < 0 || path > 6) return W8A8_ERR_INVALID_ARG;
   g_forced_path.store(path);
   return W8A8_OK;
 }
