@@ -61,6 +61,12 @@ w8a8_status launch_gemm2sm(const int8_t *q, const float *a_scale, const void *pa
                            const float *w_scale, const void *bias, void *y, int64_t M, int64_t N,
                            int64_t K, cudaStream_t stream, bool pdl, int split);
 int64_t pair_tiles(int64_t M, int64_t N);
+// Small-M weight-streaming kernel (decode.cu).
+int64_t decode_workspace_bytes(int64_t N, int64_t K);
+bool use_decode_path(int64_t M);
+w8a8_status launch_decode(const int8_t *q, const float *a_scale, const void *packed_w,
+                          const float *w_scale, const void *bias, void *y, int64_t M,
+                          int64_t N, int64_t K, void *workspace, cudaStream_t stream, bool pdl);
 // Quantisation launcher (quant.cu).
 w8a8_status launch_quant(const void *x, int64_t M, int64_t K, int64_t ldx, int8_t *q,
                          float *a_scale, cudaStream_t stream);

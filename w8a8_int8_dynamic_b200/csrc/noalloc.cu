@@ -65,8 +65,8 @@ extern "C" w8a8_status w8a8_linear_noalloc(const void *x, int64_t ldx, const voi
   const w8a8_status sa = scratch_address(&scratch);
   if (sa != W8A8_OK) return sa;
   // Everything the layer reads from the scratch is written first in the same
-  // call (codes, scales), and the split-K counters are cleared at the start
-  // of every small-M call, so what a previous call left there does not matter.
+  // call (codes, scales, partials), and the small-M split-K counters carry a
+  // per-call tag, so what a previous call left there does not matter.
   return w8a8_linear(x, ldx, packed_w, w_scale, bias, y, M, N, K, scratch, kNoAllocScratchBytes,
                      stream);
 }

@@ -33,23 +33,24 @@ namespace {
 __device__ __forceinline__ float bf16_lo(uint32_t v) { return __uint_as_float(v << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t v) { return __uint_as_float(v & 0xFFFF0000u); }
 
+// Code of one element: rint(RN(x / s)).  y = RN(x * inv) is within 2.3e-5 of
+// RN(x / s), so rint(y) is the answer unless y lies within 1e-4 of a
+// half-integer, i.e. |y - rint(y)| > 0.4999 (it is always <= 0.5); only then
+// is the IEEE quotient formed.  |x| <= amax makes |y| <= 127 (1 + 2^-22), so
+// the result is always in [-127, 127] and needs no clamp.
 __device__ __forceinline__ int quant_one(float x, float s, float inv, bool exact_only) {
-  float r;
-  if (exact_only) {
-    r = rintf(__fdiv_rn(x, s));
-  } else {
-    const float y = __fmul_rn(x, inv);
-    r = rintf(y);
-    const float d = fabsf(y - r);  // exact: y and r are within 1/2 of each other
-    if (fabsf(d - 0.5f) < 1e-4f) r = rintf(__fdiv_rn(x, s));
-  }
-  r = fminf(fmaxf(r, -127.0f), 127.0f);
-  return static_cast<int>(r);
+  if (exact_only) return __float2int_rn(__fdiv_rn(x, s));
+  const float y = __fmul_rn(x, inv);
+  const float r = rintf(y);
+  if (fabsf(y - r) > 0.4999f) return __float2int_rn(__fdiv_rn(x, s));
+  return (int)r;
 }
 
+// Low bytes of four ints -> one word (byte permutes).
 __device__ __forceinline__ uint32_t pack4(int a, int b, int c, int d) {
-  return (uint32_t)(a & 0xFF) | ((uint32_t)(b & 0xFF) << 8) | ((uint32_t)(c & 0xFF) << 16) |
-         ((uint32_t)(d & 0xFF) << 24);
+  const uint32_t ab = __byte_perm((uint32_t)a, (uint32_t)b, 0x0040);
+  const uint32_t cd = __byte_perm((uint32_t)c, (uint32_t)d, 0x0040);
+  return __byte_perm(ab, cd, 0x5410);
 }
 
 template <int CHUNKS>
