@@ -146,7 +146,7 @@ def test_gemm_i32_extreme_values():
 
 @pytest.mark.parametrize("bias", [False, True])
 @pytest.mark.parametrize("path", [w8.PATH_LARGE_BN128, w8.PATH_LARGE_BN256, w8.PATH_LARGE_PAIR,
-                                  w8.PATH_LARGE_PAIR_SPLIT])
+                                  w8.PATH_LARGE_PAIR128, w8.PATH_LARGE_PAIR_SPLIT])
 @pytest.mark.parametrize("M,N,K", [(64, 128, 256), (129, 392, 400), (300, 1000, 528), (512, 1024, 4096),
                                    (257, 264, 272), (700, 520, 144)])
 def test_scaled_mm_matches_oracle(M, N, K, path, bias):
@@ -162,7 +162,8 @@ def test_scaled_mm_matches_oracle(M, N, K, path, bias):
     assert np.array_equal(y_h, y_ref), "expected bit-exact bf16"
 
 
-@pytest.mark.parametrize("path", [w8.PATH_LARGE_BN128, w8.PATH_LARGE_PAIR, w8.PATH_LARGE_PAIR_SPLIT])
+@pytest.mark.parametrize("path", [w8.PATH_LARGE_BN128, w8.PATH_LARGE_PAIR, w8.PATH_LARGE_PAIR128,
+                                  w8.PATH_LARGE_PAIR_SPLIT])
 def test_scaled_mm_does_not_write_outside_y(path):
     w8.set_path(path)
     M, N, K = 130, 264, 272
@@ -198,7 +199,8 @@ def test_decode_path_matches_oracle(M, N, K):
 
 
 # ---------------------------------------------------------------- fused layer
-@pytest.mark.parametrize("path", [w8.PATH_AUTO, w8.PATH_LARGE_PAIR, w8.PATH_LARGE_PAIR_SPLIT])
+@pytest.mark.parametrize("path", [w8.PATH_AUTO, w8.PATH_LARGE_PAIR, w8.PATH_LARGE_PAIR128,
+                                  w8.PATH_LARGE_PAIR_SPLIT])
 @pytest.mark.parametrize("M,N,K", [(1, 264, 400), (16, 1024, 1024), (17, 1024, 1024),
                                    (64, 128, 256), (300, 1000, 528), (512, 4096, 4096)])
 def test_linear_matches_oracle(M, N, K, path):

@@ -293,32 +293,42 @@ w8a8_status run_large(const CUtensorMap &tmap, const CUtensorMap &tmap_y, GemmAr
 // ~128 B/clk per SM, the 128 x 256 tile ~94, the 2-SM 256 x 256 tile ~64),
 // so the cost of a shape is its wave count times its per-SM tile work divided
 // by the fraction of the rate it sustains.
-enum class LargeKind { k128, k256, kPair, kPairSplit };
+enum class LargeKind { k128, k256, kPair, kPair128, kPairSplit };
 
+// Kernel choice for large M: (waves of tiles) x (per-SM time of one tile).
+// The per-SM time of a stage of two k-blocks is set by what has to reach the
+// SM from L2 (measured ~114 GB/s per SM with ~190 KB in flight) or by the
+// MMAs, whichever is slower: 1-SM 128x128: 64 KB / 512 cycles; 1-SM 128x256:
+// 96 KB / 1024; pair 256x256: 64 KB / 1024; pair 256x128: 48 KB / 512 per SM.
 LargeKind choose_large(int64_t M, int64_t N, int64_t K) {
   const int path = forced_path();
   if (path == 3) return LargeKind::k128;
   if (path == 4) return LargeKind::k256;
   if (path == 5) return LargeKind::kPair;
   if (path == 6) return LargeKind::kPairSplit;
-  const int64_t sms = sm_count();
+  if (path == 7) return LargeKind::kPair128;
+  (void)K;
+  const int64_t sms = sm_count(), pairs = sms / 2;
+  const double feed_us_per_kb = 1.0 / 114e3;  // us per byte per SM
+  const double mma_us_per_cycle = 1.0 / 1900.0;
+  auto stage_us = [&](double bytes, double cycles) {
+    return std::max(bytes * feed_us_per_kb, cycles * mma_us_per_cycle);
+  };
   const int64_t tm = (M + kBM - 1) / kBM;
   const int64_t t128 = tm * ((N + 127) / 128), t256 = tm * ((N + 255) / 256);
-  const int64_t tpair = pair_tiles(M, N), pairs = sms / 2, quads = sms / 4;
-  const double c128 = (double)((t128 + sms - 1) / sms) * 128.0 / 0.45;
-  const double c256 = (double)((t256 + sms - 1) / sms) * 256.0 / 0.60;
-  const double cpair = (double)((tpair + pairs - 1) / pairs) * 256.0 / 0.85;
-  // Half the K per cluster of two pairs, plus the exchange of one 128 KB
-  // partial per CTA over DSMEM, measured at ~5 us on this part: it does not
-  // pay on the shapes at hand, so automatic selection leaves it off.
-  (void)quads;
-  (void)K;
-  const double csplit = 1e30;
+  const int64_t tp256 = pair_tiles(M, N, 256), tp128 = pair_tiles(M, N, 128);
+  const double c128 = (double)((t128 + sms - 1) / sms) * stage_us(65536, 512);
+  const double c256 = (double)((t256 + sms - 1) / sms) * stage_us(98304, 1024);
+  const double cp256 = (double)((tp256 + pairs - 1) / pairs) * stage_us(65536, 1024);
+  const double cp128 = (double)((tp128 + pairs - 1) / pairs) * stage_us(49152, 512);
   double best = c128;
   LargeKind kind = LargeKind::k128;
   if (c256 < best) best = c256, kind = LargeKind::k256;
-  if (cpair <= best) best = cpair, kind = LargeKind::kPair;
-  if (csplit < best) best = csplit, kind = LargeKind::kPairSplit;
+  if (cp256 <= best) best = cp256, kind = LargeKind::kPair;
+  if (cp128 < best * 0.97) best = cp128, kind = LargeKind::kPair128;
+  // The K-split pair variant exchanges a 128 KB partial per CTA over DSMEM
+  // (measured ~5 us): it does not pay on the shapes at hand and is never
+  // chosen automatically.
   return kind;
 }
 
@@ -356,9 +366,11 @@ w8a8_status launch_scaled_mm(const int8_t *q, const float *a_scale, const void *
   if (!make_tmap_out_bf16(&tmap_y, out, (uint64_t)M, (uint64_t)N)) return W8A8_ERR_CUDA;
   switch (choose_large(M, N, K)) {
     case LargeKind::kPair:
-      return launch_gemm2sm(q, a_scale, packed_w, w_scale, bias, out, M, N, K, stream, pdl, 1);
+      return launch_gemm2sm(q, a_scale, packed_w, w_scale, bias, out, M, N, K, stream, pdl, 1, 256);
+    case LargeKind::kPair128:
+      return launch_gemm2sm(q, a_scale, packed_w, w_scale, bias, out, M, N, K, stream, pdl, 1, 128);
     case LargeKind::kPairSplit:
-      return launch_gemm2sm(q, a_scale, packed_w, w_scale, bias, out, M, N, K, stream, pdl, 2);
+      return launch_gemm2sm(q, a_scale, packed_w, w_scale, bias, out, M, N, K, stream, pdl, 2, 256);
     case LargeKind::k256:
       return run_large<256, kLargeStages256, false>(tmap, tmap_y, a, stream, pdl, 2);
     default:

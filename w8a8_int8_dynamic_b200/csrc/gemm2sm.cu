@@ -37,24 +37,28 @@
 namespace w8a8 {
 namespace {
 
-constexpr int kPairBN = 256;                      // tile N (both CTAs)
 constexpr int kStageK = 2;                        // k-blocks per stage
-constexpr int kHalfStage = kStageK * kTileBytes;  // 32 KB: one operand of one stage
-constexpr int kPartialBytes = 128 * kPairBN * 4;  // one CTA's int32 partial: 128 KB
+constexpr int kHalfStage = kStageK * kTileBytes;  // 32 KB: the q part of one stage
+constexpr int kPartialBytes = 128 * 256 * 4;      // one CTA's int32 partial (BN = 256): 128 KB
 
-template <int STAGES>
+// BN = tile N of the pair (256 or 128); each CTA holds BN/2 weight rows.
+template <int BN, int STAGES>
 struct PairSmem {
+  static constexpr int kBRows = BN / 2;                 // weight rows per CTA
+  static constexpr int kBTile = kBRows * kBK;           // weight bytes per k-block per CTA
+  static constexpr int kBStage = kStageK * kBTile;
   static constexpr int kA = 0;                          // STAGES x 32 KB q tiles
-  static constexpr int kB = STAGES * kHalfStage;        // STAGES x 32 KB weight tiles
-  static constexpr int kEpiPerWarp = kPairBN * 4 + kPairBN * 2;
-  static constexpr int kEpi = kB + STAGES * kHalfStage;
+  static constexpr int kB = STAGES * kHalfStage;        // STAGES x kBStage weight tiles
+  static constexpr int kEpiPerWarp = BN * 4 + BN * 2;
+  static constexpr int kEpi = kB + STAGES * kBStage;
   static constexpr int kOut = kEpi + 4 * kEpiPerWarp + 1024 - (kEpi + 4 * kEpiPerWarp) % 1024;
   // full[S], empty[S], tfull[2], tempty[2], done, ready, recv
   static constexpr int kBars = kOut + 4 * kEpiStagePerWarp;
   static constexpr int kMisc = kBars + (2 * STAGES + 7) * 8;
   static constexpr int kUsed = kMisc + 16;
   static constexpr int kAlloc = kUsed + 1024;
-  static_assert(2 * STAGES * kHalfStage >= kPartialBytes, "partial must fit the stage buffers");
+  static_assert(BN != 256 || STAGES * (kHalfStage + kBStage) >= kPartialBytes,
+                "partial must fit the stage buffers");
 };
 
 // int32 partial layout in shared memory: element (row r, column j) at
@@ -65,14 +69,16 @@ struct PartialIndex {
   __device__ int operator()(int r, int j) const { return partial_index(r, j); }
 };
 
-template <int STAGES, int SPLIT>
+template <int BN, int STAGES, int SPLIT>
 __global__ void __launch_bounds__(kThreads, 1)
     gemm2sm_kernel(const __grid_constant__ CUtensorMap tmap_q,
                    const __grid_constant__ CUtensorMap tmap_w,
                    const __grid_constant__ CUtensorMap tmap_y, const GemmArgs args) {
-  using L = PairSmem<STAGES>;
-  constexpr uint32_t kTmemCols = 2 * kPairBN;
-  constexpr uint32_t kIdesc = idesc_i8(256, kPairBN);
+  using L = PairSmem<BN, STAGES>;
+  constexpr int kPairBN = BN;
+  constexpr uint32_t kTmemCols = 2 * BN;
+  constexpr uint32_t kIdesc = idesc_i8(256, BN);
+  static_assert(SPLIT == 1 || BN == 256, "the K split is built for 256-wide tiles");
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>(
@@ -147,9 +153,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int nk = min(kStageK, num_kb - kb0);
         const uint32_t bar = full0 + s * 8;
         if (weights) {
-          // two contiguous packed tiles (k-blocks kb0, kb0+1) of this CTA's slab
-          const int wslab = nb * 2 + (int)rank;
-          tma_load_2d_pair(sB + s * kHalfStage, &tmap_w, 0, (wslab * num_kb + kb0) * 128, bar);
+          if (BN == 256) {
+            // two contiguous packed tiles (k-blocks kb0, kb0+1) of this CTA's slab
+            const int wslab = nb * 2 + (int)rank;
+            tma_load_2d_pair(sB + s * L::kBStage, &tmap_w, 0, (wslab * num_kb + kb0) * 128, bar);
+          } else {
+            // this CTA's 64-row half of each of the two tiles of slab nb
+            for (int h = 0; h < nk; ++h)
+              tma_load_2d_pair(sB + s * L::kBStage + h * L::kBTile, &tmap_w, 0,
+                               (nb * num_kb + kb0 + h) * 128 + (int)rank * 64, bar);
+          }
         }
         if (acts) {
           const int row0 = mb * 256 + (int)rank * 128;
@@ -160,7 +173,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       };
       auto stage_bytes = [&](uint32_t it) {
         const int kb0 = (st_begin + (int)(it % nst)) * kStageK;
-        return (uint32_t)(kHalfStage + min(kStageK, num_kb - kb0) * kTileBytes);
+        const int nk = min(kStageK, num_kb - kb0);
+        // the 256-wide weight box always moves two tiles (zero-filled past the end)
+        return (uint32_t)(nk * kTileBytes + (BN == 256 ? L::kBStage : nk * L::kBTile));
       };
       uint32_t last_par[STAGES];
       bool ok = true;
@@ -216,7 +231,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int nk = min(kStageK, num_kb - (st_begin + j) * kStageK);
           for (int h = 0; h < nk; ++h) {
             const uint64_t a_desc = sw128_kmajor_desc(sA + s * kHalfStage + h * kTileBytes);
-            const uint64_t b_desc = sw128_kmajor_desc(sB + s * kHalfStage + h * kTileBytes);
+            const uint64_t b_desc = sw128_kmajor_desc(sB + s * L::kBStage + h * L::kBTile);
 #pragma unroll
             for (int k = 0; k < kBK / 32; ++k)
               mma_i8_pair(d_tmem, a_desc + 2 * k, b_desc + 2 * k, kIdesc, (j | h | k) != 0);
@@ -316,20 +331,19 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-constexpr int kPairStages = 3;
-bool g_pair_attr_done[64][2];
+bool g_pair_attr_done[64][3];
 
-template <int SPLIT>
+template <int BN, int STAGES, int SPLIT>
 w8a8_status run_pair(const CUtensorMap &tq, const CUtensorMap &tw, const CUtensorMap &ty,
-                     const GemmArgs &a, cudaStream_t stream, bool pdl) {
-  using L = PairSmem<kPairStages>;
-  auto k = gemm2sm_kernel<kPairStages, SPLIT>;
+                     const GemmArgs &a, cudaStream_t stream, bool pdl, int slot_id) {
+  using L = PairSmem<BN, STAGES>;
+  auto k = gemm2sm_kernel<BN, STAGES, SPLIT>;
   const int d = current_device();
-  if (d < 0 || d >= 64 || !g_pair_attr_done[d][SPLIT - 1]) {
+  if (d < 0 || d >= 64 || !g_pair_attr_done[d][slot_id]) {
     if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kAlloc) !=
         cudaSuccess)
       return W8A8_ERR_CUDA;
-    if (d >= 0 && d < 64) g_pair_attr_done[d][SPLIT - 1] = true;
+    if (d >= 0 && d < 64) g_pair_attr_done[d][slot_id] = true;
   }
   const int tiles = a.tiles_m * a.tiles_n;
   const int cta_per_cluster = 2 * SPLIT;
@@ -356,18 +370,19 @@ w8a8_status run_pair(const CUtensorMap &tq, const CUtensorMap &tw, const CUtenso
 
 }  // namespace
 
-// Number of 256 x 256 tiles the pair kernel would process.
-int64_t pair_tiles(int64_t M, int64_t N) { return ((M + 255) / 256) * ((N + 255) / 256); }
+// Number of 256 x bn tiles the pair kernel would process.
+int64_t pair_tiles(int64_t M, int64_t N, int bn) { return ((M + 255) / 256) * ((N + bn - 1) / bn); }
 
 w8a8_status launch_gemm2sm(const int8_t *q, const float *a_scale, const void *packed_w,
                            const float *w_scale, const void *bias, void *y, int64_t M, int64_t N,
-                           int64_t K, cudaStream_t stream, bool pdl, int split) {
+                           int64_t K, cudaStream_t stream, bool pdl, int split, int bn) {
   CUtensorMap tq, tw, ty;
   if (!make_tmap_u8_2d(&tq, q, (uint64_t)M, (uint64_t)K, (uint64_t)K, kBM, kBK))
     return W8A8_ERR_CUDA;
   if (!make_tmap_out_bf16(&ty, y, (uint64_t)M, (uint64_t)N)) return W8A8_ERR_CUDA;
   const uint64_t wrows = (uint64_t)(packed_rows(N) * packed_cols(K) / 128);
-  if (!make_tmap_u8_2d_plain(&tw, packed_w, wrows, 128, 128, 256, 128)) return W8A8_ERR_CUDA;
+  if (!make_tmap_u8_2d_plain(&tw, packed_w, wrows, 128, 128, bn == 128 ? 64 : 256, 128))
+    return W8A8_ERR_CUDA;
   GemmArgs a;
   a.packed_w = static_cast<const uint8_t *>(packed_w);
   a.a_scale = a_scale;
@@ -378,13 +393,14 @@ w8a8_status launch_gemm2sm(const int8_t *q, const float *a_scale, const void *pa
   a.N = (int)N;
   a.num_kb = (int)(packed_cols(K) / 128);
   a.tiles_m = (int)((M + 255) / 256);
-  a.tiles_n = (int)((N + 255) / 256);
+  a.tiles_n = (int)((N + bn - 1) / bn);
   a.status = status_word();
   if (!a.status) return W8A8_ERR_CUDA;
+  if (bn == 128) return run_pair<128, 4, 1>(tq, tw, ty, a, stream, pdl, 2);
   // the split needs at least one stage per half
   if (split == 2 && (a.num_kb + kStageK - 1) / kStageK >= 2)
-    return run_pair<2>(tq, tw, ty, a, stream, pdl);
-  return run_pair<1>(tq, tw, ty, a, stream, pdl);
+    return run_pair<256, 3, 2>(tq, tw, ty, a, stream, pdl, 1);
+  return run_pair<256, 3, 1>(tq, tw, ty, a, stream, pdl, 0);
 }
 
 }  // namespace w8a8

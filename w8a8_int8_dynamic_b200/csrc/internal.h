@@ -59,8 +59,8 @@ w8a8_status launch_scaled_mm(const int8_t *q, const float *a_scale, const void *
 // 2-SM (CTA pair) GEMM with the bf16 epilogue (gemm2sm.cu).
 w8a8_status launch_gemm2sm(const int8_t *q, const float *a_scale, const void *packed_w,
                            const float *w_scale, const void *bias, void *y, int64_t M, int64_t N,
-                           int64_t K, cudaStream_t stream, bool pdl, int split);
-int64_t pair_tiles(int64_t M, int64_t N);
+                           int64_t K, cudaStream_t stream, bool pdl, int split, int bn);
+int64_t pair_tiles(int64_t M, int64_t N, int bn);
 // Small-M weight-streaming kernel (decode.cu).
 int64_t decode_workspace_bytes(int64_t N, int64_t K);
 bool use_decode_path(int64_t M);
