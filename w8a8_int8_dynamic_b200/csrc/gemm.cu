@@ -310,17 +310,29 @@ LargeKind choose_large(int64_t M, int64_t N, int64_t K) {
   (void)K;
   const int64_t sms = sm_count(), pairs = sms / 2;
   const double feed_us_per_kb = 1.0 / 114e3;  // us per byte per SM
+  const double l2_us_per_byte = 1.0 / 10.5e6;  // us per byte, whole chip
   const double mma_us_per_cycle = 1.0 / 1900.0;
-  auto stage_us = [&](double bytes, double cycles) {
-    return std::max(bytes * feed_us_per_kb, cycles * mma_us_per_cycle);
+  // one stage of every busy SM: per-SM feed, aggregate L2 and MMA bounds
+  auto stage_us_on = [&](double bytes, double cycles, int64_t busy_sms) {
+    return std::max({bytes * feed_us_per_kb, bytes * (double)busy_sms * l2_us_per_byte,
+                     cycles * mma_us_per_cycle});
   };
   const int64_t tm = (M + kBM - 1) / kBM;
   const int64_t t128 = tm * ((N + 127) / 128), t256 = tm * ((N + 255) / 256);
   const int64_t tp256 = pair_tiles(M, N, 256), tp128 = pair_tiles(M, N, 128);
-  const double c128 = (double)((t128 + sms - 1) / sms) * stage_us(65536, 512);
-  const double c256 = (double)((t256 + sms - 1) / sms) * stage_us(98304, 1024);
-  const double cp256 = (double)((tp256 + pairs - 1) / pairs) * stage_us(65536, 1024);
-  const double cp128 = (double)((tp128 + pairs - 1) / pairs) * stage_us(49152, 512);
+  auto cost = [&](int64_t tiles, int64_t slots, int ctas_per_tile, double bytes, double cycles) {
+    const int64_t waves = (tiles + slots - 1) / slots;
+    const int64_t busy = std::min(tiles, slots) * ctas_per_tile;
+    return (double)waves * stage_us_on(bytes, cycles, busy);
+  };
+  const double c128 = cost(t128, sms, 1, 65536, 512);
+  const double c256 = cost(t256, sms, 1, 98304, 1024);
+  const double cp256 = cost(tp256, pairs, 2, 65536, 1024);
+  const double cp128 = cost(tp128, pairs, 2, 49152, 512);
+  // Few 256-wide pair tiles (half the GPU or less) but 128x128 tiles that fit
+  // one wave: with cold operands, twice as many SMs pulling from DRAM wins
+  // (measured on 512 x 4096 x 4096: 16.6 us vs 19.1 us).
+  if (tp256 * 2 <= pairs && t128 <= sms) return LargeKind::k128;
   double best = c128;
   LargeKind kind = LargeKind::k128;
   if (c256 < best) best = c256, kind = LargeKind::k256;

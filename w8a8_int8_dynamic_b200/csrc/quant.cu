@@ -9,8 +9,8 @@
 //             q = clamp(rint_half_even(x / s), -127, 127);  amax == 0 -> s = 0, q = 0.
 //
 // One CTA per row.  The row is read once with 128-bit streaming loads and
-// held in registers (up to 4 16-byte chunks per thread, rows of up to 32768
-// elements; longer rows take a two-pass kernel); the row
+// held in registers (1, 2 or 4 16-byte chunks per thread for rows of up to
+// 8192 / 16384 / 32768 elements; longer rows take a two-pass kernel); the row
 // maximum is a packed 16-bit integer max on the bf16 magnitudes (|x| order
 // equals the order of the 15 low bits for finite bf16), reduced with warp
 // shuffles and one shared-memory step; each thread then writes its codes as
@@ -189,16 +189,26 @@ __global__ void __launch_bounds__(1024) quant_rows_two_pass_kernel(
 
 w8a8_status launch_quant(const void *x, int64_t M, int64_t K, int64_t ldx, int8_t *q,
                          float *a_scale, cudaStream_t stream) {
+  // One CTA per row with as many threads as the row has 16-byte chunks (up
+  // to 1024): the row is read in one wave of loads and each warp has little
+  // serial work, which is what this latency-bound kernel needs.
   const int64_t nchunks = K / 8;
+  const uint16_t *xp = static_cast<const uint16_t *>(x);
   auto threads_for = [&](int per) {
     int64_t t = (nchunks + per - 1) / per;
-    t = round_up(t < 32 ? 32 : t, 32);
-    return t;
+    return round_up(t < 32 ? 32 : t, 32);
   };
-  const uint16_t *xp = static_cast<const uint16_t *>(x);
-  const int64_t t = threads_for(4);
-  if (t <= 1024) {
-    quant_rows_kernel<4><<<(unsigned)M, (unsigned)t, 0, stream>>>(xp, ldx, (int)K, q, a_scale);
+  // at most 512 threads per row-CTA (measured: 768-thread CTAs fit only two
+  // per SM and run the 12288-wide rows slower than 384-thread ones)
+  if (threads_for(1) <= 512) {
+    quant_rows_kernel<1><<<(unsigned)M, (unsigned)threads_for(1), 0, stream>>>(xp, ldx, (int)K, q,
+                                                                                 a_scale);
+  } else if (threads_for(2) <= 512) {
+    quant_rows_kernel<2><<<(unsigned)M, (unsigned)threads_for(2), 0, stream>>>(xp, ldx, (int)K, q,
+                                                                                 a_scale);
+  } else if (threads_for(4) <= 1024) {
+    quant_rows_kernel<4><<<(unsigned)M, (unsigned)threads_for(4), 0, stream>>>(xp, ldx, (int)K, q,
+                                                                                 a_scale);
   } else {
     quant_rows_two_pass_kernel<<<(unsigned)M, 1024, 0, stream>>>(xp, ldx, (int)K, q, a_scale);
   }
