@@ -41,27 +41,32 @@ namespace {
 // ============================================================================
 // Large-M persistent GEMM
 // ============================================================================
-template <int BN, int STAGES>
+// KPS = k-blocks per pipeline stage.  With 128-wide tiles the KPS weight
+// tiles of a stage are contiguous in the packed image (one bulk copy); fewer,
+// larger stages halve the per-stage barrier round trips that bound the feed.
+template <int BN, int STAGES, int KPS>
 struct LargeSmem {
+  static constexpr int kAStage = KPS * kTileBytes;
+  static constexpr int kBStage = KPS * BN * kBK;
   static constexpr int kA = 0;
-  static constexpr int kB = STAGES * kTileBytes;
+  static constexpr int kB = STAGES * kAStage;
   // per epilogue warp: the tile's BN w_scale (fp32) and BN bias (bf16) values
   static constexpr int kEpiPerWarp = BN * 4 + BN * 2;
-  static constexpr int kEpi = kB + STAGES * BN * kBK;
+  static constexpr int kEpi = kB + STAGES * kBStage;
   static constexpr int kOut = kEpi + 4 * kEpiPerWarp + 1024 - (kEpi + 4 * kEpiPerWarp) % 1024;
   static constexpr int kBars = kOut + 4 * kEpiStagePerWarp;  // full[S], empty[S], tfull[2], tempty[2], done
   static constexpr int kMisc = kBars + (2 * STAGES + 5) * 8;
   static constexpr int kUsed = kMisc + 16;
   static constexpr int kAlloc = kUsed + 1024;  // slack for 1024-byte alignment
+  static_assert(KPS == 1 || BN == 128, "multi-k-block stages need contiguous weight tiles");
 };
 
-template <int BN, int STAGES, bool OUT_I32>
+template <int BN, int STAGES, int KPS, bool OUT_I32>
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_kernel(const __grid_constant__ CUtensorMap tmap_q,
                 const __grid_constant__ CUtensorMap tmap_y, const GemmArgs args) {
-  using L = LargeSmem<BN, STAGES>;
+  using L = LargeSmem<BN, STAGES, KPS>;
   constexpr uint32_t kTmemCols = 2 * BN;  // two accumulator buffers
-  constexpr uint32_t kStageBytes = kTileBytes + BN * kBK;
   constexpr uint32_t kIdesc = idesc_i8(kBM, BN);
 
   extern __shared__ uint8_t smem_raw[];
@@ -100,8 +105,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   const int num_tiles = args.tiles_m * args.tiles_n;
   const int num_kb = args.num_kb;
+  const int nsk = (num_kb + KPS - 1) / KPS;  // stages per tile
   const int my_tiles = blockIdx.x < num_tiles ? (num_tiles - 1 - blockIdx.x) / gridDim.x + 1 : 0;
-  const uint32_t my_iters = (uint32_t)my_tiles * num_kb;
+  const uint32_t my_iters = (uint32_t)my_tiles * nsk;
 
   // Roles: lane 0 of warps 0 and 1 runs the producer / MMA loop alone; the
   // rest of those warps wait at __syncwarp so every warp reaches the block
@@ -109,42 +115,47 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 0) {
     if (lane == 0) {
       // ---------------- producer ----------------
+      auto stage_nk = [&](uint32_t it) { return min(KPS, num_kb - (int)(it % nsk) * KPS); };
+      auto weights = [&](uint32_t it, uint32_t s) {
+        const int tile = blockIdx.x + (int)(it / nsk) * gridDim.x;
+        const int nb = tile / args.tiles_m, kb0 = (int)(it % nsk) * KPS;
+        const int nk = stage_nk(it);
+#pragma unroll
+        for (int h = 0; h < BN / 128; ++h)
+          bulk_load(sB + s * L::kBStage + h * kTileBytes,
+                    args.packed_w + (((size_t)nb * (BN / 128) + h) * num_kb + kb0) * kTileBytes,
+                    (uint32_t)(nk * kTileBytes), &full[s]);
+      };
+      auto acts = [&](uint32_t it, uint32_t s) {
+        const int tile = blockIdx.x + (int)(it / nsk) * gridDim.x;
+        const int kb0 = (int)(it % nsk) * KPS;
+        const int nk = stage_nk(it);
+        for (int i = 0; i < nk; ++i)
+          tma_load_2d(sA + s * L::kAStage + i * kTileBytes, &tmap_q, (kb0 + i) * kBK,
+                      (tile % args.tiles_m) * kBM, &full[s]);
+      };
+      auto bytes = [&](uint32_t it) { return (uint32_t)(stage_nk(it) * (kTileBytes + BN * kBK)); };
       uint32_t last_par[STAGES];
       bool ok = true;
-      auto b_src = [&](uint32_t it, int h) {
-        const int tile = blockIdx.x + (int)(it / num_kb) * gridDim.x;
-        const int nb = tile / args.tiles_m, kb = (int)(it % num_kb);
-        return args.packed_w + (((size_t)nb * (BN / 128) + h) * num_kb + kb) * kTileBytes;
-      };
       // The weight tiles of the first stages do not depend on the preceding
       // kernel of the stream: issue them before waiting for it.
       const uint32_t pre = my_iters < (uint32_t)STAGES ? my_iters : (uint32_t)STAGES;
       for (uint32_t it = 0; it < pre; ++it) {
-        mbar_arrive_expect_tx(&full[it], kStageBytes);
-#pragma unroll
-        for (int h = 0; h < BN / 128; ++h)
-          bulk_load(sB + it * (BN * kBK) + h * kTileBytes, b_src(it, h), kTileBytes, &full[it]);
+        mbar_arrive_expect_tx(&full[it], bytes(it));
+        weights(it, it);
         last_par[it] = 0;
       }
       griddep_wait();
-      for (uint32_t it = 0; it < pre; ++it) {
-        const int tile = blockIdx.x + (int)(it / num_kb) * gridDim.x;
-        tma_load_2d(sA + it * kTileBytes, &tmap_q, (int)(it % num_kb) * kBK,
-                    (tile % args.tiles_m) * kBM, &full[it]);
-      }
+      for (uint32_t it = 0; it < pre; ++it) acts(it, it);
       for (uint32_t it = pre; it < my_iters; ++it) {
         const uint32_t s = it % STAGES, ph = (it / STAGES) & 1;
         if (!mbar_wait(&empty[s], ph ^ 1, abort_flag, args.status)) {
           ok = false;
           break;
         }
-        const int tile = blockIdx.x + (int)(it / num_kb) * gridDim.x;
-        mbar_arrive_expect_tx(&full[s], kStageBytes);
-        tma_load_2d(sA + s * kTileBytes, &tmap_q, (int)(it % num_kb) * kBK,
-                    (tile % args.tiles_m) * kBM, &full[s]);
-#pragma unroll
-        for (int h = 0; h < BN / 128; ++h)
-          bulk_load(sB + s * (BN * kBK) + h * kTileBytes, b_src(it, h), kTileBytes, &full[s]);
+        mbar_arrive_expect_tx(&full[s], bytes(it));
+        acts(it, s);
+        weights(it, s);
         last_par[s] = ph;
       }
       if (!ok) {
@@ -169,18 +180,21 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + b * BN;
-        for (int kb = 0; kb < num_kb; ++kb, ++it) {
+        for (int j = 0; j < nsk; ++j, ++it) {
           const uint32_t s = it % STAGES, ph = (it / STAGES) & 1;
           if (!mbar_wait(&full[s], ph, abort_flag, args.status)) {
             ok = false;
             break;
           }
           tc_fence_after();
-          const uint64_t a_desc = sw128_kmajor_desc(sA + s * kTileBytes);
-          const uint64_t b_desc = sw128_kmajor_desc(sB + s * (BN * kBK));
+          const int nk = min(KPS, num_kb - j * KPS);
+          for (int i = 0; i < nk; ++i) {
+            const uint64_t a_desc = sw128_kmajor_desc(sA + s * L::kAStage + i * kTileBytes);
+            const uint64_t b_desc = sw128_kmajor_desc(sB + s * L::kBStage + i * BN * kBK);
 #pragma unroll
-          for (int k = 0; k < kBK / 32; ++k)
-            mma_i8(d_tmem, a_desc + 2 * k, b_desc + 2 * k, kIdesc, (kb | k) != 0);
+            for (int k = 0; k < kBK / 32; ++k)
+              mma_i8(d_tmem, a_desc + 2 * k, b_desc + 2 * k, kIdesc, (j | i | k) != 0);
+          }
           mma_commit(&empty[s]);  // frees the stage when these MMAs finish
         }
         if (ok) mma_commit(&tfull[b]);
@@ -243,8 +257,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 // ============================================================================
 // host side
 // ============================================================================
-constexpr int kLargeStages128 = 6;
-constexpr int kLargeStages256 = 4;
+constexpr int kLargeStages128 = 3;  // 3 x (2 k-blocks): 64 KB stages
+constexpr int kKps128 = 2;
+constexpr int kLargeStages256 = 4;  // 4 x (1 k-block): 48 KB stages
 
 bool g_attr_done[64][8];
 
@@ -276,8 +291,9 @@ cudaError_t launch_ex(Kernel k, int grid, int smem, cudaStream_t stream, bool pd
 template <int BN, int STAGES, bool OUT_I32>
 w8a8_status run_large(const CUtensorMap &tmap, const CUtensorMap &tmap_y, GemmArgs args,
                       cudaStream_t stream, bool pdl, int slot) {
-  using L = LargeSmem<BN, STAGES>;
-  auto k = gemm_kernel<BN, STAGES, OUT_I32>;
+  constexpr int KPS = BN == 128 ? kKps128 : 1;
+  using L = LargeSmem<BN, STAGES, KPS>;
+  auto k = gemm_kernel<BN, STAGES, KPS, OUT_I32>;
   cudaError_t e = set_smem_attr(k, L::kAlloc, slot);
   if (e != cudaSuccess) return W8A8_ERR_CUDA;
   args.tiles_n = (int)((args.N + BN - 1) / BN);
