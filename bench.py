@@ -314,7 +314,7 @@ def run_ours(args, rank, world, device):
     gemm_tops = ops / base["t_gemm"] / 1e12
     roofline = {"bound": "tensor", "achieved": round(gemm_tops, 2), "peak": round(int8_peak, 1),
                 "unit": "TOPS", "frac": round(gemm_tops / int8_peak, 4), "traffic": None,
-                "kernel": "gemm_kernel (persistent tcgen05 kind::i8 + epilogue)",
+                "kernel": w8.gemm_kernel_name(wl.M, wl.N, wl.K),
                 "peak_note": f"int8 = 2 x {peaks['source']} bf16 burst {peaks['bf16_tflops']} TFLOP/s",
                 "frac_vs_spec_4500": round(gemm_tops / SPEC_INT8_TOPS, 4),
                 "gemm_us": round(base["t_gemm"] * 1e6, 3),
@@ -412,6 +412,7 @@ def sweep(w8, args, device, stream, peaks, int8_peak):
             "quant_frac_hbm": round(quant_bytes / r["t_quant"] / 1e9 / peaks["hbm_gbs"], 4),
             "step_frac_roofline": round(t_roof_fused / r["t_step"], 4),
             "l2_sets": r["nsets"],
+            "kernel": w8.gemm_kernel_name(wl.M, wl.N, wl.K),
         }
         del ls, loop
         torch.cuda.empty_cache()

@@ -178,6 +178,10 @@ w8a8_status w8a8_linear_noalloc(const void *x, int64_t ldx, const void *packed_w
  * Process-wide; not synchronised with concurrent calls. */
 w8a8_status w8a8_set_path(int path);
 
+/* Name of the GEMM kernel w8a8_scaled_mm / w8a8_linear would run for this
+ * shape under the current path setting (static string, for reports). */
+const char *w8a8_gemm_kernel_name(int64_t M, int64_t N, int64_t K);
+
 /* ---- harness kernel: GELU (tanh form), bf16 -> bf16 ------------------------
  * Not on the pages; it joins the up and down projections of the DiT MLP
  * workload.  y = 0.5 x (1 + tanh(sqrt(2/pi)(x + 0.044715 x^3))) in fp32,

@@ -59,6 +59,7 @@ _SIGNATURES = {
     "w8a8_linear_noalloc_max_bytes": ([], _SZ),
     "w8a8_linear_noalloc": ([_P, _I64, _P, _P, _P, _P, _I64, _I64, _I64, _P], ctypes.c_int),
     "w8a8_set_path": ([ctypes.c_int], ctypes.c_int),
+    "w8a8_gemm_kernel_name": ([_I64, _I64, _I64], ctypes.c_char_p),
     "w8a8_gelu_tanh": ([_P, _P, _I64, _P], ctypes.c_int),
     "w8a8_poll_status": ([_P], ctypes.c_int),
     "w8a8_selftest_wait_timeout": ([_I64, _P], ctypes.c_int),
@@ -246,6 +247,10 @@ def gelu_tanh(x: torch.Tensor, out: Optional[torch.Tensor] = None, stream=None) 
         out = torch.empty_like(x)
     _check(lib().w8a8_gelu_tanh(_ptr(x), _ptr(out), x.numel(), _stream(stream)), "w8a8_gelu_tanh")
     return out
+
+
+def gemm_kernel_name(M: int, N: int, K: int) -> str:
+    return lib().w8a8_gemm_kernel_name(M, N, K).decode()
 
 
 def set_path(path: int):

@@ -447,6 +447,18 @@ w8a8_status w8a8_scaled_mm(const int8_t *q, const float *a_scale, const void *pa
   return launch_scaled_mm(q, a_scale, packed_w, w_scale, bias, y, false, M, N, K, s, false);
 }
 
+const char *w8a8_gemm_kernel_name(int64_t M, int64_t N, int64_t K) {
+  if (M < 1 || N < 1 || K < 1) return "invalid";
+  if (use_decode_path(M)) return "decode_kernel (swap-AB stream-K, needs a workspace)";
+  switch (choose_large(M, N, K)) {
+    case LargeKind::kPair: return "gemm2sm_kernel<256, 3, 1> (2-SM pair, 256x256 tiles)";
+    case LargeKind::kPair128: return "gemm2sm_kernel<128, 4, 1> (2-SM pair, 256x128 tiles)";
+    case LargeKind::kPairSplit: return "gemm2sm_kernel<256, 3, 2> (2-SM pairs, K split)";
+    case LargeKind::k256: return "gemm_kernel<256, 4, 1> (1-SM, 128x256 tiles)";
+    default: return "gemm_kernel<128, 3, 2> (1-SM, 128x128 tiles, 2 k-blocks per stage)";
+  }
+}
+
 w8a8_status w8a8_scaled_mm_i32(const int8_t *q, const void *packed_w, int32_t *acc, int64_t M,
                                int64_t N, int64_t K, w8a8_stream_t stream) {
   w8a8_status st = check_gemm_args(q, packed_w, acc, M, N, K);
