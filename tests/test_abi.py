@@ -91,7 +91,8 @@ def test_gemm_rejects_bad_arguments(L):
     assert g(FAKE, 16, FAKE, FAKE, None, FAKE, 4, 8, 16, None, 0, None) == 1       # no workspace
     assert g(FAKE, 16, FAKE, FAKE, None, FAKE, 4, 8, 16, FAKE, 1, None) == 6       # too small
     assert g(FAKE, 8, FAKE, FAKE, None, FAKE, 4, 8, 16, FAKE, 1 << 30, None) == 1  # ldx < K
-    assert L.w8a8_set_path(7) == 1
+    assert L.w8a8_set_path(8) == 1
+    assert L.w8a8_set_path(7) == 0
     assert L.w8a8_set_path(0) == 0
 
 
