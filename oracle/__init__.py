@@ -40,6 +40,9 @@ def lib():
         L.w8a8o_bf16_to_f32.argtypes = [ctypes.c_uint16]
         L.w8a8o_bf16_to_f32.restype = ctypes.c_float
         L.w8a8o_num_threads.restype = ctypes.c_int
+        L.w8a8o_quant_weight.argtypes = [P, I64, I64, P, P]
+        L.w8a8o_quant_act_static.argtypes = [P, I64, I64, I64, ctypes.c_float, P, P]
+        L.w8a8o_unpack_int32.argtypes = [P, I64, I64, P]
         _lib = L
     return _lib
 
@@ -159,3 +162,33 @@ def f64_to_bf16(v: float) -> int:
 
 def bf16_to_f32(h: int) -> float:
     return float(lib().w8a8o_bf16_to_f32(h))
+
+
+def quant_weight(w_bf16: np.ndarray):
+    """bf16 bits [N, K] -> (int8 [N, K], fp32 per-output-channel scale [N])."""
+    w = np.ascontiguousarray(w_bf16, dtype=np.uint16)
+    N, K = w.shape
+    q = np.empty((N, K), np.int8)
+    s = np.empty((N,), np.float32)
+    _check(lib().w8a8o_quant_weight(_p(w), N, K, _p(q), _p(s)), "quant_weight")
+    return q, s
+
+
+def quant_act_static(x_bf16: np.ndarray, scale: float):
+    """Per-tensor calibrated scale -> (q int8 [M, K], a_scale fp32 [M])."""
+    x = np.ascontiguousarray(x_bf16, dtype=np.uint16)
+    M, K = x.shape
+    q = np.empty((M, K), np.int8)
+    s = np.empty((M,), np.float32)
+    _check(lib().w8a8o_quant_act_static(_p(x), M, K, K, float(np.float32(scale)), _p(q), _p(s)),
+           "quant_act_static")
+    return q, s
+
+
+def unpack_int32(packed: np.ndarray, K: int) -> np.ndarray:
+    """compressed-tensors int32 words [N, K/4] -> int8 [N, K]."""
+    p = np.ascontiguousarray(packed, dtype=np.int32)
+    N = p.shape[0]
+    w = np.empty((N, K), np.int8)
+    _check(lib().w8a8o_unpack_int32(_p(p), N, K, _p(w)), "unpack_int32")
+    return w

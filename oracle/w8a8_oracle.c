@@ -278,6 +278,64 @@ int w8a8o_gelu_tanh(const uint16_t *x, int64_t n, uint16_t *y) {
   return ORACLE_OK;
 }
 
+/* ---- online weight quantisation ------------------------------------------
+ * "Online Quantization", Overview: quantised weights and scales are computed
+ * while the model loads, from bf16 weights.  "Issue 5 probe ...", Round one:
+ * the weights are per-output-channel symmetric.  So each output channel (a row
+ * of W[N, K]) follows the rule of the activation rows: scale = amax / 127,
+ * code = clamp(rne(w / scale), -127, 127), a zero row gets scale 0.
+ * w: bf16 [N, K]; q: int8 [N, K]; w_scale: fp32 [N]. */
+int w8a8o_quant_weight(const uint16_t *w, int64_t N, int64_t K, int8_t *q, float *w_scale) {
+  return w8a8o_quant_act(w, N, K, K, q, w_scale);
+}
+
+/* ---- static (calibrated) per-tensor activation scale ------------------------
+ * "Online Quantization", Parameters: activation_scheme "dynamic" selects run-
+ * time activation scaling; the other scheme keeps one calibrated fp32 scale
+ * for the whole tensor.  code = clamp(rne(x / scale), -127, 127); values
+ * beyond the calibrated range saturate.  A scale that is not > 0 (0, negative,
+ * NaN) gives codes 0 (reading: no usable scale).  a_scale_out[m] = scale (or
+ * 0) so the scaled GEMM applies it per row unchanged. */
+int w8a8o_quant_act_static(const uint16_t *x, int64_t M, int64_t K, int64_t ldx, float scale,
+                           int8_t *q, float *a_scale_out) {
+  if (!x || !q || M < 0 || K < 0 || ldx < K) return ORACLE_EINVAL;
+  const int usable = scale > 0.0f; /* false for NaN too */
+  int64_t m;
+#pragma omp parallel for schedule(static)
+  for (m = 0; m < M; ++m) {
+    for (int64_t k = 0; k < K; ++k) {
+      if (!usable) {
+        q[m * K + k] = 0;
+        continue;
+      }
+      float v = bf16_to_f32(x[m * ldx + k]) / scale;
+      float r = nearbyintf(v);
+      if (r > 127.0f) r = 127.0f;
+      if (r < -127.0f) r = -127.0f;
+      q[m * K + k] = (int8_t)r;
+    }
+    if (a_scale_out) a_scale_out[m] = usable ? scale : 0.0f;
+  }
+  return ORACLE_OK;
+}
+
+/* ---- compressed-tensors int32 weight storage -----------------------------
+ * "Issue 5 probe ...", Artifact: weights stored with pack_to_int32, "uint8
+ * biased by 128, 4 per int32".  Reading (the page gives no bit order): the
+ * four consecutive K elements k = 4j .. 4j+3 of a row share int32 word j,
+ * element 4j+i in bits [8i, 8i+8) as the unsigned byte (w + 128).
+ * packed: int32 [N, K/4]; w: int8 [N, K]. */
+int w8a8o_unpack_int32(const int32_t *packed, int64_t N, int64_t K, int8_t *w) {
+  if (!packed || !w || N < 0 || K < 0 || K % 4 != 0) return ORACLE_EINVAL;
+  for (int64_t n = 0; n < N; ++n)
+    for (int64_t k = 0; k < K; ++k) {
+      uint32_t word = (uint32_t)packed[n * (K / 4) + k / 4];
+      uint32_t byte = (word >> (8 * (k % 4))) & 0xFFu;
+      w[n * K + k] = (int8_t)((int)byte - 128);
+    }
+  return ORACLE_OK;
+}
+
 int w8a8o_num_threads(void) {
 #ifdef _OPENMP
   extern int omp_get_max_threads(void);
