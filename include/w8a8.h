@@ -78,6 +78,22 @@ int w8a8_abi_version(void);
 w8a8_status w8a8_quant_act(const void *x, int64_t M, int64_t K, int64_t ldx,
                            int8_t *q, float *a_scale, w8a8_stream_t stream);
 
+/* Static (calibrated) activation scale, the other activation scheme of
+ * "Online Quantization", Parameters: one fp32 scale for the whole tensor,
+ * computed offline.  code = clamp(rint_half_even(x / scale), -127, 127)
+ * (values outside the calibrated range saturate); a scale that is not > 0
+ * (zero, negative, NaN) gives all codes 0 and a_scale 0.
+ *   x       device, bf16 [M, K], row stride ldx >= K elements (ldx % 8 == 0)
+ *   scale   device, one fp32 (4-byte aligned); read by the kernel, so a new
+ *           calibration needs no host synchronisation
+ *   q       device, int8 [M, K] dense (output)
+ *   a_scale device, fp32 [M] (output; may be NULL): every entry = the scale
+ *           used, so w8a8_scaled_mm applies it unchanged
+ * Same shape rules and errors as w8a8_quant_act. */
+w8a8_status w8a8_quant_act_static(const void *x, int64_t M, int64_t K, int64_t ldx,
+                                  const float *scale, int8_t *q, float *a_scale,
+                                  w8a8_stream_t stream);
+
 /* ---- step 2 (load time): weight repack ------------------------------------
  * Source: "Issue 5 probe ...", Round two, kernel-path verification
  * ("load -> transpose-repack -> apply"); the layout is this library's own:
@@ -98,6 +114,35 @@ w8a8_status w8a8_pack_weight(const int8_t *w, int64_t N, int64_t K,
 /* Inverse of w8a8_pack_weight (test and inspection use): packed -> w [N, K]. */
 w8a8_status w8a8_unpack_weight(const void *packed, int64_t N, int64_t K,
                                int8_t *w, w8a8_stream_t stream);
+
+/* ---- load time: online weight quantisation + repack in one pass -------------
+ * Source: "Online Quantization", Overview (quantised weights and their scales
+ * computed while the model loads, from a higher-precision checkpoint);
+ * "Issue 5 probe ...", Round one (per-output-channel symmetric int8 weights).
+ * Per output channel n: w_scale[n] = max_k |W[n,k]| / 127 (IEEE fp32
+ * division), code = rint_half_even(W[n,k] / w_scale[n]) in [-127, 127]; an
+ * all-zero channel gets scale 0 and codes 0.  Same rule as w8a8_quant_act
+ * applied to the rows of W.
+ *   w       device, bf16 [N, K] row-major
+ *   packed  device, packed_bytes >= w8a8_packed_weight_bytes(N, K); every byte
+ *           written, same image as w8a8_pack_weight of the int8 codes
+ *   w_scale device, fp32 [N] (output)
+ * Shape rules as w8a8_pack_weight; w, packed, w_scale 16-byte aligned. */
+w8a8_status w8a8_quant_pack_weight(const void *w, int64_t N, int64_t K,
+                                   void *packed, size_t packed_bytes,
+                                   float *w_scale, w8a8_stream_t stream);
+
+/* ---- load time: repack from compressed-tensors int32 storage ----------------
+ * Source: "Issue 5 probe ...", Artifact (weights stored with pack_to_int32:
+ * uint8 biased by 128, four per int32).  Bit order (not printed there; this
+ * library's reading): element 4j+i of a row is bits [8i, 8i+8) of word j,
+ * holding the unsigned byte (w + 128).
+ *   w_i32   device, int32 [N, K/4] row-major, 16-byte aligned
+ *   packed  as w8a8_pack_weight; the result equals w8a8_pack_weight of the
+ *           decoded int8 [N, K] weight. */
+w8a8_status w8a8_pack_weight_int32(const int32_t *w_i32, int64_t N, int64_t K,
+                                   void *packed, size_t packed_bytes,
+                                   w8a8_stream_t stream);
 
 /* ---- steps 3+4: int8 GEMM with the dequantising epilogue -----------------
  * Source: "Issue 5 probe ...", Round two (op cutlass_scaled_mm: int8 x int8

@@ -48,9 +48,12 @@ _SIGNATURES = {
     "w8a8_status_string": ([ctypes.c_int], ctypes.c_char_p),
     "w8a8_abi_version": ([], ctypes.c_int),
     "w8a8_quant_act": ([_P, _I64, _I64, _I64, _P, _P, _P], ctypes.c_int),
+    "w8a8_quant_act_static": ([_P, _I64, _I64, _I64, _P, _P, _P, _P], ctypes.c_int),
     "w8a8_packed_weight_bytes": ([_I64, _I64, ctypes.POINTER(_SZ)], ctypes.c_int),
     "w8a8_pack_weight": ([_P, _I64, _I64, _P, _SZ, _P], ctypes.c_int),
     "w8a8_unpack_weight": ([_P, _I64, _I64, _P, _P], ctypes.c_int),
+    "w8a8_quant_pack_weight": ([_P, _I64, _I64, _P, _SZ, _P, _P], ctypes.c_int),
+    "w8a8_pack_weight_int32": ([_P, _I64, _I64, _P, _SZ, _P], ctypes.c_int),
     "w8a8_scaled_mm_workspace_bytes": ([_I64, _I64, _I64, ctypes.POINTER(_SZ)], ctypes.c_int),
     "w8a8_scaled_mm": ([_P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _P, _SZ, _P], ctypes.c_int),
     "w8a8_scaled_mm_i32": ([_P, _P, _P, _I64, _I64, _I64, _P], ctypes.c_int),
@@ -141,6 +144,56 @@ def quant_act(x: torch.Tensor, q: Optional[torch.Tensor] = None,
     _check(lib().w8a8_quant_act(_ptr(x), M, K, x.stride(0), _ptr(q), _ptr(a_scale), _stream(stream)),
            "w8a8_quant_act")
     return q, a_scale
+
+
+def quant_act_static(x: torch.Tensor, scale: torch.Tensor, q: Optional[torch.Tensor] = None,
+                     a_scale: Optional[torch.Tensor] = None,
+                     stream=None) -> Tuple[torch.Tensor, torch.Tensor]:
+    """x bf16 [M, K] with one calibrated fp32 scale (a 1-element CUDA tensor)
+    -> (q int8 [M, K], a_scale fp32 [M] filled with the scale used)."""
+    _need_cuda(x, "x", torch.bfloat16)
+    _need_cuda(scale, "scale", torch.float32)
+    if scale.numel() != 1:
+        raise ValueError("scale must hold exactly one value")
+    M, K = x.shape
+    if x.stride(1) != 1:
+        raise ValueError("x must have unit stride along K")
+    if q is None:
+        q = torch.empty((M, K), dtype=torch.int8, device=x.device)
+    if a_scale is None:
+        a_scale = torch.empty((M,), dtype=torch.float32, device=x.device)
+    _check(lib().w8a8_quant_act_static(_ptr(x), M, K, x.stride(0), _ptr(scale), _ptr(q),
+                                       _ptr(a_scale), _stream(stream)), "w8a8_quant_act_static")
+    return q, a_scale
+
+
+def quant_pack_weight(w: torch.Tensor, stream=None) -> Tuple[torch.Tensor, torch.Tensor]:
+    """bf16 [N, K] -> (packed int8 tile image, fp32 per-channel w_scale [N]):
+    quantisation at load time, in one pass."""
+    _need_cuda(w, "w", torch.bfloat16)
+    w = w.contiguous()
+    N, K = w.shape
+    nbytes = packed_weight_bytes(N, K)
+    packed = torch.empty((nbytes,), dtype=torch.uint8, device=w.device)
+    w_scale = torch.empty((N,), dtype=torch.float32, device=w.device)
+    _check(lib().w8a8_quant_pack_weight(_ptr(w), N, K, _ptr(packed), nbytes, _ptr(w_scale),
+                                        _stream(stream)), "w8a8_quant_pack_weight")
+    return packed, w_scale
+
+
+def pack_weight_int32(w_i32: torch.Tensor, K: int, stream=None) -> torch.Tensor:
+    """int32 [N, K/4] biased-uint8 storage (four elements per word) -> packed
+    tile image."""
+    _need_cuda(w_i32, "w_i32", torch.int32)
+    w_i32 = w_i32.contiguous()
+    N = w_i32.shape[0]
+    if w_i32.shape[1] * 4 != K:
+        raise ValueError("w_i32 must be [N, K/4]")
+    nbytes = packed_weight_bytes(N, K)
+    packed = torch.empty((nbytes,), dtype=torch.uint8, device=w_i32.device)
+    _check(lib().w8a8_pack_weight_int32(_ptr(w_i32), N, K, _ptr(packed), nbytes, _stream(stream)),
+           "w8a8_pack_weight_int32")
+    return packed
 
 
 def pack_weight(w: torch.Tensor, stream=None) -> torch.Tensor:
@@ -285,6 +338,19 @@ class W8A8Linear:
         self.bias = None if bias is None else bias.to(device=w.device, dtype=torch.bfloat16).contiguous()
         self.splits = tuple(splits) if splits else (self.N,)
         self._ws = None
+
+    @classmethod
+    def from_float(cls, w: torch.Tensor, bias: Optional[torch.Tensor] = None):
+        """Online quantisation: a bf16 [N, K] weight quantised per output
+        channel and packed on the device at load time."""
+        self = cls.__new__(cls)
+        _need_cuda(w, "w", torch.bfloat16)
+        self.N, self.K = w.shape
+        self.packed, self.w_scale = quant_pack_weight(w)
+        self.bias = None if bias is None else bias.to(device=w.device, dtype=torch.bfloat16).contiguous()
+        self.splits = (self.N,)
+        self._ws = None
+        return self
 
     @classmethod
     def from_blocks(cls, blocks, scales, biases=None):

@@ -21,8 +21,10 @@ namespace {
 
 // One thread per 16-byte chunk of the packed buffer (coalesced writes; the
 // 8 threads of one row read one contiguous 128-byte row segment).
+// `flip` is XORed into every source word: 0 for int8 input, 0x80808080 for
+// the biased-uint8 int32 storage (byte (w + 128) XOR 0x80 is w as int8).
 __global__ void pack_kernel(const int8_t *__restrict__ w, int64_t N, int64_t K, int64_t kblocks,
-                            int64_t total_chunks, uint4 *__restrict__ out) {
+                            int64_t total_chunks, uint32_t flip, uint4 *__restrict__ out) {
   for (int64_t o = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; o < total_chunks;
        o += (int64_t)gridDim.x * blockDim.x) {
     const int64_t tile = o >> 10;          // 1024 chunks per tile
@@ -32,7 +34,13 @@ __global__ void pack_kernel(const int8_t *__restrict__ w, int64_t N, int64_t K, 
     const int64_t n = (tile / kblocks) * 128 + r;
     const int64_t k = (tile % kblocks) * 128 + j * 16;
     uint4 v = make_uint4(0, 0, 0, 0);
-    if (n < N && k < K) v = *reinterpret_cast<const uint4 *>(w + n * K + k);
+    if (n < N && k < K) {
+      v = *reinterpret_cast<const uint4 *>(w + n * K + k);
+      v.x ^= flip;
+      v.y ^= flip;
+      v.z ^= flip;
+      v.w ^= flip;
+    }
     out[o] = v;
   }
 }
@@ -49,6 +57,16 @@ __global__ void unpack_kernel(const uint4 *__restrict__ in, int64_t N, int64_t K
     const int64_t k = (tile % kblocks) * 128 + j * 16;
     if (n < N && k < K) *reinterpret_cast<uint4 *>(w + n * K + k) = in[o];
   }
+}
+
+w8a8_status launch_pack(const int8_t *w, int64_t N, int64_t K, void *packed, uint32_t flip,
+                        cudaStream_t stream) {
+  const int64_t chunks = packed_rows(N) * packed_cols(K) / 16;
+  const int64_t blocks = std::min<int64_t>((chunks + 255) / 256, (int64_t)sm_count() * 16);
+  pack_kernel<<<(unsigned)blocks, 256, 0, stream>>>(w, N, K, packed_cols(K) / 128, chunks, flip,
+                                                    static_cast<uint4 *>(packed));
+  count_launch();
+  return from_cuda(cudaGetLastError());
 }
 
 w8a8_status check_weight_shape(int64_t N, int64_t K) {
@@ -81,12 +99,19 @@ w8a8_status w8a8_pack_weight(const int8_t *w, int64_t N, int64_t K, void *packed
   if (!aligned16(w) || !aligned16(packed)) return W8A8_ERR_ALIGNMENT;
   const int64_t need = packed_rows(N) * packed_cols(K);
   if ((int64_t)packed_bytes < need) return W8A8_ERR_BUFFER_TOO_SMALL;
-  const int64_t chunks = need / 16;
-  const int64_t blocks = std::min<int64_t>((chunks + 255) / 256, (int64_t)sm_count() * 16);
-  pack_kernel<<<(unsigned)blocks, 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
-      w, N, K, packed_cols(K) / 128, chunks, static_cast<uint4 *>(packed));
-  count_launch();
-  return from_cuda(cudaGetLastError());
+  return launch_pack(w, N, K, packed, 0u, reinterpret_cast<cudaStream_t>(stream));
+}
+
+w8a8_status w8a8_pack_weight_int32(const int32_t *w_i32, int64_t N, int64_t K, void *packed,
+                                   size_t packed_bytes, w8a8_stream_t stream) {
+  if (!w_i32 || !packed) return W8A8_ERR_INVALID_ARG;
+  const w8a8_status st = check_weight_shape(N, K);
+  if (st != W8A8_OK) return st;
+  if (!aligned16(w_i32) || !aligned16(packed)) return W8A8_ERR_ALIGNMENT;
+  const int64_t need = packed_rows(N) * packed_cols(K);
+  if ((int64_t)packed_bytes < need) return W8A8_ERR_BUFFER_TOO_SMALL;
+  return launch_pack(reinterpret_cast<const int8_t *>(w_i32), N, K, packed, 0x80808080u,
+                     reinterpret_cast<cudaStream_t>(stream));
 }
 
 w8a8_status w8a8_unpack_weight(const void *packed, int64_t N, int64_t K, int8_t *w,

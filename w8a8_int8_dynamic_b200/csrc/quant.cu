@@ -24,6 +24,8 @@
 // (where 1/s could overflow) always take the IEEE quotient.
 #include <cuda_bf16.h>
 
+#include <algorithm>
+
 #include "internal.h"
 #include "ptx.cuh"
 
@@ -185,6 +187,72 @@ __global__ void __launch_bounds__(1024) quant_rows_two_pass_kernel(
   }
 }
 
+// Static (calibrated) per-tensor scale: code = clamp(rint(RN(x / scale)),
+// -127, 127); a scale that is not > 0 gives codes 0 and a_scale 0.  The scale
+// is read from device memory, so a calibrated value can change without a host
+// round trip.  One thread per 16-element chunk (32 bytes in, 16 bytes out),
+// grid-stride over all M * K/16 chunks.  The reciprocal shortcut holds while
+// |y| <= 256 (error < 256 * 3 * 2^-24 < 1e-4 of the quotient); beyond that
+// the code saturates either way.  Scales outside [1e-30, 1e30] (where RN(1/s)
+// overflows or goes subnormal) always take the IEEE quotient.
+__device__ __forceinline__ int quant_static_one(float x, float s, float inv, bool exact_only) {
+  float v;
+  if (exact_only) {
+    v = rintf(__fdiv_rn(x, s));
+  } else {
+    const float y = __fmul_rn(x, inv);
+    if (fabsf(y) > 256.0f) return y > 0.0f ? 127 : -127;
+    v = rintf(y);
+    if (fabsf(y - v) > 0.4999f) v = rintf(__fdiv_rn(x, s));
+  }
+  v = fminf(fmaxf(v, -127.0f), 127.0f);
+  return (int)v;
+}
+
+__global__ void __launch_bounds__(256) quant_static_kernel(const uint16_t *__restrict__ x,
+                                                           int64_t ldx, int64_t M, int K,
+                                                           const float *__restrict__ scale_ptr,
+                                                           int8_t *__restrict__ q,
+                                                           float *__restrict__ a_scale) {
+  griddep_launch_dependents();
+  const float s_in = *scale_ptr;
+  const bool usable = s_in > 0.0f;  // false for NaN
+  const float s = usable ? s_in : 0.0f;
+  const bool exact_only = !(s >= 1e-30f && s <= 1e30f);
+  const float inv = exact_only ? 0.0f : __frcp_rn(s);
+  const int per_row = K >> 4;
+  const int64_t total = M * per_row;
+  for (int64_t c = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; c < total;
+       c += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t m = c / per_row;
+    const int k = (int)(c - m * per_row) * 16;
+    if (k == 0 && a_scale) a_scale[m] = s;
+    uint4 out = make_uint4(0, 0, 0, 0);
+    if (usable) {
+      const uint16_t *src = x + m * ldx + k;
+      const uint4 a = ld_stream_u4(src);
+      const uint4 b = ld_stream_u4(src + 8);
+      out.x = pack4(quant_static_one(bf16_lo(a.x), s, inv, exact_only),
+                    quant_static_one(bf16_hi(a.x), s, inv, exact_only),
+                    quant_static_one(bf16_lo(a.y), s, inv, exact_only),
+                    quant_static_one(bf16_hi(a.y), s, inv, exact_only));
+      out.y = pack4(quant_static_one(bf16_lo(a.z), s, inv, exact_only),
+                    quant_static_one(bf16_hi(a.z), s, inv, exact_only),
+                    quant_static_one(bf16_lo(a.w), s, inv, exact_only),
+                    quant_static_one(bf16_hi(a.w), s, inv, exact_only));
+      out.z = pack4(quant_static_one(bf16_lo(b.x), s, inv, exact_only),
+                    quant_static_one(bf16_hi(b.x), s, inv, exact_only),
+                    quant_static_one(bf16_lo(b.y), s, inv, exact_only),
+                    quant_static_one(bf16_hi(b.y), s, inv, exact_only));
+      out.w = pack4(quant_static_one(bf16_lo(b.z), s, inv, exact_only),
+                    quant_static_one(bf16_hi(b.z), s, inv, exact_only),
+                    quant_static_one(bf16_lo(b.w), s, inv, exact_only),
+                    quant_static_one(bf16_hi(b.w), s, inv, exact_only));
+    }
+    *reinterpret_cast<uint4 *>(q + m * K + k) = out;
+  }
+}
+
 }  // namespace
 
 w8a8_status launch_quant(const void *x, int64_t M, int64_t K, int64_t ldx, int8_t *q,
@@ -228,4 +296,22 @@ extern "C" w8a8_status w8a8_quant_act(const void *x, int64_t M, int64_t K, int64
   if (!aligned16(x) || !aligned16(q) || !aligned16(a_scale) || ldx % 8 != 0)
     return W8A8_ERR_ALIGNMENT;
   return launch_quant(x, M, K, ldx, q, a_scale, reinterpret_cast<cudaStream_t>(stream));
+}
+
+
+extern "C" w8a8_status w8a8_quant_act_static(const void *x, int64_t M, int64_t K, int64_t ldx,
+                                             const float *scale, int8_t *q, float *a_scale,
+                                             w8a8_stream_t stream) {
+  if (!x || !q || !scale) return W8A8_ERR_INVALID_ARG;
+  if (M < 1 || M > 0x7FFFFFFF || K < 1 || ldx < K) return W8A8_ERR_INVALID_ARG;
+  if (K % 16 != 0 || K > kMaxK) return W8A8_ERR_UNSUPPORTED_SHAPE;
+  if (!aligned16(x) || !aligned16(q) || ldx % 8 != 0 ||
+      (reinterpret_cast<uintptr_t>(scale) & 3u) || (a_scale && !aligned16(a_scale)))
+    return W8A8_ERR_ALIGNMENT;
+  const int64_t chunks = M * (K / 16);
+  const int64_t blocks = std::min<int64_t>((chunks + 255) / 256, (int64_t)sm_count() * 8);
+  quant_static_kernel<<<(unsigned)blocks, 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+      static_cast<const uint16_t *>(x), ldx, M, (int)K, scale, q, a_scale);
+  count_launch();
+  return from_cuda(cudaGetLastError());
 }
