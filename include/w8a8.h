@@ -62,6 +62,17 @@ typedef enum w8a8_status {
   W8A8_ERR_BUFFER_TOO_SMALL = 6   /* packed or workspace buffer too small */
 } w8a8_status;
 
+/* Activation applied to the layer output inside the GEMM epilogue.
+ * W8A8_ACT_GELU_TANH: the output is bf16(GELU_tanh(bf16(y))), i.e. exactly
+ * the result of the plain layer followed by w8a8_gelu_tanh, without the
+ * round trip of y through memory.  GELU_tanh(v) = 0.5 v (1 + tanh(sqrt(2/pi)
+ * (v + 0.044715 v^3))) in fp32; it joins the up- and down-projections of a
+ * transformer MLP and is not part of the quantisation method. */
+typedef enum {
+  W8A8_ACT_NONE = 0,
+  W8A8_ACT_GELU_TANH = 1
+} w8a8_act;
+
 /* Human-readable name of a status code (static string, never NULL). */
 const char *w8a8_status_string(int status);
 
@@ -168,6 +179,16 @@ w8a8_status w8a8_scaled_mm(const int8_t *q, const float *a_scale,
                            int64_t K, void *workspace, size_t ws_bytes,
                            w8a8_stream_t stream);
 
+/* w8a8_scaled_mm with an activation (w8a8_act) applied in the epilogue:
+ * act = W8A8_ACT_GELU_TANH writes bf16(GELU_tanh(y)) instead of y (the
+ * fused form of the MLP up-projection followed by its GELU).  Any other
+ * value than the w8a8_act members -> W8A8_ERR_INVALID_ARG. */
+w8a8_status w8a8_scaled_mm_act(const int8_t *q, const float *a_scale,
+                               const void *packed_w, const float *w_scale,
+                               const void *bias, void *y, int64_t M, int64_t N,
+                               int64_t K, int act, void *workspace,
+                               size_t ws_bytes, w8a8_stream_t stream);
+
 /* The int32 accumulators acc[M, N] of the same GEMM, without the epilogue
  * (test and inspection use; acc device, int32 [M, N]). */
 w8a8_status w8a8_scaled_mm_i32(const int8_t *q, const void *packed_w,
@@ -192,6 +213,14 @@ w8a8_status w8a8_linear(const void *x, int64_t ldx, const void *packed_w,
                         const float *w_scale, const void *bias, void *y,
                         int64_t M, int64_t N, int64_t K, void *workspace,
                         size_t ws_bytes, w8a8_stream_t stream);
+
+/* w8a8_linear with an activation applied in the epilogue (see
+ * w8a8_scaled_mm_act); same workspace. */
+w8a8_status w8a8_linear_act(const void *x, int64_t ldx, const void *packed_w,
+                            const float *w_scale, const void *bias, void *y,
+                            int64_t M, int64_t N, int64_t K, int act,
+                            void *workspace, size_t ws_bytes,
+                            w8a8_stream_t stream);
 
 /* ---- the whole layer without a caller-provided workspace ---------------------
  * No counterpart on the pages: an addition for callers that cannot allocate

@@ -30,6 +30,8 @@ STATUS_NAMES = {
 PATH_AUTO, PATH_LARGE, PATH_SMALL, PATH_LARGE_BN128, PATH_LARGE_BN256, PATH_LARGE_PAIR = 0, 1, 2, 3, 4, 5
 PATH_LARGE_PAIR_SPLIT = 6
 PATH_LARGE_PAIR128 = 7
+# activations fused into the GEMM epilogue (w8a8_act)
+ACT_NONE, ACT_GELU_TANH = 0, 1
 
 
 class W8A8Error(RuntimeError):
@@ -56,9 +58,13 @@ _SIGNATURES = {
     "w8a8_pack_weight_int32": ([_P, _I64, _I64, _P, _SZ, _P], ctypes.c_int),
     "w8a8_scaled_mm_workspace_bytes": ([_I64, _I64, _I64, ctypes.POINTER(_SZ)], ctypes.c_int),
     "w8a8_scaled_mm": ([_P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _P, _SZ, _P], ctypes.c_int),
+    "w8a8_scaled_mm_act": ([_P, _P, _P, _P, _P, _P, _I64, _I64, _I64, ctypes.c_int, _P, _SZ, _P],
+                           ctypes.c_int),
     "w8a8_scaled_mm_i32": ([_P, _P, _P, _I64, _I64, _I64, _P], ctypes.c_int),
     "w8a8_linear_workspace_bytes": ([_I64, _I64, _I64, ctypes.POINTER(_SZ)], ctypes.c_int),
     "w8a8_linear": ([_P, _I64, _P, _P, _P, _P, _I64, _I64, _I64, _P, _SZ, _P], ctypes.c_int),
+    "w8a8_linear_act": ([_P, _I64, _P, _P, _P, _P, _I64, _I64, _I64, ctypes.c_int, _P, _SZ, _P],
+                        ctypes.c_int),
     "w8a8_linear_noalloc_max_bytes": ([], _SZ),
     "w8a8_linear_noalloc": ([_P, _I64, _P, _P, _P, _P, _I64, _I64, _I64, _P], ctypes.c_int),
     "w8a8_set_path": ([ctypes.c_int], ctypes.c_int),
@@ -219,16 +225,17 @@ def unpack_weight(packed: torch.Tensor, N: int, K: int, stream=None) -> torch.Te
 def scaled_mm(q: torch.Tensor, a_scale: torch.Tensor, packed_w: torch.Tensor,
               w_scale: torch.Tensor, bias: Optional[torch.Tensor], N: int,
               out: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None,
-              stream=None) -> torch.Tensor:
-    """q int8 [M, K] x packed W -> y bf16 [M, N]."""
+              stream=None, act: int = ACT_NONE) -> torch.Tensor:
+    """q int8 [M, K] x packed W -> y bf16 [M, N] (``act``: epilogue activation)."""
     _need_cuda(q, "q", torch.int8)
     M, K = q.shape
     if out is None:
         out = torch.empty((M, N), dtype=torch.bfloat16, device=q.device)
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
-    _check(lib().w8a8_scaled_mm(_ptr(q), _ptr(a_scale), _ptr(packed_w), _ptr(w_scale), _ptr(bias),
-                                _ptr(out), M, N, K, _ptr(workspace), ws_bytes, _stream(stream)),
-           "w8a8_scaled_mm")
+    _check(lib().w8a8_scaled_mm_act(_ptr(q), _ptr(a_scale), _ptr(packed_w), _ptr(w_scale),
+                                    _ptr(bias), _ptr(out), M, N, K, act, _ptr(workspace), ws_bytes,
+                                    _stream(stream)),
+           "w8a8_scaled_mm_act")
     return out
 
 
@@ -245,8 +252,9 @@ def scaled_mm_i32(q: torch.Tensor, packed_w: torch.Tensor, N: int,
 
 def linear(x: torch.Tensor, packed_w: torch.Tensor, w_scale: torch.Tensor,
            bias: Optional[torch.Tensor], N: int, out: Optional[torch.Tensor] = None,
-           workspace: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
-    """The whole layer: y[..., N] = W8A8(x[..., K])."""
+           workspace: Optional[torch.Tensor] = None, stream=None,
+           act: int = ACT_NONE) -> torch.Tensor:
+    """The whole layer: y[..., N] = W8A8(x[..., K]) (``act``: epilogue activation)."""
     _need_cuda(x, "x", torch.bfloat16)
     lead = x.shape[:-1]
     K = x.shape[-1]
@@ -260,9 +268,10 @@ def linear(x: torch.Tensor, packed_w: torch.Tensor, w_scale: torch.Tensor,
     if workspace is None:
         workspace = torch.empty((need,), dtype=torch.uint8, device=x.device)
     ws_bytes = workspace.numel() * workspace.element_size()
-    _check(lib().w8a8_linear(_ptr(x2), x2.stride(0), _ptr(packed_w), _ptr(w_scale), _ptr(bias),
-                             _ptr(out), M, N, K, _ptr(workspace), ws_bytes, _stream(stream)),
-           "w8a8_linear")
+    _check(lib().w8a8_linear_act(_ptr(x2), x2.stride(0), _ptr(packed_w), _ptr(w_scale), _ptr(bias),
+                                 _ptr(out), M, N, K, act, _ptr(workspace), ws_bytes,
+                                 _stream(stream)),
+           "w8a8_linear_act")
     return out.view(*lead, N)
 
 
@@ -330,8 +339,9 @@ class W8A8Linear:
     """
 
     def __init__(self, w: torch.Tensor, w_scale: torch.Tensor, bias: Optional[torch.Tensor] = None,
-                 splits: Optional[Tuple[int, ...]] = None):
+                 splits: Optional[Tuple[int, ...]] = None, act: int = ACT_NONE):
         _need_cuda(w, "w", torch.int8)
+        self.act = act
         self.N, self.K = w.shape
         self.packed = pack_weight(w)
         self.w_scale = w_scale.to(device=w.device, dtype=torch.float32).contiguous()
@@ -340,10 +350,12 @@ class W8A8Linear:
         self._ws = None
 
     @classmethod
-    def from_float(cls, w: torch.Tensor, bias: Optional[torch.Tensor] = None):
+    def from_float(cls, w: torch.Tensor, bias: Optional[torch.Tensor] = None,
+                   act: int = ACT_NONE):
         """Online quantisation: a bf16 [N, K] weight quantised per output
         channel and packed on the device at load time."""
         self = cls.__new__(cls)
+        self.act = act
         _need_cuda(w, "w", torch.bfloat16)
         self.N, self.K = w.shape
         self.packed, self.w_scale = quant_pack_weight(w)
@@ -364,7 +376,8 @@ class W8A8Linear:
         need = linear_workspace_bytes(M, self.N, self.K)
         if self._ws is None or self._ws.numel() < need or self._ws.device != x.device:
             self._ws = torch.empty((need,), dtype=torch.uint8, device=x.device)
-        return linear(x, self.packed, self.w_scale, self.bias, self.N, workspace=self._ws)
+        return linear(x, self.packed, self.w_scale, self.bias, self.N, workspace=self._ws,
+                      act=self.act)
 
     def split(self, y: torch.Tensor):
         return torch.split(y, list(self.splits), dim=-1)

@@ -60,6 +60,7 @@ struct DecodeArgs {
   int32_t *partials;             // [num_nb][max_contrib][16][128]
   unsigned long long *counters;  // [num_nb]: (tag << 8) | arrivals
   unsigned long long tag;        // this call's tag (56 bits)
+  int act;                       // w8a8_act applied after the dequantisation
   int *status;
 };
 
@@ -309,6 +310,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (m < args.M) {
             float t = dequant((int32_t)r[m], as[m], ws);
             if (args.bias) t = __fadd_rn(t, bv);
+            t = apply_act(t, args.act);
             const __nv_bfloat16 h = __float2bfloat16_rn(t);
             args.y[(int64_t)m * args.N + n] = *reinterpret_cast<const uint16_t *>(&h);
           }
@@ -362,7 +364,8 @@ bool use_decode_path(int64_t M) {
 
 w8a8_status launch_decode(const int8_t *q, const float *a_scale, const void *packed_w,
                           const float *w_scale, const void *bias, void *y, int64_t M,
-                          int64_t N, int64_t K, void *workspace, cudaStream_t stream, bool pdl) {
+                          int64_t N, int64_t K, void *workspace, cudaStream_t stream, bool pdl,
+                          int act) {
   CUtensorMap tmap;
   if (!make_tmap_u8_2d(&tmap, q, (uint64_t)M, (uint64_t)K, (uint64_t)K, kDecodeNT, kBK))
     return W8A8_ERR_CUDA;
@@ -386,6 +389,7 @@ w8a8_status launch_decode(const int8_t *q, const float *a_scale, const void *pac
   a.counters = reinterpret_cast<unsigned long long *>(ws);
   a.partials = reinterpret_cast<int32_t *>(ws + round_up(nb * 8, 256));
   a.tag = (g_tag.fetch_add(1) + 1) & ((1ull << 56) - 1);
+  a.act = act;
   a.status = status_word();
   if (!a.status) return W8A8_ERR_CUDA;
   cudaError_t e = cudaSuccess;

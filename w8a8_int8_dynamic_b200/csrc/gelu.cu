@@ -6,27 +6,15 @@
 // element; 8 elements per thread with 128-bit loads and stores.
 #include <cuda_bf16.h>
 
+#include "act.cuh"
 #include "internal.h"
 
 namespace w8a8 {
 namespace {
 
-// GELU_tanh(x) = 0.5 x (1 + tanh(u)), u = sqrt(2/pi)(x + 0.044715 x^3),
-// evaluated as x * sigma(2u) (the same function: 0.5(1 + tanh(u)) = 1/(1 + e^-2u)),
-// with sigma written so nothing cancels: 1 + tanh(u) in fp32 is exactly 0
-// once tanh(u) rounds to -1 (u < -9), which would flush whole ranges of
-// small negative outputs to -0.
-__device__ __forceinline__ float gelu_f(float x) {
-  const float c = 0.7978845608028654f;  // sqrt(2 / pi)
-  const float u = c * (x + 0.044715f * x * x * x);
-  const float e = expf(-2.0f * fabsf(u));  // in (0, 1]
-  const float sig = u >= 0.0f ? 1.0f / (1.0f + e) : e / (1.0f + e);
-  return x * sig;
-}
-
 __device__ __forceinline__ uint32_t gelu2(uint32_t v) {
-  const float a = gelu_f(__uint_as_float(v << 16));
-  const float b = gelu_f(__uint_as_float(v & 0xFFFF0000u));
+  const float a = gelu_tanh_f(__uint_as_float(v << 16));
+  const float b = gelu_tanh_f(__uint_as_float(v & 0xFFFF0000u));
   const __nv_bfloat162 r = __floats2bfloat162_rn(a, b);
   return *reinterpret_cast<const uint32_t *>(&r);
 }
@@ -40,7 +28,7 @@ __global__ void gelu_kernel(const uint4 *__restrict__ x, uint4 *__restrict__ y, 
     y[i] = make_uint4(gelu2(v.x), gelu2(v.y), gelu2(v.z), gelu2(v.w));
   }
   if (blockIdx.x == 0 && threadIdx.x < tail) {
-    const float a = gelu_f(__uint_as_float((uint32_t)xt[threadIdx.x] << 16));
+    const float a = gelu_tanh_f(__uint_as_float((uint32_t)xt[threadIdx.x] << 16));
     const __nv_bfloat16 r = __float2bfloat16_rn(a);
     yt[threadIdx.x] = *reinterpret_cast<const uint16_t *>(&r);
   }

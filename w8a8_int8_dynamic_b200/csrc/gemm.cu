@@ -364,7 +364,8 @@ LargeKind choose_large(int64_t M, int64_t N, int64_t K) {
 
 w8a8_status launch_scaled_mm(const int8_t *q, const float *a_scale, const void *packed_w,
                              const float *w_scale, const void *bias, void *out, bool out_i32,
-                             int64_t M, int64_t N, int64_t K, cudaStream_t stream, bool pdl) {
+                             int64_t M, int64_t N, int64_t K, cudaStream_t stream, bool pdl,
+                             int act) {
   CUtensorMap tmap;
   if (!make_tmap_u8_2d(&tmap, q, (uint64_t)M, (uint64_t)K, (uint64_t)K, kBM, kBK))
     return W8A8_ERR_CUDA;
@@ -379,6 +380,7 @@ w8a8_status launch_scaled_mm(const int8_t *q, const float *a_scale, const void *
   a.num_kb = (int)(packed_cols(K) / 128);
   a.tiles_m = (int)((M + kBM - 1) / kBM);
   a.tiles_n = 0;
+  a.act = out_i32 ? W8A8_ACT_NONE : act;
   a.status = status_word();
   if (!a.status) return W8A8_ERR_CUDA;
   CUtensorMap tmap_y;
@@ -394,11 +396,14 @@ w8a8_status launch_scaled_mm(const int8_t *q, const float *a_scale, const void *
   if (!make_tmap_out_bf16(&tmap_y, out, (uint64_t)M, (uint64_t)N)) return W8A8_ERR_CUDA;
   switch (choose_large(M, N, K)) {
     case LargeKind::kPair:
-      return launch_gemm2sm(q, a_scale, packed_w, w_scale, bias, out, M, N, K, stream, pdl, 1, 256);
+      return launch_gemm2sm(q, a_scale, packed_w, w_scale, bias, out, M, N, K, stream, pdl, 1, 256,
+                            act);
     case LargeKind::kPair128:
-      return launch_gemm2sm(q, a_scale, packed_w, w_scale, bias, out, M, N, K, stream, pdl, 1, 128);
+      return launch_gemm2sm(q, a_scale, packed_w, w_scale, bias, out, M, N, K, stream, pdl, 1, 128,
+                            act);
     case LargeKind::kPairSplit:
-      return launch_gemm2sm(q, a_scale, packed_w, w_scale, bias, out, M, N, K, stream, pdl, 2, 256);
+      return launch_gemm2sm(q, a_scale, packed_w, w_scale, bias, out, M, N, K, stream, pdl, 2, 256,
+                            act);
     case LargeKind::k256:
       return run_large<256, kLargeStages256, false>(tmap, tmap_y, a, stream, pdl, 2);
     default:
@@ -429,22 +434,32 @@ w8a8_status w8a8_scaled_mm_workspace_bytes(int64_t M, int64_t N, int64_t K, size
   return W8A8_OK;
 }
 
-w8a8_status w8a8_scaled_mm(const int8_t *q, const float *a_scale, const void *packed_w,
-                           const float *w_scale, const void *bias, void *y, int64_t M, int64_t N,
-                           int64_t K, void *workspace, size_t ws_bytes, w8a8_stream_t stream) {
+w8a8_status w8a8_scaled_mm_act(const int8_t *q, const float *a_scale, const void *packed_w,
+                               const float *w_scale, const void *bias, void *y, int64_t M,
+                               int64_t N, int64_t K, int act, void *workspace, size_t ws_bytes,
+                               w8a8_stream_t stream) {
   w8a8_status st = check_gemm_args(q, packed_w, y, M, N, K);
   if (st != W8A8_OK) return st;
   if (!a_scale || !w_scale) return W8A8_ERR_INVALID_ARG;
+  if (act != W8A8_ACT_NONE && act != W8A8_ACT_GELU_TANH) return W8A8_ERR_INVALID_ARG;
   if (!aligned16(a_scale) || !aligned16(w_scale) || (bias && !aligned16(bias)))
     return W8A8_ERR_ALIGNMENT;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   if (use_decode_path(M) && workspace) {
     if (!aligned16(workspace)) return W8A8_ERR_ALIGNMENT;
     if ((int64_t)ws_bytes < decode_workspace_bytes(N, K)) return W8A8_ERR_BUFFER_TOO_SMALL;
-    return launch_decode(q, a_scale, packed_w, w_scale, bias, y, M, N, K, workspace, s, false);
+    return launch_decode(q, a_scale, packed_w, w_scale, bias, y, M, N, K, workspace, s, false,
+                         act);
   }
   if (forced_path() == 2) return W8A8_ERR_INVALID_ARG;  // small path needs M <= 16 and a workspace
-  return launch_scaled_mm(q, a_scale, packed_w, w_scale, bias, y, false, M, N, K, s, false);
+  return launch_scaled_mm(q, a_scale, packed_w, w_scale, bias, y, false, M, N, K, s, false, act);
+}
+
+w8a8_status w8a8_scaled_mm(const int8_t *q, const float *a_scale, const void *packed_w,
+                           const float *w_scale, const void *bias, void *y, int64_t M, int64_t N,
+                           int64_t K, void *workspace, size_t ws_bytes, w8a8_stream_t stream) {
+  return w8a8_scaled_mm_act(q, a_scale, packed_w, w_scale, bias, y, M, N, K, W8A8_ACT_NONE,
+                            workspace, ws_bytes, stream);
 }
 
 const char *w8a8_gemm_kernel_name(int64_t M, int64_t N, int64_t K) {
@@ -476,13 +491,15 @@ w8a8_status w8a8_linear_workspace_bytes(int64_t M, int64_t N, int64_t K, size_t 
   return W8A8_OK;
 }
 
-w8a8_status w8a8_linear(const void *x, int64_t ldx, const void *packed_w, const float *w_scale,
-                        const void *bias, void *y, int64_t M, int64_t N, int64_t K,
-                        void *workspace, size_t ws_bytes, w8a8_stream_t stream) {
+w8a8_status w8a8_linear_act(const void *x, int64_t ldx, const void *packed_w,
+                            const float *w_scale, const void *bias, void *y, int64_t M, int64_t N,
+                            int64_t K, int act, void *workspace, size_t ws_bytes,
+                            w8a8_stream_t stream) {
   w8a8_status st = check_gemm_args(x, packed_w, y, M, N, K);
   if (st != W8A8_OK) return st;
   if (!w_scale || !workspace) return W8A8_ERR_INVALID_ARG;
   if (ldx < K) return W8A8_ERR_INVALID_ARG;
+  if (act != W8A8_ACT_NONE && act != W8A8_ACT_GELU_TANH) return W8A8_ERR_INVALID_ARG;
   if (ldx % 8 != 0 || !aligned16(w_scale) || !aligned16(workspace) ||
       (bias && !aligned16(bias)))
     return W8A8_ERR_ALIGNMENT;
@@ -498,10 +515,17 @@ w8a8_status w8a8_linear(const void *x, int64_t ldx, const void *packed_w, const 
   if (st != W8A8_OK) return st;
   if (use_decode_path(M)) {
     void *dws = ws + round_up(M * K, 256) + round_up(M * 4, 256);
-    return launch_decode(q, a_scale, packed_w, w_scale, bias, y, M, N, K, dws, s, true);
+    return launch_decode(q, a_scale, packed_w, w_scale, bias, y, M, N, K, dws, s, true, act);
   }
   if (forced_path() == 2) return W8A8_ERR_INVALID_ARG;
-  return launch_scaled_mm(q, a_scale, packed_w, w_scale, bias, y, false, M, N, K, s, true);
+  return launch_scaled_mm(q, a_scale, packed_w, w_scale, bias, y, false, M, N, K, s, true, act);
+}
+
+w8a8_status w8a8_linear(const void *x, int64_t ldx, const void *packed_w, const float *w_scale,
+                        const void *bias, void *y, int64_t M, int64_t N, int64_t K,
+                        void *workspace, size_t ws_bytes, w8a8_stream_t stream) {
+  return w8a8_linear_act(x, ldx, packed_w, w_scale, bias, y, M, N, K, W8A8_ACT_NONE, workspace,
+                         ws_bytes, stream);
 }
 
 }  // extern "C"

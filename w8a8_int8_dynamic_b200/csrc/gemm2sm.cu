@@ -375,7 +375,8 @@ int64_t pair_tiles(int64_t M, int64_t N, int bn) { return ((M + 255) / 256) * ((
 
 w8a8_status launch_gemm2sm(const int8_t *q, const float *a_scale, const void *packed_w,
                            const float *w_scale, const void *bias, void *y, int64_t M, int64_t N,
-                           int64_t K, cudaStream_t stream, bool pdl, int split, int bn) {
+                           int64_t K, cudaStream_t stream, bool pdl, int split, int bn,
+                           int act) {
   CUtensorMap tq, tw, ty;
   if (!make_tmap_u8_2d(&tq, q, (uint64_t)M, (uint64_t)K, (uint64_t)K, kBM, kBK))
     return W8A8_ERR_CUDA;
@@ -394,6 +395,7 @@ w8a8_status launch_gemm2sm(const int8_t *q, const float *a_scale, const void *pa
   a.num_kb = (int)(packed_cols(K) / 128);
   a.tiles_m = (int)((M + 255) / 256);
   a.tiles_n = (int)((N + bn - 1) / bn);
+  a.act = act;
   a.status = status_word();
   if (!a.status) return W8A8_ERR_CUDA;
   if (bn == 128) return run_pair<128, 4, 1>(tq, tw, ty, a, stream, pdl, 2);

@@ -7,6 +7,7 @@
 
 #include <cuda_bf16.h>
 
+#include "act.cuh"
 #include "internal.h"
 #include "ptx.cuh"
 
@@ -27,6 +28,7 @@ struct GemmArgs {
   int M, N;
   int num_kb;            // K blocks of 128 bytes (= packed K / 128)
   int tiles_m, tiles_n;
+  int act;               // w8a8_act applied after the dequantisation
   int *status;
 };
 
@@ -115,6 +117,10 @@ __device__ __forceinline__ void epilogue_tile(const GemmArgs &a, uint32_t tmem_c
             t[2 * h + 1] = __fadd_rn(t[2 * h + 1], __uint_as_float(bw[h] & 0xFFFF0000u));
           }
         }
+        if (a.act != W8A8_ACT_NONE) {
+#pragma unroll
+          for (int h = 0; h < 8; ++h) t[h] = apply_act(t[h], a.act);
+        }
         if (row_ok) {
           uint16_t *dst = static_cast<uint16_t *>(a.out) + (int64_t)row * a.N + nn;
           *reinterpret_cast<uint4 *>(dst) =
@@ -197,6 +203,10 @@ __device__ __forceinline__ void epilogue_tile_tma(const GemmArgs &a, const CUten
           t[2 * h] = __fadd_rn(t[2 * h], __uint_as_float(bw[h] << 16));
           t[2 * h + 1] = __fadd_rn(t[2 * h + 1], __uint_as_float(bw[h] & 0xFFFF0000u));
         }
+      }
+      if (a.act != W8A8_ACT_NONE) {
+#pragma unroll
+        for (int h = 0; h < 8; ++h) t[h] = apply_act(t[h], a.act);
       }
       *reinterpret_cast<uint4 *>(buf + swz64_offset(lane, g)) =
           make_uint4(pack_bf16x2(t[0], t[1]), pack_bf16x2(t[2], t[3]), pack_bf16x2(t[4], t[5]),

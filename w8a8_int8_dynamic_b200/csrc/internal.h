@@ -55,18 +55,21 @@ inline int64_t packed_cols(int64_t K) { return round_up(K, 128); }
 // GEMM launchers (gemm.cu).
 w8a8_status launch_scaled_mm(const int8_t *q, const float *a_scale, const void *packed_w,
                              const float *w_scale, const void *bias, void *out, bool out_i32,
-                             int64_t M, int64_t N, int64_t K, cudaStream_t stream, bool pdl);
+                             int64_t M, int64_t N, int64_t K, cudaStream_t stream, bool pdl,
+                             int act = W8A8_ACT_NONE);
 // 2-SM (CTA pair) GEMM with the bf16 epilogue (gemm2sm.cu).
 w8a8_status launch_gemm2sm(const int8_t *q, const float *a_scale, const void *packed_w,
                            const float *w_scale, const void *bias, void *y, int64_t M, int64_t N,
-                           int64_t K, cudaStream_t stream, bool pdl, int split, int bn);
+                           int64_t K, cudaStream_t stream, bool pdl, int split, int bn,
+                           int act = W8A8_ACT_NONE);
 int64_t pair_tiles(int64_t M, int64_t N, int bn);
 // Small-M weight-streaming kernel (decode.cu).
 int64_t decode_workspace_bytes(int64_t N, int64_t K);
 bool use_decode_path(int64_t M);
 w8a8_status launch_decode(const int8_t *q, const float *a_scale, const void *packed_w,
                           const float *w_scale, const void *bias, void *y, int64_t M,
-                          int64_t N, int64_t K, void *workspace, cudaStream_t stream, bool pdl);
+                          int64_t N, int64_t K, void *workspace, cudaStream_t stream, bool pdl,
+                          int act = W8A8_ACT_NONE);
 // Quantisation launcher (quant.cu).
 w8a8_status launch_quant(const void *x, int64_t M, int64_t K, int64_t ldx, int8_t *q,
                          float *a_scale, cudaStream_t stream);
