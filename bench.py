@@ -78,14 +78,15 @@ class ClockSampler:
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
-    def __init__(self, index: int):
+    def __init__(self, index: int, tag: str = ""):
         self.index = index
+        self.tag = tag
         self.proc = None
         self.path = None
 
     def start(self):
         os.makedirs(os.path.join(HERE, "gpurun_out"), exist_ok=True)
-        self.path = os.path.join(HERE, "gpurun_out", f"clocks_rank{self.index}.csv")
+        self.path = os.path.join(HERE, "gpurun_out", f"clocks_rank{self.index}{self.tag}.csv")
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}",
@@ -129,6 +130,10 @@ class ClockSampler:
 
 
 # ----------------------------------------------------------------------------- helpers
+def smi_index(device):
+    return torch.cuda.current_device() if "CUDA_VISIBLE_DEVICES" in os.environ else device.index or 0
+
+
 def bf16_dev(a_u16: np.ndarray, device) -> torch.Tensor:
     return torch.from_numpy(np.ascontiguousarray(a_u16).view(np.int16)).to(device).view(torch.bfloat16)
 
@@ -282,8 +287,7 @@ def run_ours(args, rank, world, device):
 
     ls, layer_loop, base = run_workload(w8, wl, 2000, args.warmup, device, stream)
     # ---- the timed region: exactly K steps, barrier + sync on both sides
-    sampler = ClockSampler(torch.cuda.current_device() if "CUDA_VISIBLE_DEVICES" in os.environ
-                           else device.index or 0)
+    sampler = ClockSampler(smi_index(device))
     sampler.start()
     time_loop(layer_loop, args.warmup, stream)  # W untimed warm-up steps
     if world > 1:
@@ -351,6 +355,7 @@ def run_ours(args, rank, world, device):
         out["cpu_baseline"] = cpu_baseline(wl, budget_s=args.cpu_seconds)
     if not args.no_sweep:
         out["sweep"] = sweep(w8, args, device, stream, peaks, int8_peak)
+        out["mlp_chain"] = mlp_chain(w8, device, stream)
     return out
 
 
@@ -416,6 +421,74 @@ def sweep(w8, args, device, stream, peaks, int8_peak):
         }
         del ls, loop
         torch.cuda.empty_cache()
+    return out
+
+
+def mlp_chain(w8, device, stream, steps=128, nsets=2):
+    """The DiT MLP block (4096 tokens, 3072 -> 12288 -> 3072): the two W8A8
+    layers with the GELU between them, unfused (layer, GELU kernel, layer)
+    and with the GELU in the up-projection's epilogue."""
+    up_wl = WORKLOADS["dit_mlp_up_4096x12288x3072"]
+    dn_wl = WORKLOADS["dit_mlp_down_4096x3072x12288"]
+    up, dn = make_inputs(up_wl), make_inputs(dn_wl)
+    M, H, D = up_wl.M, up_wl.N, up_wl.K
+    sets = []
+    for i in range(nsets):
+        s = {"x": bf16_dev(up.x, device),
+             "pu": w8.pack_weight(torch.from_numpy(up.w).to(device)),
+             "su": torch.from_numpy(up.w_scale).to(device), "bu": bf16_dev(up.bias, device),
+             "pd": w8.pack_weight(torch.from_numpy(dn.w).to(device)),
+             "sd": torch.from_numpy(dn.w_scale).to(device), "bd": bf16_dev(dn.bias, device),
+             "h": torch.empty((M, H), dtype=torch.bfloat16, device=device),
+             "g": torch.empty((M, H), dtype=torch.bfloat16, device=device),
+             "y": torch.empty((M, D), dtype=torch.bfloat16, device=device),
+             "wsu": torch.empty((w8.linear_workspace_bytes(M, H, D),), dtype=torch.uint8,
+                                device=device),
+             "wsd": torch.empty((w8.linear_workspace_bytes(M, D, H),), dtype=torch.uint8,
+                                device=device)}
+        sets.append(s)
+    def unfused(s):
+        w8.linear(s["x"], s["pu"], s["su"], s["bu"], H, out=s["h"], workspace=s["wsu"], stream=stream)
+        w8.gelu_tanh(s["h"], out=s["g"], stream=stream)
+        w8.linear(s["g"], s["pd"], s["sd"], s["bd"], D, out=s["y"], workspace=s["wsd"], stream=stream)
+    def fused(s):
+        w8.linear(s["x"], s["pu"], s["su"], s["bu"], H, out=s["g"], workspace=s["wsu"],
+                  stream=stream, act=w8.ACT_GELU_TANH)
+        w8.linear(s["g"], s["pd"], s["sd"], s["bd"], D, out=s["y"], workspace=s["wsd"], stream=stream)
+    def up_only(s, act):
+        w8.linear(s["x"], s["pu"], s["su"], s["bu"], H, out=s["g"], workspace=s["wsu"],
+                  stream=stream, act=act)
+    loops = {
+        "unfused": GraphLoop([lambda s=s: unfused(s) for s in sets], stream, per_graph=8),
+        "fused": GraphLoop([lambda s=s: fused(s) for s in sets], stream, per_graph=8),
+        "up_layer": GraphLoop([lambda s=s: up_only(s, w8.ACT_NONE) for s in sets], stream, 16),
+        "up_layer_gelu": GraphLoop([lambda s=s: up_only(s, w8.ACT_GELU_TANH) for s in sets],
+                                   stream, 16),
+        "gelu_kernel": GraphLoop([lambda s=s: w8.gelu_tanh(s["h"], out=s["g"], stream=stream)
+                                  for s in sets], stream, 16),
+    }
+    torch.cuda.synchronize()
+    for lp in loops.values():
+        time_loop(lp, 3 * lp.per_graph, stream)
+    ops = 2 * (2 * M * H * D)
+    out = {"tokens": M, "dims": [D, H, D]}
+    for name, lp in loops.items():
+        # long enough (>= 0.6 s) for the clock sampler to see the loop
+        t0 = time_loop(lp, lp.per_graph, stream) / lp.per_graph
+        n = max(steps, int(0.6 / t0) // lp.per_graph * lp.per_graph)
+        cs = ClockSampler(smi_index(device), tag="_mlp_" + name)
+        cs.start()
+        t = time_loop(lp, n, stream) / n
+        clk = cs.stop()
+        out[name + "_us"] = round(t * 1e6, 2)
+        out[name + "_sm_mhz"] = clk["sm_mhz"]
+        if clk["reasons"]:
+            out[name + "_clock_reasons"] = clk["reasons"]
+    for name in ("unfused", "fused"):
+        out[name + "_tops"] = round(ops / (out[name + "_us"] * 1e-6) / 1e12, 1)
+    assert w8.poll_status() == 0
+    del sets, loops
+    torch.cuda.empty_cache()
     return out
 
 

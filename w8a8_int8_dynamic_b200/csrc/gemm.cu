@@ -50,11 +50,12 @@ struct LargeSmem {
   static constexpr int kBStage = KPS * BN * kBK;
   static constexpr int kA = 0;
   static constexpr int kB = STAGES * kAStage;
-  // per epilogue warp: the tile's BN w_scale (fp32) and BN bias (bf16) values
-  static constexpr int kEpiPerWarp = BN * 4 + BN * 2;
+  // per epilogue warp: its BN/2 columns' w_scale (fp32) and bias (bf16) values
+  static constexpr int kEpiPerWarp = (BN / 2) * 6;
   static constexpr int kEpi = kB + STAGES * kBStage;
-  static constexpr int kOut = kEpi + 4 * kEpiPerWarp + 1024 - (kEpi + 4 * kEpiPerWarp) % 1024;
-  static constexpr int kBars = kOut + 4 * kEpiStagePerWarp;  // full[S], empty[S], tfull[2], tempty[2], done
+  static constexpr int kEpiEnd = kEpi + kEpiWarps * kEpiPerWarp;
+  static constexpr int kOut = kEpiEnd + 1024 - kEpiEnd % 1024;
+  static constexpr int kBars = kOut + kEpiWarps * kEpiStagePerWarp;  // full[S], empty[S], tfull[2], tempty[2], done
   static constexpr int kMisc = kBars + (2 * STAGES + 5) * 8;
   static constexpr int kUsed = kMisc + 16;
   static constexpr int kAlloc = kUsed + 1024;  // slack for 1024-byte alignment
@@ -62,7 +63,7 @@ struct LargeSmem {
 };
 
 template <int BN, int STAGES, int KPS, bool OUT_I32>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kGemmThreads, 1)
     gemm_kernel(const __grid_constant__ CUtensorMap tmap_q,
                 const __grid_constant__ CUtensorMap tmap_y, const GemmArgs args) {
   using L = LargeSmem<BN, STAGES, KPS>;
@@ -90,7 +91,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&tfull[b], 1);
-      mbar_init(&tempty[b], 4);  // one arrival per epilogue warp
+      mbar_init(&tempty[b], kEpiWarps);  // one arrival per epilogue warp
     }
     mbar_init(mma_done, 1);
     *abort_flag = 0;
@@ -208,23 +209,24 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     __syncwarp();
   } else {
-    // ---------------- epilogue (warps 2..5) ----------------
+    // ---------------- epilogue (warps 2..9) ----------------
     griddep_wait();  // a_scale comes from the preceding kernel
-    const int quarter = warp & 3;  // TMEM lanes this warp may access
+    constexpr int kCols = BN / 2;  // columns of the tile this warp drains
+    const EpiWarp ew(warp);
     float *s_ws = reinterpret_cast<float *>(smem + L::kEpi + (warp - 2) * L::kEpiPerWarp);
-    uint16_t *s_bias = reinterpret_cast<uint16_t *>(s_ws + BN);
+    uint16_t *s_bias = reinterpret_cast<uint16_t *>(s_ws + kCols);
     uint8_t *s_out = smem + L::kOut + (warp - 2) * kEpiStagePerWarp;
-    uint32_t out_count = 0;
     for (int t = 0; t < my_tiles; ++t) {
       const int tile = blockIdx.x + t * gridDim.x;
       const int mb = tile % args.tiles_m, nb = tile / args.tiles_m;
       const uint32_t b = t & 1, bph = (t >> 1) & 1;
+      const int n0 = nb * BN + ew.half * kCols;
+      const int row0 = mb * kBM + ew.quarter * 32;
       // operands of the epilogue, fetched while the main loop runs
       float as = 0.0f;
       if (!OUT_I32) {
-        stage_columns<BN>(args, nb, lane, s_ws, s_bias);
-        const int row = mb * kBM + quarter * 32 + lane;
-        if (row < args.M) as = __ldg(args.a_scale + row);
+        stage_columns<kCols>(args, n0, lane, s_ws, s_bias);
+        if (row0 + lane < args.M) as = __ldg(args.a_scale + row0 + lane);
       }
       __syncwarp();
       int ok = 0;
@@ -232,12 +234,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
       if (!ok) break;
       tc_fence_after();
+      const uint32_t taddr =
+          tmem_base + b * BN + ew.half * kCols + ((uint32_t)(ew.quarter * 32) << 16);
       if (OUT_I32)
-        epilogue_tile<BN, true>(args, tmem_base + b * BN, quarter, lane, mb * kBM, nb, as, s_ws,
-                                s_bias);
+        epilogue_i32<kCols>(args, taddr, row0 + lane, n0);
       else
-        epilogue_tile_tma<BN>(args, &tmap_y, tmem_base + b * BN, quarter, lane, mb * kBM, nb, as,
-                              s_ws, s_bias, s_out, out_count, nullptr, NoExtra());
+        epilogue_tma<kCols>(args, &tmap_y, taddr, lane, row0, n0, as, s_ws, s_bias, s_out,
+                            nullptr, NoExtra());
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&tempty[b]);
@@ -277,7 +280,7 @@ cudaError_t launch_ex(Kernel k, int grid, int smem, cudaStream_t stream, bool pd
                       const Args &...args) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)grid);
-  cfg.blockDim = dim3(kThreads);
+  cfg.blockDim = dim3(kGemmThreads);
   cfg.dynamicSmemBytes = (size_t)smem;
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];

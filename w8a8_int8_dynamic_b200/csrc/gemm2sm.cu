@@ -49,11 +49,12 @@ struct PairSmem {
   static constexpr int kBStage = kStageK * kBTile;
   static constexpr int kA = 0;                          // STAGES x 32 KB q tiles
   static constexpr int kB = STAGES * kHalfStage;        // STAGES x kBStage weight tiles
-  static constexpr int kEpiPerWarp = BN * 4 + BN * 2;
+  static constexpr int kEpiPerWarp = (BN / 2) * 6;  // BN/2 columns: fp32 scale + bf16 bias
   static constexpr int kEpi = kB + STAGES * kBStage;
-  static constexpr int kOut = kEpi + 4 * kEpiPerWarp + 1024 - (kEpi + 4 * kEpiPerWarp) % 1024;
+  static constexpr int kEpiEnd = kEpi + kEpiWarps * kEpiPerWarp;
+  static constexpr int kOut = kEpiEnd + 1024 - kEpiEnd % 1024;
   // full[S], empty[S], tfull[2], tempty[2], done, ready, recv
-  static constexpr int kBars = kOut + 4 * kEpiStagePerWarp;
+  static constexpr int kBars = kOut + kEpiWarps * kEpiStagePerWarp;
   static constexpr int kMisc = kBars + (2 * STAGES + 7) * 8;
   static constexpr int kUsed = kMisc + 16;
   static constexpr int kAlloc = kUsed + 1024;
@@ -65,12 +66,15 @@ struct PairSmem {
 // ((j / 4) * 128 + r) * 4 + j % 4, so the 32 lanes (rows) of a warp move 512
 // contiguous bytes per 16-byte access.
 __device__ __forceinline__ int partial_index(int r, int j) { return ((j >> 2) * 128 + r) * 4 + (j & 3); }
+// Partial element of row r for column j0 + j (the epilogue's column index j
+// counts from the warp's first column j0).
 struct PartialIndex {
-  __device__ int operator()(int r, int j) const { return partial_index(r, j); }
+  int r, j0;
+  __device__ int operator()(int j) const { return partial_index(r, j0 + j); }
 };
 
 template <int BN, int STAGES, int SPLIT>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kGemmThreads, 1)
     gemm2sm_kernel(const __grid_constant__ CUtensorMap tmap_q,
                    const __grid_constant__ CUtensorMap tmap_w,
                    const __grid_constant__ CUtensorMap tmap_y, const GemmArgs args) {
@@ -111,7 +115,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&tfull[b], 1);
-      mbar_init(&tempty[b], 8);  // four epilogue warps in each CTA
+      mbar_init(&tempty[b], 2 * kEpiWarps);  // the epilogue warps of both CTAs
     }
     mbar_init(mma_done, 1);
     mbar_init(ready, 1);
@@ -248,48 +252,48 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     __syncwarp();
   } else {
-    // ---------------- epilogue (warps 2..5, every CTA) ----------------
+    // ---------------- epilogue (warps 2..9, every CTA) ----------------
     griddep_wait();  // a_scale comes from the preceding kernel
-    const int quarter = warp & 3;
-    const int et = threadIdx.x - 64;  // 0..127
+    constexpr int kCols = kPairBN / 2;  // columns of the tile this warp drains
+    const EpiWarp ew(warp);
+    const bool first_epi_thread = threadIdx.x == 64;
     float *s_ws = reinterpret_cast<float *>(smem + L::kEpi + (warp - 2) * L::kEpiPerWarp);
-    uint16_t *s_bias = reinterpret_cast<uint16_t *>(s_ws + kPairBN);
+    uint16_t *s_bias = reinterpret_cast<uint16_t *>(s_ws + kCols);
     uint8_t *s_out = smem + L::kOut + (warp - 2) * kEpiStagePerWarp;
-    uint32_t out_count = 0;
+    const int r = ew.quarter * 32 + lane;  // row within this CTA's 128
+    const int j0 = ew.half * kCols;        // first tile column of this warp
     for (int t = 0; t < my_tiles; ++t) {
       const int tile = slot + t * nslots;
       const int mb = tile % args.tiles_m, nb = tile / args.tiles_m;
-      const int row_base = mb * 256 + (int)rank * 128;
+      const int row0 = mb * 256 + (int)rank * 128 + ew.quarter * 32;
+      const int n0 = nb * kPairBN + j0;
       const uint32_t b = t & 1, bph = (t >> 1) & 1;
-      if (SPLIT == 1 || ksplit == 0) stage_columns<kPairBN>(args, nb, lane, s_ws, s_bias);
-      const int row = row_base + quarter * 32 + lane;
-      const float as = row < args.M ? __ldg(args.a_scale + row) : 0.0f;
+      if (SPLIT == 1 || ksplit == 0) stage_columns<kCols>(args, n0, lane, s_ws, s_bias);
+      const float as = row0 + lane < args.M ? __ldg(args.a_scale + row0 + lane) : 0.0f;
       __syncwarp();
       int ok = 0;
       if (lane == 0) ok = mbar_wait(&tfull[b], bph, abort_flag, args.status);
       ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
       if (!ok) break;
       tc_fence_after();
-      const uint32_t taddr = tmem_base + b * kPairBN + ((uint32_t)(quarter * 32) << 16);
-      const int r = quarter * 32 + lane;  // row within this CTA's 128
+      const uint32_t taddr =
+          tmem_base + b * kPairBN + j0 + ((uint32_t)(ew.quarter * 32) << 16);
       if (SPLIT == 2 && ksplit == 1) {
         // Second pair: stage the int32 partial in this CTA's stage buffers
         // (all consumed: the producer waited for that) and ship it to the
         // first pair's CTA of the same rank once its buffers are free.
-#pragma unroll 1
-        for (int c = 0; c < kPairBN / 32; ++c) {
-          uint32_t v[32];
-          tmem_ld_32x32b_x32(taddr + c * 32, v);
-          tmem_ld_wait();
+        for_tmem_chunks<kCols / 32>(
+            taddr, [](int) { return true; },
+            [&](const uint32_t(&v)[32], int c) {
 #pragma unroll
-          for (int g = 0; g < 8; ++g)
-            *reinterpret_cast<uint4 *>(partial + partial_index(r, c * 32 + 4 * g)) =
-                make_uint4(v[4 * g], v[4 * g + 1], v[4 * g + 2], v[4 * g + 3]);
-        }
+              for (int g = 0; g < 8; ++g)
+                *reinterpret_cast<uint4 *>(partial + partial_index(r, j0 + c * 32 + 4 * g)) =
+                    make_uint4(v[4 * g], v[4 * g + 1], v[4 * g + 2], v[4 * g + 3]);
+            });
         fence_proxy_async_smem();
         __syncwarp();
-        asm volatile("bar.sync 1, 128;" ::: "memory");
-        if (et == 0) {
+        named_barrier_sync(1, 32 * kEpiWarps);
+        if (first_epi_thread) {
           if (mbar_wait(ready, 0, abort_flag, args.status)) {
             const uint32_t dst_cta = crank - 2;
             bulk_copy_s2cluster(map_to_cta(smem_addr(partial), dst_cta), partial, kPartialBytes,
@@ -301,7 +305,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (SPLIT == 2) {
           // First pair: every stage is consumed (tfull), so the stage buffers
           // may receive the partner pair's partial now.
-          if (et == 0) {
+          if (first_epi_thread) {
             mbar_arrive_expect_tx(recv, kPartialBytes);
             mbar_arrive_cluster(map_to_cta(smem_addr(ready), crank + 2));
           }
@@ -311,9 +315,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (!got) break;
         }
         // dequantise: (acc [+ partner partial]) * a_scale * w_scale + bias
-        epilogue_tile_tma<kPairBN>(args, &tmap_y, tmem_base + b * kPairBN, quarter, lane,
-                                   row_base, nb, as, s_ws, s_bias, s_out, out_count,
-                                   SPLIT == 2 ? partial : nullptr, PartialIndex());
+        epilogue_tma<kCols>(args, &tmap_y, taddr, lane, row0, n0, as, s_ws, s_bias, s_out,
+                            SPLIT == 2 ? partial : nullptr, PartialIndex{r, j0});
       }
       tc_fence_before();
       __syncwarp();
@@ -351,7 +354,7 @@ w8a8_status run_pair(const CUtensorMap &tq, const CUtensorMap &tw, const CUtenso
   const int clusters = SPLIT == 1 ? std::max(1, std::min(tiles, sm_count() / 2)) : tiles;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)(cta_per_cluster * clusters));
-  cfg.blockDim = dim3(kThreads);
+  cfg.blockDim = dim3(kGemmThreads);
   cfg.dynamicSmemBytes = (size_t)L::kAlloc;
   cfg.stream = stream;
   cudaLaunchAttribute attr[2];

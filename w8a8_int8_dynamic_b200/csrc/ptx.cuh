@@ -211,6 +211,21 @@ __device__ __forceinline__ void tmem_ld_wait() {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
 
+// The same wait, with the destination registers of the load it completes as
+// operands: no use of `r` can be scheduled above it (for loads issued ahead
+// of the computation on an earlier chunk).
+__device__ __forceinline__ void tmem_ld_wait_regs(uint32_t (&r)[32]) {
+  asm volatile("tcgen05.wait::ld.sync.aligned;"
+               : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]),
+                 "+r"(r[6]), "+r"(r[7]), "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]),
+                 "+r"(r[12]), "+r"(r[13]), "+r"(r[14]), "+r"(r[15]), "+r"(r[16]), "+r"(r[17]),
+                 "+r"(r[18]), "+r"(r[19]), "+r"(r[20]), "+r"(r[21]), "+r"(r[22]), "+r"(r[23]),
+                 "+r"(r[24]), "+r"(r[25]), "+r"(r[26]), "+r"(r[27]), "+r"(r[28]), "+r"(r[29]),
+                 "+r"(r[30]), "+r"(r[31])
+               :
+               : "memory");
+}
+
 // Shared-memory matrix descriptor for a K-major operand stored in the
 // 128-byte-swizzled canonical layout: 8-row x 128-byte swizzle atoms stacked
 // along M/N at a stride of 1024 bytes.  Fields: start address >> 4 (bits
@@ -323,6 +338,11 @@ __device__ __forceinline__ void bulk_copy_s2cluster(uint32_t dst_cluster, const 
 
 // Makes this thread's generic-proxy shared-memory writes visible to the async
 // proxy (bulk copies) issued after a following barrier.
+// Named barrier `id` among `threads` threads (a multiple of 32) of the block.
+__device__ __forceinline__ void named_barrier_sync(int id, int threads) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
+}
+
 __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
