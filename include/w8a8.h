@@ -166,11 +166,16 @@ w8a8_status w8a8_pack_weight_int32(const int32_t *w_i32, int64_t N, int64_t K,
  *   bias     device, bf16 [N], or NULL for no bias
  *   y        device, bf16 [M, N] (output)
  *   workspace device scratch of ws_bytes >= w8a8_scaled_mm_workspace_bytes,
- *            or NULL.  Only the small-M (decode) kernel uses it: int32 split-K
- *            partials and one counter per 128-row weight block.  With NULL,
- *            every M runs the large-M kernel.
- * Large M runs the persistent tcgen05 GEMM; M <= 16 with a workspace runs
- * the weight-streaming swap-AB kernel.  Both give bit-identical results. */
+ *            or NULL (16-byte aligned; contents on entry do not matter).  It
+ *            holds int32 K-split partials and call-tagged counters: for
+ *            M <= 16 those of the weight-streaming kernel; for problems with
+ *            too few 256 x 256 tiles to fill the GPU, those of the K-split
+ *            pair kernel (one 128 KB partial per 128 output rows of a tile).
+ *            The size query returns 0 when the chosen kernel needs none.
+ *            With NULL (or too small), M <= 16 and the K split fall back to
+ *            the large-M kernels without a split.
+ * All kernels give bit-identical results (the partials are summed exactly
+ * in int32 before the scale arithmetic). */
 w8a8_status w8a8_scaled_mm_workspace_bytes(int64_t M, int64_t N, int64_t K,
                                            size_t *bytes);
 w8a8_status w8a8_scaled_mm(const int8_t *q, const float *a_scale,
@@ -202,8 +207,10 @@ w8a8_status w8a8_scaled_mm_i32(const int8_t *q, const void *packed_w,
  * set-up overlaps the quantisation's tail.
  *   x         device, bf16 [M, K], row stride ldx
  *   workspace device, ws_bytes >= w8a8_linear_workspace_bytes(M, N, K); holds
- *             q and a_scale (and split-K partials for small M).  Its contents
- *             on entry do not matter.
+ *             q and a_scale, then the GEMM's workspace (see w8a8_scaled_mm).
+ *             Its contents on entry do not matter.  A smaller workspace that
+ *             still holds q, a_scale and, for M <= 16, the small-M partials
+ *             works too: the GEMM then runs without the K split.
  * N-D activations [..., K] are flattened by the caller to [M, K] and y is
  * viewed back as [..., N] (the "Diffusion Quantization Reference", GGUF
  * rules and the output-rank failure in "Common Failures"). */
@@ -232,7 +239,10 @@ w8a8_status w8a8_linear_act(const void *x, int64_t ldx, const void *packed_w,
  * to one scratch array of w8a8_linear_noalloc_max_bytes() bytes (8 MiB) that
  * every GPU loading this library holds until the process exits.  Nothing is
  * allocated.  Returns W8A8_ERR_BUFFER_TOO_SMALL, launching nothing, when
- * w8a8_linear_workspace_bytes(M, N, K) exceeds that size.  The first call on
+ * the codes, scales and small-M partials alone exceed that size (M * K plus
+ * 4 M bytes, each rounded up to 256, plus for M <= 16 the small-M kernel's
+ * partials); room left over serves the GEMM's K split, which is skipped
+ * when it does not fit.  The first call on
  * each device looks up the array's device address (make it before any stream
  * capture).  All calls on a device share the array: calls that overlap on the
  * GPU (different streams without ordering) race and corrupt each other. */

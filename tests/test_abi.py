@@ -97,8 +97,21 @@ def test_gemm_rejects_bad_arguments(L):
 
 
 def test_workspace_sizes(L):
+    """Host-side sizing (no GPU: the SM count falls back to the B200's 148).
+    The automatic choice never splits K for large M, so the GEMM needs no
+    workspace there; with the K-split pair kernel forced, 512 x 4096 x 4096
+    (32 tiles of 256 x 256) needs two 16-byte sync slots and one 128 KB int32
+    partial per 128 output rows of each tile.  Small M needs the split-K
+    partials of the weight-streaming kernel."""
     from w8a8_int8_dynamic_b200 import binding
-    ws = binding.linear_workspace_bytes(512, 4096, 4096)
-    assert ws >= 512 * 4096 + 512 * 4
     assert binding.scaled_mm_workspace_bytes(512, 4096, 4096) == 0
+    assert binding.linear_workspace_bytes(512, 4096, 4096) == 512 * 4096 + 2048
+    assert binding.linear_workspace_bytes(4096, 12288, 3072) == 4096 * 3072 + 4096 * 4
     assert binding.scaled_mm_workspace_bytes(16, 27648, 5120) > 0
+    assert L.w8a8_set_path(6) == 0
+    try:
+        split = 1024 + 64 * 128 * 1024
+        assert binding.scaled_mm_workspace_bytes(512, 4096, 4096) == split
+        assert binding.linear_workspace_bytes(512, 4096, 4096) == 512 * 4096 + 2048 + split
+    finally:
+        assert L.w8a8_set_path(0) == 0

@@ -162,6 +162,31 @@ def test_scaled_mm_matches_oracle(M, N, K, path, bias):
     assert np.array_equal(y_h, y_ref), "expected bit-exact bf16"
 
 
+@pytest.mark.parametrize("M,N,K", [(512, 1024, 4096), (300, 776, 2064), (512, 4096, 4096)])
+def test_k_split_pairs_with_garbage_workspace_repeated(M, N, K):
+    """The K-split pair kernel (two pairs per tile, one per half of K, the
+    first half's int32 partial handed over through the workspace).  The
+    workspace starts as random bytes and is reused by three calls; the
+    call-tagged counters must ignore every leftover, and each call must match
+    the oracle bit for bit."""
+    w8.set_path(w8.PATH_LARGE_PAIR_SPLIT)
+    assert "K split" in w8.gemm_kernel_name(M, N, K)
+    inp = random_case(M * 5 + N + K, M, N, K, bias=True, n_outliers=K // 64, zero_row=True)
+    q_ref, s_ref = oracle.quant_act(inp.x)
+    y_ref = oracle.epilogue(oracle.gemm_i32(q_ref, inp.w), s_ref, inp.w_scale, inp.bias)
+    need = w8.scaled_mm_workspace_bytes(M, N, K)
+    assert need > 0
+    ws = torch.randint(0, 256, (need,), dtype=torch.uint8, device="cuda")
+    args = (dev(q_ref), dev(s_ref), w8.pack_weight(dev(inp.w)), dev(inp.w_scale),
+            dev_bf16(inp.bias), N)
+    for _ in range(3):
+        y = w8.scaled_mm(*args, workspace=ws)
+        assert np.array_equal(host_u16(y), y_ref)
+    # without a workspace the same problem runs unsplit, with the same result
+    small = torch.empty((16,), dtype=torch.uint8, device="cuda")
+    assert np.array_equal(host_u16(w8.scaled_mm(*args, workspace=small)), y_ref)
+
+
 @pytest.mark.parametrize("path", [w8.PATH_LARGE_BN128, w8.PATH_LARGE_PAIR, w8.PATH_LARGE_PAIR128,
                                   w8.PATH_LARGE_PAIR_SPLIT])
 def test_scaled_mm_does_not_write_outside_y(path):

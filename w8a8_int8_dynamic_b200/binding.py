@@ -231,6 +231,10 @@ def scaled_mm(q: torch.Tensor, a_scale: torch.Tensor, packed_w: torch.Tensor,
     M, K = q.shape
     if out is None:
         out = torch.empty((M, N), dtype=torch.bfloat16, device=q.device)
+    if workspace is None:
+        need = scaled_mm_workspace_bytes(M, N, K)
+        if need:
+            workspace = torch.empty((need,), dtype=torch.uint8, device=q.device)
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     _check(lib().w8a8_scaled_mm_act(_ptr(q), _ptr(a_scale), _ptr(packed_w), _ptr(w_scale),
                                     _ptr(bias), _ptr(out), M, N, K, act, _ptr(workspace), ws_bytes,

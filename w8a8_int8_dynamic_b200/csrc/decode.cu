@@ -64,18 +64,6 @@ struct DecodeArgs {
   int *status;
 };
 
-// Counts this CTA's arrival on a slab counter and returns the count after it:
-// a word whose tag is not this call's counts as zero arrivals.
-__device__ __forceinline__ uint32_t arrive_tagged(unsigned long long *ctr, unsigned long long tag) {
-  unsigned long long cur = *reinterpret_cast<volatile unsigned long long *>(ctr);
-  while (true) {
-    const unsigned long long next = ((cur >> 8) == tag) ? cur + 1 : ((tag << 8) | 1ull);
-    const unsigned long long prev = atomicCAS(ctr, cur, next);
-    if (prev == cur) return (uint32_t)(next & 0xFF);
-    cur = prev;
-  }
-}
-
 __device__ __forceinline__ int64_t unit_begin(int64_t units, int grid, int c) {
   return units * c / grid;
 }
@@ -330,7 +318,6 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 bool g_decode_attr_done[64];
-std::atomic<unsigned long long> g_tag{0};
 
 int64_t units_of(int64_t N, int64_t K) {
   const int64_t nkb = packed_cols(K) / 128;
@@ -388,7 +375,7 @@ w8a8_status launch_decode(const int8_t *q, const float *a_scale, const void *pac
   a.max_contrib = mc;
   a.counters = reinterpret_cast<unsigned long long *>(ws);
   a.partials = reinterpret_cast<int32_t *>(ws + round_up(nb * 8, 256));
-  a.tag = (g_tag.fetch_add(1) + 1) & ((1ull << 56) - 1);
+  a.tag = next_call_tag();
   a.act = act;
   a.status = status_word();
   if (!a.status) return W8A8_ERR_CUDA;

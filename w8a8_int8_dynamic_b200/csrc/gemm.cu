@@ -319,14 +319,14 @@ enum class LargeKind { k128, k256, kPair, kPair128, kPairSplit };
 // SM from L2 (measured ~114 GB/s per SM with ~190 KB in flight) or by the
 // MMAs, whichever is slower: 1-SM 128x128: 64 KB / 512 cycles; 1-SM 128x256:
 // 96 KB / 1024; pair 256x256: 64 KB / 1024; pair 256x128: 48 KB / 512 per SM.
-LargeKind choose_large(int64_t M, int64_t N, int64_t K) {
+// `split_ok`: a workspace for the K-split pair kernel is available.
+LargeKind choose_large(int64_t M, int64_t N, int64_t K, bool split_ok) {
   const int path = forced_path();
   if (path == 3) return LargeKind::k128;
   if (path == 4) return LargeKind::k256;
   if (path == 5) return LargeKind::kPair;
-  if (path == 6) return LargeKind::kPairSplit;
+  if (path == 6) return split_ok ? LargeKind::kPairSplit : LargeKind::kPair;
   if (path == 7) return LargeKind::kPair128;
-  (void)K;
   const int64_t sms = sm_count(), pairs = sms / 2;
   const double feed_us_per_kb = 1.0 / 114e3;  // us per byte per SM
   const double l2_us_per_byte = 1.0 / 10.5e6;  // us per byte, whole chip
@@ -350,7 +350,13 @@ LargeKind choose_large(int64_t M, int64_t N, int64_t K) {
   const double cp128 = cost(tp128, pairs, 2, 49152, 512);
   // Few 256-wide pair tiles (half the GPU or less) but 128x128 tiles that fit
   // one wave: with cold operands, twice as many SMs pulling from DRAM wins
-  // (measured on 512 x 4096 x 4096: 16.6 us vs 19.1 us).
+  // (measured on 512 x 4096 x 4096: 16.6 us vs 19.1 us for 256x256 pairs).
+  // Splitting K over two pairs per tile halves the operand traffic but its
+  // int32 partial handoff (about 4 us for 128 KB per CTA through L2) costs
+  // more than it saves at these sizes (512 x 4096 x K, measured: 19.1 vs
+  // 14.3 us at K = 4096, even at K = 8192), so it is never chosen here.
+  (void)split_ok;
+  (void)K;
   if (tp256 * 2 <= pairs && t128 <= sms) return LargeKind::k128;
   double best = c128;
   LargeKind kind = LargeKind::k128;
@@ -368,7 +374,7 @@ LargeKind choose_large(int64_t M, int64_t N, int64_t K) {
 w8a8_status launch_scaled_mm(const int8_t *q, const float *a_scale, const void *packed_w,
                              const float *w_scale, const void *bias, void *out, bool out_i32,
                              int64_t M, int64_t N, int64_t K, cudaStream_t stream, bool pdl,
-                             int act) {
+                             int act, void *workspace, size_t ws_bytes) {
   CUtensorMap tmap;
   if (!make_tmap_u8_2d(&tmap, q, (uint64_t)M, (uint64_t)K, (uint64_t)K, kBM, kBK))
     return W8A8_ERR_CUDA;
@@ -391,13 +397,14 @@ w8a8_status launch_scaled_mm(const int8_t *q, const float *a_scale, const void *
     // the int32 export always uses the 1-SM kernel (tests and inspection); it
     // stores from registers and takes no output tensor map
     memset(&tmap_y, 0, sizeof(tmap_y));
-    const LargeKind kind = choose_large(M, N, K);
+    const LargeKind kind = choose_large(M, N, K, false);
     return kind == LargeKind::k128
                ? run_large<128, kLargeStages128, true>(tmap, tmap_y, a, stream, pdl, 1)
                : run_large<256, kLargeStages256, true>(tmap, tmap_y, a, stream, pdl, 0);
   }
   if (!make_tmap_out_bf16(&tmap_y, out, (uint64_t)M, (uint64_t)N)) return W8A8_ERR_CUDA;
-  switch (choose_large(M, N, K)) {
+  const bool split_ok = workspace && (int64_t)ws_bytes >= split_workspace_bytes(M, N);
+  switch (choose_large(M, N, K, split_ok)) {
     case LargeKind::kPair:
       return launch_gemm2sm(q, a_scale, packed_w, w_scale, bias, out, M, N, K, stream, pdl, 1, 256,
                             act);
@@ -406,12 +413,24 @@ w8a8_status launch_scaled_mm(const int8_t *q, const float *a_scale, const void *
                             act);
     case LargeKind::kPairSplit:
       return launch_gemm2sm(q, a_scale, packed_w, w_scale, bias, out, M, N, K, stream, pdl, 2, 256,
-                            act);
+                            act, workspace, ws_bytes);
     case LargeKind::k256:
       return run_large<256, kLargeStages256, false>(tmap, tmap_y, a, stream, pdl, 2);
     default:
       return run_large<128, kLargeStages128, false>(tmap, tmap_y, a, stream, pdl, 3);
   }
+}
+
+int64_t large_workspace_bytes(int64_t M, int64_t N, int64_t K) {
+  return choose_large(M, N, K, true) == LargeKind::kPairSplit ? split_workspace_bytes(M, N) : 0;
+}
+
+// Workspace w8a8_linear cannot do without: the codes, the scales and (small
+// M) the split-K partials of the weight-streaming kernel.
+int64_t linear_workspace_min(int64_t M, int64_t N, int64_t K) {
+  int64_t b = round_up(M * K, 256) + round_up(M * 4, 256);
+  if (M <= kDecodeNT) b += decode_workspace_bytes(N, K);
+  return b;
 }
 
 static w8a8_status check_gemm_args(const void *q, const void *packed_w, const void *out,
@@ -433,7 +452,7 @@ extern "C" {
 w8a8_status w8a8_scaled_mm_workspace_bytes(int64_t M, int64_t N, int64_t K, size_t *bytes) {
   if (!bytes || M < 1 || N < 1 || K < 1) return W8A8_ERR_INVALID_ARG;
   if (K % 16 != 0 || K > kMaxK || N % 8 != 0) return W8A8_ERR_UNSUPPORTED_SHAPE;
-  *bytes = M <= kDecodeNT ? (size_t)decode_workspace_bytes(N, K) : 0;
+  *bytes = (size_t)(M <= kDecodeNT ? decode_workspace_bytes(N, K) : large_workspace_bytes(M, N, K));
   return W8A8_OK;
 }
 
@@ -455,7 +474,9 @@ w8a8_status w8a8_scaled_mm_act(const int8_t *q, const float *a_scale, const void
                          act);
   }
   if (forced_path() == 2) return W8A8_ERR_INVALID_ARG;  // small path needs M <= 16 and a workspace
-  return launch_scaled_mm(q, a_scale, packed_w, w_scale, bias, y, false, M, N, K, s, false, act);
+  if (workspace && !aligned16(workspace)) return W8A8_ERR_ALIGNMENT;
+  return launch_scaled_mm(q, a_scale, packed_w, w_scale, bias, y, false, M, N, K, s, false, act,
+                          workspace, ws_bytes);
 }
 
 w8a8_status w8a8_scaled_mm(const int8_t *q, const float *a_scale, const void *packed_w,
@@ -468,7 +489,7 @@ w8a8_status w8a8_scaled_mm(const int8_t *q, const float *a_scale, const void *pa
 const char *w8a8_gemm_kernel_name(int64_t M, int64_t N, int64_t K) {
   if (M < 1 || N < 1 || K < 1) return "invalid";
   if (use_decode_path(M)) return "decode_kernel (swap-AB stream-K, needs a workspace)";
-  switch (choose_large(M, N, K)) {
+  switch (choose_large(M, N, K, true)) {
     case LargeKind::kPair: return "gemm2sm_kernel<256, 3, 1> (2-SM pair, 256x256 tiles)";
     case LargeKind::kPair128: return "gemm2sm_kernel<128, 4, 1> (2-SM pair, 256x128 tiles)";
     case LargeKind::kPairSplit: return "gemm2sm_kernel<256, 3, 2> (2-SM pairs, K split)";
@@ -488,8 +509,8 @@ w8a8_status w8a8_scaled_mm_i32(const int8_t *q, const void *packed_w, int32_t *a
 w8a8_status w8a8_linear_workspace_bytes(int64_t M, int64_t N, int64_t K, size_t *bytes) {
   if (!bytes || M < 1 || N < 1 || K < 1) return W8A8_ERR_INVALID_ARG;
   if (K % 16 != 0 || K > kMaxK || N % 8 != 0) return W8A8_ERR_UNSUPPORTED_SHAPE;
-  int64_t b = round_up(M * K, 256) + round_up(M * 4, 256);
-  if (M <= kDecodeNT) b += decode_workspace_bytes(N, K);
+  int64_t b = linear_workspace_min(M, N, K);
+  if (M > kDecodeNT) b += large_workspace_bytes(M, N, K);
   *bytes = (size_t)b;
   return W8A8_OK;
 }
@@ -506,10 +527,9 @@ w8a8_status w8a8_linear_act(const void *x, int64_t ldx, const void *packed_w,
   if (ldx % 8 != 0 || !aligned16(w_scale) || !aligned16(workspace) ||
       (bias && !aligned16(bias)))
     return W8A8_ERR_ALIGNMENT;
-  size_t need = 0;
-  st = w8a8_linear_workspace_bytes(M, N, K, &need);
-  if (st != W8A8_OK) return st;
-  if (ws_bytes < need) return W8A8_ERR_BUFFER_TOO_SMALL;
+  // Anything beyond the minimum may hold the K-split partials of the GEMM.
+  const int64_t need = linear_workspace_min(M, N, K);
+  if ((int64_t)ws_bytes < need) return W8A8_ERR_BUFFER_TOO_SMALL;
   uint8_t *ws = static_cast<uint8_t *>(workspace);
   int8_t *q = reinterpret_cast<int8_t *>(ws);
   float *a_scale = reinterpret_cast<float *>(ws + round_up(M * K, 256));
@@ -521,7 +541,9 @@ w8a8_status w8a8_linear_act(const void *x, int64_t ldx, const void *packed_w,
     return launch_decode(q, a_scale, packed_w, w_scale, bias, y, M, N, K, dws, s, true, act);
   }
   if (forced_path() == 2) return W8A8_ERR_INVALID_ARG;
-  return launch_scaled_mm(q, a_scale, packed_w, w_scale, bias, y, false, M, N, K, s, true, act);
+  const int64_t head = round_up(M * K, 256) + round_up(M * 4, 256);
+  return launch_scaled_mm(q, a_scale, packed_w, w_scale, bias, y, false, M, N, K, s, true, act,
+                          ws + head, ws_bytes - (size_t)head);
 }
 
 w8a8_status w8a8_linear(const void *x, int64_t ldx, const void *packed_w, const float *w_scale,

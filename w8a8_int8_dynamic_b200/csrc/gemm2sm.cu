@@ -20,11 +20,15 @@
 //   * both CTAs run the epilogue on their own 128 TMEM lanes.
 //
 // SPLIT = 1: persistent clusters of 2 CTAs, double-buffered accumulators.
-// SPLIT = 2: clusters of 4 CTAs = two pairs computing one tile over the two
-//   halves of K (for problems with too few tiles to fill the GPU).  The second
-//   pair writes its int32 partial into its own (then idle) stage buffers and
-//   ships it with one DSMEM bulk copy into the first pair's stage buffers; the
-//   first pair adds it -- exactly, in int32 -- before the scale arithmetic.
+// SPLIT = 2: (for problems with too few tiles to fill the GPU) every tile is
+//   computed by two pairs, one per half of K, one work item per pair.  Per
+//   (tile, CTA rank) a call-tagged counter in the workspace tells the two
+//   CTAs that hold the same 128 output rows which of them finished first: the
+//   first publishes its int32 partial to the workspace and raises a flag; the
+//   second waits for that flag (its partner is already past its main loop),
+//   bulk-copies the partial into its idle stage buffers and adds it -- exactly,
+//   in int32 -- before the scale arithmetic.  No CTA ever waits for one that
+//   may not have started.
 //
 // No TMA load uses cluster multicast.  Every wait is time-bounded (the waits
 // between the two pairs of a cluster are safe: a cluster's CTAs are
@@ -40,6 +44,7 @@ namespace {
 constexpr int kStageK = 2;                        // k-blocks per stage
 constexpr int kHalfStage = kStageK * kTileBytes;  // 32 KB: the q part of one stage
 constexpr int kPartialBytes = 128 * 256 * 4;      // one CTA's int32 partial (BN = 256): 128 KB
+constexpr int kPartialInts = kPartialBytes / 4;
 
 // BN = tile N of the pair (256 or 128); each CTA holds BN/2 weight rows.
 template <int BN, int STAGES>
@@ -53,9 +58,9 @@ struct PairSmem {
   static constexpr int kEpi = kB + STAGES * kBStage;
   static constexpr int kEpiEnd = kEpi + kEpiWarps * kEpiPerWarp;
   static constexpr int kOut = kEpiEnd + 1024 - kEpiEnd % 1024;
-  // full[S], empty[S], tfull[2], tempty[2], done, ready, recv
+  // full[S], empty[S], tfull[2], tempty[2], done, recv
   static constexpr int kBars = kOut + kEpiWarps * kEpiStagePerWarp;
-  static constexpr int kMisc = kBars + (2 * STAGES + 7) * 8;
+  static constexpr int kMisc = kBars + (2 * STAGES + 6) * 8;
   static constexpr int kUsed = kMisc + 16;
   static constexpr int kAlloc = kUsed + 1024;
   static_assert(BN != 256 || STAGES * (kHalfStage + kBStage) >= kPartialBytes,
@@ -94,16 +99,15 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   uint64_t *tfull = empty + STAGES;
   uint64_t *tempty = tfull + 2;
   uint64_t *mma_done = tempty + 2;
-  uint64_t *ready = mma_done + 1;  // (second pair) the first pair's buffers are free
-  uint64_t *recv = ready + 1;      // (first pair) the partial has arrived
+  uint64_t *recv = mma_done + 1;  // (SPLIT = 2) the partner's partial has arrived
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + L::kMisc);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + L::kMisc + 4);
+  volatile int *arrival = reinterpret_cast<volatile int *>(smem + L::kMisc + 8);
   int32_t *partial = reinterpret_cast<int32_t *>(smem);  // aliases the stage buffers
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t crank = cluster_ctarank();
   const uint32_t rank = crank & 1;      // 0: even CTA of the pair (issues the MMAs)
-  const uint32_t ksplit = crank >> 1;   // which K part this pair computes (SPLIT = 2)
   const uint32_t lead = crank & ~1u;    // cluster rank of this pair's even CTA
   // commit multicast masks are in cluster-rank space
   const uint16_t pair_mask = (uint16_t)(0x3u << lead);
@@ -118,7 +122,6 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       mbar_init(&tempty[b], 2 * kEpiWarps);  // the epilogue warps of both CTAs
     }
     mbar_init(mma_done, 1);
-    mbar_init(ready, 1);
     mbar_init(recv, 1);
     *abort_flag = 0;
     fence_barrier_init();
@@ -133,16 +136,20 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
 
-  const int num_tiles = args.tiles_m * args.tiles_n;  // 256 x 256 tiles
+  const int num_tiles = args.tiles_m * args.tiles_n;  // 256 x BN tiles
   const int num_kb = args.num_kb;
   const int stages_total = (num_kb + kStageK - 1) / kStageK;
-  // this pair's share of the K stages
-  const int st_begin = SPLIT == 1 ? 0 : (ksplit == 0 ? 0 : stages_total / 2);
-  const int st_end = SPLIT == 1 ? stages_total : (ksplit == 0 ? stages_total / 2 : stages_total);
+  const int slot = (int)(blockIdx.x >> 1);
+  const int nslots = (int)(gridDim.x >> 1);
+  // SPLIT = 2: one work item per pair, item = tile * 2 + K half
+  const int khalf = SPLIT == 2 ? (slot & 1) : 0;
+  const int st_begin = khalf == 0 ? 0 : stages_total / 2;
+  const int st_end = SPLIT == 1 ? stages_total : (khalf == 0 ? stages_total / 2 : stages_total);
   const int nst = st_end - st_begin;
-  const int slot = SPLIT == 1 ? (int)(blockIdx.x >> 1) : (int)(blockIdx.x >> 2);
-  const int nslots = SPLIT == 1 ? (int)(gridDim.x >> 1) : (int)(gridDim.x >> 2);
-  const int my_tiles = slot < num_tiles ? (num_tiles - 1 - slot) / nslots + 1 : 0;
+  const int my_tiles = SPLIT == 1
+                           ? (slot < num_tiles ? (num_tiles - 1 - slot) / nslots + 1 : 0)
+                           : (slot < 2 * num_tiles ? 1 : 0);
+  auto tile_of = [&](int t) { return SPLIT == 1 ? slot + t * nslots : slot >> 1; };
   const uint32_t my_iters = (uint32_t)my_tiles * nst;
   const uint32_t full0 = map_to_cta(smem_addr(full), lead);  // pair leader's full[0]
   const uint32_t tempty0 = map_to_cta(smem_addr(tempty), lead);
@@ -151,7 +158,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     if (lane == 0) {
       // ---------------- producer (every CTA) ----------------
       auto issue = [&](uint32_t it, uint32_t s, bool weights, bool acts) {
-        const int tile = slot + (int)(it / nst) * nslots;
+        const int tile = tile_of((int)(it / nst));
         const int mb = tile % args.tiles_m, nb = tile / args.tiles_m;
         const int kb0 = (st_begin + (int)(it % nst)) * kStageK;
         const int nk = min(kStageK, num_kb - kb0);
@@ -204,8 +211,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       }
       // Wait until every stage this CTA filled has been consumed: the MMA
       // commits that release them also arrive here, and must land before the
-      // CTA may leave (and, with SPLIT = 2, before the stage buffers are
-      // reused for the partial).
+      // CTA may leave.
       for (uint32_t s = 0; s < (uint32_t)STAGES && s < my_iters; ++s) {
         volatile int no_abort = 0;
         if (ok) (void)mbar_wait_bounded(&empty[s], last_par[s], &no_abort, args.status);
@@ -263,12 +269,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     const int r = ew.quarter * 32 + lane;  // row within this CTA's 128
     const int j0 = ew.half * kCols;        // first tile column of this warp
     for (int t = 0; t < my_tiles; ++t) {
-      const int tile = slot + t * nslots;
+      const int tile = tile_of(t);
       const int mb = tile % args.tiles_m, nb = tile / args.tiles_m;
       const int row0 = mb * 256 + (int)rank * 128 + ew.quarter * 32;
       const int n0 = nb * kPairBN + j0;
       const uint32_t b = t & 1, bph = (t >> 1) & 1;
-      if (SPLIT == 1 || ksplit == 0) stage_columns<kCols>(args, n0, lane, s_ws, s_bias);
+      stage_columns<kCols>(args, n0, lane, s_ws, s_bias);
       const float as = row0 + lane < args.M ? __ldg(args.a_scale + row0 + lane) : 0.0f;
       __syncwarp();
       int ok = 0;
@@ -278,45 +284,48 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       tc_fence_after();
       const uint32_t taddr =
           tmem_base + b * kPairBN + j0 + ((uint32_t)(ew.quarter * 32) << 16);
-      if (SPLIT == 2 && ksplit == 1) {
-        // Second pair: stage the int32 partial in this CTA's stage buffers
-        // (all consumed: the producer waited for that) and ship it to the
-        // first pair's CTA of the same rank once its buffers are free.
-        for_tmem_chunks<kCols / 32>(
-            taddr, [](int) { return true; },
-            [&](const uint32_t(&v)[32], int c) {
-#pragma unroll
-              for (int g = 0; g < 8; ++g)
-                *reinterpret_cast<uint4 *>(partial + partial_index(r, j0 + c * 32 + 4 * g)) =
-                    make_uint4(v[4 * g], v[4 * g + 1], v[4 * g + 2], v[4 * g + 3]);
-            });
-        fence_proxy_async_smem();
-        __syncwarp();
+      if (SPLIT == 2) {
+        // Which of the two K halves of these 128 rows finished first?
+        const int sidx = tile * 2 + (int)rank;
+        unsigned long long *ctr = args.sync + 2 * sidx;  // [0] arrivals, [1] published
+        int32_t *gpart = args.partials + (size_t)sidx * kPartialInts;
+        if (first_epi_thread) *arrival = (int)arrive_tagged(ctr, args.tag);
         named_barrier_sync(1, 32 * kEpiWarps);
-        if (first_epi_thread) {
-          if (mbar_wait(ready, 0, abort_flag, args.status)) {
-            const uint32_t dst_cta = crank - 2;
-            bulk_copy_s2cluster(map_to_cta(smem_addr(partial), dst_cta), partial, kPartialBytes,
-                                map_to_cta(smem_addr(recv), dst_cta));
-          }
-        }
-        __syncwarp();
-      } else {
-        if (SPLIT == 2) {
-          // First pair: every stage is consumed (tfull), so the stage buffers
-          // may receive the partner pair's partial now.
+        if (*arrival == 1) {
+          // First: publish the int32 partial (the layout of partial_index),
+          // then raise the flag once every epilogue thread's stores are out.
+          for_tmem_chunks<kCols / 32>(
+              taddr, [](int) { return true; },
+              [&](const uint32_t(&v)[32], int c) {
+#pragma unroll
+                for (int g = 0; g < 8; ++g)
+                  *reinterpret_cast<uint4 *>(gpart + partial_index(r, j0 + c * 32 + 4 * g)) =
+                      make_uint4(v[4 * g], v[4 * g + 1], v[4 * g + 2], v[4 * g + 3]);
+              });
+          __threadfence();
+          named_barrier_sync(1, 32 * kEpiWarps);
+          if (first_epi_thread) st_release_gpu(ctr + 1, args.tag);
+        } else {
+          // Second: the partner has arrived, so its partial is being or has
+          // been published; copy it into the idle stage buffers and finish.
           if (first_epi_thread) {
-            mbar_arrive_expect_tx(recv, kPartialBytes);
-            mbar_arrive_cluster(map_to_cta(smem_addr(ready), crank + 2));
+            if (flag_wait_bounded(ctr + 1, args.tag, abort_flag, args.status)) {
+              fence_proxy_async_global();
+              mbar_arrive_expect_tx(recv, kPartialBytes);
+              bulk_load(partial, gpart, kPartialBytes, recv);
+            }
           }
           int got = 0;
           if (lane == 0) got = mbar_wait(recv, 0, abort_flag, args.status);
           got = __shfl_sync(0xFFFFFFFFu, got, 0);
           if (!got) break;
+          epilogue_tma<kCols>(args, &tmap_y, taddr, lane, row0, n0, as, s_ws, s_bias, s_out,
+                              partial, PartialIndex{r, j0});
         }
-        // dequantise: (acc [+ partner partial]) * a_scale * w_scale + bias
+      } else {
+        // dequantise: acc * a_scale * w_scale + bias
         epilogue_tma<kCols>(args, &tmap_y, taddr, lane, row0, n0, as, s_ws, s_bias, s_out,
-                            SPLIT == 2 ? partial : nullptr, PartialIndex{r, j0});
+                            nullptr, PartialIndex{r, j0});
       }
       tc_fence_before();
       __syncwarp();
@@ -349,17 +358,17 @@ w8a8_status run_pair(const CUtensorMap &tq, const CUtensorMap &tw, const CUtenso
     if (d >= 0 && d < 64) g_pair_attr_done[d][slot_id] = true;
   }
   const int tiles = a.tiles_m * a.tiles_n;
-  const int cta_per_cluster = 2 * SPLIT;
-  // SPLIT = 1: persistent, one pair per two SMs; SPLIT = 2: one tile per cluster.
-  const int clusters = SPLIT == 1 ? std::max(1, std::min(tiles, sm_count() / 2)) : tiles;
+  // SPLIT = 1: persistent, one pair per two SMs; SPLIT = 2: one pair per
+  // (tile, K half).
+  const int pairs = SPLIT == 1 ? std::max(1, std::min(tiles, sm_count() / 2)) : 2 * tiles;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((unsigned)(cta_per_cluster * clusters));
+  cfg.gridDim = dim3((unsigned)(2 * pairs));
   cfg.blockDim = dim3(kGemmThreads);
   cfg.dynamicSmemBytes = (size_t)L::kAlloc;
   cfg.stream = stream;
   cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = (unsigned)cta_per_cluster;
+  attr[0].val.clusterDim.x = 2;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
   attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
@@ -376,10 +385,17 @@ w8a8_status run_pair(const CUtensorMap &tq, const CUtensorMap &tw, const CUtenso
 // Number of 256 x bn tiles the pair kernel would process.
 int64_t pair_tiles(int64_t M, int64_t N, int bn) { return ((M + 255) / 256) * ((N + bn - 1) / bn); }
 
+// Workspace of the K-split pair kernel: per (tile, CTA rank) two 8-byte sync
+// words, then one 128 KB int32 partial.
+int64_t split_workspace_bytes(int64_t M, int64_t N) {
+  const int64_t slots = 2 * pair_tiles(M, N, 256);
+  return round_up(slots * 16, 256) + slots * kPartialBytes;
+}
+
 w8a8_status launch_gemm2sm(const int8_t *q, const float *a_scale, const void *packed_w,
                            const float *w_scale, const void *bias, void *y, int64_t M, int64_t N,
                            int64_t K, cudaStream_t stream, bool pdl, int split, int bn,
-                           int act) {
+                           int act, void *workspace, size_t ws_bytes) {
   CUtensorMap tq, tw, ty;
   if (!make_tmap_u8_2d(&tq, q, (uint64_t)M, (uint64_t)K, (uint64_t)K, kBM, kBK))
     return W8A8_ERR_CUDA;
@@ -400,11 +416,21 @@ w8a8_status launch_gemm2sm(const int8_t *q, const float *a_scale, const void *pa
   a.tiles_n = (int)((N + bn - 1) / bn);
   a.act = act;
   a.status = status_word();
+  a.sync = nullptr;
+  a.partials = nullptr;
+  a.tag = 0;
   if (!a.status) return W8A8_ERR_CUDA;
   if (bn == 128) return run_pair<128, 4, 1>(tq, tw, ty, a, stream, pdl, 2);
-  // the split needs at least one stage per half
-  if (split == 2 && (a.num_kb + kStageK - 1) / kStageK >= 2)
+  // the split needs at least one stage per half and the workspace
+  if (split == 2 && (a.num_kb + kStageK - 1) / kStageK >= 2 && workspace &&
+      (int64_t)ws_bytes >= split_workspace_bytes(M, N)) {
+    const int64_t slots = 2 * pair_tiles(M, N, 256);
+    uint8_t *ws = static_cast<uint8_t *>(workspace);
+    a.sync = reinterpret_cast<unsigned long long *>(ws);
+    a.partials = reinterpret_cast<int32_t *>(ws + round_up(slots * 16, 256));
+    a.tag = next_call_tag();
     return run_pair<256, 3, 2>(tq, tw, ty, a, stream, pdl, 1);
+  }
   return run_pair<256, 3, 1>(tq, tw, ty, a, stream, pdl, 0);
 }
 

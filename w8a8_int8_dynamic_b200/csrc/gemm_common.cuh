@@ -36,6 +36,11 @@ struct GemmArgs {
   int tiles_m, tiles_n;
   int act;               // w8a8_act applied after the dequantisation
   int *status;
+  // K-split pair kernel only: per (tile, CTA rank) a call-tagged arrival
+  // counter and a "partial published" flag, and the published int32 partials
+  unsigned long long *sync;
+  int32_t *partials;
+  unsigned long long tag;
 };
 
 // Epilogue warp ew (0..7): TMEM lane quarter and which half of the columns.

@@ -25,6 +25,10 @@ void count_launch(int n = 1);
 // Path override set by w8a8_set_path: 0 auto, 1 large-M GEMM, 2 small-M.
 int forced_path();
 
+// A fresh 56-bit tag per call of a kernel that synchronises CTAs through
+// workspace words (so words left by earlier calls never need clearing).
+unsigned long long next_call_tag();
+
 // 2-D tiled tensor map over a row-major uint8 matrix [rows, cols] with row
 // stride ld bytes, box {box_cols, box_rows}, 128-byte swizzle, zero fill out
 // of bounds.  Returns false if the driver rejects it.
@@ -56,13 +60,22 @@ inline int64_t packed_cols(int64_t K) { return round_up(K, 128); }
 w8a8_status launch_scaled_mm(const int8_t *q, const float *a_scale, const void *packed_w,
                              const float *w_scale, const void *bias, void *out, bool out_i32,
                              int64_t M, int64_t N, int64_t K, cudaStream_t stream, bool pdl,
-                             int act = W8A8_ACT_NONE);
+                             int act = W8A8_ACT_NONE, void *workspace = nullptr,
+                             size_t ws_bytes = 0);
+// Workspace w8a8_scaled_mm can use for (M, N, K) with M above the small-M
+// range (0 when the chosen kernel needs none).
+int64_t large_workspace_bytes(int64_t M, int64_t N, int64_t K);
+// The part of w8a8_linear's workspace it cannot run without.
+int64_t linear_workspace_min(int64_t M, int64_t N, int64_t K);
 // 2-SM (CTA pair) GEMM with the bf16 epilogue (gemm2sm.cu).
 w8a8_status launch_gemm2sm(const int8_t *q, const float *a_scale, const void *packed_w,
                            const float *w_scale, const void *bias, void *y, int64_t M, int64_t N,
                            int64_t K, cudaStream_t stream, bool pdl, int split, int bn,
-                           int act = W8A8_ACT_NONE);
+                           int act = W8A8_ACT_NONE, void *workspace = nullptr,
+                           size_t ws_bytes = 0);
 int64_t pair_tiles(int64_t M, int64_t N, int bn);
+// Workspace the K-split pair kernel needs (sync words + int32 partials).
+int64_t split_workspace_bytes(int64_t M, int64_t N);
 // Small-M weight-streaming kernel (decode.cu).
 int64_t decode_workspace_bytes(int64_t N, int64_t K);
 bool use_decode_path(int64_t M);

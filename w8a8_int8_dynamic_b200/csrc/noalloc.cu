@@ -60,7 +60,10 @@ extern "C" w8a8_status w8a8_linear_noalloc(const void *x, int64_t ldx, const voi
   size_t need = 0;
   const w8a8_status st = w8a8_linear_workspace_bytes(M, N, K, &need);
   if (st != W8A8_OK) return st;
-  if (need > kNoAllocScratchBytes) return W8A8_ERR_BUFFER_TOO_SMALL;
+  // the layer runs in any workspace of at least the minimum; the rest of the
+  // scratch serves the GEMM's K-split partials when they fit
+  if (linear_workspace_min(M, N, K) > (int64_t)kNoAllocScratchBytes)
+    return W8A8_ERR_BUFFER_TOO_SMALL;
   void *scratch = nullptr;
   const w8a8_status sa = scratch_address(&scratch);
   if (sa != W8A8_OK) return sa;

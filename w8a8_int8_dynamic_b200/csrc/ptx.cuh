@@ -92,6 +92,57 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity,
   return mbar_wait_bounded(bar, parity, abort_flag, status);
 }
 
+// ---- flags in global memory between CTAs of one grid -------------------------
+__device__ __forceinline__ unsigned long long ld_acquire_gpu(const unsigned long long *p) {
+  unsigned long long v;
+  asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+  return v;
+}
+
+__device__ __forceinline__ void st_release_gpu(unsigned long long *p, unsigned long long v) {
+  asm volatile("st.release.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
+}
+
+// Waits until *flag == want (acquire).  Gives up like mbar_wait_bounded: on
+// *abort_flag, or after kWaitLimitNs (then sets *abort_flag and records
+// W8A8_ERR_TIMEOUT).  Only ever used to wait for a CTA that has already
+// announced itself running, so the wait is short unless something failed.
+static __device__ __noinline__ bool flag_wait_bounded(const unsigned long long *flag,
+                                                      unsigned long long want,
+                                                      volatile int *abort_flag, int *status) {
+  if (ld_acquire_gpu(flag) == want) return true;
+  const uint64_t t0 = global_timer_ns();
+  while (true) {
+    __nanosleep(64);
+    if (ld_acquire_gpu(flag) == want) return true;
+    if (*abort_flag) return false;
+    if (global_timer_ns() - t0 > kWaitLimitNs) {
+      *abort_flag = 1;
+      atomicExch(status, (int)W8A8_ERR_TIMEOUT);
+      return false;
+    }
+  }
+}
+
+// Counts this CTA's arrival on a call-tagged counter word ((tag << 8) |
+// arrivals) and returns the count after it; a word carrying another call's
+// tag counts as zero arrivals, so the words never need clearing.
+__device__ __forceinline__ uint32_t arrive_tagged(unsigned long long *ctr, unsigned long long tag) {
+  unsigned long long cur = *reinterpret_cast<volatile unsigned long long *>(ctr);
+  while (true) {
+    const unsigned long long next = ((cur >> 8) == tag) ? cur + 1 : ((tag << 8) | 1ull);
+    const unsigned long long prev = atomicCAS(ctr, cur, next);
+    if (prev == cur) return (uint32_t)(next & 0xFF);
+    cur = prev;
+  }
+}
+
+// Orders this thread's generic-proxy accesses to global memory before its
+// later async-proxy (bulk copy) accesses.
+__device__ __forceinline__ void fence_proxy_async_global() {
+  asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+
 // ---- TMA and bulk copies (global -> shared, completion on an mbarrier) ------
 __device__ __forceinline__ void prefetch_tmap(const CUtensorMap *map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");

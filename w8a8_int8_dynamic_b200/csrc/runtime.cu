@@ -19,6 +19,7 @@ int g_sm_count[kMaxDevices];
 std::mutex g_mu;
 std::atomic<int64_t> g_launches{0};
 std::atomic<int> g_forced_path{0};
+std::atomic<unsigned long long> g_call_tag{0};
 PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
 }  // namespace
 
@@ -56,6 +57,10 @@ int sm_count() {
 void count_launch(int n) { g_launches.fetch_add(n, std::memory_order_relaxed); }
 
 int forced_path() { return g_forced_path.load(std::memory_order_relaxed); }
+
+unsigned long long next_call_tag() {
+  return (g_call_tag.fetch_add(1, std::memory_order_relaxed) + 1) & ((1ull << 56) - 1);
+}
 
 static bool encode_u8_2d(CUtensorMap *map, const void *base, uint64_t rows, uint64_t cols,
                          uint64_t ld, uint32_t box_rows, uint32_t box_cols,
