@@ -53,6 +53,10 @@ def load_peaks():
             "source": "fallback"}
 
 
+# the sources the dominant kernel is compiled from (a change voids the record)
+TRAFFIC_SOURCES = ("gemm.cu", "gemm_common.cuh", "act.cuh", "ptx.cuh")
+
+
 def recorded_traffic(workload):
     """DRAM bytes per launch of the GEMM from the committed ncu capture, or
     None when there is none or the kernel sources changed since it was taken."""
@@ -65,7 +69,7 @@ def recorded_traffic(workload):
         return None
     csrc = os.path.join(HERE, "w8a8_int8_dynamic_b200", "csrc")
     h = hashlib.sha256()
-    for f in ("gemm.cu", "ptx.cuh"):
+    for f in TRAFFIC_SOURCES:
         h.update(open(os.path.join(csrc, f), "rb").read())
     if h.hexdigest()[:16] != rec.get("source_sha256_16"):
         return None
