@@ -257,8 +257,9 @@ w8a8_status w8a8_linear_noalloc(const void *x, int64_t ldx, const void *packed_w
  * tile width); 2 = the small-M weight-streaming kernel (M <= 16 only, else
  * W8A8_ERR_INVALID_ARG); 3 / 4 = the 1-SM large-M GEMM with 128- / 256-wide
  * output tiles; 5 = the 2-SM (CTA pair) GEMM with 256 x 256 tiles; 6 = the
- * same with K split over two pairs of a 4-CTA cluster (one tile per cluster);
- * 7 = the 2-SM GEMM with 256 x 128 tiles.
+ * same with K split over two pairs per tile, the first half's int32 partial
+ * handed over through the workspace (which w8a8_scaled_mm_workspace_bytes
+ * then sizes); 7 = the 2-SM GEMM with 256 x 128 tiles.
  * Process-wide; not synchronised with concurrent calls. */
 w8a8_status w8a8_set_path(int path);
 

@@ -271,6 +271,54 @@ def test_gelu_within_one_ulp():
     assert_bf16_close(host_u16(y), oracle.gelu_tanh(x), max_ulp=1, what="gelu")
 
 
+# ---------------------------------------------------------------- CUDA graph replay
+@pytest.mark.parametrize("case", ["layer", "decode_layer", "k_split"])
+def test_cuda_graph_replay_with_new_inputs(case):
+    """Kernels that count CTAs on call-tagged workspace words (the small-M
+    kernel's slab reduction, the K-split handoff) see the same tag on every
+    replay of a captured CUDA graph.  They must leave those words cleared:
+    capture one call, then replay it three times with new inputs copied into
+    the captured buffers, each replay checked against the oracle bit for bit
+    (the large-M layer, quantisation + GEMM, alongside)."""
+    M, N, K = {"layer": (512, 1024, 1024), "decode_layer": (4, 2056, 1040),
+               "k_split": (512, 1024, 4096)}[case]
+    if case == "k_split":
+        w8.set_path(w8.PATH_LARGE_PAIR_SPLIT)
+    inp = random_case(7, M, N, K, bias=True, n_outliers=K // 64)
+    packed = w8.pack_weight(dev(inp.w))
+    ws_s, b = dev(inp.w_scale), dev_bf16(inp.bias)
+    x = torch.empty((M, K), dtype=torch.bfloat16, device="cuda")
+    q = torch.empty((M, K), dtype=torch.int8, device="cuda")
+    a = torch.empty((M,), dtype=torch.float32, device="cuda")
+    y = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+    if case == "k_split":
+        ws = torch.empty((w8.scaled_mm_workspace_bytes(M, N, K),), dtype=torch.uint8, device="cuda")
+        call = lambda: w8.scaled_mm(q, a, packed, ws_s, b, N, out=y, workspace=ws)  # noqa: E731
+    else:
+        ws = torch.empty((w8.linear_workspace_bytes(M, N, K),), dtype=torch.uint8, device="cuda")
+        call = lambda: w8.linear(x, packed, ws_s, b, N, out=y, workspace=ws)  # noqa: E731
+    stream = torch.cuda.Stream()
+    with torch.cuda.stream(stream):
+        call()  # warm the launch path before capture
+        stream.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            call()
+    torch.cuda.synchronize()
+    for i in range(3):
+        xi = random_case(100 + i, M, N, K, bias=False, n_outliers=K // 64).x
+        y_ref, q_ref, s_ref, _ = oracle.linear(xi, inp.w, inp.w_scale, inp.bias)
+        x.copy_(dev_bf16(xi))
+        q.copy_(dev(q_ref))
+        a.copy_(dev(s_ref))
+        torch.cuda.synchronize()
+        g.replay()
+        torch.cuda.synchronize()
+        assert w8.poll_status() == 0
+        assert np.array_equal(host_u16(y), y_ref), f"replay {i}"
+    del g
+
+
 # ---------------------------------------------------------------- bounded waits
 def test_timeout_is_reported_and_context_survives():
     w8.selftest_wait_timeout(2_000_000)  # 2 ms

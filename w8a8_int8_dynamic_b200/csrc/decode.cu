@@ -272,8 +272,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         __threadfence();
         __syncwarp();
         asm volatile("bar.sync 1, 128;" ::: "memory");
-        if (et == 0)
-          *last_flag = arrive_tagged(args.counters + nb, args.tag) == (uint32_t)contributors ? 1 : 0;
+        if (et == 0) {
+          const bool last = arrive_tagged(args.counters + nb, args.tag) == (uint32_t)contributors;
+          // The last arrival of this call: nothing else touches the word in
+          // this launch, so clear it.  A replayed CUDA graph relaunches with
+          // the same tag and must find the count at zero, not at its total.
+          if (last) args.counters[nb] = 0ull;
+          *last_flag = last ? 1 : 0;
+        }
         __syncwarp();
         asm volatile("bar.sync 1, 128;" ::: "memory");
         finish = *last_flag != 0;

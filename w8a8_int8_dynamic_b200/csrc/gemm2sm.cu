@@ -319,6 +319,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           if (lane == 0) got = mbar_wait(recv, 0, abort_flag, args.status);
           got = __shfl_sync(0xFFFFFFFFu, got, 0);
           if (!got) break;
+          // Both CTAs are done with the two words for this call: clear them,
+          // so a replayed CUDA graph (same tag) starts from zero.
+          if (first_epi_thread) {
+            ctr[0] = 0ull;
+            ctr[1] = 0ull;
+          }
           epilogue_tma<kCols>(args, &tmap_y, taddr, lane, row0, n0, as, s_ws, s_bias, s_out,
                               partial, PartialIndex{r, j0});
         }

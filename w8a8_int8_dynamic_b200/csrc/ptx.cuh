@@ -125,14 +125,22 @@ static __device__ __noinline__ bool flag_wait_bounded(const unsigned long long *
 }
 
 // Counts this CTA's arrival on a call-tagged counter word ((tag << 8) |
-// arrivals) and returns the count after it; a word carrying another call's
-// tag counts as zero arrivals, so the words never need clearing.
+// arrivals, at most 255 arrivals per call) and returns the count after it; a
+// word carrying another call's tag (or cleared to 0) counts as zero arrivals,
+// so words left by earlier calls never need clearing.  Only the first arrival
+// on a stale word installs the tag with a compare-and-swap; every other one
+// is a single atomic add (many CTAs arriving together on one word would
+// otherwise retry their compare-and-swaps for microseconds).  Within a call
+// only this call's tag is ever written to the word until its last arrival.
 __device__ __forceinline__ uint32_t arrive_tagged(unsigned long long *ctr, unsigned long long tag) {
   unsigned long long cur = *reinterpret_cast<volatile unsigned long long *>(ctr);
   while (true) {
-    const unsigned long long next = ((cur >> 8) == tag) ? cur + 1 : ((tag << 8) | 1ull);
-    const unsigned long long prev = atomicCAS(ctr, cur, next);
-    if (prev == cur) return (uint32_t)(next & 0xFF);
+    if ((cur >> 8) == tag) {
+      const unsigned long long old = atomicAdd(ctr, 1ull);
+      return (uint32_t)((old & 0xFF) + 1);
+    }
+    const unsigned long long prev = atomicCAS(ctr, cur, (tag << 8) | 1ull);
+    if (prev == cur) return 1;
     cur = prev;
   }
 }

@@ -21,66 +21,19 @@
 // share an SM with it.  Rows longer than 65536 elements take a two-pass
 // kernel.  HBM-bound: 2 bytes read + 1 byte written per element.
 //
-// Exact quotient without a division: the code of x is rint(RN(x / s)).
-// RN(x / s) is formed from inv = RN(1/s) by reciprocal refinement (P. W.
-// Markstein, "Computation of elementary functions on the IBM RISC System/6000
-// processor", IBM J. Res. Dev. 34(1), 1990, Theorem 1: if y is 1/b rounded to
-// nearest and q is within one ulp of a/b, then r = a - b q is exact and
-// RN(q + r y) = RN(a/b)).  q0 = RN(x inv) is within 1.5 ulp of x / s, so one
-// refinement step first brings it within one ulp (q1 = RN(q0 + r0 inv) with
-// r0 = RN(x - s q0): |q1 - x/s| <= ulp/2 + 1.5 ulp * 2^-24), and a second
-// step, Markstein's, gives RN(x / s) exactly: 1 multiply + 4 FMAs per
-// element, no branch.  rint is then one addition (see kRound).  Rows with
-// s < 1e-30 (where 1/s could overflow) take the IEEE quotient.  |x| <= amax
-// makes |x / s| <= 127 (1 + 2^-23), so no clamp is needed.
+// The per-element arithmetic (the exact quotient by reciprocal refinement,
+// rint by one addition) is in quant_common.cuh, shared with the GEMM that
+// quantises its own rows.
 #include <cuda_bf16.h>
 
 #include <algorithm>
 
 #include "internal.h"
 #include "ptx.cuh"
+#include "quant_common.cuh"
 
 namespace w8a8 {
 namespace {
-
-__device__ __forceinline__ float bf16_lo(uint32_t v) { return __uint_as_float(v << 16); }
-__device__ __forceinline__ float bf16_hi(uint32_t v) { return __uint_as_float(v & 0xFFFF0000u); }
-
-// Code of one element: rint(RN(x / s)).  y = RN(x * inv) is within 2.3e-5 of
-// RN(x / s), so rint(y) is the answer unless y lies within 1e-4 of a
-// half-integer, i.e. |y - rint(y)| > 0.4999 (it is always <= 0.5); only then
-// is the IEEE quotient formed.  |x| <= amax makes |y| <= 127 (1 + 2^-22), so
-// the result is always in [-127, 127] and needs no clamp.
-// The IEEE quotient path, out of line: it runs rarely, and inlined at every
-// element of an unrolled row it would bloat the kernel past the instruction
-// cache.
-static __device__ __noinline__ int exact_code(float x, float s) {
-  return __float2int_rn(__fdiv_rn(x, s));
-}
-
-__device__ __forceinline__ int quant_one(float x, float s, float inv, bool exact_only) {
-  if (exact_only) return exact_code(x, s);
-  const float y = __fmul_rn(x, inv);
-  const float r = rintf(y);
-  if (fabsf(y - r) > 0.49997f) return exact_code(x, s);
-  return (int)r;
-}
-
-// Low bytes of four ints -> one word (byte permutes).
-// RN(x / s) from inv = RN(1/s) (Markstein refinement, see above).
-__device__ __forceinline__ float quotient_rn(float x, float s, float inv) {
-  const float q0 = __fmul_rn(x, inv);
-  const float r0 = __fmaf_rn(-s, q0, x);
-  const float q1 = __fmaf_rn(r0, inv, q0);
-  const float r1 = __fmaf_rn(-s, q1, x);
-  return __fmaf_rn(r1, inv, q1);
-}
-
-__device__ __forceinline__ uint32_t pack4(int a, int b, int c, int d) {
-  const uint32_t ab = __byte_perm((uint32_t)a, (uint32_t)b, 0x0040);
-  const uint32_t cd = __byte_perm((uint32_t)c, (uint32_t)d, 0x0040);
-  return __byte_perm(ab, cd, 0x5410);
-}
 
 // W warps per row, R rows per CTA (blockDim = 32 * W * R), CPL chunks per
 // lane.  Warp w of a row covers chunks [w * 32 * CPL, (w + 1) * 32 * CPL),
@@ -110,13 +63,8 @@ __global__ void __launch_bounds__(512) quant_warps_kernel(const uint16_t *__rest
   }
   uint32_t mx = 0;  // packed pair of 16-bit magnitudes
 #pragma unroll
-  for (int j = 0; j < CPL; ++j) {
-    mx = __vmaxu2(mx, v[j].x & 0x7FFF7FFFu);
-    mx = __vmaxu2(mx, v[j].y & 0x7FFF7FFFu);
-    mx = __vmaxu2(mx, v[j].z & 0x7FFF7FFFu);
-    mx = __vmaxu2(mx, v[j].w & 0x7FFF7FFFu);
-  }
-  uint32_t m = max(mx & 0xFFFFu, mx >> 16);
+  for (int j = 0; j < CPL; ++j) mx = absmax_chunk(mx, v[j]);
+  uint32_t m = absmax_fold(mx);
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
   if (W > 1) {
@@ -141,43 +89,13 @@ __global__ void __launch_bounds__(512) quant_warps_kernel(const uint16_t *__rest
   const float s = __fdiv_rn(amax, 127.0f);
   const float inv = __frcp_rn(s);
   if (w == 0 && lane == 0) a_scale[row] = s;
-  // Rounding: for |y| < 2^22, RN(y + 1.5 * 2^23) is 1.5 * 2^23 + rint(y)
-  // (round-half-even: the unit in the last place is 1 there), so its low
-  // byte is the two's-complement code: no conversion instruction needed.
-  constexpr float kRound = 12582912.0f;  // 1.5 * 2^23
   uint2 out[CPL];
   if (s >= 1e-30f) {
 #pragma unroll
-    for (int j = 0; j < CPL; ++j) {
-      const uint32_t e[4] = {v[j].x, v[j].y, v[j].z, v[j].w};
-      uint32_t code[8];
-#pragma unroll
-      for (int h = 0; h < 4; ++h) {
-        code[2 * h] = __float_as_uint(__fadd_rn(quotient_rn(bf16_lo(e[h]), s, inv), kRound));
-        code[2 * h + 1] = __float_as_uint(__fadd_rn(quotient_rn(bf16_hi(e[h]), s, inv), kRound));
-      }
-      out[j] = make_uint2(pack4((int)code[0], (int)code[1], (int)code[2], (int)code[3]),
-                          pack4((int)code[4], (int)code[5], (int)code[6], (int)code[7]));
-    }
+    for (int j = 0; j < CPL; ++j) out[j] = codes8(v[j], s, inv);
   } else {
-    // subnormal-scale rows: the IEEE quotient (rolled: a single copy of the
-    // division code)
 #pragma unroll
-    for (int j = 0; j < CPL; ++j) {
-      uint32_t o0 = 0, o1 = 0;
-#pragma unroll 1
-      for (int h = 0; h < 8; ++h) {
-        const uint32_t word = h < 2 ? v[j].x : h < 4 ? v[j].y : h < 6 ? v[j].z : v[j].w;
-        const float xv = (h & 1) ? bf16_hi(word) : bf16_lo(word);
-        const uint32_t code = (uint32_t)__float2int_rn(__fdiv_rn(xv, s)) & 0xFFu;
-        const int sh = (h & 3) * 8;
-        if (h < 4)
-          o0 |= code << sh;
-        else
-          o1 |= code << sh;
-      }
-      out[j] = make_uint2(o0, o1);
-    }
+    for (int j = 0; j < CPL; ++j) out[j] = codes8_ieee(v[j], s);
   }
 #pragma unroll
   for (int j = 0; j < CPL; ++j) {
@@ -198,12 +116,9 @@ __global__ void __launch_bounds__(1024) quant_rows_two_pass_kernel(
   uint32_t mx = 0;
   for (int i = threadIdx.x; i < nchunks; i += blockDim.x) {
     const uint4 c = *reinterpret_cast<const uint4 *>(xr + (int64_t)i * 8);
-    mx = __vmaxu2(mx, c.x & 0x7FFF7FFFu);
-    mx = __vmaxu2(mx, c.y & 0x7FFF7FFFu);
-    mx = __vmaxu2(mx, c.z & 0x7FFF7FFFu);
-    mx = __vmaxu2(mx, c.w & 0x7FFF7FFFu);
+    mx = absmax_chunk(mx, c);
   }
-  uint32_t m = max(mx & 0xFFFFu, mx >> 16);
+  uint32_t m = absmax_fold(mx);
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
   __shared__ uint32_t warp_max[32];
@@ -229,14 +144,7 @@ __global__ void __launch_bounds__(1024) quant_rows_two_pass_kernel(
     uint2 out = make_uint2(0, 0);
     if (amax != 0.0f) {
       const uint4 c = *reinterpret_cast<const uint4 *>(xr + (int64_t)i * 8);
-      out.x = pack4(quant_one(bf16_lo(c.x), s, inv, exact_only),
-                    quant_one(bf16_hi(c.x), s, inv, exact_only),
-                    quant_one(bf16_lo(c.y), s, inv, exact_only),
-                    quant_one(bf16_hi(c.y), s, inv, exact_only));
-      out.y = pack4(quant_one(bf16_lo(c.z), s, inv, exact_only),
-                    quant_one(bf16_hi(c.z), s, inv, exact_only),
-                    quant_one(bf16_lo(c.w), s, inv, exact_only),
-                    quant_one(bf16_hi(c.w), s, inv, exact_only));
+      out = exact_only ? codes8_ieee(c, s) : codes8(c, s, inv);
     }
     *reinterpret_cast<uint2 *>(qr + (int64_t)i * 8) = out;
   }
@@ -287,22 +195,22 @@ __global__ void __launch_bounds__(256) quant_static_kernel(const uint16_t *__res
       const uint16_t *src = x + m * ldx + k;
       const uint4 a = ld_stream_u4(src);
       const uint4 b = ld_stream_u4(src + 8);
-      out.x = pack4(quant_static_one(bf16_lo(a.x), s, inv, exact_only),
-                    quant_static_one(bf16_hi(a.x), s, inv, exact_only),
-                    quant_static_one(bf16_lo(a.y), s, inv, exact_only),
-                    quant_static_one(bf16_hi(a.y), s, inv, exact_only));
-      out.y = pack4(quant_static_one(bf16_lo(a.z), s, inv, exact_only),
-                    quant_static_one(bf16_hi(a.z), s, inv, exact_only),
-                    quant_static_one(bf16_lo(a.w), s, inv, exact_only),
-                    quant_static_one(bf16_hi(a.w), s, inv, exact_only));
-      out.z = pack4(quant_static_one(bf16_lo(b.x), s, inv, exact_only),
-                    quant_static_one(bf16_hi(b.x), s, inv, exact_only),
-                    quant_static_one(bf16_lo(b.y), s, inv, exact_only),
-                    quant_static_one(bf16_hi(b.y), s, inv, exact_only));
-      out.w = pack4(quant_static_one(bf16_lo(b.z), s, inv, exact_only),
-                    quant_static_one(bf16_hi(b.z), s, inv, exact_only),
-                    quant_static_one(bf16_lo(b.w), s, inv, exact_only),
-                    quant_static_one(bf16_hi(b.w), s, inv, exact_only));
+      out.x = pack4((uint32_t)quant_static_one(bf16_lo(a.x), s, inv, exact_only),
+                    (uint32_t)quant_static_one(bf16_hi(a.x), s, inv, exact_only),
+                    (uint32_t)quant_static_one(bf16_lo(a.y), s, inv, exact_only),
+                    (uint32_t)quant_static_one(bf16_hi(a.y), s, inv, exact_only));
+      out.y = pack4((uint32_t)quant_static_one(bf16_lo(a.z), s, inv, exact_only),
+                    (uint32_t)quant_static_one(bf16_hi(a.z), s, inv, exact_only),
+                    (uint32_t)quant_static_one(bf16_lo(a.w), s, inv, exact_only),
+                    (uint32_t)quant_static_one(bf16_hi(a.w), s, inv, exact_only));
+      out.z = pack4((uint32_t)quant_static_one(bf16_lo(b.x), s, inv, exact_only),
+                    (uint32_t)quant_static_one(bf16_hi(b.x), s, inv, exact_only),
+                    (uint32_t)quant_static_one(bf16_lo(b.y), s, inv, exact_only),
+                    (uint32_t)quant_static_one(bf16_hi(b.y), s, inv, exact_only));
+      out.w = pack4((uint32_t)quant_static_one(bf16_lo(b.z), s, inv, exact_only),
+                    (uint32_t)quant_static_one(bf16_hi(b.z), s, inv, exact_only),
+                    (uint32_t)quant_static_one(bf16_lo(b.w), s, inv, exact_only),
+                    (uint32_t)quant_static_one(bf16_hi(b.w), s, inv, exact_only));
     }
     *reinterpret_cast<uint4 *>(q + m * K + k) = out;
   }

@@ -1,0 +1,92 @@
+// quant_common.cuh -- the per-element arithmetic of the dynamic per-token
+// activation quantisation ("Issue 5 probe: int8 quantized DiT serve paths on
+// the RTX 3090", Round two: dynamic per-token symmetric int8 activations),
+// shared by the standalone kernel (quant.cu) and the GEMM that quantises its
+// own input rows (gemm.cu).
+//
+// Per row: amax = max |x|, s = RN(amax / 127), code = rint_half_even(RN(x / s)).
+//
+// Exact quotient without a division.  RN(x / s) is formed from inv = RN(1/s)
+// by reciprocal refinement (P. W. Markstein, "Computation of elementary
+// functions on the IBM RISC System/6000 processor", IBM J. Res. Dev. 34(1),
+// 1990, Theorem 1: if y is 1/b rounded to nearest and q is within one ulp of
+// a/b, then r = a - b q is exact and RN(q + r y) = RN(a/b)).  q0 = RN(x inv)
+// is within 1.5 ulp of x / s, so one refinement step first brings it within
+// one ulp (q1 = RN(q0 + r0 inv), r0 = RN(x - s q0): |q1 - x/s| <= ulp/2 +
+// 1.5 ulp * 2^-24), and a second step, Markstein's, gives RN(x / s) exactly:
+// one multiply and four FMAs per element, no branch.  Valid for s >= 1e-30
+// (1/s finite and normal); smaller scales take the IEEE quotient.  |x| <= amax
+// makes |x / s| <= 127 (1 + 2^-23), so no clamp is needed.
+//
+// rint without a conversion: for |y| < 2^22, RN(y + 1.5 * 2^23) is
+// 1.5 * 2^23 + rint(y) (round-half-even, the unit in the last place being 1
+// there), so the low byte of its bit pattern is the two's-complement code.
+#pragma once
+
+#include <stdint.h>
+
+namespace w8a8 {
+
+__device__ __forceinline__ float bf16_lo(uint32_t v) { return __uint_as_float(v << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t v) { return __uint_as_float(v & 0xFFFF0000u); }
+
+// Running maximum of the bf16 magnitudes of one 16-byte chunk, as two packed
+// 16-bit lanes (for finite bf16, |x| order is the order of the 15 low bits).
+__device__ __forceinline__ uint32_t absmax_chunk(uint32_t m, const uint4 &v) {
+  m = __vmaxu2(m, v.x & 0x7FFF7FFFu);
+  m = __vmaxu2(m, v.y & 0x7FFF7FFFu);
+  m = __vmaxu2(m, v.z & 0x7FFF7FFFu);
+  return __vmaxu2(m, v.w & 0x7FFF7FFFu);
+}
+
+// The two packed lanes of absmax_chunk -> one magnitude's bit pattern.
+__device__ __forceinline__ uint32_t absmax_fold(uint32_t m) { return max(m & 0xFFFFu, m >> 16); }
+
+// RN(x / s) from inv = RN(1/s) (reciprocal refinement, see above).
+__device__ __forceinline__ float quotient_rn(float x, float s, float inv) {
+  const float q0 = __fmul_rn(x, inv);
+  const float r0 = __fmaf_rn(-s, q0, x);
+  const float q1 = __fmaf_rn(r0, inv, q0);
+  const float r1 = __fmaf_rn(-s, q1, x);
+  return __fmaf_rn(r1, inv, q1);
+}
+
+// Low bytes of four ints -> one word.
+__device__ __forceinline__ uint32_t pack4(uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+  const uint32_t ab = __byte_perm(a, b, 0x0040);
+  const uint32_t cd = __byte_perm(c, d, 0x0040);
+  return __byte_perm(ab, cd, 0x5410);
+}
+
+constexpr float kRound = 12582912.0f;  // 1.5 * 2^23
+
+__device__ __forceinline__ uint32_t code_bits(float x, float s, float inv) {
+  return __float_as_uint(__fadd_rn(quotient_rn(x, s, inv), kRound));
+}
+
+// One 16-byte chunk (8 bf16) -> its 8 codes, for s >= 1e-30.
+__device__ __forceinline__ uint2 codes8(const uint4 &v, float s, float inv) {
+  return make_uint2(pack4(code_bits(bf16_lo(v.x), s, inv), code_bits(bf16_hi(v.x), s, inv),
+                          code_bits(bf16_lo(v.y), s, inv), code_bits(bf16_hi(v.y), s, inv)),
+                    pack4(code_bits(bf16_lo(v.z), s, inv), code_bits(bf16_hi(v.z), s, inv),
+                          code_bits(bf16_lo(v.w), s, inv), code_bits(bf16_hi(v.w), s, inv)));
+}
+
+// The same with the IEEE quotient (rows with s < 1e-30).  A rolled loop keeps
+// a single copy of the division code.
+__device__ __forceinline__ uint2 codes8_ieee(const uint4 &v, float s) {
+  uint32_t o0 = 0, o1 = 0;
+#pragma unroll 1
+  for (int h = 0; h < 8; ++h) {
+    const uint32_t word = h < 2 ? v.x : h < 4 ? v.y : h < 6 ? v.z : v.w;
+    const float xv = (h & 1) ? bf16_hi(word) : bf16_lo(word);
+    const uint32_t code = (uint32_t)__float2int_rn(__fdiv_rn(xv, s)) & 0xFFu;
+    if (h < 4)
+      o0 |= code << ((h & 3) * 8);
+    else
+      o1 |= code << ((h & 3) * 8);
+  }
+  return make_uint2(o0, o1);
+}
+
+}  // namespace w8a8
