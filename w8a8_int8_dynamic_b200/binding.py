@@ -268,9 +268,9 @@ def linear(x: torch.Tensor, packed_w: torch.Tensor, w_scale: torch.Tensor,
     M = x2.shape[0]
     if out is None:
         out = torch.empty((M, N), dtype=torch.bfloat16, device=x.device)
-    need = linear_workspace_bytes(M, N, K)
     if workspace is None:
-        workspace = torch.empty((need,), dtype=torch.uint8, device=x.device)
+        workspace = torch.empty((linear_workspace_bytes(M, N, K),), dtype=torch.uint8,
+                                device=x.device)
     ws_bytes = workspace.numel() * workspace.element_size()
     _check(lib().w8a8_linear_act(_ptr(x2), x2.stride(0), _ptr(packed_w), _ptr(w_scale), _ptr(bias),
                                  _ptr(out), M, N, K, act, _ptr(workspace), ws_bytes,
