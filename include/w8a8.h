@@ -259,7 +259,12 @@ w8a8_status w8a8_linear_noalloc(const void *x, int64_t ldx, const void *packed_w
  * output tiles; 5 = the 2-SM (CTA pair) GEMM with 256 x 256 tiles; 6 = the
  * same with K split over two pairs per tile, the first half's int32 partial
  * handed over through the workspace (which w8a8_scaled_mm_workspace_bytes
- * then sizes); 7 = the 2-SM GEMM with 256 x 128 tiles.
+ * then sizes); 7 = the 2-SM GEMM with 256 x 128 tiles; 8 = the 256 x 256
+ * 2-SM GEMM with stream-K: the tiles' k-blocks cut into equal contiguous
+ * ranges, one per SM pair, tiles split between two pairs summing their int32
+ * partials through the workspace (chosen automatically, given the workspace,
+ * when the tiles outnumber the SM pairs and the last wave would leave pairs
+ * idle).
  * Process-wide; not synchronised with concurrent calls. */
 w8a8_status w8a8_set_path(int path);
 

@@ -146,9 +146,10 @@ def test_gemm_i32_extreme_values():
 
 @pytest.mark.parametrize("bias", [False, True])
 @pytest.mark.parametrize("path", [w8.PATH_LARGE_BN128, w8.PATH_LARGE_BN256, w8.PATH_LARGE_PAIR,
-                                  w8.PATH_LARGE_PAIR128, w8.PATH_LARGE_PAIR_SPLIT])
+                                  w8.PATH_LARGE_PAIR128, w8.PATH_LARGE_PAIR_SPLIT,
+                                  w8.PATH_LARGE_PAIR_STREAMK])
 @pytest.mark.parametrize("M,N,K", [(64, 128, 256), (129, 392, 400), (300, 1000, 528), (512, 1024, 4096),
-                                   (257, 264, 272), (700, 520, 144)])
+                                   (257, 264, 272), (700, 520, 144), (1000, 2056, 1040)])
 def test_scaled_mm_matches_oracle(M, N, K, path, bias):
     w8.set_path(path)
     inp = random_case(M + N + K, M, N, K, bias=bias, n_outliers=K // 64, zero_row=True)
@@ -188,7 +189,7 @@ def test_k_split_pairs_with_garbage_workspace_repeated(M, N, K):
 
 
 @pytest.mark.parametrize("path", [w8.PATH_LARGE_BN128, w8.PATH_LARGE_PAIR, w8.PATH_LARGE_PAIR128,
-                                  w8.PATH_LARGE_PAIR_SPLIT])
+                                  w8.PATH_LARGE_PAIR_SPLIT, w8.PATH_LARGE_PAIR_STREAMK])
 def test_scaled_mm_does_not_write_outside_y(path):
     w8.set_path(path)
     M, N, K = 130, 264, 272
@@ -272,7 +273,7 @@ def test_gelu_within_one_ulp():
 
 
 # ---------------------------------------------------------------- CUDA graph replay
-@pytest.mark.parametrize("case", ["layer", "decode_layer", "k_split"])
+@pytest.mark.parametrize("case", ["layer", "decode_layer", "k_split", "stream_k"])
 def test_cuda_graph_replay_with_new_inputs(case):
     """Kernels that count CTAs on call-tagged workspace words (the small-M
     kernel's slab reduction, the K-split handoff) see the same tag on every
@@ -281,9 +282,11 @@ def test_cuda_graph_replay_with_new_inputs(case):
     the captured buffers, each replay checked against the oracle bit for bit
     (the large-M layer, quantisation + GEMM, alongside)."""
     M, N, K = {"layer": (512, 1024, 1024), "decode_layer": (4, 2056, 1040),
-               "k_split": (512, 1024, 4096)}[case]
+               "k_split": (512, 1024, 4096), "stream_k": (1000, 2056, 1040)}[case]
     if case == "k_split":
         w8.set_path(w8.PATH_LARGE_PAIR_SPLIT)
+    if case == "stream_k":
+        w8.set_path(w8.PATH_LARGE_PAIR_STREAMK)
     inp = random_case(7, M, N, K, bias=True, n_outliers=K // 64)
     packed = w8.pack_weight(dev(inp.w))
     ws_s, b = dev(inp.w_scale), dev_bf16(inp.bias)
@@ -291,7 +294,7 @@ def test_cuda_graph_replay_with_new_inputs(case):
     q = torch.empty((M, K), dtype=torch.int8, device="cuda")
     a = torch.empty((M,), dtype=torch.float32, device="cuda")
     y = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
-    if case == "k_split":
+    if case in ("k_split", "stream_k"):
         ws = torch.empty((w8.scaled_mm_workspace_bytes(M, N, K),), dtype=torch.uint8, device="cuda")
         call = lambda: w8.scaled_mm(q, a, packed, ws_s, b, N, out=y, workspace=ws)  # noqa: E731
     else:

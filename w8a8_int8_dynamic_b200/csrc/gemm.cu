@@ -240,7 +240,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         epilogue_i32<kCols>(args, taddr, row0 + lane, n0);
       else
         epilogue_tma<kCols>(args, &tmap_y, taddr, lane, row0, n0, as, s_ws, s_bias, s_out,
-                            nullptr, NoExtra());
+                            false, NoExtra());
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&tempty[b]);
@@ -312,7 +312,7 @@ w8a8_status run_large(const CUtensorMap &tmap, const CUtensorMap &tmap_y, GemmAr
 // ~128 B/clk per SM, the 128 x 256 tile ~94, the 2-SM 256 x 256 tile ~64),
 // so the cost of a shape is its wave count times its per-SM tile work divided
 // by the fraction of the rate it sustains.
-enum class LargeKind { k128, k256, kPair, kPair128, kPairSplit };
+enum class LargeKind { k128, k256, kPair, kPair128, kPairSplit, kPairStreamK };
 
 // Kernel choice for large M: (waves of tiles) x (per-SM time of one tile).
 // The per-SM time of a stage of two k-blocks is set by what has to reach the
@@ -327,6 +327,7 @@ LargeKind choose_large(int64_t M, int64_t N, int64_t K, bool split_ok) {
   if (path == 5) return LargeKind::kPair;
   if (path == 6) return split_ok ? LargeKind::kPairSplit : LargeKind::kPair;
   if (path == 7) return LargeKind::kPair128;
+  if (path == 8) return split_ok ? LargeKind::kPairStreamK : LargeKind::kPair;
   const int64_t sms = sm_count(), pairs = sms / 2;
   const double feed_us_per_kb = 1.0 / 114e3;  // us per byte per SM
   const double l2_us_per_byte = 1.0 / 10.5e6;  // us per byte, whole chip
@@ -363,6 +364,11 @@ LargeKind choose_large(int64_t M, int64_t N, int64_t K, bool split_ok) {
   if (c256 < best) best = c256, kind = LargeKind::k256;
   if (cp256 <= best) best = cp256, kind = LargeKind::kPair;
   if (cp128 < best * 0.97) best = cp128, kind = LargeKind::kPair128;
+  // Stream-K (equal k-block ranges per SM pair, path 8) is not chosen: these
+  // kernels are bound by L2 -> SM delivery, so a last wave with few busy pairs
+  // runs each of them faster and costs little, while stream-K's int32
+  // partials add about a fifth to the L2 traffic (measured on 512 x 12288 x
+  // 4096: 35.3 us against 31.8 us with whole tiles).
   // The K-split pair variant exchanges a 128 KB partial per CTA over DSMEM
   // (measured ~5 us): it does not pay on the shapes at hand and is never
   // chosen automatically.
@@ -403,7 +409,10 @@ w8a8_status launch_scaled_mm(const int8_t *q, const float *a_scale, const void *
                : run_large<256, kLargeStages256, true>(tmap, tmap_y, a, stream, pdl, 0);
   }
   if (!make_tmap_out_bf16(&tmap_y, out, (uint64_t)M, (uint64_t)N)) return W8A8_ERR_CUDA;
-  const bool split_ok = workspace && (int64_t)ws_bytes >= split_workspace_bytes(M, N);
+  // enough workspace for the K split / stream-K (both partial layouts)
+  const bool split_ok =
+      workspace && (int64_t)ws_bytes >= std::min(split_workspace_bytes(M, N, 2),
+                                                  split_workspace_bytes(M, N, 3));
   switch (choose_large(M, N, K, split_ok)) {
     case LargeKind::kPair:
       return launch_gemm2sm(q, a_scale, packed_w, w_scale, bias, out, M, N, K, stream, pdl, 1, 256,
@@ -414,6 +423,9 @@ w8a8_status launch_scaled_mm(const int8_t *q, const float *a_scale, const void *
     case LargeKind::kPairSplit:
       return launch_gemm2sm(q, a_scale, packed_w, w_scale, bias, out, M, N, K, stream, pdl, 2, 256,
                             act, workspace, ws_bytes);
+    case LargeKind::kPairStreamK:
+      return launch_gemm2sm(q, a_scale, packed_w, w_scale, bias, out, M, N, K, stream, pdl, 3, 256,
+                            act, workspace, ws_bytes);
     case LargeKind::k256:
       return run_large<256, kLargeStages256, false>(tmap, tmap_y, a, stream, pdl, 2);
     default:
@@ -422,7 +434,10 @@ w8a8_status launch_scaled_mm(const int8_t *q, const float *a_scale, const void *
 }
 
 int64_t large_workspace_bytes(int64_t M, int64_t N, int64_t K) {
-  return choose_large(M, N, K, true) == LargeKind::kPairSplit ? split_workspace_bytes(M, N) : 0;
+  const LargeKind kind = choose_large(M, N, K, true);
+  return kind == LargeKind::kPairSplit    ? split_workspace_bytes(M, N, 2)
+         : kind == LargeKind::kPairStreamK ? split_workspace_bytes(M, N, 3)
+                                           : 0;
 }
 
 // Workspace w8a8_linear cannot do without: the codes, the scales and (small
@@ -493,6 +508,8 @@ const char *w8a8_gemm_kernel_name(int64_t M, int64_t N, int64_t K) {
     case LargeKind::kPair: return "gemm2sm_kernel<256, 3, 1> (2-SM pair, 256x256 tiles)";
     case LargeKind::kPair128: return "gemm2sm_kernel<128, 4, 1> (2-SM pair, 256x128 tiles)";
     case LargeKind::kPairSplit: return "gemm2sm_kernel<256, 3, 2> (2-SM pairs, K split)";
+    case LargeKind::kPairStreamK:
+      return "gemm2sm_kernel<256, 3, 3> (2-SM pairs, 256x256 tiles, stream-K)";
     case LargeKind::k256: return "gemm_kernel<256, 4, 1> (1-SM, 128x256 tiles)";
     default: return "gemm_kernel<128, 3, 2> (1-SM, 128x128 tiles, 2 k-blocks per stage)";
   }

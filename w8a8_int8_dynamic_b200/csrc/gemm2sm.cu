@@ -71,11 +71,17 @@ struct PairSmem {
 // ((j / 4) * 128 + r) * 4 + j % 4, so the 32 lanes (rows) of a warp move 512
 // contiguous bytes per 16-byte access.
 __device__ __forceinline__ int partial_index(int r, int j) { return ((j >> 2) * 128 + r) * 4 + (j & 3); }
-// Partial element of row r for column j0 + j (the epilogue's column index j
-// counts from the warp's first column j0).
-struct PartialIndex {
+// Four partial values of row r at columns j0 + j .. j0 + j + 3 (the
+// epilogue's column index j counts from the warp's first column j0), from
+// shared memory or, bypassing L1, from the workspace in global memory.
+struct PartialLoad {
+  const int32_t *p;
   int r, j0;
-  __device__ int operator()(int j) const { return partial_index(r, j0 + j); }
+  bool global;
+  __device__ uint4 operator()(int j) const {
+    const uint4 *q = reinterpret_cast<const uint4 *>(p + partial_index(r, j0 + j));
+    return global ? __ldcg(q) : *q;
+  }
 };
 
 template <int BN, int STAGES, int SPLIT>
@@ -88,6 +94,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   constexpr uint32_t kTmemCols = 2 * BN;
   constexpr uint32_t kIdesc = idesc_i8(256, BN);
   static_assert(SPLIT == 1 || BN == 256, "the K split is built for 256-wide tiles");
+  static_assert(SPLIT >= 1 && SPLIT <= 3, "1: whole tiles, 2: K halves, 3: stream-K");
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>(
@@ -138,29 +145,53 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 
   const int num_tiles = args.tiles_m * args.tiles_n;  // 256 x BN tiles
   const int num_kb = args.num_kb;
-  const int stages_total = (num_kb + kStageK - 1) / kStageK;
+  const int S = (num_kb + kStageK - 1) / kStageK;  // stages per tile
   const int slot = (int)(blockIdx.x >> 1);
   const int nslots = (int)(gridDim.x >> 1);
-  // SPLIT = 2: one work item per pair, item = tile * 2 + K half
-  const int khalf = SPLIT == 2 ? (slot & 1) : 0;
-  const int st_begin = khalf == 0 ? 0 : stages_total / 2;
-  const int st_end = SPLIT == 1 ? stages_total : (khalf == 0 ? stages_total / 2 : stages_total);
-  const int nst = st_end - st_begin;
-  const int my_tiles = SPLIT == 1
-                           ? (slot < num_tiles ? (num_tiles - 1 - slot) / nslots + 1 : 0)
-                           : (slot < 2 * num_tiles ? 1 : 0);
-  auto tile_of = [&](int t) { return SPLIT == 1 ? slot + t * nslots : slot >> 1; };
-  const uint32_t my_iters = (uint32_t)my_tiles * nst;
+  // This pair's work as segments (tile, first stage, end stage), in order:
+  //   SPLIT = 1: whole tiles slot, slot + nslots, ...
+  //   SPLIT = 2: one segment, tile slot / 2, K half slot % 2
+  //   SPLIT = 3: stream-K -- the tiles' T * S stages cut into nslots equal
+  //              contiguous ranges; a range starts inside a tile (its tail),
+  //              covers whole tiles and ends inside another (its head).  With
+  //              at least S stages per range a tile has at most two parts.
+  // Segment i: tile t_first + i * t_step, stages [i == 0 ? st_first : 0,
+  // i == nseg - 1 ? st_last : S).
+  int nseg = 0, t_first = 0, t_step = 1, st_first = 0, st_last = S;
+  if (SPLIT == 1) {
+    nseg = slot < num_tiles ? (num_tiles - 1 - slot) / nslots + 1 : 0;
+    t_first = slot;
+    t_step = nslots;
+  } else if (SPLIT == 2) {
+    nseg = slot < 2 * num_tiles ? 1 : 0;
+    t_first = slot >> 1;
+    st_first = (slot & 1) ? S / 2 : 0;
+    st_last = (slot & 1) ? S : S / 2;
+  } else {
+    const int64_t units = (int64_t)num_tiles * S;
+    const int64_t u0 = units * slot / nslots, u1 = units * (slot + 1) / nslots;
+    if (u1 > u0) {
+      t_first = (int)(u0 / S);
+      const int t_last = (int)((u1 - 1) / S);
+      nseg = t_last - t_first + 1;
+      st_first = (int)(u0 - (int64_t)t_first * S);
+      st_last = (int)(u1 - (int64_t)t_last * S);
+    }
+  }
+  auto seg_tile = [&](int i) -> int { return t_first + i * t_step; };
+  auto seg_begin = [&](int i) -> int { return i == 0 ? st_first : 0; };
+  auto seg_end = [&](int i) -> int { return i == nseg - 1 ? st_last : S; };
+  uint32_t my_iters = 0;
+  for (int i = 0; i < nseg; ++i) my_iters += (uint32_t)(seg_end(i) - seg_begin(i));
   const uint32_t full0 = map_to_cta(smem_addr(full), lead);  // pair leader's full[0]
   const uint32_t tempty0 = map_to_cta(smem_addr(tempty), lead);
 
   if (warp == 0) {
     if (lane == 0) {
       // ---------------- producer (every CTA) ----------------
-      auto issue = [&](uint32_t it, uint32_t s, bool weights, bool acts) {
-        const int tile = tile_of((int)(it / nst));
+      auto issue = [&](int tile, int st, uint32_t s, bool weights, bool acts) {
         const int mb = tile % args.tiles_m, nb = tile / args.tiles_m;
-        const int kb0 = (st_begin + (int)(it % nst)) * kStageK;
+        const int kb0 = st * kStageK;
         const int nk = min(kStageK, num_kb - kb0);
         const uint32_t bar = full0 + s * 8;
         if (weights) {
@@ -182,31 +213,38 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                              bar);
         }
       };
-      auto stage_bytes = [&](uint32_t it) {
-        const int kb0 = (st_begin + (int)(it % nst)) * kStageK;
-        const int nk = min(kStageK, num_kb - kb0);
+      auto stage_bytes = [&](int st) {
+        const int nk = min(kStageK, num_kb - st * kStageK);
         // the 256-wide weight box always moves two tiles (zero-filled past the end)
         return (uint32_t)(nk * kTileBytes + (BN == 256 ? L::kBStage : nk * L::kBTile));
       };
+      // cursor over (segment, stage) in the order the MMAs consume them
+      int ci = 0, cst = nseg > 0 ? seg_begin(0) : 0;
+      auto advance = [&]() {
+        if (++cst >= seg_end(ci) && ++ci < nseg) cst = seg_begin(ci);
+      };
       uint32_t last_par[STAGES];
+      int pre_tile[STAGES], pre_st[STAGES];
       bool ok = true;
       const uint32_t pre = my_iters < (uint32_t)STAGES ? my_iters : (uint32_t)STAGES;
       // weight tiles do not depend on the preceding kernel: issue them first
-      for (uint32_t it = 0; it < pre; ++it) {
-        mbar_arrive_expect_tx_cluster(full0 + it * 8, stage_bytes(it));
-        issue(it, it, true, false);
+      for (uint32_t it = 0; it < pre; ++it, advance()) {
+        pre_tile[it] = seg_tile(ci);
+        pre_st[it] = cst;
+        mbar_arrive_expect_tx_cluster(full0 + it * 8, stage_bytes(cst));
+        issue(pre_tile[it], cst, it, true, false);
         last_par[it] = 0;
       }
       griddep_wait();
-      for (uint32_t it = 0; it < pre; ++it) issue(it, it, false, true);
-      for (uint32_t it = pre; it < my_iters; ++it) {
+      for (uint32_t it = 0; it < pre; ++it) issue(pre_tile[it], pre_st[it], it, false, true);
+      for (uint32_t it = pre; it < my_iters; ++it, advance()) {
         const uint32_t s = it % STAGES, ph = (it / STAGES) & 1;
         if (!mbar_wait(&empty[s], ph ^ 1, abort_flag, args.status)) {
           ok = false;
           break;
         }
-        mbar_arrive_expect_tx_cluster(full0 + s * 8, stage_bytes(it));
-        issue(it, s, true, true);
+        mbar_arrive_expect_tx_cluster(full0 + s * 8, stage_bytes(cst));
+        issue(seg_tile(ci), cst, s, true, true);
         last_par[s] = ph;
       }
       // Wait until every stage this CTA filled has been consumed: the MMA
@@ -223,28 +261,30 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       // ---------------- MMA issuer (even CTA of each pair) ----------------
       uint32_t it = 0;
       bool ok = true;
-      for (int t = 0; ok && t < my_tiles; ++t) {
-        const uint32_t b = t & 1, bph = (t >> 1) & 1;
+      for (int i = 0; ok && i < nseg; ++i) {
+        const uint32_t b = i & 1, bph = (i >> 1) & 1;
         if (!mbar_wait(&tempty[b], bph ^ 1, abort_flag, args.status)) {
           ok = false;
           break;
         }
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + b * kPairBN;
-        for (int j = 0; j < nst; ++j, ++it) {
+        const int sb = seg_begin(i), se = seg_end(i);
+        for (int st = sb; st < se; ++st, ++it) {
           const uint32_t s = it % STAGES, ph = (it / STAGES) & 1;
           if (!mbar_wait(&full[s], ph, abort_flag, args.status)) {
             ok = false;
             break;
           }
           tc_fence_after();
-          const int nk = min(kStageK, num_kb - (st_begin + j) * kStageK);
+          const int nk = min(kStageK, num_kb - st * kStageK);
           for (int h = 0; h < nk; ++h) {
             const uint64_t a_desc = sw128_kmajor_desc(sA + s * kHalfStage + h * kTileBytes);
             const uint64_t b_desc = sw128_kmajor_desc(sB + s * L::kBStage + h * L::kBTile);
 #pragma unroll
             for (int k = 0; k < kBK / 32; ++k)
-              mma_i8_pair(d_tmem, a_desc + 2 * k, b_desc + 2 * k, kIdesc, (j | h | k) != 0);
+              mma_i8_pair(d_tmem, a_desc + 2 * k, b_desc + 2 * k, kIdesc,
+                          (st != sb) || h != 0 || k != 0);
           }
           mma_commit_pair(&empty[s], pair_mask);  // frees the stage in both CTAs
         }
@@ -268,12 +308,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     uint8_t *s_out = smem + L::kOut + (warp - 2) * kEpiStagePerWarp;
     const int r = ew.quarter * 32 + lane;  // row within this CTA's 128
     const int j0 = ew.half * kCols;        // first tile column of this warp
-    for (int t = 0; t < my_tiles; ++t) {
-      const int tile = tile_of(t);
+    for (int i = 0; i < nseg; ++i) {
+      const int tile = seg_tile(i);
       const int mb = tile % args.tiles_m, nb = tile / args.tiles_m;
       const int row0 = mb * 256 + (int)rank * 128 + ew.quarter * 32;
       const int n0 = nb * kPairBN + j0;
-      const uint32_t b = t & 1, bph = (t >> 1) & 1;
+      const uint32_t b = i & 1, bph = (i >> 1) & 1;
+      const bool whole = seg_begin(i) == 0 && seg_end(i) == S;
       stage_columns<kCols>(args, n0, lane, s_ws, s_bias);
       const float as = row0 + lane < args.M ? __ldg(args.a_scale + row0 + lane) : 0.0f;
       __syncwarp();
@@ -284,14 +325,23 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       tc_fence_after();
       const uint32_t taddr =
           tmem_base + b * kPairBN + j0 + ((uint32_t)(ew.quarter * 32) << 16);
-      if (SPLIT == 2) {
-        // Which of the two K halves of these 128 rows finished first?
-        const int sidx = tile * 2 + (int)rank;
+      bool add_partial = false, partial_in_l2 = false;
+      int32_t *gpart = nullptr;
+      if (!whole) {
+        // This tile's 128 rows have one other part (the other K range).
+        // Which of the two finished first?  Sync words and partial slot: per
+        // (tile, CTA rank) for the K split; for stream-K per (range boundary,
+        // CTA rank) -- the tile cut at the boundary between pairs p - 1 and p
+        // is pair p's first segment and pair p - 1's last.
+        const int part_key = SPLIT == 3 ? ((i == 0 && st_first > 0) ? slot : slot + 1) : tile;
+        const int sidx = part_key * 2 + (int)rank;
         unsigned long long *ctr = args.sync + 2 * sidx;  // [0] arrivals, [1] published
-        int32_t *gpart = args.partials + (size_t)sidx * kPartialInts;
+        gpart = args.partials + (size_t)sidx * kPartialInts;
         if (first_epi_thread) *arrival = (int)arrive_tagged(ctr, args.tag);
         named_barrier_sync(1, 32 * kEpiWarps);
-        if (*arrival == 1) {
+        const int order = *arrival;
+        named_barrier_sync(1, 32 * kEpiWarps);  // the word is reused by the next part
+        if (order == 1) {
           // First: publish the int32 partial (the layout of partial_index),
           // then raise the flag once every epilogue thread's stores are out.
           for_tmem_chunks<kCols / 32>(
@@ -306,36 +356,49 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           named_barrier_sync(1, 32 * kEpiWarps);
           if (first_epi_thread) st_release_gpu(ctr + 1, args.tag);
         } else {
-          // Second: the partner has arrived, so its partial is being or has
-          // been published; copy it into the idle stage buffers and finish.
+          // Second: the other part has arrived, so its partial is being or
+          // has been published.  In this CTA's last segment the stage
+          // buffers are idle and take it in one bulk copy; otherwise (rare:
+          // stream-K parts normally finish tail first) the epilogue reads it
+          // from L2.
+          const bool last = i == nseg - 1;
+          int got = 1;
           if (first_epi_thread) {
-            if (flag_wait_bounded(ctr + 1, args.tag, abort_flag, args.status)) {
+            got = flag_wait_bounded(ctr + 1, args.tag, abort_flag, args.status);
+            if (got && last) {
               fence_proxy_async_global();
               mbar_arrive_expect_tx(recv, kPartialBytes);
               bulk_load(partial, gpart, kPartialBytes, recv);
             }
+            *arrival = got;
           }
-          int got = 0;
-          if (lane == 0) got = mbar_wait(recv, 0, abort_flag, args.status);
-          got = __shfl_sync(0xFFFFFFFFu, got, 0);
+          named_barrier_sync(1, 32 * kEpiWarps);
+          got = *arrival;
+          named_barrier_sync(1, 32 * kEpiWarps);
           if (!got) break;
-          // Both CTAs are done with the two words for this call: clear them,
+          if (last) {
+            if (lane == 0) got = mbar_wait(recv, 0, abort_flag, args.status);
+            got = __shfl_sync(0xFFFFFFFFu, got, 0);
+            if (!got) break;
+          }
+          // Both parts are done with the two words for this call: clear them,
           // so a replayed CUDA graph (same tag) starts from zero.
           if (first_epi_thread) {
             ctr[0] = 0ull;
             ctr[1] = 0ull;
           }
-          epilogue_tma<kCols>(args, &tmap_y, taddr, lane, row0, n0, as, s_ws, s_bias, s_out,
-                              partial, PartialIndex{r, j0});
+          add_partial = true;
+          partial_in_l2 = !last;
         }
-      } else {
-        // dequantise: acc * a_scale * w_scale + bias
-        epilogue_tma<kCols>(args, &tmap_y, taddr, lane, row0, n0, as, s_ws, s_bias, s_out,
-                            nullptr, PartialIndex{r, j0});
       }
+      if (whole || add_partial)
+        // dequantise: (acc [+ the other part's partial]) * a_scale * w_scale + bias
+        epilogue_tma<kCols>(args, &tmap_y, taddr, lane, row0, n0, as, s_ws, s_bias, s_out,
+                            add_partial,
+                            PartialLoad{partial_in_l2 ? gpart : partial, r, j0, partial_in_l2});
       tc_fence_before();
       __syncwarp();
-      if (SPLIT == 1 && lane == 0) mbar_arrive_cluster(tempty0 + b * 8);
+      if (lane == 0) mbar_arrive_cluster(tempty0 + b * 8);
     }
     if (lane == 0) bulk_wait_group_all();  // output stores complete before exit
     __syncwarp();
@@ -349,7 +412,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   }
 }
 
-bool g_pair_attr_done[64][3];
+bool g_pair_attr_done[64][4];
 
 template <int BN, int STAGES, int SPLIT>
 w8a8_status run_pair(const CUtensorMap &tq, const CUtensorMap &tw, const CUtensorMap &ty,
@@ -365,8 +428,13 @@ w8a8_status run_pair(const CUtensorMap &tq, const CUtensorMap &tw, const CUtenso
   }
   const int tiles = a.tiles_m * a.tiles_n;
   // SPLIT = 1: persistent, one pair per two SMs; SPLIT = 2: one pair per
-  // (tile, K half).
-  const int pairs = SPLIT == 1 ? std::max(1, std::min(tiles, sm_count() / 2)) : 2 * tiles;
+  // (tile, K half); SPLIT = 3: persistent stream-K over all SM pairs when
+  // there are more tiles than pairs (a tile then has at most two parts);
+  // with fewer tiles (a forced path, for tests) two pairs per three tiles.
+  const int sm_pairs = sm_count() / 2;
+  const int pairs = SPLIT == 1   ? std::max(1, std::min(tiles, sm_pairs))
+                    : SPLIT == 2 ? 2 * tiles
+                                 : (tiles >= sm_pairs ? sm_pairs : std::max(1, 2 * tiles / 3));
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)(2 * pairs));
   cfg.blockDim = dim3(kGemmThreads);
@@ -391,10 +459,16 @@ w8a8_status run_pair(const CUtensorMap &tq, const CUtensorMap &tw, const CUtenso
 // Number of 256 x bn tiles the pair kernel would process.
 int64_t pair_tiles(int64_t M, int64_t N, int bn) { return ((M + 255) / 256) * ((N + bn - 1) / bn); }
 
-// Workspace of the K-split pair kernel: per (tile, CTA rank) two 8-byte sync
-// words, then one 128 KB int32 partial.
-int64_t split_workspace_bytes(int64_t M, int64_t N) {
-  const int64_t slots = 2 * pair_tiles(M, N, 256);
+// Workspace of the K-split and stream-K pair kernels: per slot two 8-byte
+// sync words, then one 128 KB int32 partial per slot.  Slots: (tile, CTA
+// rank) for the K split; (range boundary, CTA rank) for stream-K, at most
+// one per SM pair plus one.
+int64_t split_slots(int64_t M, int64_t N, int split) {
+  return split == 3 ? 2 * (int64_t)(sm_count() / 2 + 1) : 2 * pair_tiles(M, N, 256);
+}
+
+int64_t split_workspace_bytes(int64_t M, int64_t N, int split) {
+  const int64_t slots = split_slots(M, N, split);
   return round_up(slots * 16, 256) + slots * kPartialBytes;
 }
 
@@ -427,15 +501,18 @@ w8a8_status launch_gemm2sm(const int8_t *q, const float *a_scale, const void *pa
   a.tag = 0;
   if (!a.status) return W8A8_ERR_CUDA;
   if (bn == 128) return run_pair<128, 4, 1>(tq, tw, ty, a, stream, pdl, 2);
-  // the split needs at least one stage per half and the workspace
-  if (split == 2 && (a.num_kb + kStageK - 1) / kStageK >= 2 && workspace &&
-      (int64_t)ws_bytes >= split_workspace_bytes(M, N)) {
-    const int64_t slots = 2 * pair_tiles(M, N, 256);
+  // the K split needs at least one stage per half, stream-K at least two
+  // stages per tile; both need the workspace
+  const int S = (a.num_kb + kStageK - 1) / kStageK;
+  if ((split == 2 || split == 3) && S >= split && workspace &&
+      (int64_t)ws_bytes >= split_workspace_bytes(M, N, split)) {
+    const int64_t slots = split_slots(M, N, split);
     uint8_t *ws = static_cast<uint8_t *>(workspace);
     a.sync = reinterpret_cast<unsigned long long *>(ws);
     a.partials = reinterpret_cast<int32_t *>(ws + round_up(slots * 16, 256));
     a.tag = next_call_tag();
-    return run_pair<256, 3, 2>(tq, tw, ty, a, stream, pdl, 1);
+    return split == 2 ? run_pair<256, 3, 2>(tq, tw, ty, a, stream, pdl, 1)
+                      : run_pair<256, 3, 3>(tq, tw, ty, a, stream, pdl, 3);
   }
   return run_pair<256, 3, 1>(tq, tw, ty, a, stream, pdl, 0);
 }

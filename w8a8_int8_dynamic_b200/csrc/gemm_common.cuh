@@ -175,21 +175,21 @@ __device__ __forceinline__ uint32_t swz64_offset(int r, int c16) {
 //   taddr   TMEM address of the first column, this warp's lane quarter
 //   row0    output row of lane 0;  n0: output column of the first column
 //   s_ws / s_bias: the COLS columns' scales and bias, staged in smem
-//   extra   when non-null, an int32 partial in shared memory added to the
-//           accumulator first; element (lane, column j) at extra_index(j)
-template <int COLS, typename ExtraIndex>
+//   has_extra / extra_load: an int32 partial added to the accumulator first;
+//           extra_load(j) returns this lane's four values at column j..j+3
+template <int COLS, typename ExtraLoad>
 __device__ __forceinline__ void epilogue_tma(const GemmArgs &a, const CUtensorMap *tmap_y,
                                              uint32_t taddr, int lane, int row0, int n0, float as,
                                              const float *s_ws, const uint16_t *s_bias,
-                                             uint8_t *stage, const int32_t *extra,
-                                             ExtraIndex extra_index) {
+                                             uint8_t *stage, bool has_extra,
+                                             ExtraLoad extra_load) {
   for_tmem_chunks<COLS / 32>(
       taddr, [&](int c) { return n0 + c * 32 < a.N; },
       [&](uint32_t(&v)[32], int c) {
-        if (extra) {
+        if (has_extra) {
 #pragma unroll
           for (int g = 0; g < 8; ++g) {
-            const uint4 p = *reinterpret_cast<const uint4 *>(extra + extra_index(c * 32 + 4 * g));
+            const uint4 p = extra_load(c * 32 + 4 * g);
             v[4 * g] += p.x;
             v[4 * g + 1] += p.y;
             v[4 * g + 2] += p.z;
@@ -215,7 +215,7 @@ __device__ __forceinline__ void epilogue_tma(const GemmArgs &a, const CUtensorMa
 }
 
 struct NoExtra {
-  __device__ int operator()(int) const { return 0; }
+  __device__ uint4 operator()(int) const { return make_uint4(0, 0, 0, 0); }
 };
 
 }  // namespace w8a8

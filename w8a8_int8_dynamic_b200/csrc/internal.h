@@ -74,8 +74,9 @@ w8a8_status launch_gemm2sm(const int8_t *q, const float *a_scale, const void *pa
                            int act = W8A8_ACT_NONE, void *workspace = nullptr,
                            size_t ws_bytes = 0);
 int64_t pair_tiles(int64_t M, int64_t N, int bn);
-// Workspace the K-split pair kernel needs (sync words + int32 partials).
-int64_t split_workspace_bytes(int64_t M, int64_t N);
+// Workspace the K-split (split = 2) or stream-K (split = 3) pair kernel needs
+// (sync words + int32 partials).
+int64_t split_workspace_bytes(int64_t M, int64_t N, int split);
 // Small-M weight-streaming kernel (decode.cu).
 int64_t decode_workspace_bytes(int64_t N, int64_t K);
 bool use_decode_path(int64_t M);

@@ -153,7 +153,7 @@ const char *w8a8_status_string(int status) {
 int w8a8_abi_version(void) { return (1 << 16) | 0; }
 
 w8a8_status w8a8_set_path(int path) {
-  if (path < 0 || path > 7) return W8A8_ERR_INVALID_ARG;
+  if (path < 0 || path > 8) return W8A8_ERR_INVALID_ARG;
   g_forced_path.store(path);
   return W8A8_OK;
 }
