@@ -316,9 +316,12 @@ enum class LargeKind { k128, k256, kPair, kPair128, kPairSplit, kPairStreamK };
 
 // Kernel choice for large M: (waves of tiles) x (per-SM time of one tile).
 // The per-SM time of a stage of two k-blocks is set by what has to reach the
-// SM from L2 (measured ~114 GB/s per SM with ~190 KB in flight) or by the
-// MMAs, whichever is slower: 1-SM 128x128: 64 KB / 512 cycles; 1-SM 128x256:
-// 96 KB / 1024; pair 256x256: 64 KB / 1024; pair 256x128: 48 KB / 512 per SM.
+// SM (about 100-115 GB/s per SM in these kernels: stage slots of ~190 KB
+// cycle through the loaded-L2 latency and the MMAs), by a whole-chip delivery
+// term, or by the MMAs, whichever is slowest: 1-SM 128x128: 64 KB / 512
+// cycles; 1-SM 128x256: 96 KB / 1024; pair 256x256: 64 KB / 1024; pair
+// 256x128: 48 KB / 512 per SM.  The constants are calibrated against timings
+// on this B200, not derived.
 // `split_ok`: a workspace for the K-split pair kernel is available.
 LargeKind choose_large(int64_t M, int64_t N, int64_t K, bool split_ok) {
   const int path = forced_path();
@@ -352,26 +355,20 @@ LargeKind choose_large(int64_t M, int64_t N, int64_t K, bool split_ok) {
   // Few 256-wide pair tiles (half the GPU or less) but 128x128 tiles that fit
   // one wave: with cold operands, twice as many SMs pulling from DRAM wins
   // (measured on 512 x 4096 x 4096: 16.6 us vs 19.1 us for 256x256 pairs).
-  // Splitting K over two pairs per tile halves the operand traffic but its
-  // int32 partial handoff (about 4 us for 128 KB per CTA through L2) costs
-  // more than it saves at these sizes (512 x 4096 x K, measured: 19.1 vs
-  // 14.3 us at K = 4096, even at K = 8192), so it is never chosen here.
-  (void)split_ok;
-  (void)K;
   if (tp256 * 2 <= pairs && t128 <= sms) return LargeKind::k128;
   double best = c128;
   LargeKind kind = LargeKind::k128;
   if (c256 < best) best = c256, kind = LargeKind::k256;
   if (cp256 <= best) best = cp256, kind = LargeKind::kPair;
   if (cp128 < best * 0.97) best = cp128, kind = LargeKind::kPair128;
-  // Stream-K (equal k-block ranges per SM pair, path 8) is not chosen: these
-  // kernels are bound by L2 -> SM delivery, so a last wave with few busy pairs
-  // runs each of them faster and costs little, while stream-K's int32
-  // partials add about a fifth to the L2 traffic (measured on 512 x 12288 x
-  // 4096: 35.3 us against 31.8 us with whole tiles).
-  // The K-split pair variant exchanges a 128 KB partial per CTA over DSMEM
-  // (measured ~5 us): it does not pay on the shapes at hand and is never
-  // chosen automatically.
+  // Never chosen here, both measured slower on the shapes at hand: the K
+  // split over two pairs per tile (paths 6; 512 x 4096 x 4096: 19.1 vs
+  // 14.3 us -- the 128 KB int32 handoff per CTA costs about 4 us) and
+  // stream-K (path 8; 512 x 12288 x 4096: 35.3 vs 31.8 us -- the partials add
+  // about a fifth to the L2 traffic, while a last wave with few busy SMs
+  // runs each of its tiles faster and costs little).
+  (void)split_ok;
+  (void)K;
   return kind;
 }
 
