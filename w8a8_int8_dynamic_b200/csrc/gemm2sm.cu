@@ -483,7 +483,7 @@ w8a8_status launch_gemm2sm(const int8_t *q, const float *a_scale, const void *pa
   const uint64_t wrows = (uint64_t)(packed_rows(N) * packed_cols(K) / 128);
   if (!make_tmap_u8_2d_plain(&tw, packed_w, wrows, 128, 128, bn == 128 ? 64 : 256, 128))
     return W8A8_ERR_CUDA;
-  GemmArgs a;
+  GemmArgs a{};
   a.packed_w = static_cast<const uint8_t *>(packed_w);
   a.a_scale = a_scale;
   a.w_scale = w_scale;

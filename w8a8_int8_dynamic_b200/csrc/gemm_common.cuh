@@ -35,6 +35,9 @@ struct GemmArgs {
   int num_kb;            // K blocks of 128 bytes (= packed K / 128)
   int tiles_m, tiles_n;
   int act;               // w8a8_act applied after the dequantisation
+  // 1-SM kernel: k-blocks of its first weight slab past the first stages that
+  // a CTA asks L2 to fetch before waiting for the preceding kernel (0: none)
+  int prefetch_kb;
   int *status;
   // K-split pair kernel only: per (tile, CTA rank) a call-tagged arrival
   // counter and a "partial published" flag, and the published int32 partials
