@@ -98,6 +98,14 @@ __global__ void __launch_bounds__(kThreads, 1)
   volatile int *last_flag = reinterpret_cast<volatile int *>(smem + L::kMisc + 8);
   volatile int *seg_ok = reinterpret_cast<volatile int *>(smem + L::kMisc + 16);  // [2]
 
+  // Release the next kernel of the stream at once: the activation
+  // quantisation of the next layer becomes resident beside this kernel and
+  // waits on the device for it to finish, and the next layer's GEMM takes
+  // each SM as soon as this kernel's CTA there exits, streaming its weights
+  // while the last CTAs here still sum their partials.  (The large-M kernels
+  // do not: the next quantisation's CTAs would crowd onto the SMs they leave
+  // idle.)
+  griddep_launch_dependents();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {

@@ -21,6 +21,11 @@
 // share an SM with it.  Rows longer than 65536 elements take a two-pass
 // kernel.  HBM-bound: 2 bytes read + 1 byte written per element.
 //
+// Both kernels are programmatic dependent launches: their CTAs may become
+// resident while the preceding kernel of the stream is still running (the
+// decode GEMM releases its dependents early), and wait on the device for it
+// to complete before reading x, which may be that kernel's output.
+//
 // The per-element arithmetic (the exact quotient by reciprocal refinement,
 // rint by one addition) is in quant_common.cuh, shared with the GEMM that
 // quantises its own rows.
@@ -45,6 +50,7 @@ __global__ void __launch_bounds__(512) quant_warps_kernel(const uint16_t *__rest
                                                           float *__restrict__ a_scale) {
   // Let a dependent GEMM start its prologue while the rows are quantised.
   griddep_launch_dependents();
+  griddep_wait();  // x may be the preceding kernel's output
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int rl = warp / W, w = warp - rl * W;
@@ -110,6 +116,7 @@ __global__ void __launch_bounds__(1024) quant_rows_two_pass_kernel(
     const uint16_t *__restrict__ x, int64_t ldx, int K, int8_t *__restrict__ q,
     float *__restrict__ a_scale) {
   griddep_launch_dependents();
+  griddep_wait();  // x may be the preceding kernel's output
   const int64_t row = blockIdx.x;
   const int nchunks = K >> 3;
   const uint16_t *xr = x + row * ldx;
@@ -216,6 +223,23 @@ __global__ void __launch_bounds__(256) quant_static_kernel(const uint16_t *__res
   }
 }
 
+// Launches k as a programmatic dependent of the preceding kernel of the stream.
+template <typename... Params, typename... Args>
+cudaError_t launch_dependent(void (*k)(Params...), dim3 grid, dim3 block, cudaStream_t stream,
+                             Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, k, static_cast<Params>(args)...);
+}
+
 }  // namespace
 
 w8a8_status launch_quant(const void *x, int64_t M, int64_t K, int64_t ldx, int8_t *q,
@@ -231,17 +255,19 @@ w8a8_status launch_quant(const void *x, int64_t M, int64_t K, int64_t ldx, int8_
   while (cpl < per_lane && (cpl < 4 || (nchunks + 32 * cpl - 1) / (32 * cpl) > 16) && cpl < 16)
     cpl *= 2;
   const int64_t W = (nchunks + 32 * cpl - 1) / (32 * cpl);
+  cudaError_t e = cudaSuccess;
   if (W > 16) {
-    quant_rows_two_pass_kernel<<<(unsigned)M, 1024, 0, stream>>>(xp, ldx, (int)K, q, a_scale);
+    e = launch_dependent(quant_rows_two_pass_kernel, dim3((unsigned)M), dim3(1024), stream, xp,
+                         ldx, (int)K, q, a_scale);
   } else {
     const int R = W >= 4 ? 1 : (int)(4 / W);  // rows per CTA: about 128 threads
     const unsigned grid = (unsigned)((M + R - 1) / R);
     const unsigned threads = (unsigned)(32 * W * R);
     switch (cpl) {
-#define W8A8_QUANT_CASE(C)                                                                     \
-  case C:                                                                                      \
-    quant_warps_kernel<C><<<grid, threads, 0, stream>>>(xp, ldx, (int)M, (int)K, (int)W, R, q, \
-                                                        a_scale);                              \
+#define W8A8_QUANT_CASE(C)                                                                   \
+  case C:                                                                                    \
+    e = launch_dependent(quant_warps_kernel<C>, dim3(grid), dim3(threads), stream, xp, ldx, \
+                         (int)M, (int)K, (int)W, R, q, a_scale);                             \
     break;
       W8A8_QUANT_CASE(1)
       W8A8_QUANT_CASE(2)
@@ -253,6 +279,7 @@ w8a8_status launch_quant(const void *x, int64_t M, int64_t K, int64_t ldx, int8_
         return W8A8_ERR_INVALID_ARG;
     }
   }
+  if (e != cudaSuccess) return from_cuda(e);
   count_launch();
   return from_cuda(cudaGetLastError());
 }
