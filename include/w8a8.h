@@ -262,9 +262,9 @@ w8a8_status w8a8_linear_noalloc(const void *x, int64_t ldx, const void *packed_w
  * then sizes); 7 = the 2-SM GEMM with 256 x 128 tiles; 8 = the 256 x 256
  * 2-SM GEMM with stream-K: the tiles' k-blocks cut into equal contiguous
  * ranges, one per SM pair, tiles split between two pairs summing their int32
- * partials through the workspace (chosen automatically, given the workspace,
- * when the tiles outnumber the SM pairs and the last wave would leave pairs
- * idle).
+ * partials through the workspace (sized by w8a8_scaled_mm_workspace_bytes
+ * while the path is set).  Paths 6 and 8 are never chosen automatically; the
+ * others are, by shape.
  * Process-wide; not synchronised with concurrent calls. */
 w8a8_status w8a8_set_path(int path);
 
