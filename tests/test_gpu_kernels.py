@@ -193,6 +193,10 @@ def test_k_split_pairs_with_garbage_workspace_repeated(M, N, K):
 def test_scaled_mm_does_not_write_outside_y(path):
     w8.set_path(path)
     M, N, K = 130, 264, 272
+    _guarded_scaled_mm(M, N, K)
+
+
+def _guarded_scaled_mm(M, N, K):
     inp = random_case(9, M, N, K, bias=True)
     q_ref, s_ref = oracle.quant_act(inp.x)
     guard = 4096
@@ -203,6 +207,23 @@ def test_scaled_mm_does_not_write_outside_y(path):
     y_ref = oracle.epilogue(oracle.gemm_i32(q_ref, inp.w), s_ref, inp.w_scale, inp.bias)
     assert np.array_equal(host_u16(y), y_ref)
     assert (ybuf[M * N:].cpu().numpy() == -1).all()
+
+
+@pytest.mark.parametrize("M,N,K", [(300, 20480, 528), (600, 8200, 400)])
+def test_pair_tail_split_matches_oracle(M, N, K):
+    """Shapes whose 256 x 256 pair tiles fill the SM pairs once and leave a
+    short last round (160 tiles: 12 left over; 99 tiles: 25 left over, the
+    last one ragged in N and M): those tiles run as two 256 x 128 halves.
+    Bit-exact against the oracle, automatic and forced pair path, nothing
+    written past y."""
+    pairs = torch.cuda.get_device_properties(0).multi_processor_count // 2
+    tiles = ((M + 255) // 256) * ((N + 255) // 256)
+    if not (tiles > pairs and 0 < tiles % pairs <= pairs // 2):
+        pytest.skip(f"{tiles} tiles on {pairs} SM pairs leave no short last round")
+    for path in (w8.PATH_AUTO, w8.PATH_LARGE_PAIR):
+        w8.set_path(path)
+        assert "256x256" in w8.gemm_kernel_name(M, N, K)
+        _guarded_scaled_mm(M, N, K)
 
 
 # ---------------------------------------------------------------- decode path

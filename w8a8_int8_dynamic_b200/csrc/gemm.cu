@@ -374,7 +374,9 @@ LargeKind choose_large(int64_t M, int64_t N, int64_t K, bool split_ok) {
   };
   const double c128 = cost(t128, sms, 1, 65536, 512);
   const double c256 = cost(t256, sms, 1, 98304, 1024);
-  const double cp256 = cost(tp256, pairs, 2, 65536, 1024);
+  double cp256 = cost(tp256, pairs, 2, 65536, 1024);
+  if (pair_full_tiles(tp256, pairs) < tp256)  // a short last round runs as half tiles
+    cp256 -= 0.25 * cost(pairs, pairs, 2, 65536, 1024);
   const double cp128 = cost(tp128, pairs, 2, 49152, 512);
   // Few 256-wide pair tiles (half the GPU or less) but 128x128 tiles that fit
   // one wave: with cold operands, twice as many SMs pulling from DRAM wins

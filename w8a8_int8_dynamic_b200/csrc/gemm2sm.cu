@@ -20,6 +20,10 @@
 //   * both CTAs run the epilogue on their own 128 TMEM lanes.
 //
 // SPLIT = 1: persistent clusters of 2 CTAs, double-buffered accumulators.
+//   When the 256 x 256 tiles fill the SM pairs a few times over plus a short
+//   last round (at most half the pairs), the tiles of that round run as their
+//   two 256 x 128 halves instead (MMA N = 128, each CTA loading 64 weight
+//   rows), spread over twice as many pairs.
 // SPLIT = 2: (for problems with too few tiles to fill the GPU) every tile is
 //   computed by two pairs, one per half of K, one work item per pair.  Per
 //   (tile, CTA rank) a call-tagged counter in the workspace tells the two
@@ -88,11 +92,14 @@ template <int BN, int STAGES, int SPLIT>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     gemm2sm_kernel(const __grid_constant__ CUtensorMap tmap_q,
                    const __grid_constant__ CUtensorMap tmap_w,
+                   const __grid_constant__ CUtensorMap tmap_w64,
                    const __grid_constant__ CUtensorMap tmap_y, const GemmArgs args) {
   using L = PairSmem<BN, STAGES>;
   constexpr int kPairBN = BN;
   constexpr uint32_t kTmemCols = 2 * BN;
   constexpr uint32_t kIdesc = idesc_i8(256, BN);
+  constexpr uint32_t kIdescHalf = idesc_i8(256, 128);  // a 256 x 128 half of a 256-wide tile
+  constexpr int kHalfBTile = 64 * kBK;                   // its weight rows per CTA per k-block
   static_assert(SPLIT == 1 || BN == 256, "the K split is built for 256-wide tiles");
   static_assert(SPLIT >= 1 && SPLIT <= 3, "1: whole tiles, 2: K halves, 3: stream-K");
 
@@ -136,6 +143,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   if (warp == 0 && lane == 0) {
     prefetch_tmap(&tmap_q);
     prefetch_tmap(&tmap_w);
+    if (BN == 256 && args.full_tiles < args.tiles_m * args.tiles_n) prefetch_tmap(&tmap_w64);
   }
   if (warp == 1) tmem_alloc_pair(tmem_slot, kTmemCols);
   tc_fence_before();
@@ -148,8 +156,18 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   const int S = (num_kb + kStageK - 1) / kStageK;  // stages per tile
   const int slot = (int)(blockIdx.x >> 1);
   const int nslots = (int)(gridDim.x >> 1);
-  // This pair's work as segments (tile, first stage, end stage), in order:
-  //   SPLIT = 1: whole tiles slot, slot + nslots, ...
+  // Work items: tiles [0, full_tiles) whole, then item full_tiles + 2 j + h
+  // is N half h of tile full_tiles + j (SPLIT = 1 only; otherwise full_tiles
+  // is the tile count).
+  const int num_items = args.full_tiles + 2 * (num_tiles - args.full_tiles);
+  auto item_tile = [&](int item) -> int {
+    return item < args.full_tiles ? item : args.full_tiles + ((item - args.full_tiles) >> 1);
+  };
+  auto item_half = [&](int item) -> int {  // -1: the whole tile
+    return item < args.full_tiles ? -1 : ((item - args.full_tiles) & 1);
+  };
+  // This pair's work as segments (item, first stage, end stage), in order:
+  //   SPLIT = 1: items slot, slot + nslots, ...
   //   SPLIT = 2: one segment, tile slot / 2, K half slot % 2
   //   SPLIT = 3: stream-K -- the tiles' T * S stages cut into nslots equal
   //              contiguous ranges; a range starts inside a tile (its tail),
@@ -159,7 +177,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   // i == nseg - 1 ? st_last : S).
   int nseg = 0, t_first = 0, t_step = 1, st_first = 0, st_last = S;
   if (SPLIT == 1) {
-    nseg = slot < num_tiles ? (num_tiles - 1 - slot) / nslots + 1 : 0;
+    nseg = slot < num_items ? (num_items - 1 - slot) / nslots + 1 : 0;
     t_first = slot;
     t_step = nslots;
   } else if (SPLIT == 2) {
@@ -189,13 +207,19 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   if (warp == 0) {
     if (lane == 0) {
       // ---------------- producer (every CTA) ----------------
-      auto issue = [&](int tile, int st, uint32_t s, bool weights, bool acts) {
+      auto issue = [&](int item, int st, uint32_t s, bool weights, bool acts) {
+        const int tile = item_tile(item), half = item_half(item);
         const int mb = tile % args.tiles_m, nb = tile / args.tiles_m;
         const int kb0 = st * kStageK;
         const int nk = min(kStageK, num_kb - kb0);
         const uint32_t bar = full0 + s * 8;
         if (weights) {
-          if (BN == 256) {
+          if (BN == 256 && half >= 0) {
+            // this CTA's 64-row half of slab 2 nb + half, per k-block
+            for (int h = 0; h < nk; ++h)
+              tma_load_2d_pair(sB + s * L::kBStage + h * kHalfBTile, &tmap_w64, 0,
+                               ((nb * 2 + half) * num_kb + kb0 + h) * 128 + (int)rank * 64, bar);
+          } else if (BN == 256) {
             // two contiguous packed tiles (k-blocks kb0, kb0+1) of this CTA's slab
             const int wslab = nb * 2 + (int)rank;
             tma_load_2d_pair(sB + s * L::kBStage, &tmap_w, 0, (wslab * num_kb + kb0) * 128, bar);
@@ -213,10 +237,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                              bar);
         }
       };
-      auto stage_bytes = [&](int st) {
+      auto stage_bytes = [&](int item, int st) {
         const int nk = min(kStageK, num_kb - st * kStageK);
         // the 256-wide weight box always moves two tiles (zero-filled past the end)
-        return (uint32_t)(nk * kTileBytes + (BN == 256 ? L::kBStage : nk * L::kBTile));
+        const int wb = BN == 256 ? (item_half(item) >= 0 ? nk * kHalfBTile : L::kBStage)
+                                 : nk * L::kBTile;
+        return (uint32_t)(nk * kTileBytes + wb);
       };
       // cursor over (segment, stage) in the order the MMAs consume them
       int ci = 0, cst = nseg > 0 ? seg_begin(0) : 0;
@@ -231,7 +257,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       for (uint32_t it = 0; it < pre; ++it, advance()) {
         pre_tile[it] = seg_tile(ci);
         pre_st[it] = cst;
-        mbar_arrive_expect_tx_cluster(full0 + it * 8, stage_bytes(cst));
+        mbar_arrive_expect_tx_cluster(full0 + it * 8, stage_bytes(pre_tile[it], cst));
         issue(pre_tile[it], cst, it, true, false);
         last_par[it] = 0;
       }
@@ -243,7 +269,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           ok = false;
           break;
         }
-        mbar_arrive_expect_tx_cluster(full0 + s * 8, stage_bytes(cst));
+        mbar_arrive_expect_tx_cluster(full0 + s * 8, stage_bytes(seg_tile(ci), cst));
         issue(seg_tile(ci), cst, s, true, true);
         last_par[s] = ph;
       }
@@ -270,6 +296,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + b * kPairBN;
         const int sb = seg_begin(i), se = seg_end(i);
+        const bool half = BN == 256 && item_half(seg_tile(i)) >= 0;
+        const uint32_t idesc = half ? kIdescHalf : kIdesc;
+        const int b_step = half ? kHalfBTile : L::kBTile;
         for (int st = sb; st < se; ++st, ++it) {
           const uint32_t s = it % STAGES, ph = (it / STAGES) & 1;
           if (!mbar_wait(&full[s], ph, abort_flag, args.status)) {
@@ -280,10 +309,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           const int nk = min(kStageK, num_kb - st * kStageK);
           for (int h = 0; h < nk; ++h) {
             const uint64_t a_desc = sw128_kmajor_desc(sA + s * kHalfStage + h * kTileBytes);
-            const uint64_t b_desc = sw128_kmajor_desc(sB + s * L::kBStage + h * L::kBTile);
+            const uint64_t b_desc = sw128_kmajor_desc(sB + s * L::kBStage + h * b_step);
 #pragma unroll
             for (int k = 0; k < kBK / 32; ++k)
-              mma_i8_pair(d_tmem, a_desc + 2 * k, b_desc + 2 * k, kIdesc,
+              mma_i8_pair(d_tmem, a_desc + 2 * k, b_desc + 2 * k, idesc,
                           (st != sb) || h != 0 || k != 0);
           }
           mma_commit_pair(&empty[s], pair_mask);  // frees the stage in both CTAs
@@ -309,10 +338,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     const int r = ew.quarter * 32 + lane;  // row within this CTA's 128
     const int j0 = ew.half * kCols;        // first tile column of this warp
     for (int i = 0; i < nseg; ++i) {
-      const int tile = seg_tile(i);
+      const int tile = item_tile(seg_tile(i)), half = item_half(seg_tile(i));
       const int mb = tile % args.tiles_m, nb = tile / args.tiles_m;
       const int row0 = mb * 256 + (int)rank * 128 + ew.quarter * 32;
-      const int n0 = nb * kPairBN + j0;
+      // a half tile's 128 columns: 64 per warp
+      const int jw = half >= 0 ? half * 128 + ew.half * 64 : j0;  // warp's first tile column
+      const int ncols = half >= 0 ? 64 : kCols;
+      const int n0 = nb * kPairBN + jw;
       const uint32_t b = i & 1, bph = (i >> 1) & 1;
       const bool whole = seg_begin(i) == 0 && seg_end(i) == S;
       stage_columns<kCols>(args, n0, lane, s_ws, s_bias);
@@ -323,8 +355,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
       if (!ok) break;
       tc_fence_after();
-      const uint32_t taddr =
-          tmem_base + b * kPairBN + j0 + ((uint32_t)(ew.quarter * 32) << 16);
+      const uint32_t taddr = tmem_base + b * kPairBN + (half >= 0 ? ew.half * 64 : j0) +
+                             ((uint32_t)(ew.quarter * 32) << 16);
       bool add_partial = false, partial_in_l2 = false;
       int32_t *gpart = nullptr;
       if (!whole) {
@@ -395,7 +427,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         // dequantise: (acc [+ the other part's partial]) * a_scale * w_scale + bias
         epilogue_tma<kCols>(args, &tmap_y, taddr, lane, row0, n0, as, s_ws, s_bias, s_out,
                             add_partial,
-                            PartialLoad{partial_in_l2 ? gpart : partial, r, j0, partial_in_l2});
+                            PartialLoad{partial_in_l2 ? gpart : partial, r, j0, partial_in_l2},
+                            ncols);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive_cluster(tempty0 + b * 8);
@@ -415,8 +448,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 bool g_pair_attr_done[64][4];
 
 template <int BN, int STAGES, int SPLIT>
-w8a8_status run_pair(const CUtensorMap &tq, const CUtensorMap &tw, const CUtensorMap &ty,
-                     const GemmArgs &a, cudaStream_t stream, bool pdl, int slot_id) {
+w8a8_status run_pair(const CUtensorMap &tq, const CUtensorMap &tw, const CUtensorMap &tw64,
+                     const CUtensorMap &ty, const GemmArgs &a, cudaStream_t stream, bool pdl,
+                     int slot_id) {
   using L = PairSmem<BN, STAGES>;
   auto k = gemm2sm_kernel<BN, STAGES, SPLIT>;
   const int d = current_device();
@@ -427,12 +461,13 @@ w8a8_status run_pair(const CUtensorMap &tq, const CUtensorMap &tw, const CUtenso
     if (d >= 0 && d < 64) g_pair_attr_done[d][slot_id] = true;
   }
   const int tiles = a.tiles_m * a.tiles_n;
+  const int items = a.full_tiles + 2 * (tiles - a.full_tiles);
   // SPLIT = 1: persistent, one pair per two SMs; SPLIT = 2: one pair per
   // (tile, K half); SPLIT = 3: persistent stream-K over all SM pairs when
   // there are more tiles than pairs (a tile then has at most two parts);
   // with fewer tiles (a forced path, for tests) two pairs per three tiles.
   const int sm_pairs = sm_count() / 2;
-  const int pairs = SPLIT == 1   ? std::max(1, std::min(tiles, sm_pairs))
+  const int pairs = SPLIT == 1   ? std::max(1, std::min(items, sm_pairs))
                     : SPLIT == 2 ? 2 * tiles
                                  : (tiles >= sm_pairs ? sm_pairs : std::max(1, 2 * tiles / 3));
   cudaLaunchConfig_t cfg = {};
@@ -449,7 +484,7 @@ w8a8_status run_pair(const CUtensorMap &tq, const CUtensorMap &tw, const CUtenso
   attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = pdl ? 2 : 1;
-  const cudaError_t e = cudaLaunchKernelEx(&cfg, k, tq, tw, ty, a);
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, k, tq, tw, tw64, ty, a);
   count_launch();
   return from_cuda(e);
 }
@@ -458,6 +493,15 @@ w8a8_status run_pair(const CUtensorMap &tq, const CUtensorMap &tw, const CUtenso
 
 // Number of 256 x bn tiles the pair kernel would process.
 int64_t pair_tiles(int64_t M, int64_t N, int bn) { return ((M + 255) / 256) * ((N + bn - 1) / bn); }
+
+// Whole 256 x 256 tiles before the ones that run as two 256 x 128 halves:
+// when the tiles fill the SM pairs more than once and leave a last round of
+// at most half the pairs, that round's tiles are split (twice as many items,
+// each about 3/4 of a tile's time: the halves move 3/4 of the bytes).
+int64_t pair_full_tiles(int64_t tiles, int64_t pairs) {
+  const int64_t rem = tiles % pairs;
+  return (tiles > pairs && rem > 0 && 2 * rem <= pairs) ? tiles - rem : tiles;
+}
 
 // Workspace of the K-split and stream-K pair kernels: per slot two 8-byte
 // sync words, then one 128 KB int32 partial per slot.  Slots: (tile, CTA
@@ -476,13 +520,14 @@ w8a8_status launch_gemm2sm(const int8_t *q, const float *a_scale, const void *pa
                            const float *w_scale, const void *bias, void *y, int64_t M, int64_t N,
                            int64_t K, cudaStream_t stream, bool pdl, int split, int bn,
                            int act, void *workspace, size_t ws_bytes) {
-  CUtensorMap tq, tw, ty;
+  CUtensorMap tq, tw, tw64, ty;
   if (!make_tmap_u8_2d(&tq, q, (uint64_t)M, (uint64_t)K, (uint64_t)K, kBM, kBK))
     return W8A8_ERR_CUDA;
   if (!make_tmap_out_bf16(&ty, y, (uint64_t)M, (uint64_t)N)) return W8A8_ERR_CUDA;
   const uint64_t wrows = (uint64_t)(packed_rows(N) * packed_cols(K) / 128);
   if (!make_tmap_u8_2d_plain(&tw, packed_w, wrows, 128, 128, bn == 128 ? 64 : 256, 128))
     return W8A8_ERR_CUDA;
+  if (!make_tmap_u8_2d_plain(&tw64, packed_w, wrows, 128, 128, 64, 128)) return W8A8_ERR_CUDA;
   GemmArgs a{};
   a.packed_w = static_cast<const uint8_t *>(packed_w);
   a.a_scale = a_scale;
@@ -494,13 +539,14 @@ w8a8_status launch_gemm2sm(const int8_t *q, const float *a_scale, const void *pa
   a.num_kb = (int)(packed_cols(K) / 128);
   a.tiles_m = (int)((M + 255) / 256);
   a.tiles_n = (int)((N + bn - 1) / bn);
+  a.full_tiles = a.tiles_m * a.tiles_n;
   a.act = act;
   a.status = status_word();
   a.sync = nullptr;
   a.partials = nullptr;
   a.tag = 0;
   if (!a.status) return W8A8_ERR_CUDA;
-  if (bn == 128) return run_pair<128, 4, 1>(tq, tw, ty, a, stream, pdl, 2);
+  if (bn == 128) return run_pair<128, 4, 1>(tq, tw, tw64, ty, a, stream, pdl, 2);
   // the K split needs at least one stage per half, stream-K at least two
   // stages per tile; both need the workspace
   const int S = (a.num_kb + kStageK - 1) / kStageK;
@@ -511,10 +557,11 @@ w8a8_status launch_gemm2sm(const int8_t *q, const float *a_scale, const void *pa
     a.sync = reinterpret_cast<unsigned long long *>(ws);
     a.partials = reinterpret_cast<int32_t *>(ws + round_up(slots * 16, 256));
     a.tag = next_call_tag();
-    return split == 2 ? run_pair<256, 3, 2>(tq, tw, ty, a, stream, pdl, 1)
-                      : run_pair<256, 3, 3>(tq, tw, ty, a, stream, pdl, 3);
+    return split == 2 ? run_pair<256, 3, 2>(tq, tw, tw64, ty, a, stream, pdl, 1)
+                      : run_pair<256, 3, 3>(tq, tw, tw64, ty, a, stream, pdl, 3);
   }
-  return run_pair<256, 3, 1>(tq, tw, ty, a, stream, pdl, 0);
+  a.full_tiles = (int)pair_full_tiles(a.full_tiles, sm_count() / 2);
+  return run_pair<256, 3, 1>(tq, tw, tw64, ty, a, stream, pdl, 0);
 }
 
 }  // namespace w8a8

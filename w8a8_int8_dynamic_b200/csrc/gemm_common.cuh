@@ -38,6 +38,9 @@ struct GemmArgs {
   // 1-SM kernel: k-blocks of its first weight slab past the first stages that
   // a CTA asks L2 to fetch before waiting for the preceding kernel (0: none)
   int prefetch_kb;
+  // pair kernel, whole tiles: tiles [0, full_tiles) run whole, each later one
+  // as its two 128-column halves (a short last round spread over more pairs)
+  int full_tiles;
   int *status;
   // K-split pair kernel only: per (tile, CTA rank) a call-tagged arrival
   // counter and a "partial published" flag, and the published int32 partials
@@ -180,14 +183,15 @@ __device__ __forceinline__ uint32_t swz64_offset(int r, int c16) {
 //   s_ws / s_bias: the COLS columns' scales and bias, staged in smem
 //   has_extra / extra_load: an int32 partial added to the accumulator first;
 //           extra_load(j) returns this lane's four values at column j..j+3
+//   ncols   columns actually drained (a multiple of 32, at most COLS)
 template <int COLS, typename ExtraLoad>
 __device__ __forceinline__ void epilogue_tma(const GemmArgs &a, const CUtensorMap *tmap_y,
                                              uint32_t taddr, int lane, int row0, int n0, float as,
                                              const float *s_ws, const uint16_t *s_bias,
                                              uint8_t *stage, bool has_extra,
-                                             ExtraLoad extra_load) {
+                                             ExtraLoad extra_load, int ncols = COLS) {
   for_tmem_chunks<COLS / 32>(
-      taddr, [&](int c) { return n0 + c * 32 < a.N; },
+      taddr, [&](int c) { return c * 32 < ncols && n0 + c * 32 < a.N; },
       [&](uint32_t(&v)[32], int c) {
         if (has_extra) {
 #pragma unroll

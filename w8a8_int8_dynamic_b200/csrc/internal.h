@@ -74,6 +74,7 @@ w8a8_status launch_gemm2sm(const int8_t *q, const float *a_scale, const void *pa
                            int act = W8A8_ACT_NONE, void *workspace = nullptr,
                            size_t ws_bytes = 0);
 int64_t pair_tiles(int64_t M, int64_t N, int bn);
+int64_t pair_full_tiles(int64_t tiles, int64_t pairs);
 // Workspace the K-split (split = 2) or stream-K (split = 3) pair kernel needs
 // (sync words + int32 partials).
 int64_t split_workspace_bytes(int64_t M, int64_t N, int split);
