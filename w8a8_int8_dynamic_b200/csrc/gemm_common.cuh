@@ -112,7 +112,7 @@ __device__ __forceinline__ uint4 epilogue8(const GemmArgs &a, const uint32_t *v,
   }
   if (a.act != W8A8_ACT_NONE) {
 #pragma unroll
-    for (int h = 0; h < 8; ++h) t[h] = apply_act(t[h], a.act);
+    for (int h = 0; h < 4; ++h) apply_act_pair(t[2 * h], t[2 * h + 1], a.act);
   }
   return make_uint4(pack_bf16x2(t[0], t[1]), pack_bf16x2(t[2], t[3]), pack_bf16x2(t[4], t[5]),
                     pack_bf16x2(t[6], t[7]));
