@@ -1,5 +1,7 @@
 // gemm.cu -- int8 x int8 -> int32 GEMM on the sm_100a tensor cores with the
-// dequantising epilogue, plus the fused quantise+GEMM layer entry point.
+// dequantising epilogue; the kernel choice for large M; and the C entry points
+// of the GEMM and of the whole layer (quantisation kernel, then the GEMM as a
+// programmatic dependent launch).
 //
 // Source: "Issue 5 probe: int8 quantized DiT serve paths on the RTX 3090",
 // Round two: the cutlass_scaled_mm op (int8 activations x int8 weights,
@@ -11,18 +13,23 @@
 //   acc[m,n] = sum_k q[m,k] w[n,k]                     (exact int32, TMEM)
 //   y[m,n]   = bf16_rne(((float)acc * a_scale[m]) * w_scale[n] + bias[n])
 //
-// Two kernels share the tile image, descriptors and epilogue arithmetic:
-//
-// 1. gemm_kernel (large M): persistent, one CTA per SM, 192 threads.
-//    warp 0: producer -- TMA 2-D load of the q tile (128 rows x 128 bytes,
-//            128-byte swizzle) and a 16 KB bulk copy per 128-row weight slab
-//            from the packed image, onto a STAGES-deep mbarrier ring;
+// 1. gemm_kernel (large M): persistent, one CTA per SM, 320 threads.
+//    warp 0: producer -- per stage of KPS k-blocks, TMA 2-D loads of the q
+//            tiles (128 rows x 128 bytes, 128-byte swizzle) and one bulk copy
+//            of the KPS contiguous weight tiles of each 128-row slab from the
+//            packed image, onto a STAGES-deep mbarrier ring.  Behind the
+//            quantisation kernel it first issues the weight copies of the
+//            first stages and an L2 prefetch of more of its slab, then waits
+//            for the codes;
 //    warp 1: MMA issuer -- 4 x tcgen05.mma.kind::i8 (M=128, N=BN, K=32) per
-//            stage, int32 accumulators in TMEM, double-buffered so the
+//            k-block, int32 accumulators in TMEM, double-buffered so the
 //            epilogue of tile i overlaps the main loop of tile i+1;
-//    warps 2-5: epilogue -- tcgen05.ld of 32 columns at a time, the scale /
-//            bias arithmetic in fp32 (each step rounded separately, so the
-//            result is bit-identical to the definition), bf16 stores.
+//    warps 2-9: epilogue -- two warps per TMEM lane quarter, half the columns
+//            each; tcgen05.ld of 32 columns at a time with the next load in
+//            flight, the scale / bias (/ GELU) arithmetic in fp32 (each step
+//            rounded separately, so the result is bit-identical to the
+//            definition), bf16 through swizzled shared-memory boxes and TMA
+//            stores.
 // 2. The 2-SM pair kernel (gemm2sm.cu) and the small-M weight-streaming
 //    kernel (decode.cu) share the tile image and epilogue arithmetic.
 //

@@ -9,9 +9,10 @@
 //             q = clamp(rint_half_even(x / s), -127, 127);  amax == 0 -> s = 0, q = 0.
 //
 // Each row is handled by W warps (W = 1 for rows of up to 1024 elements,
-// more for longer rows), each lane holding up to 4 16-byte chunks of the row
-// in registers (8 or 16 for rows longer than 16384), all loaded at once with
-// 128-bit streaming loads: the row is read exactly once and many loads are in
+// more for longer rows), each lane holding 4 16-byte chunks of the row in
+// registers (8 when the input has enough rows that fewer, fatter warps pay;
+// 16 for rows too long for 16 warps), all loaded at once with 128-bit
+// streaming loads: the row is read exactly once and many loads are in
 // flight per warp.  The row
 // maximum is a packed 16-bit integer max on the bf16 magnitudes (|x| order
 // equals the order of the 15 low bits for finite bf16), reduced with warp
@@ -26,9 +27,8 @@
 // decode GEMM releases its dependents early), and wait on the device for it
 // to complete before reading x, which may be that kernel's output.
 //
-// The per-element arithmetic (the exact quotient by reciprocal refinement,
-// rint by one addition) is in quant_common.cuh, shared with the GEMM that
-// quantises its own rows.
+// The per-element arithmetic (the code from one step of reciprocal
+// refinement, rint by one addition) is in quant_common.cuh.
 #include <cuda_bf16.h>
 
 #include <algorithm>
