@@ -93,6 +93,28 @@ def test_dit_mlp_up_fused_gelu_full_size():
     assert torch.equal(g_fused, g_chain)
 
 
+def test_gelu_epilogue_on_half_tiles():
+    """A shape whose last round of 256 x 256 pair tiles runs as 256 x 128
+    halves (99 tiles on 74 pairs; the last tile ragged in M and N): the GELU
+    epilogue on the halves equals the layer followed by the GELU kernel, bit
+    for bit, and the oracle's chain within one bf16 ulp."""
+    M, N, K = 600, 8200, 400
+    pairs = torch.cuda.get_device_properties(0).multi_processor_count // 2
+    tiles = ((M + 255) // 256) * ((N + 255) // 256)
+    if not (tiles > pairs and 0 < tiles % pairs <= pairs // 2):
+        pytest.skip(f"{tiles} tiles on {pairs} SM pairs leave no short last round")
+    inp, q_ref, s_ref, y_ref = _case(M, N, K, True, 41)
+    args = (dev(q_ref), dev(s_ref), w8.pack_weight(dev(inp.w)), dev(inp.w_scale),
+            dev_bf16(inp.bias), N)
+    y = w8.scaled_mm(*args)
+    g_chain = w8.gelu_tanh(y)
+    g_fused = w8.scaled_mm(*args, act=w8.ACT_GELU_TANH)
+    torch.cuda.synchronize()
+    assert np.array_equal(host_u16(y), y_ref)
+    assert torch.equal(g_fused, g_chain)
+    assert_bf16_close(host_u16(g_fused), oracle.gelu_tanh(y_ref), max_ulp=1, what="gelu")
+
+
 def test_act_rejects_unknown_value():
     inp, q_ref, s_ref, _ = _case(64, 128, 256, False, 1)
     with pytest.raises(w8.W8A8Error):

@@ -294,7 +294,7 @@ def test_gelu_within_one_ulp():
 
 
 # ---------------------------------------------------------------- CUDA graph replay
-@pytest.mark.parametrize("case", ["layer", "decode_layer", "k_split", "stream_k"])
+@pytest.mark.parametrize("case", ["layer", "decode_layer", "k_split", "stream_k", "tail_split"])
 def test_cuda_graph_replay_with_new_inputs(case):
     """Kernels that count CTAs on call-tagged workspace words (the small-M
     kernel's slab reduction, the K-split handoff) see the same tag on every
@@ -303,7 +303,8 @@ def test_cuda_graph_replay_with_new_inputs(case):
     the captured buffers, each replay checked against the oracle bit for bit
     (the large-M layer, quantisation + GEMM, alongside)."""
     M, N, K = {"layer": (512, 1024, 1024), "decode_layer": (4, 2056, 1040),
-               "k_split": (512, 1024, 4096), "stream_k": (1000, 2056, 1040)}[case]
+               "k_split": (512, 1024, 4096), "stream_k": (1000, 2056, 1040),
+               "tail_split": (600, 8200, 400)}[case]
     if case == "k_split":
         w8.set_path(w8.PATH_LARGE_PAIR_SPLIT)
     if case == "stream_k":
