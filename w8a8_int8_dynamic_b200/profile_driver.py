@@ -1,6 +1,6 @@
 """Run one workload's kernels a few times, for profiling under ncu.
 
-    python -m w8a8_int8_dynamic_b200.profile_driver <workload> <reps> [gemm|decode|quant|linear]
+    python -m w8a8_int8_dynamic_b200.profile_driver <workload> <reps> [gemm|decode|quant|linear|gelu]
 
 Draws the workload's seeded inputs, packs the weights, then launches the
 quantisation and the GEMM `reps` times (no CUDA graphs, so each kernel is a
@@ -29,8 +29,14 @@ def main(argv):
                        device="cuda")
     y = torch.empty((wl.M, wl.N), dtype=torch.bfloat16, device="cuda")
     layer_ws = torch.empty(w8.linear_workspace_bytes(wl.M, wl.N, wl.K), dtype=torch.uint8, device="cuda")
+    g_in = None
+    if mode == "gelu":  # the GELU kernel over an [M, N] activation (the MLP's up output)
+        g_in = torch.randn(wl.M, wl.N, device="cuda",
+                           generator=torch.Generator("cuda").manual_seed(0)).to(torch.bfloat16)
     for _ in range(reps):
-        if mode == "linear":
+        if mode == "gelu":
+            w8.gelu_tanh(g_in, out=y)
+        elif mode == "linear":
             w8.linear(x, packed, ws, b, wl.N, out=y, workspace=layer_ws)
         else:
             w8.quant_act(x, q=q, a_scale=a)
