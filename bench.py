@@ -190,11 +190,19 @@ class LayerSets:
 
 
 def sets_needed(w8, wl, M=None):
+    """Input sets to rotate over so that every timed loop -- the layer, the
+    GEMM alone, the quantisation alone -- touches more than L2 (x 1.5)
+    between two uses of the same set.  A quantisation too small to exceed L2
+    even over 16 sets (it is latency-bound then) does not count."""
     probe_M = wl.M if M is None else M
-    per = (probe_M * wl.K * 3 + wl.N * wl.K + 2 * probe_M * wl.N + 8 * wl.N
-           + w8.linear_workspace_bytes(probe_M, wl.N, wl.K))
+    M, N, K = probe_M, wl.N, wl.K
+    per = (M * K * 3 + N * K + 2 * M * N + 8 * N + w8.linear_workspace_bytes(M, N, K))
+    footprints = [per, M * K + N * K + 2 * M * N]  # the layer; the GEMM alone (q, W, y)
+    if 16 * 3 * M * K > 1.5 * L2_BYTES:
+        footprints.append(3 * M * K)  # the quantisation alone (x, q)
+    smallest = min(footprints)
     n = 1
-    while n * per <= 1.5 * L2_BYTES and n < 16:
+    while n * smallest <= 1.5 * L2_BYTES and n < 16:
         n += 1
     return n, per
 
@@ -240,7 +248,8 @@ def time_loop(loop, steps, stream):
 
 
 # ----------------------------------------------------------------------------- our arm
-def run_workload(w8, wl, steps, warmup, device, stream, M=None, with_quant=True):
+def run_workload(w8, wl, steps, warmup, device, stream, M=None, with_quant=True,
+                 gemm_clock_tag=None):
     nsets, _ = sets_needed(w8, wl, M)
     ls = LayerSets(w8, wl, nsets, device, M)
     steps_fns, mm_fns, q_fns = [], [], []
@@ -274,6 +283,15 @@ def run_workload(w8, wl, steps, warmup, device, stream, M=None, with_quant=True)
            "M": ls.M, "N": ls.N, "K": ls.K}
     res["t_step"] = time_loop(layer_loop, steps, stream) / steps
     res["t_gemm"] = time_loop(mm_loop, steps, stream) / steps
+    if gemm_clock_tag is not None:
+        # the GEMM alone again, long enough (>= 0.6 s) for the clock sampler:
+        # a tensor-bound loop may run under the power cap
+        per = mm_loop.per_graph
+        n = max(steps, int(0.6 / res["t_gemm"]) // per * per)
+        cs = ClockSampler(smi_index(device), tag=gemm_clock_tag)
+        cs.start()
+        res["t_gemm_long"] = time_loop(mm_loop, n, stream) / n
+        res["gemm_clock"] = cs.stop()
     if with_quant:
         res["t_quant"] = time_loop(q_loop, steps, stream) / steps
     assert w8.poll_status() == 0, "device-side timeout during the benchmark"
@@ -436,10 +454,11 @@ def sweep(w8, args, device, stream, peaks, int8_peak):
         wl = WORKLOADS[name]
         ops, gemm_bytes, quant_bytes, fused_bytes = algorithmic(wl)
         steps = 256 if wl.M * wl.N * wl.K > 1e11 else 2048
-        ls, loop, r = run_workload(w8, wl, steps, 3, device, stream)
+        bound = "tensor" if ops / (int8_peak * 1e12) >= gemm_bytes / (peaks["hbm_gbs"] * 1e9) else "hbm"
+        ls, loop, r = run_workload(w8, wl, steps, 3, device, stream,
+                                   gemm_clock_tag=("_gemm_" + name) if bound == "tensor" else None)
         t_roof_gemm = max(ops / (int8_peak * 1e12), gemm_bytes / (peaks["hbm_gbs"] * 1e9))
         t_roof_fused = max(ops / (int8_peak * 1e12), fused_bytes / (peaks["hbm_gbs"] * 1e9))
-        bound = "tensor" if ops / (int8_peak * 1e12) >= gemm_bytes / (peaks["hbm_gbs"] * 1e9) else "hbm"
         out[name] = {
             "M": wl.M, "N": wl.N, "K": wl.K, "bound": bound,
             "step_us": round(r["t_step"] * 1e6, 3), "gemm_us": round(r["t_gemm"] * 1e6, 3),
@@ -455,6 +474,16 @@ def sweep(w8, args, device, stream, peaks, int8_peak):
             "l2_sets": r["nsets"],
             "kernel": w8.gemm_kernel_name(wl.M, wl.N, wl.K),
         }
+        if "gemm_clock" in r:
+            # a long GEMM loop with its clocks: under the power cap the
+            # sustained bf16 rate (x 2 for int8) is the ceiling it can reach
+            sustained = 2.0 * peaks["bf16_tflops_sustained"]
+            tops_long = ops / r["t_gemm_long"] / 1e12
+            out[name]["gemm_long_loop"] = {
+                "us": round(r["t_gemm_long"] * 1e6, 3), "tops": round(tops_long, 1),
+                "sm_mhz": r["gemm_clock"]["sm_mhz"], "reasons": r["gemm_clock"]["reasons"],
+                "frac_of_sustained": round(tops_long / sustained, 4),
+                "sustained_peak_tops": round(sustained, 1)}
         del ls, loop
         torch.cuda.empty_cache()
     return out
