@@ -13,7 +13,7 @@ import torch
 
 import oracle
 import w8a8_int8_dynamic_b200 as w8
-from gpu_util import dev, dev_bf16, host_u16, require_gpu
+from gpu_util import assert_bf16_close, dev, dev_bf16, host_u16, require_gpu
 from w8a8_int8_dynamic_b200.workloads import random_case
 
 pytestmark = pytest.mark.gpu
@@ -99,3 +99,35 @@ def test_quant_after_decode_reads_its_output():
         torch.cuda.synchronize()
         assert np.array_equal(q2.cpu().numpy(), q2_ref)
         assert np.array_equal(s2.cpu().numpy(), s2_ref)
+
+
+@pytest.mark.parametrize("M", [4, 300])
+def test_mlp_block_chain(M):
+    """The MLP pattern: up-projection with the GELU epilogue, then the
+    down-projection on its output, queued back to back (the down-projection's
+    quantisation waits on the device for the up-projection).  The up output
+    is within one bf16 ulp of the oracle's GELU chain; the down-projection is
+    checked bit for bit against the oracle fed the GPU's own GELU output (the
+    two sides' GELU may differ by an ulp)."""
+    D, H = 1024, 2064
+    up = random_case(21 + M, M, H, D, bias=True, n_outliers=D // 64)
+    dn = random_case(22 + M, M, D, H, bias=True)
+    y_up_ref, *_ = oracle.linear(up.x, up.w, up.w_scale, up.bias)
+    g_ref = oracle.gelu_tanh(y_up_ref)
+    ws_up = torch.empty((w8.linear_workspace_bytes(M, H, D),), dtype=torch.uint8, device="cuda")
+    ws_dn = torch.empty((w8.linear_workspace_bytes(M, D, H),), dtype=torch.uint8, device="cuda")
+    p_up, p_dn = w8.pack_weight(dev(up.w)), w8.pack_weight(dev(dn.w))
+    x = dev_bf16(up.x)
+    g = torch.empty((M, H), dtype=torch.bfloat16, device="cuda")
+    y = torch.empty((M, D), dtype=torch.bfloat16, device="cuda")
+    for _ in range(3):
+        g.fill_(0)
+        y.fill_(0)
+        w8.linear(x, p_up, dev(up.w_scale), dev_bf16(up.bias), H, out=g, workspace=ws_up,
+                  act=w8.ACT_GELU_TANH)
+        w8.linear(g, p_dn, dev(dn.w_scale), dev_bf16(dn.bias), D, out=y, workspace=ws_dn)
+        torch.cuda.synchronize()
+        g_h = host_u16(g)
+        assert_bf16_close(g_h, g_ref, max_ulp=1, what="gelu chain")
+        y_ref, *_ = oracle.linear(g_h, dn.w, dn.w_scale, dn.bias)
+        assert np.array_equal(host_u16(y), y_ref)
