@@ -18,7 +18,8 @@ constexpr int kBK = 128;                 // bytes of K per pipeline stage
 constexpr int kTileBytes = 128 * kBK;    // one 128 x 128 int8 tile = 16 KB
 constexpr int kThreads = 192;            // small-M kernel: 6 warps
 constexpr int kDecodeNT = 16;            // activation rows per decode MMA (N)
-// Large-M kernels: warp 0 producer, warp 1 MMA issuer, warps 2..9 epilogue.
+// Large-M kernels: warp 1 MMA issuer, warps 2..9 epilogue, warp 0 idle, and
+// the producer alone in an eleventh, one-thread warp (block kGemmThreads + 1).
 // A warp may only read the TMEM lanes of its quarter (warp id mod 4), so the
 // eight epilogue warps form two per lane quarter, each draining half of the
 // tile's columns: two warps per SM sub-partition hide each other's latency.
