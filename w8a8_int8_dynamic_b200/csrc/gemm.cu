@@ -128,41 +128,58 @@ __global__ void __launch_bounds__(kGemmThreads + 1, 1)
   // reaches the block barrier below converged; the warp also owns the TMEM
   // allocation); warp 0 is idle.
   if (threadIdx.x == kGemmThreads) {
-    {
-      // ---------------- producer ----------------
-      auto stage_nk = [&](uint32_t it) { return min(KPS, num_kb - (int)(it % nsk) * KPS); };
-      auto weights = [&](uint32_t it, uint32_t s) {
-        const int tile = blockIdx.x + (int)(it / nsk) * gridDim.x;
-        const int nb = tile / args.tiles_m, kb0 = (int)(it % nsk) * KPS;
-        const int nk = stage_nk(it);
+    // ---------------- producer ----------------
+    // A cursor walks this CTA's stages in order; the divisions by runtime
+    // tile counts and the 64-bit slab offsets are taken once per tile, after
+    // a stage's copies are issued.  Between a slot's release and its refill
+    // only the copies themselves remain: the issuing thread is on the ring's
+    // critical path (a scratch microbenchmark of 64 KB stages moves 118 GB/s
+    // per SM with a 64-bit modulo per stage in that thread, 170 GB/s without).
+    const size_t slab_bytes = (size_t)num_kb * kTileBytes;  // one 128-row weight slab
+    struct Cursor {
+      int tile, j, q_row;       // tile index, stage within the tile, first q row
+      const uint8_t *w;         // the tile's first weight slab
+    };
+    auto at_tile = [&](int tile) {
+      Cursor c;
+      c.tile = tile;
+      c.j = 0;
+      c.q_row = (tile % args.tiles_m) * kBM;
+      c.w = args.packed_w + (size_t)(tile / args.tiles_m) * (BN / 128) * slab_bytes;
+      return c;
+    };
+    auto advance = [&](Cursor &c) {
+      if (++c.j == nsk) c = at_tile(c.tile + (int)gridDim.x);
+    };
+    auto stage_nk = [&](const Cursor &c) { return min(KPS, num_kb - c.j * KPS); };
+    auto weights = [&](const Cursor &c, uint32_t s, int nk) {
+      const uint8_t *src = c.w + (size_t)(c.j * KPS) * kTileBytes;
 #pragma unroll
-        for (int h = 0; h < BN / 128; ++h)
-          bulk_load(sB + s * L::kBStage + h * kTileBytes,
-                    args.packed_w + (((size_t)nb * (BN / 128) + h) * num_kb + kb0) * kTileBytes,
-                    (uint32_t)(nk * kTileBytes), &full[s]);
-      };
-      auto acts = [&](uint32_t it, uint32_t s) {
-        const int tile = blockIdx.x + (int)(it / nsk) * gridDim.x;
-        const int kb0 = (int)(it % nsk) * KPS;
-        const int nk = stage_nk(it);
-        for (int i = 0; i < nk; ++i)
-          tma_load_2d(sA + s * L::kAStage + i * kTileBytes, &tmap_q, (kb0 + i) * kBK,
-                      (tile % args.tiles_m) * kBM, &full[s]);
-      };
-      auto bytes = [&](uint32_t it) { return (uint32_t)(stage_nk(it) * (kTileBytes + BN * kBK)); };
-      uint32_t last_par[STAGES];
-      bool ok = true;
+      for (int h = 0; h < BN / 128; ++h)
+        bulk_load(sB + s * L::kBStage + h * kTileBytes, src + h * slab_bytes,
+                  (uint32_t)(nk * kTileBytes), &full[s]);
+    };
+    auto acts = [&](const Cursor &c, uint32_t s, int nk) {
+      for (int i = 0; i < nk; ++i)
+        tma_load_2d(sA + s * L::kAStage + i * kTileBytes, &tmap_q, (c.j * KPS + i) * kBK, c.q_row,
+                    &full[s]);
+    };
+    constexpr uint32_t kBytesPerKb = kTileBytes + BN * kBK;
+    const uint32_t pre = my_iters < (uint32_t)STAGES ? my_iters : (uint32_t)STAGES;
+    if (my_tiles > 0) {
+      Cursor cur = at_tile(blockIdx.x);
       // The weight tiles of the first stages do not depend on the preceding
       // kernel of the stream: issue them before waiting for it.
-      const uint32_t pre = my_iters < (uint32_t)STAGES ? my_iters : (uint32_t)STAGES;
+      const Cursor first = cur;
       for (uint32_t it = 0; it < pre; ++it) {
-        mbar_arrive_expect_tx(&full[it], bytes(it));
-        weights(it, it);
-        last_par[it] = 0;
+        const int nk = stage_nk(cur);
+        mbar_arrive_expect_tx(&full[it], (uint32_t)nk * kBytesPerKb);
+        weights(cur, it, nk);
+        advance(cur);
       }
-      if (args.prefetch_kb > 0 && my_tiles > 0) {
+      if (args.prefetch_kb > 0) {
         // CTAs blockIdx.x / tiles_m read the same slab: each warms its share.
-        const int nb = blockIdx.x / args.tiles_m, mb = blockIdx.x % args.tiles_m;
+        const int mb = blockIdx.x % args.tiles_m;
         const int kb_lo = STAGES * KPS, kb_hi = min(num_kb, kb_lo + args.prefetch_kb);
         if (kb_hi > kb_lo) {
           const int per = (kb_hi - kb_lo + args.tiles_m - 1) / args.tiles_m;
@@ -170,29 +187,43 @@ __global__ void __launch_bounds__(kGemmThreads + 1, 1)
           if (k1 > k0)
 #pragma unroll
             for (int h = 0; h < BN / 128; ++h)
-              bulk_prefetch_l2(
-                  args.packed_w + (((size_t)nb * (BN / 128) + h) * num_kb + k0) * kTileBytes,
-                  (uint32_t)((k1 - k0) * kTileBytes));
+              bulk_prefetch_l2(first.w + h * slab_bytes + (size_t)k0 * kTileBytes,
+                               (uint32_t)((k1 - k0) * kTileBytes));
         }
       }
       griddep_wait();
-      for (uint32_t it = 0; it < pre; ++it) acts(it, it);
-      for (uint32_t it = pre; it < my_iters; ++it) {
-        const uint32_t s = it % STAGES, ph = (it / STAGES) & 1;
+      {
+        Cursor c = first;
+        for (uint32_t it = 0; it < pre; ++it) {
+          acts(c, it, stage_nk(c));
+          advance(c);
+        }
+      }
+      uint32_t issued = pre, s = 0, ph = 1;  // stage `pre` (if any) reuses slot 0, second round
+      bool ok = true;
+      for (; issued < my_iters; ++issued) {
+        const int nk = stage_nk(cur);
+        const uint32_t bytes = (uint32_t)nk * kBytesPerKb;
         if (!mbar_wait(&empty[s], ph ^ 1, abort_flag, args.status)) {
           ok = false;
           break;
         }
-        mbar_arrive_expect_tx(&full[s], bytes(it));
-        acts(it, s);
-        weights(it, s);
-        last_par[s] = ph;
+        mbar_arrive_expect_tx(&full[s], bytes);
+        acts(cur, s, nk);
+        weights(cur, s, nk);
+        advance(cur);
+        if (++s == (uint32_t)STAGES) {
+          s = 0;
+          ph ^= 1;
+        }
       }
       if (!ok) {
-        // Drain: wait (bounded) for the copies still in flight into our smem.
-        for (uint32_t s = 0; s < (uint32_t)STAGES && s < my_iters; ++s) {
+        // Drain: wait (bounded) for the copies still in flight into our smem:
+        // the last stage issued into each slot.
+        for (uint32_t sl = 0; sl < (uint32_t)STAGES && sl < issued; ++sl) {
+          const uint32_t last = sl + ((issued - 1 - sl) / STAGES) * STAGES;
           volatile int no_abort = 0;
-          (void)mbar_wait_bounded(&full[s], last_par[s], &no_abort, args.status);
+          (void)mbar_wait_bounded(&full[sl], (last / STAGES) & 1, &no_abort, args.status);
         }
       }
     }
@@ -201,7 +232,11 @@ __global__ void __launch_bounds__(kGemmThreads + 1, 1)
   } else if (warp == 1) {
     if (lane == 0) {
       // ---------------- MMA issuer ----------------
-      uint32_t it = 0;
+      // Slot, phase and operand descriptors advance by counters, so a full
+      // stage is answered by its MMAs at once.  A descriptor's address field
+      // is the shared-memory address / 16, linear below 256 KB.
+      const uint64_t a_desc0 = sw128_kmajor_desc(sA), b_desc0 = sw128_kmajor_desc(sB);
+      uint32_t s = 0, ph = 0;
       bool ok = true;
       for (int t = 0; ok && t < my_tiles; ++t) {
         const uint32_t b = t & 1, bph = (t >> 1) & 1;
@@ -211,22 +246,26 @@ __global__ void __launch_bounds__(kGemmThreads + 1, 1)
         }
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + b * BN;
-        for (int j = 0; j < nsk; ++j, ++it) {
-          const uint32_t s = it % STAGES, ph = (it / STAGES) & 1;
+        for (int j = 0; j < nsk; ++j) {
+          const int nk = min(KPS, num_kb - j * KPS);
+          const uint64_t a_desc = a_desc0 + ((s * L::kAStage) >> 4);
+          const uint64_t b_desc = b_desc0 + ((s * L::kBStage) >> 4);
           if (!mbar_wait(&full[s], ph, abort_flag, args.status)) {
             ok = false;
             break;
           }
           tc_fence_after();
-          const int nk = min(KPS, num_kb - j * KPS);
           for (int i = 0; i < nk; ++i) {
-            const uint64_t a_desc = sw128_kmajor_desc(sA + s * L::kAStage + i * kTileBytes);
-            const uint64_t b_desc = sw128_kmajor_desc(sB + s * L::kBStage + i * BN * kBK);
 #pragma unroll
             for (int k = 0; k < kBK / 32; ++k)
-              mma_i8(d_tmem, a_desc + 2 * k, b_desc + 2 * k, kIdesc, (j | i | k) != 0);
+              mma_i8(d_tmem, a_desc + ((i * kTileBytes) >> 4) + 2 * k,
+                     b_desc + ((i * BN * kBK) >> 4) + 2 * k, kIdesc, (j | i | k) != 0);
           }
           mma_commit(&empty[s]);  // frees the stage when these MMAs finish
+          if (++s == (uint32_t)STAGES) {
+            s = 0;
+            ph ^= 1;
+          }
         }
         if (ok) mma_commit(&tfull[b]);
       }

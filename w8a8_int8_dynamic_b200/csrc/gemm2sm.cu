@@ -209,88 +209,125 @@ __global__ void __launch_bounds__(kGemmThreads + 1, 1)
   // loop (fused QKV 28.7 -> 28.0 us); lane 0 of warp 1 issues the MMAs; warp
   // 0 is idle.
   if (threadIdx.x == kGemmThreads) {
-    {
-      // ---------------- producer (every CTA) ----------------
-      auto issue = [&](int item, int st, uint32_t s, bool weights, bool acts) {
-        const int tile = item_tile(item), half = item_half(item);
-        const int mb = tile % args.tiles_m, nb = tile / args.tiles_m;
-        const int kb0 = st * kStageK;
-        const int nk = min(kStageK, num_kb - kb0);
-        const uint32_t bar = full0 + s * 8;
-        if (weights) {
-          if (BN == 256 && half >= 0) {
-            // this CTA's 64-row half of slab 2 nb + half, per k-block
-            for (int h = 0; h < nk; ++h)
-              tma_load_2d_pair(sB + s * L::kBStage + h * kHalfBTile, &tmap_w64, 0,
-                               ((nb * 2 + half) * num_kb + kb0 + h) * 128 + (int)rank * 64, bar);
-          } else if (BN == 256) {
-            // two contiguous packed tiles (k-blocks kb0, kb0+1) of this CTA's slab
-            const int wslab = nb * 2 + (int)rank;
-            tma_load_2d_pair(sB + s * L::kBStage, &tmap_w, 0, (wslab * num_kb + kb0) * 128, bar);
-          } else {
-            // this CTA's 64-row half of each of the two tiles of slab nb
-            for (int h = 0; h < nk; ++h)
-              tma_load_2d_pair(sB + s * L::kBStage + h * L::kBTile, &tmap_w, 0,
-                               (nb * num_kb + kb0 + h) * 128 + (int)rank * 64, bar);
-          }
-        }
-        if (acts) {
-          const int row0 = mb * 256 + (int)rank * 128;
-          for (int h = 0; h < nk; ++h)
-            tma_load_2d_pair(sA + s * kHalfStage + h * kTileBytes, &tmap_q, (kb0 + h) * kBK, row0,
-                             bar);
-        }
-      };
-      auto stage_bytes = [&](int item, int st) {
-        const int nk = min(kStageK, num_kb - st * kStageK);
-        // the 256-wide weight box always moves two tiles (zero-filled past the end)
-        const int wb = BN == 256 ? (item_half(item) >= 0 ? nk * kHalfBTile : L::kBStage)
-                                 : nk * L::kBTile;
-        return (uint32_t)(nk * kTileBytes + wb);
-      };
-      // cursor over (segment, stage) in the order the MMAs consume them
-      int ci = 0, cst = nseg > 0 ? seg_begin(0) : 0;
-      auto advance = [&]() {
-        if (++cst >= seg_end(ci) && ++ci < nseg) cst = seg_begin(ci);
-      };
-      uint32_t last_par[STAGES];
-      int pre_tile[STAGES], pre_st[STAGES];
-      bool ok = true;
-      const uint32_t pre = my_iters < (uint32_t)STAGES ? my_iters : (uint32_t)STAGES;
+    // ---------------- producer (every CTA) ----------------
+    // A cursor walks this CTA's (segment, stage) list in the order the MMAs
+    // consume it.  A segment's box coordinates (divisions by the runtime tile
+    // counts) are formed when the cursor enters it, after the previous
+    // stage's copies are issued, so a released slot is refilled with the
+    // copies alone (the issuing thread is on the ring's critical path).
+    struct Cursor {
+      int seg, st;  // segment index, stage within the tile
+      int kind;     // 0: 256 x BN tile, 1: 256 x 128 half of a 256-wide tile
+      int wrow;     // weight box row of k-block 0 (plus 128 per k-block)
+      int qrow;     // first q row of this CTA
+    };
+    auto enter = [&](int i, int st) {
+      Cursor c;
+      c.seg = i;
+      c.st = st;
+      if (i >= nseg) {
+        c.kind = 0;
+        c.wrow = c.qrow = 0;
+        return c;
+      }
+      const int item = seg_tile(i), tile = item_tile(item), half = item_half(item);
+      const int mb = tile % args.tiles_m, nb = tile / args.tiles_m;
+      c.kind = (BN == 256 && half >= 0) ? 1 : 0;
+      c.qrow = mb * 256 + (int)rank * 128;
+      if (BN == 256 && half >= 0)
+        c.wrow = (nb * 2 + half) * num_kb * 128 + (int)rank * 64;  // this CTA's 64 rows
+      else if (BN == 256)
+        c.wrow = (nb * 2 + (int)rank) * num_kb * 128;  // this CTA's 128-row slab
+      else
+        c.wrow = nb * num_kb * 128 + (int)rank * 64;  // this CTA's 64 rows of slab nb
+      return c;
+    };
+    auto advance = [&](Cursor &c) {
+      if (++c.st >= seg_end(c.seg)) c = enter(c.seg + 1, c.seg + 1 < nseg ? seg_begin(c.seg + 1) : 0);
+    };
+    auto stage_nk = [&](const Cursor &c) { return min(kStageK, num_kb - c.st * kStageK); };
+    auto stage_bytes = [&](const Cursor &c, int nk) {
+      // the 256-wide weight box always moves two tiles (zero-filled past the end)
+      const int wb = BN == 256 ? (c.kind == 1 ? nk * kHalfBTile : L::kBStage) : nk * L::kBTile;
+      return (uint32_t)(nk * kTileBytes + wb);
+    };
+    auto weights = [&](const Cursor &c, uint32_t s, int nk) {
+      const uint32_t bar = full0 + s * 8;
+      const int row = c.wrow + c.st * kStageK * 128;
+      if (BN == 256 && c.kind == 0) {
+        // two contiguous packed tiles (k-blocks kb0, kb0+1) of this CTA's slab
+        tma_load_2d_pair(sB + s * L::kBStage, &tmap_w, 0, row, bar);
+      } else {
+        const int step = (BN == 256) ? kHalfBTile : L::kBTile;
+        for (int h = 0; h < nk; ++h)
+          tma_load_2d_pair(sB + s * L::kBStage + h * step, BN == 256 ? &tmap_w64 : &tmap_w, 0,
+                           row + h * 128, bar);
+      }
+    };
+    auto acts = [&](const Cursor &c, uint32_t s, int nk) {
+      const uint32_t bar = full0 + s * 8;
+      for (int h = 0; h < nk; ++h)
+        tma_load_2d_pair(sA + s * kHalfStage + h * kTileBytes, &tmap_q, (c.st * kStageK + h) * kBK,
+                         c.qrow, bar);
+    };
+    const uint32_t pre = my_iters < (uint32_t)STAGES ? my_iters : (uint32_t)STAGES;
+    uint32_t issued = 0;
+    bool ok = true;
+    if (my_iters > 0) {
+      Cursor cur = enter(0, seg_begin(0));
+      const Cursor first = cur;
       // weight tiles do not depend on the preceding kernel: issue them first
-      for (uint32_t it = 0; it < pre; ++it, advance()) {
-        pre_tile[it] = seg_tile(ci);
-        pre_st[it] = cst;
-        mbar_arrive_expect_tx_cluster(full0 + it * 8, stage_bytes(pre_tile[it], cst));
-        issue(pre_tile[it], cst, it, true, false);
-        last_par[it] = 0;
+      for (uint32_t it = 0; it < pre; ++it) {
+        const int nk = stage_nk(cur);
+        mbar_arrive_expect_tx_cluster(full0 + it * 8, stage_bytes(cur, nk));
+        weights(cur, it, nk);
+        advance(cur);
       }
       griddep_wait();
-      for (uint32_t it = 0; it < pre; ++it) issue(pre_tile[it], pre_st[it], it, false, true);
-      for (uint32_t it = pre; it < my_iters; ++it, advance()) {
-        const uint32_t s = it % STAGES, ph = (it / STAGES) & 1;
+      {
+        Cursor c = first;
+        for (uint32_t it = 0; it < pre; ++it) {
+          acts(c, it, stage_nk(c));
+          advance(c);
+        }
+      }
+      uint32_t s = 0, ph = 1;  // stage `pre` (if any) reuses slot 0, second round
+      for (issued = pre; issued < my_iters; ++issued) {
+        const int nk = stage_nk(cur);
+        const uint32_t bytes = stage_bytes(cur, nk);
         if (!mbar_wait(&empty[s], ph ^ 1, abort_flag, args.status)) {
           ok = false;
           break;
         }
-        mbar_arrive_expect_tx_cluster(full0 + s * 8, stage_bytes(seg_tile(ci), cst));
-        issue(seg_tile(ci), cst, s, true, true);
-        last_par[s] = ph;
-      }
-      // Wait until every stage this CTA filled has been consumed: the MMA
-      // commits that release them also arrive here, and must land before the
-      // CTA may leave.
-      for (uint32_t s = 0; s < (uint32_t)STAGES && s < my_iters; ++s) {
-        volatile int no_abort = 0;
-        if (ok) (void)mbar_wait_bounded(&empty[s], last_par[s], &no_abort, args.status);
+        mbar_arrive_expect_tx_cluster(full0 + s * 8, bytes);
+        weights(cur, s, nk);
+        acts(cur, s, nk);
+        advance(cur);
+        if (++s == (uint32_t)STAGES) {
+          s = 0;
+          ph ^= 1;
+        }
       }
     }
+    // Wait until every stage this CTA filled has been consumed: the MMA
+    // commits that release them also arrive here, and must land before the
+    // CTA may leave.  The last stage issued into slot sl has parity
+    // (last / STAGES) & 1.
+    if (ok)
+      for (uint32_t sl = 0; sl < (uint32_t)STAGES && sl < issued; ++sl) {
+        const uint32_t last = sl + ((issued - 1 - sl) / STAGES) * STAGES;
+        volatile int no_abort = 0;
+        (void)mbar_wait_bounded(&empty[sl], (last / STAGES) & 1, &no_abort, args.status);
+      }
   } else if (warp == 0) {
     // idle
   } else if (warp == 1) {
     if (lane == 0 && rank == 0) {
       // ---------------- MMA issuer (even CTA of each pair) ----------------
-      uint32_t it = 0;
+      // Slot, phase and operand descriptors advance by counters (a
+      // descriptor's address field is the shared-memory address / 16).
+      const uint64_t a_desc0 = sw128_kmajor_desc(sA), b_desc0 = sw128_kmajor_desc(sB);
+      uint32_t s = 0, ph = 0;
       bool ok = true;
       for (int i = 0; ok && i < nseg; ++i) {
         const uint32_t b = i & 1, bph = (i >> 1) & 1;
@@ -304,23 +341,27 @@ __global__ void __launch_bounds__(kGemmThreads + 1, 1)
         const bool half = BN == 256 && item_half(seg_tile(i)) >= 0;
         const uint32_t idesc = half ? kIdescHalf : kIdesc;
         const int b_step = half ? kHalfBTile : L::kBTile;
-        for (int st = sb; st < se; ++st, ++it) {
-          const uint32_t s = it % STAGES, ph = (it / STAGES) & 1;
+        for (int st = sb; st < se; ++st) {
+          const int nk = min(kStageK, num_kb - st * kStageK);
+          const uint64_t a_desc = a_desc0 + ((s * kHalfStage) >> 4);
+          const uint64_t b_desc = b_desc0 + ((s * L::kBStage) >> 4);
           if (!mbar_wait(&full[s], ph, abort_flag, args.status)) {
             ok = false;
             break;
           }
           tc_fence_after();
-          const int nk = min(kStageK, num_kb - st * kStageK);
           for (int h = 0; h < nk; ++h) {
-            const uint64_t a_desc = sw128_kmajor_desc(sA + s * kHalfStage + h * kTileBytes);
-            const uint64_t b_desc = sw128_kmajor_desc(sB + s * L::kBStage + h * b_step);
 #pragma unroll
             for (int k = 0; k < kBK / 32; ++k)
-              mma_i8_pair(d_tmem, a_desc + 2 * k, b_desc + 2 * k, idesc,
+              mma_i8_pair(d_tmem, a_desc + ((h * kTileBytes) >> 4) + 2 * k,
+                          b_desc + ((h * b_step) >> 4) + 2 * k, idesc,
                           (st != sb) || h != 0 || k != 0);
           }
           mma_commit_pair(&empty[s], pair_mask);  // frees the stage in both CTAs
+          if (++s == (uint32_t)STAGES) {
+            s = 0;
+            ph ^= 1;
+          }
         }
         if (ok) mma_commit_pair(&tfull[b], pair_mask);
       }
