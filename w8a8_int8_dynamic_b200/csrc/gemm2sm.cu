@@ -88,8 +88,11 @@ struct PartialLoad {
   }
 };
 
+// At most kGemmRegs registers a thread, so that a CTA (11 warps) fits on an
+// SM beside the blocks of the quantisation kernel it is launched behind and
+// starts its prologue and first weight copies while they run.
 template <int BN, int STAGES, int SPLIT>
-__global__ void __launch_bounds__(kGemmThreads + 1, 1)
+__global__ void __maxnreg__(kGemmRegs)
     gemm2sm_kernel(const __grid_constant__ CUtensorMap tmap_q,
                    const __grid_constant__ CUtensorMap tmap_w,
                    const __grid_constant__ CUtensorMap tmap_w64,

@@ -25,6 +25,10 @@ constexpr int kDecodeNT = 16;            // activation rows per decode MMA (N)
 // tile's columns: two warps per SM sub-partition hide each other's latency.
 constexpr int kEpiWarps = 8;
 constexpr int kGemmThreads = 64 + 32 * kEpiWarps;
+// Register cap of the large-M GEMM kernels: 128 x 32 x 11 warps = 45,056 of an
+// SM's 65,536 registers, which leaves room for four 4-warp quantisation blocks
+// of 40 registers (20,480) on the same SM.
+constexpr int kGemmRegs = 128;
 
 struct GemmArgs {
   const uint8_t *packed_w;

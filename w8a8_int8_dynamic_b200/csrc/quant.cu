@@ -223,10 +223,31 @@ __global__ void __launch_bounds__(256) quant_static_kernel(const uint16_t *__res
   }
 }
 
-// Launches k as a programmatic dependent of the preceding kernel of the stream.
+// Every SM that runs quantisation blocks is set up for the largest shared
+// memory share.  The GEMM launched behind them needs about 214 KB of shared
+// memory a CTA; an SM configured for a small share (the default for a kernel
+// that uses 64 bytes) takes such a CTA only after it has drained, so the GEMM
+// would start no earlier than the quantisation ends.
+bool g_carveout_done[64][8];
+
+template <typename Kernel>
+void prefer_max_shared(Kernel k, int slot) {
+  const int d = current_device();
+  if (d >= 0 && d < 64 && g_carveout_done[d][slot]) return;
+  if (cudaFuncSetAttribute(k, cudaFuncAttributePreferredSharedMemoryCarveout,
+                           (int)cudaSharedmemCarveoutMaxShared) == cudaSuccess) {
+    if (d >= 0 && d < 64) g_carveout_done[d][slot] = true;
+  } else {
+    (void)cudaGetLastError();  // a preference only: the launch goes ahead without it
+  }
+}
+
+// Launches k as a programmatic dependent of the preceding kernel of the
+// stream.  `slot` names k for the one-time carveout setting.
 template <typename... Params, typename... Args>
-cudaError_t launch_dependent(void (*k)(Params...), dim3 grid, dim3 block, cudaStream_t stream,
-                             Args... args) {
+cudaError_t launch_dependent(void (*k)(Params...), int slot, dim3 grid, dim3 block,
+                             cudaStream_t stream, Args... args) {
+  prefer_max_shared(k, slot);
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = grid;
   cfg.blockDim = block;
@@ -268,23 +289,23 @@ w8a8_status launch_quant(const void *x, int64_t M, int64_t K, int64_t ldx, int8_
   const int64_t W = (nchunks + 32 * cpl - 1) / (32 * cpl);
   cudaError_t e = cudaSuccess;
   if (W > 16) {
-    e = launch_dependent(quant_rows_two_pass_kernel, dim3((unsigned)M), dim3(1024), stream, xp,
+    e = launch_dependent(quant_rows_two_pass_kernel, 5, dim3((unsigned)M), dim3(1024), stream, xp,
                          ldx, (int)K, q, a_scale);
   } else {
     const int R = W >= 4 ? 1 : (int)(4 / W);  // rows per CTA: about 128 threads
     const unsigned grid = (unsigned)((M + R - 1) / R);
     const unsigned threads = (unsigned)(32 * W * R);
     switch (cpl) {
-#define W8A8_QUANT_CASE(C)                                                                   \
+#define W8A8_QUANT_CASE(C, SLOT)                                                             \
   case C:                                                                                    \
-    e = launch_dependent(quant_warps_kernel<C>, dim3(grid), dim3(threads), stream, xp, ldx, \
-                         (int)M, (int)K, (int)W, R, q, a_scale);                             \
+    e = launch_dependent(quant_warps_kernel<C>, SLOT, dim3(grid), dim3(threads), stream, xp, \
+                         ldx, (int)M, (int)K, (int)W, R, q, a_scale);                        \
     break;
-      W8A8_QUANT_CASE(1)
-      W8A8_QUANT_CASE(2)
-      W8A8_QUANT_CASE(4)
-      W8A8_QUANT_CASE(8)
-      W8A8_QUANT_CASE(16)
+      W8A8_QUANT_CASE(1, 0)
+      W8A8_QUANT_CASE(2, 1)
+      W8A8_QUANT_CASE(4, 2)
+      W8A8_QUANT_CASE(8, 3)
+      W8A8_QUANT_CASE(16, 4)
 #undef W8A8_QUANT_CASE
       default:
         return W8A8_ERR_INVALID_ARG;
@@ -321,6 +342,7 @@ extern "C" w8a8_status w8a8_quant_act_static(const void *x, int64_t M, int64_t K
     return W8A8_ERR_ALIGNMENT;
   const int64_t chunks = M * (K / 16);
   const int64_t blocks = std::min<int64_t>((chunks + 255) / 256, (int64_t)sm_count() * 8);
+  prefer_max_shared(quant_static_kernel, 6);
   quant_static_kernel<<<(unsigned)blocks, 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
       static_cast<const uint16_t *>(x), ldx, M, (int)K, scale, q, a_scale);
   count_launch();
