@@ -635,7 +635,7 @@ w8a8_status w8a8_linear_act(const void *x, int64_t ldx, const void *packed_w,
   int8_t *q = reinterpret_cast<int8_t *>(ws);
   float *a_scale = reinterpret_cast<float *>(ws + round_up(M * K, 256));
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  st = launch_quant(x, M, K, ldx, q, a_scale, s);
+  st = launch_quant(x, M, K, ldx, q, a_scale, s, true);
   if (st != W8A8_OK) return st;
   if (use_decode_path(M)) {
     void *dws = ws + round_up(M * K, 256) + round_up(M * 4, 256);

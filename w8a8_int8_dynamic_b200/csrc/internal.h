@@ -85,8 +85,9 @@ w8a8_status launch_decode(const int8_t *q, const float *a_scale, const void *pac
                           const float *w_scale, const void *bias, void *y, int64_t M,
                           int64_t N, int64_t K, void *workspace, cudaStream_t stream, bool pdl,
                           int act = W8A8_ACT_NONE);
-// Quantisation launcher (quant.cu).
+// Quantisation launcher (quant.cu).  ahead_of_gemm: the launch is followed by
+// a GEMM launched as its programmatic dependent (the layer).
 w8a8_status launch_quant(const void *x, int64_t M, int64_t K, int64_t ldx, int8_t *q,
-                         float *a_scale, cudaStream_t stream);
+                         float *a_scale, cudaStream_t stream, bool ahead_of_gemm);
 
 }  // namespace w8a8
