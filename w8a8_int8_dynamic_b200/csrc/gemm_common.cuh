@@ -26,8 +26,10 @@ constexpr int kDecodeNT = 16;            // activation rows per decode MMA (N)
 constexpr int kEpiWarps = 8;
 constexpr int kGemmThreads = 64 + 32 * kEpiWarps;
 // Register cap of the large-M GEMM kernels: 128 x 32 x 11 warps = 45,056 of an
-// SM's 65,536 registers, which leaves room for four 4-warp quantisation blocks
-// of 40 registers (20,480) on the same SM.
+// SM's 65,536 registers.  The 20,480 left hold four 4-warp quantisation
+// blocks of 40 registers on paper; measured, a GEMM CTA starts early on SMs
+// that hold three of them (most SMs, for 512 rows of 4096), not on those with
+// four.
 constexpr int kGemmRegs = 128;
 
 struct GemmArgs {

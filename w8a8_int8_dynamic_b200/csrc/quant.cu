@@ -113,8 +113,7 @@ __global__ void __launch_bounds__(512) quant_warps_kernel(const uint16_t *__rest
 }
 
 // Rows longer than 65536 elements: two passes over the row (the second one
-// hits L2), same arithmetic.  AHEAD as for quant_warps_kernel.
-template <bool AHEAD>
+// hits L2), same arithmetic.
 __global__ void __launch_bounds__(1024) quant_rows_two_pass_kernel(
     const uint16_t *__restrict__ x, int64_t ldx, int K, int8_t *__restrict__ q,
     float *__restrict__ a_scale) {
@@ -295,24 +294,28 @@ w8a8_status launch_quant(const void *x, int64_t M, int64_t K, int64_t ldx, int8_
   const int64_t W = (nchunks + 32 * cpl - 1) / (32 * cpl);
   cudaError_t e = cudaSuccess;
   if (W > 16) {
-    e = ahead_of_gemm
-            ? launch_dependent(quant_rows_two_pass_kernel<true>, 5, dim3((unsigned)M),
-                               dim3(1024), stream, xp, ldx, (int)K, q, a_scale)
-            : launch_dependent(quant_rows_two_pass_kernel<false>, -1, dim3((unsigned)M),
-                               dim3(1024), stream, xp, ldx, (int)K, q, a_scale);
+    // 1024-thread CTAs never leave room for a GEMM CTA: default carveout.
+    e = launch_dependent(quant_rows_two_pass_kernel, -1, dim3((unsigned)M), dim3(1024), stream,
+                         xp, ldx, (int)K, q, a_scale);
   } else {
     const int R = W >= 4 ? 1 : (int)(4 / W);  // rows per CTA: about 128 threads
     const unsigned grid = (unsigned)((M + R - 1) / R);
     const unsigned threads = (unsigned)(32 * W * R);
+    // The instance with the largest carveout where the GEMM behind it can
+    // start beside it: every CTA resident at once, at most 16 warps a SM on
+    // average (the 512-row layers).  Longer inputs run in several waves, in
+    // which the GEMM could start only during the last; they keep the default
+    // carveout and its larger L1.
+    const bool wide = ahead_of_gemm && M * W <= (int64_t)sm_count() * 16;
     switch (cpl) {
 #define W8A8_QUANT_CASE(C, SLOT)                                                          \
   case C:                                                                                 \
-    e = ahead_of_gemm ? launch_dependent(quant_warps_kernel<C, true>, SLOT, dim3(grid),   \
-                                         dim3(threads), stream, xp, ldx, (int)M, (int)K,  \
-                                         (int)W, R, q, a_scale)                           \
-                      : launch_dependent(quant_warps_kernel<C, false>, -1, dim3(grid),    \
-                                         dim3(threads), stream, xp, ldx, (int)M, (int)K,  \
-                                         (int)W, R, q, a_scale);                          \
+    e = wide ? launch_dependent(quant_warps_kernel<C, true>, SLOT, dim3(grid),            \
+                                dim3(threads), stream, xp, ldx, (int)M, (int)K,           \
+                                (int)W, R, q, a_scale)                                    \
+             : launch_dependent(quant_warps_kernel<C, false>, -1, dim3(grid),             \
+                                dim3(threads), stream, xp, ldx, (int)M, (int)K,           \
+                                (int)W, R, q, a_scale);                                   \
     break;
       W8A8_QUANT_CASE(1, 0)
       W8A8_QUANT_CASE(2, 1)
