@@ -13,15 +13,17 @@
 //   acc[m,n] = sum_k q[m,k] w[n,k]                     (exact int32, TMEM)
 //   y[m,n]   = bf16_rne(((float)acc * a_scale[m]) * w_scale[n] + bias[n])
 //
-// 1. gemm_kernel (large M): persistent, one CTA per SM, 321 threads.
+// 1. gemm_kernel (large M): persistent, one CTA per SM, 321 threads of at
+//    most 128 registers (room for quantisation CTAs beside it).
 //    thread 320, alone in the last warp: producer -- per stage of KPS
 //            k-blocks, TMA 2-D loads of the q tiles (128 rows x 128 bytes,
 //            128-byte swizzle) and one bulk copy
 //            of the KPS contiguous weight tiles of each 128-row slab from the
-//            packed image, onto a STAGES-deep mbarrier ring.  Behind the
+//            packed image, onto a STAGES-deep mbarrier ring; a cursor keeps
+//            the address arithmetic out of the slot turnaround.  Behind the
 //            quantisation kernel it first issues the weight copies of the
-//            first stages and an L2 prefetch of more of its slab, then waits
-//            for the codes;
+//            first stages, waits for the codes, then asks L2 to prefetch
+//            more of its slab;
 //    warp 1: MMA issuer -- 4 x tcgen05.mma.kind::i8 (M=128, N=BN, K=32) per
 //            k-block, int32 accumulators in TMEM, double-buffered so the
 //            epilogue of tile i overlaps the main loop of tile i+1;
