@@ -17,7 +17,10 @@
 //     (M = 256, N = 256, K = 32), which reads both CTAs' shared memory and
 //     accumulates into both CTAs' TMEM; its commits arrive on the "empty" and
 //     "accumulator full" barriers of both CTAs (commit multicast);
-//   * both CTAs run the epilogue on their own 128 TMEM lanes.
+//   * both CTAs run the epilogue on their own 128 TMEM lanes;
+//   * roles and limits as in gemm.cu: the producer is the lone thread of a
+//     last, one-thread warp and walks its (segment, stage) list with a cursor;
+//     at most 128 registers a thread.
 //
 // SPLIT = 1: persistent clusters of 2 CTAs, double-buffered accumulators.
 //   When the 256 x 256 tiles fill the SM pairs a few times over plus a short
