@@ -20,7 +20,9 @@ _lib = None
 def lib():
     global _lib
     if _lib is None:
-        path = _build.build()
+        # The mutation test points W8A8_ORACLE_LIB at a deliberately altered
+        # build of this oracle, to check that the pins catch the alteration.
+        path = os.environ.get("W8A8_ORACLE_LIB") or _build.build()
         L = ctypes.CDLL(path)
         P = ctypes.c_void_p
         I64 = ctypes.c_int64

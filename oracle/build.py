@@ -13,16 +13,22 @@ SRC = os.path.join(HERE, "w8a8_oracle.c")
 LIB = os.path.join(HERE, "liboracle.so")
 
 
+def compile_lib(src: str, out: str) -> str:
+    """Compile an oracle source file into a shared library (also used by the
+    mutation test, which compiles deliberately altered copies)."""
+    cmd = ["gcc", "-O2", "-fopenmp", "-ffp-contract=off", "-fno-fast-math",
+           "-std=gnu11", "-Wall", "-Wextra", "-shared", "-fPIC",
+           "-o", out + ".tmp", src, "-lm"]
+    subprocess.run(cmd, check=True)
+    os.replace(out + ".tmp", out)
+    return out
+
+
 def build(force: bool = False) -> str:
     if (not force and os.path.exists(LIB)
             and os.path.getmtime(LIB) >= os.path.getmtime(SRC)):
         return LIB
-    cmd = ["gcc", "-O2", "-fopenmp", "-ffp-contract=off", "-fno-fast-math",
-           "-std=gnu11", "-Wall", "-Wextra", "-shared", "-fPIC",
-           "-o", LIB + ".tmp", SRC, "-lm"]
-    subprocess.run(cmd, check=True)
-    os.replace(LIB + ".tmp", LIB)
-    return LIB
+    return compile_lib(SRC, LIB)
 
 
 if __name__ == "__main__":
