@@ -26,6 +26,7 @@ import os
 import statistics
 import subprocess
 import sys
+import tempfile
 import time
 
 import numpy as np
@@ -37,6 +38,9 @@ sys.path.insert(0, HERE)
 from w8a8_int8_dynamic_b200.workloads import WORKLOADS, make_inputs  # noqa: E402
 
 MAIN_WORKLOAD = "square_512x4096x4096"
+# where the raw nvidia-smi clock samples go (--clocks-dir); the JSON line
+# carries their summary either way
+CLOCKS_DIR = os.path.join(tempfile.gettempdir(), "w8a8_bench_clocks")
 L2_BYTES = 126 * 1024 * 1024
 SPEC_INT8_TOPS = 4500.0
 
@@ -89,8 +93,8 @@ class ClockSampler:
         self.path = None
 
     def start(self):
-        os.makedirs(os.path.join(HERE, "gpurun_out"), exist_ok=True)
-        self.path = os.path.join(HERE, "gpurun_out", f"clocks_rank{self.index}{self.tag}.csv")
+        os.makedirs(CLOCKS_DIR, exist_ok=True)
+        self.path = os.path.join(CLOCKS_DIR, f"clocks_rank{self.index}{self.tag}.csv")
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}",
@@ -637,6 +641,7 @@ def run_reference(args):
 
 # ----------------------------------------------------------------------------- main
 def main():
+    global CLOCKS_DIR
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=20000)
@@ -647,7 +652,11 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--ref-rows", type=int, default=64)
+    ap.add_argument("--clocks-dir", default=None,
+                    help="directory for the raw clock samples (default: a temporary one)")
     args = ap.parse_args()
+    if args.clocks_dir:
+        CLOCKS_DIR = os.path.abspath(args.clocks_dir)
     args.warmup = max(args.warmup, 3)
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
