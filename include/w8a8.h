@@ -166,14 +166,11 @@ w8a8_status w8a8_pack_weight_int32(const int32_t *w_i32, int64_t N, int64_t K,
  *   bias     device, bf16 [N], or NULL for no bias
  *   y        device, bf16 [M, N] (output)
  *   workspace device scratch of ws_bytes >= w8a8_scaled_mm_workspace_bytes,
- *            or NULL (16-byte aligned; contents on entry do not matter).  It
- *            holds int32 K-split partials and call-tagged counters: for
- *            M <= 16 those of the weight-streaming kernel; for problems with
- *            too few 256 x 256 tiles to fill the GPU, those of the K-split
- *            pair kernel (one 128 KB partial per 128 output rows of a tile).
- *            The size query returns 0 when the chosen kernel needs none.
- *            With NULL (or too small), M <= 16 and the K split fall back to
- *            the large-M kernels without a split.
+ *            or NULL (16-byte aligned; contents on entry do not matter).  For
+ *            M <= 16 it holds the weight-streaming kernel's int32 split-K
+ *            partials and call-tagged counters; the size query returns 0
+ *            for larger M, whose kernels need none.  With NULL (or too
+ *            small), M <= 16 falls back to the large-M kernels.
  * All kernels give bit-identical results (the partials are summed exactly
  * in int32 before the scale arithmetic). */
 w8a8_status w8a8_scaled_mm_workspace_bytes(int64_t M, int64_t N, int64_t K,
@@ -207,10 +204,9 @@ w8a8_status w8a8_scaled_mm_i32(const int8_t *q, const void *packed_w,
  * set-up overlaps the quantisation's tail.
  *   x         device, bf16 [M, K], row stride ldx
  *   workspace device, ws_bytes >= w8a8_linear_workspace_bytes(M, N, K); holds
- *             q and a_scale, then the GEMM's workspace (see w8a8_scaled_mm).
- *             Its contents on entry do not matter.  A smaller workspace that
- *             still holds q, a_scale and, for M <= 16, the small-M partials
- *             works too: the GEMM then runs without the K split.
+ *             q and a_scale (each rounded up to 256 bytes), then for M <= 16
+ *             the small-M kernel's partials (see w8a8_scaled_mm).  Its
+ *             contents on entry do not matter.
  * N-D activations [..., K] are flattened by the caller to [M, K] and y is
  * viewed back as [..., N] (the "Diffusion Quantization Reference", GGUF
  * rules and the output-rank failure in "Common Failures"). */
@@ -239,13 +235,15 @@ w8a8_status w8a8_linear_act(const void *x, int64_t ldx, const void *packed_w,
  * to one scratch array of w8a8_linear_noalloc_max_bytes() bytes (8 MiB) that
  * every GPU loading this library holds until the process exits.  Nothing is
  * allocated.  Returns W8A8_ERR_BUFFER_TOO_SMALL, launching nothing, when
- * the codes, scales and small-M partials alone exceed that size (M * K plus
- * 4 M bytes, each rounded up to 256, plus for M <= 16 the small-M kernel's
- * partials); room left over serves the GEMM's K split, which is skipped
- * when it does not fit.  The first call on
- * each device looks up the array's device address (make it before any stream
- * capture).  All calls on a device share the array: calls that overlap on the
- * GPU (different streams without ordering) race and corrupt each other. */
+ * the codes, scales and small-M partials exceed that size
+ * (w8a8_linear_workspace_bytes: M * K plus 4 M bytes, each rounded up to 256,
+ * plus for M <= 16 the small-M kernel's partials).  The first call on each
+ * device looks up the array's device address in the current CUDA context
+ * (make it before any stream capture); the address is looked up again when
+ * a call finds another context current (after a device reset, or under a
+ * context the caller pushed).  All calls on a device share the array: calls
+ * that overlap on the GPU (different streams without ordering) race and
+ * corrupt each other. */
 size_t w8a8_linear_noalloc_max_bytes(void);
 w8a8_status w8a8_linear_noalloc(const void *x, int64_t ldx, const void *packed_w,
                                 const float *w_scale, const void *bias, void *y,
@@ -256,15 +254,9 @@ w8a8_status w8a8_linear_noalloc(const void *x, int64_t ldx, const void *packed_w
  * 0 = automatic (default); 1 = always the persistent large-M GEMM (automatic
  * tile width); 2 = the small-M weight-streaming kernel (M <= 16 only, else
  * W8A8_ERR_INVALID_ARG); 3 / 4 = the 1-SM large-M GEMM with 128- / 256-wide
- * output tiles; 5 = the 2-SM (CTA pair) GEMM with 256 x 256 tiles; 6 = the
- * same with K split over two pairs per tile, the first half's int32 partial
- * handed over through the workspace (which w8a8_scaled_mm_workspace_bytes
- * then sizes); 7 = the 2-SM GEMM with 256 x 128 tiles; 8 = the 256 x 256
- * 2-SM GEMM with stream-K: the tiles' k-blocks cut into equal contiguous
- * ranges, one per SM pair, tiles split between two pairs summing their int32
- * partials through the workspace (sized by w8a8_scaled_mm_workspace_bytes
- * while the path is set).  Paths 6 and 8 are never chosen automatically; the
- * others are, by shape.
+ * output tiles; 5 = the 2-SM (CTA pair) GEMM with 256 x 256 tiles; 7 = the
+ * 2-SM GEMM with 256 x 128 tiles.  6 (and anything above 7) is not a path:
+ * W8A8_ERR_INVALID_ARG.  Each path is also chosen automatically, by shape.
  * Process-wide; not synchronised with concurrent calls. */
 w8a8_status w8a8_set_path(int path);
 

@@ -92,35 +92,28 @@ def test_gemm_rejects_bad_arguments(L):
     assert g(FAKE, 16, FAKE, FAKE, None, FAKE, 4, 8, 16, FAKE, 1, None) == 6       # too small
     assert g(FAKE, 8, FAKE, FAKE, None, FAKE, 4, 8, 16, FAKE, 1 << 30, None) == 1  # ldx < K
     assert L.w8a8_set_path(9) == 1
-    assert L.w8a8_set_path(8) == 0
+    assert L.w8a8_set_path(8) == 1
+    assert L.w8a8_set_path(6) == 1
+    assert L.w8a8_set_path(7) == 0
     assert L.w8a8_set_path(0) == 0
 
 
 def test_workspace_sizes(L):
     """Host-side sizing (no GPU: the SM count falls back to the B200's 148).
-    The automatic choice needs no GEMM workspace above the small-M range; the
-    forced stream-K path needs its partials; with the K-split pair kernel
-    forced, 512 x 4096 x 4096 (32
-    tiles) needs two 16-byte sync slots and one 128 KB int32 partial per 128
-    output rows of each tile.  Small M needs the split-K partials of the
-    weight-streaming kernel."""
+    The large-M kernels need no GEMM workspace, under every path setting; the
+    layer's workspace is then the codes and scales, each rounded up to 256
+    bytes.  Small M needs the split-K partials of the weight-streaming
+    kernel."""
     from w8a8_int8_dynamic_b200 import binding
     assert binding.scaled_mm_workspace_bytes(512, 4096, 4096) == 0
     assert binding.linear_workspace_bytes(512, 4096, 4096) == 512 * 4096 + 2048
     assert binding.scaled_mm_workspace_bytes(4096, 12288, 3072) == 0
     assert binding.linear_workspace_bytes(4096, 12288, 3072) == 4096 * 3072 + 4096 * 4
     assert binding.scaled_mm_workspace_bytes(16, 27648, 5120) > 0
-    # stream-K forced: two sync words and one 128 KB partial per (range
-    # boundary, CTA rank), at most 74 + 1 boundaries
-    assert L.w8a8_set_path(8) == 0
-    try:
-        assert binding.scaled_mm_workspace_bytes(4096, 12288, 3072) == 2560 + 150 * 128 * 1024
-    finally:
-        assert L.w8a8_set_path(0) == 0
-    assert L.w8a8_set_path(6) == 0
-    try:
-        split = 1024 + 64 * 128 * 1024
-        assert binding.scaled_mm_workspace_bytes(512, 4096, 4096) == split
-        assert binding.linear_workspace_bytes(512, 4096, 4096) == 512 * 4096 + 2048 + split
-    finally:
-        assert L.w8a8_set_path(0) == 0
+    for path in (1, 3, 4, 5, 7):
+        assert L.w8a8_set_path(path) == 0
+        try:
+            assert binding.scaled_mm_workspace_bytes(512, 4096, 4096) == 0
+            assert binding.linear_workspace_bytes(512, 4096, 4096) == 512 * 4096 + 2048
+        finally:
+            assert L.w8a8_set_path(0) == 0

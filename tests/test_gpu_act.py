@@ -35,8 +35,7 @@ def _case(M, N, K, bias, seed):
 
 @pytest.mark.parametrize("bias", [False, True])
 @pytest.mark.parametrize("path", [w8.PATH_LARGE_BN128, w8.PATH_LARGE_BN256, w8.PATH_LARGE_PAIR,
-                                  w8.PATH_LARGE_PAIR128, w8.PATH_LARGE_PAIR_SPLIT,
-                                  w8.PATH_LARGE_PAIR_STREAMK])
+                                  w8.PATH_LARGE_PAIR128])
 @pytest.mark.parametrize("M,N,K", [(64, 128, 256), (129, 392, 400), (300, 1000, 528),
                                    (512, 1024, 4096), (700, 520, 144)])
 def test_scaled_mm_gelu_fused_equals_chain(M, N, K, path, bias):

@@ -146,8 +146,7 @@ def test_gemm_i32_extreme_values():
 
 @pytest.mark.parametrize("bias", [False, True])
 @pytest.mark.parametrize("path", [w8.PATH_LARGE_BN128, w8.PATH_LARGE_BN256, w8.PATH_LARGE_PAIR,
-                                  w8.PATH_LARGE_PAIR128, w8.PATH_LARGE_PAIR_SPLIT,
-                                  w8.PATH_LARGE_PAIR_STREAMK])
+                                  w8.PATH_LARGE_PAIR128])
 @pytest.mark.parametrize("M,N,K", [(64, 128, 256), (129, 392, 400), (300, 1000, 528), (512, 1024, 4096),
                                    (257, 264, 272), (700, 520, 144), (1000, 2056, 1040)])
 def test_scaled_mm_matches_oracle(M, N, K, path, bias):
@@ -163,33 +162,31 @@ def test_scaled_mm_matches_oracle(M, N, K, path, bias):
     assert np.array_equal(y_h, y_ref), "expected bit-exact bf16"
 
 
-@pytest.mark.parametrize("M,N,K", [(512, 1024, 4096), (300, 776, 2064), (512, 4096, 4096)])
-def test_k_split_pairs_with_garbage_workspace_repeated(M, N, K):
-    """The K-split pair kernel (two pairs per tile, one per half of K, the
-    first half's int32 partial handed over through the workspace).  The
-    workspace starts as random bytes and is reused by three calls; the
-    call-tagged counters must ignore every leftover, and each call must match
-    the oracle bit for bit."""
-    w8.set_path(w8.PATH_LARGE_PAIR_SPLIT)
-    assert "K split" in w8.gemm_kernel_name(M, N, K)
-    inp = random_case(M * 5 + N + K, M, N, K, bias=True, n_outliers=K // 64, zero_row=True)
-    q_ref, s_ref = oracle.quant_act(inp.x)
-    y_ref = oracle.epilogue(oracle.gemm_i32(q_ref, inp.w), s_ref, inp.w_scale, inp.bias)
+@pytest.mark.parametrize("M,N,K", [(1, 27648, 5120), (4, 2056, 1040), (16, 4096, 12288)])
+def test_decode_with_garbage_workspace_repeated(M, N, K):
+    """The small-M kernel counts the CTAs that share a weight slab on
+    call-tagged workspace words.  Here the workspace starts as random bytes
+    (stale tags, counts in every state) and serves four calls with new
+    activations; each call must match the oracle bit for bit."""
+    w8.set_path(w8.PATH_SMALL)
+    inp = random_case(M * 7 + N + K, M, N, K, bias=True, n_outliers=K // 64)
+    packed = w8.pack_weight(dev(inp.w))
     need = w8.scaled_mm_workspace_bytes(M, N, K)
     assert need > 0
     ws = torch.randint(0, 256, (need,), dtype=torch.uint8, device="cuda")
-    args = (dev(q_ref), dev(s_ref), w8.pack_weight(dev(inp.w)), dev(inp.w_scale),
-            dev_bf16(inp.bias), N)
-    for _ in range(3):
-        y = w8.scaled_mm(*args, workspace=ws)
-        assert np.array_equal(host_u16(y), y_ref)
-    # without a workspace the same problem runs unsplit, with the same result
-    small = torch.empty((16,), dtype=torch.uint8, device="cuda")
-    assert np.array_equal(host_u16(w8.scaled_mm(*args, workspace=small)), y_ref)
+    for i in range(4):
+        xi = random_case(500 + i, M, N, K, bias=False, n_outliers=K // 64).x
+        q_ref, s_ref = oracle.quant_act(xi)
+        y_ref = oracle.epilogue(oracle.gemm_i32(q_ref, inp.w), s_ref, inp.w_scale, inp.bias)
+        y = w8.scaled_mm(dev(q_ref), dev(s_ref), packed, dev(inp.w_scale), dev_bf16(inp.bias), N,
+                         workspace=ws)
+        assert np.array_equal(host_u16(y), y_ref), f"call {i}"
+        # and a fresh scramble of the words between calls
+        if i == 1:
+            ws.random_(0, 256)
 
 
-@pytest.mark.parametrize("path", [w8.PATH_LARGE_BN128, w8.PATH_LARGE_PAIR, w8.PATH_LARGE_PAIR128,
-                                  w8.PATH_LARGE_PAIR_SPLIT, w8.PATH_LARGE_PAIR_STREAMK])
+@pytest.mark.parametrize("path", [w8.PATH_LARGE_BN128, w8.PATH_LARGE_PAIR, w8.PATH_LARGE_PAIR128])
 def test_scaled_mm_does_not_write_outside_y(path):
     w8.set_path(path)
     M, N, K = 130, 264, 272
@@ -246,8 +243,7 @@ def test_decode_path_matches_oracle(M, N, K):
 
 
 # ---------------------------------------------------------------- fused layer
-@pytest.mark.parametrize("path", [w8.PATH_AUTO, w8.PATH_LARGE_PAIR, w8.PATH_LARGE_PAIR128,
-                                  w8.PATH_LARGE_PAIR_SPLIT])
+@pytest.mark.parametrize("path", [w8.PATH_AUTO, w8.PATH_LARGE_PAIR, w8.PATH_LARGE_PAIR128])
 @pytest.mark.parametrize("M,N,K", [(1, 264, 400), (16, 1024, 1024), (17, 1024, 1024),
                                    (64, 128, 256), (300, 1000, 528), (512, 4096, 4096)])
 def test_linear_matches_oracle(M, N, K, path):
@@ -294,21 +290,16 @@ def test_gelu_within_one_ulp():
 
 
 # ---------------------------------------------------------------- CUDA graph replay
-@pytest.mark.parametrize("case", ["layer", "decode_layer", "k_split", "stream_k", "tail_split"])
+@pytest.mark.parametrize("case", ["layer", "decode_layer", "tail_split"])
 def test_cuda_graph_replay_with_new_inputs(case):
     """Kernels that count CTAs on call-tagged workspace words (the small-M
-    kernel's slab reduction, the K-split handoff) see the same tag on every
-    replay of a captured CUDA graph.  They must leave those words cleared:
-    capture one call, then replay it three times with new inputs copied into
-    the captured buffers, each replay checked against the oracle bit for bit
-    (the large-M layer, quantisation + GEMM, alongside)."""
+    kernel's slab reduction) see the same tag on every replay of a captured
+    CUDA graph.  They must leave those words cleared: capture one call, then
+    replay it three times with new inputs copied into the captured buffers,
+    each replay checked against the oracle bit for bit (the large-M layer,
+    quantisation + GEMM, alongside)."""
     M, N, K = {"layer": (512, 1024, 1024), "decode_layer": (4, 2056, 1040),
-               "k_split": (512, 1024, 4096), "stream_k": (1000, 2056, 1040),
                "tail_split": (600, 8200, 400)}[case]
-    if case == "k_split":
-        w8.set_path(w8.PATH_LARGE_PAIR_SPLIT)
-    if case == "stream_k":
-        w8.set_path(w8.PATH_LARGE_PAIR_STREAMK)
     inp = random_case(7, M, N, K, bias=True, n_outliers=K // 64)
     packed = w8.pack_weight(dev(inp.w))
     ws_s, b = dev(inp.w_scale), dev_bf16(inp.bias)
@@ -316,12 +307,8 @@ def test_cuda_graph_replay_with_new_inputs(case):
     q = torch.empty((M, K), dtype=torch.int8, device="cuda")
     a = torch.empty((M,), dtype=torch.float32, device="cuda")
     y = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
-    if case in ("k_split", "stream_k"):
-        ws = torch.empty((w8.scaled_mm_workspace_bytes(M, N, K),), dtype=torch.uint8, device="cuda")
-        call = lambda: w8.scaled_mm(q, a, packed, ws_s, b, N, out=y, workspace=ws)  # noqa: E731
-    else:
-        ws = torch.empty((w8.linear_workspace_bytes(M, N, K),), dtype=torch.uint8, device="cuda")
-        call = lambda: w8.linear(x, packed, ws_s, b, N, out=y, workspace=ws)  # noqa: E731
+    ws = torch.empty((w8.linear_workspace_bytes(M, N, K),), dtype=torch.uint8, device="cuda")
+    call = lambda: w8.linear(x, packed, ws_s, b, N, out=y, workspace=ws)  # noqa: E731
     stream = torch.cuda.Stream()
     with torch.cuda.stream(stream):
         call()  # warm the launch path before capture

@@ -28,9 +28,7 @@ STATUS_NAMES = {
 }
 
 PATH_AUTO, PATH_LARGE, PATH_SMALL, PATH_LARGE_BN128, PATH_LARGE_BN256, PATH_LARGE_PAIR = 0, 1, 2, 3, 4, 5
-PATH_LARGE_PAIR_SPLIT = 6
 PATH_LARGE_PAIR128 = 7
-PATH_LARGE_PAIR_STREAMK = 8
 # activations fused into the GEMM epilogue (w8a8_act)
 ACT_NONE, ACT_GELU_TANH = 0, 1
 

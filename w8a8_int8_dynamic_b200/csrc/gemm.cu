@@ -316,8 +316,7 @@ __global__ void __maxnreg__(kGemmRegs)
       if (OUT_I32)
         epilogue_i32<kCols>(args, taddr, row0 + lane, n0);
       else
-        epilogue_tma<kCols>(args, &tmap_y, taddr, lane, row0, n0, as, s_ws, s_bias, s_out,
-                            false, NoExtra());
+        epilogue_tma<kCols>(args, &tmap_y, taddr, lane, row0, n0, as, s_ws, s_bias, s_out);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&tempty[b]);
@@ -398,7 +397,7 @@ w8a8_status run_large(const CUtensorMap &tmap, const CUtensorMap &tmap_y, GemmAr
 // ~128 B/clk per SM, the 128 x 256 tile ~94, the 2-SM 256 x 256 tile ~64),
 // so the cost of a shape is its wave count times its per-SM tile work divided
 // by the fraction of the rate it sustains.
-enum class LargeKind { k128, k256, kPair, kPair128, kPairSplit, kPairStreamK };
+enum class LargeKind { k128, k256, kPair, kPair128 };
 
 // Kernel choice for large M: (waves of tiles) x (per-SM time of one tile).
 // The per-SM time of a stage of two k-blocks is set by what has to reach the
@@ -408,15 +407,12 @@ enum class LargeKind { k128, k256, kPair, kPair128, kPairSplit, kPairStreamK };
 // cycles; 1-SM 128x256: 96 KB / 1024; pair 256x256: 64 KB / 1024; pair
 // 256x128: 48 KB / 512 per SM.  The constants are calibrated against timings
 // on this B200, not derived.
-// `split_ok`: a workspace for the K-split pair kernel is available.
-LargeKind choose_large(int64_t M, int64_t N, int64_t K, bool split_ok) {
+LargeKind choose_large(int64_t M, int64_t N) {
   const int path = forced_path();
   if (path == 3) return LargeKind::k128;
   if (path == 4) return LargeKind::k256;
   if (path == 5) return LargeKind::kPair;
-  if (path == 6) return split_ok ? LargeKind::kPairSplit : LargeKind::kPair;
   if (path == 7) return LargeKind::kPair128;
-  if (path == 8) return split_ok ? LargeKind::kPairStreamK : LargeKind::kPair;
   const int64_t sms = sm_count(), pairs = sms / 2;
   const double feed_us_per_kb = 1.0 / 114e3;  // us per byte per SM
   const double l2_us_per_byte = 1.0 / 10.5e6;  // us per byte, whole chip
@@ -449,14 +445,6 @@ LargeKind choose_large(int64_t M, int64_t N, int64_t K, bool split_ok) {
   if (c256 < best) best = c256, kind = LargeKind::k256;
   if (cp256 <= best) best = cp256, kind = LargeKind::kPair;
   if (cp128 < best * 0.97) best = cp128, kind = LargeKind::kPair128;
-  // Never chosen here, both measured slower on the shapes at hand: the K
-  // split over two pairs per tile (paths 6; 512 x 4096 x 4096: 19.1 vs
-  // 14.3 us -- the 128 KB int32 handoff per CTA costs about 4 us) and
-  // stream-K (path 8; 512 x 12288 x 4096: 35.3 vs 31.8 us -- the partials add
-  // about a fifth to the L2 traffic, while a last wave with few busy SMs
-  // runs each of its tiles faster and costs little).
-  (void)split_ok;
-  (void)K;
   return kind;
 }
 
@@ -465,7 +453,7 @@ LargeKind choose_large(int64_t M, int64_t N, int64_t K, bool split_ok) {
 w8a8_status launch_scaled_mm(const int8_t *q, const float *a_scale, const void *packed_w,
                              const float *w_scale, const void *bias, void *out, bool out_i32,
                              int64_t M, int64_t N, int64_t K, cudaStream_t stream, bool pdl,
-                             int act, void *workspace, size_t ws_bytes) {
+                             int act) {
   CUtensorMap tmap;
   if (!make_tmap_u8_2d(&tmap, q, (uint64_t)M, (uint64_t)K, (uint64_t)K, kBM, kBK))
     return W8A8_ERR_CUDA;
@@ -489,29 +477,19 @@ w8a8_status launch_scaled_mm(const int8_t *q, const float *a_scale, const void *
     // the int32 export always uses the 1-SM kernel (tests and inspection); it
     // stores from registers and takes no output tensor map
     memset(&tmap_y, 0, sizeof(tmap_y));
-    const LargeKind kind = choose_large(M, N, K, false);
+    const LargeKind kind = choose_large(M, N);
     return kind == LargeKind::k128
                ? run_large<128, kLargeStages128, true>(tmap, tmap_y, a, stream, pdl, 1)
                : run_large<256, kLargeStages256, true>(tmap, tmap_y, a, stream, pdl, 0);
   }
   if (!make_tmap_out_bf16(&tmap_y, out, (uint64_t)M, (uint64_t)N)) return W8A8_ERR_CUDA;
-  // enough workspace for the K split / stream-K (both partial layouts)
-  const bool split_ok =
-      workspace && (int64_t)ws_bytes >= std::min(split_workspace_bytes(M, N, 2),
-                                                  split_workspace_bytes(M, N, 3));
-  switch (choose_large(M, N, K, split_ok)) {
+  switch (choose_large(M, N)) {
     case LargeKind::kPair:
-      return launch_gemm2sm(q, a_scale, packed_w, w_scale, bias, out, M, N, K, stream, pdl, 1, 256,
+      return launch_gemm2sm(q, a_scale, packed_w, w_scale, bias, out, M, N, K, stream, pdl, 256,
                             act);
     case LargeKind::kPair128:
-      return launch_gemm2sm(q, a_scale, packed_w, w_scale, bias, out, M, N, K, stream, pdl, 1, 128,
+      return launch_gemm2sm(q, a_scale, packed_w, w_scale, bias, out, M, N, K, stream, pdl, 128,
                             act);
-    case LargeKind::kPairSplit:
-      return launch_gemm2sm(q, a_scale, packed_w, w_scale, bias, out, M, N, K, stream, pdl, 2, 256,
-                            act, workspace, ws_bytes);
-    case LargeKind::kPairStreamK:
-      return launch_gemm2sm(q, a_scale, packed_w, w_scale, bias, out, M, N, K, stream, pdl, 3, 256,
-                            act, workspace, ws_bytes);
     case LargeKind::k256:
       return run_large<256, kLargeStages256, false>(tmap, tmap_y, a, stream, pdl, 2);
     default:
@@ -519,16 +497,9 @@ w8a8_status launch_scaled_mm(const int8_t *q, const float *a_scale, const void *
   }
 }
 
-int64_t large_workspace_bytes(int64_t M, int64_t N, int64_t K) {
-  const LargeKind kind = choose_large(M, N, K, true);
-  return kind == LargeKind::kPairSplit    ? split_workspace_bytes(M, N, 2)
-         : kind == LargeKind::kPairStreamK ? split_workspace_bytes(M, N, 3)
-                                           : 0;
-}
-
-// Workspace w8a8_linear cannot do without: the codes, the scales and (small
-// M) the split-K partials of the weight-streaming kernel.
-int64_t linear_workspace_min(int64_t M, int64_t N, int64_t K) {
+// Workspace of w8a8_linear: the codes, the scales and (small M) the split-K
+// partials of the weight-streaming kernel.
+int64_t linear_workspace_bytes(int64_t M, int64_t N, int64_t K) {
   int64_t b = round_up(M * K, 256) + round_up(M * 4, 256);
   if (M <= kDecodeNT) b += decode_workspace_bytes(N, K);
   return b;
@@ -553,7 +524,7 @@ extern "C" {
 w8a8_status w8a8_scaled_mm_workspace_bytes(int64_t M, int64_t N, int64_t K, size_t *bytes) {
   if (!bytes || M < 1 || N < 1 || K < 1) return W8A8_ERR_INVALID_ARG;
   if (K % 16 != 0 || K > kMaxK || N % 8 != 0) return W8A8_ERR_UNSUPPORTED_SHAPE;
-  *bytes = (size_t)(M <= kDecodeNT ? decode_workspace_bytes(N, K) : large_workspace_bytes(M, N, K));
+  *bytes = (size_t)(M <= kDecodeNT ? decode_workspace_bytes(N, K) : 0);
   return W8A8_OK;
 }
 
@@ -576,8 +547,7 @@ w8a8_status w8a8_scaled_mm_act(const int8_t *q, const float *a_scale, const void
   }
   if (forced_path() == 2) return W8A8_ERR_INVALID_ARG;  // small path needs M <= 16 and a workspace
   if (workspace && !aligned16(workspace)) return W8A8_ERR_ALIGNMENT;
-  return launch_scaled_mm(q, a_scale, packed_w, w_scale, bias, y, false, M, N, K, s, false, act,
-                          workspace, ws_bytes);
+  return launch_scaled_mm(q, a_scale, packed_w, w_scale, bias, y, false, M, N, K, s, false, act);
 }
 
 w8a8_status w8a8_scaled_mm(const int8_t *q, const float *a_scale, const void *packed_w,
@@ -590,12 +560,9 @@ w8a8_status w8a8_scaled_mm(const int8_t *q, const float *a_scale, const void *pa
 const char *w8a8_gemm_kernel_name(int64_t M, int64_t N, int64_t K) {
   if (M < 1 || N < 1 || K < 1) return "invalid";
   if (use_decode_path(M)) return "decode_kernel (swap-AB stream-K, needs a workspace)";
-  switch (choose_large(M, N, K, true)) {
-    case LargeKind::kPair: return "gemm2sm_kernel<256, 3, 1> (2-SM pair, 256x256 tiles)";
-    case LargeKind::kPair128: return "gemm2sm_kernel<128, 4, 1> (2-SM pair, 256x128 tiles)";
-    case LargeKind::kPairSplit: return "gemm2sm_kernel<256, 3, 2> (2-SM pairs, K split)";
-    case LargeKind::kPairStreamK:
-      return "gemm2sm_kernel<256, 3, 3> (2-SM pairs, 256x256 tiles, stream-K)";
+  switch (choose_large(M, N)) {
+    case LargeKind::kPair: return "gemm2sm_kernel<256, 3> (2-SM pair, 256x256 tiles)";
+    case LargeKind::kPair128: return "gemm2sm_kernel<128, 4> (2-SM pair, 256x128 tiles)";
     case LargeKind::k256: return "gemm_kernel<256, 4, 1> (1-SM, 128x256 tiles)";
     default: return "gemm_kernel<128, 3, 2> (1-SM, 128x128 tiles, 2 k-blocks per stage)";
   }
@@ -612,9 +579,7 @@ w8a8_status w8a8_scaled_mm_i32(const int8_t *q, const void *packed_w, int32_t *a
 w8a8_status w8a8_linear_workspace_bytes(int64_t M, int64_t N, int64_t K, size_t *bytes) {
   if (!bytes || M < 1 || N < 1 || K < 1) return W8A8_ERR_INVALID_ARG;
   if (K % 16 != 0 || K > kMaxK || N % 8 != 0) return W8A8_ERR_UNSUPPORTED_SHAPE;
-  int64_t b = linear_workspace_min(M, N, K);
-  if (M > kDecodeNT) b += large_workspace_bytes(M, N, K);
-  *bytes = (size_t)b;
+  *bytes = (size_t)linear_workspace_bytes(M, N, K);
   return W8A8_OK;
 }
 
@@ -630,9 +595,7 @@ w8a8_status w8a8_linear_act(const void *x, int64_t ldx, const void *packed_w,
   if (ldx % 8 != 0 || !aligned16(w_scale) || !aligned16(workspace) ||
       (bias && !aligned16(bias)))
     return W8A8_ERR_ALIGNMENT;
-  // Anything beyond the minimum may hold the K-split partials of the GEMM.
-  const int64_t need = linear_workspace_min(M, N, K);
-  if ((int64_t)ws_bytes < need) return W8A8_ERR_BUFFER_TOO_SMALL;
+  if ((int64_t)ws_bytes < linear_workspace_bytes(M, N, K)) return W8A8_ERR_BUFFER_TOO_SMALL;
   uint8_t *ws = static_cast<uint8_t *>(workspace);
   int8_t *q = reinterpret_cast<int8_t *>(ws);
   float *a_scale = reinterpret_cast<float *>(ws + round_up(M * K, 256));
@@ -644,9 +607,7 @@ w8a8_status w8a8_linear_act(const void *x, int64_t ldx, const void *packed_w,
     return launch_decode(q, a_scale, packed_w, w_scale, bias, y, M, N, K, dws, s, true, act);
   }
   if (forced_path() == 2) return W8A8_ERR_INVALID_ARG;
-  const int64_t head = round_up(M * K, 256) + round_up(M * 4, 256);
-  return launch_scaled_mm(q, a_scale, packed_w, w_scale, bias, y, false, M, N, K, s, true, act,
-                          ws + head, ws_bytes - (size_t)head);
+  return launch_scaled_mm(q, a_scale, packed_w, w_scale, bias, y, false, M, N, K, s, true, act);
 }
 
 w8a8_status w8a8_linear(const void *x, int64_t ldx, const void *packed_w, const float *w_scale,

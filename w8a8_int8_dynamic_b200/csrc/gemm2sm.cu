@@ -22,23 +22,14 @@
 //     last, one-thread warp and walks its (segment, stage) list with a cursor;
 //     at most 128 registers a thread.
 //
-// SPLIT = 1: persistent clusters of 2 CTAs, double-buffered accumulators.
-//   When the 256 x 256 tiles fill the SM pairs a few times over plus a short
-//   last round (at most half the pairs), the tiles of that round run as their
-//   two 256 x 128 halves instead (MMA N = 128, each CTA loading 64 weight
-//   rows), spread over twice as many pairs.
-// SPLIT = 2: (for problems with too few tiles to fill the GPU) every tile is
-//   computed by two pairs, one per half of K, one work item per pair.  Per
-//   (tile, CTA rank) a call-tagged counter in the workspace tells the two
-//   CTAs that hold the same 128 output rows which of them finished first: the
-//   first publishes its int32 partial to the workspace and raises a flag; the
-//   second waits for that flag (its partner is already past its main loop),
-//   bulk-copies the partial into its idle stage buffers and adds it -- exactly,
-//   in int32 -- before the scale arithmetic.  No CTA ever waits for one that
-//   may not have started.
+// Persistent clusters of 2 CTAs, double-buffered accumulators.  When the
+// 256 x 256 tiles fill the SM pairs a few times over plus a short last round
+// (at most half the pairs), the tiles of that round run as their two
+// 256 x 128 halves instead (MMA N = 128, each CTA loading 64 weight rows),
+// spread over twice as many pairs.
 //
 // No TMA load uses cluster multicast.  Every wait is time-bounded (the waits
-// between the two pairs of a cluster are safe: a cluster's CTAs are
+// between the two CTAs of a pair are safe: a cluster's CTAs are
 // co-scheduled); a block that gives up drains its copies, the cluster meets
 // at a barrier and frees TMEM.
 #include <algorithm>
@@ -50,8 +41,6 @@ namespace {
 
 constexpr int kStageK = 2;                        // k-blocks per stage
 constexpr int kHalfStage = kStageK * kTileBytes;  // 32 KB: the q part of one stage
-constexpr int kPartialBytes = 128 * 256 * 4;      // one CTA's int32 partial (BN = 256): 128 KB
-constexpr int kPartialInts = kPartialBytes / 4;
 
 // BN = tile N of the pair (256 or 128); each CTA holds BN/2 weight rows.
 template <int BN, int STAGES>
@@ -65,36 +54,17 @@ struct PairSmem {
   static constexpr int kEpi = kB + STAGES * kBStage;
   static constexpr int kEpiEnd = kEpi + kEpiWarps * kEpiPerWarp;
   static constexpr int kOut = kEpiEnd + 1024 - kEpiEnd % 1024;
-  // full[S], empty[S], tfull[2], tempty[2], done, recv
+  // full[S], empty[S], tfull[2], tempty[2], done
   static constexpr int kBars = kOut + kEpiWarps * kEpiStagePerWarp;
-  static constexpr int kMisc = kBars + (2 * STAGES + 6) * 8;
+  static constexpr int kMisc = kBars + (2 * STAGES + 5) * 8;
   static constexpr int kUsed = kMisc + 16;
   static constexpr int kAlloc = kUsed + 1024;
-  static_assert(BN != 256 || STAGES * (kHalfStage + kBStage) >= kPartialBytes,
-                "partial must fit the stage buffers");
-};
-
-// int32 partial layout in shared memory: element (row r, column j) at
-// ((j / 4) * 128 + r) * 4 + j % 4, so the 32 lanes (rows) of a warp move 512
-// contiguous bytes per 16-byte access.
-__device__ __forceinline__ int partial_index(int r, int j) { return ((j >> 2) * 128 + r) * 4 + (j & 3); }
-// Four partial values of row r at columns j0 + j .. j0 + j + 3 (the
-// epilogue's column index j counts from the warp's first column j0), from
-// shared memory or, bypassing L1, from the workspace in global memory.
-struct PartialLoad {
-  const int32_t *p;
-  int r, j0;
-  bool global;
-  __device__ uint4 operator()(int j) const {
-    const uint4 *q = reinterpret_cast<const uint4 *>(p + partial_index(r, j0 + j));
-    return global ? __ldcg(q) : *q;
-  }
 };
 
 // At most kGemmRegs registers a thread, so that a CTA (11 warps) fits on an
 // SM beside the blocks of the quantisation kernel it is launched behind and
 // starts its prologue and first weight copies while they run.
-template <int BN, int STAGES, int SPLIT>
+template <int BN, int STAGES>
 __global__ void __maxnreg__(kGemmRegs)
     gemm2sm_kernel(const __grid_constant__ CUtensorMap tmap_q,
                    const __grid_constant__ CUtensorMap tmap_w,
@@ -106,8 +76,6 @@ __global__ void __maxnreg__(kGemmRegs)
   constexpr uint32_t kIdesc = idesc_i8(256, BN);
   constexpr uint32_t kIdescHalf = idesc_i8(256, 128);  // a 256 x 128 half of a 256-wide tile
   constexpr int kHalfBTile = 64 * kBK;                   // its weight rows per CTA per k-block
-  static_assert(SPLIT == 1 || BN == 256, "the K split is built for 256-wide tiles");
-  static_assert(SPLIT >= 1 && SPLIT <= 3, "1: whole tiles, 2: K halves, 3: stream-K");
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>(
@@ -119,11 +87,8 @@ __global__ void __maxnreg__(kGemmRegs)
   uint64_t *tfull = empty + STAGES;
   uint64_t *tempty = tfull + 2;
   uint64_t *mma_done = tempty + 2;
-  uint64_t *recv = mma_done + 1;  // (SPLIT = 2) the partner's partial has arrived
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + L::kMisc);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + L::kMisc + 4);
-  volatile int *arrival = reinterpret_cast<volatile int *>(smem + L::kMisc + 8);
-  int32_t *partial = reinterpret_cast<int32_t *>(smem);  // aliases the stage buffers
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t crank = cluster_ctarank();
@@ -142,7 +107,6 @@ __global__ void __maxnreg__(kGemmRegs)
       mbar_init(&tempty[b], 2 * kEpiWarps);  // the epilogue warps of both CTAs
     }
     mbar_init(mma_done, 1);
-    mbar_init(recv, 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -163,8 +127,8 @@ __global__ void __maxnreg__(kGemmRegs)
   const int slot = (int)(blockIdx.x >> 1);
   const int nslots = (int)(gridDim.x >> 1);
   // Work items: tiles [0, full_tiles) whole, then item full_tiles + 2 j + h
-  // is N half h of tile full_tiles + j (SPLIT = 1 only; otherwise full_tiles
-  // is the tile count).
+  // is N half h of tile full_tiles + j.  This pair takes items slot,
+  // slot + nslots, ... (one segment of S stages each).
   const int num_items = args.full_tiles + 2 * (num_tiles - args.full_tiles);
   auto item_tile = [&](int item) -> int {
     return item < args.full_tiles ? item : args.full_tiles + ((item - args.full_tiles) >> 1);
@@ -172,41 +136,9 @@ __global__ void __maxnreg__(kGemmRegs)
   auto item_half = [&](int item) -> int {  // -1: the whole tile
     return item < args.full_tiles ? -1 : ((item - args.full_tiles) & 1);
   };
-  // This pair's work as segments (item, first stage, end stage), in order:
-  //   SPLIT = 1: items slot, slot + nslots, ...
-  //   SPLIT = 2: one segment, tile slot / 2, K half slot % 2
-  //   SPLIT = 3: stream-K -- the tiles' T * S stages cut into nslots equal
-  //              contiguous ranges; a range starts inside a tile (its tail),
-  //              covers whole tiles and ends inside another (its head).  With
-  //              at least S stages per range a tile has at most two parts.
-  // Segment i: tile t_first + i * t_step, stages [i == 0 ? st_first : 0,
-  // i == nseg - 1 ? st_last : S).
-  int nseg = 0, t_first = 0, t_step = 1, st_first = 0, st_last = S;
-  if (SPLIT == 1) {
-    nseg = slot < num_items ? (num_items - 1 - slot) / nslots + 1 : 0;
-    t_first = slot;
-    t_step = nslots;
-  } else if (SPLIT == 2) {
-    nseg = slot < 2 * num_tiles ? 1 : 0;
-    t_first = slot >> 1;
-    st_first = (slot & 1) ? S / 2 : 0;
-    st_last = (slot & 1) ? S : S / 2;
-  } else {
-    const int64_t units = (int64_t)num_tiles * S;
-    const int64_t u0 = units * slot / nslots, u1 = units * (slot + 1) / nslots;
-    if (u1 > u0) {
-      t_first = (int)(u0 / S);
-      const int t_last = (int)((u1 - 1) / S);
-      nseg = t_last - t_first + 1;
-      st_first = (int)(u0 - (int64_t)t_first * S);
-      st_last = (int)(u1 - (int64_t)t_last * S);
-    }
-  }
-  auto seg_tile = [&](int i) -> int { return t_first + i * t_step; };
-  auto seg_begin = [&](int i) -> int { return i == 0 ? st_first : 0; };
-  auto seg_end = [&](int i) -> int { return i == nseg - 1 ? st_last : S; };
-  uint32_t my_iters = 0;
-  for (int i = 0; i < nseg; ++i) my_iters += (uint32_t)(seg_end(i) - seg_begin(i));
+  const int nseg = slot < num_items ? (num_items - 1 - slot) / nslots + 1 : 0;
+  auto seg_tile = [&](int i) -> int { return slot + i * nslots; };
+  const uint32_t my_iters = (uint32_t)nseg * (uint32_t)S;
   const uint32_t full0 = map_to_cta(smem_addr(full), lead);  // pair leader's full[0]
   const uint32_t tempty0 = map_to_cta(smem_addr(tempty), lead);
 
@@ -249,7 +181,7 @@ __global__ void __maxnreg__(kGemmRegs)
       return c;
     };
     auto advance = [&](Cursor &c) {
-      if (++c.st >= seg_end(c.seg)) c = enter(c.seg + 1, c.seg + 1 < nseg ? seg_begin(c.seg + 1) : 0);
+      if (++c.st >= S) c = enter(c.seg + 1, 0);
     };
     auto stage_nk = [&](const Cursor &c) { return min(kStageK, num_kb - c.st * kStageK); };
     auto stage_bytes = [&](const Cursor &c, int nk) {
@@ -280,7 +212,7 @@ __global__ void __maxnreg__(kGemmRegs)
     uint32_t issued = 0;
     bool ok = true;
     if (my_iters > 0) {
-      Cursor cur = enter(0, seg_begin(0));
+      Cursor cur = enter(0, 0);
       const Cursor first = cur;
       // weight tiles do not depend on the preceding kernel: issue them first
       for (uint32_t it = 0; it < pre; ++it) {
@@ -343,11 +275,10 @@ __global__ void __maxnreg__(kGemmRegs)
         }
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + b * kPairBN;
-        const int sb = seg_begin(i), se = seg_end(i);
         const bool half = BN == 256 && item_half(seg_tile(i)) >= 0;
         const uint32_t idesc = half ? kIdescHalf : kIdesc;
         const int b_step = half ? kHalfBTile : L::kBTile;
-        for (int st = sb; st < se; ++st) {
+        for (int st = 0; st < S; ++st) {
           const int nk = min(kStageK, num_kb - st * kStageK);
           const uint64_t a_desc = a_desc0 + ((s * kHalfStage) >> 4);
           const uint64_t b_desc = b_desc0 + ((s * L::kBStage) >> 4);
@@ -361,7 +292,7 @@ __global__ void __maxnreg__(kGemmRegs)
             for (int k = 0; k < kBK / 32; ++k)
               mma_i8_pair(d_tmem, a_desc + ((h * kTileBytes) >> 4) + 2 * k,
                           b_desc + ((h * b_step) >> 4) + 2 * k, idesc,
-                          (st != sb) || h != 0 || k != 0);
+                          st != 0 || h != 0 || k != 0);
           }
           mma_commit_pair(&empty[s], pair_mask);  // frees the stage in both CTAs
           if (++s == (uint32_t)STAGES) {
@@ -383,12 +314,10 @@ __global__ void __maxnreg__(kGemmRegs)
     griddep_wait();  // a_scale comes from the preceding kernel
     constexpr int kCols = kPairBN / 2;  // columns of the tile this warp drains
     const EpiWarp ew(warp);
-    const bool first_epi_thread = threadIdx.x == 64;
     float *s_ws = reinterpret_cast<float *>(smem + L::kEpi + (warp - 2) * L::kEpiPerWarp);
     uint16_t *s_bias = reinterpret_cast<uint16_t *>(s_ws + kCols);
     uint8_t *s_out = smem + L::kOut + (warp - 2) * kEpiStagePerWarp;
-    const int r = ew.quarter * 32 + lane;  // row within this CTA's 128
-    const int j0 = ew.half * kCols;        // first tile column of this warp
+    const int j0 = ew.half * kCols;  // first tile column of this warp
     for (int i = 0; i < nseg; ++i) {
       const int tile = item_tile(seg_tile(i)), half = item_half(seg_tile(i));
       const int mb = tile % args.tiles_m, nb = tile / args.tiles_m;
@@ -398,7 +327,6 @@ __global__ void __maxnreg__(kGemmRegs)
       const int ncols = half >= 0 ? 64 : kCols;
       const int n0 = nb * kPairBN + jw;
       const uint32_t b = i & 1, bph = (i >> 1) & 1;
-      const bool whole = seg_begin(i) == 0 && seg_end(i) == S;
       stage_columns<kCols>(args, n0, lane, s_ws, s_bias);
       const float as = row0 + lane < args.M ? __ldg(args.a_scale + row0 + lane) : 0.0f;
       __syncwarp();
@@ -409,78 +337,8 @@ __global__ void __maxnreg__(kGemmRegs)
       tc_fence_after();
       const uint32_t taddr = tmem_base + b * kPairBN + (half >= 0 ? ew.half * 64 : j0) +
                              ((uint32_t)(ew.quarter * 32) << 16);
-      bool add_partial = false, partial_in_l2 = false;
-      int32_t *gpart = nullptr;
-      if (!whole) {
-        // This tile's 128 rows have one other part (the other K range).
-        // Which of the two finished first?  Sync words and partial slot: per
-        // (tile, CTA rank) for the K split; for stream-K per (range boundary,
-        // CTA rank) -- the tile cut at the boundary between pairs p - 1 and p
-        // is pair p's first segment and pair p - 1's last.
-        const int part_key = SPLIT == 3 ? ((i == 0 && st_first > 0) ? slot : slot + 1) : tile;
-        const int sidx = part_key * 2 + (int)rank;
-        unsigned long long *ctr = args.sync + 2 * sidx;  // [0] arrivals, [1] published
-        gpart = args.partials + (size_t)sidx * kPartialInts;
-        if (first_epi_thread) *arrival = (int)arrive_tagged(ctr, args.tag);
-        named_barrier_sync(1, 32 * kEpiWarps);
-        const int order = *arrival;
-        named_barrier_sync(1, 32 * kEpiWarps);  // the word is reused by the next part
-        if (order == 1) {
-          // First: publish the int32 partial (the layout of partial_index),
-          // then raise the flag once every epilogue thread's stores are out.
-          for_tmem_chunks<kCols / 32>(
-              taddr, [](int) { return true; },
-              [&](const uint32_t(&v)[32], int c) {
-#pragma unroll
-                for (int g = 0; g < 8; ++g)
-                  *reinterpret_cast<uint4 *>(gpart + partial_index(r, j0 + c * 32 + 4 * g)) =
-                      make_uint4(v[4 * g], v[4 * g + 1], v[4 * g + 2], v[4 * g + 3]);
-              });
-          __threadfence();
-          named_barrier_sync(1, 32 * kEpiWarps);
-          if (first_epi_thread) st_release_gpu(ctr + 1, args.tag);
-        } else {
-          // Second: the other part has arrived, so its partial is being or
-          // has been published.  In this CTA's last segment the stage
-          // buffers are idle and take it in one bulk copy; otherwise (rare:
-          // stream-K parts normally finish tail first) the epilogue reads it
-          // from L2.
-          const bool last = i == nseg - 1;
-          int got = 1;
-          if (first_epi_thread) {
-            got = flag_wait_bounded(ctr + 1, args.tag, abort_flag, args.status);
-            if (got && last) {
-              fence_proxy_async_global();
-              mbar_arrive_expect_tx(recv, kPartialBytes);
-              bulk_load(partial, gpart, kPartialBytes, recv);
-            }
-            *arrival = got;
-          }
-          named_barrier_sync(1, 32 * kEpiWarps);
-          got = *arrival;
-          named_barrier_sync(1, 32 * kEpiWarps);
-          if (!got) break;
-          if (last) {
-            if (lane == 0) got = mbar_wait(recv, 0, abort_flag, args.status);
-            got = __shfl_sync(0xFFFFFFFFu, got, 0);
-            if (!got) break;
-          }
-          // Both parts are done with the two words for this call: clear them,
-          // so a replayed CUDA graph (same tag) starts from zero.
-          if (first_epi_thread) {
-            ctr[0] = 0ull;
-            ctr[1] = 0ull;
-          }
-          add_partial = true;
-          partial_in_l2 = !last;
-        }
-      }
-      if (whole || add_partial)
-        // dequantise: (acc [+ the other part's partial]) * a_scale * w_scale + bias
-        epilogue_tma<kCols>(args, &tmap_y, taddr, lane, row0, n0, as, s_ws, s_bias, s_out,
-                            add_partial,
-                            PartialLoad{partial_in_l2 ? gpart : partial, r, j0, partial_in_l2},
-                            ncols);
+      // dequantise: acc * a_scale * w_scale + bias
+      epilogue_tma<kCols>(args, &tmap_y, taddr, lane, row0, n0, as, s_ws, s_bias, s_out, ncols);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive_cluster(tempty0 + b * 8);
@@ -497,14 +355,14 @@ __global__ void __maxnreg__(kGemmRegs)
   }
 }
 
-bool g_pair_attr_done[64][4];
+bool g_pair_attr_done[64][2];
 
-template <int BN, int STAGES, int SPLIT>
+template <int BN, int STAGES>
 w8a8_status run_pair(const CUtensorMap &tq, const CUtensorMap &tw, const CUtensorMap &tw64,
                      const CUtensorMap &ty, const GemmArgs &a, cudaStream_t stream, bool pdl,
                      int slot_id) {
   using L = PairSmem<BN, STAGES>;
-  auto k = gemm2sm_kernel<BN, STAGES, SPLIT>;
+  auto k = gemm2sm_kernel<BN, STAGES>;
   const int d = current_device();
   if (d < 0 || d >= 64 || !g_pair_attr_done[d][slot_id]) {
     if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kAlloc) !=
@@ -514,14 +372,8 @@ w8a8_status run_pair(const CUtensorMap &tq, const CUtensorMap &tw, const CUtenso
   }
   const int tiles = a.tiles_m * a.tiles_n;
   const int items = a.full_tiles + 2 * (tiles - a.full_tiles);
-  // SPLIT = 1: persistent, one pair per two SMs; SPLIT = 2: one pair per
-  // (tile, K half); SPLIT = 3: persistent stream-K over all SM pairs when
-  // there are more tiles than pairs (a tile then has at most two parts);
-  // with fewer tiles (a forced path, for tests) two pairs per three tiles.
-  const int sm_pairs = sm_count() / 2;
-  const int pairs = SPLIT == 1   ? std::max(1, std::min(items, sm_pairs))
-                    : SPLIT == 2 ? 2 * tiles
-                                 : (tiles >= sm_pairs ? sm_pairs : std::max(1, 2 * tiles / 3));
+  // persistent: one pair per two SMs, at most one per work item
+  const int pairs = std::max(1, std::min(items, sm_count() / 2));
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)(2 * pairs));
   cfg.blockDim = dim3(kGemmThreads + 1);  // + the producer's one-thread warp
@@ -555,23 +407,9 @@ int64_t pair_full_tiles(int64_t tiles, int64_t pairs) {
   return (tiles > pairs && rem > 0 && 2 * rem <= pairs) ? tiles - rem : tiles;
 }
 
-// Workspace of the K-split and stream-K pair kernels: per slot two 8-byte
-// sync words, then one 128 KB int32 partial per slot.  Slots: (tile, CTA
-// rank) for the K split; (range boundary, CTA rank) for stream-K, at most
-// one per SM pair plus one.
-int64_t split_slots(int64_t M, int64_t N, int split) {
-  return split == 3 ? 2 * (int64_t)(sm_count() / 2 + 1) : 2 * pair_tiles(M, N, 256);
-}
-
-int64_t split_workspace_bytes(int64_t M, int64_t N, int split) {
-  const int64_t slots = split_slots(M, N, split);
-  return round_up(slots * 16, 256) + slots * kPartialBytes;
-}
-
 w8a8_status launch_gemm2sm(const int8_t *q, const float *a_scale, const void *packed_w,
                            const float *w_scale, const void *bias, void *y, int64_t M, int64_t N,
-                           int64_t K, cudaStream_t stream, bool pdl, int split, int bn,
-                           int act, void *workspace, size_t ws_bytes) {
+                           int64_t K, cudaStream_t stream, bool pdl, int bn, int act) {
   CUtensorMap tq, tw, tw64, ty;
   if (!make_tmap_u8_2d(&tq, q, (uint64_t)M, (uint64_t)K, (uint64_t)K, kBM, kBK))
     return W8A8_ERR_CUDA;
@@ -594,26 +432,10 @@ w8a8_status launch_gemm2sm(const int8_t *q, const float *a_scale, const void *pa
   a.full_tiles = a.tiles_m * a.tiles_n;
   a.act = act;
   a.status = status_word();
-  a.sync = nullptr;
-  a.partials = nullptr;
-  a.tag = 0;
   if (!a.status) return W8A8_ERR_CUDA;
-  if (bn == 128) return run_pair<128, 4, 1>(tq, tw, tw64, ty, a, stream, pdl, 2);
-  // the K split needs at least one stage per half, stream-K at least two
-  // stages per tile; both need the workspace
-  const int S = (a.num_kb + kStageK - 1) / kStageK;
-  if ((split == 2 || split == 3) && S >= split && workspace &&
-      (int64_t)ws_bytes >= split_workspace_bytes(M, N, split)) {
-    const int64_t slots = split_slots(M, N, split);
-    uint8_t *ws = static_cast<uint8_t *>(workspace);
-    a.sync = reinterpret_cast<unsigned long long *>(ws);
-    a.partials = reinterpret_cast<int32_t *>(ws + round_up(slots * 16, 256));
-    a.tag = next_call_tag();
-    return split == 2 ? run_pair<256, 3, 2>(tq, tw, tw64, ty, a, stream, pdl, 1)
-                      : run_pair<256, 3, 3>(tq, tw, tw64, ty, a, stream, pdl, 3);
-  }
+  if (bn == 128) return run_pair<128, 4>(tq, tw, tw64, ty, a, stream, pdl, 1);
   a.full_tiles = (int)pair_full_tiles(a.full_tiles, sm_count() / 2);
-  return run_pair<256, 3, 1>(tq, tw, tw64, ty, a, stream, pdl, 0);
+  return run_pair<256, 3>(tq, tw, tw64, ty, a, stream, pdl, 0);
 }
 
 }  // namespace w8a8

@@ -49,11 +49,6 @@ struct GemmArgs {
   // as its two 128-column halves (a short last round spread over more pairs)
   int full_tiles;
   int *status;
-  // K-split pair kernel only: per (tile, CTA rank) a call-tagged arrival
-  // counter and a "partial published" flag, and the published int32 partials
-  unsigned long long *sync;
-  int32_t *partials;
-  unsigned long long tag;
 };
 
 // Epilogue warp ew (0..7): TMEM lane quarter and which half of the columns.
@@ -188,28 +183,15 @@ __device__ __forceinline__ uint32_t swz64_offset(int r, int c16) {
 //   taddr   TMEM address of the first column, this warp's lane quarter
 //   row0    output row of lane 0;  n0: output column of the first column
 //   s_ws / s_bias: the COLS columns' scales and bias, staged in smem
-//   has_extra / extra_load: an int32 partial added to the accumulator first;
-//           extra_load(j) returns this lane's four values at column j..j+3
 //   ncols   columns actually drained (a multiple of 32, at most COLS)
-template <int COLS, typename ExtraLoad>
+template <int COLS>
 __device__ __forceinline__ void epilogue_tma(const GemmArgs &a, const CUtensorMap *tmap_y,
                                              uint32_t taddr, int lane, int row0, int n0, float as,
                                              const float *s_ws, const uint16_t *s_bias,
-                                             uint8_t *stage, bool has_extra,
-                                             ExtraLoad extra_load, int ncols = COLS) {
+                                             uint8_t *stage, int ncols = COLS) {
   for_tmem_chunks<COLS / 32>(
       taddr, [&](int c) { return c * 32 < ncols && n0 + c * 32 < a.N; },
-      [&](uint32_t(&v)[32], int c) {
-        if (has_extra) {
-#pragma unroll
-          for (int g = 0; g < 8; ++g) {
-            const uint4 p = extra_load(c * 32 + 4 * g);
-            v[4 * g] += p.x;
-            v[4 * g + 1] += p.y;
-            v[4 * g + 2] += p.z;
-            v[4 * g + 3] += p.w;
-          }
-        }
+      [&](const uint32_t(&v)[32], int c) {
         uint4 out[4];
 #pragma unroll
         for (int g = 0; g < 4; ++g)
@@ -227,9 +209,5 @@ __device__ __forceinline__ void epilogue_tma(const GemmArgs &a, const CUtensorMa
         }
       });
 }
-
-struct NoExtra {
-  __device__ uint4 operator()(int) const { return make_uint4(0, 0, 0, 0); }
-};
 
 }  // namespace w8a8

@@ -6,12 +6,31 @@
 #include <stddef.h>
 #include <stdint.h>
 
+#include <mutex>
+
 #include "w8a8.h"
 
 namespace w8a8 {
 
 // Device pointer to this device's status word (0 = OK, else a w8a8_status).
 int *status_word();
+
+// Unique ID of the current CUDA context (false if none is current).
+bool current_context_id(unsigned long long *id);
+
+// One cached device address of a __device__ variable, valid for the context
+// it was looked up in.
+struct SymbolCache {
+  std::mutex mu;
+  bool valid = false;
+  unsigned long long ctx_id = 0;
+  void *addr = nullptr;
+};
+
+// The device address of `symbol` (the host-side name of a __device__
+// variable) in the current context, from the cache while that context is the
+// one it was looked up in, else from cudaGetSymbolAddress.
+bool symbol_address(SymbolCache *cache, const void *symbol, void **out);
 
 // Number of SMs of the current device (cached per device).
 int sm_count();
@@ -60,24 +79,16 @@ inline int64_t packed_cols(int64_t K) { return round_up(K, 128); }
 w8a8_status launch_scaled_mm(const int8_t *q, const float *a_scale, const void *packed_w,
                              const float *w_scale, const void *bias, void *out, bool out_i32,
                              int64_t M, int64_t N, int64_t K, cudaStream_t stream, bool pdl,
-                             int act = W8A8_ACT_NONE, void *workspace = nullptr,
-                             size_t ws_bytes = 0);
-// Workspace w8a8_scaled_mm can use for (M, N, K) with M above the small-M
-// range (0 when the chosen kernel needs none).
-int64_t large_workspace_bytes(int64_t M, int64_t N, int64_t K);
-// The part of w8a8_linear's workspace it cannot run without.
-int64_t linear_workspace_min(int64_t M, int64_t N, int64_t K);
-// 2-SM (CTA pair) GEMM with the bf16 epilogue (gemm2sm.cu).
+                             int act = W8A8_ACT_NONE);
+// Workspace of w8a8_linear: codes, scales and (small M) the decode partials.
+int64_t linear_workspace_bytes(int64_t M, int64_t N, int64_t K);
+// 2-SM (CTA pair) GEMM with the bf16 epilogue (gemm2sm.cu); bn = 256 or 128.
 w8a8_status launch_gemm2sm(const int8_t *q, const float *a_scale, const void *packed_w,
                            const float *w_scale, const void *bias, void *y, int64_t M, int64_t N,
-                           int64_t K, cudaStream_t stream, bool pdl, int split, int bn,
-                           int act = W8A8_ACT_NONE, void *workspace = nullptr,
-                           size_t ws_bytes = 0);
+                           int64_t K, cudaStream_t stream, bool pdl, int bn,
+                           int act = W8A8_ACT_NONE);
 int64_t pair_tiles(int64_t M, int64_t N, int bn);
 int64_t pair_full_tiles(int64_t tiles, int64_t pairs);
-// Workspace the K-split (split = 2) or stream-K (split = 3) pair kernel needs
-// (sync words + int32 partials).
-int64_t split_workspace_bytes(int64_t M, int64_t N, int split);
 // Small-M weight-streaming kernel (decode.cu).
 int64_t decode_workspace_bytes(int64_t N, int64_t K);
 bool use_decode_path(int64_t M);

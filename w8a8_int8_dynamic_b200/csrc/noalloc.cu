@@ -14,7 +14,10 @@
 // library holds kNoAllocScratchBytes of it until the process exits.  Host code
 // cannot use the array's name as a device address (it is a host-side stand-in),
 // so the first call on each device looks the address up with
-// cudaGetSymbolAddress while that device is current and caches it.
+// cudaGetSymbolAddress while that device is current and keeps it.  The kept
+// address belongs to the CUDA context it was looked up in: it is reused only
+// while that same context (by its process-wide unique ID) is current, and
+// looked up again after a device reset or under another context.
 #include <mutex>
 
 #include "internal.h"
@@ -27,22 +30,34 @@ constexpr size_t kNoAllocScratchBytes = size_t(8) << 20;  // 8 MiB per device
 __device__ __align__(256) uint8_t g_noalloc_scratch[kNoAllocScratchBytes];
 
 constexpr int kMaxDevices = 64;
-void *g_scratch_addr[kMaxDevices];
-std::mutex g_scratch_mu;
+struct ScratchSlot {
+  bool valid;
+  unsigned long long ctx_id;
+  void *addr;
+};
+ScratchSlot g_scratch[kMaxDevices];
+std::mutex g_scratch_mu;  // guards every read and write of g_scratch
 
-// Device address of this device's scratch array (set-up on first use).
+// Device address of the scratch array in the current context (set-up on the
+// first call in each context).
 w8a8_status scratch_address(void **out) {
   const int d = current_device();
   if (d < 0 || d >= kMaxDevices) return W8A8_ERR_CUDA;
-  if (!g_scratch_addr[d]) {
-    std::lock_guard<std::mutex> lk(g_scratch_mu);
-    if (!g_scratch_addr[d]) {
-      void *p = nullptr;
-      if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return W8A8_ERR_CUDA;
-      g_scratch_addr[d] = p;
-    }
+  std::lock_guard<std::mutex> lk(g_scratch_mu);
+  ScratchSlot &slot = g_scratch[d];
+  unsigned long long id = 0;
+  bool have_id = current_context_id(&id);
+  if (have_id && slot.valid && slot.ctx_id == id) {
+    *out = slot.addr;
+    return W8A8_OK;
   }
-  *out = g_scratch_addr[d];
+  void *p = nullptr;
+  if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return W8A8_ERR_CUDA;
+  if (!have_id) have_id = current_context_id(&id);  // the lookup may have created it
+  slot.valid = have_id;
+  slot.ctx_id = id;
+  slot.addr = p;
+  *out = p;
   return W8A8_OK;
 }
 
@@ -60,10 +75,7 @@ extern "C" w8a8_status w8a8_linear_noalloc(const void *x, int64_t ldx, const voi
   size_t need = 0;
   const w8a8_status st = w8a8_linear_workspace_bytes(M, N, K, &need);
   if (st != W8A8_OK) return st;
-  // the layer runs in any workspace of at least the minimum; the rest of the
-  // scratch serves the GEMM's K-split partials when they fit
-  if (linear_workspace_min(M, N, K) > (int64_t)kNoAllocScratchBytes)
-    return W8A8_ERR_BUFFER_TOO_SMALL;
+  if (need > kNoAllocScratchBytes) return W8A8_ERR_BUFFER_TOO_SMALL;
   void *scratch = nullptr;
   const w8a8_status sa = scratch_address(&scratch);
   if (sa != W8A8_OK) return sa;

@@ -14,13 +14,21 @@ __device__ int g_status_word;
 
 namespace {
 constexpr int kMaxDevices = 64;
-int *g_status_ptr[kMaxDevices];
 int g_sm_count[kMaxDevices];
 std::mutex g_mu;
 std::atomic<int64_t> g_launches{0};
 std::atomic<int> g_forced_path{0};
 std::atomic<unsigned long long> g_call_tag{0};
 PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+
+// Driver entry points that identify the current CUDA context.
+using CtxGetCurrentFn = CUresult (*)(CUcontext *);
+using CtxGetIdFn = CUresult (*)(CUcontext, unsigned long long *);
+std::once_flag g_ctx_fns_once;
+CtxGetCurrentFn g_ctx_get_current = nullptr;
+CtxGetIdFn g_ctx_get_id = nullptr;
+
+SymbolCache g_status_cache;
 }  // namespace
 
 int current_device() {
@@ -29,18 +37,53 @@ int current_device() {
   return d;
 }
 
-int *status_word() {
-  const int d = current_device();
-  if (d < 0 || d >= kMaxDevices) return nullptr;
-  if (!g_status_ptr[d]) {
-    std::lock_guard<std::mutex> lk(g_mu);
-    if (!g_status_ptr[d]) {
-      void *p = nullptr;
-      if (cudaGetSymbolAddress(&p, g_status_word) != cudaSuccess) return nullptr;
-      g_status_ptr[d] = static_cast<int *>(p);
-    }
+bool current_context_id(unsigned long long *id) {
+  std::call_once(g_ctx_fns_once, [] {
+    void *fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &fn, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      g_ctx_get_current = reinterpret_cast<CtxGetCurrentFn>(fn);
+    fn = nullptr;
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &fn, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      g_ctx_get_id = reinterpret_cast<CtxGetIdFn>(fn);
+  });
+  if (!g_ctx_get_current || !g_ctx_get_id) return false;
+  CUcontext c = nullptr;
+  if (g_ctx_get_current(&c) != CUDA_SUCCESS || !c) return false;
+  return g_ctx_get_id(c, id) == CUDA_SUCCESS;
+}
+
+// The device address of a __device__ variable in the current context.  A
+// cached address is reused only while the same context (by its process-wide
+// unique ID, which a context created after a device reset does not share) is
+// current; otherwise it is looked up again.  The mutex covers every read and
+// write of the cache.
+bool symbol_address(SymbolCache *cache, const void *symbol, void **out) {
+  std::lock_guard<std::mutex> lk(cache->mu);
+  unsigned long long id = 0;
+  bool have_id = current_context_id(&id);
+  if (have_id && cache->valid && cache->ctx_id == id) {
+    *out = cache->addr;
+    return true;
   }
-  return g_status_ptr[d];
+  void *p = nullptr;
+  if (cudaGetSymbolAddress(&p, symbol) != cudaSuccess || !p) return false;
+  // the lookup may itself have made the device's primary context current
+  if (!have_id) have_id = current_context_id(&id);
+  cache->valid = have_id;
+  cache->ctx_id = id;
+  cache->addr = p;
+  *out = p;
+  return true;
+}
+
+int *status_word() {
+  void *p = nullptr;
+  if (!symbol_address(&g_status_cache, reinterpret_cast<const void *>(&g_status_word), &p))
+    return nullptr;
+  return static_cast<int *>(p);
 }
 
 int sm_count() {
@@ -153,7 +196,7 @@ const char *w8a8_status_string(int status) {
 int w8a8_abi_version(void) { return (1 << 16) | 0; }
 
 w8a8_status w8a8_set_path(int path) {
-  if (path < 0 || path > 8) return W8A8_ERR_INVALID_ARG;
+  if (path < 0 || path > 7 || path == 6) return W8A8_ERR_INVALID_ARG;
   g_forced_path.store(path);
   return W8A8_OK;
 }
