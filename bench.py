@@ -1,22 +1,29 @@
 """Benchmark of the W8A8 int8-dynamic linear path on B200.
 
-One step = one pass of the hot path over one batch: dynamic per-token int8
-quantisation of the activations, the int8 x int8 -> int32 tensor-core GEMM
-against pre-packed int8 weights, and the dequantising bf16 epilogue
-(w8a8_linear), on the square 512 x 4096 x 4096 projection with bias and an
-all-zero row.  Weights are packed once before timing (load time).
+One step = one pass of the hot path over one batch.  The default step is the
+DiT transformer-block MLP at image-token scale (4096 tokens): the
+up-projection 3072 -> 12288 with GELU(tanh) in its epilogue, then the
+row-parallel down-projection 12288 -> 3072 fed its bf16 output.  Each layer
+is w8a8_linear: dynamic per-token int8 quantisation of its input, the
+int8 x int8 -> int32 tensor-core GEMM against weights packed once before
+timing (load time), and the dequantising bf16 epilogue.  ``--workload NAME``
+times a single layer of another workload instead.
 
-Prints ONE JSON line (rank 0).  ``value`` is whole-job int8 TOPS (2*M*N*K per
-step, summed over ranks, divided by the max-over-ranks device time).  Inputs
-rotate over enough buffer sets to exceed the 126 MB L2, and each set's step is
-replayed from a CUDA graph so host launch overhead stays out of the device
-timing.  Also reported: the dominant kernel's roofline (GEMM alone, CUDA
-events on its stream), an end-to-end figure through the public API with
-host buffers, the oracle's CPU throughput, SM clocks sampled during the timed
-region, and a sweep over the other workloads.
+Prints ONE JSON line (rank 0).  ``value`` is whole-job int8 TOPS (2*M*N*K of
+every layer of every step, summed over ranks, divided by the max-over-ranks
+device time).  Inputs rotate over enough buffer sets to exceed the 126 MB L2
+between two uses, and consecutive steps are replayed from CUDA graphs so host
+launch overhead stays out of the device timing.  Also reported: the dominant
+kernel's roofline (the GEMM, timed alone with CUDA events on its stream), an
+end-to-end figure through the public API with host buffers, the oracle's CPU
+throughput, SM clocks sampled during the timed region, and a compact sweep
+over the other workloads.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                  [--no-sweep] [--workload NAME]
+                  [--workload NAME] [--no-sweep] [--no-cpu-baseline]
+  python bench.py --profile MODE --workload NAME [--reps R]
+      runs one workload's kernels R times as separate launches, without
+      graphs, for ncu (MODE: layer, gemm, quant, gelu, block)
 """
 from __future__ import annotations
 
@@ -37,12 +44,26 @@ sys.path.insert(0, HERE)
 
 from w8a8_int8_dynamic_b200.workloads import WORKLOADS, make_inputs  # noqa: E402
 
-MAIN_WORKLOAD = "square_512x4096x4096"
+ACT_NONE, ACT_GELU = 0, 1  # w8a8_act
+# The DiT MLP block: (layer workload, epilogue activation), each layer fed the
+# previous one's output.
+BLOCK = "dit_mlp_block_4096x3072x12288"
+CHAINS = {BLOCK: (("dit_mlp_up_4096x12288x3072", ACT_GELU),
+                  ("dit_mlp_down_4096x3072x12288", ACT_NONE))}
+MAIN_WORKLOAD = BLOCK
+METRIC = "W8A8 quant+scaled-GEMM TOPS and % of int8 roofline on one B200"
 # where the raw nvidia-smi clock samples go (--clocks-dir); the JSON line
 # carries their summary either way
 CLOCKS_DIR = os.path.join(tempfile.gettempdir(), "w8a8_bench_clocks")
 L2_BYTES = 126 * 1024 * 1024
 SPEC_INT8_TOPS = 4500.0
+
+
+def chain_of(name):
+    """The layers of a workload name: a chain, or one plain layer."""
+    if name in CHAINS:
+        return CHAINS[name]
+    return ((name, ACT_NONE),)
 
 
 # ----------------------------------------------------------------------------- peaks
@@ -57,25 +78,34 @@ def load_peaks():
             "source": "fallback"}
 
 
-# the sources the dominant kernel is compiled from (a change voids the record)
-TRAFFIC_SOURCES = ("gemm.cu", "gemm_common.cuh", "act.cuh", "ptx.cuh")
+# the sources each GEMM kernel is compiled from (a change voids its record)
+TRAFFIC_SOURCES = {
+    "gemm_kernel": ("gemm.cu", "gemm_common.cuh", "act.cuh", "ptx.cuh"),
+    "gemm2sm_kernel": ("gemm2sm.cu", "gemm_common.cuh", "act.cuh", "ptx.cuh"),
+    "decode_kernel": ("decode.cu", "gemm_common.cuh", "act.cuh", "ptx.cuh"),
+}
+
+
+def sources_hash(kernel):
+    import hashlib
+    csrc = os.path.join(HERE, "w8a8_int8_dynamic_b200", "csrc")
+    h = hashlib.sha256()
+    for f in TRAFFIC_SOURCES[kernel]:
+        h.update(open(os.path.join(csrc, f), "rb").read())
+    return h.hexdigest()[:16]
 
 
 def recorded_traffic(workload):
-    """DRAM bytes per launch of the GEMM from the committed ncu capture, or
-    None when there is none or the kernel sources changed since it was taken."""
-    import hashlib
+    """DRAM bytes per launch of a workload's GEMM from the committed ncu
+    capture, or None when there is none or the kernel's sources changed
+    since it was taken."""
     path = os.path.join(HERE, "profiles", "traffic.json")
     if not os.path.exists(path):
         return None
     rec = json.load(open(path)).get(workload)
-    if not rec:
+    if not rec or rec.get("kernel_family") not in TRAFFIC_SOURCES:
         return None
-    csrc = os.path.join(HERE, "w8a8_int8_dynamic_b200", "csrc")
-    h = hashlib.sha256()
-    for f in TRAFFIC_SOURCES:
-        h.update(open(os.path.join(csrc, f), "rb").read())
-    if h.hexdigest()[:16] != rec.get("source_sha256_16"):
+    if sources_hash(rec["kernel_family"]) != rec.get("source_sha256_16"):
         return None
     return rec.get("gemm_bytes_per_launch")
 
@@ -146,69 +176,49 @@ def bf16_dev(a_u16: np.ndarray, device) -> torch.Tensor:
     return torch.from_numpy(np.ascontiguousarray(a_u16).view(np.int16)).to(device).view(torch.bfloat16)
 
 
-def algorithmic(wl, M=None):
-    M = wl.M if M is None else M
-    N, K = wl.N, wl.K
-    bias = 2 * N if wl.bias else 0
+def algorithmic(M, N, K, bias):
+    """2MNK ops; GEMM bytes MK + NK + 2MN + scales (+ bias); quantisation
+    bytes 3MK + 4M; the layer's bytes without the int8 round trip of q."""
+    b = 2 * N if bias else 0
     ops = 2 * M * N * K
-    gemm_bytes = M * K + N * K + 2 * M * N + 4 * M + 4 * N + bias
+    gemm_bytes = M * K + N * K + 2 * M * N + 4 * M + 4 * N + b
     quant_bytes = 3 * M * K + 4 * M
-    fused_bytes = 2 * M * K + N * K + 2 * M * N + 4 * N + bias
+    fused_bytes = 2 * M * K + N * K + 2 * M * N + 4 * N + b
     return ops, gemm_bytes, quant_bytes, fused_bytes
 
 
-class LayerSets:
-    """``nsets`` independent copies of a workload's tensors on the device."""
-
-    def __init__(self, w8, wl, nsets, device, M=None):
-        inp = make_inputs(wl, M)
-        self.M, self.N, self.K = inp.x.shape[0], wl.N, wl.K
-        self.sets = []
-        x0 = bf16_dev(inp.x, device)
-        w0 = torch.from_numpy(inp.w).to(device)
-        packed0 = w8.pack_weight(w0)
-        del w0
-        ws0 = torch.from_numpy(inp.w_scale).to(device)
-        b0 = None if inp.bias is None else bf16_dev(inp.bias, device)
-        wsb = w8.linear_workspace_bytes(self.M, self.N, self.K)
-        mmws = w8.scaled_mm_workspace_bytes(self.M, self.N, self.K)
-        for i in range(nsets):
-            s = {
-                "x": x0 if i == 0 else x0.clone(),
-                "packed": packed0 if i == 0 else packed0.clone(),
-                "w_scale": ws0 if i == 0 else ws0.clone(),
-                "bias": None if b0 is None else (b0 if i == 0 else b0.clone()),
-                "y": torch.empty((self.M, self.N), dtype=torch.bfloat16, device=device),
-                "ws": torch.empty((wsb,), dtype=torch.uint8, device=device),
-                "mmws": torch.empty((max(mmws, 16),), dtype=torch.uint8, device=device)
-                if mmws else None,
-            }
-            s["q"], s["a_scale"] = w8.quant_act(s["x"])
-            self.sets.append(s)
-        torch.cuda.synchronize()
-
-    def set_bytes(self):
-        s = self.sets[0]
-        return sum(t.numel() * t.element_size() for k, t in s.items()
-                   if isinstance(t, torch.Tensor))
+def chain_shapes(names, M=None):
+    """(M, N, K, bias) of each layer of a chain."""
+    out = []
+    for name, _ in names:
+        wl = WORKLOADS[name]
+        out.append((wl.M if M is None else M, wl.N, wl.K, wl.bias))
+    return out
 
 
-def sets_needed(w8, wl, M=None):
-    """Input sets to rotate over so that every timed loop -- the layer, the
-    GEMM alone, the quantisation alone -- touches more than L2 (x 1.5)
-    between two uses of the same set.  A quantisation too small to exceed L2
-    even over 16 sets (it is latency-bound then) does not count."""
-    probe_M = wl.M if M is None else M
-    M, N, K = probe_M, wl.N, wl.K
-    per = (M * K * 3 + N * K + 2 * M * N + 8 * N + w8.linear_workspace_bytes(M, N, K))
-    footprints = [per, M * K + N * K + 2 * M * N]  # the layer; the GEMM alone (q, W, y)
-    if 16 * 3 * M * K > 1.5 * L2_BYTES:
-        footprints.append(3 * M * K)  # the quantisation alone (x, q)
-    smallest = min(footprints)
+def footprints(shapes, layer_ws):
+    """Bytes each timed loop touches per input set: the whole step, each
+    layer's GEMM alone (q, W, y) and each layer's quantisation alone (x, q).
+    A quantisation too small to exceed L2 even over 16 sets (it is
+    latency-bound then) does not count."""
+    step = sum(3 * M * K + N * K + 2 * M * N + 8 * N + ws
+               for (M, N, K, _), ws in zip(shapes, layer_ws))
+    fp = {"step": step}
+    for i, (M, N, K, _) in enumerate(shapes):
+        fp[f"gemm{i}"] = M * K + N * K + 2 * M * N
+        if 16 * 3 * M * K > 1.5 * L2_BYTES:
+            fp[f"quant{i}"] = 3 * M * K
+    return fp
+
+
+def sets_needed(fp):
+    """Input sets to rotate over so that every timed loop touches more than
+    L2 (x 1.5) between two uses of the same set (at most 16)."""
+    smallest = min(fp.values())
     n = 1
     while n * smallest <= 1.5 * L2_BYTES and n < 16:
         n += 1
-    return n, per
+    return n
 
 
 def capture(fns, stream):
@@ -270,75 +280,164 @@ def time_loop(loop, steps, stream):
     return start.elapsed_time(end) / 1e3  # seconds
 
 
-# ----------------------------------------------------------------------------- our arm
-def run_workload(w8, wl, steps, warmup, device, stream, M=None, with_quant=True,
-                 gemm_clock_tag=None):
-    nsets, _ = sets_needed(w8, wl, M)
-    ls = LayerSets(w8, wl, nsets, device, M)
-    steps_fns, mm_fns, q_fns = [], [], []
-    for s in ls.sets:
-        def step(s=s):
-            w8.linear(s["x"], s["packed"], s["w_scale"], s["bias"], ls.N, out=s["y"],
-                      workspace=s["ws"], stream=stream)
-        def mm(s=s):
-            w8.scaled_mm(s["q"], s["a_scale"], s["packed"], s["w_scale"], s["bias"], ls.N,
-                         out=s["y"], workspace=s["mmws"], stream=stream)
-        def qa(s=s):
-            w8.quant_act(s["x"], q=s["q"], a_scale=s["a_scale"], stream=stream)
-        steps_fns.append(step)
-        mm_fns.append(mm)
-        q_fns.append(qa)
+def per_graph_for(t_step_estimate):
+    """Steps per captured graph: about 1 ms of work, between 4 and 64."""
+    return int(min(64, max(4, 1e-3 / max(t_step_estimate, 1e-7))))
+
+
+# ----------------------------------------------------------------------------- chains
+class Layer:
+    """One W8A8 layer of one input set on the device."""
+
+    def __init__(self, w8, wl, act, inp, device, clone_of=None):
+        self.wl, self.act = wl, act
+        self.M, self.N, self.K = inp.x.shape[0], wl.N, wl.K
+        if clone_of is None:
+            self.packed = w8.pack_weight(torch.from_numpy(inp.w).to(device))
+            self.w_scale = torch.from_numpy(inp.w_scale).to(device)
+            self.bias = None if inp.bias is None else bf16_dev(inp.bias, device)
+        else:
+            self.packed = clone_of.packed.clone()
+            self.w_scale = clone_of.w_scale.clone()
+            self.bias = None if clone_of.bias is None else clone_of.bias.clone()
+        M, N, K = self.M, self.N, self.K
+        self.y = torch.empty((M, N), dtype=torch.bfloat16, device=device)
+        self.ws = torch.empty((w8.linear_workspace_bytes(M, N, K),), dtype=torch.uint8,
+                              device=device)
+        mm = w8.scaled_mm_workspace_bytes(M, N, K)
+        self.mmws = torch.empty((mm,), dtype=torch.uint8, device=device) if mm else None
+        self.q = torch.empty((M, K), dtype=torch.int8, device=device)
+        self.a = torch.empty((M,), dtype=torch.float32, device=device)
+
+
+class ChainSets:
+    """``nsets`` independent copies of a chain's tensors on the device (the
+    first layer's input x, every layer's packed weight, scales, bias, output
+    and workspaces)."""
+
+    def __init__(self, w8, names, nsets, device, M=None):
+        self.names = names
+        inps = [make_inputs(WORKLOADS[n], M) for n, _ in names]
+        self.M = inps[0].x.shape[0]
+        x0 = bf16_dev(inps[0].x, device)
+        self.sets = []
+        for i in range(nsets):
+            first = self.sets[0] if self.sets else None
+            layers = [Layer(w8, WORKLOADS[n], act, inp, device,
+                            None if first is None else first["layers"][j])
+                      for j, ((n, act), inp) in enumerate(zip(names, inps))]
+            self.sets.append({"x": x0 if i == 0 else x0.clone(), "layers": layers})
+        del inps
+        torch.cuda.synchronize()
+
+    def inputs(self, s):
+        """The input tensor of each layer of set s."""
+        return [s["x"]] + [L.y for L in s["layers"][:-1]]
+
+    def set_bytes(self):
+        s = self.sets[0]
+        n = s["x"].numel() * 2
+        for L in s["layers"]:
+            for t in (L.packed, L.w_scale, L.bias, L.y, L.ws, L.mmws, L.q, L.a):
+                if t is not None:
+                    n += t.numel() * t.element_size()
+        return n
+
+
+def run_chain(w8, cs, s, stream):
+    x = s["x"]
+    for L in s["layers"]:
+        w8.linear(x, L.packed, L.w_scale, L.bias, L.N, out=L.y, workspace=L.ws, stream=stream,
+                  act=L.act)
+        x = L.y
+
+
+def measure_chain(w8, names, steps, warmup, device, stream, with_layers=True, M=None,
+                  long_gemm_clock=False, warm_gemm=False):
+    """Times the chain step, and (with_layers) each layer's GEMM alone and
+    quantisation alone, each over rotated input sets in CUDA graphs."""
+    shapes = chain_shapes(names, M)
+    ws_bytes = [w8.linear_workspace_bytes(m, n, k) for m, n, k, _ in shapes]
+    nsets = sets_needed(footprints(shapes, ws_bytes))
+    cs = ChainSets(w8, names, nsets, device, M)
     with torch.cuda.stream(stream):
-        for f in steps_fns[:1] + mm_fns[:1] + q_fns[:1]:
-            f()  # warm the launch path (attributes, tensor maps) before capture
+        for s in cs.sets:
+            run_chain(w8, cs, s, stream)  # warm the launch path; layer inputs exist
+        for s in cs.sets:
+            for L, x in zip(s["layers"], cs.inputs(s)):
+                w8.quant_act(x, q=L.q, a_scale=L.a, stream=stream)
     torch.cuda.synchronize()
     c0 = w8.launch_count()
-    capture([steps_fns[0]], stream)
+    capture([lambda: run_chain(w8, cs, cs.sets[0], stream)], stream)
     per_step = w8.launch_count() - c0
-    layer_loop = GraphLoop(steps_fns, stream)
-    mm_loop = GraphLoop(mm_fns, stream)
-    q_loop = GraphLoop(q_fns, stream)
-    for loop in (layer_loop, mm_loop, q_loop):
-        loop.prepare(steps)
+    ops = [algorithmic(*sh)[0] for sh in shapes]
+    est = sum(ops) / 2.0e15
+    step_loop = GraphLoop([lambda s=s: run_chain(w8, cs, s, stream) for s in cs.sets], stream,
+                          per_graph_for(est))
+    loops = {"step": step_loop}
+    if with_layers:
+        for i in range(len(names)):
+            def mm(s, i=i):
+                L = s["layers"][i]
+                w8.scaled_mm(L.q, L.a, L.packed, L.w_scale, L.bias, L.N, out=L.y,
+                             workspace=L.mmws, stream=stream, act=L.act)
+
+            def qa(s, i=i):
+                L = s["layers"][i]
+                w8.quant_act(cs.inputs(s)[i], q=L.q, a_scale=L.a, stream=stream)
+            # (each callable binds this layer's functions: the loops' tail
+            # graphs are captured after this loop has moved on)
+            loops[f"gemm{i}"] = GraphLoop([lambda s=s, f=mm: f(s) for s in cs.sets], stream,
+                                          per_graph_for(ops[i] / 2.0e15))
+            loops[f"quant{i}"] = GraphLoop([lambda s=s, f=qa: f(s) for s in cs.sets], stream,
+                                           per_graph_for(3e-6))
+            if warm_gemm:
+                # the same set over and over: operands resident in L2 when they fit
+                loops[f"gemm{i}_warm"] = GraphLoop([lambda f=mm: f(cs.sets[0])], stream,
+                                                   per_graph_for(ops[i] / 2.0e15))
+    for lp in loops.values():
+        lp.prepare(steps)
     torch.cuda.synchronize()
     assert w8.poll_status() == 0
-    for loop in (layer_loop, mm_loop, q_loop):
-        time_loop(loop, max(warmup, 3) * loop.per_graph, stream)
-    res = {"launches_per_step": per_step, "nsets": nsets, "set_bytes": ls.set_bytes(),
-           "M": ls.M, "N": ls.N, "K": ls.K}
-    res["t_step"] = time_loop(layer_loop, steps, stream) / steps
-    res["t_gemm"] = time_loop(mm_loop, steps, stream) / steps
-    if gemm_clock_tag is not None:
-        # the GEMM alone again, long enough (>= 0.6 s) for the clock sampler:
-        # a tensor-bound loop may run under the power cap
-        per = mm_loop.per_graph
-        n = max(steps, int(0.6 / res["t_gemm"]) // per * per)
-        cs = ClockSampler(smi_index(device), tag=gemm_clock_tag)
-        cs.start()
-        res["t_gemm_long"] = time_loop(mm_loop, n, stream) / n
-        res["gemm_clock"] = cs.stop()
-    if with_quant:
-        res["t_quant"] = time_loop(q_loop, steps, stream) / steps
+    for lp in loops.values():
+        time_loop(lp, max(warmup, 3) * lp.per_graph, stream)
+    res = {"launches_per_step": per_step, "nsets": nsets, "set_bytes": cs.set_bytes(),
+           "shapes": shapes, "ops": ops}
+    for k, lp in loops.items():
+        res["t_" + k] = time_loop(lp, steps, stream) / steps
+    if long_gemm_clock:
+        # each GEMM again, long enough (>= 0.6 s) for the clock sampler: a
+        # tensor-bound loop may run under the power cap
+        for i in range(len(names)):
+            lp = loops[f"gemm{i}"]
+            n = max(steps, int(0.6 / res[f"t_gemm{i}"]) // lp.per_graph * lp.per_graph)
+            cs_ = ClockSampler(smi_index(device), tag=f"_gemm{i}")
+            cs_.start()
+            res[f"t_gemm{i}_long"] = time_loop(lp, n, stream) / n
+            res[f"gemm{i}_clock"] = cs_.stop()
     assert w8.poll_status() == 0, "device-side timeout during the benchmark"
-    return ls, layer_loop, res
+    return cs, step_loop, res
 
 
+# ----------------------------------------------------------------------------- our arm
 def run_ours(args, rank, world, device):
     import w8a8_int8_dynamic_b200 as w8
     w8.lib()
     peaks = load_peaks()
     int8_peak = 2.0 * peaks["bf16_tflops"]  # nominal int8 : bf16 dense rate = 2
     stream = torch.cuda.Stream(device=device)
-    wl = WORKLOADS[args.workload]
-    ops, gemm_bytes, quant_bytes, fused_bytes = algorithmic(wl)
+    names = chain_of(args.workload)
 
-    ls, layer_loop, base = run_workload(w8, wl, 2000, args.warmup, device, stream)
-    layer_loop.prepare(args.steps)
+    cs, step_loop, base = measure_chain(w8, names, 2000 if len(names) == 1 else 400,
+                                        args.warmup, device, stream, long_gemm_clock=True)
+    shapes, ops_l = base["shapes"], base["ops"]
+    ops = sum(ops_l)
+    step_loop.prepare(args.steps)
     torch.cuda.synchronize()
     # ---- the timed region: exactly K steps, barrier + sync on both sides
     sampler = ClockSampler(smi_index(device))
     sampler.start()
-    time_loop(layer_loop, args.warmup, stream)  # W untimed warm-up steps
+    time_loop(step_loop, args.warmup, stream)  # W untimed warm-up steps
     if world > 1:
         torch.distributed.barrier()
     torch.cuda.synchronize()
@@ -346,7 +445,7 @@ def run_ours(args, rank, world, device):
     end = torch.cuda.Event(enable_timing=True)
     with torch.cuda.stream(stream):
         start.record(stream)
-        layer_loop.run(args.steps)
+        step_loop.run(args.steps)
         end.record(stream)
     end.synchronize()
     torch.cuda.synchronize()
@@ -355,74 +454,110 @@ def run_ours(args, rank, world, device):
     elapsed = start.elapsed_time(end) / 1e3
     clocks = sampler.stop()
     assert w8.poll_status() == 0, "device-side timeout during the timed region"
-    t_max = elapsed
-    if world > 1:
-        t = torch.tensor([elapsed], dtype=torch.float64, device=device)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        t_max = float(t.item())
-    value = ops * args.steps * world / t_max / 1e12
+    t_max = max_over_ranks(elapsed, world, device)
+    value = whole_job_tops(ops, args.steps, world, t_max)
     ms_per_step = t_max / args.steps * 1e3
+    per_graph = step_loop.per_graph
 
-    # ---- dominant kernel (the GEMM) alone, CUDA events on its stream
-    gemm_tops = ops / base["t_gemm"] / 1e12
-    roofline = {"bound": "tensor", "achieved": round(gemm_tops, 2), "peak": round(int8_peak, 1),
-                "unit": "TOPS", "frac": round(gemm_tops / int8_peak, 4), "traffic": None,
-                "kernel": w8.gemm_kernel_name(wl.M, wl.N, wl.K),
-                "peak_note": f"int8 = 2 x {peaks['source']} bf16 burst {peaks['bf16_tflops']} TFLOP/s",
-                "frac_vs_spec_4500": round(gemm_tops / SPEC_INT8_TOPS, 4),
-                "gemm_us": round(base["t_gemm"] * 1e6, 3),
-                "quant_us": round(base["t_quant"] * 1e6, 3),
-                "quant_gbs": round(quant_bytes / base["t_quant"] / 1e9, 1),
-                "quant_frac_hbm": round(quant_bytes / base["t_quant"] / 1e9 / peaks["hbm_gbs"], 4)}
-    roofline["traffic"] = recorded_traffic(args.workload)
+    # ---- dominant kernel: the GEMM of every layer, each timed alone; the
+    # algorithmic ops of one launch over the mean launch duration
+    t_g = [base[f"t_gemm{i}"] for i in range(len(names))]
+    gemm_tops = ops / sum(t_g) / 1e12
+    kernels = [w8.gemm_kernel_name(M, N, K) for M, N, K, _ in shapes]
+    traffic = [recorded_traffic(n) for n, _ in names]
+    roofline = {
+        "bound": "tensor", "achieved": round(gemm_tops, 1), "peak": round(int8_peak, 1),
+        "unit": "TOPS", "frac": round(gemm_tops / int8_peak, 4),
+        "traffic": None if None in traffic else int(sum(traffic) / len(traffic)),
+        "kernel": kernels[0].split(" (")[0] if len(set(kernels)) == 1 else kernels,
+        "peak_note": f"2 x {peaks['source']} bf16 burst",
+        "frac_vs_spec_4500": round(gemm_tops / SPEC_INT8_TOPS, 4),
+        "ops_per_launch": ops_l[0] if len(set(ops_l)) == 1 else ops_l,
+        "gemm_us": [round(t * 1e6, 2) for t in t_g],
+        "quant_us": [round(base[f"t_quant{i}"] * 1e6, 2) for i in range(len(names))],
+        "quant_frac_hbm": [round(algorithmic(*sh)[2] / base[f"t_quant{i}"] / 1e9 /
+                                 peaks["hbm_gbs"], 4) for i, sh in enumerate(shapes)],
+    }
+    sustained = 2.0 * peaks["bf16_tflops_sustained"]
+    t_long = [base[f"t_gemm{i}_long"] for i in range(len(names))]
+    clk = [base[f"gemm{i}_clock"] for i in range(len(names))]
+    roofline["long_loop"] = {
+        "frac_of_sustained": round(ops / sum(t_long) / 1e12 / sustained, 4),
+        "sustained_peak": round(sustained, 1),
+        "sm_mhz": [c["sm_mhz"] for c in clk],
+        "reasons": sorted({r for c in clk for r in c["reasons"]})}
+    t_roof = 0.0
+    for sh in shapes:
+        o, _, _, fused = algorithmic(*sh)
+        t_roof += max(o / (int8_peak * 1e12), fused / (peaks["hbm_gbs"] * 1e9))
 
     # ---- end to end through the public API, host buffers
-    e2e = run_e2e(w8, ls, args, stream, ops)
+    e2e = run_e2e(w8, cs, args, stream, ops)
+    del cs, step_loop
+    torch.cuda.empty_cache()
 
+    first = WORKLOADS[names[0][0]]
     out = {
-        "metric": "W8A8 quant+scaled-GEMM TOPS and % of int8 roofline on one B200",
+        "metric": METRIC,
         "value": round(value, 2), "unit": "TOPS", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(ms_per_step, 5), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "int8 x int8 -> int32, bf16 in/out",
-        "data": "synthetic (seeded; N(0,1) activations with 1% outlier channels x10, "
-                "int8 weights uniform [-127,127], fp32 scales, bf16 bias)",
-        "config": {"workload": args.workload, "M": wl.M, "N": wl.N, "K": wl.K,
-                   "step": "w8a8_linear = quant kernel + tcgen05 GEMM/epilogue (2 launches, PDL)",
-                   "l2": f"rotating {base['nsets']} input sets of {base['set_bytes'] / 2**20:.1f} MiB "
-                         f"(> 126 MB L2)",
-                   "launch": "CUDA graphs of 64 consecutive steps over the rotated sets",
+        "data": "synthetic, seeded (workloads.py recipe)",
+        "config": {"workload": args.workload, "M": first.M if len(names) > 1 else shapes[0][0],
+                   "layers": [f"{M}x{N}x{K}" + ("+gelu" if a else "")
+                              for (M, N, K, _), (_, a) in zip(shapes, names)],
+                   "step": f"{len(names)} x w8a8_linear (quant kernel + tcgen05 GEMM/epilogue, PDL)",
+                   "l2": f"{base['nsets']} rotated input sets of "
+                         f"{base['set_bytes'] / 2**20:.0f} MiB (> 126 MB L2)",
+                   "launch": f"CUDA graphs of {per_graph} steps",
                    "parallelism": f"replicas x{world}"},
         "roofline": roofline,
-        "fused_frac_of_roofline": round(max(ops / (int8_peak * 1e12),
-                                            fused_bytes / (peaks["hbm_gbs"] * 1e9)) / (t_max / args.steps),
-                                        4),
+        "step_frac_of_roofline": round(t_roof / (t_max / args.steps), 4),
         "e2e": e2e,
         "gpu_launches": int(base["launches_per_step"] * args.steps),
-        "clocks": clocks,
+        "clocks": {k: clocks[k] for k in ("sm_mhz", "sm_max_mhz", "reasons")},
     }
     if rank == 0 and not args.no_cpu_baseline:
-        out["cpu_baseline"] = cpu_baseline(wl, budget_s=args.cpu_seconds)
+        out["cpu_baseline"] = cpu_baseline(names, budget_s=args.cpu_seconds)
     if not args.no_sweep:
+        out["sweep_cols"] = SWEEP_COLS
         out["sweep"] = sweep(w8, args, device, stream, peaks, int8_peak)
-        out["mlp_chain"] = mlp_chain(w8, device, stream)
+        if args.workload == BLOCK:
+            out["block_unfused_us"] = block_unfused(w8, device, stream)
     return out
 
 
-def run_e2e(w8, ls, args, stream, ops):
-    """Public API, host buffers: per step H2D of x from pinned memory, the
-    layer call, D2H of y into pinned memory, all inside the timed region.
-    Steps are pipelined the way a serving loop would run them: the upload of
-    step i+1, the layer of step i and the download of step i-1 overlap on
-    three streams (PCIe is full duplex), with three device buffer sets."""
-    s0 = ls.sets[0]
-    M, N, K = ls.M, ls.N, ls.K
+def max_over_ranks(elapsed, world, device):
+    """The slowest rank's time: every rank takes part (one all-reduce)."""
+    if world == 1:
+        return elapsed
+    t = torch.tensor([elapsed], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_tops(ops_per_step, steps, world, t_max):
+    """Replicas: every rank runs `steps` steps; the job's throughput is all
+    ranks' work over the slowest rank's time."""
+    return ops_per_step * steps * world / t_max / 1e12
+
+
+def run_e2e(w8, cs, args, stream, ops):
+    """Public API, host buffers: per step H2D of the first layer's input from
+    pinned memory, the layers, D2H of the last layer's output into pinned
+    memory, all inside the timed region.  Steps are pipelined the way a
+    serving loop would run them: the upload of step i+1, the layers of step
+    i and the download of step i-1 overlap on three streams (PCIe is full
+    duplex), with three device buffer sets."""
+    s0 = cs.sets[0]
+    ndev = min(3, len(cs.sets))
+    nhost = 4
     dev = s0["x"].device
-    nhost, ndev = 4, 3
+    x_shape = tuple(s0["x"].shape)
+    y_shape = tuple(s0["layers"][-1].y.shape)
     xs = [s0["x"].cpu().pin_memory() for _ in range(nhost)]
-    ys = [torch.empty((M, N), dtype=torch.bfloat16).pin_memory() for _ in range(nhost)]
-    xd = [torch.empty_like(s0["x"]) for _ in range(ndev)]
-    yd = [torch.empty((M, N), dtype=torch.bfloat16, device=dev) for _ in range(ndev)]
-    layer_args = (s0["packed"], s0["w_scale"], s0["bias"], N)
+    ys = [torch.empty(y_shape, dtype=torch.bfloat16).pin_memory() for _ in range(nhost)]
+    dsets = [cs.sets[i] for i in range(ndev)]
     up, down = torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev)
     comp = stream
     ev_in = [torch.cuda.Event() for _ in range(ndev)]
@@ -431,23 +566,24 @@ def run_e2e(w8, ls, args, stream, ops):
 
     def step(i, first):
         b = i % ndev
+        d = dsets[b]
         if not first[b]:
-            up.wait_event(ev_done[b])        # x[b] free: the layer that read it is done
+            up.wait_event(ev_done[b])        # x[b] free: the layers that read it are done
         with torch.cuda.stream(up):
-            xd[b].copy_(xs[i % nhost], non_blocking=True)
+            d["x"].copy_(xs[i % nhost], non_blocking=True)
             ev_in[b].record(up)
         comp.wait_event(ev_in[b])
         if not first[b]:
             comp.wait_event(ev_out[b])       # y[b] free: its download is done
-        w8.linear(xd[b], *layer_args, out=yd[b], workspace=s0["ws"], stream=comp)
+        run_chain(w8, cs, d, comp)
         ev_done[b].record(comp)
         down.wait_event(ev_done[b])
         with torch.cuda.stream(down):
-            ys[i % nhost].copy_(yd[b], non_blocking=True)
+            ys[i % nhost].copy_(d["layers"][-1].y, non_blocking=True)
             ev_out[b].record(down)
         first[b] = False
 
-    steps = max(10, min(args.steps, 2000))
+    steps = max(10, min(args.steps, 200))
     first = [True] * ndev
     for i in range(3):
         step(i, first)
@@ -465,178 +601,207 @@ def run_e2e(w8, ls, args, stream, ops):
     end.synchronize()
     t = start.elapsed_time(end) / 1e3 / steps
     # the last step's output must have arrived
-    assert torch.equal(ys[(steps - 1) % nhost].to(dev), yd[(steps - 1) % ndev])
-    return {"value": round(ops / t / 1e12, 3), "unit": "TOPS", "h2d_bytes_per_step": M * K * 2,
-            "d2h_bytes_per_step": M * N * 2, "steps": steps, "ms_per_step": round(t * 1e3, 4),
-            "pipelining": "H2D of step i+1, layer of step i and D2H of step i-1 on three streams",
-            "api": "w8a8_int8_dynamic_b200.linear (ctypes -> w8a8_linear)"}
+    last = dsets[(steps - 1) % ndev]["layers"][-1].y
+    assert torch.equal(ys[(steps - 1) % nhost].to(dev), last)
+    xb = int(np.prod(x_shape)) * 2
+    yb = int(np.prod(y_shape)) * 2
+    return {"value": round(ops / t / 1e12, 2), "unit": "TOPS", "h2d_bytes_per_step": xb,
+            "d2h_bytes_per_step": yb, "steps": steps, "ms_per_step": round(t * 1e3, 4),
+            "overlap": "H2D i+1 | layers i | D2H i-1, 3 streams", "api": "w8a8_linear_act"}
+
+
+# compact sweep rows: one list per workload, columns named once
+SWEEP_COLS = ["kernel", "step_us", "gemm_us", "quant_us", "gemm_frac", "quant_frac_hbm",
+              "step_frac", "gemm_us_warm"]
+SWEEP = ["small_64x128x256", "square_512x4096x4096", "fused_qkv_512x12288x4096",
+         "dit_mlp_up_4096x12288x3072", "dit_mlp_down_4096x3072x12288",
+         "decode_m1_27648x5120", "decode_m4_27648x5120", "decode_m16_27648x5120"]
+
+
+def short_kernel(name):
+    """'gemm2sm_kernel<256, 3> (...)' -> 'pair256'."""
+    if name.startswith("decode"):
+        return "decode"
+    if name.startswith("gemm2sm"):
+        return "pair" + name.split("<")[1].split(",")[0]
+    return "1sm" + name.split("<")[1].split(",")[0]
 
 
 def sweep(w8, args, device, stream, peaks, int8_peak):
+    """Every workload as one layer: step (quant + GEMM), GEMM alone (cold
+    operands; warm too where they fit L2), quantisation alone.  gemm_frac is
+    t_roof / t for the GEMM (tensor or HBM bound, whichever is slower),
+    quant_frac_hbm the quantisation's fraction of HBM bandwidth, step_frac the
+    layer's fraction of its roofline."""
     out = {}
-    names = ["small_64x128x256", "square_512x4096x4096", "fused_qkv_512x12288x4096",
-             "dit_mlp_up_4096x12288x3072", "dit_mlp_down_4096x3072x12288",
-             "decode_m1_27648x5120", "decode_m4_27648x5120", "decode_m16_27648x5120"]
-    for name in names:
+    for name in SWEEP:
         wl = WORKLOADS[name]
-        ops, gemm_bytes, quant_bytes, fused_bytes = algorithmic(wl)
-        steps = 256 if wl.M * wl.N * wl.K > 1e11 else 2048
-        bound = "tensor" if ops / (int8_peak * 1e12) >= gemm_bytes / (peaks["hbm_gbs"] * 1e9) else "hbm"
-        ls, loop, r = run_workload(w8, wl, steps, 3, device, stream,
-                                   gemm_clock_tag=("_gemm_" + name) if bound == "tensor" else None)
+        ops, gemm_bytes, quant_bytes, fused_bytes = algorithmic(wl.M, wl.N, wl.K, wl.bias)
+        steps = 200 if ops > 1e11 else 2000
+        warm = wl.N * wl.K + wl.M * wl.K + 2 * wl.M * wl.N < L2_BYTES // 2
+        cs, loop, r = measure_chain(w8, ((name, ACT_NONE),), steps, 3, device, stream,
+                                    warm_gemm=warm)
         t_roof_gemm = max(ops / (int8_peak * 1e12), gemm_bytes / (peaks["hbm_gbs"] * 1e9))
-        t_roof_fused = max(ops / (int8_peak * 1e12), fused_bytes / (peaks["hbm_gbs"] * 1e9))
-        out[name] = {
-            "M": wl.M, "N": wl.N, "K": wl.K, "bound": bound,
-            "step_us": round(r["t_step"] * 1e6, 3), "gemm_us": round(r["t_gemm"] * 1e6, 3),
-            "quant_us": round(r["t_quant"] * 1e6, 3),
-            "step_tops": round(ops / r["t_step"] / 1e12, 2),
-            "gemm_tops": round(ops / r["t_gemm"] / 1e12, 2),
-            "gemm_gbs": round(gemm_bytes / r["t_gemm"] / 1e9, 1),
-            "gemm_frac_roofline": round(t_roof_gemm / r["t_gemm"], 4),
-            "gemm_frac_spec_int8": round(ops / r["t_gemm"] / 1e12 / SPEC_INT8_TOPS, 4),
-            "quant_gbs": round(quant_bytes / r["t_quant"] / 1e9, 1),
-            "quant_frac_hbm": round(quant_bytes / r["t_quant"] / 1e9 / peaks["hbm_gbs"], 4),
-            "step_frac_roofline": round(t_roof_fused / r["t_step"], 4),
-            "l2_sets": r["nsets"],
-            "kernel": w8.gemm_kernel_name(wl.M, wl.N, wl.K),
-        }
-        if "gemm_clock" in r:
-            # a long GEMM loop with its clocks: under the power cap the
-            # sustained bf16 rate (x 2 for int8) is the ceiling it can reach
-            sustained = 2.0 * peaks["bf16_tflops_sustained"]
-            tops_long = ops / r["t_gemm_long"] / 1e12
-            out[name]["gemm_long_loop"] = {
-                "us": round(r["t_gemm_long"] * 1e6, 3), "tops": round(tops_long, 1),
-                "sm_mhz": r["gemm_clock"]["sm_mhz"], "reasons": r["gemm_clock"]["reasons"],
-                "frac_of_sustained": round(tops_long / sustained, 4),
-                "sustained_peak_tops": round(sustained, 1)}
-        del ls, loop
+        t_roof_step = max(ops / (int8_peak * 1e12), fused_bytes / (peaks["hbm_gbs"] * 1e9))
+        row = [short_kernel(w8.gemm_kernel_name(wl.M, wl.N, wl.K)),
+               round(r["t_step"] * 1e6, 2), round(r["t_gemm0"] * 1e6, 2),
+               round(r["t_quant0"] * 1e6, 2), round(t_roof_gemm / r["t_gemm0"], 3),
+               round(quant_bytes / r["t_quant0"] / 1e9 / peaks["hbm_gbs"], 3),
+               round(t_roof_step / r["t_step"], 3)]
+        if warm:
+            row.append(round(r["t_gemm0_warm"] * 1e6, 2))
+        out[name] = row
+        del cs, loop
         torch.cuda.empty_cache()
     return out
 
 
-def mlp_chain(w8, device, stream, steps=128, nsets=2):
-    """The DiT MLP block (4096 tokens, 3072 -> 12288 -> 3072): the two W8A8
-    layers with the GELU between them, unfused (layer, GELU kernel, layer)
-    and with the GELU in the up-projection's epilogue."""
-    up_wl = WORKLOADS["dit_mlp_up_4096x12288x3072"]
-    dn_wl = WORKLOADS["dit_mlp_down_4096x3072x12288"]
-    up, dn = make_inputs(up_wl), make_inputs(dn_wl)
-    M, H, D = up_wl.M, up_wl.N, up_wl.K
-    sets = []
-    for i in range(nsets):
-        s = {"x": bf16_dev(up.x, device),
-             "pu": w8.pack_weight(torch.from_numpy(up.w).to(device)),
-             "su": torch.from_numpy(up.w_scale).to(device), "bu": bf16_dev(up.bias, device),
-             "pd": w8.pack_weight(torch.from_numpy(dn.w).to(device)),
-             "sd": torch.from_numpy(dn.w_scale).to(device), "bd": bf16_dev(dn.bias, device),
-             "h": torch.empty((M, H), dtype=torch.bfloat16, device=device),
-             "g": torch.empty((M, H), dtype=torch.bfloat16, device=device),
-             "y": torch.empty((M, D), dtype=torch.bfloat16, device=device),
-             "wsu": torch.empty((w8.linear_workspace_bytes(M, H, D),), dtype=torch.uint8,
-                                device=device),
-             "wsd": torch.empty((w8.linear_workspace_bytes(M, D, H),), dtype=torch.uint8,
-                                device=device)}
-        sets.append(s)
-    def unfused(s):
-        w8.linear(s["x"], s["pu"], s["su"], s["bu"], H, out=s["h"], workspace=s["wsu"], stream=stream)
-        w8.gelu_tanh(s["h"], out=s["g"], stream=stream)
-        w8.linear(s["g"], s["pd"], s["sd"], s["bd"], D, out=s["y"], workspace=s["wsd"], stream=stream)
-    def fused(s):
-        w8.linear(s["x"], s["pu"], s["su"], s["bu"], H, out=s["g"], workspace=s["wsu"],
-                  stream=stream, act=w8.ACT_GELU_TANH)
-        w8.linear(s["g"], s["pd"], s["sd"], s["bd"], D, out=s["y"], workspace=s["wsd"], stream=stream)
-    def up_only(s, act):
-        w8.linear(s["x"], s["pu"], s["su"], s["bu"], H, out=s["g"], workspace=s["wsu"],
-                  stream=stream, act=act)
-    loops = {
-        "unfused": GraphLoop([lambda s=s: unfused(s) for s in sets], stream, per_graph=8),
-        "fused": GraphLoop([lambda s=s: fused(s) for s in sets], stream, per_graph=8),
-        "up_layer": GraphLoop([lambda s=s: up_only(s, w8.ACT_NONE) for s in sets], stream, 16),
-        "up_layer_gelu": GraphLoop([lambda s=s: up_only(s, w8.ACT_GELU_TANH) for s in sets],
-                                   stream, 16),
-        "gelu_kernel": GraphLoop([lambda s=s: w8.gelu_tanh(s["h"], out=s["g"], stream=stream)
-                                  for s in sets], stream, 16),
-    }
-    torch.cuda.synchronize()
-    for lp in loops.values():
-        time_loop(lp, 3 * lp.per_graph, stream)
-    ops = 2 * (2 * M * H * D)
-    out = {"tokens": M, "dims": [D, H, D]}
-    for name, lp in loops.items():
-        # long enough (>= 0.6 s) for the clock sampler to see the loop
-        t0 = time_loop(lp, lp.per_graph, stream) / lp.per_graph
-        n = max(steps, int(0.6 / t0) // lp.per_graph * lp.per_graph)
-        cs = ClockSampler(smi_index(device), tag="_mlp_" + name)
-        cs.start()
-        t = time_loop(lp, n, stream) / n
-        clk = cs.stop()
-        out[name + "_us"] = round(t * 1e6, 2)
-        out[name + "_sm_mhz"] = clk["sm_mhz"]
-        if clk["reasons"]:
-            out[name + "_clock_reasons"] = clk["reasons"]
-    for name in ("unfused", "fused"):
-        out[name + "_tops"] = round(ops / (out[name + "_us"] * 1e-6) / 1e12, 1)
+def block_unfused(w8, device, stream, nsets=2, steps=64):
+    """The DiT MLP block with the GELU as a kernel of its own between the
+    layers (layer, GELU kernel, layer), for comparison with the headline
+    step, where the GELU runs in the up-projection's epilogue."""
+    names = CHAINS[BLOCK]
+    cs = ChainSets(w8, names, nsets, device)
+    gs = [torch.empty_like(s["layers"][0].y) for s in cs.sets]
+
+    def unfused(s, g):
+        Lu, Ld = s["layers"]
+        w8.linear(s["x"], Lu.packed, Lu.w_scale, Lu.bias, Lu.N, out=Lu.y, workspace=Lu.ws,
+                  stream=stream)
+        w8.gelu_tanh(Lu.y, out=g, stream=stream)
+        w8.linear(g, Ld.packed, Ld.w_scale, Ld.bias, Ld.N, out=Ld.y, workspace=Ld.ws,
+                  stream=stream)
+    lp = GraphLoop([lambda s=s, g=g: unfused(s, g) for s, g in zip(cs.sets, gs)], stream, 4)
+    lp.prepare(steps)
+    time_loop(lp, 3 * lp.per_graph, stream)
+    t = time_loop(lp, steps, stream) / steps
     assert w8.poll_status() == 0
-    del sets, loops
+    del cs, gs, lp
     torch.cuda.empty_cache()
-    return out
+    return round(t * 1e6, 2)
 
 
 # ----------------------------------------------------------------------------- CPU oracle
-def cpu_baseline(wl, budget_s=12.0):
-    """The oracle as it stands, on the host cores: whole layers of the same
-    workload, repeated until about budget_s seconds have elapsed."""
+def oracle_chain(oracle, names, x, inps):
+    """The chain through the oracle: each layer, then GELU where it has one."""
+    for (name, act), inp in zip(names, inps):
+        x = oracle.linear(x, inp.w, inp.w_scale, inp.bias)[0]
+        if act == ACT_GELU:
+            x = oracle.gelu_tanh(x)
+    return x
+
+
+def cpu_baseline(names, budget_s=12.0):
+    """The oracle as it stands, on the host cores: whole steps of the same
+    workload (every layer at full size), repeated until about budget_s
+    seconds have elapsed; plus single-thread figures for the three smaller
+    workloads (a row sample of each)."""
     import oracle
-    inp = make_inputs(wl)
-    ops = 2 * wl.M * wl.N * wl.K
-    oracle.linear(inp.x[:8], inp.w[:64], inp.w_scale[:64], None if inp.bias is None else inp.bias[:64])
+    inps = [make_inputs(WORKLOADS[n]) for n, _ in names]
+    ops = sum(algorithmic(*sh)[0] for sh in chain_shapes(names))
+    oracle_chain(oracle, names, inps[0].x[:4], inps)  # load and touch
     t0 = time.perf_counter()
     reps = 0
     while True:
-        oracle.linear(inp.x, inp.w, inp.w_scale, inp.bias)
+        oracle_chain(oracle, names, inps[0].x, inps)
         reps += 1
         if time.perf_counter() - t0 >= budget_s or reps >= 50:
             break
     t = (time.perf_counter() - t0) / reps
-    return {"value": round(ops / t / 1e12, 5), "unit": "TOPS", "cores": oracle.num_threads(),
+    cores = oracle.num_threads()
+    single = {}
+    oracle.set_num_threads(1)
+    try:
+        for name, rows in (("small_64x128x256", 64), ("square_512x4096x4096", 32),
+                           ("fused_qkv_512x12288x4096", 16)):
+            wl = WORKLOADS[name]
+            inp = make_inputs(wl)
+            x = inp.x[:rows]
+            t1 = time.perf_counter()
+            oracle.linear(x, inp.w, inp.w_scale, inp.bias)
+            dt = time.perf_counter() - t1
+            single[name] = [round(2 * rows * wl.N * wl.K / dt / 1e12, 5), rows]
+    finally:
+        oracle.set_num_threads(cores)
+    del inps
+    return {"value": round(ops / t / 1e12, 5), "unit": "TOPS", "cores": cores,
             "kind": "oracle",
-            "sample": f"{reps} full {wl.name} layers (quant + int32 GEMM + epilogue), "
-                      f"{t:.3f} s each, OpenMP over rows"}
+            "sample": f"{reps} whole step(s) of {len(names)} full layer(s), {t:.2f} s each",
+            "single_thread_tops_rows": single}
 
 
 def run_reference(args):
-    wl = WORKLOADS[args.workload]
+    """The oracle, as it stands, on the host cores: each step a bounded
+    sample of the same workload (its first rows through every layer)."""
     import oracle
-    inp = make_inputs(wl)
-    ops = 2 * wl.M * wl.N * wl.K
-    # bounded sample per step: a slice of rows of the same workload
-    rows = max(1, min(wl.M, int(args.ref_rows)))
-    x = inp.x[:rows]
+    names = chain_of(args.workload)
+    inps = [make_inputs(WORKLOADS[n]) for n, _ in names]
+    shapes = chain_shapes(names)
+    M = shapes[0][0]
+    rows = max(1, min(M, int(args.ref_rows)))
+    x = inps[0].x[:rows]
     for _ in range(args.warmup):
-        oracle.linear(x, inp.w, inp.w_scale, inp.bias)
+        oracle_chain(oracle, names, x, inps)
     t0 = time.perf_counter()
     for _ in range(args.steps):
-        oracle.linear(x, inp.w, inp.w_scale, inp.bias)
+        oracle_chain(oracle, names, x, inps)
     t = (time.perf_counter() - t0) / args.steps
-    sample_ops = 2 * rows * wl.N * wl.K
+    sample_ops = sum(2 * rows * N * K for _, N, K, _ in shapes)
+    full_ops = sum(algorithmic(*sh)[0] for sh in shapes)
     value = sample_ops / t / 1e12
     return {
-        "metric": "W8A8 quant+scaled-GEMM TOPS and % of int8 roofline on one B200",
-        "impl": "reference", "value": round(value, 5), "unit": "TOPS", "n_gpus": 1,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(t * 1e3, 3),
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-        "dtype": "int8 x int8 -> int32, bf16 in/out", "data": "synthetic (seeded)",
-        "config": {"workload": args.workload, "M": wl.M, "N": wl.N, "K": wl.K,
+        "metric": METRIC, "impl": "reference", "value": round(value, 5), "unit": "TOPS",
+        "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(t * 1e3, 3), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "int8 x int8 -> int32, bf16 in/out",
+        "data": "synthetic (seeded)",
+        "config": {"workload": args.workload, "M": M,
+                   "layers": [f"{m}x{n}x{k}" for m, n, k, _ in shapes],
                    "sample_rows_per_step": rows},
         "cpu_baseline": {"value": round(value, 5), "unit": "TOPS", "cores": oracle.num_threads(),
                          "kind": "oracle",
-                         "sample": f"{rows} of {wl.M} rows of {wl.name} per step "
-                                   f"({sample_ops / ops:.3f} of a layer)"},
+                         "sample": f"{rows} of {M} rows through every layer per step "
+                                   f"({sample_ops / full_ops:.4f} of a step)"},
         "e2e": {"value": round(value, 5), "unit": "TOPS", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
     }
+
+
+# ----------------------------------------------------------------------------- profiling
+def run_profile(args):
+    """A workload's kernels as separate launches (no graphs), so that ncu can
+    select them with -k / -s / -c.  MODE layer: w8a8_linear; gemm: the
+    quantisation then the GEMM alone; quant: the quantisation; gelu: the
+    GELU kernel over the layer's output shape; block: the chain."""
+    import w8a8_int8_dynamic_b200 as w8
+    device = torch.device("cuda", 0)
+    torch.cuda.set_device(device)
+    stream = torch.cuda.current_stream()
+    names = chain_of(args.workload)
+    cs = ChainSets(w8, names, 1, device)
+    s = cs.sets[0]
+    mode = args.profile
+    L0 = s["layers"][0]
+    g_in = None
+    if mode == "gelu":
+        g_in = torch.randn(L0.M, L0.N, device=device,
+                           generator=torch.Generator(device).manual_seed(0)).to(torch.bfloat16)
+    for _ in range(args.reps):
+        if mode in ("block", "layer"):
+            run_chain(w8, cs, s, stream)
+        elif mode == "gelu":
+            w8.gelu_tanh(g_in, out=L0.y)
+        else:
+            for L, x in zip(s["layers"], cs.inputs(s)):
+                w8.quant_act(x, q=L.q, a_scale=L.a)
+                if mode == "gemm":
+                    w8.scaled_mm(L.q, L.a, L.packed, L.w_scale, L.bias, L.N, out=L.y,
+                                 workspace=L.mmws, act=L.act)
+    torch.cuda.synchronize()
+    st = w8.poll_status()
+    if st != 0:
+        raise SystemExit(f"device status {st}")
+    print("done", args.workload, mode, args.reps)
 
 
 # ----------------------------------------------------------------------------- main
@@ -644,20 +809,26 @@ def main():
     global CLOCKS_DIR
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20000)
+    ap.add_argument("--steps", type=int, default=4000)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", default=MAIN_WORKLOAD, choices=list(WORKLOADS))
+    ap.add_argument("--workload", default=MAIN_WORKLOAD, choices=list(CHAINS) + list(WORKLOADS))
     ap.add_argument("--no-sweep", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--cpu-seconds", type=float, default=12.0)
-    ap.add_argument("--ref-rows", type=int, default=64)
+    ap.add_argument("--cpu-seconds", type=float, default=5.0)
+    ap.add_argument("--ref-rows", type=int, default=32)
+    ap.add_argument("--profile", choices=["layer", "gemm", "quant", "gelu", "block"], default=None)
+    ap.add_argument("--reps", type=int, default=3)
     ap.add_argument("--clocks-dir", default=None,
                     help="directory for the raw clock samples (default: a temporary one)")
     args = ap.parse_args()
     if args.clocks_dir:
         CLOCKS_DIR = os.path.abspath(args.clocks_dir)
     args.warmup = max(args.warmup, 3)
+
+    if args.profile:
+        run_profile(args)
+        return 0
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -677,7 +848,7 @@ def main():
     try:
         out = run_ours(args, rank, world, device)
         if rank == 0:
-            print(json.dumps(out), flush=True)
+            print(json.dumps(out, separators=(",", ":")), flush=True)
     finally:
         if world > 1:
             torch.distributed.destroy_process_group()

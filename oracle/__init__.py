@@ -42,6 +42,8 @@ def lib():
         L.w8a8o_bf16_to_f32.argtypes = [ctypes.c_uint16]
         L.w8a8o_bf16_to_f32.restype = ctypes.c_float
         L.w8a8o_num_threads.restype = ctypes.c_int
+        L.w8a8o_set_num_threads.argtypes = [ctypes.c_int]
+        L.w8a8o_set_num_threads.restype = None
         L.w8a8o_quant_weight.argtypes = [P, I64, I64, P, P]
         L.w8a8o_quant_act_static.argtypes = [P, I64, I64, I64, ctypes.c_float, P, P]
         L.w8a8o_unpack_int32.argtypes = [P, I64, I64, P]
@@ -62,6 +64,11 @@ def _check(rc, what):
 
 def num_threads() -> int:
     return lib().w8a8o_num_threads()
+
+
+def set_num_threads(n: int) -> None:
+    """Threads used by later calls (OpenMP); for timing the oracle alone."""
+    lib().w8a8o_set_num_threads(int(n))
 
 
 def quant_act(x_bf16: np.ndarray):

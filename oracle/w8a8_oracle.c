@@ -344,3 +344,13 @@ int w8a8o_num_threads(void) {
   return 1;
 #endif
 }
+
+/* Sets the number of threads later calls use (for single-thread timings). */
+void w8a8o_set_num_threads(int n) {
+#ifdef _OPENMP
+  extern void omp_set_num_threads(int);
+  if (n > 0) omp_set_num_threads(n);
+#else
+  (void)n;
+#endif
+}

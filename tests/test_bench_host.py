@@ -89,48 +89,69 @@ def test_graph_loop_prepare_is_idempotent(fake_capture):
     assert len(captured) == n
 
 
-class FakeW8:
-    def __init__(self, ws):
-        self.ws = ws
-
-    def linear_workspace_bytes(self, M, N, K):
-        return self.ws
-
-
 def test_sets_needed_exceeds_l2_for_every_timed_loop():
-    wl = bench.WORKLOADS[bench.MAIN_WORKLOAD]
-    w8 = FakeW8(ws=wl.M * wl.K + 4 * wl.M)
-    n, per = bench.sets_needed(w8, wl)
-    M, N, K = wl.M, wl.N, wl.K
-    gemm_alone = M * K + N * K + 2 * M * N
-    # the smallest timed footprint (the GEMM alone) times n exceeds 1.5 x L2 ...
-    assert n * min(per, gemm_alone) > 1.5 * bench.L2_BYTES
+    names = bench.chain_of(bench.MAIN_WORKLOAD)
+    shapes = bench.chain_shapes(names)
+    ws = [M * K + 4 * M for M, N, K, _ in shapes]
+    fp = bench.footprints(shapes, ws)
+    # the step, both GEMMs and both quantisations are timed loops of the block
+    assert set(fp) == {"step", "gemm0", "gemm1", "quant0", "quant1"}
+    n = bench.sets_needed(fp)
+    smallest = min(fp.values())
+    # the smallest timed footprint times n exceeds 1.5 x L2 ...
+    assert n * smallest > 1.5 * bench.L2_BYTES
     # ... and n is the smallest count that does
-    assert (n - 1) * min(per, gemm_alone) <= 1.5 * bench.L2_BYTES
-    assert per > gemm_alone
+    assert (n - 1) * smallest <= 1.5 * bench.L2_BYTES
+    (M0, N0, K0, _), (M1, N1, K1, _) = shapes
+    assert fp["gemm0"] == M0 * K0 + N0 * K0 + 2 * M0 * N0
+    assert fp["quant0"] == 3 * M0 * K0
+    assert fp["step"] > fp["gemm0"] + fp["gemm1"]
 
 
 def test_sets_needed_is_capped_for_tiny_workloads():
-    class WL:
-        M, N, K = 16, 256, 256
-    n, _ = bench.sets_needed(FakeW8(ws=0), WL)
-    assert n == 16
+    fp = bench.footprints([(16, 256, 256, False)], [0])
+    assert "quant0" not in fp  # too small to exceed L2 even over 16 sets
+    assert bench.sets_needed(fp) == 16
+
+
+def test_block_chain_is_the_dit_mlp_config():
+    """The headline step: up-projection 3072 -> 12288 with GELU in its
+    epilogue, then the row-parallel down-projection 12288 -> 3072, 4096
+    tokens, each layer a full-size workload."""
+    names = bench.chain_of(bench.MAIN_WORKLOAD)
+    assert [a for _, a in names] == [bench.ACT_GELU, bench.ACT_NONE]
+    assert bench.chain_shapes(names) == [(4096, 12288, 3072, True), (4096, 3072, 12288, True)]
+    ops = sum(bench.algorithmic(*s)[0] for s in bench.chain_shapes(names))
+    assert ops == 2 * 2 * 4096 * 12288 * 3072
+    assert bench.chain_of("square_512x4096x4096") == (("square_512x4096x4096", bench.ACT_NONE),)
+
+
+def test_whole_job_value_and_compact_kernel_names():
+    assert bench.whole_job_tops(1e12, 10, 2, 0.5) == pytest.approx(40.0)
+    assert bench.short_kernel("gemm2sm_kernel<256, 3> (2-SM pair, 256x256 tiles)") == "pair256"
+    assert bench.short_kernel("gemm_kernel<128, 3, 2> (1-SM, 128x128 tiles)") == "1sm128"
+    assert bench.short_kernel("decode_kernel (swap-AB stream-K, needs a workspace)") == "decode"
 
 
 def test_recorded_traffic_only_while_the_sources_match(tmp_path, monkeypatch):
     csrc = tmp_path / "w8a8_int8_dynamic_b200" / "csrc"
     csrc.mkdir(parents=True)
-    for i, f in enumerate(bench.TRAFFIC_SOURCES):
+    fam = "gemm2sm_kernel"
+    for i, f in enumerate(bench.TRAFFIC_SOURCES[fam]):
         (csrc / f).write_bytes(f"// source {i}\n".encode())
     h = hashlib.sha256()
-    for f in bench.TRAFFIC_SOURCES:
+    for f in bench.TRAFFIC_SOURCES[fam]:
         h.update((csrc / f).read_bytes())
     (tmp_path / "profiles").mkdir()
-    rec = {"square": {"gemm_bytes_per_launch": 123, "source_sha256_16": h.hexdigest()[:16]}}
+    rec = {"mlp": {"gemm_bytes_per_launch": 123, "kernel_family": fam,
+                   "source_sha256_16": h.hexdigest()[:16]},
+           "odd": {"gemm_bytes_per_launch": 5, "kernel_family": "unknown",
+                   "source_sha256_16": h.hexdigest()[:16]}}
     (tmp_path / "profiles" / "traffic.json").write_text(json.dumps(rec))
     monkeypatch.setattr(bench, "HERE", str(tmp_path))
-    assert bench.recorded_traffic("square") == 123
+    assert bench.sources_hash(fam) == h.hexdigest()[:16]
+    assert bench.recorded_traffic("mlp") == 123
     assert bench.recorded_traffic("other") is None
-    (csrc / bench.TRAFFIC_SOURCES[-1]).write_bytes(b"// changed\n")
-    assert bench.recorded_traffic("square") is None
-
+    assert bench.recorded_traffic("odd") is None
+    (csrc / bench.TRAFFIC_SOURCES[fam][-1]).write_bytes(b"// changed\n")
+    assert bench.recorded_traffic("mlp") is None
