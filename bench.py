@@ -45,11 +45,15 @@ sys.path.insert(0, HERE)
 from w8a8_int8_dynamic_b200.workloads import WORKLOADS, make_inputs  # noqa: E402
 
 ACT_NONE, ACT_GELU = 0, 1  # w8a8_act
-# The DiT MLP block: (layer workload, epilogue activation), each layer fed the
-# previous one's output.
+# A chain of layers, each fed the previous one's output: (layer workload,
+# epilogue activation, whether the layer also forms the next layer's codes).
+# A layer that does runs w8a8_linear_act_quant, and the next one then runs
+# the scaled GEMM on those codes; any other layer runs w8a8_linear_act.
+# The DiT MLP block: the up-projection with GELU in its epilogue and the
+# down-projection's quantisation fused in, then the down-projection.
 BLOCK = "dit_mlp_block_4096x3072x12288"
-CHAINS = {BLOCK: (("dit_mlp_up_4096x12288x3072", ACT_GELU),
-                  ("dit_mlp_down_4096x3072x12288", ACT_NONE))}
+CHAINS = {BLOCK: (("dit_mlp_up_4096x12288x3072", ACT_GELU, True),
+                  ("dit_mlp_down_4096x3072x12288", ACT_NONE, False))}
 MAIN_WORKLOAD = BLOCK
 METRIC = "W8A8 quant+scaled-GEMM TOPS and % of int8 roofline on one B200"
 # where the raw nvidia-smi clock samples go (--clocks-dir); the JSON line
@@ -63,7 +67,7 @@ def chain_of(name):
     """The layers of a workload name: a chain, or one plain layer."""
     if name in CHAINS:
         return CHAINS[name]
-    return ((name, ACT_NONE),)
+    return ((name, ACT_NONE, False),)
 
 
 # ----------------------------------------------------------------------------- peaks
@@ -190,7 +194,7 @@ def algorithmic(M, N, K, bias):
 def chain_shapes(names, M=None):
     """(M, N, K, bias) of each layer of a chain."""
     out = []
-    for name, _ in names:
+    for name, *_ in names:
         wl = WORKLOADS[name]
         out.append((wl.M if M is None else M, wl.N, wl.K, wl.bias))
     return out
@@ -289,8 +293,9 @@ def per_graph_for(t_step_estimate):
 class Layer:
     """One W8A8 layer of one input set on the device."""
 
-    def __init__(self, w8, wl, act, inp, device, clone_of=None):
-        self.wl, self.act = wl, act
+    def __init__(self, w8, wl, act, inp, device, clone_of=None, fuse_next=False):
+        self.wl, self.act, self.fuse_next = wl, act, fuse_next
+        self.from_codes = False  # set by the chain: the previous layer forms its codes
         self.M, self.N, self.K = inp.x.shape[0], wl.N, wl.K
         if clone_of is None:
             self.packed = w8.pack_weight(torch.from_numpy(inp.w).to(device))
@@ -308,6 +313,8 @@ class Layer:
         self.mmws = torch.empty((mm,), dtype=torch.uint8, device=device) if mm else None
         self.q = torch.empty((M, K), dtype=torch.int8, device=device)
         self.a = torch.empty((M,), dtype=torch.float32, device=device)
+        self.aqws = (torch.empty((w8.linear_act_quant_workspace_bytes(M, N, K),),
+                                 dtype=torch.uint8, device=device) if fuse_next else None)
 
 
 class ChainSets:
@@ -317,15 +324,17 @@ class ChainSets:
 
     def __init__(self, w8, names, nsets, device, M=None):
         self.names = names
-        inps = [make_inputs(WORKLOADS[n], M) for n, _ in names]
+        inps = [make_inputs(WORKLOADS[n], M) for n, *_ in names]
         self.M = inps[0].x.shape[0]
         x0 = bf16_dev(inps[0].x, device)
         self.sets = []
         for i in range(nsets):
             first = self.sets[0] if self.sets else None
             layers = [Layer(w8, WORKLOADS[n], act, inp, device,
-                            None if first is None else first["layers"][j])
-                      for j, ((n, act), inp) in enumerate(zip(names, inps))]
+                            None if first is None else first["layers"][j], fuse)
+                      for j, ((n, act, fuse), inp) in enumerate(zip(names, inps))]
+            for prev, L in zip(layers, layers[1:]):
+                L.from_codes = prev.fuse_next
             self.sets.append({"x": x0 if i == 0 else x0.clone(), "layers": layers})
         del inps
         torch.cuda.synchronize()
@@ -338,7 +347,7 @@ class ChainSets:
         s = self.sets[0]
         n = s["x"].numel() * 2
         for L in s["layers"]:
-            for t in (L.packed, L.w_scale, L.bias, L.y, L.ws, L.mmws, L.q, L.a):
+            for t in (L.packed, L.w_scale, L.bias, L.y, L.ws, L.mmws, L.q, L.a, L.aqws):
                 if t is not None:
                     n += t.numel() * t.element_size()
         return n
@@ -346,9 +355,19 @@ class ChainSets:
 
 def run_chain(w8, cs, s, stream):
     x = s["x"]
-    for L in s["layers"]:
-        w8.linear(x, L.packed, L.w_scale, L.bias, L.N, out=L.y, workspace=L.ws, stream=stream,
-                  act=L.act)
+    layers = s["layers"]
+    for i, L in enumerate(layers):
+        if L.from_codes:
+            # codes and scales formed by the previous layer
+            w8.scaled_mm(L.q, L.a, L.packed, L.w_scale, L.bias, L.N, out=L.y,
+                         workspace=L.mmws, stream=stream, act=L.act)
+        elif L.fuse_next:
+            nxt = layers[i + 1]
+            w8.linear_act_quant(x, L.packed, L.w_scale, L.bias, L.N, out=L.y, q_next=nxt.q,
+                                a_scale_next=nxt.a, workspace=L.aqws, stream=stream, act=L.act)
+        else:
+            w8.linear(x, L.packed, L.w_scale, L.bias, L.N, out=L.y, workspace=L.ws, stream=stream,
+                      act=L.act)
         x = L.y
 
 
@@ -459,12 +478,13 @@ def run_ours(args, rank, world, device):
     ms_per_step = t_max / args.steps * 1e3
     per_graph = step_loop.per_graph
 
-    # ---- dominant kernel: the GEMM of every layer, each timed alone; the
-    # algorithmic ops of one launch over the mean launch duration
+    # ---- dominant kernel: the GEMM of every layer, each timed alone (without
+    # the fused quantisation); the algorithmic ops of one launch over the mean
+    # launch duration
     t_g = [base[f"t_gemm{i}"] for i in range(len(names))]
     gemm_tops = ops / sum(t_g) / 1e12
     kernels = [w8.gemm_kernel_name(M, N, K) for M, N, K, _ in shapes]
-    traffic = [recorded_traffic(n) for n, _ in names]
+    traffic = [recorded_traffic(n) for n, *_ in names]
     roofline = {
         "bound": "tensor", "achieved": round(gemm_tops, 1), "peak": round(int8_peak, 1),
         "unit": "TOPS", "frac": round(gemm_tops / int8_peak, 4),
@@ -504,9 +524,9 @@ def run_ours(args, rank, world, device):
         "scaling": "weak", "vs_baseline": None, "dtype": "int8 x int8 -> int32, bf16 in/out",
         "data": "synthetic, seeded (workloads.py recipe)",
         "config": {"workload": args.workload, "M": first.M if len(names) > 1 else shapes[0][0],
-                   "layers": [f"{M}x{N}x{K}" + ("+gelu" if a else "")
-                              for (M, N, K, _), (_, a) in zip(shapes, names)],
-                   "step": f"{len(names)} x w8a8_linear (quant kernel + tcgen05 GEMM/epilogue, PDL)",
+                   "layers": [f"{M}x{N}x{K}" + ("+gelu" if a else "") + ("+quant_next" if f else "")
+                              for (M, N, K, _), (_, a, f) in zip(shapes, names)],
+                   "step": step_description(names),
                    "l2": f"{base['nsets']} rotated input sets of "
                          f"{base['set_bytes'] / 2**20:.0f} MiB (> 126 MB L2)",
                    "launch": f"CUDA graphs of {per_graph} steps",
@@ -523,8 +543,15 @@ def run_ours(args, rank, world, device):
         out["sweep_cols"] = SWEEP_COLS
         out["sweep"] = sweep(w8, args, device, stream, peaks, int8_peak)
         if args.workload == BLOCK:
-            out["block_unfused_us"] = block_unfused(w8, device, stream)
+            out["block_variants_us"] = block_variants(w8, device, stream)
     return out
+
+
+def step_description(names):
+    if len(names) == 1:
+        return "w8a8_linear: quant kernel + tcgen05 GEMM/epilogue (PDL)"
+    return ("w8a8_linear_act_quant (quant, GEMM+GELU, codes of its output beside it) + "
+            "w8a8_scaled_mm on those codes" if names[0][2] else f"{len(names)} x w8a8_linear")
 
 
 def max_over_ranks(elapsed, world, device):
@@ -607,7 +634,10 @@ def run_e2e(w8, cs, args, stream, ops):
     yb = int(np.prod(y_shape)) * 2
     return {"value": round(ops / t / 1e12, 2), "unit": "TOPS", "h2d_bytes_per_step": xb,
             "d2h_bytes_per_step": yb, "steps": steps, "ms_per_step": round(t * 1e3, 4),
-            "overlap": "H2D i+1 | layers i | D2H i-1, 3 streams", "api": "w8a8_linear_act"}
+            "overlap": "H2D i+1 | layers i | D2H i-1, 3 streams",
+            "api": "+".join(sorted({"w8a8_linear_act_quant" if L.fuse_next else
+                                    "w8a8_scaled_mm" if L.from_codes else "w8a8_linear_act"
+                                    for L in s0["layers"]}))}
 
 
 # compact sweep rows: one list per workload, columns named once
@@ -639,7 +669,7 @@ def sweep(w8, args, device, stream, peaks, int8_peak):
         ops, gemm_bytes, quant_bytes, fused_bytes = algorithmic(wl.M, wl.N, wl.K, wl.bias)
         steps = 200 if ops > 1e11 else 2000
         warm = wl.N * wl.K + wl.M * wl.K + 2 * wl.M * wl.N < L2_BYTES // 2
-        cs, loop, r = measure_chain(w8, ((name, ACT_NONE),), steps, 3, device, stream,
+        cs, loop, r = measure_chain(w8, chain_of(name), steps, 3, device, stream,
                                     warm_gemm=warm)
         t_roof_gemm = max(ops / (int8_peak * 1e12), gemm_bytes / (peaks["hbm_gbs"] * 1e9))
         t_roof_step = max(ops / (int8_peak * 1e12), fused_bytes / (peaks["hbm_gbs"] * 1e9))
@@ -656,13 +686,22 @@ def sweep(w8, args, device, stream, peaks, int8_peak):
     return out
 
 
-def block_unfused(w8, device, stream, nsets=2, steps=64):
-    """The DiT MLP block with the GELU as a kernel of its own between the
-    layers (layer, GELU kernel, layer), for comparison with the headline
-    step, where the GELU runs in the up-projection's epilogue."""
+def block_variants(w8, device, stream, nsets=4, steps=64):
+    """The DiT MLP block without the fusions of the headline step, same
+    inputs and loop: "layers" -- two w8a8_linear calls, the GELU in the
+    up-projection's epilogue but the down-projection quantising its input in
+    a pass of its own; "unfused" -- layer, GELU kernel, layer.  Microseconds
+    a step."""
     names = CHAINS[BLOCK]
     cs = ChainSets(w8, names, nsets, device)
     gs = [torch.empty_like(s["layers"][0].y) for s in cs.sets]
+
+    def layers(s, g):
+        Lu, Ld = s["layers"]
+        w8.linear(s["x"], Lu.packed, Lu.w_scale, Lu.bias, Lu.N, out=Lu.y, workspace=Lu.ws,
+                  stream=stream, act=Lu.act)
+        w8.linear(Lu.y, Ld.packed, Ld.w_scale, Ld.bias, Ld.N, out=Ld.y, workspace=Ld.ws,
+                  stream=stream)
 
     def unfused(s, g):
         Lu, Ld = s["layers"]
@@ -671,20 +710,24 @@ def block_unfused(w8, device, stream, nsets=2, steps=64):
         w8.gelu_tanh(Lu.y, out=g, stream=stream)
         w8.linear(g, Ld.packed, Ld.w_scale, Ld.bias, Ld.N, out=Ld.y, workspace=Ld.ws,
                   stream=stream)
-    lp = GraphLoop([lambda s=s, g=g: unfused(s, g) for s, g in zip(cs.sets, gs)], stream, 4)
-    lp.prepare(steps)
-    time_loop(lp, 3 * lp.per_graph, stream)
-    t = time_loop(lp, steps, stream) / steps
+    out = {}
+    for name, fn in (("layers", layers), ("unfused", unfused)):
+        lp = GraphLoop([lambda s=s, g=g, f=fn: f(s, g) for s, g in zip(cs.sets, gs)], stream, 4)
+        lp.prepare(steps)
+        time_loop(lp, 3 * lp.per_graph, stream)
+        out[name] = round(time_loop(lp, steps, stream) / steps * 1e6, 2)
+        del lp
     assert w8.poll_status() == 0
-    del cs, gs, lp
+    del cs, gs
     torch.cuda.empty_cache()
-    return round(t * 1e6, 2)
+    return out
 
 
 # ----------------------------------------------------------------------------- CPU oracle
 def oracle_chain(oracle, names, x, inps):
-    """The chain through the oracle: each layer, then GELU where it has one."""
-    for (name, act), inp in zip(names, inps):
+    """The chain through the oracle: each layer, then GELU where it has one
+    (the codes a layer forms for the next are the next layer's own)."""
+    for (name, act, _), inp in zip(names, inps):
         x = oracle.linear(x, inp.w, inp.w_scale, inp.bias)[0]
         if act == ACT_GELU:
             x = oracle.gelu_tanh(x)
@@ -697,7 +740,7 @@ def cpu_baseline(names, budget_s=12.0):
     seconds have elapsed; plus single-thread figures for the three smaller
     workloads (a row sample of each)."""
     import oracle
-    inps = [make_inputs(WORKLOADS[n]) for n, _ in names]
+    inps = [make_inputs(WORKLOADS[n]) for n, *_ in names]
     ops = sum(algorithmic(*sh)[0] for sh in chain_shapes(names))
     oracle_chain(oracle, names, inps[0].x[:4], inps)  # load and touch
     t0 = time.perf_counter()
@@ -735,7 +778,7 @@ def run_reference(args):
     sample of the same workload (its first rows through every layer)."""
     import oracle
     names = chain_of(args.workload)
-    inps = [make_inputs(WORKLOADS[n]) for n, _ in names]
+    inps = [make_inputs(WORKLOADS[n]) for n, *_ in names]
     shapes = chain_shapes(names)
     M = shapes[0][0]
     rows = max(1, min(M, int(args.ref_rows)))

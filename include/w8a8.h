@@ -225,6 +225,39 @@ w8a8_status w8a8_linear_act(const void *x, int64_t ldx, const void *packed_w,
                             void *workspace, size_t ws_bytes,
                             w8a8_stream_t stream);
 
+/* ---- a layer whose output feeds the next W8A8 layer ---------------------------
+ * Source: "Issue 5 probe ...", Kernel isolation (the DiT MLP pair: the
+ * up-projection img_mlp.proj feeds img_mlp.out) and Round two (step 1, the
+ * dynamic per-token quantisation, applied to the next layer's input).  The
+ * next layer's quantisation of this layer's output, fused with this layer:
+ * the results equal, bit for bit, w8a8_linear_act(..., y, ...) followed by
+ * w8a8_quant_act(y, M, N, N, q_next, a_scale_next).  The next layer then runs
+ * w8a8_scaled_mm(q_next, a_scale_next, ...) on them.
+ * How: the GEMM epilogue folds every row's largest output magnitude while it
+ * stores y, and reports each 128-row block once its stores are complete; a
+ * codes kernel running beside the GEMM quantises each block as it completes,
+ * reading the rows back from L2, so that no separate pass over y follows the
+ * layer.  Three launches on `stream` (for M <= 16: the layer, then the
+ * quantisation kernel on y).
+ *   x, ldx, packed_w, w_scale, bias, y, M, N, K, act: as w8a8_linear_act
+ *   q_next       device, int8 [M, N] dense (output): the codes of y
+ *   a_scale_next device, fp32 [M] (output): their per-row scales
+ *   workspace    device, ws_bytes >= w8a8_linear_act_quant_workspace_bytes(M,
+ *                N, K): w8a8_linear's workspace, then the row maxima and one
+ *                call-tagged completion word per 128-row block (contents on
+ *                entry do not matter; the last CTA of each call clears the
+ *                words, so a replayed CUDA graph finds them at zero)
+ * Limits as w8a8_linear, plus N <= 2^28.  After a call that timed out
+ * (W8A8_ERR_TIMEOUT) the words may be left set: capture CUDA graphs of this
+ * call again (a new capture draws a new tag) before replaying them. */
+w8a8_status w8a8_linear_act_quant_workspace_bytes(int64_t M, int64_t N, int64_t K,
+                                                  size_t *bytes);
+w8a8_status w8a8_linear_act_quant(const void *x, int64_t ldx, const void *packed_w,
+                                  const float *w_scale, const void *bias, void *y,
+                                  int64_t M, int64_t N, int64_t K, int act,
+                                  int8_t *q_next, float *a_scale_next, void *workspace,
+                                  size_t ws_bytes, w8a8_stream_t stream);
+
 /* ---- the whole layer without a caller-provided workspace ---------------------
  * No counterpart on the pages: an addition for callers that cannot allocate
  * device memory when they run a layer (a plugin whose host framework owns all

@@ -117,3 +117,34 @@ def test_workspace_sizes(L):
             assert binding.linear_workspace_bytes(512, 4096, 4096) == 512 * 4096 + 2048
         finally:
             assert L.w8a8_set_path(0) == 0
+
+
+def test_act_quant_rejects_bad_arguments_and_sizes_its_workspace(L):
+    """w8a8_linear_act_quant: host-side checks before any launch, and the
+    workspace: w8a8_linear's, then the row maxima (4 bytes a row), one 8-byte
+    completion word per 128-row block and one exit word, each rounded up to
+    256 bytes."""
+    from w8a8_int8_dynamic_b200 import binding
+    f = L.w8a8_linear_act_quant
+    big = 1 << 30
+    ok = (FAKE, 16, FAKE, FAKE, None, FAKE, 4, 8, 16, 0, FAKE, FAKE, FAKE, big, None)
+    # every argument valid but the one under test (nothing may launch)
+    def call(**kw):
+        a = list(ok)
+        for i, v in kw.items():
+            a[int(i[1:])] = v
+        return f(*a)
+    assert call(a10=None) == 1                 # no q_next
+    assert call(a11=None) == 1                 # no a_scale_next
+    assert call(a12=None) == 1                 # no workspace
+    assert call(a9=7) == 1                     # unknown activation
+    assert call(a10=FAKE_MIS) == 2             # q_next misaligned
+    assert call(a11=FAKE_MIS) == 2             # a_scale_next misaligned
+    assert call(a13=1) == 6                    # workspace too small
+    assert call(a7=(1 << 28) + 8) == 3         # N beyond the fused limit
+    assert call(a8=40) == 3                    # K % 16
+    for M, N, K in [(4096, 12288, 3072), (1000, 2056, 1040), (16, 4096, 4096)]:
+        lin = binding.linear_workspace_bytes(M, N, K)
+        rnd = lambda v: (v + 255) // 256 * 256  # noqa: E731
+        extra = rnd(4 * M) + rnd(8 * ((M + 127) // 128)) + 256
+        assert binding.linear_act_quant_workspace_bytes(M, N, K) == lin + extra

@@ -133,3 +133,28 @@ def test_rel_l2_reproduces_page_figure(name):
     ref = qh @ wdq.T + bias
     err = np.linalg.norm(yf - ref) / np.linalg.norm(ref)
     assert 0.0010 <= err <= 0.0025, err
+
+
+def test_dit_mlp_block_fused_quant_full():
+    """The benchmark's step at full size: the up-projection with GELU in its
+    epilogue and the down-projection's quantisation fused in
+    (w8a8_linear_act_quant), then the down-projection as a scaled GEMM on
+    those codes.  The same bits as the two layers run one after the other,
+    with the codes and scales equal to the oracle's quantisation of the GPU's
+    GELU output, in full."""
+    up = make_inputs(WORKLOADS["dit_mlp_up_4096x12288x3072"])
+    down = make_inputs(WORKLOADS["dit_mlp_down_4096x3072x12288"])
+    l_up = w8.W8A8Linear(dev(up.w), dev(up.w_scale), dev_bf16(up.bias), act=w8.ACT_GELU_TANH)
+    l_down = w8.W8A8Linear(dev(down.w), dev(down.w_scale), dev_bf16(down.bias))
+    x = dev_bf16(up.x)
+    g, q, s = w8.linear_act_quant(x, l_up.packed, l_up.w_scale, l_up.bias, 12288,
+                                  act=w8.ACT_GELU_TANH)
+    y = w8.scaled_mm(q, s, l_down.packed, l_down.w_scale, l_down.bias, 3072)
+    g_ref = l_up(x)
+    y_ref = l_down(g_ref)
+    torch.cuda.synchronize()
+    assert torch.equal(g, g_ref)
+    assert torch.equal(y, y_ref)
+    q_o, s_o = oracle.quant_act(host_u16(g))
+    assert np.array_equal(q.cpu().numpy(), q_o)
+    assert np.array_equal(s.cpu().numpy().view(np.uint32), s_o.view(np.uint32))

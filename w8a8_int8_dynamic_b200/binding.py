@@ -64,6 +64,10 @@ _SIGNATURES = {
     "w8a8_linear": ([_P, _I64, _P, _P, _P, _P, _I64, _I64, _I64, _P, _SZ, _P], ctypes.c_int),
     "w8a8_linear_act": ([_P, _I64, _P, _P, _P, _P, _I64, _I64, _I64, ctypes.c_int, _P, _SZ, _P],
                         ctypes.c_int),
+    "w8a8_linear_act_quant_workspace_bytes": ([_I64, _I64, _I64, ctypes.POINTER(_SZ)],
+                                              ctypes.c_int),
+    "w8a8_linear_act_quant": ([_P, _I64, _P, _P, _P, _P, _I64, _I64, _I64, ctypes.c_int, _P, _P, _P,
+                               _SZ, _P], ctypes.c_int),
     "w8a8_linear_noalloc_max_bytes": ([], _SZ),
     "w8a8_linear_noalloc": ([_P, _I64, _P, _P, _P, _P, _I64, _I64, _I64, _P], ctypes.c_int),
     "w8a8_set_path": ([ctypes.c_int], ctypes.c_int),
@@ -124,6 +128,13 @@ def linear_workspace_bytes(M: int, N: int, K: int) -> int:
     out = _SZ()
     _check(lib().w8a8_linear_workspace_bytes(M, N, K, ctypes.byref(out)),
            "w8a8_linear_workspace_bytes")
+    return out.value
+
+
+def linear_act_quant_workspace_bytes(M: int, N: int, K: int) -> int:
+    out = _SZ()
+    _check(lib().w8a8_linear_act_quant_workspace_bytes(M, N, K, ctypes.byref(out)),
+           "w8a8_linear_act_quant_workspace_bytes")
     return out.value
 
 
@@ -276,6 +287,39 @@ def linear(x: torch.Tensor, packed_w: torch.Tensor, w_scale: torch.Tensor,
                                  _stream(stream)),
            "w8a8_linear_act")
     return out.view(*lead, N)
+
+
+def linear_act_quant(x: torch.Tensor, packed_w: torch.Tensor, w_scale: torch.Tensor,
+                     bias: Optional[torch.Tensor], N: int, out: Optional[torch.Tensor] = None,
+                     q_next: Optional[torch.Tensor] = None,
+                     a_scale_next: Optional[torch.Tensor] = None,
+                     workspace: Optional[torch.Tensor] = None, stream=None,
+                     act: int = ACT_NONE) -> Tuple[torch.Tensor, torch.Tensor, torch.Tensor]:
+    """A layer whose output feeds another W8A8 layer: y = act(W8A8(x)) and
+    the next layer's codes and scales of y, (y, q_next, a_scale_next), equal
+    to ``linear`` followed by ``quant_act`` of its output."""
+    _need_cuda(x, "x", torch.bfloat16)
+    K = x.shape[-1]
+    x2 = x.reshape(-1, K)
+    if x2.stride(1) != 1:
+        x2 = x2.contiguous()
+    M = x2.shape[0]
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.bfloat16, device=x.device)
+    if q_next is None:
+        q_next = torch.empty((M, N), dtype=torch.int8, device=x.device)
+    if a_scale_next is None:
+        a_scale_next = torch.empty((M,), dtype=torch.float32, device=x.device)
+    if workspace is None:
+        workspace = torch.empty((linear_act_quant_workspace_bytes(M, N, K),), dtype=torch.uint8,
+                                device=x.device)
+    ws_bytes = workspace.numel() * workspace.element_size()
+    _check(lib().w8a8_linear_act_quant(_ptr(x2), x2.stride(0), _ptr(packed_w), _ptr(w_scale),
+                                       _ptr(bias), _ptr(out), M, N, K, act, _ptr(q_next),
+                                       _ptr(a_scale_next), _ptr(workspace), ws_bytes,
+                                       _stream(stream)),
+           "w8a8_linear_act_quant")
+    return out, q_next, a_scale_next
 
 
 def linear_noalloc(x: torch.Tensor, packed_w: torch.Tensor, w_scale: torch.Tensor,

@@ -75,8 +75,9 @@ struct LargeSmem {
 // At most kGemmRegs registers a thread, so that a CTA (11 warps) fits on an
 // SM beside the blocks of the quantisation kernel it is launched behind and
 // starts its prologue and first weight copies while they run.
-template <int BN, int STAGES, int KPS, bool OUT_I32>
-__global__ void __maxnreg__(kGemmRegs)
+// ROWMAX: the next layer's quantisation is fused in (GemmArgs::row_amax).
+template <int BN, int STAGES, int KPS, bool OUT_I32, bool ROWMAX>
+__global__ void __maxnreg__(ROWMAX ? kGemmRegsRowmax : kGemmRegs)
     gemm_kernel(const __grid_constant__ CUtensorMap tmap_q,
                 const __grid_constant__ CUtensorMap tmap_y, const GemmArgs args) {
   using L = LargeSmem<BN, STAGES, KPS>;
@@ -96,6 +97,9 @@ __global__ void __maxnreg__(kGemmRegs)
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + L::kMisc);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + L::kMisc + 4);
 
+  // With the next layer's quantisation fused in, the codes kernel behind
+  // this one becomes resident beside it and follows its row blocks.
+  if (ROWMAX) griddep_launch_dependents();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -313,13 +317,17 @@ __global__ void __maxnreg__(kGemmRegs)
       tc_fence_after();
       const uint32_t taddr =
           tmem_base + b * BN + ew.half * kCols + ((uint32_t)(ew.quarter * 32) << 16);
+      uint32_t rmax = 0;
       if (OUT_I32)
         epilogue_i32<kCols>(args, taddr, row0 + lane, n0);
       else
-        epilogue_tma<kCols>(args, &tmap_y, taddr, lane, row0, n0, as, s_ws, s_bias, s_out);
+        epilogue_tma<kCols, ROWMAX>(args, &tmap_y, taddr, lane, row0, n0, as, s_ws, s_bias, s_out,
+                                    rmax);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&tempty[b]);
+      if (ROWMAX && n0 < args.N && (row0 >> 7) * 128 < args.M)
+        publish_rows(args, lane, row0, row_max_bits(rmax), min(kCols, args.N - n0));
     }
     if (lane == 0) bulk_wait_group_all();  // output stores complete before exit
     __syncwarp();
@@ -376,12 +384,12 @@ cudaError_t launch_ex(Kernel k, int grid, int smem, cudaStream_t stream, bool pd
   return cudaLaunchKernelEx(&cfg, k, args...);
 }
 
-template <int BN, int STAGES, bool OUT_I32>
+template <int BN, int STAGES, bool OUT_I32, bool ROWMAX = false>
 w8a8_status run_large(const CUtensorMap &tmap, const CUtensorMap &tmap_y, GemmArgs args,
                       cudaStream_t stream, bool pdl, int slot) {
   constexpr int KPS = BN == 128 ? kKps128 : 1;
   using L = LargeSmem<BN, STAGES, KPS>;
-  auto k = gemm_kernel<BN, STAGES, KPS, OUT_I32>;
+  auto k = gemm_kernel<BN, STAGES, KPS, OUT_I32, ROWMAX>;
   cudaError_t e = set_smem_attr(k, L::kAlloc, slot);
   if (e != cudaSuccess) return W8A8_ERR_CUDA;
   args.tiles_n = (int)((args.N + BN - 1) / BN);
@@ -453,7 +461,7 @@ LargeKind choose_large(int64_t M, int64_t N) {
 w8a8_status launch_scaled_mm(const int8_t *q, const float *a_scale, const void *packed_w,
                              const float *w_scale, const void *bias, void *out, bool out_i32,
                              int64_t M, int64_t N, int64_t K, cudaStream_t stream, bool pdl,
-                             int act) {
+                             int act, bool prefetch, const RowSignal *sig) {
   CUtensorMap tmap;
   if (!make_tmap_u8_2d(&tmap, q, (uint64_t)M, (uint64_t)K, (uint64_t)K, kBM, kBK))
     return W8A8_ERR_CUDA;
@@ -469,9 +477,14 @@ w8a8_status launch_scaled_mm(const int8_t *q, const float *a_scale, const void *
   a.tiles_m = (int)((M + kBM - 1) / kBM);
   a.tiles_n = 0;
   a.act = out_i32 ? W8A8_ACT_NONE : act;
-  a.prefetch_kb = pdl ? kPrefetchKb : 0;
+  a.prefetch_kb = (pdl && prefetch) ? kPrefetchKb : 0;
   a.status = status_word();
   if (!a.status) return W8A8_ERR_CUDA;
+  if (sig && !out_i32) {
+    a.row_amax = sig->row_amax;
+    a.row_done = sig->row_done;
+    a.done_tag = sig->tag;
+  }
   CUtensorMap tmap_y;
   if (out_i32) {
     // the int32 export always uses the 1-SM kernel (tests and inspection); it
@@ -486,16 +499,26 @@ w8a8_status launch_scaled_mm(const int8_t *q, const float *a_scale, const void *
   switch (choose_large(M, N)) {
     case LargeKind::kPair:
       return launch_gemm2sm(q, a_scale, packed_w, w_scale, bias, out, M, N, K, stream, pdl, 256,
-                            act);
+                            act, sig);
     case LargeKind::kPair128:
       return launch_gemm2sm(q, a_scale, packed_w, w_scale, bias, out, M, N, K, stream, pdl, 128,
-                            act);
+                            act, sig);
     case LargeKind::k256:
-      return run_large<256, kLargeStages256, false>(tmap, tmap_y, a, stream, pdl, 2);
+      return sig ? run_large<256, kLargeStages256, false, true>(tmap, tmap_y, a, stream, pdl, 4)
+                 : run_large<256, kLargeStages256, false>(tmap, tmap_y, a, stream, pdl, 2);
     default:
-      return run_large<128, kLargeStages128, false>(tmap, tmap_y, a, stream, pdl, 3);
+      return sig ? run_large<128, kLargeStages128, false, true>(tmap, tmap_y, a, stream, pdl, 5)
+                 : run_large<128, kLargeStages128, false>(tmap, tmap_y, a, stream, pdl, 3);
   }
 }
+
+// Largest N of the fused next-layer quantisation (a row block's completion
+// count, 4 N, stays in 32 bits).
+constexpr int64_t kMaxFusedN = (int64_t)1 << 28;
+
+// Workspace of w8a8_linear_act_quant: as w8a8_linear's, then (large M) the
+// row maxima, one completion word per 128-row block and one exit word.
+int64_t act_quant_workspace_bytes(int64_t M, int64_t N, int64_t K);
 
 // Workspace of w8a8_linear: the codes, the scales and (small M) the split-K
 // partials of the weight-streaming kernel.
@@ -503,6 +526,11 @@ int64_t linear_workspace_bytes(int64_t M, int64_t N, int64_t K) {
   int64_t b = round_up(M * K, 256) + round_up(M * 4, 256);
   if (M <= kDecodeNT) b += decode_workspace_bytes(N, K);
   return b;
+}
+
+int64_t act_quant_workspace_bytes(int64_t M, int64_t N, int64_t K) {
+  return linear_workspace_bytes(M, N, K) + round_up(M * 4, 256) +
+         round_up(((M + 127) / 128) * 8, 256) + 256;
 }
 
 static w8a8_status check_gemm_args(const void *q, const void *packed_w, const void *out,
@@ -547,7 +575,10 @@ w8a8_status w8a8_scaled_mm_act(const int8_t *q, const float *a_scale, const void
   }
   if (forced_path() == 2) return W8A8_ERR_INVALID_ARG;  // small path needs M <= 16 and a workspace
   if (workspace && !aligned16(workspace)) return W8A8_ERR_ALIGNMENT;
-  return launch_scaled_mm(q, a_scale, packed_w, w_scale, bias, y, false, M, N, K, s, false, act);
+  // A programmatic dependent of the preceding kernel: behind the codes kernel
+  // of a fused next-layer quantisation its CTAs take SMs as the previous
+  // GEMM leaves them and issue their first weight copies while it finishes.
+  return launch_scaled_mm(q, a_scale, packed_w, w_scale, bias, y, false, M, N, K, s, true, act);
 }
 
 w8a8_status w8a8_scaled_mm(const int8_t *q, const float *a_scale, const void *packed_w,
@@ -596,6 +627,7 @@ w8a8_status w8a8_linear_act(const void *x, int64_t ldx, const void *packed_w,
       (bias && !aligned16(bias)))
     return W8A8_ERR_ALIGNMENT;
   if ((int64_t)ws_bytes < linear_workspace_bytes(M, N, K)) return W8A8_ERR_BUFFER_TOO_SMALL;
+  if (!use_decode_path(M) && forced_path() == 2) return W8A8_ERR_INVALID_ARG;
   uint8_t *ws = static_cast<uint8_t *>(workspace);
   int8_t *q = reinterpret_cast<int8_t *>(ws);
   float *a_scale = reinterpret_cast<float *>(ws + round_up(M * K, 256));
@@ -606,8 +638,8 @@ w8a8_status w8a8_linear_act(const void *x, int64_t ldx, const void *packed_w,
     void *dws = ws + round_up(M * K, 256) + round_up(M * 4, 256);
     return launch_decode(q, a_scale, packed_w, w_scale, bias, y, M, N, K, dws, s, true, act);
   }
-  if (forced_path() == 2) return W8A8_ERR_INVALID_ARG;
-  return launch_scaled_mm(q, a_scale, packed_w, w_scale, bias, y, false, M, N, K, s, true, act);
+  return launch_scaled_mm(q, a_scale, packed_w, w_scale, bias, y, false, M, N, K, s, true, act,
+                          true);
 }
 
 w8a8_status w8a8_linear(const void *x, int64_t ldx, const void *packed_w, const float *w_scale,
@@ -615,6 +647,58 @@ w8a8_status w8a8_linear(const void *x, int64_t ldx, const void *packed_w, const 
                         void *workspace, size_t ws_bytes, w8a8_stream_t stream) {
   return w8a8_linear_act(x, ldx, packed_w, w_scale, bias, y, M, N, K, W8A8_ACT_NONE, workspace,
                          ws_bytes, stream);
+}
+
+w8a8_status w8a8_linear_act_quant_workspace_bytes(int64_t M, int64_t N, int64_t K,
+                                                  size_t *bytes) {
+  if (!bytes || M < 1 || N < 1 || K < 1) return W8A8_ERR_INVALID_ARG;
+  if (K % 16 != 0 || K > kMaxK || N % 8 != 0) return W8A8_ERR_UNSUPPORTED_SHAPE;
+  *bytes = (size_t)act_quant_workspace_bytes(M, N, K);
+  return W8A8_OK;
+}
+
+w8a8_status w8a8_linear_act_quant(const void *x, int64_t ldx, const void *packed_w,
+                                  const float *w_scale, const void *bias, void *y, int64_t M,
+                                  int64_t N, int64_t K, int act, int8_t *q_next,
+                                  float *a_scale_next, void *workspace, size_t ws_bytes,
+                                  w8a8_stream_t stream) {
+  w8a8_status st = check_gemm_args(x, packed_w, y, M, N, K);
+  if (st != W8A8_OK) return st;
+  if (!w_scale || !workspace || !q_next || !a_scale_next) return W8A8_ERR_INVALID_ARG;
+  if (ldx < K) return W8A8_ERR_INVALID_ARG;
+  if (act != W8A8_ACT_NONE && act != W8A8_ACT_GELU_TANH) return W8A8_ERR_INVALID_ARG;
+  if (N > kMaxFusedN) return W8A8_ERR_UNSUPPORTED_SHAPE;
+  if (ldx % 8 != 0 || !aligned16(w_scale) || !aligned16(workspace) ||
+      (bias && !aligned16(bias)) || !aligned16(q_next) || !aligned16(a_scale_next))
+    return W8A8_ERR_ALIGNMENT;
+  if ((int64_t)ws_bytes < act_quant_workspace_bytes(M, N, K)) return W8A8_ERR_BUFFER_TOO_SMALL;
+  if (!use_decode_path(M) && forced_path() == 2) return W8A8_ERR_INVALID_ARG;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (use_decode_path(M)) {
+    // Few rows: the layer, then the quantisation of its output.
+    st = w8a8_linear_act(x, ldx, packed_w, w_scale, bias, y, M, N, K, act, workspace, ws_bytes,
+                         stream);
+    if (st != W8A8_OK) return st;
+    return launch_quant(y, M, N, N, q_next, a_scale_next, s, false);
+  }
+  uint8_t *ws = static_cast<uint8_t *>(workspace);
+  int8_t *q = reinterpret_cast<int8_t *>(ws);
+  int64_t off = round_up(M * K, 256);
+  float *a_scale = reinterpret_cast<float *>(ws + off);
+  off += round_up(M * 4, 256);
+  uint32_t *row_amax = reinterpret_cast<uint32_t *>(ws + off);
+  off += round_up(M * 4, 256);
+  unsigned long long *row_done = reinterpret_cast<unsigned long long *>(ws + off);
+  off += round_up(((M + 127) / 128) * 8, 256);
+  unsigned long long *exit_word = reinterpret_cast<unsigned long long *>(ws + off);
+  RowSignal sig{row_amax, row_done, next_call_tag() & 0xFFFFFFFFull};
+  if (sig.tag == 0) sig.tag = 1;
+  st = launch_quant(x, M, K, ldx, q, a_scale, s, true, row_amax);
+  if (st != W8A8_OK) return st;
+  st = launch_scaled_mm(q, a_scale, packed_w, w_scale, bias, y, false, M, N, K, s, true, act, true,
+                        &sig);
+  if (st != W8A8_OK) return st;
+  return launch_codes(y, M, N, row_amax, row_done, sig.tag, q_next, a_scale_next, exit_word, s);
 }
 
 }  // extern "C"

@@ -64,8 +64,9 @@ struct PairSmem {
 // At most kGemmRegs registers a thread, so that a CTA (11 warps) fits on an
 // SM beside the blocks of the quantisation kernel it is launched behind and
 // starts its prologue and first weight copies while they run.
-template <int BN, int STAGES>
-__global__ void __maxnreg__(kGemmRegs)
+// ROWMAX: the next layer's quantisation is fused in (GemmArgs::row_amax).
+template <int BN, int STAGES, bool ROWMAX>
+__global__ void __maxnreg__(ROWMAX ? kGemmRegsRowmax : kGemmRegs)
     gemm2sm_kernel(const __grid_constant__ CUtensorMap tmap_q,
                    const __grid_constant__ CUtensorMap tmap_w,
                    const __grid_constant__ CUtensorMap tmap_w64,
@@ -90,6 +91,9 @@ __global__ void __maxnreg__(kGemmRegs)
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + L::kMisc);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + L::kMisc + 4);
 
+  // With the next layer's quantisation fused in, the codes kernel behind
+  // this one becomes resident beside it and follows its row blocks.
+  if (ROWMAX) griddep_launch_dependents();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t crank = cluster_ctarank();
   const uint32_t rank = crank & 1;      // 0: even CTA of the pair (issues the MMAs)
@@ -338,10 +342,15 @@ __global__ void __maxnreg__(kGemmRegs)
       const uint32_t taddr = tmem_base + b * kPairBN + (half >= 0 ? ew.half * 64 : j0) +
                              ((uint32_t)(ew.quarter * 32) << 16);
       // dequantise: acc * a_scale * w_scale + bias
-      epilogue_tma<kCols>(args, &tmap_y, taddr, lane, row0, n0, as, s_ws, s_bias, s_out, ncols);
+      uint32_t rmax = 0;
+      epilogue_tma<kCols, ROWMAX>(args, &tmap_y, taddr, lane, row0, n0, as, s_ws, s_bias, s_out,
+                                  rmax, ncols);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive_cluster(tempty0 + b * 8);
+      // (the odd CTA of the last row tile may hold rows wholly past M)
+      if (ROWMAX && n0 < args.N && (row0 >> 7) * 128 < args.M)
+        publish_rows(args, lane, row0, row_max_bits(rmax), min(ncols, args.N - n0));
     }
     if (lane == 0) bulk_wait_group_all();  // output stores complete before exit
     __syncwarp();
@@ -355,14 +364,14 @@ __global__ void __maxnreg__(kGemmRegs)
   }
 }
 
-bool g_pair_attr_done[64][2];
+bool g_pair_attr_done[64][4];
 
-template <int BN, int STAGES>
+template <int BN, int STAGES, bool ROWMAX = false>
 w8a8_status run_pair(const CUtensorMap &tq, const CUtensorMap &tw, const CUtensorMap &tw64,
                      const CUtensorMap &ty, const GemmArgs &a, cudaStream_t stream, bool pdl,
                      int slot_id) {
   using L = PairSmem<BN, STAGES>;
-  auto k = gemm2sm_kernel<BN, STAGES>;
+  auto k = gemm2sm_kernel<BN, STAGES, ROWMAX>;
   const int d = current_device();
   if (d < 0 || d >= 64 || !g_pair_attr_done[d][slot_id]) {
     if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kAlloc) !=
@@ -409,7 +418,8 @@ int64_t pair_full_tiles(int64_t tiles, int64_t pairs) {
 
 w8a8_status launch_gemm2sm(const int8_t *q, const float *a_scale, const void *packed_w,
                            const float *w_scale, const void *bias, void *y, int64_t M, int64_t N,
-                           int64_t K, cudaStream_t stream, bool pdl, int bn, int act) {
+                           int64_t K, cudaStream_t stream, bool pdl, int bn, int act,
+                           const RowSignal *sig) {
   CUtensorMap tq, tw, tw64, ty;
   if (!make_tmap_u8_2d(&tq, q, (uint64_t)M, (uint64_t)K, (uint64_t)K, kBM, kBK))
     return W8A8_ERR_CUDA;
@@ -433,9 +443,17 @@ w8a8_status launch_gemm2sm(const int8_t *q, const float *a_scale, const void *pa
   a.act = act;
   a.status = status_word();
   if (!a.status) return W8A8_ERR_CUDA;
-  if (bn == 128) return run_pair<128, 4>(tq, tw, tw64, ty, a, stream, pdl, 1);
+  if (sig) {
+    a.row_amax = sig->row_amax;
+    a.row_done = sig->row_done;
+    a.done_tag = sig->tag;
+  }
+  if (bn == 128)
+    return sig ? run_pair<128, 4, true>(tq, tw, tw64, ty, a, stream, pdl, 3)
+               : run_pair<128, 4>(tq, tw, tw64, ty, a, stream, pdl, 1);
   a.full_tiles = (int)pair_full_tiles(a.full_tiles, sm_count() / 2);
-  return run_pair<256, 3>(tq, tw, tw64, ty, a, stream, pdl, 0);
+  return sig ? run_pair<256, 3, true>(tq, tw, tw64, ty, a, stream, pdl, 2)
+             : run_pair<256, 3>(tq, tw, tw64, ty, a, stream, pdl, 0);
 }
 
 }  // namespace w8a8

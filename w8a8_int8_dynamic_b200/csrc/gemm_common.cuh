@@ -31,6 +31,11 @@ constexpr int kGemmThreads = 64 + 32 * kEpiWarps;
 // that hold three of them (most SMs, for 512 rows of 4096), not on those with
 // four.
 constexpr int kGemmRegs = 128;
+// The instances with the next layer's quantisation fused in (ROWMAX) keep
+// one more value a lane through the epilogue and spill below 144 (the pair
+// kernel at 136 too).  At 144 a CTA takes 50,688 registers, and the codes
+// kernel's two 4-warp CTAs of 56 registers (14,336) still fit beside it.
+constexpr int kGemmRegsRowmax = 144;
 
 struct GemmArgs {
   const uint8_t *packed_w;
@@ -49,7 +54,43 @@ struct GemmArgs {
   // as its two 128-column halves (a short last round spread over more pairs)
   int full_tiles;
   int *status;
+  // Next-layer quantisation fused with this layer (the kernels' ROWMAX
+  // instances): the epilogue folds each row's largest bf16 output magnitude
+  // into row_amax (atomicMax on the bf16 magnitude bits; zeroed by the
+  // quantisation kernel ahead of this GEMM), and once a warp's output stores
+  // for a tile are complete it adds the columns it stored to its 128-row
+  // block's word in row_done ((done_tag << 32) | columns; a block is complete
+  // at 4 N).  Those instances also release their dependents at their start,
+  // so that the codes kernel behind them becomes resident and follows the
+  // blocks.
+  uint32_t *row_amax;
+  unsigned long long *row_done;
+  unsigned long long done_tag;
 };
+
+// After a tile: the epilogue warp that drained rows [row0, row0 + 32) and
+// `cols` of their columns (at least 1) publishes them to the codes kernel.
+// Callers skip warps whose 128-row block lies wholly past M (no word exists
+// for it); every warp of an existing block arrives, rows past M included, so
+// that each block's count reaches 4 N.
+// Each lane folds its row's maximum magnitude (bf16 magnitude bits) into
+// row_amax; lane 0 waits
+// until the warp's TMA stores of the tile have completed, orders them (async
+// proxy) and the lanes' maxima before its arrival on the row block's word.
+__device__ __forceinline__ void publish_rows(const GemmArgs &a, int lane, int row0,
+                                             uint32_t max_bits, int cols) {
+  const int row = row0 + lane;
+  if (row < a.M) atomicMax(a.row_amax + row, max_bits);
+  __threadfence();
+  __syncwarp();
+  if (lane == 0) {
+    bulk_wait_group_all();
+    fence_proxy_async_global();
+    __threadfence();
+    arrive_tagged32(a.row_done + (row0 >> 7), a.done_tag, (uint32_t)cols);
+  }
+  __syncwarp();
+}
 
 // Epilogue warp ew (0..7): TMEM lane quarter and which half of the columns.
 struct EpiWarp {
@@ -173,6 +214,12 @@ __device__ __forceinline__ void epilogue_i32(const GemmArgs &a, uint32_t taddr, 
 constexpr int kEpiStageBytes = 32 * 32 * 2;
 constexpr int kEpiStagePerWarp = kEpiStageBytes;
 
+// The two packed 16-bit magnitudes of epilogue_tma's rmax -> one bf16
+// magnitude bit pattern (finite bf16 order by magnitude = order of these bits).
+__device__ __forceinline__ uint32_t row_max_bits(uint32_t rmax) {
+  return max(rmax & 0xFFFFu, rmax >> 16);
+}
+
 __device__ __forceinline__ uint32_t swz64_offset(int r, int c16) {
   return (uint32_t)(r * 64 + ((c16 ^ ((r >> 1) & 3)) << 4));
 }
@@ -183,12 +230,14 @@ __device__ __forceinline__ uint32_t swz64_offset(int r, int c16) {
 //   taddr   TMEM address of the first column, this warp's lane quarter
 //   row0    output row of lane 0;  n0: output column of the first column
 //   s_ws / s_bias: the COLS columns' scales and bias, staged in smem
+//   rmax    (ROWMAX) the running maximum of this lane's row's bf16 output
+//           magnitudes, as two packed 16-bit lanes (see row_max_bits)
 //   ncols   columns actually drained (a multiple of 32, at most COLS)
-template <int COLS>
+template <int COLS, bool ROWMAX>
 __device__ __forceinline__ void epilogue_tma(const GemmArgs &a, const CUtensorMap *tmap_y,
                                              uint32_t taddr, int lane, int row0, int n0, float as,
                                              const float *s_ws, const uint16_t *s_bias,
-                                             uint8_t *stage, int ncols = COLS) {
+                                             uint8_t *stage, uint32_t &rmax, int ncols = COLS) {
   for_tmem_chunks<COLS / 32>(
       taddr, [&](int c) { return c * 32 < ncols && n0 + c * 32 < a.N; },
       [&](const uint32_t(&v)[32], int c) {
@@ -196,6 +245,16 @@ __device__ __forceinline__ void epilogue_tma(const GemmArgs &a, const CUtensorMa
 #pragma unroll
         for (int g = 0; g < 4; ++g)
           out[g] = epilogue8(a, v + 8 * g, as, s_ws + c * 32 + 8 * g, s_bias + c * 32 + 8 * g);
+        if (ROWMAX) {
+          // Columns past N hold exact zeros (zero weights, scale and bias).
+#pragma unroll
+          for (int g = 0; g < 4; ++g) {
+            rmax = __vmaxu2(rmax, out[g].x & 0x7FFF7FFFu);
+            rmax = __vmaxu2(rmax, out[g].y & 0x7FFF7FFFu);
+            rmax = __vmaxu2(rmax, out[g].z & 0x7FFF7FFFu);
+            rmax = __vmaxu2(rmax, out[g].w & 0x7FFF7FFFu);
+          }
+        }
         // the box was last read by this warp's previous store
         if (lane == 0) bulk_wait_group_read<0>();
         __syncwarp();

@@ -76,17 +76,28 @@ inline int64_t packed_rows(int64_t N) { return round_up(N, 256); }
 inline int64_t packed_cols(int64_t K) { return round_up(K, 128); }
 
 // GEMM launchers (gemm.cu).
+// The next layer's quantisation fused with a GEMM (see GemmArgs::row_amax):
+// per-row maxima (zeroed by the quantisation kernel ahead of the GEMM), per
+// 128-row block call-tagged completion words, and the call's tag.
+struct RowSignal {
+  uint32_t *row_amax;
+  unsigned long long *row_done;
+  unsigned long long tag;
+};
+// pdl: a programmatic dependent of the preceding kernel; prefetch: (1-SM
+// kernel) warm L2 with weights while waiting behind the quantisation kernel.
 w8a8_status launch_scaled_mm(const int8_t *q, const float *a_scale, const void *packed_w,
                              const float *w_scale, const void *bias, void *out, bool out_i32,
                              int64_t M, int64_t N, int64_t K, cudaStream_t stream, bool pdl,
-                             int act = W8A8_ACT_NONE);
+                             int act = W8A8_ACT_NONE, bool prefetch = false,
+                             const RowSignal *sig = nullptr);
 // Workspace of w8a8_linear: codes, scales and (small M) the decode partials.
 int64_t linear_workspace_bytes(int64_t M, int64_t N, int64_t K);
 // 2-SM (CTA pair) GEMM with the bf16 epilogue (gemm2sm.cu); bn = 256 or 128.
 w8a8_status launch_gemm2sm(const int8_t *q, const float *a_scale, const void *packed_w,
                            const float *w_scale, const void *bias, void *y, int64_t M, int64_t N,
                            int64_t K, cudaStream_t stream, bool pdl, int bn,
-                           int act = W8A8_ACT_NONE);
+                           int act = W8A8_ACT_NONE, const RowSignal *sig = nullptr);
 int64_t pair_tiles(int64_t M, int64_t N, int bn);
 int64_t pair_full_tiles(int64_t tiles, int64_t pairs);
 // Small-M weight-streaming kernel (decode.cu).
@@ -97,8 +108,17 @@ w8a8_status launch_decode(const int8_t *q, const float *a_scale, const void *pac
                           int64_t N, int64_t K, void *workspace, cudaStream_t stream, bool pdl,
                           int act = W8A8_ACT_NONE);
 // Quantisation launcher (quant.cu).  ahead_of_gemm: the launch is followed by
-// a GEMM launched as its programmatic dependent (the layer).
+// a GEMM launched as its programmatic dependent (the layer).  zero_rows
+// (nullable): a per-row word the kernel sets to 0 (the row maxima of a GEMM
+// with the next layer's quantisation fused in).
 w8a8_status launch_quant(const void *x, int64_t M, int64_t K, int64_t ldx, int8_t *q,
-                         float *a_scale, cudaStream_t stream, bool ahead_of_gemm);
+                         float *a_scale, cudaStream_t stream, bool ahead_of_gemm,
+                         uint32_t *zero_rows = nullptr);
+// The codes kernel of the fused next-layer quantisation (quant.cu): the codes
+// and scales of y [M, N] from the row maxima, each 128-row block once its
+// row_done word reads (tag, 4 N); exit_word counts the CTAs out.
+w8a8_status launch_codes(const void *y, int64_t M, int64_t N, const uint32_t *row_amax,
+                         unsigned long long *row_done, unsigned long long tag, int8_t *q,
+                         float *a_scale, unsigned long long *exit_word, cudaStream_t stream);
 
 }  // namespace w8a8

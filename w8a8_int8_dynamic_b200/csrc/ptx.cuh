@@ -103,27 +103,6 @@ __device__ __forceinline__ void st_release_gpu(unsigned long long *p, unsigned l
   asm volatile("st.release.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
 }
 
-// Waits until *flag == want (acquire).  Gives up like mbar_wait_bounded: on
-// *abort_flag, or after kWaitLimitNs (then sets *abort_flag and records
-// W8A8_ERR_TIMEOUT).  Only ever used to wait for a CTA that has already
-// announced itself running, so the wait is short unless something failed.
-static __device__ __noinline__ bool flag_wait_bounded(const unsigned long long *flag,
-                                                      unsigned long long want,
-                                                      volatile int *abort_flag, int *status) {
-  if (ld_acquire_gpu(flag) == want) return true;
-  const uint64_t t0 = global_timer_ns();
-  while (true) {
-    __nanosleep(64);
-    if (ld_acquire_gpu(flag) == want) return true;
-    if (*abort_flag) return false;
-    if (global_timer_ns() - t0 > kWaitLimitNs) {
-      *abort_flag = 1;
-      atomicExch(status, (int)W8A8_ERR_TIMEOUT);
-      return false;
-    }
-  }
-}
-
 // Counts this CTA's arrival on a call-tagged counter word ((tag << 8) |
 // arrivals, at most 255 arrivals per call) and returns the count after it; a
 // word carrying another call's tag (or cleared to 0) counts as zero arrivals,
@@ -145,8 +124,30 @@ __device__ __forceinline__ uint32_t arrive_tagged(unsigned long long *ctr, unsig
   }
 }
 
-// Orders this thread's generic-proxy accesses to global memory before its
-// later async-proxy (bulk copy) accesses.
+// Counts `n` on a call-tagged word ((tag << 32) | count, 32-bit count) and
+// returns the count after it: a word carrying another call's tag (or
+// cleared to 0) counts as zero, so words left by earlier calls need no
+// clearing.  Only the first arrival of a call installs the tag, by
+// compare-and-swap; later ones are single adds.  The caller orders its
+// earlier writes before this with a fence.
+__device__ __forceinline__ uint32_t arrive_tagged32(unsigned long long *ctr, unsigned long long tag,
+                                                    uint32_t n) {
+  unsigned long long cur = *reinterpret_cast<volatile unsigned long long *>(ctr);
+  while (true) {
+    if ((cur >> 32) == tag) {
+      const unsigned long long old = atomicAdd(ctr, (unsigned long long)n);
+      return (uint32_t)old + n;
+    }
+    const unsigned long long prev = atomicCAS(ctr, cur, (tag << 32) | n);
+    if (prev == cur) return n;
+    cur = prev;
+  }
+}
+
+// Orders this thread's global-memory accesses through the generic proxy and
+// through the async proxy (bulk copies, TMA) against each other, in both
+// directions: before later bulk loads of data written by generic stores, and
+// after completed TMA stores, before a generic release that publishes them.
 __device__ __forceinline__ void fence_proxy_async_global() {
   asm volatile("fence.proxy.async.global;" ::: "memory");
 }

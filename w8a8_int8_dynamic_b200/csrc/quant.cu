@@ -29,6 +29,13 @@
 //
 // The per-element arithmetic (the code from one step of reciprocal
 // refinement, rint by one addition) is in quant_common.cuh.
+//
+// quant_codes_kernel quantises the output of a layer whose GEMM epilogue has
+// already folded every row's maximum magnitude (the next layer's activation
+// quantisation fused with this one): it runs beside that GEMM and takes each
+// 128-row block as soon as the GEMM reports it complete, reading the rows
+// back while they are still in L2.  Same scale and codes as the kernels
+// above, from the same row maximum.
 #include <cuda_bf16.h>
 
 #include <algorithm>
@@ -45,11 +52,14 @@ namespace {
 // lane l the chunks w * 32 * CPL + 32 j + l.  AHEAD: the instance launched
 // ahead of a GEMM (same code; a function of its own, since the shared-memory
 // carveout is a property of the function).
+// zero_rows (nullable): a per-row word set to 0 here, before the GEMM behind
+// this kernel folds its output maxima into it.
 template <int CPL, bool AHEAD>
 __global__ void __launch_bounds__(512) quant_warps_kernel(const uint16_t *__restrict__ x,
                                                           int64_t ldx, int M, int K, int W, int R,
                                                           int8_t *__restrict__ q,
-                                                          float *__restrict__ a_scale) {
+                                                          float *__restrict__ a_scale,
+                                                          uint32_t *__restrict__ zero_rows) {
   // Let a dependent GEMM start its prologue while the rows are quantised.
   griddep_launch_dependents();
   griddep_wait();  // x may be the preceding kernel's output
@@ -58,6 +68,7 @@ __global__ void __launch_bounds__(512) quant_warps_kernel(const uint16_t *__rest
   const int rl = warp / W, w = warp - rl * W;
   const int64_t row = (int64_t)blockIdx.x * R + rl;
   const bool row_ok = row < M;
+  if (zero_rows && row_ok && w == 0 && lane == 0) zero_rows[row] = 0u;
   const int nchunks = K >> 3;  // 8 bf16 per 16-byte chunk
   const int c0 = w * 32 * CPL + lane;
   const uint16_t *xr = x + (row_ok ? row : 0) * ldx;
@@ -116,10 +127,11 @@ __global__ void __launch_bounds__(512) quant_warps_kernel(const uint16_t *__rest
 // hits L2), same arithmetic.
 __global__ void __launch_bounds__(1024) quant_rows_two_pass_kernel(
     const uint16_t *__restrict__ x, int64_t ldx, int K, int8_t *__restrict__ q,
-    float *__restrict__ a_scale) {
+    float *__restrict__ a_scale, uint32_t *__restrict__ zero_rows) {
   griddep_launch_dependents();
   griddep_wait();  // x may be the preceding kernel's output
   const int64_t row = blockIdx.x;
+  if (zero_rows && threadIdx.x == 0) zero_rows[row] = 0u;
   const int nchunks = K >> 3;
   const uint16_t *xr = x + row * ldx;
   uint32_t mx = 0;
@@ -156,6 +168,122 @@ __global__ void __launch_bounds__(1024) quant_rows_two_pass_kernel(
       out = exact_only ? codes8_ieee(c, s) : codes8(c, s, inv);
     }
     *reinterpret_cast<uint2 *>(qr + (int64_t)i * 8) = out;
+  }
+}
+
+// ---- codes of a GEMM's output whose row maxima its epilogue folded ----------
+// A unit is one row x kCodesSlice columns, handled by one warp (each lane
+// kCodesCPL 16-byte chunks); units are taken in row order, so a warp waits
+// for row blocks in the order the GEMM tends to finish them.  Rows are read
+// through L2 only (.cg): they are written by the GEMM running beside this
+// kernel.  The last CTA to finish clears the block words, so that a replayed
+// CUDA graph (same tag) finds them at zero.
+constexpr int kCodesCPL = 4;
+constexpr int kCodesSlice = 32 * kCodesCPL * 8;  // 1024 columns
+constexpr int kCodesWarps = 4;
+
+__device__ __forceinline__ uint4 ld_cg_u4(const void *p) {
+  uint4 v;
+  asm volatile("ld.global.cg.v4.u32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "l"(p));
+  return v;
+}
+
+// Waits until *word == want (acquire), polling every 256 ns (a block
+// completes every few microseconds).  The words are written by the GEMM this
+// kernel follows, every CTA of which has started before this kernel is
+// launched, so the wait ends unless something failed; it gives up like
+// mbar_wait_bounded: on *abort_flag, or after kWaitLimitNs (then it sets
+// *abort_flag and records W8A8_ERR_TIMEOUT).
+__device__ __noinline__ bool wait_block(const unsigned long long *word, unsigned long long want,
+                                        volatile int *abort_flag, int *status) {
+  if (ld_acquire_gpu(word) == want) return true;
+  const uint64_t t0 = global_timer_ns();
+  while (true) {
+    __nanosleep(256);
+    if (ld_acquire_gpu(word) == want) return true;
+    if (*abort_flag) return false;
+    if (global_timer_ns() - t0 > kWaitLimitNs) {
+      *abort_flag = 1;
+      atomicExch(status, (int)W8A8_ERR_TIMEOUT);
+      return false;
+    }
+  }
+}
+
+__global__ void __maxnreg__(56) quant_codes_kernel(
+    const uint16_t *__restrict__ y, int M, int N, const uint32_t *row_amax,
+    unsigned long long *row_done, unsigned long long tag, unsigned long long target,
+    int8_t *__restrict__ q, float *__restrict__ a_scale, unsigned long long *exit_word,
+    int *status) {
+  // The next layer's GEMM may take each SM as the GEMM beside this kernel
+  // leaves it; it waits on the device for this kernel to complete.
+  griddep_launch_dependents();
+  __shared__ int abort_flag;
+  __shared__ int last_cta;
+  if (threadIdx.x == 0) abort_flag = 0;
+  __syncthreads();
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int slices = (N + kCodesSlice - 1) / kCodesSlice;
+  const int nchunks = N >> 3;
+  const int64_t units = (int64_t)M * slices;
+  const int64_t stride = (int64_t)gridDim.x * kCodesWarps;
+  const unsigned long long want = (tag << 32) | target;
+  int ready = -1;  // the last row block this warp saw complete
+  for (int64_t u = (int64_t)blockIdx.x * kCodesWarps + warp; u < units; u += stride) {
+    const int row = (int)(u / slices), slice = (int)(u - (int64_t)row * slices);
+    const int blk = row >> 7;
+    if (blk != ready) {
+      int ok = 1;
+      if (lane == 0) ok = wait_block(row_done + blk, want, &abort_flag, status) ? 1 : 0;
+      ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
+      if (!ok) break;
+      (void)ld_acquire_gpu(row_done + blk);  // every lane acquires the block's rows
+      ready = blk;
+    }
+    const float amax = __uint_as_float(__ldcg(row_amax + row) << 16);
+    const float s = amax == 0.0f ? 0.0f : __fdiv_rn(amax, 127.0f);
+    if (slice == 0 && lane == 0) a_scale[row] = s;
+    const uint16_t *yr = y + (int64_t)row * N;
+    int8_t *qr = q + (int64_t)row * N;
+    const int c0 = slice * (kCodesSlice / 8) + lane;
+    uint4 v[kCodesCPL];
+#pragma unroll
+    for (int j = 0; j < kCodesCPL; ++j) {
+      const int c = c0 + 32 * j;
+      v[j] = make_uint4(0, 0, 0, 0);
+      if (c < nchunks) v[j] = ld_cg_u4(yr + (int64_t)c * 8);
+    }
+    uint2 out[kCodesCPL];
+    if (amax == 0.0f) {
+#pragma unroll
+      for (int j = 0; j < kCodesCPL; ++j) out[j] = make_uint2(0, 0);
+    } else if (s >= 1e-30f) {
+      const float inv = __frcp_rn(s);
+#pragma unroll
+      for (int j = 0; j < kCodesCPL; ++j) out[j] = codes8(v[j], s, inv);
+    } else {
+#pragma unroll
+      for (int j = 0; j < kCodesCPL; ++j) out[j] = codes8_ieee(v[j], s);
+    }
+#pragma unroll
+    for (int j = 0; j < kCodesCPL; ++j) {
+      const int c = c0 + 32 * j;
+      if (c < nchunks) *reinterpret_cast<uint2 *>(qr + (int64_t)c * 8) = out[j];
+    }
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    __threadfence();
+    last_cta = arrive_tagged32(exit_word, tag, 1u) == gridDim.x ? 1 : 0;
+  }
+  __syncthreads();
+  if (last_cta) {
+    // every CTA is past its waits: clear the words for the next call
+    const int nblk = (M + 127) >> 7;
+    for (int b = threadIdx.x; b < nblk; b += blockDim.x) row_done[b] = 0ull;
+    if (threadIdx.x == 0) *exit_word = 0ull;
   }
 }
 
@@ -269,7 +397,8 @@ cudaError_t launch_dependent(void (*k)(Params...), int slot, dim3 grid, dim3 blo
 }  // namespace
 
 w8a8_status launch_quant(const void *x, int64_t M, int64_t K, int64_t ldx, int8_t *q,
-                         float *a_scale, cudaStream_t stream, bool ahead_of_gemm) {
+                         float *a_scale, cudaStream_t stream, bool ahead_of_gemm,
+                         uint32_t *zero_rows) {
   const int64_t nchunks = K / 8;
   const uint16_t *xp = static_cast<const uint16_t *>(x);
   // Chunks per lane (a power of two): 4 where the row has that many per lane;
@@ -296,7 +425,7 @@ w8a8_status launch_quant(const void *x, int64_t M, int64_t K, int64_t ldx, int8_
   if (W > 16) {
     // 1024-thread CTAs never leave room for a GEMM CTA: default carveout.
     e = launch_dependent(quant_rows_two_pass_kernel, -1, dim3((unsigned)M), dim3(1024), stream,
-                         xp, ldx, (int)K, q, a_scale);
+                         xp, ldx, (int)K, q, a_scale, zero_rows);
   } else {
     const int R = W >= 4 ? 1 : (int)(4 / W);  // rows per CTA: about 128 threads
     const unsigned grid = (unsigned)((M + R - 1) / R);
@@ -312,10 +441,10 @@ w8a8_status launch_quant(const void *x, int64_t M, int64_t K, int64_t ldx, int8_
   case C:                                                                                 \
     e = wide ? launch_dependent(quant_warps_kernel<C, true>, SLOT, dim3(grid),            \
                                 dim3(threads), stream, xp, ldx, (int)M, (int)K,           \
-                                (int)W, R, q, a_scale)                                    \
+                                (int)W, R, q, a_scale, zero_rows)                         \
              : launch_dependent(quant_warps_kernel<C, false>, -1, dim3(grid),             \
                                 dim3(threads), stream, xp, ldx, (int)M, (int)K,           \
-                                (int)W, R, q, a_scale);                                   \
+                                (int)W, R, q, a_scale, zero_rows);                        \
     break;
       W8A8_QUANT_CASE(1, 0)
       W8A8_QUANT_CASE(2, 1)
@@ -332,6 +461,25 @@ w8a8_status launch_quant(const void *x, int64_t M, int64_t K, int64_t ldx, int8_
   return from_cuda(cudaGetLastError());
 }
 
+w8a8_status launch_codes(const void *y, int64_t M, int64_t N, const uint32_t *row_amax,
+                         unsigned long long *row_done, unsigned long long tag, int8_t *q,
+                         float *a_scale, unsigned long long *exit_word, cudaStream_t stream) {
+  int *status = status_word();
+  if (!status) return W8A8_ERR_CUDA;
+  const int64_t slices = (N + kCodesSlice - 1) / kCodesSlice;
+  const int64_t warps = M * slices;
+  // two CTAs an SM fit beside a GEMM CTA (registers: 2 x 128 x 56)
+  const int64_t grid = std::max<int64_t>(
+      1, std::min<int64_t>((warps + kCodesWarps - 1) / kCodesWarps, 2 * (int64_t)sm_count()));
+  const cudaError_t e = launch_dependent(
+      quant_codes_kernel, 5, dim3((unsigned)grid), dim3(32 * kCodesWarps), stream,
+      static_cast<const uint16_t *>(y), (int)M, (int)N, row_amax, row_done, tag,
+      (unsigned long long)(4 * N), q, a_scale, exit_word, status);
+  if (e != cudaSuccess) return from_cuda(e);
+  count_launch();
+  return from_cuda(cudaGetLastError());
+}
+
 }  // namespace w8a8
 
 using namespace w8a8;
@@ -343,7 +491,8 @@ extern "C" w8a8_status w8a8_quant_act(const void *x, int64_t M, int64_t K, int64
   if (K % 16 != 0 || K > kMaxK) return W8A8_ERR_UNSUPPORTED_SHAPE;
   if (!aligned16(x) || !aligned16(q) || !aligned16(a_scale) || ldx % 8 != 0)
     return W8A8_ERR_ALIGNMENT;
-  return launch_quant(x, M, K, ldx, q, a_scale, reinterpret_cast<cudaStream_t>(stream), false);
+  return launch_quant(x, M, K, ldx, q, a_scale, reinterpret_cast<cudaStream_t>(stream), false,
+                      nullptr);
 }
 
 
