@@ -247,7 +247,8 @@ w8a8_status w8a8_linear_act(const void *x, int64_t ldx, const void *packed_w,
  *                call-tagged completion word per 128-row block (contents on
  *                entry do not matter; the last CTA of each call clears the
  *                words, so a replayed CUDA graph finds them at zero)
- * Limits as w8a8_linear, plus N <= 2^28.  After a call that timed out
+ * Limits as w8a8_linear, plus N % 16 == 0 (q_next is the next layer's GEMM
+ * input, whose K = N) and N <= 2^28.  After a call that timed out
  * (W8A8_ERR_TIMEOUT) the words may be left set: capture CUDA graphs of this
  * call again (a new capture draws a new tag) before replaying them. */
 w8a8_status w8a8_linear_act_quant_workspace_bytes(int64_t M, int64_t N, int64_t K,

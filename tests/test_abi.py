@@ -127,7 +127,7 @@ def test_act_quant_rejects_bad_arguments_and_sizes_its_workspace(L):
     from w8a8_int8_dynamic_b200 import binding
     f = L.w8a8_linear_act_quant
     big = 1 << 30
-    ok = (FAKE, 16, FAKE, FAKE, None, FAKE, 4, 8, 16, 0, FAKE, FAKE, FAKE, big, None)
+    ok = (FAKE, 16, FAKE, FAKE, None, FAKE, 4, 16, 16, 0, FAKE, FAKE, FAKE, big, None)
     # every argument valid but the one under test (nothing may launch)
     def call(**kw):
         a = list(ok)
@@ -141,9 +141,10 @@ def test_act_quant_rejects_bad_arguments_and_sizes_its_workspace(L):
     assert call(a10=FAKE_MIS) == 2             # q_next misaligned
     assert call(a11=FAKE_MIS) == 2             # a_scale_next misaligned
     assert call(a13=1) == 6                    # workspace too small
-    assert call(a7=(1 << 28) + 8) == 3         # N beyond the fused limit
+    assert call(a7=(1 << 28) + 16) == 3        # N beyond the fused limit
+    assert call(a7=24) == 3                    # N % 16 (the next layer's K)
     assert call(a8=40) == 3                    # K % 16
-    for M, N, K in [(4096, 12288, 3072), (1000, 2056, 1040), (16, 4096, 4096)]:
+    for M, N, K in [(4096, 12288, 3072), (1000, 2064, 1040), (16, 4096, 4096)]:
         lin = binding.linear_workspace_bytes(M, N, K)
         rnd = lambda v: (v + 255) // 256 * 256  # noqa: E731
         extra = rnd(4 * M) + rnd(8 * ((M + 127) // 128)) + 256

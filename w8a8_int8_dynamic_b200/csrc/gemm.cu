@@ -667,7 +667,8 @@ w8a8_status w8a8_linear_act_quant(const void *x, int64_t ldx, const void *packed
   if (!w_scale || !workspace || !q_next || !a_scale_next) return W8A8_ERR_INVALID_ARG;
   if (ldx < K) return W8A8_ERR_INVALID_ARG;
   if (act != W8A8_ACT_NONE && act != W8A8_ACT_GELU_TANH) return W8A8_ERR_INVALID_ARG;
-  if (N > kMaxFusedN) return W8A8_ERR_UNSUPPORTED_SHAPE;
+  // the codes are the next layer's GEMM input, K = N
+  if (N > kMaxFusedN || N % 16 != 0) return W8A8_ERR_UNSUPPORTED_SHAPE;
   if (ldx % 8 != 0 || !aligned16(w_scale) || !aligned16(workspace) ||
       (bias && !aligned16(bias)) || !aligned16(q_next) || !aligned16(a_scale_next))
     return W8A8_ERR_ALIGNMENT;
