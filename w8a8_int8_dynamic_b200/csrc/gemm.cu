@@ -77,7 +77,7 @@ struct LargeSmem {
 // starts its prologue and first weight copies while they run.
 // ROWMAX: the next layer's quantisation is fused in (GemmArgs::row_amax).
 template <int BN, int STAGES, int KPS, bool OUT_I32, bool ROWMAX>
-__global__ void __maxnreg__(ROWMAX ? kGemmRegsRowmax : kGemmRegs)
+__global__ void __maxnreg__(kGemmRegs)
     gemm_kernel(const __grid_constant__ CUtensorMap tmap_q,
                 const __grid_constant__ CUtensorMap tmap_y, const GemmArgs args) {
   using L = LargeSmem<BN, STAGES, KPS>;
@@ -153,8 +153,10 @@ __global__ void __maxnreg__(ROWMAX ? kGemmRegsRowmax : kGemmRegs)
       Cursor c;
       c.tile = tile;
       c.j = 0;
-      c.q_row = (tile % args.tiles_m) * kBM;
-      c.w = args.packed_w + (size_t)(tile / args.tiles_m) * (BN / 128) * slab_bytes;
+      int mb, nb;
+      tile_coords<ROWMAX>(args, tile, mb, nb);
+      c.q_row = mb * kBM;
+      c.w = args.packed_w + (size_t)nb * (BN / 128) * slab_bytes;
       return c;
     };
     auto advance = [&](Cursor &c) {
@@ -299,7 +301,8 @@ __global__ void __maxnreg__(ROWMAX ? kGemmRegsRowmax : kGemmRegs)
     uint8_t *s_out = smem + L::kOut + (warp - 2) * kEpiStagePerWarp;
     for (int t = 0; t < my_tiles; ++t) {
       const int tile = blockIdx.x + t * gridDim.x;
-      const int mb = tile % args.tiles_m, nb = tile / args.tiles_m;
+      int mb, nb;
+      tile_coords<ROWMAX>(args, tile, mb, nb);
       const uint32_t b = t & 1, bph = (t >> 1) & 1;
       const int n0 = nb * BN + ew.half * kCols;
       const int row0 = mb * kBM + ew.quarter * 32;
@@ -477,7 +480,8 @@ w8a8_status launch_scaled_mm(const int8_t *q, const float *a_scale, const void *
   a.tiles_m = (int)((M + kBM - 1) / kBM);
   a.tiles_n = 0;
   a.act = out_i32 ? W8A8_ACT_NONE : act;
-  a.prefetch_kb = (pdl && prefetch) ? kPrefetchKb : 0;
+  // (the prefetch shares slabs out by the plain tile order)
+  a.prefetch_kb = (pdl && prefetch && !sig) ? kPrefetchKb : 0;
   a.status = status_word();
   if (!a.status) return W8A8_ERR_CUDA;
   if (sig && !out_i32) {
@@ -668,7 +672,8 @@ w8a8_status w8a8_linear_act_quant(const void *x, int64_t ldx, const void *packed
   if (ldx < K) return W8A8_ERR_INVALID_ARG;
   if (act != W8A8_ACT_NONE && act != W8A8_ACT_GELU_TANH) return W8A8_ERR_INVALID_ARG;
   // the codes are the next layer's GEMM input, K = N
-  if (N > kMaxFusedN || N % 16 != 0) return W8A8_ERR_UNSUPPORTED_SHAPE;
+  if (N > kMaxFusedN || N % 16 != 0 || codes_units(M, N) >= ((int64_t)1 << 31))
+    return W8A8_ERR_UNSUPPORTED_SHAPE;
   if (ldx % 8 != 0 || !aligned16(w_scale) || !aligned16(workspace) ||
       (bias && !aligned16(bias)) || !aligned16(q_next) || !aligned16(a_scale_next))
     return W8A8_ERR_ALIGNMENT;
@@ -691,7 +696,7 @@ w8a8_status w8a8_linear_act_quant(const void *x, int64_t ldx, const void *packed
   off += round_up(M * 4, 256);
   unsigned long long *row_done = reinterpret_cast<unsigned long long *>(ws + off);
   off += round_up(((M + 127) / 128) * 8, 256);
-  unsigned long long *exit_word = reinterpret_cast<unsigned long long *>(ws + off);
+  unsigned long long *words = reinterpret_cast<unsigned long long *>(ws + off);  // [2]
   RowSignal sig{row_amax, row_done, next_call_tag() & 0xFFFFFFFFull};
   if (sig.tag == 0) sig.tag = 1;
   st = launch_quant(x, M, K, ldx, q, a_scale, s, true, row_amax);
@@ -699,7 +704,7 @@ w8a8_status w8a8_linear_act_quant(const void *x, int64_t ldx, const void *packed
   st = launch_scaled_mm(q, a_scale, packed_w, w_scale, bias, y, false, M, N, K, s, true, act, true,
                         &sig);
   if (st != W8A8_OK) return st;
-  return launch_codes(y, M, N, row_amax, row_done, sig.tag, q_next, a_scale_next, exit_word, s);
+  return launch_codes(y, M, N, row_amax, row_done, sig.tag, q_next, a_scale_next, words, s);
 }
 
 }  // extern "C"

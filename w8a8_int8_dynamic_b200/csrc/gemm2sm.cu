@@ -66,7 +66,7 @@ struct PairSmem {
 // starts its prologue and first weight copies while they run.
 // ROWMAX: the next layer's quantisation is fused in (GemmArgs::row_amax).
 template <int BN, int STAGES, bool ROWMAX>
-__global__ void __maxnreg__(ROWMAX ? kGemmRegsRowmax : kGemmRegs)
+__global__ void __maxnreg__(kGemmRegs)
     gemm2sm_kernel(const __grid_constant__ CUtensorMap tmap_q,
                    const __grid_constant__ CUtensorMap tmap_w,
                    const __grid_constant__ CUtensorMap tmap_w64,
@@ -173,7 +173,8 @@ __global__ void __maxnreg__(ROWMAX ? kGemmRegsRowmax : kGemmRegs)
         return c;
       }
       const int item = seg_tile(i), tile = item_tile(item), half = item_half(item);
-      const int mb = tile % args.tiles_m, nb = tile / args.tiles_m;
+      int mb, nb;
+      tile_coords<ROWMAX>(args, tile, mb, nb);
       c.kind = (BN == 256 && half >= 0) ? 1 : 0;
       c.qrow = mb * 256 + (int)rank * 128;
       if (BN == 256 && half >= 0)
@@ -324,7 +325,8 @@ __global__ void __maxnreg__(ROWMAX ? kGemmRegsRowmax : kGemmRegs)
     const int j0 = ew.half * kCols;  // first tile column of this warp
     for (int i = 0; i < nseg; ++i) {
       const int tile = item_tile(seg_tile(i)), half = item_half(seg_tile(i));
-      const int mb = tile % args.tiles_m, nb = tile / args.tiles_m;
+      int mb, nb;
+      tile_coords<ROWMAX>(args, tile, mb, nb);
       const int row0 = mb * 256 + (int)rank * 128 + ew.quarter * 32;
       // a half tile's 128 columns: 64 per warp
       const int jw = half >= 0 ? half * 128 + ew.half * 64 : j0;  // warp's first tile column

@@ -31,11 +31,6 @@ constexpr int kGemmThreads = 64 + 32 * kEpiWarps;
 // that hold three of them (most SMs, for 512 rows of 4096), not on those with
 // four.
 constexpr int kGemmRegs = 128;
-// The instances with the next layer's quantisation fused in (ROWMAX) keep
-// one more value a lane through the epilogue and spill below 144 (the pair
-// kernel at 136 too).  At 144 a CTA takes 50,688 registers, and the codes
-// kernel's two 4-warp CTAs of 56 registers (14,336) still fit beside it.
-constexpr int kGemmRegsRowmax = 144;
 
 struct GemmArgs {
   const uint8_t *packed_w;
@@ -90,6 +85,22 @@ __device__ __forceinline__ void publish_rows(const GemmArgs &a, int lane, int ro
     arrive_tagged32(a.row_done + (row0 >> 7), a.done_tag, (uint32_t)cols);
   }
   __syncwarp();
+}
+
+// The (row tile, column tile) of a linear tile index.  Plain instances walk
+// the tiles column tile by column tile (row tile fastest: tiles running at
+// the same time share a weight slab in L2).  ROWMAX instances walk them row
+// tile by row tile, so that their row blocks complete one after another
+// while the GEMM runs and the codes kernel beside it can follow.
+template <bool ROWMAX>
+__device__ __forceinline__ void tile_coords(const GemmArgs &a, int tile, int &mb, int &nb) {
+  if (ROWMAX) {
+    mb = tile / a.tiles_n;
+    nb = tile - mb * a.tiles_n;
+  } else {
+    nb = tile / a.tiles_m;
+    mb = tile - nb * a.tiles_m;
+  }
 }
 
 // Epilogue warp ew (0..7): TMEM lane quarter and which half of the columns.
@@ -188,6 +199,20 @@ __device__ __forceinline__ void for_tmem_chunks(uint32_t taddr, Valid valid, Bod
   }
 }
 
+// As for_tmem_chunks, one chunk in flight at a time.
+template <int NCH, typename Valid, typename Body>
+__device__ __forceinline__ void for_tmem_chunks_single(uint32_t taddr, Valid valid, Body body) {
+  uint32_t v[32];
+#pragma unroll 1
+  for (int c = 0; c < NCH; ++c) {
+    if (!valid(c)) return;
+    tmem_ld_32x32b_x32(taddr + c * 32, v);
+    tmem_ld_wait_regs(v);
+    body(v, c);
+    __syncwarp();  // converged for the next .sync.aligned tcgen05 instruction
+  }
+}
+
 // int32 accumulators straight to global memory (inspection export): COLS
 // columns of this warp's 32 rows, starting at global column n0.
 template <int COLS>
@@ -238,8 +263,17 @@ __device__ __forceinline__ void epilogue_tma(const GemmArgs &a, const CUtensorMa
                                              uint32_t taddr, int lane, int row0, int n0, float as,
                                              const float *s_ws, const uint16_t *s_bias,
                                              uint8_t *stage, uint32_t &rmax, int ncols = COLS) {
-  for_tmem_chunks<COLS / 32>(
-      taddr, [&](int c) { return c * 32 < ncols && n0 + c * 32 < a.N; },
+  // ROWMAX instances load one chunk at a time: their tiles are long (large
+  // M, N and K), so the epilogue is far off the critical path, and the
+  // registers of the second chunk buffer leave room beside the GEMM for the
+  // codes kernel's warps.
+  auto run = [&](auto valid, auto body) {
+    if (ROWMAX)
+      for_tmem_chunks_single<COLS / 32>(taddr, valid, body);
+    else
+      for_tmem_chunks<COLS / 32>(taddr, valid, body);
+  };
+  run([&](int c) { return c * 32 < ncols && n0 + c * 32 < a.N; },
       [&](const uint32_t(&v)[32], int c) {
         uint4 out[4];
 #pragma unroll

@@ -116,9 +116,12 @@ w8a8_status launch_quant(const void *x, int64_t M, int64_t K, int64_t ldx, int8_
                          uint32_t *zero_rows = nullptr);
 // The codes kernel of the fused next-layer quantisation (quant.cu): the codes
 // and scales of y [M, N] from the row maxima, each 128-row block once its
-// row_done word reads (tag, 4 N); exit_word counts the CTAs out.
+// row_done word reads (tag, 4 N); words[0] hands out the work units,
+// words[1] counts the CTAs out.
 w8a8_status launch_codes(const void *y, int64_t M, int64_t N, const uint32_t *row_amax,
                          unsigned long long *row_done, unsigned long long tag, int8_t *q,
-                         float *a_scale, unsigned long long *exit_word, cudaStream_t stream);
+                         float *a_scale, unsigned long long *words, cudaStream_t stream);
+// Work units of the codes kernel (must stay below 2^32).
+int64_t codes_units(int64_t M, int64_t N);
 
 }  // namespace w8a8

@@ -173,13 +173,16 @@ __global__ void __launch_bounds__(1024) quant_rows_two_pass_kernel(
 
 // ---- codes of a GEMM's output whose row maxima its epilogue folded ----------
 // A unit is one row x kCodesSlice columns, handled by one warp (each lane
-// kCodesCPL 16-byte chunks); units are taken in row order, so a warp waits
-// for row blocks in the order the GEMM tends to finish them.  Rows are read
-// through L2 only (.cg): they are written by the GEMM running beside this
-// kernel.  The last CTA to finish clears the block words, so that a replayed
+// kCodesCPL 16-byte chunks, all loads in flight together).  Warps take units
+// in row order from a call-tagged counter, the next one asked for before the
+// current one is processed, so that whichever warps are resident beside the
+// GEMM share the work as its row blocks complete, and a CTA that only
+// becomes resident after the GEMM finds the work done.  Rows are read
+// through L2 only (.cg): the GEMM beside this kernel writes them.  The last
+// CTA to finish clears the counter and the block words, so that a replayed
 // CUDA graph (same tag) finds them at zero.
-constexpr int kCodesCPL = 4;
-constexpr int kCodesSlice = 32 * kCodesCPL * 8;  // 1024 columns
+constexpr int kCodesCPL = 8;
+constexpr int kCodesSlice = 32 * kCodesCPL * 8;  // 2048 columns
 constexpr int kCodesWarps = 4;
 
 __device__ __forceinline__ uint4 ld_cg_u4(const void *p) {
@@ -212,10 +215,13 @@ __device__ __noinline__ bool wait_block(const unsigned long long *word, unsigned
   }
 }
 
-__global__ void __maxnreg__(56) quant_codes_kernel(
+// At most 64 registers: two 4-warp CTAs fit beside a GEMM CTA of 128
+// registers a thread (its 11 warps leave 4,096 registers on each of three SM
+// sub-partitions and more on the fourth).
+__global__ void __maxnreg__(64) quant_codes_kernel(
     const uint16_t *__restrict__ y, int M, int N, const uint32_t *row_amax,
     unsigned long long *row_done, unsigned long long tag, unsigned long long target,
-    int8_t *__restrict__ q, float *__restrict__ a_scale, unsigned long long *exit_word,
+    int8_t *__restrict__ q, float *__restrict__ a_scale, unsigned long long *words,
     int *status) {
   // The next layer's GEMM may take each SM as the GEMM beside this kernel
   // leaves it; it waits on the device for this kernel to complete.
@@ -224,15 +230,22 @@ __global__ void __maxnreg__(56) quant_codes_kernel(
   __shared__ int last_cta;
   if (threadIdx.x == 0) abort_flag = 0;
   __syncthreads();
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  unsigned long long *next_unit = words;  // (tag << 32) | units handed out
+  unsigned long long *exit_word = words + 1;
+  const int lane = threadIdx.x & 31;
   const int slices = (N + kCodesSlice - 1) / kCodesSlice;
   const int nchunks = N >> 3;
-  const int64_t units = (int64_t)M * slices;
-  const int64_t stride = (int64_t)gridDim.x * kCodesWarps;
+  const uint32_t units = (uint32_t)M * (uint32_t)slices;
   const unsigned long long want = (tag << 32) | target;
   int ready = -1;  // the last row block this warp saw complete
-  for (int64_t u = (int64_t)blockIdx.x * kCodesWarps + warp; u < units; u += stride) {
-    const int row = (int)(u / slices), slice = (int)(u - (int64_t)row * slices);
+  uint32_t u = 0;
+  if (lane == 0) u = arrive_tagged32(next_unit, tag, 1u) - 1u;
+  u = __shfl_sync(0xFFFFFFFFu, u, 0);
+  while (u < units) {
+    uint32_t nu = 0;
+    if (lane == 0) nu = arrive_tagged32(next_unit, tag, 1u) - 1u;  // in flight meanwhile
+    const int row = (int)(u / (uint32_t)slices);
+    const int slice = (int)(u - (uint32_t)row * (uint32_t)slices);
     const int blk = row >> 7;
     if (blk != ready) {
       int ok = 1;
@@ -242,9 +255,6 @@ __global__ void __maxnreg__(56) quant_codes_kernel(
       (void)ld_acquire_gpu(row_done + blk);  // every lane acquires the block's rows
       ready = blk;
     }
-    const float amax = __uint_as_float(__ldcg(row_amax + row) << 16);
-    const float s = amax == 0.0f ? 0.0f : __fdiv_rn(amax, 127.0f);
-    if (slice == 0 && lane == 0) a_scale[row] = s;
     const uint16_t *yr = y + (int64_t)row * N;
     int8_t *qr = q + (int64_t)row * N;
     const int c0 = slice * (kCodesSlice / 8) + lane;
@@ -255,23 +265,31 @@ __global__ void __maxnreg__(56) quant_codes_kernel(
       v[j] = make_uint4(0, 0, 0, 0);
       if (c < nchunks) v[j] = ld_cg_u4(yr + (int64_t)c * 8);
     }
-    uint2 out[kCodesCPL];
+    const float amax = __uint_as_float(__ldcg(row_amax + row) << 16);
+    const float s = amax == 0.0f ? 0.0f : __fdiv_rn(amax, 127.0f);
+    if (slice == 0 && lane == 0) a_scale[row] = s;
     if (amax == 0.0f) {
 #pragma unroll
-      for (int j = 0; j < kCodesCPL; ++j) out[j] = make_uint2(0, 0);
+      for (int j = 0; j < kCodesCPL; ++j) {
+        const int c = c0 + 32 * j;
+        if (c < nchunks) *reinterpret_cast<uint2 *>(qr + (int64_t)c * 8) = make_uint2(0, 0);
+      }
     } else if (s >= 1e-30f) {
       const float inv = __frcp_rn(s);
 #pragma unroll
-      for (int j = 0; j < kCodesCPL; ++j) out[j] = codes8(v[j], s, inv);
+      for (int j = 0; j < kCodesCPL; ++j) {
+        const int c = c0 + 32 * j;
+        if (c < nchunks) *reinterpret_cast<uint2 *>(qr + (int64_t)c * 8) = codes8(v[j], s, inv);
+      }
     } else {
+      // (unrolled: a runtime index into v would move it to local memory)
 #pragma unroll
-      for (int j = 0; j < kCodesCPL; ++j) out[j] = codes8_ieee(v[j], s);
+      for (int j = 0; j < kCodesCPL; ++j) {
+        const int c = c0 + 32 * j;
+        if (c < nchunks) *reinterpret_cast<uint2 *>(qr + (int64_t)c * 8) = codes8_ieee(v[j], s);
+      }
     }
-#pragma unroll
-    for (int j = 0; j < kCodesCPL; ++j) {
-      const int c = c0 + 32 * j;
-      if (c < nchunks) *reinterpret_cast<uint2 *>(qr + (int64_t)c * 8) = out[j];
-    }
+    u = __shfl_sync(0xFFFFFFFFu, nu, 0);
   }
   __syncthreads();
   if (threadIdx.x == 0) {
@@ -280,10 +298,13 @@ __global__ void __maxnreg__(56) quant_codes_kernel(
   }
   __syncthreads();
   if (last_cta) {
-    // every CTA is past its waits: clear the words for the next call
+    // every CTA is past its waits and grabs: clear the words for the next call
     const int nblk = (M + 127) >> 7;
     for (int b = threadIdx.x; b < nblk; b += blockDim.x) row_done[b] = 0ull;
-    if (threadIdx.x == 0) *exit_word = 0ull;
+    if (threadIdx.x == 0) {
+      *next_unit = 0ull;
+      *exit_word = 0ull;
+    }
   }
 }
 
@@ -461,20 +482,21 @@ w8a8_status launch_quant(const void *x, int64_t M, int64_t K, int64_t ldx, int8_
   return from_cuda(cudaGetLastError());
 }
 
+int64_t codes_units(int64_t M, int64_t N) { return M * ((N + kCodesSlice - 1) / kCodesSlice); }
+
 w8a8_status launch_codes(const void *y, int64_t M, int64_t N, const uint32_t *row_amax,
                          unsigned long long *row_done, unsigned long long tag, int8_t *q,
-                         float *a_scale, unsigned long long *exit_word, cudaStream_t stream) {
+                         float *a_scale, unsigned long long *words, cudaStream_t stream) {
   int *status = status_word();
   if (!status) return W8A8_ERR_CUDA;
-  const int64_t slices = (N + kCodesSlice - 1) / kCodesSlice;
-  const int64_t warps = M * slices;
-  // two CTAs an SM fit beside a GEMM CTA (registers: 2 x 128 x 56)
+  const int64_t units = codes_units(M, N);
+  // two 4-warp CTAs an SM fit beside a GEMM CTA
   const int64_t grid = std::max<int64_t>(
-      1, std::min<int64_t>((warps + kCodesWarps - 1) / kCodesWarps, 2 * (int64_t)sm_count()));
+      1, std::min<int64_t>((units + kCodesWarps - 1) / kCodesWarps, 2 * (int64_t)sm_count()));
   const cudaError_t e = launch_dependent(
       quant_codes_kernel, 5, dim3((unsigned)grid), dim3(32 * kCodesWarps), stream,
       static_cast<const uint16_t *>(y), (int)M, (int)N, row_amax, row_done, tag,
-      (unsigned long long)(4 * N), q, a_scale, exit_word, status);
+      (unsigned long long)(4 * N), q, a_scale, words, status);
   if (e != cudaSuccess) return from_cuda(e);
   count_launch();
   return from_cuda(cudaGetLastError());
