@@ -233,20 +233,23 @@ w8a8_status w8a8_linear_act(const void *x, int64_t ldx, const void *packed_w,
  * the results equal, bit for bit, w8a8_linear_act(..., y, ...) followed by
  * w8a8_quant_act(y, M, N, N, q_next, a_scale_next).  The next layer then runs
  * w8a8_scaled_mm(q_next, a_scale_next, ...) on them.
- * How: the GEMM epilogue folds every row's largest output magnitude while it
- * stores y, and reports each 128-row block once its stores are complete; a
- * codes kernel running beside the GEMM quantises each block as it completes,
- * reading the rows back from L2, so that no separate pass over y follows the
- * layer.  Three launches on `stream` (for M <= 16: the layer, then the
- * quantisation kernel on y).
+ * How: the GEMM walks its output tiles row block by row block; its epilogue
+ * folds every row's largest output magnitude while it stores y and reports
+ * each 128-row block once its stores are complete, and the GEMM's own warps
+ * (an otherwise idle warp throughout, the epilogue warps between their
+ * tiles and after their last) quantise each block as it completes, reading
+ * the rows back from L2, so that no separate pass over y follows the layer.
+ * Two launches on `stream`, as w8a8_linear_act (for M <= 16: the layer, then
+ * the quantisation kernel on y).
  *   x, ldx, packed_w, w_scale, bias, y, M, N, K, act: as w8a8_linear_act
  *   q_next       device, int8 [M, N] dense (output): the codes of y
  *   a_scale_next device, fp32 [M] (output): their per-row scales
  *   workspace    device, ws_bytes >= w8a8_linear_act_quant_workspace_bytes(M,
- *                N, K): w8a8_linear's workspace, then the row maxima and one
- *                call-tagged completion word per 128-row block (contents on
- *                entry do not matter; the last CTA of each call clears the
- *                words, so a replayed CUDA graph finds them at zero)
+ *                N, K): w8a8_linear's workspace, then the row maxima, one
+ *                call-tagged completion word per 128-row block and two words
+ *                that hand out the codes' work (contents on entry do not
+ *                matter; the last CTA of each call clears the words, so a
+ *                replayed CUDA graph finds them at zero)
  * Limits as w8a8_linear, plus N % 16 == 0 (q_next is the next layer's GEMM
  * input, whose K = N) and N <= 2^28.  After a call that timed out
  * (W8A8_ERR_TIMEOUT) the words may be left set: capture CUDA graphs of this

@@ -97,8 +97,8 @@ __global__ void __maxnreg__(kGemmRegs)
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + L::kMisc);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + L::kMisc + 4);
 
-  // With the next layer's quantisation fused in, the codes kernel behind
-  // this one becomes resident beside it and follows its row blocks.
+  // With the next layer's quantisation fused in, the next layer's GEMM (a
+  // programmatic dependent) takes each SM as this kernel leaves it.
   if (ROWMAX) griddep_launch_dependents();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
@@ -242,7 +242,11 @@ __global__ void __maxnreg__(kGemmRegs)
       }
     }
   } else if (warp == 0) {
-    // idle
+    // idle, or (next-layer quantisation fused in) forming codes of the
+    // output's row blocks as they complete
+    if (ROWMAX)
+      while (codes_take_one(args, lane, abort_flag)) {
+      }
   } else if (warp == 1) {
     if (lane == 0) {
       // ---------------- MMA issuer ----------------
@@ -313,6 +317,7 @@ __global__ void __maxnreg__(kGemmRegs)
         if (row0 + lane < args.M) as = __ldg(args.a_scale + row0 + lane);
       }
       __syncwarp();
+      if (ROWMAX) codes_while_waiting(args, lane, &tfull[b], bph);
       int ok = 0;
       if (lane == 0) ok = mbar_wait(&tfull[b], bph, abort_flag, args.status);
       ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
@@ -334,6 +339,9 @@ __global__ void __maxnreg__(kGemmRegs)
     }
     if (lane == 0) bulk_wait_group_all();  // output stores complete before exit
     __syncwarp();
+    if (ROWMAX)  // help with the codes still to form
+      while (codes_take_one(args, lane, abort_flag)) {
+      }
   }
 
   tc_fence_before();
@@ -342,6 +350,7 @@ __global__ void __maxnreg__(kGemmRegs)
     tc_fence_after();
     tmem_dealloc(tmem_base, kTmemCols);
   }
+  if (ROWMAX) codes_exit(args);
 }
 
 // ============================================================================
@@ -488,6 +497,9 @@ w8a8_status launch_scaled_mm(const int8_t *q, const float *a_scale, const void *
     a.row_amax = sig->row_amax;
     a.row_done = sig->row_done;
     a.done_tag = sig->tag;
+    a.q_next = sig->q_next;
+    a.a_scale_next = sig->a_scale_next;
+    a.codes_words = sig->words;
   }
   CUtensorMap tmap_y;
   if (out_i32) {
@@ -671,8 +683,9 @@ w8a8_status w8a8_linear_act_quant(const void *x, int64_t ldx, const void *packed
   if (!w_scale || !workspace || !q_next || !a_scale_next) return W8A8_ERR_INVALID_ARG;
   if (ldx < K) return W8A8_ERR_INVALID_ARG;
   if (act != W8A8_ACT_NONE && act != W8A8_ACT_GELU_TANH) return W8A8_ERR_INVALID_ARG;
-  // the codes are the next layer's GEMM input, K = N
-  if (N > kMaxFusedN || N % 16 != 0 || codes_units(M, N) >= ((int64_t)1 << 31))
+  // the codes are the next layer's GEMM input, K = N; the codes' work units
+  // (rows x 2048 columns) are counted in 32 bits
+  if (N > kMaxFusedN || N % 16 != 0 || M * ((N + 2047) / 2048) >= ((int64_t)1 << 31))
     return W8A8_ERR_UNSUPPORTED_SHAPE;
   if (ldx % 8 != 0 || !aligned16(w_scale) || !aligned16(workspace) ||
       (bias && !aligned16(bias)) || !aligned16(q_next) || !aligned16(a_scale_next))
@@ -697,14 +710,12 @@ w8a8_status w8a8_linear_act_quant(const void *x, int64_t ldx, const void *packed
   unsigned long long *row_done = reinterpret_cast<unsigned long long *>(ws + off);
   off += round_up(((M + 127) / 128) * 8, 256);
   unsigned long long *words = reinterpret_cast<unsigned long long *>(ws + off);  // [2]
-  RowSignal sig{row_amax, row_done, next_call_tag() & 0xFFFFFFFFull};
+  RowSignal sig{row_amax, row_done, next_call_tag() & 0xFFFFFFFFull, q_next, a_scale_next, words};
   if (sig.tag == 0) sig.tag = 1;
   st = launch_quant(x, M, K, ldx, q, a_scale, s, true, row_amax);
   if (st != W8A8_OK) return st;
-  st = launch_scaled_mm(q, a_scale, packed_w, w_scale, bias, y, false, M, N, K, s, true, act, true,
-                        &sig);
-  if (st != W8A8_OK) return st;
-  return launch_codes(y, M, N, row_amax, row_done, sig.tag, q_next, a_scale_next, words, s);
+  return launch_scaled_mm(q, a_scale, packed_w, w_scale, bias, y, false, M, N, K, s, true, act,
+                          true, &sig);
 }
 
 }  // extern "C"

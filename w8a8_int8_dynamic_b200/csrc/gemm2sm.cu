@@ -91,8 +91,8 @@ __global__ void __maxnreg__(kGemmRegs)
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + L::kMisc);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + L::kMisc + 4);
 
-  // With the next layer's quantisation fused in, the codes kernel behind
-  // this one becomes resident beside it and follows its row blocks.
+  // With the next layer's quantisation fused in, the next layer's GEMM (a
+  // programmatic dependent) takes each SM as this kernel leaves it.
   if (ROWMAX) griddep_launch_dependents();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t crank = cluster_ctarank();
@@ -263,7 +263,11 @@ __global__ void __maxnreg__(kGemmRegs)
         (void)mbar_wait_bounded(&empty[sl], (last / STAGES) & 1, &no_abort, args.status);
       }
   } else if (warp == 0) {
-    // idle
+    // idle, or (next-layer quantisation fused in) forming codes of the
+    // output's row blocks as they complete
+    if (ROWMAX)
+      while (codes_take_one(args, lane, abort_flag)) {
+      }
   } else if (warp == 1) {
     if (lane == 0 && rank == 0) {
       // ---------------- MMA issuer (even CTA of each pair) ----------------
@@ -336,6 +340,7 @@ __global__ void __maxnreg__(kGemmRegs)
       stage_columns<kCols>(args, n0, lane, s_ws, s_bias);
       const float as = row0 + lane < args.M ? __ldg(args.a_scale + row0 + lane) : 0.0f;
       __syncwarp();
+      if (ROWMAX) codes_while_waiting(args, lane, &tfull[b], bph);
       int ok = 0;
       if (lane == 0) ok = mbar_wait(&tfull[b], bph, abort_flag, args.status);
       ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
@@ -356,6 +361,9 @@ __global__ void __maxnreg__(kGemmRegs)
     }
     if (lane == 0) bulk_wait_group_all();  // output stores complete before exit
     __syncwarp();
+    if (ROWMAX)  // help with the codes still to form
+      while (codes_take_one(args, lane, abort_flag)) {
+      }
   }
 
   tc_fence_before();
@@ -364,6 +372,7 @@ __global__ void __maxnreg__(kGemmRegs)
     tc_fence_after();
     tmem_dealloc_pair(tmem_base, kTmemCols);
   }
+  if (ROWMAX) codes_exit(args);
 }
 
 bool g_pair_attr_done[64][4];
@@ -449,6 +458,9 @@ w8a8_status launch_gemm2sm(const int8_t *q, const float *a_scale, const void *pa
     a.row_amax = sig->row_amax;
     a.row_done = sig->row_done;
     a.done_tag = sig->tag;
+    a.q_next = sig->q_next;
+    a.a_scale_next = sig->a_scale_next;
+    a.codes_words = sig->words;
   }
   if (bn == 128)
     return sig ? run_pair<128, 4, true>(tq, tw, tw64, ty, a, stream, pdl, 3)

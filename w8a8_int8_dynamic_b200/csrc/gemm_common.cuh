@@ -10,6 +10,7 @@
 #include "act.cuh"
 #include "internal.h"
 #include "ptx.cuh"
+#include "quant_common.cuh"
 
 namespace w8a8 {
 
@@ -55,12 +56,16 @@ struct GemmArgs {
   // quantisation kernel ahead of this GEMM), and once a warp's output stores
   // for a tile are complete it adds the columns it stored to its 128-row
   // block's word in row_done ((done_tag << 32) | columns; a block is complete
-  // at 4 N).  Those instances also release their dependents at their start,
-  // so that the codes kernel behind them becomes resident and follows the
-  // blocks.
+  // at 4 N).  The kernel's own warps then form the codes q_next [M, N] and
+  // scales a_scale_next [M] of each complete block (see codes_* below);
+  // codes_words[0] hands out their work units, codes_words[1] counts the CTAs
+  // out (the last one clears the words for the next call).
   uint32_t *row_amax;
   unsigned long long *row_done;
   unsigned long long done_tag;
+  int8_t *q_next;
+  float *a_scale_next;
+  unsigned long long *codes_words;
 };
 
 // After a tile: the epilogue warp that drained rows [row0, row0 + 32) and
@@ -238,6 +243,183 @@ __device__ __forceinline__ void epilogue_i32(const GemmArgs &a, uint32_t taddr, 
 // c ^ ((r >> 1) & 3)), so the 32 lanes' 16-byte writes spread over all banks.
 constexpr int kEpiStageBytes = 32 * 32 * 2;
 constexpr int kEpiStagePerWarp = kEpiStageBytes;
+
+// ---- the next layer's codes, formed by the fused GEMM's own warps ------------
+// A unit is one row x kCodesSlice columns of the output, handled by one warp
+// (each lane kCodesCPL 16-byte chunks, all loads in flight together), with
+// the arithmetic of the quantisation kernel (quant_common.cuh) on the row's
+// maximum from row_amax.  Units are handed out in row order.  The idle warp
+// 0 takes them one after another, waiting for each row block to complete;
+// the epilogue warps take only units whose block is already complete, in the
+// gaps between their tiles, and after their last tile help with the rest.
+// Rows are read through L2 only (.cg): other CTAs of the grid write them.
+constexpr int kCodesCPL = 8;
+constexpr int kCodesSlice = 32 * kCodesCPL * 8;  // 2048 columns
+
+__device__ __forceinline__ uint4 ld_cg_u4(const void *p) {
+  uint4 v;
+  asm volatile("ld.global.cg.v4.u32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "l"(p));
+  return v;
+}
+
+__device__ __forceinline__ int codes_slices(const GemmArgs &a) {
+  return (a.N + kCodesSlice - 1) / kCodesSlice;
+}
+__device__ __forceinline__ unsigned long long codes_want(const GemmArgs &a) {
+  return (a.done_tag << 32) | (unsigned long long)(4 * a.N);
+}
+
+// Waits until *word == want (acquire), the pause between reads doubling from
+// 128 ns to 2 us: a row block completes every few microseconds, and many
+// warps wait on the same word, whose L2 slice the GEMM's own traffic also
+// uses.  The blocks are completed by CTAs of this grid, which is a single
+// wave (at most one CTA or CTA pair per SM), so the wait ends unless
+// something failed; it gives up like mbar_wait_bounded.
+static __device__ __noinline__ bool wait_block(const unsigned long long *word,
+                                               unsigned long long want,
+                                               volatile int *abort_flag, int *status) {
+  if (ld_acquire_gpu(word) == want) return true;
+  const uint64_t t0 = global_timer_ns();
+  unsigned pause = 128;
+  while (true) {
+    __nanosleep(pause);
+    if (pause < 2048) pause *= 2;
+    if (ld_acquire_gpu(word) == want) return true;
+    if (*abort_flag) return false;
+    if (global_timer_ns() - t0 > kWaitLimitNs) {
+      *abort_flag = 1;
+      atomicExch(status, (int)W8A8_ERR_TIMEOUT);
+      return false;
+    }
+  }
+}
+
+// Unit u, whose row block is complete, by the whole warp.
+__device__ __forceinline__ void codes_unit(const GemmArgs &a, uint32_t u, int lane) {
+  const int slices = codes_slices(a);
+  const int row = (int)(u / (uint32_t)slices);
+  const int slice = (int)(u - (uint32_t)row * (uint32_t)slices);
+  (void)ld_acquire_gpu(a.row_done + (row >> 7));  // this lane acquires the block's rows
+  const uint16_t *yr = static_cast<const uint16_t *>(a.out) + (int64_t)row * a.N;
+  int8_t *qr = a.q_next + (int64_t)row * a.N;
+  const int nchunks = a.N >> 3;
+  const int c0 = slice * (kCodesSlice / 8) + lane;
+  uint4 v[kCodesCPL];
+#pragma unroll
+  for (int j = 0; j < kCodesCPL; ++j) {
+    const int c = c0 + 32 * j;
+    v[j] = make_uint4(0, 0, 0, 0);
+    if (c < nchunks) v[j] = ld_cg_u4(yr + (int64_t)c * 8);
+  }
+  const float amax = __uint_as_float(__ldcg(a.row_amax + row) << 16);
+  const float s = amax == 0.0f ? 0.0f : __fdiv_rn(amax, 127.0f);
+  if (slice == 0 && lane == 0) a.a_scale_next[row] = s;
+  if (amax == 0.0f) {
+#pragma unroll
+    for (int j = 0; j < kCodesCPL; ++j) {
+      const int c = c0 + 32 * j;
+      if (c < nchunks) *reinterpret_cast<uint2 *>(qr + (int64_t)c * 8) = make_uint2(0, 0);
+    }
+  } else if (s >= 1e-30f) {
+    const float inv = __frcp_rn(s);
+#pragma unroll
+    for (int j = 0; j < kCodesCPL; ++j) {
+      const int c = c0 + 32 * j;
+      if (c < nchunks) *reinterpret_cast<uint2 *>(qr + (int64_t)c * 8) = codes8(v[j], s, inv);
+    }
+  } else {
+    // (unrolled: a runtime index into v would move it to local memory)
+#pragma unroll
+    for (int j = 0; j < kCodesCPL; ++j) {
+      const int c = c0 + 32 * j;
+      if (c < nchunks) *reinterpret_cast<uint2 *>(qr + (int64_t)c * 8) = codes8_ieee(v[j], s);
+    }
+  }
+}
+
+// Takes the next unit only if its row block is already complete (a
+// compare-and-swap on the counter, so that nothing is taken otherwise) and
+// processes it.  False: none taken.
+__device__ __forceinline__ bool codes_try_one(const GemmArgs &a, int lane) {
+  const uint32_t units = (uint32_t)a.M * (uint32_t)codes_slices(a);
+  uint32_t u = 0xFFFFFFFFu;
+  if (lane == 0) {
+    unsigned long long cur = *reinterpret_cast<volatile unsigned long long *>(a.codes_words);
+    for (int tries = 0; tries < 4; ++tries) {
+      const uint32_t n = (cur >> 32) == a.done_tag ? (uint32_t)cur : 0u;
+      if (n >= units) break;
+      const int blk = (int)(n / (uint32_t)codes_slices(a)) >> 7;
+      if (ld_acquire_gpu(a.row_done + blk) != codes_want(a)) break;
+      const unsigned long long prev =
+          atomicCAS(a.codes_words, cur, (a.done_tag << 32) | (unsigned long long)(n + 1));
+      if (prev == cur) {
+        u = n;
+        break;
+      }
+      cur = prev;
+    }
+  }
+  u = __shfl_sync(0xFFFFFFFFu, u, 0);
+  if (u == 0xFFFFFFFFu) return false;
+  codes_unit(a, u, lane);
+  return true;
+}
+
+// Takes the next unit, waits (bounded) for its row block and processes it.
+// False once every unit has been handed out, or on abort.
+__device__ __forceinline__ bool codes_take_one(const GemmArgs &a, int lane,
+                                                   volatile int *abort_flag) {
+  const uint32_t units = (uint32_t)a.M * (uint32_t)codes_slices(a);
+  uint32_t u = 0;
+  int ok = 1;
+  if (lane == 0) {
+    u = arrive_tagged32(a.codes_words, a.done_tag, 1u) - 1u;
+    if (u < units) {
+      const int blk = (int)(u / (uint32_t)codes_slices(a)) >> 7;
+      ok = wait_block(a.row_done + blk, codes_want(a), abort_flag, a.status) ? 1 : 0;
+    }
+  }
+  u = __shfl_sync(0xFFFFFFFFu, u, 0);
+  ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
+  if (u >= units || !ok) return false;
+  codes_unit(a, u, lane);
+  return true;
+}
+
+// An epilogue warp about to wait for its next tile's accumulators forms codes
+// of complete row blocks while they are not ready yet.
+__device__ __forceinline__ void codes_while_waiting(const GemmArgs &a, int lane, uint64_t *tfull,
+                                                    uint32_t parity) {
+  while (true) {
+    int ready = 0;
+    if (lane == 0) ready = mbar_try_wait(smem_addr(tfull), parity) ? 1 : 0;
+    ready = __shfl_sync(0xFFFFFFFFu, ready, 0);
+    if (ready || !codes_try_one(a, lane)) return;
+  }
+}
+
+// After the CTA's last barrier: thread 0 counts the CTA out; the last CTA of
+// the grid clears the counter and the block words (every CTA is past its
+// waits), so that a replayed CUDA graph, which keeps the tag, starts from
+// zero.
+__device__ __forceinline__ void codes_exit(const GemmArgs &a) {
+  __shared__ int last_cta;
+  if (threadIdx.x == 0) {
+    __threadfence();
+    last_cta = arrive_tagged32(a.codes_words + 1, a.done_tag, 1u) == gridDim.x ? 1 : 0;
+  }
+  __syncthreads();
+  if (last_cta) {
+    const int nblk = (a.M + 127) >> 7;
+    for (int b = threadIdx.x; b < nblk; b += blockDim.x) a.row_done[b] = 0ull;
+    if (threadIdx.x == 0) {
+      a.codes_words[0] = 0ull;
+      a.codes_words[1] = 0ull;
+    }
+  }
+}
 
 // The two packed 16-bit magnitudes of epilogue_tma's rmax -> one bf16
 // magnitude bit pattern (finite bf16 order by magnitude = order of these bits).

@@ -78,11 +78,15 @@ inline int64_t packed_cols(int64_t K) { return round_up(K, 128); }
 // GEMM launchers (gemm.cu).
 // The next layer's quantisation fused with a GEMM (see GemmArgs::row_amax):
 // per-row maxima (zeroed by the quantisation kernel ahead of the GEMM), per
-// 128-row block call-tagged completion words, and the call's tag.
+// 128-row block call-tagged completion words, the call's tag, the codes and
+// scales to form, and two words: the work counter and the exit count.
 struct RowSignal {
   uint32_t *row_amax;
   unsigned long long *row_done;
   unsigned long long tag;
+  int8_t *q_next;
+  float *a_scale_next;
+  unsigned long long *words;
 };
 // pdl: a programmatic dependent of the preceding kernel; prefetch: (1-SM
 // kernel) warm L2 with weights while waiting behind the quantisation kernel.
@@ -114,14 +118,6 @@ w8a8_status launch_decode(const int8_t *q, const float *a_scale, const void *pac
 w8a8_status launch_quant(const void *x, int64_t M, int64_t K, int64_t ldx, int8_t *q,
                          float *a_scale, cudaStream_t stream, bool ahead_of_gemm,
                          uint32_t *zero_rows = nullptr);
-// The codes kernel of the fused next-layer quantisation (quant.cu): the codes
-// and scales of y [M, N] from the row maxima, each 128-row block once its
-// row_done word reads (tag, 4 N); words[0] hands out the work units,
-// words[1] counts the CTAs out.
-w8a8_status launch_codes(const void *y, int64_t M, int64_t N, const uint32_t *row_amax,
-                         unsigned long long *row_done, unsigned long long tag, int8_t *q,
-                         float *a_scale, unsigned long long *words, cudaStream_t stream);
-// Work units of the codes kernel (must stay below 2^32).
-int64_t codes_units(int64_t M, int64_t N);
+
 
 }  // namespace w8a8

@@ -29,13 +29,7 @@
 //
 // The per-element arithmetic (the code from one step of reciprocal
 // refinement, rint by one addition) is in quant_common.cuh.
-//
-// quant_codes_kernel quantises the output of a layer whose GEMM epilogue has
-// already folded every row's maximum magnitude (the next layer's activation
-// quantisation fused with this one): it runs beside that GEMM and takes each
-// 128-row block as soon as the GEMM reports it complete, reading the rows
-// back while they are still in L2.  Same scale and codes as the kernels
-// above, from the same row maximum.
+
 #include <cuda_bf16.h>
 
 #include <algorithm>
@@ -168,143 +162,6 @@ __global__ void __launch_bounds__(1024) quant_rows_two_pass_kernel(
       out = exact_only ? codes8_ieee(c, s) : codes8(c, s, inv);
     }
     *reinterpret_cast<uint2 *>(qr + (int64_t)i * 8) = out;
-  }
-}
-
-// ---- codes of a GEMM's output whose row maxima its epilogue folded ----------
-// A unit is one row x kCodesSlice columns, handled by one warp (each lane
-// kCodesCPL 16-byte chunks, all loads in flight together).  Warps take units
-// in row order from a call-tagged counter, the next one asked for before the
-// current one is processed, so that whichever warps are resident beside the
-// GEMM share the work as its row blocks complete, and a CTA that only
-// becomes resident after the GEMM finds the work done.  Rows are read
-// through L2 only (.cg): the GEMM beside this kernel writes them.  The last
-// CTA to finish clears the counter and the block words, so that a replayed
-// CUDA graph (same tag) finds them at zero.
-constexpr int kCodesCPL = 8;
-constexpr int kCodesSlice = 32 * kCodesCPL * 8;  // 2048 columns
-constexpr int kCodesWarps = 4;
-
-__device__ __forceinline__ uint4 ld_cg_u4(const void *p) {
-  uint4 v;
-  asm volatile("ld.global.cg.v4.u32 {%0, %1, %2, %3}, [%4];"
-               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-               : "l"(p));
-  return v;
-}
-
-// Waits until *word == want (acquire), polling every 256 ns (a block
-// completes every few microseconds).  The words are written by the GEMM this
-// kernel follows, every CTA of which has started before this kernel is
-// launched, so the wait ends unless something failed; it gives up like
-// mbar_wait_bounded: on *abort_flag, or after kWaitLimitNs (then it sets
-// *abort_flag and records W8A8_ERR_TIMEOUT).
-__device__ __noinline__ bool wait_block(const unsigned long long *word, unsigned long long want,
-                                        volatile int *abort_flag, int *status) {
-  if (ld_acquire_gpu(word) == want) return true;
-  const uint64_t t0 = global_timer_ns();
-  while (true) {
-    __nanosleep(256);
-    if (ld_acquire_gpu(word) == want) return true;
-    if (*abort_flag) return false;
-    if (global_timer_ns() - t0 > kWaitLimitNs) {
-      *abort_flag = 1;
-      atomicExch(status, (int)W8A8_ERR_TIMEOUT);
-      return false;
-    }
-  }
-}
-
-// At most 64 registers: two 4-warp CTAs fit beside a GEMM CTA of 128
-// registers a thread (its 11 warps leave 4,096 registers on each of three SM
-// sub-partitions and more on the fourth).
-__global__ void __maxnreg__(64) quant_codes_kernel(
-    const uint16_t *__restrict__ y, int M, int N, const uint32_t *row_amax,
-    unsigned long long *row_done, unsigned long long tag, unsigned long long target,
-    int8_t *__restrict__ q, float *__restrict__ a_scale, unsigned long long *words,
-    int *status) {
-  // The next layer's GEMM may take each SM as the GEMM beside this kernel
-  // leaves it; it waits on the device for this kernel to complete.
-  griddep_launch_dependents();
-  __shared__ int abort_flag;
-  __shared__ int last_cta;
-  if (threadIdx.x == 0) abort_flag = 0;
-  __syncthreads();
-  unsigned long long *next_unit = words;  // (tag << 32) | units handed out
-  unsigned long long *exit_word = words + 1;
-  const int lane = threadIdx.x & 31;
-  const int slices = (N + kCodesSlice - 1) / kCodesSlice;
-  const int nchunks = N >> 3;
-  const uint32_t units = (uint32_t)M * (uint32_t)slices;
-  const unsigned long long want = (tag << 32) | target;
-  int ready = -1;  // the last row block this warp saw complete
-  uint32_t u = 0;
-  if (lane == 0) u = arrive_tagged32(next_unit, tag, 1u) - 1u;
-  u = __shfl_sync(0xFFFFFFFFu, u, 0);
-  while (u < units) {
-    uint32_t nu = 0;
-    if (lane == 0) nu = arrive_tagged32(next_unit, tag, 1u) - 1u;  // in flight meanwhile
-    const int row = (int)(u / (uint32_t)slices);
-    const int slice = (int)(u - (uint32_t)row * (uint32_t)slices);
-    const int blk = row >> 7;
-    if (blk != ready) {
-      int ok = 1;
-      if (lane == 0) ok = wait_block(row_done + blk, want, &abort_flag, status) ? 1 : 0;
-      ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
-      if (!ok) break;
-      (void)ld_acquire_gpu(row_done + blk);  // every lane acquires the block's rows
-      ready = blk;
-    }
-    const uint16_t *yr = y + (int64_t)row * N;
-    int8_t *qr = q + (int64_t)row * N;
-    const int c0 = slice * (kCodesSlice / 8) + lane;
-    uint4 v[kCodesCPL];
-#pragma unroll
-    for (int j = 0; j < kCodesCPL; ++j) {
-      const int c = c0 + 32 * j;
-      v[j] = make_uint4(0, 0, 0, 0);
-      if (c < nchunks) v[j] = ld_cg_u4(yr + (int64_t)c * 8);
-    }
-    const float amax = __uint_as_float(__ldcg(row_amax + row) << 16);
-    const float s = amax == 0.0f ? 0.0f : __fdiv_rn(amax, 127.0f);
-    if (slice == 0 && lane == 0) a_scale[row] = s;
-    if (amax == 0.0f) {
-#pragma unroll
-      for (int j = 0; j < kCodesCPL; ++j) {
-        const int c = c0 + 32 * j;
-        if (c < nchunks) *reinterpret_cast<uint2 *>(qr + (int64_t)c * 8) = make_uint2(0, 0);
-      }
-    } else if (s >= 1e-30f) {
-      const float inv = __frcp_rn(s);
-#pragma unroll
-      for (int j = 0; j < kCodesCPL; ++j) {
-        const int c = c0 + 32 * j;
-        if (c < nchunks) *reinterpret_cast<uint2 *>(qr + (int64_t)c * 8) = codes8(v[j], s, inv);
-      }
-    } else {
-      // (unrolled: a runtime index into v would move it to local memory)
-#pragma unroll
-      for (int j = 0; j < kCodesCPL; ++j) {
-        const int c = c0 + 32 * j;
-        if (c < nchunks) *reinterpret_cast<uint2 *>(qr + (int64_t)c * 8) = codes8_ieee(v[j], s);
-      }
-    }
-    u = __shfl_sync(0xFFFFFFFFu, nu, 0);
-  }
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    __threadfence();
-    last_cta = arrive_tagged32(exit_word, tag, 1u) == gridDim.x ? 1 : 0;
-  }
-  __syncthreads();
-  if (last_cta) {
-    // every CTA is past its waits and grabs: clear the words for the next call
-    const int nblk = (M + 127) >> 7;
-    for (int b = threadIdx.x; b < nblk; b += blockDim.x) row_done[b] = 0ull;
-    if (threadIdx.x == 0) {
-      *next_unit = 0ull;
-      *exit_word = 0ull;
-    }
   }
 }
 
@@ -477,26 +334,6 @@ w8a8_status launch_quant(const void *x, int64_t M, int64_t K, int64_t ldx, int8_
         return W8A8_ERR_INVALID_ARG;
     }
   }
-  if (e != cudaSuccess) return from_cuda(e);
-  count_launch();
-  return from_cuda(cudaGetLastError());
-}
-
-int64_t codes_units(int64_t M, int64_t N) { return M * ((N + kCodesSlice - 1) / kCodesSlice); }
-
-w8a8_status launch_codes(const void *y, int64_t M, int64_t N, const uint32_t *row_amax,
-                         unsigned long long *row_done, unsigned long long tag, int8_t *q,
-                         float *a_scale, unsigned long long *words, cudaStream_t stream) {
-  int *status = status_word();
-  if (!status) return W8A8_ERR_CUDA;
-  const int64_t units = codes_units(M, N);
-  // two 4-warp CTAs an SM fit beside a GEMM CTA
-  const int64_t grid = std::max<int64_t>(
-      1, std::min<int64_t>((units + kCodesWarps - 1) / kCodesWarps, 2 * (int64_t)sm_count()));
-  const cudaError_t e = launch_dependent(
-      quant_codes_kernel, 5, dim3((unsigned)grid), dim3(32 * kCodesWarps), stream,
-      static_cast<const uint16_t *>(y), (int)M, (int)N, row_amax, row_done, tag,
-      (unsigned long long)(4 * N), q, a_scale, words, status);
   if (e != cudaSuccess) return from_cuda(e);
   count_launch();
   return from_cuda(cudaGetLastError());
