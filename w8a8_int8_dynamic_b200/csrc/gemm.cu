@@ -244,9 +244,11 @@ __global__ void __maxnreg__(kGemmRegs)
   } else if (warp == 0) {
     // idle, or (next-layer quantisation fused in) forming codes of the
     // output's row blocks as they complete
-    if (ROWMAX)
-      while (codes_take_one(args, lane, abort_flag)) {
+    if (ROWMAX) {
+      int cursor = 0;
+      while (codes_one(args, lane, cursor, true, abort_flag)) {
       }
+    }
   } else if (warp == 1) {
     if (lane == 0) {
       // ---------------- MMA issuer ----------------
@@ -303,6 +305,7 @@ __global__ void __maxnreg__(kGemmRegs)
     float *s_ws = reinterpret_cast<float *>(smem + L::kEpi + (warp - 2) * L::kEpiPerWarp);
     uint16_t *s_bias = reinterpret_cast<uint16_t *>(s_ws + kCols);
     uint8_t *s_out = smem + L::kOut + (warp - 2) * kEpiStagePerWarp;
+    int cursor = 0;  // (ROWMAX) the lowest row block not seen exhausted of codes work
     for (int t = 0; t < my_tiles; ++t) {
       const int tile = blockIdx.x + t * gridDim.x;
       int mb, nb;
@@ -317,7 +320,7 @@ __global__ void __maxnreg__(kGemmRegs)
         if (row0 + lane < args.M) as = __ldg(args.a_scale + row0 + lane);
       }
       __syncwarp();
-      if (ROWMAX) codes_while_waiting(args, lane, &tfull[b], bph);
+      if (ROWMAX) codes_while_waiting(args, lane, cursor, &tfull[b], bph);
       int ok = 0;
       if (lane == 0) ok = mbar_wait(&tfull[b], bph, abort_flag, args.status);
       ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
@@ -340,7 +343,7 @@ __global__ void __maxnreg__(kGemmRegs)
     if (lane == 0) bulk_wait_group_all();  // output stores complete before exit
     __syncwarp();
     if (ROWMAX)  // help with the codes still to form
-      while (codes_take_one(args, lane, abort_flag)) {
+      while (codes_one(args, lane, cursor, true, abort_flag)) {
       }
   }
 
@@ -499,7 +502,8 @@ w8a8_status launch_scaled_mm(const int8_t *q, const float *a_scale, const void *
     a.done_tag = sig->tag;
     a.q_next = sig->q_next;
     a.a_scale_next = sig->a_scale_next;
-    a.codes_words = sig->words;
+    a.unit_ctr = sig->unit_ctr;
+    a.exit_word = sig->exit_word;
   }
   CUtensorMap tmap_y;
   if (out_i32) {
@@ -532,8 +536,9 @@ w8a8_status launch_scaled_mm(const int8_t *q, const float *a_scale, const void *
 // count, 4 N, stays in 32 bits).
 constexpr int64_t kMaxFusedN = (int64_t)1 << 28;
 
-// Workspace of w8a8_linear_act_quant: as w8a8_linear's, then (large M) the
-// row maxima, one completion word per 128-row block and one exit word.
+// Workspace of w8a8_linear_act_quant: as w8a8_linear's, then the row maxima,
+// one completion word and one work counter per 128-row block, and an exit
+// word.
 int64_t act_quant_workspace_bytes(int64_t M, int64_t N, int64_t K);
 
 // Workspace of w8a8_linear: the codes, the scales and (small M) the split-K
@@ -546,7 +551,7 @@ int64_t linear_workspace_bytes(int64_t M, int64_t N, int64_t K) {
 
 int64_t act_quant_workspace_bytes(int64_t M, int64_t N, int64_t K) {
   return linear_workspace_bytes(M, N, K) + round_up(M * 4, 256) +
-         round_up(((M + 127) / 128) * 8, 256) + 256;
+         2 * round_up(((M + 127) / 128) * 8, 256) + 256;
 }
 
 static w8a8_status check_gemm_args(const void *q, const void *packed_w, const void *out,
@@ -709,8 +714,11 @@ w8a8_status w8a8_linear_act_quant(const void *x, int64_t ldx, const void *packed
   off += round_up(M * 4, 256);
   unsigned long long *row_done = reinterpret_cast<unsigned long long *>(ws + off);
   off += round_up(((M + 127) / 128) * 8, 256);
-  unsigned long long *words = reinterpret_cast<unsigned long long *>(ws + off);  // [2]
-  RowSignal sig{row_amax, row_done, next_call_tag() & 0xFFFFFFFFull, q_next, a_scale_next, words};
+  unsigned long long *unit_ctr = reinterpret_cast<unsigned long long *>(ws + off);
+  off += round_up(((M + 127) / 128) * 8, 256);
+  unsigned long long *exit_word = reinterpret_cast<unsigned long long *>(ws + off);
+  RowSignal sig{row_amax,     row_done, next_call_tag() & 0xFFFFFFFFull, q_next,
+                a_scale_next, unit_ctr, exit_word};
   if (sig.tag == 0) sig.tag = 1;
   st = launch_quant(x, M, K, ldx, q, a_scale, s, true, row_amax);
   if (st != W8A8_OK) return st;

@@ -265,9 +265,11 @@ __global__ void __maxnreg__(kGemmRegs)
   } else if (warp == 0) {
     // idle, or (next-layer quantisation fused in) forming codes of the
     // output's row blocks as they complete
-    if (ROWMAX)
-      while (codes_take_one(args, lane, abort_flag)) {
+    if (ROWMAX) {
+      int cursor = 0;
+      while (codes_one(args, lane, cursor, true, abort_flag)) {
       }
+    }
   } else if (warp == 1) {
     if (lane == 0 && rank == 0) {
       // ---------------- MMA issuer (even CTA of each pair) ----------------
@@ -327,6 +329,7 @@ __global__ void __maxnreg__(kGemmRegs)
     uint16_t *s_bias = reinterpret_cast<uint16_t *>(s_ws + kCols);
     uint8_t *s_out = smem + L::kOut + (warp - 2) * kEpiStagePerWarp;
     const int j0 = ew.half * kCols;  // first tile column of this warp
+    int cursor = 0;  // (ROWMAX) the lowest row block not seen exhausted of codes work
     for (int i = 0; i < nseg; ++i) {
       const int tile = item_tile(seg_tile(i)), half = item_half(seg_tile(i));
       int mb, nb;
@@ -340,7 +343,7 @@ __global__ void __maxnreg__(kGemmRegs)
       stage_columns<kCols>(args, n0, lane, s_ws, s_bias);
       const float as = row0 + lane < args.M ? __ldg(args.a_scale + row0 + lane) : 0.0f;
       __syncwarp();
-      if (ROWMAX) codes_while_waiting(args, lane, &tfull[b], bph);
+      if (ROWMAX) codes_while_waiting(args, lane, cursor, &tfull[b], bph);
       int ok = 0;
       if (lane == 0) ok = mbar_wait(&tfull[b], bph, abort_flag, args.status);
       ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
@@ -362,7 +365,7 @@ __global__ void __maxnreg__(kGemmRegs)
     if (lane == 0) bulk_wait_group_all();  // output stores complete before exit
     __syncwarp();
     if (ROWMAX)  // help with the codes still to form
-      while (codes_take_one(args, lane, abort_flag)) {
+      while (codes_one(args, lane, cursor, true, abort_flag)) {
       }
   }
 
@@ -460,7 +463,8 @@ w8a8_status launch_gemm2sm(const int8_t *q, const float *a_scale, const void *pa
     a.done_tag = sig->tag;
     a.q_next = sig->q_next;
     a.a_scale_next = sig->a_scale_next;
-    a.codes_words = sig->words;
+    a.unit_ctr = sig->unit_ctr;
+    a.exit_word = sig->exit_word;
   }
   if (bn == 128)
     return sig ? run_pair<128, 4, true>(tq, tw, tw64, ty, a, stream, pdl, 3)

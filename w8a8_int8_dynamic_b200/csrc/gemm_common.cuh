@@ -57,15 +57,17 @@ struct GemmArgs {
   // for a tile are complete it adds the columns it stored to its 128-row
   // block's word in row_done ((done_tag << 32) | columns; a block is complete
   // at 4 N).  The kernel's own warps then form the codes q_next [M, N] and
-  // scales a_scale_next [M] of each complete block (see codes_* below);
-  // codes_words[0] hands out their work units, codes_words[1] counts the CTAs
-  // out (the last one clears the words for the next call).
+  // scales a_scale_next [M] of each complete block (see codes_* below):
+  // unit_ctr holds one call-tagged counter per 128-row block that hands out
+  // its work units, exit_word counts the CTAs out (the last one clears the
+  // words for the next call).
   uint32_t *row_amax;
   unsigned long long *row_done;
   unsigned long long done_tag;
   int8_t *q_next;
   float *a_scale_next;
-  unsigned long long *codes_words;
+  unsigned long long *unit_ctr;
+  unsigned long long *exit_word;
 };
 
 // After a tile: the epilogue warp that drained rows [row0, row0 + 32) and
@@ -248,11 +250,15 @@ constexpr int kEpiStagePerWarp = kEpiStageBytes;
 // A unit is one row x kCodesSlice columns of the output, handled by one warp
 // (each lane kCodesCPL 16-byte chunks, all loads in flight together), with
 // the arithmetic of the quantisation kernel (quant_common.cuh) on the row's
-// maximum from row_amax.  Units are handed out in row order.  The idle warp
-// 0 takes them one after another, waiting for each row block to complete;
-// the epilogue warps take only units whose block is already complete, in the
-// gaps between their tiles, and after their last tile help with the rest.
-// Rows are read through L2 only (.cg): other CTAs of the grid write them.
+// maximum from row_amax.  Each 128-row block hands out its units from a
+// counter of its own: one counter for all units would see every grab of
+// every warp (tens of thousands of atomics on one address, serialised in
+// one L2 slice, tens of microseconds).  A warp keeps a cursor on the lowest
+// block it has not yet seen exhausted.  The idle warp 0 takes units one
+// after another, waiting for each block to complete; the epilogue warps take
+// only units of complete blocks, in the gaps between their tiles, and after
+// their last tile help with the rest.  Rows are read through L2 only (.cg):
+// other CTAs of the grid write them.
 constexpr int kCodesCPL = 8;
 constexpr int kCodesSlice = 32 * kCodesCPL * 8;  // 2048 columns
 
@@ -269,6 +275,10 @@ __device__ __forceinline__ int codes_slices(const GemmArgs &a) {
 }
 __device__ __forceinline__ unsigned long long codes_want(const GemmArgs &a) {
   return (a.done_tag << 32) | (unsigned long long)(4 * a.N);
+}
+// Units of row block b (its rows below M, times the slices of a row).
+__device__ __forceinline__ uint32_t codes_block_units(const GemmArgs &a, int b) {
+  return (uint32_t)min(128, a.M - b * 128) * (uint32_t)codes_slices(a);
 }
 
 // Waits until *word == want (acquire), the pause between reads doubling from
@@ -296,12 +306,12 @@ static __device__ __noinline__ bool wait_block(const unsigned long long *word,
   }
 }
 
-// Unit u, whose row block is complete, by the whole warp.
-__device__ __forceinline__ void codes_unit(const GemmArgs &a, uint32_t u, int lane) {
+// Unit u of complete row block b, by the whole warp.
+__device__ __forceinline__ void codes_unit(const GemmArgs &a, int b, uint32_t u, int lane) {
   const int slices = codes_slices(a);
-  const int row = (int)(u / (uint32_t)slices);
-  const int slice = (int)(u - (uint32_t)row * (uint32_t)slices);
-  (void)ld_acquire_gpu(a.row_done + (row >> 7));  // this lane acquires the block's rows
+  const int row = b * 128 + (int)(u / (uint32_t)slices);
+  const int slice = (int)(u % (uint32_t)slices);
+  (void)ld_acquire_gpu(a.row_done + b);  // this lane acquires the block's rows
   const uint16_t *yr = static_cast<const uint16_t *>(a.out) + (int64_t)row * a.N;
   int8_t *qr = a.q_next + (int64_t)row * a.N;
   const int nchunks = a.N >> 3;
@@ -339,85 +349,79 @@ __device__ __forceinline__ void codes_unit(const GemmArgs &a, uint32_t u, int la
   }
 }
 
-// Takes the next unit only if its row block is already complete (a
-// compare-and-swap on the counter, so that nothing is taken otherwise) and
-// processes it.  False: none taken.
-__device__ __forceinline__ bool codes_try_one(const GemmArgs &a, int lane) {
-  const uint32_t units = (uint32_t)a.M * (uint32_t)codes_slices(a);
-  uint32_t u = 0xFFFFFFFFu;
-  if (lane == 0) {
-    unsigned long long cur = *reinterpret_cast<volatile unsigned long long *>(a.codes_words);
-    for (int tries = 0; tries < 4; ++tries) {
-      const uint32_t n = (cur >> 32) == a.done_tag ? (uint32_t)cur : 0u;
-      if (n >= units) break;
-      const int blk = (int)(n / (uint32_t)codes_slices(a)) >> 7;
-      if (ld_acquire_gpu(a.row_done + blk) != codes_want(a)) break;
-      const unsigned long long prev =
-          atomicCAS(a.codes_words, cur, (a.done_tag << 32) | (unsigned long long)(n + 1));
-      if (prev == cur) {
-        u = n;
-        break;
-      }
-      cur = prev;
-    }
-  }
-  u = __shfl_sync(0xFFFFFFFFu, u, 0);
-  if (u == 0xFFFFFFFFu) return false;
-  codes_unit(a, u, lane);
-  return true;
+// Lane 0: whether block b's counter (call-tagged) has handed out all units.
+__device__ __forceinline__ bool codes_block_exhausted(const GemmArgs &a, int b) {
+  const unsigned long long cur = *reinterpret_cast<volatile unsigned long long *>(a.unit_ctr + b);
+  return (cur >> 32) == a.done_tag && (uint32_t)cur >= codes_block_units(a, b);
 }
 
-// Takes the next unit, waits (bounded) for its row block and processes it.
-// False once every unit has been handed out, or on abort.
-__device__ __forceinline__ bool codes_take_one(const GemmArgs &a, int lane,
-                                                   volatile int *abort_flag) {
-  const uint32_t units = (uint32_t)a.M * (uint32_t)codes_slices(a);
-  uint32_t u = 0;
-  int ok = 1;
+// Takes and processes one unit.  `cursor` (uniform across the warp) is the
+// lowest block this warp has not seen exhausted.  blocking: wait (bounded)
+// for the block to complete; otherwise take a unit only from a block that
+// is already complete.  False: nothing taken (blocking: no units left, or
+// abort).
+__device__ __forceinline__ bool codes_one(const GemmArgs &a, int lane, int &cursor, bool blocking,
+                                          volatile int *abort_flag) {
+  const int nblk = (a.M + 127) >> 7;
+  int b = cursor;
+  uint32_t u = 0xFFFFFFFFu;
   if (lane == 0) {
-    u = arrive_tagged32(a.codes_words, a.done_tag, 1u) - 1u;
-    if (u < units) {
-      const int blk = (int)(u / (uint32_t)codes_slices(a)) >> 7;
-      ok = wait_block(a.row_done + blk, codes_want(a), abort_flag, a.status) ? 1 : 0;
+    while (b < nblk) {
+      if (codes_block_exhausted(a, b)) {
+        ++b;
+        continue;
+      }
+      if (!blocking && ld_acquire_gpu(a.row_done + b) != codes_want(a)) break;
+      const uint32_t got = arrive_tagged32(a.unit_ctr + b, a.done_tag, 1u) - 1u;
+      if (got >= codes_block_units(a, b)) {  // taken by others meanwhile
+        ++b;
+        continue;
+      }
+      if (blocking && !wait_block(a.row_done + b, codes_want(a), abort_flag, a.status)) {
+        b = nblk;  // abort: stop
+        break;
+      }
+      u = got;
+      break;
     }
   }
+  cursor = __shfl_sync(0xFFFFFFFFu, b, 0);
   u = __shfl_sync(0xFFFFFFFFu, u, 0);
-  ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
-  if (u >= units || !ok) return false;
-  codes_unit(a, u, lane);
+  if (u == 0xFFFFFFFFu) return false;
+  codes_unit(a, cursor, u, lane);
   return true;
 }
 
 // An epilogue warp about to wait for its next tile's accumulators forms codes
 // of complete row blocks while they are not ready yet.
-__device__ __forceinline__ void codes_while_waiting(const GemmArgs &a, int lane, uint64_t *tfull,
-                                                    uint32_t parity) {
+__device__ __forceinline__ void codes_while_waiting(const GemmArgs &a, int lane, int &cursor,
+                                                    uint64_t *tfull, uint32_t parity) {
   while (true) {
     int ready = 0;
     if (lane == 0) ready = mbar_try_wait(smem_addr(tfull), parity) ? 1 : 0;
     ready = __shfl_sync(0xFFFFFFFFu, ready, 0);
-    if (ready || !codes_try_one(a, lane)) return;
+    if (ready || !codes_one(a, lane, cursor, false, nullptr)) return;
   }
 }
 
 // After the CTA's last barrier: thread 0 counts the CTA out; the last CTA of
-// the grid clears the counter and the block words (every CTA is past its
+// the grid clears the counters and the block words (every CTA is past its
 // waits), so that a replayed CUDA graph, which keeps the tag, starts from
 // zero.
 __device__ __forceinline__ void codes_exit(const GemmArgs &a) {
   __shared__ int last_cta;
   if (threadIdx.x == 0) {
     __threadfence();
-    last_cta = arrive_tagged32(a.codes_words + 1, a.done_tag, 1u) == gridDim.x ? 1 : 0;
+    last_cta = arrive_tagged32(a.exit_word, a.done_tag, 1u) == gridDim.x ? 1 : 0;
   }
   __syncthreads();
   if (last_cta) {
     const int nblk = (a.M + 127) >> 7;
-    for (int b = threadIdx.x; b < nblk; b += blockDim.x) a.row_done[b] = 0ull;
-    if (threadIdx.x == 0) {
-      a.codes_words[0] = 0ull;
-      a.codes_words[1] = 0ull;
+    for (int b = threadIdx.x; b < nblk; b += blockDim.x) {
+      a.row_done[b] = 0ull;
+      a.unit_ctr[b] = 0ull;
     }
+    if (threadIdx.x == 0) *a.exit_word = 0ull;
   }
 }
 
