@@ -311,7 +311,13 @@ w8a8_status w8a8_gelu_tanh(const void *x, void *y, int64_t n,
 /* ---- errors ----------------------------------------------------------------
  * Synchronises `stream`, then returns and clears the device status word of
  * the current device: W8A8_ERR_TIMEOUT if any kernel gave up on a wait since
- * the last poll, W8A8_ERR_CUDA on an asynchronous CUDA error, else W8A8_OK. */
+ * the last poll, W8A8_ERR_CUDA on an asynchronous CUDA error, else W8A8_OK.
+ * After W8A8_ERR_TIMEOUT the outputs of the calls since the last poll are
+ * invalid, and the call-tagged words in their workspaces (the small-M
+ * kernel's slab counters, the fused next-layer quantisation's block words)
+ * may be left mid-count.  A direct call draws a new tag and ignores them; a
+ * captured CUDA graph replays its calls with the tags it was captured with,
+ * so capture it again before replaying it. */
 w8a8_status w8a8_poll_status(w8a8_stream_t stream);
 
 /* Self-test of the bounded-wait path: launches one block that waits on a
