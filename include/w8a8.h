@@ -245,11 +245,10 @@ w8a8_status w8a8_linear_act(const void *x, int64_t ldx, const void *packed_w,
  *   q_next       device, int8 [M, N] dense (output): the codes of y
  *   a_scale_next device, fp32 [M] (output): their per-row scales
  *   workspace    device, ws_bytes >= w8a8_linear_act_quant_workspace_bytes(M,
- *                N, K): w8a8_linear's workspace, then the row maxima, and
- *                per 128-row block a call-tagged completion word and a
- *                counter that hands out the codes' work (contents on entry
- *                do not matter; the last CTA of each call clears the words,
- *                so a replayed CUDA graph finds them at zero)
+ *                N, K): w8a8_linear's workspace, then the row maxima and one
+ *                call-tagged completion word per 128-row block (contents on
+ *                entry do not matter; the last CTA of each call clears the
+ *                words, so a replayed CUDA graph finds them at zero)
  * Limits as w8a8_linear, plus N % 16 == 0 (q_next is the next layer's GEMM
  * input, whose K = N) and N <= 2^28.  After a call that timed out
  * (W8A8_ERR_TIMEOUT) the words may be left set: capture CUDA graphs of this

@@ -245,8 +245,8 @@ __global__ void __maxnreg__(kGemmRegs)
     // idle, or (next-layer quantisation fused in) forming codes of the
     // output's row blocks as they complete
     if (ROWMAX) {
-      int cursor = 0;
-      while (codes_one(args, lane, cursor, true, abort_flag)) {
+      CodesCursor cursor = codes_cursor(args, 0);
+      while (codes_next(args, lane, cursor, true, abort_flag)) {
       }
     }
   } else if (warp == 1) {
@@ -305,7 +305,7 @@ __global__ void __maxnreg__(kGemmRegs)
     float *s_ws = reinterpret_cast<float *>(smem + L::kEpi + (warp - 2) * L::kEpiPerWarp);
     uint16_t *s_bias = reinterpret_cast<uint16_t *>(s_ws + kCols);
     uint8_t *s_out = smem + L::kOut + (warp - 2) * kEpiStagePerWarp;
-    int cursor = 0;  // (ROWMAX) the lowest row block not seen exhausted of codes work
+    CodesCursor cursor = codes_cursor(args, warp - 1);  // (ROWMAX) this warp's codes units
     for (int t = 0; t < my_tiles; ++t) {
       const int tile = blockIdx.x + t * gridDim.x;
       int mb, nb;
@@ -343,7 +343,7 @@ __global__ void __maxnreg__(kGemmRegs)
     if (lane == 0) bulk_wait_group_all();  // output stores complete before exit
     __syncwarp();
     if (ROWMAX)  // help with the codes still to form
-      while (codes_one(args, lane, cursor, true, abort_flag)) {
+      while (codes_next(args, lane, cursor, true, abort_flag)) {
       }
   }
 
@@ -502,7 +502,6 @@ w8a8_status launch_scaled_mm(const int8_t *q, const float *a_scale, const void *
     a.done_tag = sig->tag;
     a.q_next = sig->q_next;
     a.a_scale_next = sig->a_scale_next;
-    a.unit_ctr = sig->unit_ctr;
     a.exit_word = sig->exit_word;
   }
   CUtensorMap tmap_y;
@@ -537,8 +536,7 @@ w8a8_status launch_scaled_mm(const int8_t *q, const float *a_scale, const void *
 constexpr int64_t kMaxFusedN = (int64_t)1 << 28;
 
 // Workspace of w8a8_linear_act_quant: as w8a8_linear's, then the row maxima,
-// one completion word and one work counter per 128-row block, and an exit
-// word.
+// one completion word per 128-row block, and an exit word.
 int64_t act_quant_workspace_bytes(int64_t M, int64_t N, int64_t K);
 
 // Workspace of w8a8_linear: the codes, the scales and (small M) the split-K
@@ -551,7 +549,7 @@ int64_t linear_workspace_bytes(int64_t M, int64_t N, int64_t K) {
 
 int64_t act_quant_workspace_bytes(int64_t M, int64_t N, int64_t K) {
   return linear_workspace_bytes(M, N, K) + round_up(M * 4, 256) +
-         2 * round_up(((M + 127) / 128) * 8, 256) + 256;
+         round_up(((M + 127) / 128) * 8, 256) + 256;
 }
 
 static w8a8_status check_gemm_args(const void *q, const void *packed_w, const void *out,
@@ -714,11 +712,9 @@ w8a8_status w8a8_linear_act_quant(const void *x, int64_t ldx, const void *packed
   off += round_up(M * 4, 256);
   unsigned long long *row_done = reinterpret_cast<unsigned long long *>(ws + off);
   off += round_up(((M + 127) / 128) * 8, 256);
-  unsigned long long *unit_ctr = reinterpret_cast<unsigned long long *>(ws + off);
-  off += round_up(((M + 127) / 128) * 8, 256);
   unsigned long long *exit_word = reinterpret_cast<unsigned long long *>(ws + off);
-  RowSignal sig{row_amax,     row_done, next_call_tag() & 0xFFFFFFFFull, q_next,
-                a_scale_next, unit_ctr, exit_word};
+  RowSignal sig{row_amax, row_done, next_call_tag() & 0xFFFFFFFFull, q_next, a_scale_next,
+                exit_word};
   if (sig.tag == 0) sig.tag = 1;
   st = launch_quant(x, M, K, ldx, q, a_scale, s, true, row_amax);
   if (st != W8A8_OK) return st;

@@ -266,8 +266,8 @@ __global__ void __maxnreg__(kGemmRegs)
     // idle, or (next-layer quantisation fused in) forming codes of the
     // output's row blocks as they complete
     if (ROWMAX) {
-      int cursor = 0;
-      while (codes_one(args, lane, cursor, true, abort_flag)) {
+      CodesCursor cursor = codes_cursor(args, 0);
+      while (codes_next(args, lane, cursor, true, abort_flag)) {
       }
     }
   } else if (warp == 1) {
@@ -329,7 +329,7 @@ __global__ void __maxnreg__(kGemmRegs)
     uint16_t *s_bias = reinterpret_cast<uint16_t *>(s_ws + kCols);
     uint8_t *s_out = smem + L::kOut + (warp - 2) * kEpiStagePerWarp;
     const int j0 = ew.half * kCols;  // first tile column of this warp
-    int cursor = 0;  // (ROWMAX) the lowest row block not seen exhausted of codes work
+    CodesCursor cursor = codes_cursor(args, warp - 1);  // (ROWMAX) this warp's codes units
     for (int i = 0; i < nseg; ++i) {
       const int tile = item_tile(seg_tile(i)), half = item_half(seg_tile(i));
       int mb, nb;
@@ -365,7 +365,7 @@ __global__ void __maxnreg__(kGemmRegs)
     if (lane == 0) bulk_wait_group_all();  // output stores complete before exit
     __syncwarp();
     if (ROWMAX)  // help with the codes still to form
-      while (codes_one(args, lane, cursor, true, abort_flag)) {
+      while (codes_next(args, lane, cursor, true, abort_flag)) {
       }
   }
 
@@ -463,7 +463,6 @@ w8a8_status launch_gemm2sm(const int8_t *q, const float *a_scale, const void *pa
     a.done_tag = sig->tag;
     a.q_next = sig->q_next;
     a.a_scale_next = sig->a_scale_next;
-    a.unit_ctr = sig->unit_ctr;
     a.exit_word = sig->exit_word;
   }
   if (bn == 128)

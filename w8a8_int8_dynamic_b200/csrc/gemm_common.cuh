@@ -57,16 +57,14 @@ struct GemmArgs {
   // for a tile are complete it adds the columns it stored to its 128-row
   // block's word in row_done ((done_tag << 32) | columns; a block is complete
   // at 4 N).  The kernel's own warps then form the codes q_next [M, N] and
-  // scales a_scale_next [M] of each complete block (see codes_* below):
-  // unit_ctr holds one call-tagged counter per 128-row block that hands out
-  // its work units, exit_word counts the CTAs out (the last one clears the
-  // words for the next call).
+  // scales a_scale_next [M] of each complete block (see codes_* below);
+  // exit_word counts the CTAs out (the last one clears the block words for
+  // the next call).
   uint32_t *row_amax;
   unsigned long long *row_done;
   unsigned long long done_tag;
   int8_t *q_next;
   float *a_scale_next;
-  unsigned long long *unit_ctr;
   unsigned long long *exit_word;
 };
 
@@ -250,17 +248,18 @@ constexpr int kEpiStagePerWarp = kEpiStageBytes;
 // A unit is one row x kCodesSlice columns of the output, handled by one warp
 // (each lane kCodesCPL 16-byte chunks, all loads in flight together), with
 // the arithmetic of the quantisation kernel (quant_common.cuh) on the row's
-// maximum from row_amax.  Each 128-row block hands out its units from a
-// counter of its own: one counter for all units would see every grab of
-// every warp (tens of thousands of atomics on one address, serialised in
-// one L2 slice, tens of microseconds).  A warp keeps a cursor on the lowest
-// block it has not yet seen exhausted.  The idle warp 0 takes units one
-// after another, waiting for each block to complete; the epilogue warps take
-// only units of complete blocks, in the gaps between their tiles, and after
-// their last tile help with the rest.  Rows are read through L2 only (.cg):
+// maximum from row_amax.  The units are dealt out in advance: of the W
+// codes workers of the grid (warp 0 and the eight epilogue warps of every
+// CTA), worker w takes units w, w + W, w + 2W, ... in that order, so that
+// handing out work costs no atomics and each unit costs one round trip to
+// learn that its row block is complete.  Warp 0, otherwise idle, waits for
+// each block in turn; the epilogue warps take their next unit only if its
+// block is already complete, in the gaps between their tiles, and after
+// their last tile finish their share.  Rows are read through L2 only (.cg):
 // other CTAs of the grid write them.
 constexpr int kCodesCPL = 8;
 constexpr int kCodesSlice = 32 * kCodesCPL * 8;  // 2048 columns
+constexpr int kCodesWorkers = 1 + kEpiWarps;     // per CTA
 
 __device__ __forceinline__ uint4 ld_cg_u4(const void *p) {
   uint4 v;
@@ -276,20 +275,28 @@ __device__ __forceinline__ int codes_slices(const GemmArgs &a) {
 __device__ __forceinline__ unsigned long long codes_want(const GemmArgs &a) {
   return (a.done_tag << 32) | (unsigned long long)(4 * a.N);
 }
-// Units of row block b (its rows below M, times the slices of a row).
-__device__ __forceinline__ uint32_t codes_block_units(const GemmArgs &a, int b) {
-  return (uint32_t)min(128, a.M - b * 128) * (uint32_t)codes_slices(a);
+
+// A warp's share of the units: its next unit and the stride.
+struct CodesCursor {
+  uint32_t u, stride, units;
+};
+// worker: 0 for warp 0, 1 + e for epilogue warp e.
+__device__ __forceinline__ CodesCursor codes_cursor(const GemmArgs &a, int worker) {
+  CodesCursor c;
+  c.stride = gridDim.x * (uint32_t)kCodesWorkers;
+  c.u = blockIdx.x * (uint32_t)kCodesWorkers + (uint32_t)worker;
+  c.units = (uint32_t)a.M * (uint32_t)codes_slices(a);
+  return c;
 }
 
-// Waits until *word == want (acquire), the pause between reads doubling from
-// 128 ns to 2 us: a row block completes every few microseconds, and many
-// warps wait on the same word, whose L2 slice the GEMM's own traffic also
-// uses.  The blocks are completed by CTAs of this grid, which is a single
-// wave (at most one CTA or CTA pair per SM), so the wait ends unless
-// something failed; it gives up like mbar_wait_bounded.
-static __device__ __noinline__ bool wait_block(const unsigned long long *word,
-                                               unsigned long long want,
-                                               volatile int *abort_flag, int *status) {
+// Waits until *word == want (acquire, every lane), the pause between reads
+// doubling from 128 ns to 2 us: a row block completes every few
+// microseconds, and many warps wait on the same word, whose L2 slice the
+// GEMM's own traffic also uses.  The blocks are completed by CTAs of this
+// grid, which is a single wave (at most one CTA or CTA pair per SM), so the
+// wait ends unless something failed; it gives up like mbar_wait_bounded.
+__device__ __forceinline__ bool wait_block(const unsigned long long *word, unsigned long long want,
+                                           volatile int *abort_flag, int *status) {
   if (ld_acquire_gpu(word) == want) return true;
   const uint64_t t0 = global_timer_ns();
   unsigned pause = 128;
@@ -306,12 +313,11 @@ static __device__ __noinline__ bool wait_block(const unsigned long long *word,
   }
 }
 
-// Unit u of complete row block b, by the whole warp.
-__device__ __forceinline__ void codes_unit(const GemmArgs &a, int b, uint32_t u, int lane) {
+// Unit u, whose row block every lane has acquired complete, by the warp.
+__device__ __forceinline__ void codes_unit(const GemmArgs &a, uint32_t u, int lane) {
   const int slices = codes_slices(a);
-  const int row = b * 128 + (int)(u / (uint32_t)slices);
-  const int slice = (int)(u % (uint32_t)slices);
-  (void)ld_acquire_gpu(a.row_done + b);  // this lane acquires the block's rows
+  const int row = (int)(u / (uint32_t)slices);
+  const int slice = (int)(u - (uint32_t)row * (uint32_t)slices);
   const uint16_t *yr = static_cast<const uint16_t *>(a.out) + (int64_t)row * a.N;
   int8_t *qr = a.q_next + (int64_t)row * a.N;
   const int nchunks = a.N >> 3;
@@ -349,65 +355,43 @@ __device__ __forceinline__ void codes_unit(const GemmArgs &a, int b, uint32_t u,
   }
 }
 
-// Lane 0: whether block b's counter (call-tagged) has handed out all units.
-__device__ __forceinline__ bool codes_block_exhausted(const GemmArgs &a, int b) {
-  const unsigned long long cur = *reinterpret_cast<volatile unsigned long long *>(a.unit_ctr + b);
-  return (cur >> 32) == a.done_tag && (uint32_t)cur >= codes_block_units(a, b);
-}
-
-// Takes and processes one unit.  `cursor` (uniform across the warp) is the
-// lowest block this warp has not seen exhausted.  blocking: wait (bounded)
-// for the block to complete; otherwise take a unit only from a block that
-// is already complete.  False: nothing taken (blocking: no units left, or
-// abort).
-__device__ __forceinline__ bool codes_one(const GemmArgs &a, int lane, int &cursor, bool blocking,
-                                          volatile int *abort_flag) {
-  const int nblk = (a.M + 127) >> 7;
-  int b = cursor;
-  uint32_t u = 0xFFFFFFFFu;
-  if (lane == 0) {
-    while (b < nblk) {
-      if (codes_block_exhausted(a, b)) {
-        ++b;
-        continue;
-      }
-      if (!blocking && ld_acquire_gpu(a.row_done + b) != codes_want(a)) break;
-      const uint32_t got = arrive_tagged32(a.unit_ctr + b, a.done_tag, 1u) - 1u;
-      if (got >= codes_block_units(a, b)) {  // taken by others meanwhile
-        ++b;
-        continue;
-      }
-      if (blocking && !wait_block(a.row_done + b, codes_want(a), abort_flag, a.status)) {
-        b = nblk;  // abort: stop
-        break;
-      }
-      u = got;
-      break;
+// The warp's next unit, if any.  blocking: wait (bounded) for its row block;
+// otherwise only if the block is already complete.  False: none processed
+// (blocking: the share is done, or abort).
+__device__ __forceinline__ bool codes_next(const GemmArgs &a, int lane, CodesCursor &c,
+                                           bool blocking, volatile int *abort_flag) {
+  if (c.u >= c.units) return false;
+  const int slices = codes_slices(a);
+  const unsigned long long *word = a.row_done + ((c.u / (uint32_t)slices) >> 7);
+  if (blocking) {
+    if (!wait_block(word, codes_want(a), abort_flag, a.status)) {
+      c.u = c.units;  // abort: stop
+      return false;
     }
+  } else if (ld_acquire_gpu(word) != codes_want(a)) {
+    return false;
   }
-  cursor = __shfl_sync(0xFFFFFFFFu, b, 0);
-  u = __shfl_sync(0xFFFFFFFFu, u, 0);
-  if (u == 0xFFFFFFFFu) return false;
-  codes_unit(a, cursor, u, lane);
+  (void)lane;
+  codes_unit(a, c.u, lane);
+  c.u += c.stride;
   return true;
 }
 
 // An epilogue warp about to wait for its next tile's accumulators forms codes
 // of complete row blocks while they are not ready yet.
-__device__ __forceinline__ void codes_while_waiting(const GemmArgs &a, int lane, int &cursor,
+__device__ __forceinline__ void codes_while_waiting(const GemmArgs &a, int lane, CodesCursor &c,
                                                     uint64_t *tfull, uint32_t parity) {
   while (true) {
     int ready = 0;
     if (lane == 0) ready = mbar_try_wait(smem_addr(tfull), parity) ? 1 : 0;
     ready = __shfl_sync(0xFFFFFFFFu, ready, 0);
-    if (ready || !codes_one(a, lane, cursor, false, nullptr)) return;
+    if (ready || !codes_next(a, lane, c, false, nullptr)) return;
   }
 }
 
 // After the CTA's last barrier: thread 0 counts the CTA out; the last CTA of
-// the grid clears the counters and the block words (every CTA is past its
-// waits), so that a replayed CUDA graph, which keeps the tag, starts from
-// zero.
+// the grid clears the block words (every CTA is past its waits), so that a
+// replayed CUDA graph, which keeps the tag, starts from zero.
 __device__ __forceinline__ void codes_exit(const GemmArgs &a) {
   __shared__ int last_cta;
   if (threadIdx.x == 0) {
@@ -417,10 +401,7 @@ __device__ __forceinline__ void codes_exit(const GemmArgs &a) {
   __syncthreads();
   if (last_cta) {
     const int nblk = (a.M + 127) >> 7;
-    for (int b = threadIdx.x; b < nblk; b += blockDim.x) {
-      a.row_done[b] = 0ull;
-      a.unit_ctr[b] = 0ull;
-    }
+    for (int b = threadIdx.x; b < nblk; b += blockDim.x) a.row_done[b] = 0ull;
     if (threadIdx.x == 0) *a.exit_word = 0ull;
   }
 }

@@ -79,14 +79,13 @@ inline int64_t packed_cols(int64_t K) { return round_up(K, 128); }
 // The next layer's quantisation fused with a GEMM (see GemmArgs::row_amax):
 // per-row maxima (zeroed by the quantisation kernel ahead of the GEMM), per
 // 128-row block call-tagged completion words, the call's tag, the codes and
-// scales to form, per-block work counters and the exit count.
+// scales to form, and the exit count.
 struct RowSignal {
   uint32_t *row_amax;
   unsigned long long *row_done;
   unsigned long long tag;
   int8_t *q_next;
   float *a_scale_next;
-  unsigned long long *unit_ctr;
   unsigned long long *exit_word;
 };
 // pdl: a programmatic dependent of the preceding kernel; prefetch: (1-SM
