@@ -49,11 +49,14 @@ ACT_NONE, ACT_GELU = 0, 1  # w8a8_act
 # epilogue activation, whether the layer also forms the next layer's codes).
 # A layer that does runs w8a8_linear_act_quant, and the next one then runs
 # the scaled GEMM on those codes; any other layer runs w8a8_linear_act.
-# The DiT MLP block: the up-projection with GELU in its epilogue and the
-# down-projection's quantisation fused in, then the down-projection.
+# The DiT MLP block: the up-projection with GELU in its epilogue, then the
+# down-projection.  (The variant with the down-projection's quantisation
+# fused into the up-projection is measured beside it: block_variants.)
 BLOCK = "dit_mlp_block_4096x3072x12288"
-CHAINS = {BLOCK: (("dit_mlp_up_4096x12288x3072", ACT_GELU, True),
+CHAINS = {BLOCK: (("dit_mlp_up_4096x12288x3072", ACT_GELU, False),
                   ("dit_mlp_down_4096x3072x12288", ACT_NONE, False))}
+BLOCK_FUSED_QUANT = (("dit_mlp_up_4096x12288x3072", ACT_GELU, True),
+                     ("dit_mlp_down_4096x3072x12288", ACT_NONE, False))
 MAIN_WORKLOAD = BLOCK
 METRIC = "W8A8 quant+scaled-GEMM TOPS and % of int8 roofline on one B200"
 # where the raw nvidia-smi clock samples go (--clocks-dir); the JSON line
@@ -550,8 +553,11 @@ def run_ours(args, rank, world, device):
 def step_description(names):
     if len(names) == 1:
         return "w8a8_linear: quant kernel + tcgen05 GEMM/epilogue (PDL)"
-    return ("w8a8_linear_act_quant (quant, GEMM+GELU, codes of its output beside it) + "
-            "w8a8_scaled_mm on those codes" if names[0][2] else f"{len(names)} x w8a8_linear")
+    if names[0][2]:
+        return ("w8a8_linear_act_quant (quant, GEMM+GELU+codes of its output) + "
+                "w8a8_scaled_mm on those codes")
+    return (f"{len(names)} x w8a8_linear_act (quant kernel + tcgen05 GEMM/epilogue, PDL), "
+            "GELU in the first epilogue")
 
 
 def max_over_ranks(elapsed, world, device):
@@ -687,13 +693,12 @@ def sweep(w8, args, device, stream, peaks, int8_peak):
 
 
 def block_variants(w8, device, stream, nsets=4, steps=64):
-    """The DiT MLP block without the fusions of the headline step, same
-    inputs and loop: "layers" -- two w8a8_linear calls, the GELU in the
-    up-projection's epilogue but the down-projection quantising its input in
-    a pass of its own; "unfused" -- layer, GELU kernel, layer.  Microseconds
-    a step."""
-    names = CHAINS[BLOCK]
-    cs = ChainSets(w8, names, nsets, device)
+    """The DiT MLP block in three forms, same inputs and loop, microseconds a
+    step: "layers" -- the headline step's two w8a8_linear_act calls;
+    "fused_quant" -- the down-projection's quantisation fused into the
+    up-projection (w8a8_linear_act_quant), then the scaled GEMM on its codes;
+    "unfused" -- layer, GELU kernel, layer."""
+    cs = ChainSets(w8, BLOCK_FUSED_QUANT, nsets, device)
     gs = [torch.empty_like(s["layers"][0].y) for s in cs.sets]
 
     def layers(s, g):
@@ -703,6 +708,9 @@ def block_variants(w8, device, stream, nsets=4, steps=64):
         w8.linear(Lu.y, Ld.packed, Ld.w_scale, Ld.bias, Ld.N, out=Ld.y, workspace=Ld.ws,
                   stream=stream)
 
+    def fused_quant(s, g):
+        run_chain(w8, cs, s, stream)
+
     def unfused(s, g):
         Lu, Ld = s["layers"]
         w8.linear(s["x"], Lu.packed, Lu.w_scale, Lu.bias, Lu.N, out=Lu.y, workspace=Lu.ws,
@@ -711,7 +719,7 @@ def block_variants(w8, device, stream, nsets=4, steps=64):
         w8.linear(g, Ld.packed, Ld.w_scale, Ld.bias, Ld.N, out=Ld.y, workspace=Ld.ws,
                   stream=stream)
     out = {}
-    for name, fn in (("layers", layers), ("unfused", unfused)):
+    for name, fn in (("layers", layers), ("fused_quant", fused_quant), ("unfused", unfused)):
         lp = GraphLoop([lambda s=s, g=g, f=fn: f(s, g) for s, g in zip(cs.sets, gs)], stream, 4)
         lp.prepare(steps)
         time_loop(lp, 3 * lp.per_graph, stream)

@@ -116,12 +116,15 @@ def test_sets_needed_is_capped_for_tiny_workloads():
 
 def test_block_chain_is_the_dit_mlp_config():
     """The headline step: up-projection 3072 -> 12288 with GELU in its
-    epilogue and the down-projection's quantisation fused in, then the
-    row-parallel down-projection 12288 -> 3072, 4096 tokens, each layer a
-    full-size workload."""
+    epilogue, then the row-parallel down-projection 12288 -> 3072, 4096
+    tokens, each layer a full-size workload; the variant with the
+    down-projection's quantisation fused into the up-projection has the same
+    layers."""
     names = bench.chain_of(bench.MAIN_WORKLOAD)
     assert [a for _, a, _ in names] == [bench.ACT_GELU, bench.ACT_NONE]
-    assert [f for _, _, f in names] == [True, False]
+    assert [f for _, _, f in names] == [False, False]
+    assert [(n, a) for n, a, _ in bench.BLOCK_FUSED_QUANT] == [(n, a) for n, a, _ in names]
+    assert [f for _, _, f in bench.BLOCK_FUSED_QUANT] == [True, False]
     assert bench.chain_shapes(names) == [(4096, 12288, 3072, True), (4096, 3072, 12288, True)]
     ops = sum(bench.algorithmic(*s)[0] for s in bench.chain_shapes(names))
     assert ops == 2 * 2 * 4096 * 12288 * 3072
