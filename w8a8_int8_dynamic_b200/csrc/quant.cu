@@ -252,11 +252,11 @@ void prefer_max_shared(Kernel k, int slot) {
   }
 }
 
-// Launches k as a programmatic dependent of the preceding kernel of the
-// stream.  `slot` >= 0 names k for the one-time carveout setting (kernels
-// launched ahead of a GEMM); -1 leaves the default.
+// Launches k, as a programmatic dependent of the preceding kernel of the
+// stream when `pdl`.  `slot` >= 0 names k for the one-time carveout setting
+// (kernels launched ahead of a GEMM); -1 leaves the default.
 template <typename... Params, typename... Args>
-cudaError_t launch_dependent(void (*k)(Params...), int slot, dim3 grid, dim3 block,
+cudaError_t launch_dependent(void (*k)(Params...), int slot, bool pdl, dim3 grid, dim3 block,
                              cudaStream_t stream, Args... args) {
   if (slot >= 0) prefer_max_shared(k, slot);
   cudaLaunchConfig_t cfg = {};
@@ -267,8 +267,8 @@ cudaError_t launch_dependent(void (*k)(Params...), int slot, dim3 grid, dim3 blo
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.attrs = pdl ? attr : nullptr;
+  cfg.numAttrs = pdl ? 1 : 0;
   return cudaLaunchKernelEx(&cfg, k, static_cast<Params>(args)...);
 }
 
@@ -299,11 +299,18 @@ w8a8_status launch_quant(const void *x, int64_t M, int64_t K, int64_t ldx, int8_
       break;
   }
   const int64_t W = (nchunks + 32 * cpl - 1) / (32 * cpl);
+  // Inside a layer the quantisation is a programmatic dependent of the
+  // preceding kernel (after the small-M kernel, which releases its
+  // dependents early, it becomes resident and waits on the device).  Alone,
+  // it is a plain launch: launches of it back to back, each released at the
+  // start of the one before, would sit resident and waiting on the slots
+  // that the running launch's later waves need.
+  const bool pdl = ahead_of_gemm;
   cudaError_t e = cudaSuccess;
   if (W > 16) {
     // 1024-thread CTAs never leave room for a GEMM CTA: default carveout.
-    e = launch_dependent(quant_rows_two_pass_kernel, -1, dim3((unsigned)M), dim3(1024), stream,
-                         xp, ldx, (int)K, q, a_scale, zero_rows);
+    e = launch_dependent(quant_rows_two_pass_kernel, -1, pdl, dim3((unsigned)M), dim3(1024),
+                         stream, xp, ldx, (int)K, q, a_scale, zero_rows);
   } else {
     const int R = W >= 4 ? 1 : (int)(4 / W);  // rows per CTA: about 128 threads
     const unsigned grid = (unsigned)((M + R - 1) / R);
@@ -317,10 +324,10 @@ w8a8_status launch_quant(const void *x, int64_t M, int64_t K, int64_t ldx, int8_
     switch (cpl) {
 #define W8A8_QUANT_CASE(C, SLOT)                                                          \
   case C:                                                                                 \
-    e = wide ? launch_dependent(quant_warps_kernel<C, true>, SLOT, dim3(grid),            \
+    e = wide ? launch_dependent(quant_warps_kernel<C, true>, SLOT, pdl, dim3(grid),       \
                                 dim3(threads), stream, xp, ldx, (int)M, (int)K,           \
                                 (int)W, R, q, a_scale, zero_rows)                         \
-             : launch_dependent(quant_warps_kernel<C, false>, -1, dim3(grid),             \
+             : launch_dependent(quant_warps_kernel<C, false>, -1, pdl, dim3(grid),        \
                                 dim3(threads), stream, xp, ldx, (int)M, (int)K,           \
                                 (int)W, R, q, a_scale, zero_rows);                        \
     break;
