@@ -339,11 +339,11 @@ __device__ __forceinline__ void codes_unit(const GemmArgs &a, uint32_t u, int la
       if (c < nchunks) *reinterpret_cast<uint2 *>(qr + (int64_t)c * 8) = make_uint2(0, 0);
     }
   } else if (s >= 1e-30f) {
-    const CodeConsts kc(s, __frcp_rn(s));
+    const float inv = __frcp_rn(s);
 #pragma unroll
     for (int j = 0; j < kCodesCPL; ++j) {
       const int c = c0 + 32 * j;
-      if (c < nchunks) *reinterpret_cast<uint2 *>(qr + (int64_t)c * 8) = codes8(v[j], kc);
+      if (c < nchunks) *reinterpret_cast<uint2 *>(qr + (int64_t)c * 8) = codes8(v[j], s, inv);
     }
   } else {
     // (unrolled: a runtime index into v would move it to local memory)

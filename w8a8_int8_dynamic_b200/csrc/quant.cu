@@ -103,10 +103,9 @@ __global__ void __launch_bounds__(512) quant_warps_kernel(const uint16_t *__rest
   const float inv = __frcp_rn(s);
   if (w == 0 && lane == 0) a_scale[row] = s;
   uint2 out[CPL];
-  const CodeConsts kc(s, inv);
   if (s >= 1e-30f) {
 #pragma unroll
-    for (int j = 0; j < CPL; ++j) out[j] = codes8(v[j], kc);
+    for (int j = 0; j < CPL; ++j) out[j] = codes8(v[j], s, inv);
   } else {
 #pragma unroll
     for (int j = 0; j < CPL; ++j) out[j] = codes8_ieee(v[j], s);
@@ -155,13 +154,12 @@ __global__ void __launch_bounds__(1024) quant_rows_two_pass_kernel(
   const float s = amax == 0.0f ? 0.0f : __fdiv_rn(amax, 127.0f);
   const float inv = amax == 0.0f ? 0.0f : __frcp_rn(s);
   const bool exact_only = s < 1e-30f;
-  const CodeConsts kc(s, inv);
   if (threadIdx.x == 0) a_scale[row] = s;
   for (int i = threadIdx.x; i < nchunks; i += blockDim.x) {
     uint2 out = make_uint2(0, 0);
     if (amax != 0.0f) {
       const uint4 c = *reinterpret_cast<const uint4 *>(xr + (int64_t)i * 8);
-      out = exact_only ? codes8_ieee(c, s) : codes8(c, kc);
+      out = exact_only ? codes8_ieee(c, s) : codes8(c, s, inv);
     }
     *reinterpret_cast<uint2 *>(qr + (int64_t)i * 8) = out;
   }

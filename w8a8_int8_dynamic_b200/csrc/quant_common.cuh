@@ -26,8 +26,6 @@
 
 #include <stdint.h>
 
-#include "act.cuh"  // the paired fp32 instructions (f2_*)
-
 namespace w8a8 {
 
 __device__ __forceinline__ float bf16_lo(uint32_t v) { return __uint_as_float(v << 16); }
@@ -45,6 +43,14 @@ __device__ __forceinline__ uint32_t absmax_chunk(uint32_t m, const uint4 &v) {
 // The two packed lanes of absmax_chunk -> one magnitude's bit pattern.
 __device__ __forceinline__ uint32_t absmax_fold(uint32_t m) { return max(m & 0xFFFFu, m >> 16); }
 
+// A quotient whose nearest integer is that of RN(x / s), from inv = RN(1/s)
+// (one refinement step, see above; for codes only).
+__device__ __forceinline__ float code_quotient(float x, float s, float inv) {
+  const float q0 = __fmul_rn(x, inv);
+  const float r0 = __fmaf_rn(-s, q0, x);
+  return __fmaf_rn(r0, inv, q0);
+}
+
 // Low bytes of four ints -> one word.
 __device__ __forceinline__ uint32_t pack4(uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
   const uint32_t ab = __byte_perm(a, b, 0x0040);
@@ -54,41 +60,16 @@ __device__ __forceinline__ uint32_t pack4(uint32_t a, uint32_t b, uint32_t c, ui
 
 constexpr float kRound = 12582912.0f;  // 1.5 * 2^23
 
-// The code bits of the two bf16 values of one 32-bit word.  Per value x:
-// q0 = RN(x inv), r0 = RN(x - s q0) (one FMA), q1 = RN(q0 + r0 inv) (one
-// FMA) -- a quotient whose nearest integer is that of RN(x / s) (the
-// refinement step above) -- then RN(q1 + 1.5 * 2^23), whose low byte is the
-// code.  Two values an instruction, on sm_100's paired fp32 instructions
-// (each lane rounded exactly like the scalar instruction): the quantisation
-// kernels are bound by instruction issue on long inputs.
-struct CodeConsts {
-  uint64_t inv2, neg_s2, round2;
-  __device__ CodeConsts(float s, float inv)
-      : inv2(f2_splat(inv)), neg_s2(f2_splat(-s)), round2(f2_splat(kRound)) {}
-};
-__device__ __forceinline__ void code_bits_pair(uint32_t w, const CodeConsts &k, uint32_t &b0,
-                                               uint32_t &b1) {
-  const uint64_t x = f2_pack(bf16_lo(w), bf16_hi(w));
-  const uint64_t q0 = f2_mul(x, k.inv2);
-  const uint64_t r0 = f2_fma(k.neg_s2, q0, x);
-  const uint64_t q1 = f2_fma(r0, k.inv2, q0);
-  float f0, f1;
-  f2_unpack(f2_add(q1, k.round2), f0, f1);
-  b0 = __float_as_uint(f0);
-  b1 = __float_as_uint(f1);
+__device__ __forceinline__ uint32_t code_bits(float x, float s, float inv) {
+  return __float_as_uint(__fadd_rn(code_quotient(x, s, inv), kRound));
 }
 
 // One 16-byte chunk (8 bf16) -> its 8 codes, for s >= 1e-30.
-__device__ __forceinline__ uint2 codes8(const uint4 &v, const CodeConsts &k) {
-  uint32_t b[8];
-  code_bits_pair(v.x, k, b[0], b[1]);
-  code_bits_pair(v.y, k, b[2], b[3]);
-  code_bits_pair(v.z, k, b[4], b[5]);
-  code_bits_pair(v.w, k, b[6], b[7]);
-  return make_uint2(pack4(b[0], b[1], b[2], b[3]), pack4(b[4], b[5], b[6], b[7]));
-}
 __device__ __forceinline__ uint2 codes8(const uint4 &v, float s, float inv) {
-  return codes8(v, CodeConsts(s, inv));
+  return make_uint2(pack4(code_bits(bf16_lo(v.x), s, inv), code_bits(bf16_hi(v.x), s, inv),
+                          code_bits(bf16_lo(v.y), s, inv), code_bits(bf16_hi(v.y), s, inv)),
+                    pack4(code_bits(bf16_lo(v.z), s, inv), code_bits(bf16_hi(v.z), s, inv),
+                          code_bits(bf16_lo(v.w), s, inv), code_bits(bf16_hi(v.w), s, inv)));
 }
 
 // The same with the IEEE quotient (rows with s < 1e-30).  A rolled loop keeps
