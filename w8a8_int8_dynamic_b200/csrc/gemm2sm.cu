@@ -454,6 +454,10 @@ w8a8_status launch_gemm2sm(const int8_t *q, const float *a_scale, const void *pa
   a.tiles_m = (int)((M + 255) / 256);
   a.tiles_n = (int)((N + bn - 1) / bn);
   a.full_tiles = a.tiles_m * a.tiles_n;
+  // Re-read the smaller operand wave after wave: with M > N the weights
+  // (DiT MLP down-projection, 4096 x 3072 x 12288: q read from DRAM 151 MB
+  // a launch in column-tile order, for 88 MB of operands; GEMM 2 % faster).
+  a.row_major = M > N ? 1 : 0;
   a.act = act;
   a.status = status_word();
   if (!a.status) return W8A8_ERR_CUDA;

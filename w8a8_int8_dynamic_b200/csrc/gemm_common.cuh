@@ -49,6 +49,7 @@ struct GemmArgs {
   // pair kernel, whole tiles: tiles [0, full_tiles) run whole, each later one
   // as its two 128-column halves (a short last round spread over more pairs)
   int full_tiles;
+  int row_major;  // tile order (tile_coords)
   int *status;
   // Next-layer quantisation fused with this layer (the kernels' ROWMAX
   // instances): the epilogue folds each row's largest bf16 output magnitude
@@ -94,12 +95,14 @@ __device__ __forceinline__ void publish_rows(const GemmArgs &a, int lane, int ro
 
 // The (row tile, column tile) of a linear tile index.  Plain instances walk
 // the tiles column tile by column tile (row tile fastest: tiles running at
-// the same time share a weight slab in L2).  ROWMAX instances walk them row
-// tile by row tile, so that their row blocks complete one after another
-// while the GEMM runs and the codes kernel beside it can follow.
+// the same time share a weight slab in L2, and each wave of tiles reads all
+// of q again), or, with row_major, row tile by row tile (each wave reads all
+// of the weights again).  ROWMAX instances walk them row tile by row tile,
+// so that their row blocks complete one after another while the GEMM runs
+// and the codes kernel beside it can follow.
 template <bool ROWMAX>
 __device__ __forceinline__ void tile_coords(const GemmArgs &a, int tile, int &mb, int &nb) {
-  if (ROWMAX) {
+  if (ROWMAX || a.row_major) {
     mb = tile / a.tiles_n;
     nb = tile - mb * a.tiles_n;
   } else {
