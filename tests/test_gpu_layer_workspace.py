@@ -136,3 +136,40 @@ def test_layers_back_to_back_share_a_workspace():
     for y in ya + [ya2]:
         assert np.array_equal(host_u16(y), ya_ref)
     assert np.array_equal(host_u16(yb), oracle.linear(ya_ref, b.w, b.w_scale, b.bias)[0])
+
+
+def test_layers_from_two_host_threads():
+    """Two host threads run layers of different shapes at the same time, each
+    on its own stream and workspace (the library's per-context caches and
+    launch settings are shared between them)."""
+    import threading
+    cases = [random_case(71, 600, 2048, 1024, bias=True, n_outliers=16),
+             random_case(72, 40, 1024, 4096, bias=True, n_outliers=64),
+             random_case(73, 8, 4096, 1024, bias=False, n_outliers=16)]
+    results, errors = {}, []
+
+    def worker(i, inp):
+        try:
+            torch.cuda.set_device(0)
+            s = torch.cuda.Stream()
+            with torch.cuda.stream(s):
+                layer = w8.W8A8Linear(dev(inp.w), dev(inp.w_scale),
+                                      None if inp.bias is None else dev_bf16(inp.bias))
+                x = dev_bf16(inp.x)
+                ys = [layer(x) for _ in range(6)]
+            s.synchronize()
+            results[i] = [host_u16(y) for y in ys]
+        except Exception as e:  # reported on the main thread
+            errors.append(repr(e))
+
+    threads = [threading.Thread(target=worker, args=(i, c)) for i, c in enumerate(cases)]
+    for t in threads:
+        t.start()
+    for t in threads:
+        t.join(timeout=120)
+    assert not errors, errors
+    for i, inp in enumerate(cases):
+        y_ref = _expect(inp.x, inp, w8.ACT_NONE)
+        assert len(results[i]) == 6
+        for y in results[i]:
+            assert np.array_equal(y, y_ref), f"thread {i}"

@@ -366,7 +366,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-bool g_decode_attr_done[64];
+FuncAttrOnce g_decode_smem_attr;
 
 int64_t units_of(int64_t N, int64_t K) {
   const int64_t nkb = packed_cols(K) / 128;
@@ -431,13 +431,10 @@ w8a8_status launch_decode(const int8_t *q, const float *a_scale, const void *pac
   cudaError_t e = cudaSuccess;
   using L = DecodeSmem<kDecodeStages>;
   auto k = decode_kernel<kDecodeStages>;
-  const int d = current_device();
-  if (d < 0 || d >= 64 || !g_decode_attr_done[d]) {
-    if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kAlloc) !=
-        cudaSuccess)
-      return W8A8_ERR_CUDA;
-    if (d >= 0 && d < 64) g_decode_attr_done[d] = true;
-  }
+  if (g_decode_smem_attr.ensure([&] {
+        return cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kAlloc);
+      }) != cudaSuccess)
+    return W8A8_ERR_CUDA;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)grid);
   cfg.blockDim = dim3(kThreads);

@@ -372,15 +372,12 @@ constexpr int kKps128 = 2;
 constexpr int kPrefetchKb = 32;
 constexpr int kLargeStages256 = 4;  // 4 x (1 k-block): 48 KB stages
 
-bool g_attr_done[64][8];
+FuncAttrOnce g_smem_attr[8];  // one per kernel instance (`slot`)
 
 template <typename Kernel>
 cudaError_t set_smem_attr(Kernel k, int bytes, int slot) {
-  const int d = current_device();
-  if (d >= 0 && d < 64 && g_attr_done[d][slot]) return cudaSuccess;
-  cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
-  if (e == cudaSuccess && d >= 0 && d < 64) g_attr_done[d][slot] = true;
-  return e;
+  return g_smem_attr[slot].ensure(
+      [&] { return cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes); });
 }
 
 template <typename Kernel, typename... Args>

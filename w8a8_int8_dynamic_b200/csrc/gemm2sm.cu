@@ -378,7 +378,7 @@ __global__ void __maxnreg__(kGemmRegs)
   if (ROWMAX) codes_exit(args);
 }
 
-bool g_pair_attr_done[64][4];
+FuncAttrOnce g_pair_smem_attr[4];  // one per kernel instance (`slot_id`)
 
 template <int BN, int STAGES, bool ROWMAX = false>
 w8a8_status run_pair(const CUtensorMap &tq, const CUtensorMap &tw, const CUtensorMap &tw64,
@@ -386,13 +386,10 @@ w8a8_status run_pair(const CUtensorMap &tq, const CUtensorMap &tw, const CUtenso
                      int slot_id) {
   using L = PairSmem<BN, STAGES>;
   auto k = gemm2sm_kernel<BN, STAGES, ROWMAX>;
-  const int d = current_device();
-  if (d < 0 || d >= 64 || !g_pair_attr_done[d][slot_id]) {
-    if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kAlloc) !=
-        cudaSuccess)
-      return W8A8_ERR_CUDA;
-    if (d >= 0 && d < 64) g_pair_attr_done[d][slot_id] = true;
-  }
+  if (g_pair_smem_attr[slot_id].ensure([&] {
+        return cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kAlloc);
+      }) != cudaSuccess)
+    return W8A8_ERR_CUDA;
   const int tiles = a.tiles_m * a.tiles_n;
   const int items = a.full_tiles + 2 * (tiles - a.full_tiles);
   // persistent: one pair per two SMs, at most one per work item

@@ -6,6 +6,7 @@
 #include <stddef.h>
 #include <stdint.h>
 
+#include <atomic>
 #include <mutex>
 
 #include "w8a8.h"
@@ -31,6 +32,28 @@ struct SymbolCache {
 // variable) in the current context, from the cache while that context is the
 // one it was looked up in, else from cudaGetSymbolAddress.
 bool symbol_address(SymbolCache *cache, const void *symbol, void **out);
+
+// A per-function setting (cudaFuncSetAttribute) made once per device and
+// CUDA context: `set` runs unless it already succeeded in the context
+// current now (by its process-wide unique ID, which a context created after
+// a device reset or pushed by the caller does not share).  Any host thread
+// may call it; two threads that find it unset both run `set`, which is
+// idempotent.
+struct FuncAttrOnce {
+  static constexpr int kDevices = 64;
+  std::atomic<unsigned long long> ctx_plus1[kDevices] = {};  // 0: not set
+  template <typename F>
+  cudaError_t ensure(F &&set) {
+    int d = 0;
+    unsigned long long id = 0;
+    const bool have = cudaGetDevice(&d) == cudaSuccess && d >= 0 && d < kDevices &&
+                      current_context_id(&id);
+    if (have && ctx_plus1[d].load(std::memory_order_acquire) == id + 1) return cudaSuccess;
+    const cudaError_t e = set();
+    if (e == cudaSuccess && have) ctx_plus1[d].store(id + 1, std::memory_order_release);
+    return e;
+  }
+};
 
 // Number of SMs of the current device (cached per device).
 int sm_count();

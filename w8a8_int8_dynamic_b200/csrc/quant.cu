@@ -238,18 +238,15 @@ __global__ void __launch_bounds__(256) quant_static_kernel(const uint16_t *__res
 // drained, so the GEMM would start no earlier than the quantisation ends.
 // Alone, the quantisation keeps the default share: with the largest one (and
 // so the smallest L1) a 512 x 4096 input takes 4.5 us instead of 3.9 us.
-bool g_carveout_done[64][8];
+FuncAttrOnce g_carveout[8];  // one per kernel instance (`slot`)
 
 template <typename Kernel>
 void prefer_max_shared(Kernel k, int slot) {
-  const int d = current_device();
-  if (d >= 0 && d < 64 && g_carveout_done[d][slot]) return;
-  if (cudaFuncSetAttribute(k, cudaFuncAttributePreferredSharedMemoryCarveout,
-                           (int)cudaSharedmemCarveoutMaxShared) == cudaSuccess) {
-    if (d >= 0 && d < 64) g_carveout_done[d][slot] = true;
-  } else {
+  if (g_carveout[slot].ensure([&] {
+        return cudaFuncSetAttribute(k, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                    (int)cudaSharedmemCarveoutMaxShared);
+      }) != cudaSuccess)
     (void)cudaGetLastError();  // a preference only: the launch goes ahead without it
-  }
 }
 
 // Launches k, as a programmatic dependent of the preceding kernel of the

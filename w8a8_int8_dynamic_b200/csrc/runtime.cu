@@ -14,7 +14,7 @@ __device__ int g_status_word;
 
 namespace {
 constexpr int kMaxDevices = 64;
-int g_sm_count[kMaxDevices];
+std::atomic<int> g_sm_count[kMaxDevices];
 std::mutex g_mu;
 std::atomic<int64_t> g_launches{0};
 std::atomic<int> g_forced_path{0};
@@ -89,12 +89,13 @@ int *status_word() {
 int sm_count() {
   const int d = current_device();
   if (d < 0 || d >= kMaxDevices) return 148;
-  if (!g_sm_count[d]) {
-    int n = 0;
+  int n = g_sm_count[d].load(std::memory_order_relaxed);
+  if (!n) {
     cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, d);
-    g_sm_count[d] = n > 0 ? n : 148;
+    if (n <= 0) n = 148;
+    g_sm_count[d].store(n, std::memory_order_relaxed);
   }
-  return g_sm_count[d];
+  return n;
 }
 
 void count_launch(int n) { g_launches.fetch_add(n, std::memory_order_relaxed); }
