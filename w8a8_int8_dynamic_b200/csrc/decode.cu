@@ -97,6 +97,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + L::kMisc + 4);
   volatile int *last_flag = reinterpret_cast<volatile int *>(smem + L::kMisc + 8);
   volatile int *seg_ok = reinterpret_cast<volatile int *>(smem + L::kMisc + 16);  // [2]
+  volatile int *early_in = reinterpret_cast<volatile int *>(smem + L::kMisc + 24);  // [2]
 
   // Release the next kernel of the stream at once: the activation
   // quantisation of the next layer becomes resident beside this kernel and
@@ -289,6 +290,46 @@ __global__ void __launch_bounds__(kThreads, 1)
       const float ws = n < args.N ? __ldg(args.w_scale + n) : 0.0f;
       const float bv =
           (args.bias && n < args.N) ? __uint_as_float((uint32_t)__ldg(args.bias + n) << 16) : 0.0f;
+      // A slab split between CTAs: this CTA's rank among those covering it.
+      // A CTA's last segment is usually the start of a slab whose other
+      // parts its neighbours finished long before, at the start of their
+      // ranges.  If every other contributor has already arrived, this CTA is
+      // the last one: it takes their partials now, while its own MMAs run,
+      // and adds them to its accumulators without publishing its own (no
+      // stores, fence, tagged arrival or partial reads at the tail of the
+      // kernel, which the next launch waits for).
+      int contributors = 1, rank = 0;
+      bool early = false;
+      int32_t pre[kDecodeNT];
+#pragma unroll
+      for (int m = 0; m < kDecodeNT; ++m) pre[m] = 0;
+      if (!whole) {
+        const int first_cta = cta_of_unit(args.units, gridDim.x, slab_begin);
+        const int last_cta = cta_of_unit(args.units, gridDim.x, slab_end - 1);
+        contributors = last_cta - first_cta + 1;
+        rank = blockIdx.x - first_cta;
+        if (et == 0) {
+          const unsigned long long v = ld_acquire_gpu(args.counters + nb);
+          const bool in =
+              (v >> 8) == args.tag && (uint32_t)(v & 0xFF) == (uint32_t)(contributors - 1);
+          // no other arrival can follow: this call is done with the word
+          if (in) args.counters[nb] = 0ull;
+          // (its own word per buffer: threads may still read last_flag of
+          // the previous segment)
+          early_in[b] = in ? 1 : 0;
+        }
+        __syncwarp();
+        asm volatile("bar.sync 1, 128;" ::: "memory");
+        early = early_in[b] != 0;
+        if (early)
+          for (int c = 0; c < contributors; ++c) {
+            if (c == rank) continue;
+            const int32_t *o = args.partials +
+                               ((size_t)nb * args.max_contrib + c) * (128 * kDecodeNT) + n_local;
+#pragma unroll
+            for (int m = 0; m < kDecodeNT; ++m) pre[m] += __ldcg(o + m * 128);
+          }
+      }
       if (et == 0) seg_ok[b] = mbar_wait(&tfull[b], bph, abort_flag, args.status) ? 1 : 0;
       __syncwarp();
       asm volatile("bar.sync 1, 128;" ::: "memory");
@@ -302,36 +343,51 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (lane == 0) mbar_arrive(&tempty[b]);
 
       bool finish = whole;
-      if (!whole) {
-        // contributor rank of this CTA among the CTAs covering this slab
-        const int first_cta = cta_of_unit(args.units, gridDim.x, slab_begin);
-        const int last_cta = cta_of_unit(args.units, gridDim.x, slab_end - 1);
-        const int contributors = last_cta - first_cta + 1;
-        const int rank = blockIdx.x - first_cta;
-        int32_t *slot = args.partials +
-                        ((size_t)nb * args.max_contrib + rank) * (128 * kDecodeNT) + n_local;
+      if (!whole && early) {
 #pragma unroll
-        for (int m = 0; m < kDecodeNT; ++m) slot[m * 128] = (int32_t)r[m];
-        __threadfence();
-        __syncwarp();
-        asm volatile("bar.sync 1, 128;" ::: "memory");
+        for (int m = 0; m < kDecodeNT; ++m) r[m] = (uint32_t)((int32_t)r[m] + pre[m]);
+        finish = true;
+      } else if (!whole) {
+        // The same check once more, now that this CTA's MMAs are done.
         if (et == 0) {
-          const bool last = arrive_tagged(args.counters + nb, args.tag) == (uint32_t)contributors;
-          // The last arrival of this call: nothing else touches the word in
-          // this launch, so clear it.  A replayed CUDA graph relaunches with
-          // the same tag and must find the count at zero, not at its total.
-          if (last) args.counters[nb] = 0ull;
-          *last_flag = last ? 1 : 0;
+          const unsigned long long v = ld_acquire_gpu(args.counters + nb);
+          const bool others_in =
+              (v >> 8) == args.tag && (uint32_t)(v & 0xFF) == (uint32_t)(contributors - 1);
+          // no other arrival can follow: this call is done with the word
+          if (others_in) args.counters[nb] = 0ull;
+          *last_flag = others_in ? 2 : 0;
         }
         __syncwarp();
         asm volatile("bar.sync 1, 128;" ::: "memory");
+        const bool others_in = *last_flag == 2;
+        if (!others_in) {
+          int32_t *slot = args.partials +
+                          ((size_t)nb * args.max_contrib + rank) * (128 * kDecodeNT) + n_local;
+#pragma unroll
+          for (int m = 0; m < kDecodeNT; ++m) slot[m * 128] = (int32_t)r[m];
+          __threadfence();
+          __syncwarp();
+          asm volatile("bar.sync 1, 128;" ::: "memory");
+          if (et == 0) {
+            const bool last =
+                arrive_tagged(args.counters + nb, args.tag) == (uint32_t)contributors;
+            // The last arrival of this call: nothing else touches the word in
+            // this launch, so clear it.  A replayed CUDA graph relaunches with
+            // the same tag and must find the count at zero, not at its total.
+            if (last) args.counters[nb] = 0ull;
+            *last_flag = last ? 1 : 0;
+          }
+          __syncwarp();
+          asm volatile("bar.sync 1, 128;" ::: "memory");
+        }
         finish = *last_flag != 0;
         if (finish) {
-          __threadfence();
+          if (!others_in) __threadfence();
           int32_t sum[kDecodeNT];
 #pragma unroll
-          for (int m = 0; m < kDecodeNT; ++m) sum[m] = 0;
+          for (int m = 0; m < kDecodeNT; ++m) sum[m] = others_in ? (int32_t)r[m] : 0;
           for (int c = 0; c < contributors; ++c) {
+            if (others_in && c == rank) continue;  // its own part is in r
             const int32_t *o = args.partials +
                                ((size_t)nb * args.max_contrib + c) * (128 * kDecodeNT) + n_local;
 #pragma unroll
