@@ -176,13 +176,16 @@ def test_layers_from_two_host_threads():
 
 
 @pytest.mark.parametrize("path", [w8.PATH_AUTO, w8.PATH_LARGE_PAIR])
-def test_row_tile_order_with_half_tile_round(path):
+@pytest.mark.parametrize("M", [8192, 8000])
+def test_row_tile_order_with_half_tile_round(path, M):
     """M > N: the pair kernel walks its tiles row tile by row tile; 8192 x
     2560 gives 320 tiles of 256 x 256 on the 74 SM pairs, the last 24 run as
-    256 x 128 halves.  Every output against the oracle."""
+    256 x 128 halves.  8000 rows: the last row tile holds 64 rows, so the odd
+    CTA of each of its pairs lies wholly past M.  Every output against the
+    oracle."""
     w8.set_path(path)
-    M, N, K = 8192, 2560, 256
-    inp = random_case(81, M, N, K, bias=True, n_outliers=4)
+    N, K = 2560, 256
+    inp = random_case(81 + M, M, N, K, bias=True, n_outliers=4)
     layer = w8.W8A8Linear(dev(inp.w), dev(inp.w_scale), dev_bf16(inp.bias))
     y = layer(dev_bf16(inp.x))
     torch.cuda.synchronize()
