@@ -486,6 +486,9 @@ def run_ours(args, rank, world, device):
     # launch duration
     t_g = [base[f"t_gemm{i}"] for i in range(len(names))]
     gemm_tops = ops / sum(t_g) / 1e12
+    # the int8 tensor-core rate with no memory traffic, measured here now
+    with torch.cuda.stream(stream):
+        mma_ceiling = w8.selftest_int8_mma_rate(20000, stream=stream)
     kernels = [w8.gemm_kernel_name(M, N, K) for M, N, K, _ in shapes]
     traffic = [recorded_traffic(n) for n, *_ in names]
     roofline = {
@@ -495,6 +498,8 @@ def run_ours(args, rank, world, device):
         "kernel": kernels[0].split(" (")[0] if len(set(kernels)) == 1 else kernels,
         "peak_note": f"2 x {peaks['source']} bf16 burst",
         "frac_vs_spec_4500": round(gemm_tops / SPEC_INT8_TOPS, 4),
+        "frac_vs_mma_ceiling": round(gemm_tops / mma_ceiling, 4),
+        "mma_ceiling": round(mma_ceiling, 1),
         "ops_per_launch": ops_l[0] if len(set(ops_l)) == 1 else ops_l,
         "gemm_us": [round(t * 1e6, 2) for t in t_g],
         "quant_us": [round(base[f"t_quant{i}"] * 1e6, 2) for i in range(len(names))],

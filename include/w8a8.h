@@ -326,6 +326,18 @@ w8a8_status w8a8_poll_status(w8a8_stream_t stream);
 w8a8_status w8a8_selftest_wait_timeout(int64_t timeout_ns,
                                        w8a8_stream_t stream);
 
+/* Self-test of the int8 tensor-core rate with no memory traffic (no
+ * counterpart on the pages; the ceiling against which the GEMM kernels'
+ * rates can be read): one CTA per SM issues `iters` (1 ... 1e6) groups of
+ * four tcgen05.mma.kind::i8 of M = 128, N = 256, K = 32 from shared memory
+ * into TMEM; the launch is timed with CUDA events on `stream` after a
+ * warm-up launch.  Synchronises the stream.  *tops: int8 TOPS (2 operations
+ * a multiply-add) over all SMs.  W8A8_ERR_INVALID_ARG for a null tops or
+ * iters out of range; a device-side wait that gave up shows in
+ * w8a8_poll_status. */
+w8a8_status w8a8_selftest_int8_mma_rate(int64_t iters, w8a8_stream_t stream,
+                                        double *tops);
+
 /* Number of kernels this library has launched in this process (all devices). */
 int64_t w8a8_launch_count(void);
 

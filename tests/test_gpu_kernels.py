@@ -331,6 +331,16 @@ def test_cuda_graph_replay_with_new_inputs(case):
     del g
 
 
+# ---------------------------------------------------------------- int8 MMA rate
+def test_int8_mma_rate_selftest():
+    """The memory-free tcgen05.mma.kind::i8 loop: a rate between the bf16
+    burst figure and twice the dense int8 spec (4.5 POPS), and no device-side
+    timeout."""
+    tops = w8.selftest_int8_mma_rate(4000)
+    assert 1500.0 < tops < 9000.0, tops
+    assert w8.poll_status() == 0
+
+
 # ---------------------------------------------------------------- bounded waits
 def test_timeout_is_reported_and_context_survives():
     w8.selftest_wait_timeout(2_000_000)  # 2 ms

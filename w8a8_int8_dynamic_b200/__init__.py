@@ -11,5 +11,5 @@ from .binding import (  # noqa: F401
     PATH_SMALL, W8A8Error, W8A8Linear,
     gelu_tanh, gemm_kernel_name, launch_count, lib, linear, linear_act_quant,
     linear_act_quant_workspace_bytes, linear_workspace_bytes, pack_weight, pack_weight_int32, packed_weight_bytes,
-    poll_status, quant_act, quant_act_static, quant_pack_weight, scaled_mm, scaled_mm_i32, scaled_mm_workspace_bytes, selftest_wait_timeout,
+    poll_status, quant_act, quant_act_static, quant_pack_weight, scaled_mm, scaled_mm_i32, scaled_mm_workspace_bytes, selftest_int8_mma_rate, selftest_wait_timeout,
     set_path, unpack_weight)

@@ -75,6 +75,7 @@ _SIGNATURES = {
     "w8a8_gelu_tanh": ([_P, _P, _I64, _P], ctypes.c_int),
     "w8a8_poll_status": ([_P], ctypes.c_int),
     "w8a8_selftest_wait_timeout": ([_I64, _P], ctypes.c_int),
+    "w8a8_selftest_int8_mma_rate": ([_I64, _P, ctypes.POINTER(ctypes.c_double)], ctypes.c_int),
     "w8a8_launch_count": ([], ctypes.c_int64),
 }
 
@@ -368,6 +369,14 @@ def set_path(path: int):
 
 def poll_status(stream=None) -> int:
     return int(lib().w8a8_poll_status(_stream(stream)))
+
+
+def selftest_int8_mma_rate(iters: int = 20000, stream=None) -> float:
+    """int8 TOPS of a memory-free tcgen05.mma loop on every SM (synchronises)."""
+    out = ctypes.c_double(0.0)
+    _check(lib().w8a8_selftest_int8_mma_rate(iters, _stream(stream), ctypes.byref(out)),
+           "w8a8_selftest_int8_mma_rate")
+    return out.value
 
 
 def selftest_wait_timeout(timeout_ns: int, stream=None):

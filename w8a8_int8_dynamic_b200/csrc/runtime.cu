@@ -175,6 +175,56 @@ __global__ void selftest_wait_kernel(int *status, uint64_t limit_ns) {
   __syncthreads();
 }
 
+// The int8 tensor-core rate with no memory traffic, the ceiling the GEMMs'
+// fractions are read against beside the measured bf16 rate: every CTA (one
+// per SM) issues `iters` groups of four tcgen05.mma.cta_group::1.kind::i8
+// (M = 128, N = 256, K = 32) from fixed shared-memory tiles into one TMEM
+// accumulator, then waits (bounded) for them.  The operand bytes are an
+// arbitrary pattern of small values (not zeros, which toggle less); the
+// int32 sums wrap and are never read.
+constexpr int kRateN = 256;
+constexpr int kRateSmem = 16384 + kRateN * 128 + 16 + 1024;
+
+__global__ void __launch_bounds__(128, 1) selftest_mma_rate_kernel(int iters, int *status) {
+  extern __shared__ uint8_t raw[];
+  uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(raw) + 1023) &
+                                            ~static_cast<uintptr_t>(1023));
+  uint8_t *sA = sm, *sB = sm + 16384;  // 128 x 128 and 256 x 128 int8 tiles (SW128 images)
+  uint64_t *bar = reinterpret_cast<uint64_t *>(sm + 16384 + kRateN * 128);
+  uint32_t *slot = reinterpret_cast<uint32_t *>(bar + 1);
+  __shared__ int abort_flag;
+  for (int i = threadIdx.x; i < (16384 + kRateN * 128) / 4; i += blockDim.x)
+    reinterpret_cast<uint32_t *>(sm)[i] = 0x01010101u * (((uint32_t)i * 2654435761u) >> 29);
+  if (threadIdx.x == 0) {
+    mbar_init(bar, 1);
+    abort_flag = 0;
+    fence_barrier_init();
+  }
+  fence_proxy_async_smem();  // the operand bytes, before the tensor core reads them
+  if (threadIdx.x < 32) tmem_alloc(slot, kRateN);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *slot;
+  if (threadIdx.x == 0) {
+    const uint64_t ad = sw128_kmajor_desc(sA), bd = sw128_kmajor_desc(sB);
+    constexpr uint32_t id = idesc_i8(128, kRateN);
+    for (int it = 0; it < iters; ++it)
+#pragma unroll
+      for (int k = 0; k < 4; ++k) mma_i8(tmem, ad + 2 * k, bd + 2 * k, id, (it | k) != 0);
+    mma_commit(bar);
+    (void)mbar_wait_bounded(bar, 0, &abort_flag, status);
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (threadIdx.x < 32) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kRateN);
+  }
+}
+
+FuncAttrOnce g_rate_smem_attr;
+
 }  // namespace w8a8
 
 using namespace w8a8;
@@ -194,7 +244,7 @@ const char *w8a8_status_string(int status) {
   }
 }
 
-int w8a8_abi_version(void) { return (1 << 16) | 0; }
+int w8a8_abi_version(void) { return (1 << 16) | 1; }
 
 w8a8_status w8a8_set_path(int path) {
   if (path < 0 || path > 7 || path == 6) return W8A8_ERR_INVALID_ARG;
@@ -220,6 +270,39 @@ w8a8_status w8a8_poll_status(w8a8_stream_t stream) {
     return static_cast<w8a8_status>(host);
   }
   return W8A8_OK;
+}
+
+w8a8_status w8a8_selftest_int8_mma_rate(int64_t iters, w8a8_stream_t stream, double *tops) {
+  if (!tops || iters < 1 || iters > 1000000) return W8A8_ERR_INVALID_ARG;
+  int *sw = status_word();
+  if (!sw) return W8A8_ERR_CUDA;
+  if (g_rate_smem_attr.ensure([] {
+        return cudaFuncSetAttribute(selftest_mma_rate_kernel,
+                                    cudaFuncAttributeMaxDynamicSharedMemorySize, kRateSmem);
+      }) != cudaSuccess)
+    return W8A8_ERR_CUDA;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const int sms = sm_count();
+  cudaEvent_t e0 = nullptr, e1 = nullptr;
+  if (cudaEventCreate(&e0) != cudaSuccess || cudaEventCreate(&e1) != cudaSuccess) {
+    if (e0) cudaEventDestroy(e0);
+    return W8A8_ERR_CUDA;
+  }
+  selftest_mma_rate_kernel<<<sms, 128, kRateSmem, s>>>(64, sw);  // warm-up
+  cudaEventRecord(e0, s);
+  selftest_mma_rate_kernel<<<sms, 128, kRateSmem, s>>>((int)iters, sw);
+  cudaEventRecord(e1, s);
+  count_launch(2);
+  cudaError_t e = cudaEventSynchronize(e1);
+  float ms = 0.0f;
+  if (e == cudaSuccess) e = cudaEventElapsedTime(&ms, e0, e1);
+  cudaEventDestroy(e0);
+  cudaEventDestroy(e1);
+  if (e != cudaSuccess) return W8A8_ERR_CUDA;
+  *tops = ms > 0.0f ? (double)sms * (double)iters * 4.0 * 2.0 * 128.0 * kRateN * 32.0 /
+                          (ms * 1e-3) / 1e12
+                    : 0.0;
+  return from_cuda(cudaGetLastError());
 }
 
 w8a8_status w8a8_selftest_wait_timeout(int64_t timeout_ns, w8a8_stream_t stream) {
