@@ -299,10 +299,14 @@ w8a8_status launch_quant(const void *x, int64_t M, int64_t K, int64_t ldx, int8_
   // Inside a layer the quantisation is a programmatic dependent of the
   // preceding kernel (after the small-M kernel, which releases its
   // dependents early, it becomes resident and waits on the device).  Alone,
-  // it is a plain launch: launches of it back to back, each released at the
-  // start of the one before, would sit resident and waiting on the slots
-  // that the running launch's later waves need.
-  const bool pdl = ahead_of_gemm;
+  // an input resident in one wave (at most 16 warps a SM on average) is a
+  // plain launch: launches of it back to back, each released at the start of
+  // the one before, would sit resident and waiting on the slots the running
+  // launch needs (512 x 4096: 3.96 -> 3.08 us).  Longer inputs are
+  // dependents there too: the next launch's first CTAs then start as the
+  // running one's last wave drains (4096 x 3072: 11.3 -> 10.7 us; 4096 x
+  // 12288: 32.3 -> 31.3 us).
+  const bool pdl = ahead_of_gemm || M * W > (int64_t)sm_count() * 16;
   cudaError_t e = cudaSuccess;
   if (W > 16) {
     // 1024-thread CTAs never leave room for a GEMM CTA: default carveout.
