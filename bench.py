@@ -695,7 +695,11 @@ def sweep(w8, args, device, stream, peaks, int8_peak):
     for name in SWEEP:
         wl = WORKLOADS[name]
         ops, gemm_bytes, quant_bytes, fused_bytes = algorithmic(wl.M, wl.N, wl.K, wl.bias)
-        steps = 200 if ops > 1e11 else 2000
+        # about 25 ms of work a loop for every row (100 to 2000 steps), so that
+        # each finishes before the power cap settles, like the burst peak it is
+        # read against (the headline's long loops give the sustained figure)
+        t_est = max(ops / (int8_peak * 1e12 * 0.6), gemm_bytes / (peaks["hbm_gbs"] * 1e9 * 0.8))
+        steps = int(min(2000, max(100, 25e-3 / t_est)))
         warm = wl.N * wl.K + wl.M * wl.K + 2 * wl.M * wl.N < L2_BYTES // 2
         cs, loop, r = measure_chain(w8, chain_of(name), steps, 3, device, stream,
                                     warm_gemm=warm)
