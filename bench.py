@@ -86,10 +86,11 @@ def load_peaks():
 
 
 # the sources each GEMM kernel is compiled from (a change voids its record)
+_GEMM_HEADERS = ("gemm_common.cuh", "act.cuh", "f32x2.cuh", "quant_common.cuh", "ptx.cuh")
 TRAFFIC_SOURCES = {
-    "gemm_kernel": ("gemm.cu", "gemm_common.cuh", "act.cuh", "ptx.cuh"),
-    "gemm2sm_kernel": ("gemm2sm.cu", "gemm_common.cuh", "act.cuh", "ptx.cuh"),
-    "decode_kernel": ("decode.cu", "gemm_common.cuh", "act.cuh", "ptx.cuh"),
+    "gemm_kernel": ("gemm.cu",) + _GEMM_HEADERS,
+    "gemm2sm_kernel": ("gemm2sm.cu",) + _GEMM_HEADERS,
+    "decode_kernel": ("decode.cu",) + _GEMM_HEADERS,
 }
 
 

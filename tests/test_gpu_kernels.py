@@ -28,8 +28,11 @@ def _gpu():
 
 
 # ---------------------------------------------------------------- quantisation
+# Every kernel instance: 1-4 chunks a lane, 8 (rows x warps beyond two waves
+# of resident warps: 1500 x 12288), 16 (rows of more than 16 warps at 8), and
+# the two-pass kernel (rows beyond 65536).
 QUANT_SHAPES = [(1, 16), (3, 48), (64, 256), (127, 4096), (129, 3072), (512, 4096),
-                (7, 12288), (16, 5120), (5, 40000), (2, 131072), (33, 32784)]
+                (7, 12288), (16, 5120), (5, 40000), (2, 131072), (33, 32784), (1500, 12288)]
 
 
 @pytest.mark.parametrize("M,K", QUANT_SHAPES)
@@ -48,10 +51,13 @@ def test_quant_matches_oracle(M, K):
     assert np.array_equal(q.cpu().numpy(), q_ref)
 
 
-def test_quant_near_ties_and_ties():
+@pytest.mark.parametrize("K,reps", [(256, 1), (12288, 28), (40000, 1)])
+def test_quant_near_ties_and_ties(K, reps):
     """Values whose quotient is exactly a half-integer, or a few fp32 ulps
-    from one: the kernel's reciprocal fast path must defer to the IEEE
-    quotient exactly as the oracle's plain division rounds."""
+    from one: the kernel's reciprocal fast path must round them exactly as
+    the oracle's plain division does.  Rows of K elements (the pattern
+    repeated), `reps` copies of the row set: short rows, the 8-chunk instance
+    (54 x 28 rows of 12288) and the 16-chunk one."""
     rows = []
     for e in range(-20, 20, 3):
         s = 2.0 ** e
@@ -68,7 +74,7 @@ def test_quant_near_ties_and_ties():
         near = (k * s).astype(np.float32)
         near = near + rng.integers(-3, 4, 255).astype(np.float32) * np.spacing(near)
         rows.append(np.concatenate([[amax], near]).astype(np.float32)[:256])
-    x = np.stack([np.resize(r, 256) for r in rows])
+    x = np.tile(np.stack([np.resize(r, K) for r in rows]), (reps, 1))
     xb = f32_to_bf16_bits(x)
     q_ref, s_ref = oracle.quant_act(xb)
     q, s = w8.quant_act(dev_bf16(xb))

@@ -104,8 +104,19 @@ __global__ void __launch_bounds__(512) quant_warps_kernel(const uint16_t *__rest
   if (w == 0 && lane == 0) a_scale[row] = s;
   uint2 out[CPL];
   if (s >= 1e-30f) {
+    if constexpr (CPL >= 8) {
+      // Long rows keep the issue slots busy (close to instruction-bound):
+      // there the paired fp32 instructions take two instructions an element
+      // off (4096 x 12288: 25.4-25.9 -> 25.0-25.5 us alone, 2048 x 12288:
+      // 14.5 -> 14.1 us, on one box).  Short rows wait on DRAM latency, and
+      // there the pair form measured no faster or slower.
+      const uint64_t ns2 = f2_splat(-s), inv2 = f2_splat(inv), rnd2 = f2_splat(kRound);
 #pragma unroll
-    for (int j = 0; j < CPL; ++j) out[j] = codes8(v[j], s, inv);
+      for (int j = 0; j < CPL; ++j) out[j] = codes8_x2(v[j], ns2, inv2, rnd2);
+    } else {
+#pragma unroll
+      for (int j = 0; j < CPL; ++j) out[j] = codes8(v[j], s, inv);
+    }
   } else {
 #pragma unroll
     for (int j = 0; j < CPL; ++j) out[j] = codes8_ieee(v[j], s);

@@ -26,6 +26,8 @@
 
 #include <stdint.h>
 
+#include "f32x2.cuh"
+
 namespace w8a8 {
 
 __device__ __forceinline__ float bf16_lo(uint32_t v) { return __uint_as_float(v << 16); }
@@ -70,6 +72,31 @@ __device__ __forceinline__ uint2 codes8(const uint4 &v, float s, float inv) {
                           code_bits(bf16_lo(v.y), s, inv), code_bits(bf16_hi(v.y), s, inv)),
                     pack4(code_bits(bf16_lo(v.z), s, inv), code_bits(bf16_hi(v.z), s, inv),
                           code_bits(bf16_lo(v.w), s, inv), code_bits(bf16_hi(v.w), s, inv)));
+}
+
+// The same two values at a time on the paired fp32 instructions (each lane
+// rounded like the scalar ones, so the codes are the same bits): the bf16
+// pair of one 32-bit word, ns2 = (-s, -s), inv2 = (inv, inv), rnd2 =
+// (kRound, kRound).  Half the floating-point instructions of codes8.
+__device__ __forceinline__ void code_bits_x2(uint32_t w, uint64_t ns2, uint64_t inv2,
+                                             uint64_t rnd2, uint32_t &lo, uint32_t &hi) {
+  const uint64_t x = f2_pack(bf16_lo(w), bf16_hi(w));
+  const uint64_t q0 = f2_mul(x, inv2);
+  const uint64_t r0 = f2_fma(ns2, q0, x);
+  float b0, b1;
+  f2_unpack(f2_add(f2_fma(r0, inv2, q0), rnd2), b0, b1);
+  lo = __float_as_uint(b0);
+  hi = __float_as_uint(b1);
+}
+
+__device__ __forceinline__ uint2 codes8_x2(const uint4 &v, uint64_t ns2, uint64_t inv2,
+                                           uint64_t rnd2) {
+  uint32_t c[8];
+  code_bits_x2(v.x, ns2, inv2, rnd2, c[0], c[1]);
+  code_bits_x2(v.y, ns2, inv2, rnd2, c[2], c[3]);
+  code_bits_x2(v.z, ns2, inv2, rnd2, c[4], c[5]);
+  code_bits_x2(v.w, ns2, inv2, rnd2, c[6], c[7]);
+  return make_uint2(pack4(c[0], c[1], c[2], c[3]), pack4(c[4], c[5], c[6], c[7]));
 }
 
 // The same with the IEEE quotient (rows with s < 1e-30).  A rolled loop keeps
