@@ -686,6 +686,16 @@ def short_kernel(name):
     return "1sm" + name.split("<")[1].split(",")[0]
 
 
+def sweep_steps(ops, gemm_bytes, int8_peak_tops, hbm_gbs, work_s=25e-3):
+    """Steps of a sweep loop: about `work_s` of work (a layer estimated at 0.6
+    of the int8 peak or 0.8 of HBM, whichever is slower), 100 to 2000 steps,
+    so that each loop finishes before the power cap settles, like the burst
+    peak it is read against (the headline's long loops give the sustained
+    figure)."""
+    t_est = max(ops / (int8_peak_tops * 1e12 * 0.6), gemm_bytes / (hbm_gbs * 1e9 * 0.8))
+    return int(min(2000, max(100, work_s / t_est)))
+
+
 def sweep(w8, args, device, stream, peaks, int8_peak):
     """Every workload as one layer: step (quant + GEMM), GEMM alone (cold
     operands; warm too where they fit L2), quantisation alone.  gemm_frac is
@@ -696,11 +706,7 @@ def sweep(w8, args, device, stream, peaks, int8_peak):
     for name in SWEEP:
         wl = WORKLOADS[name]
         ops, gemm_bytes, quant_bytes, fused_bytes = algorithmic(wl.M, wl.N, wl.K, wl.bias)
-        # about 25 ms of work a loop for every row (100 to 2000 steps), so that
-        # each finishes before the power cap settles, like the burst peak it is
-        # read against (the headline's long loops give the sustained figure)
-        t_est = max(ops / (int8_peak * 1e12 * 0.6), gemm_bytes / (peaks["hbm_gbs"] * 1e9 * 0.8))
-        steps = int(min(2000, max(100, 25e-3 / t_est)))
+        steps = sweep_steps(ops, gemm_bytes, int8_peak, peaks["hbm_gbs"])
         warm = wl.N * wl.K + wl.M * wl.K + 2 * wl.M * wl.N < L2_BYTES // 2
         cs, loop, r = measure_chain(w8, chain_of(name), steps, 3, device, stream,
                                     warm_gemm=warm)

@@ -161,3 +161,20 @@ def test_recorded_traffic_only_while_the_sources_match(tmp_path, monkeypatch):
     assert bench.recorded_traffic("odd") is None
     (csrc / bench.TRAFFIC_SOURCES[fam][-1]).write_bytes(b"// changed\n")
     assert bench.recorded_traffic("mlp") is None
+
+
+def test_sweep_loops_hold_about_25_ms_of_work():
+    peak, hbm = 3285.6, 6540.8
+    rows = {}
+    for name in bench.SWEEP:
+        wl = bench.WORKLOADS[name]
+        ops, gemm_bytes, _, _ = bench.algorithmic(wl.M, wl.N, wl.K, wl.bias)
+        n = bench.sweep_steps(ops, gemm_bytes, peak, hbm)
+        assert 100 <= n <= 2000
+        t = max(ops / (peak * 1e12 * 0.6), gemm_bytes / (hbm * 1e9 * 0.8))
+        if 100 < n < 2000:
+            assert n * t == pytest.approx(25e-3, rel=0.01)
+        rows[name] = n
+    # the 4096-token MLP layers are the longest: a few hundred steps at most
+    assert rows["dit_mlp_up_4096x12288x3072"] < 300
+    assert rows["small_64x128x256"] == 2000
