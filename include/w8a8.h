@@ -328,7 +328,7 @@ w8a8_status w8a8_selftest_wait_timeout(int64_t timeout_ns,
 
 /* Self-test of the int8 tensor-core rate with no memory traffic (no
  * counterpart on the pages; the ceiling against which the GEMM kernels'
- * rates can be read): one CTA per SM issues `iters` (1 ... 1e6) groups of
+ * rates can be read): one CTA per SM issues `iters` (1 ... 2e5) groups of
  * four tcgen05.mma.kind::i8 of M = 128, N = 256, K = 32 from shared memory
  * into TMEM; the launch is timed with CUDA events on `stream` after a
  * warm-up launch.  Synchronises the stream.  *tops: int8 TOPS (2 operations

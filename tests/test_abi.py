@@ -149,3 +149,11 @@ def test_act_quant_rejects_bad_arguments_and_sizes_its_workspace(L):
         rnd = lambda v: (v + 255) // 256 * 256  # noqa: E731
         extra = rnd(4 * M) + rnd(8 * ((M + 127) // 128)) + 256
         assert binding.linear_act_quant_workspace_bytes(M, N, K) == lin + extra
+
+
+def test_mma_rate_selftest_rejects_bad_arguments(L):
+    f = L.w8a8_selftest_int8_mma_rate
+    tops = ctypes.c_double(0.0)
+    assert f(0, None, ctypes.byref(tops)) == 1
+    assert f(200001, None, ctypes.byref(tops)) == 1   # beyond the bounded wait's reach
+    assert f(100, None, None) == 1
