@@ -4,10 +4,10 @@
  *
  * The method (sources by page title and section):
  *   "Issue 5 probe: int8 quantized DiT serve paths on the RTX 3090",
- *   Round two: int8 weights with fp32 per-output-channel scales, dynamic
- *   per-token symmetric int8 activations, an int8 scaled matmul, and the
- *   layer path "load -> transpose-repack -> apply" with fused Q/K/V and
- *   row-parallel layers.  "INT8 Quant for Dual-Max Recipe": int8 x int8 on
+ *   Round two: int8 weights with fp32 per-output-channel scales, int8
+ *   activations with one symmetric scale per token computed at run time, an
+ *   int8 scaled matmul, and weights transposed and repacked once at load
+ *   time, then applied, in fused Q/K/V and row-parallel layers as well.  "INT8 Quant for Dual-Max Recipe": int8 x int8 on
  *   the integer tensor cores with no dequantisation of the weights.
  *   "Online Quantization", Parameters: activation_scheme "dynamic".
  *
@@ -80,8 +80,9 @@ const char *w8a8_status_string(int status);
 int w8a8_abi_version(void);
 
 /* ---- step 1: dynamic per-token activation quantisation ------------------
- * Source: "Issue 5 probe ...", Round two ("dynamic per-token symmetric int8
- * activations", op scaled_int8_quant); "Online Quantization", Parameters.
+ * Source: "Issue 5 probe ...", Round two (int8 activations, one symmetric
+ * scale per token computed at run time; op scaled_int8_quant); "Online
+ * Quantization", Parameters.
  *   x       device, bf16 [M, K], row stride ldx >= K elements (ldx % 8 == 0)
  *   q       device, int8 [M, K] dense (output)
  *   a_scale device, fp32 [M]   (output)
@@ -106,8 +107,8 @@ w8a8_status w8a8_quant_act_static(const void *x, int64_t M, int64_t K, int64_t l
                                   w8a8_stream_t stream);
 
 /* ---- step 2 (load time): weight repack ------------------------------------
- * Source: "Issue 5 probe ...", Round two, kernel-path verification
- * ("load -> transpose-repack -> apply"); the layout is this library's own:
+ * Source: "Issue 5 probe ...", Round two, kernel-path verification (weights
+ * transposed and repacked once at load time); the layout is this library's own:
  * 128x128-byte tiles, each the K-major 128-byte-swizzled shared-memory image
  * the tensor core reads, N padded to 256 and K to 128 with zeros.
  *   Byte size of the packed buffer for an [N, K] weight: */
@@ -145,7 +146,7 @@ w8a8_status w8a8_quant_pack_weight(const void *w, int64_t N, int64_t K,
 
 /* ---- load time: repack from compressed-tensors int32 storage ----------------
  * Source: "Issue 5 probe ...", Artifact (weights stored with pack_to_int32:
- * uint8 biased by 128, four per int32).  Bit order (not printed there; this
+ * four unsigned bytes, each weight + 128, to an int32 word).  Bit order (not printed there; this
  * library's reading): element 4j+i of a row is bits [8i, 8i+8) of word j,
  * holding the unsigned byte (w + 128).
  *   w_i32   device, int32 [N, K/4] row-major, 16-byte aligned

@@ -219,8 +219,9 @@ int w8a8o_sampled(const int8_t *q, const float *a_scale, const int8_t *w,
 }
 
 /* ---- load-time weight repack --------------------------------------------
- * The pages name the step ("load -> transpose-repack -> apply", Round two,
- * kernel-path verification) but not a layout; the layout is this library's
+ * The pages name the step (weights are transposed and repacked once as they
+ * are loaded, then applied: Round two, kernel-path verification) but not a
+ * layout; the layout is this library's
  * own and is defined here from its written description, independently of the
  * CUDA code:
  *
@@ -320,8 +321,9 @@ int w8a8o_quant_act_static(const uint16_t *x, int64_t M, int64_t K, int64_t ldx,
 }
 
 /* ---- compressed-tensors int32 weight storage -----------------------------
- * "Issue 5 probe ...", Artifact: weights stored with pack_to_int32, "uint8
- * biased by 128, 4 per int32".  Reading (the page gives no bit order): the
+ * "Issue 5 probe ...", Artifact: weights stored with pack_to_int32, four
+ * bytes to an int32 word, each the weight plus 128 as an unsigned byte.
+ * Reading (the page gives no bit order): the
  * four consecutive K elements k = 4j .. 4j+3 of a row share int32 word j,
  * element 4j+i in bits [8i, 8i+8) as the unsigned byte (w + 128).
  * packed: int32 [N, K/4]; w: int8 [N, K]. */

@@ -1,8 +1,9 @@
 """End-to-end accuracy of the oracle against the page's printed figure.
 
 "Issue 5 probe: int8 quantized DiT serve paths on the RTX 3090", Round two,
-kernel-path verification: the raw ops match a float32 reference at 0.17%
-rel-L2 across (64,256,128) / (512,4096,4096) / (512,4096,12288).  Reading (see
+kernel-path verification: the kernel-level path agrees with a float32
+reference to within 0.17% relative L2 on the (64,256,128), (512,4096,4096) and
+(512,4096,12288) shapes.  Reading (see
 tests/golden/relL2_verification.json): the reference is the fp32 product of
 the dequantised operands, so 0.17% is the bf16 output rounding floor.  A wrong
 scale, a dropped term or a transposed operand moves the error by orders of

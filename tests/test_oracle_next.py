@@ -4,8 +4,8 @@ and compressed-tensors int32 unpacking.
 Sources: "Online Quantization", Overview (weights and scales computed at load
 time) and Parameters (activation_scheme "dynamic" vs a calibrated scale);
 "Issue 5 probe: int8 quantized DiT serve paths on the RTX 3090", Round one
-(per-output-channel symmetric weights) and Artifact (pack_to_int32: uint8
-biased by 128, 4 per int32).
+(per-output-channel symmetric weights) and Artifact (pack_to_int32: four
+unsigned bytes, weight + 128, to an int32 word).
 """
 from fractions import Fraction
 

@@ -1,9 +1,9 @@
 """Pins for the oracle's load-time weight repack.
 
 Source: "Issue 5 probe: int8 quantized DiT serve paths on the RTX 3090",
-Round two (kernel-path verification): the layer path is load ->
-transpose-repack -> apply, and the loaded weights, fused Q/K/V shards
-included, are verified bitwise.  The packed layout itself is this library's
+Round two (kernel-path verification): the layer's weights are transposed
+and repacked once as they are loaded, then applied, and the loaded weights
+(the fused Q/K/V ones too) are checked bit for bit.  The packed layout itself is this library's
 own (the UMMA K-major 128-byte-swizzled shared-memory tile image); it is
 pinned by hand-derived offsets, a bijection check, the padding rule, and the
 128-byte swizzle identity it must equal.

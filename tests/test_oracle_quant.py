@@ -1,7 +1,8 @@
 """Pins for the oracle's dynamic per-token activation quantisation.
 
 Source: "Issue 5 probe: int8 quantized DiT serve paths on the RTX 3090",
-Round two (int8 weights + dynamic per-token symmetric int8 activations);
+Round two (int8 weights; int8 activations with one symmetric scale per
+token, computed at run time);
 "Online Quantization", Parameters (activation_scheme "dynamic").
 
 The oracle is checked against the mathematics, not against a retyped copy of

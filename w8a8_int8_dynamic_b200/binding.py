@@ -388,8 +388,8 @@ def launch_count() -> int:
 
 
 class W8A8Linear:
-    """A pre-quantised linear layer: int8 weights [N, K] packed once at load
-    time ("load -> transpose-repack -> apply"), fp32 per-output-channel
+    """A pre-quantised linear layer: int8 weights [N, K] repacked once at
+    load time, then applied on every call, fp32 per-output-channel
     scales, optional bf16 bias.  For fused Q/K/V, build it from the three
     blocks with :meth:`from_blocks` and split the output with :meth:`split`.
     """

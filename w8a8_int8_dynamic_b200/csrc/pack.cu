@@ -1,9 +1,10 @@
 // pack.cu -- load-time weight repack: int8 W[N, K] -> tensor-core tile image.
 //
 // Source: "Issue 5 probe: int8 quantized DiT serve paths on the RTX 3090",
-// Round two, kernel-path verification: the layer path is "load ->
-// transpose-repack -> apply" and the loaded weights (fused Q/K/V shards
-// included) are verified bitwise.  The layout is this library's own.
+// Round two, kernel-path verification: the layer's weights are transposed
+// and repacked once as they are loaded, then applied, and the loaded weights
+// (the fused Q/K/V ones too) are checked bit for bit.  The layout is this
+// library's own.
 //
 // Layout: N padded to Np = round_up(N, 256), K to Kp = round_up(K, 128).
 // Tiles of 128 rows (n) x 128 bytes (k), tile (nb, kb) at byte offset

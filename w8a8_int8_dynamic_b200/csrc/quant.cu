@@ -1,9 +1,10 @@
-// quant.cu -- dynamic per-token symmetric int8 activation quantisation.
+// quant.cu -- int8 activation quantisation, one symmetric scale per token
+// computed at run time.
 //
 // Source: "Issue 5 probe: int8 quantized DiT serve paths on the RTX 3090",
-// Round two ("dynamic per-token symmetric int8 activations", the
-// scaled_int8_quant op); "Online Quantization", Parameters
-// (activation_scheme "dynamic": scales computed at run time).
+// Round two (the int8 activations of the W8A8 path, the scaled_int8_quant
+// op); "Online Quantization", Parameters (activation_scheme "dynamic":
+// scales computed at run time).
 //
 // Per row m:  amax = max_k |x[m,k]|;  s = amax / 127 (IEEE fp32 division);
 //             q = clamp(rint_half_even(x / s), -127, 127);  amax == 0 -> s = 0, q = 0.

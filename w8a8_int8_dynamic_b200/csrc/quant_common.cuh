@@ -1,7 +1,7 @@
-// quant_common.cuh -- the per-element arithmetic of the dynamic per-token
-// activation quantisation ("Issue 5 probe: int8 quantized DiT serve paths on
-// the RTX 3090", Round two: dynamic per-token symmetric int8 activations),
-// used by the quantisation kernels (quant.cu).
+// quant_common.cuh -- the per-element arithmetic of the activation
+// quantisation ("Issue 5 probe: int8 quantized DiT serve paths on the RTX
+// 3090", Round two: int8 activations, one symmetric scale per token computed
+// at run time), used by the quantisation kernels (quant.cu).
 //
 // Per row: amax = max |x|, s = RN(amax / 127), code = rint_half_even(RN(x / s)).
 //

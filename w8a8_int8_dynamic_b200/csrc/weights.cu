@@ -6,7 +6,8 @@
 //   symmetric): bf16 W[N, K] -> fp32 w_scale[N] and the packed int8 tile
 //   image, in one kernel (one CTA per output channel);
 // * compressed-tensors storage ("Issue 5 probe ...", Artifact: pack_to_int32,
-//   uint8 biased by 128, four per int32): int32 words -> packed int8 tiles.
+//   four unsigned bytes of weight + 128 to a word): int32 words -> packed
+//   int8 tiles.
 //   Element 4j+i of a row is byte i (bits 8i..8i+7) of word j, stored as
 //   w + 128, so in memory order the bytes are simply (w XOR 0x80): the plain
 //   repack with each byte's top bit flipped.
