@@ -94,12 +94,41 @@ TRAFFIC_SOURCES = {
 }
 
 
+def code_text(src):
+    """C / CUDA source with its comments removed and every run of whitespace
+    made one space: what the compiler sees, so that an edit of comments or
+    layout alone does not void a recorded measurement."""
+    out, i, n = [], 0, len(src)
+    while i < n:
+        c = src[i]
+        if c in "\"'":  # string or character literal, copied whole
+            j = i + 1
+            while j < n and src[j] != c:
+                j += 2 if src[j] == "\\" else 1
+            out.append(src[i:j + 1])
+            i = j + 1
+        elif src.startswith("//", i):
+            j = src.find("\n", i)
+            i = n if j < 0 else j
+        elif src.startswith("/*", i):
+            j = src.find("*/", i + 2)
+            i = n if j < 0 else j + 2
+            out.append(" ")
+        else:
+            out.append(c)
+            i += 1
+    return " ".join("".join(out).split())
+
+
 def sources_hash(kernel):
+    """First 16 hex digits of the sha256 of the code text (code_text) of a
+    kernel family's sources, in TRAFFIC_SOURCES order, one line each."""
     import hashlib
     csrc = os.path.join(HERE, "w8a8_int8_dynamic_b200", "csrc")
     h = hashlib.sha256()
     for f in TRAFFIC_SOURCES[kernel]:
-        h.update(open(os.path.join(csrc, f), "rb").read())
+        src = open(os.path.join(csrc, f), encoding="utf-8").read()
+        h.update((code_text(src) + "\n").encode())
     return h.hexdigest()[:16]
 
 

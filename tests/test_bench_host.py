@@ -144,10 +144,10 @@ def test_recorded_traffic_only_while_the_sources_match(tmp_path, monkeypatch):
     csrc.mkdir(parents=True)
     fam = "gemm2sm_kernel"
     for i, f in enumerate(bench.TRAFFIC_SOURCES[fam]):
-        (csrc / f).write_bytes(f"// source {i}\n".encode())
+        (csrc / f).write_bytes(f"// source {i}\nint  f{i}(int x) {{ return x; }}  /* end */\n".encode())
     h = hashlib.sha256()
-    for f in bench.TRAFFIC_SOURCES[fam]:
-        h.update((csrc / f).read_bytes())
+    for i, f in enumerate(bench.TRAFFIC_SOURCES[fam]):
+        h.update(f"int f{i}(int x) {{ return x; }}\n".encode())
     (tmp_path / "profiles").mkdir()
     rec = {"mlp": {"gemm_bytes_per_launch": 123, "kernel_family": fam,
                    "source_sha256_16": h.hexdigest()[:16]},
@@ -159,8 +159,18 @@ def test_recorded_traffic_only_while_the_sources_match(tmp_path, monkeypatch):
     assert bench.recorded_traffic("mlp") == 123
     assert bench.recorded_traffic("other") is None
     assert bench.recorded_traffic("odd") is None
-    (csrc / bench.TRAFFIC_SOURCES[fam][-1]).write_bytes(b"// changed\n")
+    # comments and layout do not count; code does
+    last = csrc / bench.TRAFFIC_SOURCES[fam][-1]
+    i = len(bench.TRAFFIC_SOURCES[fam]) - 1
+    last.write_bytes(f"/* reworded */ int f{i}(int x)\n{{\n  return x;  // same code\n}}\n".encode())
+    assert bench.recorded_traffic("mlp") == 123
+    last.write_bytes(f"int f{i}(int x) {{ return x + 1; }}\n".encode())
     assert bench.recorded_traffic("mlp") is None
+
+
+def test_code_text_keeps_literals_and_drops_comments():
+    src = 'a = "// not a comment"; /* gone\n */ b = \'/\'; // gone\nc  =\t"x\\"y";'
+    assert bench.code_text(src) == 'a = "// not a comment"; b = \'/\'; c = "x\\"y";'
 
 
 def test_sweep_loops_hold_about_25_ms_of_work():
