@@ -120,3 +120,27 @@ def test_bias_is_added_in_fp32():
     bias = f32_to_bf16_bits(np.array([1.0], np.float32))
     y = oracle.epilogue(acc, a_s, w_s, bias)
     assert bf16_bits_to_f32(y)[0, 0] == 126.0  # 1000*0.5*0.25 + 1 = 126
+
+
+def test_layer_reads_rows_at_their_stride():
+    """The whole layer on rows spaced ldx > K apart equals the layer on the
+    same rows packed densely: the columns past K never enter it."""
+    import ctypes
+    rng = np.random.default_rng(12)
+    M, N, K, ldx = 9, 24, 64, 80
+    big = f32_to_bf16_bits(rng.standard_normal((M, ldx)).astype(np.float32) * 2)
+    big[:, K:] = f32_to_bf16_bits(np.full((M, ldx - K), 3e4, np.float32))
+    w = rng.integers(-127, 128, (N, K), dtype=np.int8)
+    w_s = rng.uniform(5e-4, 5e-3, N).astype(np.float32)
+    bias = f32_to_bf16_bits(rng.standard_normal(N).astype(np.float32))
+    y_ref, q_ref, s_ref, acc_ref = oracle.linear(np.ascontiguousarray(big[:, :K]), w, w_s, bias)
+    y = np.empty((M, N), np.uint16)
+    q = np.empty((M, K), np.int8)
+    a_s = np.empty((M,), np.float32)
+    acc = np.empty((M, N), np.int32)
+    p_ = lambda a: a.ctypes.data_as(ctypes.c_void_p)
+    rc = oracle.lib().w8a8o_linear(p_(big), ldx, p_(w), p_(w_s), p_(bias), M, N, K,
+                                   p_(y), p_(q), p_(a_s), p_(acc))
+    assert rc == 0
+    assert (q == q_ref).all() and (a_s.view(np.uint32) == s_ref.view(np.uint32)).all()
+    assert (acc == acc_ref).all() and (y == y_ref).all()

@@ -78,10 +78,12 @@ def test_sampled_matches_full():
     w = rng.integers(-127, 128, (40, 256), dtype=np.int8)
     a_s = rng.uniform(1e-3, 1e-1, 16).astype(np.float32)
     w_s = rng.uniform(1e-3, 1e-2, 40).astype(np.float32)
+    bias = rng.integers(0x3c00, 0x4100, 40).astype(np.uint16)  # bf16 bits, 0.0078 .. 8
     acc = oracle.gemm_i32(q, w)
-    y = oracle.epilogue(acc, a_s, w_s)
     rows = rng.integers(0, 16, 50)
     cols = rng.integers(0, 40, 50)
-    acc_s, y_s = oracle.sampled(q, a_s, w, w_s, None, rows, cols)
-    assert (acc_s == acc[rows, cols]).all()
-    assert (y_s == y[rows, cols]).all()
+    for b in (None, bias):
+        y = oracle.epilogue(acc, a_s, w_s, b)
+        acc_s, y_s = oracle.sampled(q, a_s, w, w_s, b, rows, cols)
+        assert (acc_s == acc[rows, cols]).all()
+        assert (y_s == y[rows, cols]).all()

@@ -89,6 +89,29 @@ MUTANTS = [
     ("static scale accepts a negative scale",
      "  const int usable = scale > 0.0f; /* false for NaN too */",
      "  const int usable = scale != 0.0f;", [N]),
+    ("epilogue in double precision, one rounding at the end",
+     "  float t = (float)acc; /* int32 -> fp32, nearest even */\n  t = t * as;\n  t = t * ws;\n"
+     "  if (bias) t = t + bf16_to_f32(bias[n]);\n  return f32_to_bf16_rne(t);",
+     "  double t = (double)acc * as * ws;\n"
+     "  if (bias) t = t + bf16_to_f32(bias[n]);\n  return f64_to_bf16_rne(t);", [E]),
+    ("layer ignores the row stride",
+     "    rc = w8a8o_quant_act(x, M, K, ldx, q, as);",
+     "    rc = w8a8o_quant_act(x, M, K, K, q, as);", [E]),
+    ("sampled reads the weight row of the output row",
+     "    const int8_t *wr = w + cols[i] * K;",
+     "    const int8_t *wr = w + rows[i] * K;", [G]),
+    ("sampled adds the bias of the row index",
+     "w_scale[cols[i]], bias, cols[i]);",
+     "w_scale[cols[i]], bias, rows[i]);", [G]),
+    ("repack leaves the padding unzeroed",
+     "  memset(packed, 0, (size_t)(Np * Kp));",
+     "  memset(packed, 0x11, (size_t)(Np * Kp));", [P]),
+    ("packed size rounds N up to 128",
+     "  return ((N + 255) / 256 * 256) * ((K + 127) / 128 * 128);",
+     "  return ((N + 127) / 128 * 128) * ((K + 127) / 128 * 128);", [P]),
+    ("gelu multiplies the sigmoid by |x|",
+     "    y[i] = f64_to_bf16_rne(v * sig);",
+     "    y[i] = f64_to_bf16_rne(fabs(v) * sig);", [L]),
     ("static codes clamp at 126",
      "      float v = bf16_to_f32(x[m * ldx + k]) / scale;\n      float r = nearbyintf(v);\n"
      "      if (r > 127.0f) r = 127.0f;",
