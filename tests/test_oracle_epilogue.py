@@ -32,6 +32,20 @@ def test_bf16_rounding_worked_examples():
     assert oracle.f64_to_bf16(1.0 + 2.0 ** -8 + 2.0 ** -40) == 0x3F81  # single rounding
 
 
+def test_double_to_bf16_is_one_rounding_next_to_a_tie():
+    """Doubles a hair from a bf16 midpoint, closer than half an fp32 ulp: a
+    first rounding to fp32 would land on the midpoint itself, so only a
+    single correct rounding (nearest, ties even) gets these right."""
+    f = oracle.f64_to_bf16
+    eps = 2.0 ** -40
+    for sign, bits in ((1.0, 0x0000), (-1.0, 0x8000)):
+        assert f(sign * (1.0 + 2.0 ** -8 - eps)) == bits | 0x3F80   # below the tie: down
+        assert f(sign * (1.0 + 2.0 ** -8)) == bits | 0x3F80         # the tie: even (down)
+        assert f(sign * (1.0 + 2.0 ** -8 + eps)) == bits | 0x3F81   # above the tie: up
+        assert f(sign * (1.0 + 3 * 2.0 ** -8 - eps)) == bits | 0x3F81  # below the next tie
+        assert f(sign * (1.0 + 3 * 2.0 ** -8)) == bits | 0x3F82     # that tie: even (up)
+
+
 def test_bf16_rounding_matches_torch():
     rng = np.random.default_rng(0)
     v = (rng.standard_normal(20000) * rng.choice([1e-3, 1.0, 1e3], 20000)).astype(np.float32)

@@ -112,6 +112,18 @@ MUTANTS = [
     ("gelu multiplies the sigmoid by |x|",
      "    y[i] = f64_to_bf16_rne(v * sig);",
      "    y[i] = f64_to_bf16_rne(fabs(v) * sig);", [L]),
+    ("static codes clamp below at -128",
+     "      if (r < -127.0f) r = -127.0f;\n      q[m * K + k] = (int8_t)r;",
+     "      if (r < -128.0f) r = -128.0f;\n      q[m * K + k] = (int8_t)r;", [N]),
+    ("static scale reported for an unusable scale",
+     "    if (a_scale_out) a_scale_out[m] = usable ? scale : 0.0f;",
+     "    if (a_scale_out) a_scale_out[m] = scale;", [N]),
+    ("static scale reads rows at the dense stride",
+     "      float v = bf16_to_f32(x[m * ldx + k]) / scale;",
+     "      float v = bf16_to_f32(x[m * K + k]) / scale;", [N]),
+    ("round-to-odd without the truncation toward zero",
+     "    if (fabs((double)f) > fabs(g)) f = nextafterf(f, 0.0f);\n",
+     "", [L, E]),
     ("static codes clamp at 126",
      "      float v = bf16_to_f32(x[m * ldx + k]) / scale;\n      float r = nearbyintf(v);\n"
      "      if (r > 127.0f) r = 127.0f;",

@@ -87,6 +87,24 @@ def test_static_equals_dynamic_when_scale_is_the_row_scale():
     assert (qd == qs).all() and (sd == ss).all()
 
 
+def test_static_scale_reads_rows_at_their_stride():
+    """Rows spaced ldx > K apart give the codes of the same rows packed
+    densely; the columns past K (here values that would saturate) never
+    enter."""
+    import ctypes
+    rng = np.random.default_rng(6)
+    M, K, ldx = 5, 48, 64
+    big = bf(rng.standard_normal((M, ldx)).astype(np.float32))
+    big[:, K:] = bf(np.full((M, ldx - K), 500.0, np.float32))
+    q_ref, s_ref = oracle.quant_act_static(np.ascontiguousarray(big[:, :K]), 0.02)
+    q = np.empty((M, K), np.int8)
+    s = np.empty((M,), np.float32)
+    p_ = lambda a: a.ctypes.data_as(ctypes.c_void_p)
+    assert oracle.lib().w8a8o_quant_act_static(p_(big), M, K, ldx, float(np.float32(0.02)),
+                                               p_(q), p_(s)) == 0
+    assert (q == q_ref).all() and (s == s_ref).all()
+
+
 # ---------------------------------------------------------------- int32 storage
 def test_unpack_worked_example():
     # word 0x807F0081: bytes (low first) 0x81, 0x00, 0x7F, 0x80 -> 1, -128, -1, 0
