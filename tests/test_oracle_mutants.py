@@ -43,6 +43,9 @@ MUTANTS = [
     ("quant zero row gets scale 1",
      "      a_scale[m] = 0.0f;\n      for (int64_t k = 0; k < K; ++k) qr[k] = 0;",
      "      a_scale[m] = 1.0f;\n      for (int64_t k = 0; k < K; ++k) qr[k] = 0;", [Q]),
+    ("quant row maximum skips the last element",
+     "    for (int64_t k = 0; k < K; ++k) {\n      float a = fabsf(bf16_to_f32(xr[k]));",
+     "    for (int64_t k = 0; k + 1 < K; ++k) {\n      float a = fabsf(bf16_to_f32(xr[k]));", [Q]),
     ("gemm reads the weight transposed",
      "      const int8_t *wr = w + n * K;\n      int64_t s = 0;\n"
      "      for (int64_t k = 0; k < K; ++k) s += (int64_t)qr[k] * (int64_t)wr[k];",

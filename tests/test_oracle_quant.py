@@ -155,6 +155,20 @@ def test_invariants_random(seed):
     assert (err <= bound).all()
 
 
+@pytest.mark.parametrize("K", [1, 7, 256])
+def test_row_maximum_at_every_position(K):
+    """Row m of a K x K input has its largest magnitude in column m (the
+    first, a middle and the last column among them): wherever it sits, the
+    scale is that magnitude / 127 and its code is +-127."""
+    rng = np.random.default_rng(K)
+    x = rng.uniform(-1.0, 1.0, (K, K)).astype(np.float32)
+    big = np.where(rng.random(K) < 0.5, -4.0, 4.0).astype(np.float32)
+    x[np.arange(K), np.arange(K)] = big
+    q, s = oracle.quant_act(bf(x))
+    assert (s == np.float32(4.0) / np.float32(127.0)).all()
+    assert (q[np.arange(K), np.arange(K)] == np.where(big < 0, -127, 127)).all()
+
+
 def test_sign_symmetry():
     rng = np.random.default_rng(3)
     xb = bf(rng.standard_normal((8, 128)).astype(np.float32))
