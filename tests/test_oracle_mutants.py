@@ -51,6 +51,9 @@ MUTANTS = [
      "      for (int64_t k = 0; k < K; ++k) s += (int64_t)qr[k] * (int64_t)wr[k];",
      "      int64_t s = 0;\n"
      "      for (int64_t k = 0; k < K; ++k) s += (int64_t)qr[k] * (int64_t)w[k * N + n];", [G]),
+    ("gemm accumulates in int32",
+     "      const int8_t *wr = w + n * K;\n      int64_t s = 0;",
+     "      const int8_t *wr = w + n * K;\n      int32_t s = 0;", [G]),
     ("gemm drops the overflow check",
      "      if (s > INT32_MAX || s < INT32_MIN) overflow = 1;\n      acc[m * N + n] = (int32_t)s;",
      "      acc[m * N + n] = (int32_t)s;", [G]),
@@ -62,6 +65,9 @@ MUTANTS = [
     ("epilogue multiplies the two scales first",
      "  t = t * as;\n  t = t * ws;",
      "  t = t * (as * ws);", [E]),
+    ("epilogue adds the bias before the weight scale",
+     "  t = t * as;\n  t = t * ws;\n  if (bias) t = t + bf16_to_f32(bias[n]);",
+     "  t = t * as;\n  if (bias) t = t + bf16_to_f32(bias[n]);\n  t = t * ws;", [E]),
     ("epilogue drops the bias",
      "  if (bias) t = t + bf16_to_f32(bias[n]);",
      "  (void)bias;", [E]),
