@@ -550,7 +550,7 @@ def run_ours(args, rank, world, device):
         t_roof += max(o / (int8_peak * 1e12), fused / (peaks["hbm_gbs"] * 1e9))
 
     # ---- end to end through the public API, host buffers
-    e2e = run_e2e(w8, cs, args, stream, ops)
+    e2e = run_e2e(w8, cs, args, stream, ops, world, device)
     del cs, step_loop
     torch.cuda.empty_cache()
 
@@ -575,7 +575,7 @@ def run_ours(args, rank, world, device):
         "gpu_launches": int(base["launches_per_step"] * args.steps),
         "clocks": {k: clocks[k] for k in ("sm_mhz", "sm_max_mhz", "reasons")},
     }
-    if rank == 0 and not args.no_cpu_baseline:
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:  # the oracle, at N = 1 only
         out["cpu_baseline"] = cpu_baseline(names, budget_s=args.cpu_seconds)
     if not args.no_sweep:
         out["sweep_cols"] = SWEEP_COLS
@@ -610,6 +610,17 @@ def whole_job_tops(ops_per_step, steps, world, t_max):
     return ops_per_step * steps * world / t_max / 1e12
 
 
+def e2e_record(ops_per_step, steps, elapsed, world, device, h2d_bytes, d2h_bytes):
+    """The end-to-end leg as a whole-job figure, like `value`: every rank's
+    steps over the slowest rank's time, and the bytes all ranks copy a step
+    (replicas: each rank moves its own)."""
+    t_max = max_over_ranks(elapsed, world, device)
+    return {"value": round(whole_job_tops(ops_per_step, steps, world, t_max), 2),
+            "unit": "TOPS", "h2d_bytes_per_step": h2d_bytes * world,
+            "d2h_bytes_per_step": d2h_bytes * world, "steps": steps,
+            "ms_per_step": round(t_max / steps * 1e3, 4)}
+
+
 # host <-> device copies of a step, each in this many cudaMemcpyAsync pieces:
 # two halves let the two directions interleave on PCIe (DiT MLP block, 25 MB
 # each way: 0.533 ms a step against 0.573 ms with whole copies; the copies
@@ -617,7 +628,7 @@ def whole_job_tops(ops_per_step, steps, world, t_max):
 E2E_PIECES = 2
 
 
-def run_e2e(w8, cs, args, stream, ops):
+def run_e2e(w8, cs, args, stream, ops, world=1, device=None):
     """Public API, host buffers: per step H2D of the first layer's input from
     pinned memory, the layers, D2H of the last layer's output into pinned
     memory, all inside the timed region.  Steps are pipelined the way a
@@ -673,6 +684,8 @@ def run_e2e(w8, cs, args, stream, ops):
     for i in range(max(nhost, ndev)):
         step(i, first)
     torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
     start = torch.cuda.Event(enable_timing=True)
     end = torch.cuda.Event(enable_timing=True)
     start.record(up)
@@ -684,18 +697,18 @@ def run_e2e(w8, cs, args, stream, ops):
     comp.wait_stream(up)
     end.record(comp)
     end.synchronize()
-    t = start.elapsed_time(end) / 1e3 / steps
+    elapsed = start.elapsed_time(end) / 1e3
     # the last step's output must have arrived
     last = dsets[(steps - 1) % ndev]["layers"][-1].y
     assert torch.equal(ys[(steps - 1) % nhost].to(dev), last)
     xb = int(np.prod(x_shape)) * 2
     yb = int(np.prod(y_shape)) * 2
-    return {"value": round(ops / t / 1e12, 2), "unit": "TOPS", "h2d_bytes_per_step": xb,
-            "d2h_bytes_per_step": yb, "steps": steps, "ms_per_step": round(t * 1e3, 4),
-            "overlap": f"H2D i+1 | layers i | D2H i-1, 3 streams, copies in {E2E_PIECES} pieces",
-            "api": "+".join(sorted({"w8a8_linear_act_quant" if L.fuse_next else
-                                    "w8a8_scaled_mm" if L.from_codes else "w8a8_linear_act"
-                                    for L in s0["layers"]}))}
+    rec = e2e_record(ops, steps, elapsed, world, device, xb, yb)
+    rec["overlap"] = f"H2D i+1 | layers i | D2H i-1, 3 streams, copies in {E2E_PIECES} pieces"
+    rec["api"] = "+".join(sorted({"w8a8_linear_act_quant" if L.fuse_next else
+                                  "w8a8_scaled_mm" if L.from_codes else "w8a8_linear_act"
+                                  for L in s0["layers"]}))
+    return rec
 
 
 # compact sweep rows: one list per workload, columns named once
